@@ -1,0 +1,431 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against a value printed on a page (fixtures under
+tests/golden/, each with its citation), a closed form, an invariant, or a
+brute-force evaluation on tiny inputs written here independently of the
+oracle's C code.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from seeded_inputs import f32_to_bf16_bits, bf16_bits_to_f32
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _frac(s):
+    return float(Fraction(s))
+
+
+# ---------------------------------------------------------------------------
+# printed worked examples
+# ---------------------------------------------------------------------------
+def test_four_expert_renormalisation_and_combine():
+    g = _golden("four_expert_example.json")
+    p = np.array(g["probabilities"])
+    # one token, d = 1, x = 1: the router scores are the rows of W_r, and
+    # scores ln p give back p under softmax because sum(p) = 1
+    x = np.ones((1, 1), np.float32)
+    W_r = np.log(p).astype(np.float32).reshape(-1, 1)
+    r = oracle.route(x, W_r, k=g["k"], norm=oracle.NORM_RENORM)
+    assert list(r["ids"][0]) == g["chosen_experts_by_score"]
+    np.testing.assert_allclose(r["w"][0], g["weights"], rtol=0, atol=1e-6)
+    # combine with the printed expert outputs
+    E = len(p)
+    H = [None] * E
+    for e, out in g["expert_outputs"].items():
+        H[int(e)] = np.array([out], np.float64)
+    slot = np.zeros((1, g["k"]), np.int32)
+    y = oracle.combine(r["ids"], r["w"], slot, H, d=2)
+    np.testing.assert_allclose(y[0], g["y"], rtol=0, atol=1e-6)
+
+
+def _n4_setup():
+    g = _golden("n4_e3_k2_example.json")
+    P = np.array(g["probabilities"])          # [token, expert]
+    x = np.eye(4, dtype=np.float32)
+    W_r = np.log(P).T.astype(np.float32)       # stored [E_r, d]; G = X W_r^T = ln P
+    return g, x, W_r
+
+
+def _linear_expert_outputs(x, ids, slot, E):
+    """Expert outputs of the page's linear experts F_e(x) = e x (1-based e),
+    laid out per expert by slot."""
+    N, k = ids.shape
+    H = []
+    for e in range(E):
+        rows = {}
+        for t in range(N):
+            for j in range(k):
+                if ids[t, j] == e and slot[t, j] >= 0:
+                    rows[slot[t, j]] = (e + 1) * x[t].astype(np.float64)
+        H.append(np.array([rows[c] for c in range(len(rows))]) if rows else None)
+    return H
+
+
+def test_n4_example_selection_and_weights():
+    g, x, W_r = _n4_setup()
+    r = oracle.route(x, W_r, k=2, norm=oracle.NORM_RENORM)
+    for t in range(4):
+        chosen = sorted(int(e) + 1 for e in r["ids"][t])
+        assert chosen == g["chosen_sets"][t]
+        by_expert = {int(e) + 1: w for e, w in zip(r["ids"][t], r["w"][t])}
+        want = [_frac(s) for s in g["weights_by_expert_index"][t]]
+        got = [by_expert[e] for e in g["chosen_sets"][t]]
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-6)
+        assert abs(sum(r["w"][t]) - 1.0) < 1e-12
+
+
+def test_n4_example_uncapped_outputs():
+    g, x, W_r = _n4_setup()
+    r = oracle.route(x, W_r, k=2, norm=oracle.NORM_RENORM)
+    d = oracle.dispatch(r["ids"], E=3, C=4)          # C = N: nothing rejected
+    assert d["stats"]["rejected"] == 0
+    H = _linear_expert_outputs(x, r["ids"], d["slot"], 3)
+    Y = oracle.combine(r["ids"], r["w"], d["slot"], H, d=4)
+    want = np.diag([_frac(s) for s in g["uncapped_output_coefficients"]])
+    np.testing.assert_allclose(Y, want, rtol=0, atol=1e-6)
+
+
+def test_n4_example_capacity_and_statistics():
+    g, x, W_r = _n4_setup()
+    C = oracle.capacity(g["capacity_factor"], 4, 2, 3)
+    assert C == g["capacity"]
+    r = oracle.route(x, W_r, k=2, norm=oracle.NORM_RENORM)
+    d = oracle.dispatch(r["ids"], E=3, C=C)
+    assert list(d["L"]) == g["requested_loads"]
+    assert list(d["acc"]) == g["accepted_loads"]
+    # token 4's path to expert 2 is the one rejected
+    rt, re_ = g["rejected_path"]["token"] - 1, g["rejected_path"]["expert"] - 1
+    for t in range(4):
+        for j in range(2):
+            rejected = d["slot"][t, j] < 0
+            assert rejected == (t == rt and r["ids"][t, j] == re_)
+    s = d["stats"]
+    assert Fraction(s["rejected"], s["requested"]) == Fraction(g["path_reject_rate"])
+    assert Fraction(s["tokens_affected"], 4) == Fraction(g["tokens_affected_fraction"])
+    assert Fraction(s["tokens_skipped"], 4) == Fraction(g["tokens_fully_skipped_fraction"])
+    assert oracle.rho_max(d["L"], 4, 2, 3) == float(Fraction(g["rho_max"]))
+    # zero-reject output of token 4 (no renormalisation of the remaining path)
+    H = _linear_expert_outputs(x, r["ids"], d["slot"], 3)
+    Y = oracle.combine(r["ids"], r["w"], d["slot"], H, d=4)
+    assert abs(Y[3, 3] - _frac(g["token4_output_coefficient_zero_reject"])) < 1e-6
+    for t in range(3):
+        assert abs(Y[t, t] - _frac(g["uncapped_output_coefficients"][t])) < 1e-6
+
+
+def test_capacity_printed_examples():
+    for case in _golden("capacity_examples.json")["cases"]:
+        assert oracle.capacity(case["c"], case["T"], case["k"], case["E"]) == case["C"], case
+
+
+def test_capacity_closed_forms():
+    # Qwen3-shaped layer: ceil(1.25 * 8192 * 8 / 128) = 640 exactly
+    assert oracle.capacity(1.25, 8192, 8, 128) == 640
+    # Switch-shaped layer: 1.25 * 1024 / 8 = 160 exactly
+    assert oracle.capacity(1.25, 1024, 1, 8) == 160
+    # a decimal factor whose binary value is a hair above 11/10 stays at 100
+    assert oracle.capacity(1.1, 1000, 1, 11) == 100
+    # just above an integer rounds up
+    assert oracle.capacity(1.25, 1001, 1, 8) == 157
+    # no capacity limit means C = N
+    assert oracle.capacity(0.0, 4096, 2, 8) == 4096
+
+
+# ---------------------------------------------------------------------------
+# closed forms, special cases and invariants of routing
+# ---------------------------------------------------------------------------
+def test_full_probability_weight_uniform():
+    # x = 0 makes every score 0: p = 1/E_r, top-k = {0..k-1} by the index rule
+    x = np.zeros((3, 16), np.float32)
+    W_r = np.random.default_rng(0).standard_normal((8, 16)).astype(np.float32)
+    r = oracle.route(x, W_r, k=1, norm=oracle.NORM_FULLPROB)
+    assert (r["ids"][:, 0] == 0).all()
+    np.testing.assert_allclose(r["w"][:, 0], 1 / 8, rtol=0, atol=1e-15)
+    r = oracle.route(x, W_r, k=3, norm=oracle.NORM_RENORM)
+    assert (r["ids"] == np.array([0, 1, 2])).all()
+    np.testing.assert_allclose(r["w"], 1 / 3, rtol=0, atol=1e-15)
+
+
+def test_tie_rule_lower_index_first():
+    x = np.ones((1, 1), np.float32)
+    W_r = np.array([[1.0], [3.0], [3.0], [2.0]], np.float32)
+    assert list(oracle.route(x, W_r, k=1, norm=0)["ids"][0]) == [1]
+    assert list(oracle.route(x, W_r, k=2, norm=0)["ids"][0]) == [1, 2]
+    assert list(oracle.route(x, W_r, k=3, norm=0)["ids"][0]) == [1, 2, 3]
+    r = oracle.route(x, W_r, k=2, norm=0)
+    assert r["margin"][0] == 1.0                          # g_(2) - g_(3) = 3 - 2
+
+
+def _softmax_np(g):
+    z = np.exp(g - g.max(axis=1, keepdims=True))
+    return z / z.sum(axis=1, keepdims=True)
+
+
+def test_topk_by_scores_equals_topk_by_probabilities_and_full_prob_closed_form():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((64, 12)).astype(np.float32)
+    W_r = rng.standard_normal((10, 12)).astype(np.float32)
+    k = 3
+    r = oracle.route(x, W_r, k=k, norm=oracle.NORM_FULLPROB)
+    g = x.astype(np.float64) @ W_r.astype(np.float64).T
+    p = _softmax_np(g)
+    for t in range(64):
+        by_p = sorted(range(10), key=lambda e: (-p[t, e], e))[:k]
+        assert list(r["ids"][t]) == by_p
+        np.testing.assert_allclose(r["w"][t], p[t, by_p], rtol=1e-12, atol=0)
+    # renormalised weights: softmax over the chosen scores only, sum to one
+    rn = oracle.route(x, W_r, k=k, norm=oracle.NORM_RENORM)
+    for t in range(64):
+        gs = g[t, rn["ids"][t]]
+        want = np.exp(gs - gs.max()) / np.exp(gs - gs.max()).sum()
+        np.testing.assert_allclose(rn["w"][t], want, rtol=1e-12, atol=0)
+        assert abs(rn["w"][t].sum() - 1) < 1e-12
+
+
+def test_router_bias_enters_scores():
+    x = np.zeros((2, 4), np.float32)
+    W_r = np.zeros((5, 4), np.float32)
+    b = np.array([0.0, -1.0, 2.0, 2.0, 0.5], np.float32)
+    r = oracle.route(x, W_r, k=2, norm=oracle.NORM_RENORM, b_r=b)
+    assert list(r["ids"][0]) == [2, 3]
+    np.testing.assert_allclose(r["w"][0], [0.5, 0.5], atol=1e-15)
+    np.testing.assert_allclose(r["logits"][0], b, atol=0)
+
+
+def test_nonfinite_scores_are_input_failures():
+    x = np.ones((3, 2), np.float32)
+    x[1, 0] = np.inf
+    W_r = np.array([[1.0, 0.0], [0.0, 1.0], [-1.0, 0.0]], np.float32)  # inf - inf -> nan too
+    r = oracle.route(x, W_r, k=2, norm=oracle.NORM_RENORM)
+    assert r["invalid"].tolist() == [False, True, False]
+    assert (r["ids"][1] == -1).all() and (r["w"][1] == 0).all()
+    d = oracle.dispatch(r["ids"], E=3, C=3)
+    assert d["stats"]["requested"] == 4
+
+
+# ---------------------------------------------------------------------------
+# WDMoE weight-latency-ratio pruning: the pages print no worked numbers, so
+# these are hand-derived cases of the stated rule (ratio <= theta drops the
+# smallest WLR; disconnected expert has weight 0).
+# ---------------------------------------------------------------------------
+def _wlr(logit_probs, lat, k, theta):
+    p = np.array(logit_probs, np.float64)
+    x = np.ones((1, 1), np.float32)
+    W_r = np.log(p).astype(np.float32).reshape(-1, 1)
+    la = np.array([lat], np.float32)
+    return oracle.route(x, W_r, k=k, norm=oracle.NORM_WLR, theta=theta, lat=la)
+
+
+def test_wlr_prunes_slow_expert():
+    # p = (0.6, 0.4), t = (1, 4): WLR = (0.6, 0.1), ratio 1/7 <= 0.3 -> drop expert 1
+    r = _wlr([0.6, 0.4], [1.0, 4.0], k=2, theta=0.3)
+    assert list(r["ids"][0]) == [0, -1]
+    np.testing.assert_allclose(r["w"][0], [1.0, 0.0], atol=1e-12)
+    assert abs(r["wlr_gap"][0] - abs(1 / 7 - 0.3)) < 1e-6
+
+
+def test_wlr_keeps_both_when_balanced():
+    # t = (1, 1): WLR = (0.6, 0.4), ratio 0.4 > 0.3 -> keep, renormalised weights
+    r = _wlr([0.6, 0.4], [1.0, 1.0], k=2, theta=0.3)
+    assert list(r["ids"][0]) == [0, 1]
+    np.testing.assert_allclose(r["w"][0], [0.6, 0.4], atol=1e-6)
+
+
+def test_wlr_iterates_until_condition_fails():
+    # top-3 of (0.4, 0.3, 0.2, 0.1) with t = (1, 1, 10, 1): WLR (0.4, 0.3, 0.02)
+    # ratio 0.02/0.42 -> drop expert 2; then 0.3/0.7 > 0.3 -> stop
+    r = _wlr([0.4, 0.3, 0.2, 0.1], [1.0, 1.0, 10.0, 1.0], k=3, theta=0.3)
+    assert list(r["ids"][0]) == [0, 1, -1]
+    np.testing.assert_allclose(r["w"][0], [4 / 7, 3 / 7, 0.0], atol=1e-6)
+    # (0.5, 0.3, 0.2) with t = (1, 3, 4): WLR (0.5, 0.1, 0.05): drop 2, then 0.1/0.6 -> drop 1
+    r = _wlr([0.5, 0.3, 0.2], [1.0, 3.0, 4.0], k=3, theta=0.3)
+    assert list(r["ids"][0]) == [0, -1, -1]
+    np.testing.assert_allclose(r["w"][0], [1.0, 0.0, 0.0], atol=1e-12)
+
+
+def test_wlr_theta_zero_is_plain_renormalised_topk():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((32, 8)).astype(np.float32)
+    W_r = rng.standard_normal((6, 8)).astype(np.float32)
+    lat = np.exp(0.5 * rng.standard_normal((32, 6))).astype(np.float32)
+    a = oracle.route(x, W_r, k=3, norm=oracle.NORM_WLR, theta=0.0, lat=lat)
+    b = oracle.route(x, W_r, k=3, norm=oracle.NORM_RENORM)
+    assert (a["ids"] == b["ids"]).all()
+    np.testing.assert_allclose(a["w"], b["w"], rtol=1e-14, atol=0)
+
+
+def test_wlr_disconnected_expert_and_tie():
+    # infinite latency: WLR = 0, ratio 0 -> pruned first
+    r = _wlr([0.6, 0.4], [np.inf, 1.0], k=2, theta=0.3)
+    assert list(r["ids"][0]) == [-1, 1]
+    np.testing.assert_allclose(r["w"][0], [0.0, 1.0], atol=1e-12)
+    # equal WLR, ratio 1/2 <= theta = 0.6: the higher index is dropped
+    r = _wlr([0.5, 0.5], [1.0, 1.0], k=2, theta=0.6)
+    assert list(r["ids"][0]) == [0, -1]
+    # a single remaining expert is never dropped (ratio 1/2 > 0.3)
+    r = _wlr([0.9, 0.1], [1.0, 100.0], k=2, theta=0.3)
+    assert list(r["ids"][0]) == [0, -1]
+
+
+# ---------------------------------------------------------------------------
+# dispatch invariants (Algorithm 36.1) on random requests, checked by brute force
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_dispatch_invariants(seed):
+    rng = np.random.default_rng(seed)
+    N, E, k = 97, 7, 3
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(N)]).astype(np.int32)
+    ids[5, 1] = -1                                    # a pruned path is not a request
+    C = 30
+    d = oracle.dispatch(ids, E=E, C=C)
+    s = d["stats"]
+    assert s["requested"] == N * k - 1 == int(d["L"].sum())
+    assert s["requested"] == s["accepted"] + s["rejected"]
+    assert s["O"] == sum(max(0, int(L) - C) for L in d["L"])
+    assert (d["acc"] <= C).all()
+    for e in range(E):
+        owners = [(t, j) for t in range(N) for j in range(k) if ids[t, j] == e]
+        # first-come-first-served: the first C requests in token order are accepted
+        for rank, (t, j) in enumerate(owners):
+            assert d["slot"][t, j] == (rank if rank < C else -1)
+    assert d["slot"][5, 1] == -1
+
+
+def test_empty_batch():
+    x = np.zeros((0, 8), np.float32)
+    W_r = np.zeros((4, 8), np.float32)
+    Wg = np.zeros((4, 6, 8), np.float32)
+    Wd = np.zeros((4, 8, 6), np.float32)
+    out = oracle.forward(x, W_r, Wg, Wg, Wd, k=2, norm=0, c=1.0)
+    assert out["Y"].shape == (0, 8)
+    assert out["stats"]["requested"] == 0 and int(out["L"].sum()) == 0
+
+
+# ---------------------------------------------------------------------------
+# SwiGLU expert and bf16 rounding
+# ---------------------------------------------------------------------------
+def test_swiglu_closed_forms():
+    x = np.ones((1, 1), np.float32)
+    ln3 = np.float32(math.log(3.0))
+    # SiLU(ln 3) = ln3 / (1 + 1/3) = 0.75 ln 3; times up = 2, down = 0.5
+    out = oracle.swiglu_rows(x, [0], np.array([[ln3]]), np.array([[2.0]], np.float32),
+                             np.array([[0.5]], np.float32))
+    assert abs(out[0, 0] - 0.75 * math.log(3.0)) < 1e-7
+    # SiLU(z) -> z for large z, -> 0 for very negative z, SiLU(0) = 0
+    for z, want in ((40.0, 40.0), (-40.0, 0.0), (0.0, 0.0)):
+        out = oracle.swiglu_rows(x, [0], np.array([[z]], np.float32), np.array([[1.0]], np.float32),
+                                 np.array([[1.0]], np.float32))
+        assert abs(out[0, 0] - want) < 1e-12
+
+
+def test_bf16_rounding_matches_bit_rounding():
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([rng.standard_normal(2000).astype(np.float32) * np.float32(3.0),
+                           np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8),
+                                     1.0 + 2 ** -8 + 2 ** -20, 3.0e38, 1e-40], np.float32)])
+    want = bf16_bits_to_f32(f32_to_bf16_bits(vals)).astype(np.float64)
+    got = np.array([oracle.round_bf16(float(v)) for v in vals])
+    np.testing.assert_array_equal(got, want)
+    assert oracle.round_bf16(1.0 + 2 ** -8) == 1.0                # tie -> even
+    assert oracle.round_bf16(1.0 + 3 * 2 ** -8) == 1.0 + 2 ** -6  # tie -> even
+
+
+def _dense_reference(x, W_r, Wg, Wu, Wd, k, norm, C, Ws=None, b=None):
+    """Dense mixture (every expert on every token) with masked weights,
+    written with numpy matrix products; the capacity mask is a brute-force
+    token-order count."""
+    x64 = x.astype(np.float64)
+    g = x64 @ W_r.astype(np.float64).T
+    if b is not None:
+        g = g + b.astype(np.float64)
+    p = _softmax_np(g)
+    N, E = g.shape
+    A = np.zeros((N, E))
+    used = np.zeros(E, int)
+    for t in range(N):
+        S = sorted(range(E), key=lambda e: (-g[t, e], e))[:k]
+        tot = p[t, S].sum()
+        for e in S:
+            if used[e] < C:
+                A[t, e] = p[t, e] / tot if norm == oracle.NORM_RENORM else p[t, e]
+            used[e] += 1
+    Y = np.zeros((N, x.shape[1]))
+    for e in range(E):
+        G = x64 @ Wg[e].astype(np.float64).T
+        U = x64 @ Wu[e].astype(np.float64).T
+        Hh = G / (1 + np.exp(-G)) * U
+        Y += A[:, e:e + 1] * (Hh @ Wd[e].astype(np.float64).T)
+    if Ws is not None:
+        G = x64 @ Ws[0].astype(np.float64).T
+        U = x64 @ Ws[1].astype(np.float64).T
+        Y += (G / (1 + np.exp(-G)) * U) @ Ws[2].astype(np.float64).T
+    return Y
+
+
+@pytest.mark.parametrize("norm,c,shared", [(0, 0.0, False), (0, 1.0, False), (1, 1.25, False),
+                                           (0, 0.0, True), (0, 0.75, True)])
+def test_forward_matches_dense_masked_evaluation(norm, c, shared):
+    rng = np.random.default_rng(4)
+    N, d, d_f, E, k = 23, 12, 10, 5, 2 if norm == 0 else 1
+    x = rng.standard_normal((N, d)).astype(np.float32)
+    W_r = (rng.standard_normal((E, d)) / math.sqrt(d)).astype(np.float32)
+    Wg = (rng.standard_normal((E, d_f, d)) / math.sqrt(d)).astype(np.float32)
+    Wu = (rng.standard_normal((E, d_f, d)) / math.sqrt(d)).astype(np.float32)
+    Wd = (rng.standard_normal((E, d, d_f)) / math.sqrt(d_f)).astype(np.float32)
+    Ws = None
+    if shared:
+        Ws = ((rng.standard_normal((7, d)) / math.sqrt(d)).astype(np.float32),
+              (rng.standard_normal((7, d)) / math.sqrt(d)).astype(np.float32),
+              (rng.standard_normal((d, 7)) / math.sqrt(7)).astype(np.float32))
+    b = rng.standard_normal(E).astype(np.float32)
+    out = oracle.forward(x, W_r, Wg, Wu, Wd, k=k, norm=norm, c=c, Ws=Ws, b_r=b)
+    C = oracle.capacity(c, N, k, E)
+    want = _dense_reference(x, W_r, Wg, Wu, Wd, k, norm, C, Ws=Ws, b=b)
+    np.testing.assert_allclose(out["Y"], want, rtol=1e-12, atol=1e-12)
+    if c > 0:
+        assert out["stats"]["rejected"] >= 0
+    # per-token recomputation from the routing records agrees with the batch path
+    toks = np.array([0, 7, 22])
+    rows = oracle.forward_rows(x, out["ids"], out["w"], out["slot"], toks, Wg, Wu, Wd, Ws=Ws)
+    np.testing.assert_allclose(rows, out["Y"][toks], rtol=1e-13, atol=1e-13)
+
+
+def test_forward_bf16_rounds_hidden_activation():
+    # bf16 storage: h is rounded to bf16 before the down projection.  With
+    # one token, one expert and d_f = 1 the output is round_bf16(h) * W_d.
+    x = f32_to_bf16_bits(np.array([[1.0]], np.float32))
+    W_r = f32_to_bf16_bits(np.array([[0.0]], np.float32))
+    Wg = f32_to_bf16_bits(np.array([[[1.0]]], np.float32))
+    Wu = f32_to_bf16_bits(np.array([[[1.0]]], np.float32))
+    Wd = f32_to_bf16_bits(np.array([[[1.0]]], np.float32))
+    out = oracle.forward(x, W_r, Wg, Wu, Wd, k=1, norm=oracle.NORM_RENORM)
+    h = 1.0 / (1.0 + math.exp(-1.0))                  # SiLU(1) * 1
+    want = float(bf16_bits_to_f32(f32_to_bf16_bits(np.array([h], np.float32)))[0])
+    assert out["Y"][0, 0] == want
+    assert out["Y"][0, 0] != h
+
+
+# ---------------------------------------------------------------------------
+# parameter arithmetic printed on the pages
+# ---------------------------------------------------------------------------
+def test_parameter_counts():
+    # vegetog sec. 4: Mixtral d=4096, m=14336, L=32, 8 experts, top-2
+    Pe, tot, act = oracle.param_counts(4096, 14336, 8, 2, L=32)
+    assert Pe == 176_160_768
+    assert round(tot / 1e9, 2) == 45.10 and round(act / 1e9, 2) == 11.27
+    # ch. 36.5: d=1024, d_f=4096, E_r=8, k=2
+    Pe, tot, act = oracle.param_counts(1024, 4096, 8, 2)
+    assert (Pe, tot, act) == (12_582_912, 100_663_296, 25_165_824)
+    assert tot * 2 == 201_326_592 and tot * 2 // 2 ** 20 == 192 and act * 2 // 2 ** 20 == 48
