@@ -1,0 +1,399 @@
+"""Benchmark of the sparse-MoE layer forward pass on B200.
+
+Default workload: the Mixtral-shaped bf16 layer (T = 4096 tokens, d = 4096,
+d_f = 14336, E_r = 8, k = 2, renormalised top-2, no capacity limit), seeded
+synthetic inputs.  One step = one moe_forward (router, softmax, top-k,
+dispatch, gate/up GEMM + SwiGLU, down GEMM + combine) over the batch.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle on the
+host cores on a bounded sample of the same workload.  Under torchrun each
+rank runs its own token batch (weak scaling; the uncapped layer needs no
+exchange between ranks), timed on the device, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import seeded_inputs as si  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s; achieved TFLOP/s or HBM GB/s as fraction of B200 peak"
+WORKLOAD = "mixtral_bf16"
+KERNELS_PER_STEP = 7  # router, hist, scan, assign, gather, gate/up GEMM, down GEMM + combine
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def rank_workload(w: si.Workload, rank: int) -> si.Workload:
+    """Each rank draws its own token batch (seeded by rank); weights are the
+    same on every rank (tensor streams other than x keep the base seed)."""
+    return w
+
+
+def rank_x_seed(w: si.Workload, rank: int) -> int:
+    return w.seed + 1000 * rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work of one step (the roofline numerators)
+# ---------------------------------------------------------------------------
+def gate_up_flops(w: si.Workload, accepted: int) -> float:
+    """2 * A * d * (2 d_f) for the routed rows, plus the shared expert's N rows."""
+    f = 2.0 * accepted * w.d * 2 * w.d_f
+    if w.d_f_shared:
+        f += 2.0 * w.N * w.d * 2 * w.d_f_shared
+    return f
+
+
+def step_flops(w: si.Workload, accepted: int) -> float:
+    """Router 2 N d E_r + experts 2 A 3 d d_f + shared 2 N 3 d d_sh (p2 ch. 36.5 cost model)."""
+    f = 2.0 * w.N * w.d * w.E + 2.0 * accepted * 3 * w.d * w.d_f
+    if w.d_f_shared:
+        f += 2.0 * w.N * 3 * w.d * w.d_f_shared
+    return f
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    p = os.path.join(ROOT, "sparse_mixture_experts_25_b200", "csrc", "gemm_tc.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
+    None when the kernel source changed since the counters were taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        ent = t.get(kernel)
+        if ent and ent.get("source_sha256_16") == kernel_source_hash() and ent.get("workload") == WORKLOAD:
+            return ent.get("bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.out = out
+        return False
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle leg (the reference arm and the cpu_baseline key)
+# ---------------------------------------------------------------------------
+def oracle_sample(w: si.Workload, inp: dict, sample_tokens: int = 32):
+    """Times the oracle on a bounded sample: routing and dispatch of the whole
+    batch, and the expert outputs of `sample_tokens` tokens; returns the
+    extrapolated whole-batch tokens/s and a description."""
+    import oracle
+    t0 = time.perf_counter()
+    r = oracle.route(inp["x"], inp["W_r"], k=w.k, norm=w.norm, theta=w.theta, b_r=inp.get("b_r"),
+                     lat=inp.get("lat"))
+    C = oracle.capacity(w.c, w.N, w.k, w.E)
+    d = oracle.dispatch(r["ids"], E=w.E, C=C)
+    t1 = time.perf_counter()
+    toks = np.linspace(0, w.N - 1, sample_tokens).astype(np.int64)
+    Ws = (inp.get("Ws_g"), inp.get("Ws_u"), inp.get("Ws_d")) if w.d_f_shared else None
+    oracle.forward_rows(inp["x"], r["ids"], r["w"], d["slot"], toks, inp["W_g"], inp["W_u"], inp["W_d"], Ws=Ws)
+    t2 = time.perf_counter()
+    per_batch = (t1 - t0) + (t2 - t1) * w.N / sample_tokens
+    cores = si.host_threads()
+    return {"value": w.N / per_batch, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"routing+dispatch of all {w.N} tokens ({t1 - t0:.2f} s) and expert outputs "
+                       f"of {sample_tokens} tokens ({t2 - t1:.2f} s), extrapolated to {w.N} tokens"),
+            "seconds": t2 - t0}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = si.WORKLOADS[args.workload]
+    inp = si.inputs(w)
+    steps = []
+    for i in range(args.warmup + args.steps):
+        s = oracle_sample(w, inp, sample_tokens=args.ref_sample)
+        if i >= args.warmup:
+            steps.append(s)
+    val = statistics.median([s["value"] for s in steps])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * w.N / val,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, args),
+        "cpu_baseline": {k: steps[-1][k] for k in ("kind", "cores", "sample")} | {"value": val, "unit": "tokens/s"},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w: si.Workload, args):
+    return {"workload": f"{w.name}: T={w.N} d={w.d} d_f={w.d_f} E_r={w.E} k={w.k}",
+            "T": w.N, "d": w.d, "d_f": w.d_f, "E_r": w.E, "k": w.k,
+            "norm": ["renorm", "fullprob", "wlr"][w.norm], "capacity_factor": w.c or None,
+            "d_f_shared": w.d_f_shared, "seed": w.seed,
+            "parallelism": f"dp{args.gpus} (independent token batches per GPU)",
+            "l2": "inputs larger than L2 (expert weights 2.8 GB stream from HBM every step)"}
+
+
+# ---------------------------------------------------------------------------
+# GPU leg
+# ---------------------------------------------------------------------------
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    ws_n, rank, local = dist_env()
+    w = si.WORKLOADS[args.workload]
+    # host-side inputs (generated before any CUDA call; the oracle leg below
+    # uses the same buffers)
+    inp = si.inputs(w)
+    if rank:
+        inp["x"] = si.fill(rank_x_seed(w, rank), si.TID["x"], w.N * w.d, dtype=w.dt).reshape(w.N, w.d)
+    cpu_base = None
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        cpu_base = oracle_sample(w, inp, sample_tokens=args.ref_sample)
+
+    torch.cuda.set_device(local)
+    if ws_n > 1:
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    import sparse_mixture_experts_25_b200 as moe
+
+    def dev(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+    d = {k: dev(v) for k, v in inp.items()}
+    p = moe.params(w.N, w.d, w.d_f, w.E, w.k, c=w.c, norm=w.norm, theta=w.theta, dtype=w.dtype,
+                   d_f_shared=w.d_f_shared)
+    wsb = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+    Y = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(x_dev, y_dev):
+        moe.moe_forward(p, x_dev, d["W_r"], d["b_r"], d["lat"], d["W_g"], d["W_u"], d["W_d"],
+                        d["Ws_g"], d["Ws_u"], d["Ws_d"], y_dev, wsb, stream)
+
+    for _ in range(args.warmup):
+        step(d["x"], Y)
+    torch.cuda.synchronize()
+    status, stats = moe.moe_get_stats(p, wsb)
+    if status != moe.MOE_OK:
+        raise RuntimeError(f"moe_forward status: {moe.moe_status_string(status)}")
+    accepted = int(stats["accepted"])
+
+    # device-timed steps, inputs resident in HBM; stage events around each kernel group
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws_n > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        start.record(stream)
+        for i in range(args.steps):
+            moe.moe_set_stage_events(ev[i])
+            step(d["x"], Y)
+        moe.moe_set_stage_events([])
+        end.record(stream)
+        torch.cuda.synchronize()
+        time.sleep(0.2)
+    if ws_n > 1:
+        dist.barrier()
+    ms_total = start.elapsed_time(end)
+    ms_total = max_over_ranks(ms_total, device="cuda")
+    ms_step = ms_total / args.steps
+    stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(4)] for i in range(args.steps)])
+    gate_up_ms = float(stage_ms[:, 2].mean())
+    down_ms = float(stage_ms[:, 3].mean())
+
+    # end to end through the public API: pinned host x -> device, forward, Y -> pinned host
+    x_host = torch.from_numpy(np.ascontiguousarray(inp["x"]).view(np.int16)).view(torch.bfloat16) \
+        if w.dtype == si.DT_BF16 else torch.from_numpy(inp["x"])
+    x_host = x_host.pin_memory()
+    y_host = torch.empty(w.N, w.d, dtype=torch.float32).pin_memory()
+    x_dev2 = torch.empty_like(d["x"])
+    for _ in range(2):
+        x_dev2.copy_(x_host, non_blocking=True)
+        step(x_dev2, Y)
+        y_host.copy_(Y, non_blocking=True)
+    torch.cuda.synchronize()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws_n > 1:
+        dist.barrier()
+    e_start.record(stream)
+    for _ in range(args.steps):
+        x_dev2.copy_(x_host, non_blocking=True)
+        step(x_dev2, Y)
+        y_host.copy_(Y, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e_start.elapsed_time(e_end), device="cuda") / args.steps
+
+    peaks, peak_src = load_peaks()
+    timed_s = ms_total / 1000.0
+    if timed_s < 1.0:
+        peak_tf, peak_kind = peaks["bf16_tflops"], "burst"
+    else:
+        peak_tf, peak_kind = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), "sustained"
+    gu_flops = gate_up_flops(w, accepted)
+    achieved = gu_flops / (gate_up_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": ws_n * w.N / (ms_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": ws_n,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == si.DT_BF16 else "f32",
+        "data": "synthetic (seeded SplitMix64/Box-Muller; x~N(0,1), W~N(0,1/fan_in)); no dataset or checkpoint",
+        "config": config_of(w, args),
+        "roofline": {
+            "kernel": "tc_grouped_kernel<SWIGLU> (gate/up GEMM + SwiGLU)",
+            "bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+            "frac": achieved / peak_tf, "traffic": committed_traffic("gate_up"),
+            "peak_source": f"{peak_src} bf16 {peak_kind}",
+            "flops_per_launch": gu_flops, "avg_launch_ms": gate_up_ms,
+        },
+        "stages_ms": {"route": float(stage_ms[:, 0].mean()), "dispatch": float(stage_ms[:, 1].mean()),
+                      "gate_up": gate_up_ms, "down_combine": down_ms},
+        "step_tflops": step_flops(w, accepted) / (ms_step * 1e-3) / 1e12,
+        "down_tflops": 2.0 * accepted * w.d * w.d_f / (down_ms * 1e-3) / 1e12,
+        "e2e": {"value": ws_n * w.N / (e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
+                "ms_per_step": e_ms},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+        "routing": {k: stats[k] for k in ("accepted", "rejected", "near_tie", "L_max", "rho_max")},
+    }
+    if cpu_base is not None:
+        line["cpu_baseline"] = {k: cpu_base[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws_n > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(si.WORKLOADS))
+    ap.add_argument("--ref-sample", type=int, default=32)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

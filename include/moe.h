@@ -1,0 +1,241 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) sparse Mixture-of-Experts layer
+ * forward pass: router, softmax, top-k, weighting, capacity-limited
+ * token-order dispatch, SwiGLU experts, optional shared expert, weighted
+ * combine.
+ *
+ * Notation follows the pages' notation table ("LLM from scratch" ch. 36.1):
+ * N tokens in the routing group, model width d, expert hidden width d_f,
+ * E_r routed experts, k experts per token, capacity factor c (gamma on that
+ * page), router W_r and bias b_r, routing weights a_te, requested load n_e
+ * (L_e in the auturnal review), capacity C_e, expert outputs H_e, output Y.
+ *
+ * Conventions for every entry point
+ *  - Memory: every pointer argument is DEVICE memory unless marked "host".
+ *    The caller allocates and owns all buffers, including the workspace
+ *    (size from moe_workspace_size).  The library never allocates device
+ *    memory and never frees caller memory.
+ *  - Execution: every call enqueues its kernels on `stream` and returns
+ *    without waiting, except moe_get_stats, which waits for the stream.
+ *    Host-side argument checks return synchronously; a non-MOE_OK status
+ *    means nothing was enqueued (except MOE_ERR_CUDA: a launch failed).
+ *  - Layout: row-major.  Weights are stored output-major ("K-major"), the
+ *    transposes of the pages' x W convention, which ch. 36.8 of
+ *    "LLM from scratch" names an allowed transposition:
+ *      W_r [E_r, d]; W_g, W_u [E_r, d_f, d]; W_d [E_r, d, d_f];
+ *      shared Ws_g, Ws_u [d_f_shared, d]; Ws_d [d, d_f_shared].
+ *    Element type of x and all weights: params.dtype (fp32, or bf16 stored
+ *    as raw 16-bit patterns).  b_r, lat, routing weights and Y are fp32.
+ *  - Alignment: device pointers to x, weights, x_perm, H and the workspace
+ *    must be 16-byte aligned (256 recommended); d and d_f must be multiples
+ *    of 8, else MOE_ERR_UNSUPPORTED.
+ *  - Threads: calls on different streams with different workspaces may run
+ *    concurrently; one workspace must not be shared by calls in flight.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t.  NULL selects the legacy default stream. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* a size, mode or pointer violates the contract */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels implement */
+    MOE_ERR_NONFINITE = 3,    /* a router score (or WLR latency) was not finite */
+    MOE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    MOE_ERR_WORKSPACE = 5,    /* workspace missing or too small / misaligned */
+    MOE_ERR_TIMEOUT = 6       /* a bounded device wait gave up (kernel fault guard) */
+} moe_status;
+
+/* Weighting of the chosen experts ("LLM from scratch" ch. 36.2; WDMoE note). */
+typedef enum moe_norm {
+    MOE_NORM_RENORM = 0,   /* a_te = p_te / sum_{j in S_t} p_tj  (sums to 1)        */
+    MOE_NORM_FULLPROB = 1, /* a_te = p_te, the full-softmax probability (Switch)   */
+    MOE_NORM_WLR = 2       /* WDMoE weight-latency-ratio pruning with threshold theta,
+                              then softmax over the surviving scores               */
+} moe_norm;
+
+typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef struct moe_params {
+    int64_t N;          /* tokens in the routing group, N >= 0                      */
+    int32_t d;          /* model width                                               */
+    int32_t d_f;        /* routed expert hidden width                                */
+    int32_t E_r;        /* routed experts, 1..1024                                   */
+    int32_t k;          /* experts per token, 1 <= k <= min(E_r, 32)                 */
+    double c;           /* capacity factor; c <= 0 means no limit (C = N)            */
+    int32_t norm;       /* moe_norm                                                  */
+    float theta;        /* WLR threshold in [0, 1) (MOE_NORM_WLR only)               */
+    int32_t dtype;      /* moe_dtype of x and of every weight                        */
+    int32_t d_f_shared; /* hidden width of the always-on shared expert; 0 = none     */
+} moe_params;
+
+/* Routing statistics of the last moe_dispatch / moe_forward on a workspace
+ * ("LLM from scratch" ch. 36.4 load statistics and Algorithm 36.1 outputs;
+ * auturnal review equations for O and rho_max). */
+typedef struct moe_stats {
+    int64_t C;               /* capacity used                                     */
+    int64_t requested;       /* sum_e L_e (paths that asked for an expert)        */
+    int64_t accepted;        /* paths given a slot                                */
+    int64_t rejected;        /* requested - accepted                              */
+    int64_t O;               /* sum_e max(0, L_e - C)                             */
+    int64_t tokens_affected; /* tokens with at least one rejected path            */
+    int64_t tokens_skipped;  /* tokens whose every requested path was rejected    */
+    int64_t nonfinite;       /* tokens whose scores were not finite (no paths)    */
+    int64_t near_tie;        /* tokens whose k-th vs (k+1)-th score margin < 1e-5 */
+    int64_t L_max, L_p50, L_p90, L_p99; /* requested load: max, nearest-rank pct  */
+    double rho_max;          /* max_e L_e / (N k / E_r)                           */
+    double reject_rate;      /* rejected / requested                              */
+    int32_t device_error;    /* nonzero: a bounded device wait timed out          */
+    int32_t reserved;
+} moe_stats;
+
+/* Byte offsets of the regions inside the workspace (for inspection and
+ * tests; every region is 256-byte aligned). */
+typedef struct moe_ws_layout {
+    size_t ids;        /* int32 [N, k]  chosen expert per rank, -1 = none         */
+    size_t w;          /* fp32  [N, k]  weight a_te                                */
+    size_t margin;     /* fp32  [N]     score margin g_(k) - g_(k+1)               */
+    size_t slot;       /* int32 [N, k]  slot in the expert buffer, -1 = rejected   */
+    size_t offsets;    /* int32 [E_r+1] start row of each expert's accepted rows   */
+    size_t L;          /* int32 [E_r]   requested load per expert                  */
+    size_t acc;        /* int32 [E_r]   accepted rows per expert                   */
+    size_t slot_token; /* int32 [N k]   token of each accepted row                 */
+    size_t slot_w;     /* fp32  [N k]   weight of each accepted row                */
+    size_t counters;   /* int64 [16]    device counters                            */
+    size_t x_perm;     /* dtype [N k, d] gathered expert inputs                    */
+    size_t h;          /* dtype [N k, d_f] expert hidden activations               */
+    size_t h_shared;   /* dtype [N, d_f_shared]                                    */
+    size_t scratch;    /* internal                                                 */
+    size_t total;      /* bytes required                                           */
+} moe_ws_layout;
+
+/* Capacity C = ceil(c N k / E_r) (auturnal review, C_e equation; "LLM from
+ * scratch" ch. 36.3 capacity rule; vegetog sec. 6 example), on the exact
+ * value of c, taking an integer within 1e-9 (relative) of c N k / E_r as
+ * exact.  c <= 0 gives C = N.  *C is host memory. */
+MOE_API moe_status moe_capacity(const moe_params* p, int64_t* C);
+
+/* Bytes of device workspace that moe_route/moe_dispatch/moe_expert_ffn/
+ * moe_forward need for these params (host call, no device work). */
+MOE_API moe_status moe_workspace_size(const moe_params* p, size_t* bytes);
+
+/* Region offsets inside the workspace (host call). */
+MOE_API moe_status moe_workspace_layout(const moe_params* p, moe_ws_layout* out);
+
+/*
+ * Router scores G = x W_r^T + b_r, softmax over experts, top-k with ties to
+ * the lower expert index, and weights by params.norm ("LLM from scratch"
+ * ch. 36.1-36.2 and Algorithm 36.1 steps 1-2; vegetog sec. 2; WDMoE note).
+ *   x   [N, d] dtype;  W_r [E_r, d] dtype;  b_r [E_r] fp32 or NULL
+ *   lat [N, E_r] fp32 per-token per-expert latency t = t_up + t_comp + t_down,
+ *       required for MOE_NORM_WLR, ignored otherwise
+ * Outputs (rank order j = 0..k-1, score descending):
+ *   ids [N, k] int32 expert, -1 for a path pruned by WLR or an invalid token
+ *   w   [N, k] fp32 weight a_te (0 where ids = -1)
+ *   margin [N] fp32 g_(k) - g_(k+1) (+inf if k = E_r; NaN if invalid), nullable
+ * Scores are accumulated in fp32.  A token with a non-finite score (or,
+ * under WLR, a chosen expert whose latency is not a positive number) gets no
+ * paths and is counted in the workspace counters (MOE_ERR_NONFINITE from
+ * moe_get_stats).  ws: workspace of moe_workspace_size bytes.
+ */
+MOE_API moe_status moe_route(const moe_params* p, const void* x, const void* W_r, const float* b_r,
+                     const float* lat, int32_t* ids, float* w, float* margin, void* ws,
+                     moe_stream_t stream);
+
+/*
+ * Capacity check and dispatch (Algorithm 36.1 steps 3-4; ch. 36.3 dispatch
+ * matrix D_e as index lists and prefix sums).  Requests are taken in token
+ * order t = 0..N-1: path (t, e) gets slot c = number of earlier requests for
+ * e, and is accepted iff c < C.  Deterministic (a stable counting sort).
+ *   ids, w     [N, k] from moe_route (ids -1 = no request)
+ *   C          capacity, >= 1 (see moe_capacity)
+ *   slot       [N, k] int32 out: slot, or -1 if rejected / not requested
+ *   offsets    [E_r + 1] int32 out: accepted rows of expert e are rows
+ *              offsets[e] .. offsets[e+1]-1 of the expert buffers, in slot order
+ *   slot_token [N k] int32 out: source token of each accepted row
+ *   slot_w     [N k] fp32 out: weight a_te of each accepted row
+ *   x          [N, d] dtype, nullable; with x_perm [N k, d] dtype, gathers
+ *              x_perm[r] = x[slot_token[r]] for every accepted row r
+ * Statistics (L_e, accepted, O, ...) go to the workspace counters.
+ */
+MOE_API moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const float* w, int64_t C,
+                        int32_t* slot, int32_t* offsets, int32_t* slot_token, float* slot_w,
+                        const void* x, void* x_perm, void* ws, moe_stream_t stream);
+
+/*
+ * Routed SwiGLU experts on the dispatched rows (vegetog sec. 3:
+ * E_i(x) = [SiLU(x W_gate,i) (.) (x W_up,i)] W_down,i; ch. 36.3: each expert
+ * runs only on its accepted slots).
+ *   x_perm  [N k, d] dtype (rows offsets[e] .. offsets[e+1]-1 belong to e)
+ *   offsets [E_r + 1] from moe_dispatch
+ *   H       [N k, d] fp32 out: H[r] = E_e(x_perm[r]) for r < offsets[E_r]
+ * bf16 layers keep h = SiLU(.)(.)(.) in bf16 and accumulate in fp32; fp32
+ * layers compute in fp32 throughout (no TF32).
+ */
+MOE_API moe_status moe_expert_ffn(const moe_params* p, const void* x_perm, const int32_t* offsets,
+                          const void* W_g, const void* W_u, const void* W_d, float* H, void* ws,
+                          moe_stream_t stream);
+
+/*
+ * Weighted combine (Algorithm 36.1 last step; ch. 36.3 combine matrix A_e):
+ * Y[slot_token[r]] += slot_w[r] * H[r] for every accepted row r.  Y [N, d]
+ * fp32 is accumulated into (the caller zeroes it first); rejected paths add
+ * nothing and weights are not renormalised.  Summation order is free (fp32
+ * atomics).
+ */
+MOE_API moe_status moe_combine(const moe_params* p, const float* H, const int32_t* offsets,
+                       const int32_t* slot_token, const float* slot_w, float* Y,
+                       moe_stream_t stream);
+
+/*
+ * The whole layer: route, dispatch, experts and combine, with the combine
+ * fused into the down-projection epilogue, plus the shared expert
+ * (ch. 36.6; DeepSeek-V3 form y = FFN_shared(x) + sum_i g_i FFN_i(x)) when
+ * params.d_f_shared > 0.  Y [N, d] fp32 is overwritten.  Routing records
+ * and statistics stay in the workspace (moe_workspace_layout, moe_get_stats).
+ * Ws_g/Ws_u/Ws_d are required when d_f_shared > 0 and ignored otherwise.
+ */
+MOE_API moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, const float* b_r,
+                       const float* lat, const void* W_g, const void* W_u, const void* W_d,
+                       const void* Ws_g, const void* Ws_u, const void* Ws_d, float* Y, void* ws,
+                       moe_stream_t stream);
+
+/*
+ * Reads the routing statistics of the last dispatch on this workspace into
+ * *out (host memory); waits for `stream`.  Returns MOE_ERR_NONFINITE when a
+ * token had non-finite scores, MOE_ERR_TIMEOUT when a device wait gave up,
+ * else MOE_OK (out is filled in every case).
+ */
+MOE_API moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, moe_stream_t stream);
+
+/*
+ * Optional stage timing for moe_forward on the calling host thread: with
+ * n >= 5 events (cudaEvent_t handles created by the caller), the next
+ * moe_forward calls record events[0] before the router, [1] after routing,
+ * [2] after dispatch, [3] after the gate/up expert GEMM and [4] after the
+ * down-projection + combine, on the call's stream.  n = 0 turns it off.
+ */
+MOE_API moe_status moe_set_stage_events(void* const* events, int n);
+
+/* Static description of a status code. */
+MOE_API const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -1,0 +1,220 @@
+"""Python binding of libmoe, the B200 (sm_100a) sparse-MoE layer forward pass.
+
+Argument marshalling only: every function here passes device pointers of
+torch tensors (torch is used for device memory and streams) and the current
+CUDA stream to the C ABI declared in include/moe.h, under the same names.
+All computation runs in the library's CUDA kernels.  There is no fallback:
+if libmoe.so cannot be built or loaded, importing this package fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+from . import build as _build
+
+__all__ = [
+    "MoEError", "Params", "Stats", "WsLayout", "lib", "params", "moe_capacity",
+    "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_dispatch",
+    "moe_expert_ffn", "moe_combine", "moe_forward", "moe_get_stats",
+    "moe_set_stage_events", "moe_status_string", "workspace_views", "HEADER",
+]
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_NONFINITE = 0, 1, 2, 3
+MOE_ERR_CUDA, MOE_ERR_WORKSPACE, MOE_ERR_TIMEOUT = 4, 5, 6
+MOE_NORM_RENORM, MOE_NORM_FULLPROB, MOE_NORM_WLR = 0, 1, 2
+MOE_F32, MOE_BF16 = 0, 1
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {moe_status_string(status)} (status {status})")
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("d", ctypes.c_int32), ("d_f", ctypes.c_int32),
+                ("E_r", ctypes.c_int32), ("k", ctypes.c_int32), ("c", ctypes.c_double),
+                ("norm", ctypes.c_int32), ("theta", ctypes.c_float), ("dtype", ctypes.c_int32),
+                ("d_f_shared", ctypes.c_int32)]
+
+
+class Stats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "C", "requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped",
+        "nonfinite", "near_tie", "L_max", "L_p50", "L_p90", "L_p99")] + [
+        ("rho_max", ctypes.c_double), ("reject_rate", ctypes.c_double),
+        ("device_error", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_ if n != "reserved"}
+
+
+_LAYOUT_FIELDS = ("ids", "w", "margin", "slot", "offsets", "L", "acc", "slot_token", "slot_w",
+                  "counters", "x_perm", "h", "h_shared", "scratch", "total")
+
+
+class WsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in _LAYOUT_FIELDS]
+
+
+_P = ctypes.c_void_p
+_lib = None
+
+
+def lib():
+    """Load (building first if missing or stale) the in-tree libmoe.so."""
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        pp = ctypes.POINTER(Params)
+        L.moe_capacity.argtypes = [pp, ctypes.POINTER(ctypes.c_int64)]
+        L.moe_workspace_size.argtypes = [pp, ctypes.POINTER(ctypes.c_size_t)]
+        L.moe_workspace_layout.argtypes = [pp, ctypes.POINTER(WsLayout)]
+        L.moe_route.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_dispatch.argtypes = [pp, _P, _P, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_expert_ffn.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_combine.argtypes = [pp, _P, _P, _P, _P, _P, _P]
+        L.moe_forward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_get_stats.argtypes = [pp, _P, ctypes.POINTER(Stats), _P]
+        L.moe_set_stage_events.argtypes = [ctypes.POINTER(_P), ctypes.c_int]
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_status_string.restype = ctypes.c_char_p
+        for name in ("moe_capacity", "moe_workspace_size", "moe_workspace_layout", "moe_route",
+                     "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
+                     "moe_get_stats", "moe_set_stage_events"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def declared_symbols():
+    """Entry points declared in include/moe.h."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def params(N, d, d_f, E_r, k, c=0.0, norm=MOE_NORM_RENORM, theta=0.0, dtype=MOE_BF16,
+           d_f_shared=0) -> Params:
+    return Params(int(N), int(d), int(d_f), int(E_r), int(k), float(c), int(norm), float(theta),
+                  int(dtype), int(d_f_shared))
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("libmoe takes device tensors; got a host tensor")
+    if not t.is_contiguous():
+        raise ValueError("libmoe takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoEError(status, where)
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def moe_capacity(p: Params) -> int:
+    C = ctypes.c_int64()
+    _check(lib().moe_capacity(ctypes.byref(p), ctypes.byref(C)), "moe_capacity")
+    return C.value
+
+
+def moe_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().moe_workspace_size(ctypes.byref(p), ctypes.byref(n)), "moe_workspace_size")
+    return n.value
+
+
+def moe_workspace_layout(p: Params) -> dict:
+    L = WsLayout()
+    _check(lib().moe_workspace_layout(ctypes.byref(p), ctypes.byref(L)), "moe_workspace_layout")
+    return {n: getattr(L, n) for n in _LAYOUT_FIELDS}
+
+
+def moe_route(p, x, W_r, b_r, lat, ids, w, margin, ws, stream=None):
+    _check(lib().moe_route(ctypes.byref(p), _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(lat), _ptr(ids),
+                           _ptr(w), _ptr(margin), _ptr(ws), _stream(stream)), "moe_route")
+
+
+def moe_dispatch(p, ids, w, C, slot, offsets, slot_token, slot_w, x, x_perm, ws, stream=None):
+    _check(lib().moe_dispatch(ctypes.byref(p), _ptr(ids), _ptr(w), int(C), _ptr(slot), _ptr(offsets),
+                              _ptr(slot_token), _ptr(slot_w), _ptr(x), _ptr(x_perm), _ptr(ws),
+                              _stream(stream)), "moe_dispatch")
+
+
+def moe_expert_ffn(p, x_perm, offsets, W_g, W_u, W_d, H, ws, stream=None):
+    _check(lib().moe_expert_ffn(ctypes.byref(p), _ptr(x_perm), _ptr(offsets), _ptr(W_g), _ptr(W_u),
+                                _ptr(W_d), _ptr(H), _ptr(ws), _stream(stream)), "moe_expert_ffn")
+
+
+def moe_combine(p, H, offsets, slot_token, slot_w, Y, stream=None):
+    _check(lib().moe_combine(ctypes.byref(p), _ptr(H), _ptr(offsets), _ptr(slot_token), _ptr(slot_w),
+                             _ptr(Y), _stream(stream)), "moe_combine")
+
+
+def moe_forward(p, x, W_r, b_r, lat, W_g, W_u, W_d, Ws_g, Ws_u, Ws_d, Y, ws, stream=None):
+    _check(lib().moe_forward(ctypes.byref(p), _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(lat), _ptr(W_g),
+                             _ptr(W_u), _ptr(W_d), _ptr(Ws_g), _ptr(Ws_u), _ptr(Ws_d), _ptr(Y),
+                             _ptr(ws), _stream(stream)), "moe_forward")
+
+
+def moe_get_stats(p, ws, stream=None):
+    """Returns (status, stats dict); waits for the stream."""
+    s = Stats()
+    status = lib().moe_get_stats(ctypes.byref(p), _ptr(ws), ctypes.byref(s), _stream(stream))
+    if status not in (MOE_OK, MOE_ERR_NONFINITE, MOE_ERR_TIMEOUT):
+        raise MoEError(status, "moe_get_stats")
+    return status, s.as_dict()
+
+
+def moe_set_stage_events(events):
+    """events: list of torch.cuda.Event(enable_timing=True) (>= 5) or [] to stop."""
+    n = len(events)
+    arr = (_P * max(n, 1))(*[e.cuda_event for e in events])
+    _check(lib().moe_set_stage_events(arr if n else None, n), "moe_set_stage_events")
+
+
+def workspace_views(p: Params, ws):
+    """Typed torch views of the routing records inside a workspace tensor."""
+    import torch
+    L = moe_workspace_layout(p)
+    N, k, E = p.N, p.k, p.E_r
+
+    def view(name, count, dtype, shape):
+        nbytes = count * torch.empty((), dtype=dtype).element_size()
+        return ws[L[name]:L[name] + nbytes].view(dtype).view(*shape)
+
+    return {
+        "ids": view("ids", N * k, torch.int32, (N, k)),
+        "w": view("w", N * k, torch.float32, (N, k)),
+        "margin": view("margin", N, torch.float32, (N,)),
+        "slot": view("slot", N * k, torch.int32, (N, k)),
+        "offsets": view("offsets", E + 1, torch.int32, (E + 1,)),
+        "L": view("L", E, torch.int32, (E,)),
+        "acc": view("acc", E, torch.int32, (E,)),
+        "slot_token": view("slot_token", N * k, torch.int32, (N * k,)),
+        "slot_w": view("slot_w", N * k, torch.float32, (N * k,)),
+    }

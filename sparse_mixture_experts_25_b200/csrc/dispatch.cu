@@ -1,0 +1,284 @@
+// Capacity check, token-order dispatch and the row gather.
+//
+// What it computes (Algorithm 36.1 steps 3-4 of "LLM from scratch" ch. 36;
+// ch. 36.3 dispatch matrices D_e as index lists and prefix sums; auturnal
+// review equations for O and rho_max): paths (t, e) are taken in token order;
+// path (t, e) gets slot c = number of earlier requests for e and is accepted
+// iff c < C.
+//
+// Design: a stable counting sort in three short launches, with no cross-CTA
+// waiting:
+//   hist   one CTA per tile of tokens counts its requests per expert
+//          (shared-memory atomics; order does not matter for counts);
+//   scan   one CTA turns the [E][tiles] counts into exclusive per-tile bases
+//          (one warp per expert, warp-wide scans), then scans the accepted
+//          counts min(L_e, C) over experts into row offsets and the M-tile
+//          prefix used by the grouped GEMMs, and writes the statistics;
+//   assign one warp per tile walks its requests in token order, 32 at a
+//          time; __match_any_sync groups equal experts so a lane's slot is
+//          base + running count + its rank among earlier equal lanes.
+// gather then copies x rows into the per-expert row buffer with 16-byte
+// vector loads (HBM-bound, coalesced along each row).
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    return v;
+}
+
+// Exclusive scan over blockDim.x (<= 1024, multiple of 32) values; returns
+// the exclusive prefix and writes the block total to *total (all threads).
+__device__ int block_excl_scan(int v, int* warp_tot, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int inc = warp_incl_scan(v, lane);
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const int wv = lane < nw ? warp_tot[lane] : 0;
+        const int wi = warp_incl_scan(wv, lane);
+        if (lane < nw) warp_tot[lane] = wi - wv;
+        if (lane == 31) warp_tot[32] = wi;
+    }
+    __syncthreads();
+    const int ex = inc - v + warp_tot[warp];
+    *total = warp_tot[32];
+    __syncthreads();
+    return ex;
+}
+
+__global__ void hist_kernel(const int32_t* __restrict__ ids, int64_t N, int k, int E,
+                            int tile_tokens, int n_tiles, int32_t* __restrict__ hist,
+                            unsigned long long* counters) {
+    extern __shared__ int h[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    __syncthreads();
+    const int64_t t0 = (int64_t)blockIdx.x * tile_tokens;
+    const int64_t t1 = min64(N, t0 + tile_tokens);
+    bool oob = false;
+    for (int64_t i = t0 * k + threadIdx.x; i < t1 * k; i += blockDim.x) {
+        const int e = ids[i];
+        if (e >= 0 && e < E) atomicAdd(&h[e], 1);
+        else if (e >= E) oob = true;
+    }
+    if (oob) atomicOr(reinterpret_cast<unsigned long long*>(counters + CNT_DEVICE_ERROR), (unsigned long long)DEVERR_BOUNDS);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)e * n_tiles + blockIdx.x] = h[e];
+}
+
+__global__ void scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int64_t C, int bm,
+                            int32_t* __restrict__ L, int32_t* __restrict__ acc,
+                            int32_t* __restrict__ offsets, int32_t* __restrict__ mt_start,
+                            unsigned long long* counters) {
+    __shared__ int sL[kMaxExperts];
+    __shared__ int warp_tot[33];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int e = warp; e < E; e += nw) {
+        int run = 0;
+        int32_t* row = hist + (int64_t)e * n_tiles;
+        for (int b = 0; b < n_tiles; b += 32) {
+            const int i = b + lane;
+            const int v = i < n_tiles ? row[i] : 0;
+            const int inc = warp_incl_scan(v, lane);
+            if (i < n_tiles) row[i] = run + inc - v;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) sL[e] = run;
+    }
+    __syncthreads();
+    // one thread per expert (blockDim.x >= E)
+    const int e = threadIdx.x;
+    const int Le = e < E ? sL[e] : 0;
+    const int a = e < E ? (int)min64(Le, C) : 0;
+    const int mt = (a + bm - 1) / bm;
+    int tot_a, tot_mt, tot_L, tot_O;
+    const int ex_a = block_excl_scan(a, warp_tot, &tot_a);
+    const int ex_mt = block_excl_scan(mt, warp_tot, &tot_mt);
+    block_excl_scan(Le, warp_tot, &tot_L);
+    block_excl_scan(Le > C ? (int)(Le - C) : 0, warp_tot, &tot_O);
+    if (e < E) {
+        L[e] = Le;
+        acc[e] = a;
+        offsets[e] = ex_a;
+        mt_start[e] = ex_mt;
+        atomicMax(counters + CNT_L_MAX, (unsigned long long)Le);
+    }
+    if (threadIdx.x == 0) {
+        offsets[E] = tot_a;
+        mt_start[E] = tot_mt;
+        counters[CNT_REQUESTED] = (unsigned long long)tot_L;
+        counters[CNT_ACCEPTED] = (unsigned long long)tot_a;
+        counters[CNT_REJECTED] = (unsigned long long)(tot_L - tot_a);
+        counters[CNT_O] = (unsigned long long)tot_O;
+        counters[CNT_C] = (unsigned long long)C;
+    }
+}
+
+__global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w,
+                              int64_t N, int k, int E, int64_t C, int tile_tokens, int n_tiles,
+                              const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets,
+                              int32_t* __restrict__ slot, int32_t* __restrict__ slot_token,
+                              float* __restrict__ slot_w, unsigned long long* counters) {
+    extern __shared__ int run[];
+    const int lane = threadIdx.x;
+    const int tile = blockIdx.x;
+    for (int e = lane; e < E; e += 32) run[e] = hist[(int64_t)e * n_tiles + tile];
+    __syncwarp();
+    const int64_t tb = (int64_t)tile * tile_tokens;
+    const int64_t te = min64(N, tb + tile_tokens);
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int64_t base = tb * k; base < te * k; base += 32) {
+        const int64_t i = base + lane;
+        const bool valid = i < te * k;
+        int e = valid ? ids[i] : -1;
+        if (e >= E || e < 0) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(peers & lt_mask);
+        const int s = e >= 0 ? run[e] + rank : -1;
+        __syncwarp();
+        if (e >= 0 && lane == 31 - __clz(peers)) run[e] += __popc(peers);
+        __syncwarp();
+        if (valid) {
+            if (e >= 0 && s < C) {
+                const int64_t pos = (int64_t)offsets[e] + s;
+                slot_token[pos] = (int32_t)(i / k);
+                slot_w[pos] = w[i];
+                slot[i] = s;
+            } else {
+                slot[i] = -1;
+            }
+        }
+    }
+    __syncwarp();
+    unsigned long long affected = 0, skipped = 0;
+    for (int64_t t = tb + lane; t < te; t += 32) {
+        int req = 0, rej = 0;
+        for (int j = 0; j < k; ++j) {
+            const int e = ids[t * k + j];
+            if (e >= 0 && e < E) {
+                ++req;
+                if (slot[t * k + j] < 0) ++rej;
+            }
+        }
+        affected += rej > 0;
+        skipped += (req > 0 && rej == req);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        affected += __shfl_xor_sync(0xffffffffu, affected, o);
+        skipped += __shfl_xor_sync(0xffffffffu, skipped, o);
+    }
+    if (lane == 0) {
+        if (affected) atomicAdd(counters + CNT_AFFECTED, affected);
+        if (skipped) atomicAdd(counters + CNT_SKIPPED, skipped);
+    }
+}
+
+__global__ void gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ x_perm,
+                              const int32_t* __restrict__ slot_token,
+                              const int32_t* __restrict__ offsets, int E, int row_vec) {
+    const int total = offsets[E];
+    for (int r = blockIdx.x; r < total; r += gridDim.x) {
+        const int64_t t = slot_token[r];
+        const uint4* src = x + t * row_vec;
+        uint4* dst = x_perm + (int64_t)r * row_vec;
+        for (int i = threadIdx.x; i < row_vec; i += blockDim.x) dst[i] = src[i];
+    }
+}
+
+__global__ void combine_kernel(const float* __restrict__ H, const int32_t* __restrict__ offsets,
+                               int E, const int32_t* __restrict__ slot_token,
+                               const float* __restrict__ slot_w, float* Y, int d, int64_t N,
+                               int64_t max_rows) {
+    const int total = (int)min64(offsets[E], max_rows);
+    for (int r = blockIdx.x; r < total; r += gridDim.x) {
+        const int64_t t = slot_token[r];
+        if (t < 0 || t >= N) continue;
+        const float a = slot_w[r];
+        const float4* h = reinterpret_cast<const float4*>(H + (int64_t)r * d);
+        for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+            const float4 v = h[c];
+            red_add_v4(Y + t * d + 4 * c, a * v.x, a * v.y, a * v.z, a * v.w);
+        }
+    }
+}
+
+__global__ void mtile_prefix_kernel(int E, int bm, const int32_t* __restrict__ offsets,
+                                    int32_t* __restrict__ mt_start) {
+    __shared__ int warp_tot[33];
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+        const int e = e0 + threadIdx.x;
+        const int a = e < E ? offsets[e + 1] - offsets[e] : 0;
+        const int mt = (a + bm - 1) / bm;
+        int tot;
+        const int ex = block_excl_scan(mt, warp_tot, &tot);
+        if (e < E) mt_start[e] = carry + ex;
+        carry += tot;
+    }
+    if (threadIdx.x == 0) mt_start[E] = carry;
+}
+
+__global__ void zero_kernel(float4* __restrict__ Y, int64_t n4) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (int64_t)gridDim.x * blockDim.x)
+        Y[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_t* ids,
+                            const float* w, int32_t* slot, int32_t* offsets, int32_t* L,
+                            int32_t* acc, int32_t* slot_token, float* slot_w, const void* x,
+                            void* x_perm, unsigned long long* counters, const Scratch& sc,
+                            cudaStream_t st) {
+    const int E = p.E_r, k = p.k;
+    const int n_tiles = sc.n_tiles;
+    hist_kernel<<<n_tiles, 256, sizeof(int) * E, st>>>(ids, p.N, k, E, sc.tile_tokens, n_tiles,
+                                                        sc.hist, counters);
+    const int threads = ((E + 31) / 32) * 32 < 64 ? 64 : ((E + 31) / 32) * 32;
+    scan_kernel<<<1, threads, 0, st>>>(sc.hist, n_tiles, E, C, bm, L, acc, offsets, sc.mt_start,
+                                       counters);
+    assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
+                                                         n_tiles, sc.hist, offsets, slot,
+                                                         slot_token, slot_w, counters);
+    if (x && x_perm) {
+        const int row_vec = (int)(p.d * esize(p.dtype) / 16);
+        const int64_t rows = p.N * p.k;
+        const int blocks = (int)min64(rows, (int64_t)num_sms() * 8);
+        gather_kernel<<<blocks, 128, 0, st>>>(static_cast<const uint4*>(x),
+                                              static_cast<uint4*>(x_perm), slot_token, offsets, E,
+                                              row_vec);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const moe_params& p, const float* H, const int32_t* offsets,
+                           const int32_t* slot_token, const float* slot_w, float* Y,
+                           cudaStream_t st) {
+    const int64_t rows = p.N * p.k;
+    const int blocks = (int)min64(rows, (int64_t)num_sms() * 8);
+    combine_kernel<<<blocks, 256, 0, st>>>(H, offsets, p.E_r, slot_token, slot_w, Y, p.d, p.N, rows);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mtile_prefix(int E, int bm, const int32_t* offsets, int32_t* mt_start,
+                                cudaStream_t st) {
+    mtile_prefix_kernel<<<1, 1024, 0, st>>>(E, bm, offsets, mt_start);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_zero_f32(float* Y, int64_t n, cudaStream_t st) {
+    const int64_t n4 = n / 4;
+    const int blocks = (int)min64((n4 + 255) / 256, (int64_t)num_sms() * 8);
+    if (blocks > 0) zero_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<float4*>(Y), n4);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,714 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+//
+// What they compute (vegetog "MoE token routing" sec. 3, SwiGLU expert
+// E_i(x) = [SiLU(x W_gate,i) (.) (x W_up,i)] W_down,i; "LLM from scratch"
+// ch. 36.3: each expert runs only on its accepted slots, then
+// Y_t += a_te (H_e)_c; ch. 36.6: the shared expert adds F_sh(x) with weight 1):
+//   gate/up  h[r, :] = SiLU(x_r W_g^T) (.) (x_r W_u^T)        bf16 out
+//   down     Y[tok(r), :] += a(r) * (h[r, :] W_d^T)            fp32 atomics
+//            (or H[r, :] = h[r, :] W_d^T for the unfused entry point)
+//
+// Design (one persistent CTA per SM, 192 threads, warp-specialised):
+//   warp 0     TMA producer: per 64-wide K block it loads the A tile
+//              (128 rows x 64, bf16) and two 128-row B tiles into one
+//              shared-memory stage (4 stages of 48 KB, 128-byte swizzle).
+//   warp 1     MMA issuer: one elected thread issues tcgen05.mma
+//              (cta_group::1, kind::f16, M=128, N=256, K=16, fp32 accumulate)
+//              into one of two TMEM accumulators (2 x 256 columns), commits
+//              each stage back to the producer and each finished tile to the
+//              epilogue.
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator rows (one TMEM lane
+//              per row), then SwiGLU -> bf16 h (gate/up) or the weighted
+//              scatter-combine with 16-byte fp32 red.global.add (down).
+// For gate/up the two B tiles are the gate and up rows of the same 128
+// output columns, so one N=256 MMA yields both and the SwiGLU is local to a
+// thread.  For the down projection they are two consecutive 128-row halves
+// of a 256-column output tile.
+//
+// Tiles are scheduled statically (tile = blockIdx.x + i * gridDim.x) over a
+// list ordered group by group, output-column tile by column tile, with the
+// row tiles of one group fastest, so CTAs running at the same time share
+// the B (weight) tile through L2 and each weight byte leaves HBM about once.
+// The row count of each group is read from device memory (offsets and the
+// M-tile prefix written by the dispatch), so no host synchronisation is
+// needed.  Rows past a group's end are loaded (TMA zero-fills past the
+// tensor) but masked in the epilogue.
+//
+// Every wait on an mbarrier is bounded (about 2 s of %globaltimer): on
+// timeout the CTA raises an abort flag, records DEVERR_TIMEOUT, drains its
+// outstanding copies and MMAs with bounded waits, frees TMEM and returns.
+#include "moe_internal.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;   // MMA N (gate+up, or output columns of the down tile)
+constexpr int BK = 64;    // 64 bf16 = 128 bytes = one swizzle row
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_HALF_BYTES = 128 * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + 2 * B_HALF_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
+
+enum Epi { EPI_SWIGLU = 0, EPI_COMBINE = 1, EPI_STORE = 2 };
+
+struct TcArgs {
+    const int32_t* mt_start;  // [E+1] routed M-tile prefix
+    const int32_t* offsets;   // [E+1] routed row offsets
+    int E;
+    int nt_r, nkb_r;          // routed: output-column tiles, K blocks
+    int b_rows_r;             // routed B rows per expert (d_f for gate/up, d for down)
+    int M_sh, nt_sh, nkb_sh;  // shared group (M_sh = 0: none)
+    int n_valid_r, n_valid_sh;  // valid output columns
+    void* out;                // SWIGLU: h bf16 [rows, ld_out]; STORE: H fp32 [rows, ld_out]
+    void* out_sh;             // SWIGLU: h_sh bf16 [N, ld_out_sh]
+    int ld_out, ld_out_sh;
+    const int32_t* slot_token;
+    const float* slot_w;
+    float* Y;
+    int ldY;
+    int max_rows;             // rows of the routed A / output buffers (N k)
+    int n_tokens;             // N
+    unsigned long long* counters;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: true when the phase with `parity` completed; false on abort
+// (flag raised elsewhere) or timeout (raises the flag and records it).
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned long long* counters,
+                                             unsigned long long limit = kTimeoutNs) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const unsigned long long t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(a, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > limit) {
+                *abort_flag = 1;
+                atomicOr(counters + CNT_DEVICE_ERROR, (unsigned long long)DEVERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// Warp-collective bounded wait: every lane returns the same verdict, so the
+// .sync.aligned tcgen05 loads that follow are executed by the whole warp.
+__device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag,
+                                                  unsigned long long* counters) {
+    const uint32_t a = smem_u32(bar);
+    const int lane = threadIdx.x & 31;
+    unsigned long long t0 = 0;
+    if (lane == 0) t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        const bool done = mbar_try_wait(a, parity);
+        if (__all_sync(0xffffffffu, done)) return true;
+        if ((it & 63u) == 63u) {
+            int stop = 0;
+            if (lane == 0) {
+                if (*abort_flag) {
+                    stop = 1;
+                } else if (global_timer_ns() - t0 > kTimeoutNs) {
+                    *abort_flag = 1;
+                    atomicOr(counters + CNT_DEVICE_ERROR, (unsigned long long)DEVERR_TIMEOUT);
+                    stop = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
+                                            int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle,
+// 8-row core groups 1024 bytes apart (SBO), leading offset 16 bytes (unused
+// by the swizzled K-major layout), descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
+// N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Tile schedule
+// ---------------------------------------------------------------------------
+struct Tile {
+    int shared;     // 0 routed, 1 shared expert
+    int g;          // expert
+    int a_row;      // first row of the A tile in its matrix
+    int rows;       // valid rows (<= BM)
+    int n_tile;     // output-column tile
+    int nkb;        // K blocks
+};
+
+struct SchedSmem {
+    int32_t mt[kMaxExperts + 1];
+    int32_t off[kMaxExperts + 1];
+};
+
+__device__ __forceinline__ bool decode_tile(int t, const SchedSmem& s, const TcArgs& a, int routed_tiles,
+                                            Tile& ti) {
+    if (t < routed_tiles) {
+        const int q = t / a.nt_r;
+        // last group g with mt[g] <= q (non-empty, since mt[g+1] > q)
+        int lo = 0, hi = a.E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s.mt[mid] <= q) lo = mid;
+            else hi = mid - 1;
+        }
+        const int g = lo;
+        const int mtiles = s.mt[g + 1] - s.mt[g];
+        ti.shared = 0;
+        ti.g = g;
+        ti.nkb = a.nkb_r;
+        if (mtiles <= 0) {  // inconsistent prefix (caller-supplied offsets): no rows
+            ti.n_tile = 0;
+            ti.a_row = 0;
+            ti.rows = 0;
+            return true;
+        }
+        const int local = t - s.mt[g] * a.nt_r;
+        const int m_tile = local % mtiles;
+        ti.n_tile = local / mtiles;
+        ti.a_row = s.off[g] + m_tile * BM;
+        // rows of this tile inside the group and inside the row buffer
+        ti.rows = max(0, min(min(BM, s.off[g + 1] - ti.a_row), a.max_rows - ti.a_row));
+        if (ti.a_row < 0) ti.rows = 0;
+        return true;
+    }
+    const int mt_sh = (a.M_sh + BM - 1) / BM;
+    const int local = t - routed_tiles;
+    if (a.M_sh <= 0 || local >= mt_sh * a.nt_sh) return false;
+    ti.shared = 1;
+    ti.g = 0;
+    ti.n_tile = local / mt_sh;
+    ti.a_row = (local % mt_sh) * BM;
+    ti.rows = min(BM, a.M_sh - ti.a_row);
+    ti.nkb = a.nkb_sh;
+    return true;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc_grouped_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
+                      const __grid_constant__ CUtensorMap mB1,
+                      const __grid_constant__ CUtensorMap mA_sh,
+                      const __grid_constant__ CUtensorMap mB0_sh,
+                      const __grid_constant__ CUtensorMap mB1_sh, const TcArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned stage buffers (the 128-byte swizzle atom spans 8 rows)
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* stage_base = smem;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* done = tempty + 2;
+    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
+    SchedSmem* sched = reinterpret_cast<SchedSmem*>(smem + STAGES * STAGE_BYTES + 256);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    for (int i = threadIdx.x; i <= a.E; i += NUM_THREADS) {
+        sched->mt[i] = a.mt_start[i];
+        sched->off[i] = a.offsets[i];
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 128);
+        }
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc(tmem_base_s, TMEM_COLS);
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&mA);
+        tma_prefetch_desc(&mB0);
+        tma_prefetch_desc(&mB1);
+        if (a.M_sh > 0) {
+            tma_prefetch_desc(&mA_sh);
+            tma_prefetch_desc(&mB0_sh);
+            tma_prefetch_desc(&mB1_sh);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_base_s;
+
+    const int routed_tiles = sched->mt[a.E] * a.nt_r;
+    const int total_tiles = routed_tiles + (a.M_sh > 0 ? ((a.M_sh + BM - 1) / BM) * a.nt_sh : 0);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued_parity[STAGES];
+            for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                Tile ti;
+                decode_tile(t, *sched, a, routed_tiles, ti);
+                const CUtensorMap* pa = ti.shared ? &mA_sh : &mA;
+                const CUtensorMap* pb0 = ti.shared ? &mB0_sh : &mB0;
+                const CUtensorMap* pb1 = ti.shared ? &mB1_sh : &mB1;
+                int b_row0, b_row1;
+                if (EPI == EPI_SWIGLU) {
+                    b_row0 = (ti.shared ? 0 : ti.g * a.b_rows_r) + ti.n_tile * 128;
+                    b_row1 = b_row0;
+                } else {
+                    b_row0 = (ti.shared ? 0 : ti.g * a.b_rows_r) + ti.n_tile * 256;
+                    b_row1 = b_row0 + 128;
+                }
+                for (int kb = 0; kb < ti.nkb; ++kb) {
+                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, a.counters)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = stage_base + stage * STAGE_BYTES;
+                    uint8_t* sb = sa + A_BYTES;
+                    mbar_expect_tx(&full[stage], STAGE_BYTES);
+                    tma_load_2d(sa, pa, &full[stage], kb * BK, ti.a_row);
+                    tma_load_2d(sb, pb0, &full[stage], kb * BK, b_row0);
+                    tma_load_2d(sb + B_HALF_BYTES, pb1, &full[stage], kb * BK, b_row1);
+                    issued_parity[stage] = (int)phase;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (*abort_flag) {
+                // drain copies still in flight into this CTA's shared memory
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued_parity[s] >= 0)
+                        wait_bounded(&full[s], (uint32_t)issued_parity[s], abort_flag, a.counters,
+                                     kTimeoutNs / 4);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                Tile ti;
+                decode_tile(t, *sched, a, routed_tiles, ti);
+                if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, a.counters)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < ti.nkb; ++kb) {
+                    if (!wait_bounded(&full[stage], phase, abort_flag, a.counters)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+                    const uint32_t sb = sa + A_BYTES;
+                    const uint64_t ad = smem_desc_sw128(sa);
+                    const uint64_t bd = smem_desc_sw128(sb);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        // advance 16 elements (32 bytes) along K inside the swizzled row
+                        umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2),
+                                  (kb | kk) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            // all MMAs issued by this thread have completed once `done` fires
+            umma_commit(done);
+            wait_bounded(done, 0, abort_flag, a.counters, kTimeoutNs / 4);
+        }
+    } else {
+        // epilogue warps 2..5: TMEM lane quarter = warp % 4
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+            Tile ti;
+            decode_tile(t, *sched, a, routed_tiles, ti);
+            if (!warp_wait_bounded(&tfull[acc], acc_phase, abort_flag, a.counters)) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+            const bool row_ok = r < ti.rows;
+            const int grow = ti.a_row + r;
+            if (EPI == EPI_SWIGLU) {
+                const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
+                const int ld = ti.shared ? a.ld_out_sh : a.ld_out;
+                __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(ti.shared ? a.out_sh : a.out);
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 32) {
+                    uint32_t g[32], u[32];
+                    tmem_ld32(t_row + (uint32_t)c, g);
+                    tmem_ld32(t_row + 128u + (uint32_t)c, u);
+                    tmem_ld_wait();
+                    const int col0 = ti.n_tile * 128 + c;
+                    if (row_ok) {
+                        uint4* dst = reinterpret_cast<uint4*>(outp + (int64_t)grow * ld + col0);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            if (col0 + v * 8 < n_valid) {
+                                uint4 pk;
+                                float h[8];
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    h[j] = silu_f(__uint_as_float(g[v * 8 + j])) * __uint_as_float(u[v * 8 + j]);
+                                pk.x = pack_bf16(h[0], h[1]);
+                                pk.y = pack_bf16(h[2], h[3]);
+                                pk.z = pack_bf16(h[4], h[5]);
+                                pk.w = pack_bf16(h[6], h[7]);
+                                dst[v] = pk;
+                            }
+                        }
+                    }
+                }
+            } else {
+                const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
+                float wgt = 1.f;
+                float* dst_row = nullptr;
+                if (row_ok) {
+                    if (EPI == EPI_COMBINE) {
+                        int tok;
+                        if (ti.shared) {
+                            tok = grow;
+                        } else {
+                            tok = a.slot_token[grow];
+                            wgt = a.slot_w[grow];
+                        }
+                        if (tok < 0 || tok >= a.n_tokens) tok = -1;
+                        dst_row = tok >= 0 ? a.Y + (int64_t)tok * a.ldY : nullptr;
+                    } else {
+                        dst_row = static_cast<float*>(a.out) + (int64_t)grow * a.ld_out;
+                    }
+                }
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(t_row + (uint32_t)c, v);
+                    tmem_ld_wait();
+                    const int col0 = ti.n_tile * BN + c;
+                    if (row_ok && dst_row) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (col0 + q * 4 < n_valid) {
+                                float* p = dst_row + col0 + q * 4;
+                                const float x0 = __uint_as_float(v[q * 4 + 0]) * wgt;
+                                const float x1 = __uint_as_float(v[q * 4 + 1]) * wgt;
+                                const float x2 = __uint_as_float(v[q * 4 + 2]) * wgt;
+                                const float x3 = __uint_as_float(v[q * 4 + 3]) * wgt;
+                                if (EPI == EPI_COMBINE) {
+                                    red_add_v4(p, x0, x1, x2, x3);
+                                } else {
+                                    *reinterpret_cast<float4*>(p) = make_float4(x0, x1, x2, x3);
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 row-major matrix [rows, cols] read in boxes of 128 rows x 64 columns
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+    auto enc = get_encode();
+    if (!enc || rows == 0 || cols == 0) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {BK, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + sizeof(SchedSmem);
+
+template <int EPI>
+cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mB0, const CUtensorMap& mB1,
+                      const CUtensorMap& mA_sh, const CUtensorMap& mB0_sh, const CUtensorMap& mB1_sh,
+                      const TcArgs& a, int64_t max_tiles, cudaStream_t st) {
+    auto kern = tc_grouped_kernel<EPI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)min64(max_tiles, num_sms());
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, NUM_THREADS, kSmemBytes, st>>>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a);
+    return cudaGetLastError();
+}
+
+int64_t routed_mtile_bound(const moe_params& p) {
+    return (p.N * p.k + BM - 1) / BM + p.E_r;
+}
+
+}  // namespace
+
+cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
+                              const int32_t* offsets, const int32_t* mt_start,
+                              const ExpertWeights& W, void* h, void* h_shared,
+                              unsigned long long* counters, cudaStream_t st, int* status) {
+    *status = MOE_OK;
+    CUtensorMap mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh;
+    const uint64_t rows = (uint64_t)(p.N * p.k);
+    bool ok = make_map(&mA, x_perm, rows, p.d) &&
+              make_map(&mB0, W.W_g, (uint64_t)p.E_r * p.d_f, p.d) &&
+              make_map(&mB1, W.W_u, (uint64_t)p.E_r * p.d_f, p.d);
+    const bool sh = p.d_f_shared > 0;
+    if (ok && sh) {
+        ok = make_map(&mA_sh, x_shared, (uint64_t)p.N, p.d) &&
+             make_map(&mB0_sh, W.Ws_g, (uint64_t)p.d_f_shared, p.d) &&
+             make_map(&mB1_sh, W.Ws_u, (uint64_t)p.d_f_shared, p.d);
+    } else {
+        mA_sh = mA;
+        mB0_sh = mB0;
+        mB1_sh = mB1;
+    }
+    if (!ok) {
+        *status = MOE_ERR_CUDA;
+        return cudaErrorInvalidValue;
+    }
+    TcArgs a{};
+    a.mt_start = mt_start;
+    a.offsets = offsets;
+    a.E = p.E_r;
+    a.nt_r = (p.d_f + 127) / 128;
+    a.nkb_r = (p.d + BK - 1) / BK;
+    a.b_rows_r = p.d_f;
+    a.M_sh = sh ? (int)p.N : 0;
+    a.nt_sh = sh ? (p.d_f_shared + 127) / 128 : 0;
+    a.nkb_sh = a.nkb_r;
+    a.n_valid_r = p.d_f;
+    a.n_valid_sh = p.d_f_shared;
+    a.out = h;
+    a.out_sh = h_shared;
+    a.ld_out = p.d_f;
+    a.ld_out_sh = p.d_f_shared;
+    a.max_rows = (int)(p.N * p.k);
+    a.n_tokens = (int)p.N;
+    a.counters = counters;
+    int64_t max_tiles = routed_mtile_bound(p) * a.nt_r + (sh ? ((p.N + BM - 1) / BM) * a.nt_sh : 0);
+    return launch_tc<EPI_SWIGLU>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a, max_tiles, st);
+}
+
+cudaError_t launch_tc_down(const moe_params& p, int mode, const void* h, const void* h_shared,
+                           const int32_t* offsets, const int32_t* mt_start,
+                           const ExpertWeights& W, const int32_t* slot_token,
+                           const float* slot_w, float* Y, float* H_out,
+                           unsigned long long* counters, cudaStream_t st, int* status) {
+    *status = MOE_OK;
+    CUtensorMap mA, mB0, mA_sh, mB0_sh;
+    const uint64_t rows = (uint64_t)(p.N * p.k);
+    bool ok = make_map(&mA, h, rows, p.d_f) && make_map(&mB0, W.W_d, (uint64_t)p.E_r * p.d, p.d_f);
+    const bool sh = p.d_f_shared > 0 && mode == DOWN_COMBINE;
+    if (ok && sh) {
+        ok = make_map(&mA_sh, h_shared, (uint64_t)p.N, p.d_f_shared) &&
+             make_map(&mB0_sh, W.Ws_d, (uint64_t)p.d, p.d_f_shared);
+    } else {
+        mA_sh = mA;
+        mB0_sh = mB0;
+    }
+    if (!ok) {
+        *status = MOE_ERR_CUDA;
+        return cudaErrorInvalidValue;
+    }
+    TcArgs a{};
+    a.mt_start = mt_start;
+    a.offsets = offsets;
+    a.E = p.E_r;
+    a.nt_r = (p.d + BN - 1) / BN;
+    a.nkb_r = (p.d_f + BK - 1) / BK;
+    a.b_rows_r = p.d;
+    a.M_sh = sh ? (int)p.N : 0;
+    a.nt_sh = sh ? a.nt_r : 0;
+    a.nkb_sh = sh ? (p.d_f_shared + BK - 1) / BK : 0;
+    a.n_valid_r = p.d;
+    a.n_valid_sh = p.d;
+    a.out = H_out;
+    a.ld_out = p.d;
+    a.slot_token = slot_token;
+    a.slot_w = slot_w;
+    a.Y = Y;
+    a.ldY = p.d;
+    a.max_rows = (int)(p.N * p.k);
+    a.n_tokens = (int)p.N;
+    a.counters = counters;
+    int64_t max_tiles = routed_mtile_bound(p) * a.nt_r + (sh ? ((p.N + BM - 1) / BM) * a.nt_sh : 0);
+    if (mode == DOWN_COMBINE)
+        return launch_tc<EPI_COMBINE>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
+    return launch_tc<EPI_STORE>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
+}
+
+}  // namespace moe

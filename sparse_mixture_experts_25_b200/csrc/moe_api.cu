@@ -1,0 +1,399 @@
+// C ABI of the sparse-MoE layer: argument checks, workspace layout and the
+// stream-ordered launch sequence.  See include/moe.h for the contract of
+// every entry point.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+size_t esize(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
+
+int dispatch_tile_tokens(int k) {
+    // about 256 requests per dispatch tile (one warp walks a tile)
+    int t = 256 / (k > 0 ? k : 1);
+    return t < 8 ? 8 : t;
+}
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64 && cache[dev]) return cache[dev];
+    int n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+    if (dev < 64) cache[dev] = n;
+    return n;
+}
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static bool layout(const moe_params& p, moe_ws_layout& L, int& n_tiles, int& tile_tokens) {
+    const size_t Nk = (size_t)p.N * (size_t)p.k;
+    const size_t E = (size_t)p.E_r;
+    const size_t es = esize(p.dtype);
+    tile_tokens = dispatch_tile_tokens(p.k);
+    n_tiles = (int)((p.N + tile_tokens - 1) / tile_tokens);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    L.ids = take(Nk * 4);
+    L.w = take(Nk * 4);
+    L.margin = take((size_t)p.N * 4);
+    L.slot = take(Nk * 4);
+    L.offsets = take((E + 1) * 4);
+    L.L = take(E * 4);
+    L.acc = take(E * 4);
+    L.slot_token = take(Nk * 4);
+    L.slot_w = take(Nk * 4);
+    L.counters = take(CNT_COUNT * 8);
+    L.x_perm = take(Nk * (size_t)p.d * es);
+    L.h = take(Nk * (size_t)p.d_f * es);
+    L.h_shared = take((size_t)p.N * (size_t)(p.d_f_shared > 0 ? p.d_f_shared : 0) * es);
+    L.scratch = take(E * (size_t)std::max(n_tiles, 1) * 4 + (E + 1) * 4);
+    L.total = off;
+    return true;
+}
+
+bool make_view(const moe_params& p, void* ws, WsView& v) {
+    int n_tiles, tile_tokens;
+    layout(p, v.lay, n_tiles, tile_tokens);
+    char* b = static_cast<char*>(ws);
+    v.base = b;
+    v.ids = reinterpret_cast<int32_t*>(b + v.lay.ids);
+    v.w = reinterpret_cast<float*>(b + v.lay.w);
+    v.margin = reinterpret_cast<float*>(b + v.lay.margin);
+    v.slot = reinterpret_cast<int32_t*>(b + v.lay.slot);
+    v.offsets = reinterpret_cast<int32_t*>(b + v.lay.offsets);
+    v.L = reinterpret_cast<int32_t*>(b + v.lay.L);
+    v.acc = reinterpret_cast<int32_t*>(b + v.lay.acc);
+    v.slot_token = reinterpret_cast<int32_t*>(b + v.lay.slot_token);
+    v.slot_w = reinterpret_cast<float*>(b + v.lay.slot_w);
+    v.counters = reinterpret_cast<unsigned long long*>(b + v.lay.counters);
+    v.x_perm = b + v.lay.x_perm;
+    v.h = b + v.lay.h;
+    v.h_shared = b + v.lay.h_shared;
+    v.scratch.hist = reinterpret_cast<int32_t*>(b + v.lay.scratch);
+    v.scratch.mt_start = v.scratch.hist + (size_t)p.E_r * std::max(n_tiles, 1);
+    v.scratch.n_tiles = n_tiles;
+    v.scratch.tile_tokens = tile_tokens;
+    return true;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+thread_local cudaEvent_t g_stage_events[8];
+thread_local int g_stage_event_count = 0;
+
+inline void stage_mark(int i, cudaStream_t st) {
+    if (g_stage_event_count >= 5 && i < g_stage_event_count) cudaEventRecord(g_stage_events[i], st);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status check_params(const moe_params* p) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (p->N < 0 || p->d < 1 || p->d_f < 1 || p->E_r < 1 || p->k < 1 || p->k > p->E_r)
+        return MOE_ERR_INVALID_ARG;
+    if (p->norm < MOE_NORM_RENORM || p->norm > MOE_NORM_WLR) return MOE_ERR_INVALID_ARG;
+    if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (p->d_f_shared < 0) return MOE_ERR_INVALID_ARG;
+    if (!(p->c == p->c) || p->c > 1e6) return MOE_ERR_INVALID_ARG;
+    if (p->norm == MOE_NORM_WLR && !(p->theta >= 0.f && p->theta < 1.f)) return MOE_ERR_INVALID_ARG;
+    if (p->E_r > kMaxExperts || p->k > kMaxK) return MOE_ERR_UNSUPPORTED;
+    if (p->d % 8 || p->d_f % 8 || p->d_f_shared % 8) return MOE_ERR_UNSUPPORTED;
+    if ((int64_t)p->N * p->k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// exact capacity on the binary value of c (see moe.h)
+int64_t capacity_exact(double c, int64_t N, int k, int E) {
+    if (c <= 0.0) return N;
+    int ex = 0;
+    const double m = frexp(c, &ex);                      // c = m 2^ex, m in [0.5, 1)
+    const __int128 mant = (__int128)ldexp(m, 53);        // c = mant 2^(ex-53), exact
+    const int sh = ex - 53;
+    __int128 num = mant * (__int128)N * (__int128)k;
+    __int128 den = (__int128)E;
+    if (sh >= 0) {
+        num <<= sh;
+    } else {
+        int s = -sh;
+        while (s > 0 && (num & 1) == 0) {  // strip common powers of two
+            num >>= 1;
+            --s;
+        }
+        den <<= s;
+    }
+    const __int128 fl = num / den;
+    const __int128 rem = num - fl * den;
+    const __int128 r = (2 * rem >= den) ? fl + 1 : fl;   // nearest integer
+    const long double q = (long double)num / (long double)den;
+    const long double dist = fabsl(q - (long double)r);
+    const long double tol = 1e-9L * (q > 1.0L ? q : 1.0L);
+    int64_t C = (dist <= tol) ? (int64_t)r : (int64_t)(rem ? fl + 1 : fl);
+    if (N > 0 && C < 1) C = 1;
+    return C;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported size or mode";
+        case MOE_ERR_NONFINITE: return "non-finite router score (input failure)";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_WORKSPACE: return "workspace missing or misaligned";
+        case MOE_ERR_TIMEOUT: return "bounded device wait timed out";
+    }
+    return "unknown status";
+}
+
+moe_status moe_capacity(const moe_params* p, int64_t* C) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (!C) return MOE_ERR_INVALID_ARG;
+    *C = capacity_exact(p->c, p->N, p->k, p->E_r);
+    return MOE_OK;
+}
+
+moe_status moe_workspace_layout(const moe_params* p, moe_ws_layout* out) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (!out) return MOE_ERR_INVALID_ARG;
+    int n_tiles, tile_tokens;
+    layout(*p, *out, n_tiles, tile_tokens);
+    return MOE_OK;
+}
+
+moe_status moe_workspace_size(const moe_params* p, size_t* bytes) {
+    moe_ws_layout L;
+    moe_status s = moe_workspace_layout(p, &L);
+    if (s != MOE_OK) return s;
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    *bytes = L.total;
+    return MOE_OK;
+}
+
+moe_status moe_set_stage_events(void* const* events, int n) {
+    if (n < 0 || n > 8 || (n > 0 && !events)) return MOE_ERR_INVALID_ARG;
+    if (n > 0 && n < 5) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+    g_stage_event_count = n;
+    return MOE_OK;
+}
+
+moe_status moe_route(const moe_params* p, const void* x, const void* W_r, const float* b_r,
+                     const float* lat, int32_t* ids, float* w, float* margin, void* ws,
+                     moe_stream_t stream) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (p->E_r > kMaxRouterExperts) return MOE_ERR_UNSUPPORTED;
+    if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (p->N == 0) return MOE_OK;
+    if (!x || !W_r || !ids || !w || !aligned16(x) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
+    if (p->norm == MOE_NORM_WLR && !lat) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    WsView v;
+    make_view(*p, ws, v);
+    if (cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return cuda_status(launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, ids,
+                                     w, margin, v.counters, nullptr, st));
+}
+
+moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const float* w, int64_t C,
+                        int32_t* slot, int32_t* offsets, int32_t* slot_token, float* slot_w,
+                        const void* x, void* x_perm, void* ws, moe_stream_t stream) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (C < 1) return MOE_ERR_INVALID_ARG;
+    if (!offsets) return MOE_ERR_INVALID_ARG;
+    if ((x != nullptr) != (x_perm != nullptr)) return MOE_ERR_INVALID_ARG;
+    if (x && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    WsView v;
+    make_view(*p, ws, v);
+    if (p->N == 0) {
+        if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p->E_r + 1), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!ids || !w || !slot || !slot_token || !slot_w) return MOE_ERR_INVALID_ARG;
+    // dispatch-side counters start from zero; router counters are kept
+    if (cudaMemsetAsync(v.counters + CNT_REQUESTED, 0, 6 * 8, st) != cudaSuccess ||
+        cudaMemsetAsync(v.counters + CNT_L_MAX, 0, 2 * 8, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
+    return cuda_status(launch_dispatch(*p, C, bm, ids, w, slot, offsets, v.L, v.acc, slot_token,
+                                       slot_w, x, x_perm, v.counters, v.scratch, st));
+}
+
+moe_status moe_expert_ffn(const moe_params* p, const void* x_perm, const int32_t* offsets,
+                          const void* W_g, const void* W_u, const void* W_d, float* H, void* ws,
+                          moe_stream_t stream) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (p->N == 0) return MOE_OK;
+    if (!x_perm || !offsets || !W_g || !W_u || !W_d || !H) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_perm) || !aligned16(W_g) || !aligned16(W_u) || !aligned16(W_d) || !aligned16(H))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    WsView v;
+    make_view(*p, ws, v);
+    moe_params q = *p;
+    q.d_f_shared = 0;  // routed experts only
+    ExpertWeights W{W_g, W_u, W_d, nullptr, nullptr, nullptr};
+    const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
+    if (launch_mtile_prefix(p->E_r, bm, offsets, v.scratch.mt_start, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    int status = MOE_OK;
+    cudaError_t e;
+    if (p->dtype == MOE_BF16) {
+        e = launch_tc_gate_up(q, x_perm, nullptr, offsets, v.scratch.mt_start, W, v.h, nullptr,
+                              v.counters, st, &status);
+        if (e != cudaSuccess) return status != MOE_OK ? (moe_status)status : MOE_ERR_CUDA;
+        e = launch_tc_down(q, DOWN_STORE, v.h, nullptr, offsets, v.scratch.mt_start, W, nullptr,
+                           nullptr, nullptr, H, v.counters, st, &status);
+        if (e != cudaSuccess) return status != MOE_OK ? (moe_status)status : MOE_ERR_CUDA;
+    } else {
+        e = launch_simt_gate_up(q, x_perm, nullptr, offsets, v.scratch.mt_start, W, v.h, nullptr, st);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        e = launch_simt_down(q, DOWN_STORE, v.h, nullptr, offsets, v.scratch.mt_start, W, nullptr,
+                             nullptr, nullptr, H, st);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+moe_status moe_combine(const moe_params* p, const float* H, const int32_t* offsets,
+                       const int32_t* slot_token, const float* slot_w, float* Y,
+                       moe_stream_t stream) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (p->N == 0) return MOE_OK;
+    if (!H || !offsets || !slot_token || !slot_w || !Y || !aligned16(H) || !aligned16(Y))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_combine(*p, H, offsets, slot_token, slot_w, Y,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, const float* b_r,
+                       const float* lat, const void* W_g, const void* W_u, const void* W_d,
+                       const void* Ws_g, const void* Ws_u, const void* Ws_d, float* Y, void* ws,
+                       moe_stream_t stream) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (p->E_r > kMaxRouterExperts) return MOE_ERR_UNSUPPORTED;
+    if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    WsView v;
+    make_view(*p, ws, v);
+    if (cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (p->N == 0) return MOE_OK;
+    if (!x || !W_r || !W_g || !W_u || !W_d || !Y) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W_r) || !aligned16(W_g) || !aligned16(W_u) || !aligned16(W_d) ||
+        !aligned16(Y))
+        return MOE_ERR_INVALID_ARG;
+    if (p->norm == MOE_NORM_WLR && !lat) return MOE_ERR_INVALID_ARG;
+    const bool sh = p->d_f_shared > 0;
+    if (sh && (!Ws_g || !Ws_u || !Ws_d || !aligned16(Ws_g) || !aligned16(Ws_u) || !aligned16(Ws_d)))
+        return MOE_ERR_INVALID_ARG;
+    const int64_t C = capacity_exact(p->c, p->N, p->k, p->E_r);
+    ExpertWeights W{W_g, W_u, W_d, sh ? Ws_g : nullptr, sh ? Ws_u : nullptr, sh ? Ws_d : nullptr};
+
+    stage_mark(0, st);
+    cudaError_t e = launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, v.ids,
+                                  v.w, v.margin, v.counters, Y, st);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    stage_mark(1, st);
+    const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
+    e = launch_dispatch(*p, C, bm, v.ids, v.w, v.slot, v.offsets, v.L, v.acc, v.slot_token, v.slot_w,
+                        x, v.x_perm, v.counters, v.scratch, st);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    stage_mark(2, st);
+    int status = MOE_OK;
+    if (p->dtype == MOE_BF16) {
+        e = launch_tc_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared,
+                              v.counters, st, &status);
+        if (e != cudaSuccess) return status != MOE_OK ? (moe_status)status : MOE_ERR_CUDA;
+        stage_mark(3, st);
+        e = launch_tc_down(*p, DOWN_COMBINE, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
+                           v.slot_token, v.slot_w, Y, nullptr, v.counters, st, &status);
+        if (e != cudaSuccess) return status != MOE_OK ? (moe_status)status : MOE_ERR_CUDA;
+    } else {
+        e = launch_simt_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, st);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        stage_mark(3, st);
+        e = launch_simt_down(*p, DOWN_COMBINE, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
+                             v.slot_token, v.slot_w, Y, nullptr, st);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    stage_mark(4, st);
+    return MOE_OK;
+}
+
+moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, moe_stream_t stream) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (!ws || !out) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    WsView v;
+    make_view(*p, const_cast<void*>(ws), v);
+    unsigned long long cnt[CNT_COUNT];
+    std::vector<int32_t> L((size_t)p->E_r);
+    memset(out, 0, sizeof(*out));
+    if (cudaMemcpyAsync(cnt, v.counters, sizeof(cnt), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(L.data(), v.L, sizeof(int32_t) * L.size(), cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    out->C = (int64_t)cnt[CNT_C];
+    out->requested = (int64_t)cnt[CNT_REQUESTED];
+    out->accepted = (int64_t)cnt[CNT_ACCEPTED];
+    out->rejected = (int64_t)cnt[CNT_REJECTED];
+    out->O = (int64_t)cnt[CNT_O];
+    out->tokens_affected = (int64_t)cnt[CNT_AFFECTED];
+    out->tokens_skipped = (int64_t)cnt[CNT_SKIPPED];
+    out->nonfinite = (int64_t)cnt[CNT_NONFINITE];
+    out->near_tie = (int64_t)cnt[CNT_NEAR_TIE];
+    out->L_max = (int64_t)cnt[CNT_L_MAX];
+    out->device_error = (int32_t)cnt[CNT_DEVICE_ERROR];
+    if (p->N > 0) {
+        std::vector<int32_t> srt(L);
+        std::sort(srt.begin(), srt.end());
+        auto pct = [&](double q) {
+            size_t rank = (size_t)ceil(q / 100.0 * (double)srt.size());
+            if (rank < 1) rank = 1;
+            return (int64_t)srt[rank - 1];
+        };
+        out->L_p50 = pct(50);
+        out->L_p90 = pct(90);
+        out->L_p99 = pct(99);
+        out->rho_max = (double)out->L_max * (double)p->E_r / ((double)p->N * (double)p->k);
+        out->reject_rate = out->requested ? (double)out->rejected / (double)out->requested : 0.0;
+    }
+    if (cnt[CNT_DEVICE_ERROR] & DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+    if (cnt[CNT_NONFINITE]) return MOE_ERR_NONFINITE;
+    return MOE_OK;
+}
+
+}  // extern "C"

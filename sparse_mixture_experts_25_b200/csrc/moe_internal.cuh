@@ -1,0 +1,145 @@
+// Internal declarations shared by the CUDA sources of libmoe (not installed).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// Limits and workspace constants
+// ---------------------------------------------------------------------------
+constexpr int kMaxExperts = 1024;     // E_r limit of dispatch and the GEMM schedule
+constexpr int kMaxRouterExperts = 256;  // E_r limit of the fused router kernel
+constexpr int kMaxK = 32;             // k limit (warp-wide selection)
+constexpr int kTcBM = 128;            // M tile of the tcgen05 grouped GEMM
+constexpr int kSimtBM = 64;           // M tile of the fp32 grouped GEMM
+
+// indices into the int64 device counter block (moe_ws_layout.counters)
+enum Counter {
+    CNT_REQUESTED = 0,
+    CNT_ACCEPTED = 1,
+    CNT_REJECTED = 2,
+    CNT_O = 3,
+    CNT_AFFECTED = 4,
+    CNT_SKIPPED = 5,
+    CNT_NONFINITE = 6,
+    CNT_NEAR_TIE = 7,
+    CNT_L_MAX = 8,
+    CNT_C = 9,
+    CNT_DEVICE_ERROR = 10,  // bit flags, see DevErr
+    CNT_COUNT = 16
+};
+
+enum DevErr { DEVERR_TIMEOUT = 1, DEVERR_BOUNDS = 2 };
+
+constexpr float kNearTie = 1e-5f;
+
+// Scratch region of the workspace (int32 unless noted)
+struct Scratch {
+    int32_t* hist;        // [E][n_tiles] per-tile request counts -> exclusive bases
+    int32_t* mt_start;    // [E+1] prefix of M tiles (BM of the GEMM in use)
+    int n_tiles;          // dispatch tiles
+    int tile_tokens;      // tokens per dispatch tile
+};
+
+struct WsView {
+    moe_ws_layout lay;
+    char* base;
+    int32_t* ids;
+    float* w;
+    float* margin;
+    int32_t* slot;
+    int32_t* offsets;
+    int32_t* L;
+    int32_t* acc;
+    int32_t* slot_token;
+    float* slot_w;
+    unsigned long long* counters;
+    void* x_perm;
+    void* h;
+    void* h_shared;
+    Scratch scratch;
+};
+
+// Host helpers (moe_api.cu)
+int dispatch_tile_tokens(int k);
+size_t esize(int dtype);
+bool make_view(const moe_params& p, void* ws, WsView& v);
+
+// ---------------------------------------------------------------------------
+// Launchers (each returns cudaGetLastError() of its launch)
+// ---------------------------------------------------------------------------
+// router.cu
+cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, const float* b_r,
+                          const float* lat, int32_t* ids, float* w, float* margin,
+                          unsigned long long* counters, float* Y_zero, cudaStream_t st);
+// dispatch.cu
+cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_t* ids,
+                            const float* w, int32_t* slot, int32_t* offsets, int32_t* L,
+                            int32_t* acc, int32_t* slot_token, float* slot_w, const void* x,
+                            void* x_perm, unsigned long long* counters, const Scratch& sc,
+                            cudaStream_t st);
+cudaError_t launch_combine(const moe_params& p, const float* H, const int32_t* offsets,
+                           const int32_t* slot_token, const float* slot_w, float* Y,
+                           cudaStream_t st);
+cudaError_t launch_mtile_prefix(int E, int bm, const int32_t* offsets, int32_t* mt_start,
+                                cudaStream_t st);
+cudaError_t launch_zero_f32(float* Y, int64_t n, cudaStream_t st);
+
+// gemm_tc.cu (bf16, tcgen05)
+struct ExpertWeights {
+    const void* W_g;
+    const void* W_u;
+    const void* W_d;
+    const void* Ws_g;
+    const void* Ws_u;
+    const void* Ws_d;
+};
+enum DownMode { DOWN_COMBINE = 0, DOWN_STORE = 1 };
+cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
+                              const int32_t* offsets, const int32_t* mt_start,
+                              const ExpertWeights& W, void* h, void* h_shared,
+                              unsigned long long* counters, cudaStream_t st, int* status);
+cudaError_t launch_tc_down(const moe_params& p, int mode, const void* h, const void* h_shared,
+                           const int32_t* offsets, const int32_t* mt_start,
+                           const ExpertWeights& W, const int32_t* slot_token,
+                           const float* slot_w, float* Y, float* H_out,
+                           unsigned long long* counters, cudaStream_t st, int* status);
+
+// gemm_simt.cu (fp32 CUDA-core path)
+cudaError_t launch_simt_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
+                                const int32_t* offsets, const int32_t* mt_start,
+                                const ExpertWeights& W, void* h, void* h_shared,
+                                cudaStream_t st);
+cudaError_t launch_simt_down(const moe_params& p, int mode, const void* h, const void* h_shared,
+                             const int32_t* offsets, const int32_t* mt_start,
+                             const ExpertWeights& W, const int32_t* slot_token,
+                             const float* slot_w, float* Y, float* H_out, cudaStream_t st);
+
+int num_sms();
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
+}  // namespace moe

@@ -1,0 +1,337 @@
+// Router scores, softmax, top-k and routing weights, fused in one kernel.
+//
+// What it computes ("LLM from scratch" ch. 36.1-36.2, Algorithm 36.1 steps
+// 1-2; vegetog "MoE token routing" sec. 2; WDMoE note on WLR pruning):
+//   g_te = sum_i x_ti W_r[e,i] + b_e            (fp32 accumulation)
+//   p_te = exp(g_te - max_e g_te) / sum_e exp(...)
+//   S_t  = k largest scores, ties to the lower expert index
+//   a_te = p_te / sum_{S_t} p (renorm) | p_te (full prob) | WLR pruning
+//
+// Design: one CTA of 256 threads owns 32 tokens.  The score tile
+// [32 tokens x E_r] is a small FFMA GEMM staged through shared memory in
+// 64-wide K chunks, with a (TT tokens x TE experts) register tile per thread
+// chosen from E_r.  The selection then runs warp-wide: each lane holds
+// ceil(E_r/32) scores and k rounds of a (value desc, index asc) warp argmax
+// pick the experts in rank order.  For the narrow routers of the pages'
+// layers (E_r = 8 on a d = 4096 model) the kernel is bound by reading x
+// once; for E_r = 128-256 it is FFMA-bound.
+#include "moe_internal.cuh"
+
+#include <math.h>
+
+namespace moe {
+namespace {
+
+constexpr int kTok = 32;
+constexpr int kThreads = 256;
+constexpr int kKC = 64;
+
+struct RouterArgs {
+    const void* x;
+    const void* W_r;
+    const float* b_r;
+    const float* lat;
+    int32_t* ids;
+    float* w;
+    float* margin;
+    unsigned long long* counters;
+    float* Y_zero;
+    int64_t N;
+    int d, E, k, norm;
+    float theta;
+};
+
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    float4 a = *reinterpret_cast<const float4*>(p);
+    float4 b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+template <int TT, int TE, typename Tin>
+__global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
+    constexpr int EG = 8 * TT;       // expert groups across the CTA
+    constexpr int EPAD = EG * TE;    // padded expert count
+    constexpr int PER = (EPAD + 31) / 32;
+    static_assert((kTok / TT) * EG == kThreads, "thread grid");
+    extern __shared__ float smem[];
+    float* xs = smem;                 // [kKC][kTok]
+    float* wsm = smem + kKC * kTok;   // [kKC][EPAD]
+
+    const int tid = threadIdx.x;
+    const int tg = tid / EG, eg = tid % EG;
+    const int64_t t0 = (int64_t)blockIdx.x * kTok;
+    const Tin* X = static_cast<const Tin*>(a.x);
+    const Tin* W = static_cast<const Tin*>(a.W_r);
+
+    float acc[TT][TE];
+#pragma unroll
+    for (int i = 0; i < TT; ++i)
+#pragma unroll
+        for (int j = 0; j < TE; ++j) acc[i][j] = 0.f;
+
+    for (int k0 = 0; k0 < a.d; k0 += kKC) {
+        for (int i = tid; i < kTok * (kKC / 8); i += kThreads) {
+            const int tt = i / (kKC / 8), kc = (i % (kKC / 8)) * 8;
+            const int64_t t = t0 + tt;
+            float v[8];
+            if (t < a.N && k0 + kc < a.d) {
+                load8(X + t * a.d + k0 + kc, v);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) xs[(kc + j) * kTok + tt] = v[j];
+        }
+        for (int i = tid; i < EPAD * (kKC / 8); i += kThreads) {
+            const int e = i / (kKC / 8), kc = (i % (kKC / 8)) * 8;
+            float v[8];
+            if (e < a.E && k0 + kc < a.d) {
+                load8(W + (int64_t)e * a.d + k0 + kc, v);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) wsm[(kc + j) * EPAD + e] = v[j];
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kKC; ++kk) {
+            float xv[TT], wv[TE];
+#pragma unroll
+            for (int i = 0; i < TT; ++i) xv[i] = xs[kk * kTok + tg * TT + i];
+#pragma unroll
+            for (int j = 0; j < TE; ++j) wv[j] = wsm[kk * EPAD + eg + EG * j];
+#pragma unroll
+            for (int i = 0; i < TT; ++i)
+#pragma unroll
+                for (int j = 0; j < TE; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+
+    // scores -> shared memory
+    constexpr int LD = EPAD + 1;
+    float* lg = smem;  // [kTok][LD], fits inside the staging buffers
+#pragma unroll
+    for (int i = 0; i < TT; ++i)
+#pragma unroll
+        for (int j = 0; j < TE; ++j) {
+            const int e = eg + EG * j;
+            if (e < a.E) lg[(tg * TT + i) * LD + e] = acc[i][j] + (a.b_r ? a.b_r[e] : 0.f);
+        }
+    __syncthreads();
+
+    const int warp = tid >> 5, lane = tid & 31;
+    const int E = a.E, k = a.k;
+    for (int q = 0; q < kTok / 8; ++q) {
+        const int tt = warp * (kTok / 8) + q;
+        const int64_t t = t0 + tt;
+        if (t >= a.N) break;
+        const float* g = lg + tt * LD;
+        float v[PER];
+        bool bad = false;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane + 32 * i;
+            v[i] = e < E ? g[e] : -INFINITY;
+            if (e < E && !isfinite(v[i])) bad = true;
+        }
+        // selection in rank order: lane r keeps the r-th pick
+        float m = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) m = fmaxf(m, v[i]);
+        m = warp_max(m);
+        unsigned taken = 0;
+        int my_e = -1;
+        float my_g = 0.f, next_g = -INFINITY;
+        const int rounds = k < E ? k + 1 : k;
+        if (!__any_sync(0xffffffffu, bad)) {
+            for (int r = 0; r < rounds; ++r) {
+                float bv = -INFINITY;
+                int be = 0x7fffffff;
+#pragma unroll
+                for (int i = 0; i < PER; ++i) {
+                    const int e = lane + 32 * i;
+                    if (!((taken >> i) & 1u) && e < E && (v[i] > bv || (v[i] == bv && e < be))) {
+                        bv = v[i];
+                        be = e;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o; o >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                    if (ov > bv || (ov == bv && oe < be)) {
+                        bv = ov;
+                        be = oe;
+                    }
+                }
+                if (r < k) {
+                    if (lane == r) {
+                        my_e = be;
+                        my_g = bv;
+                    }
+                    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+                } else {
+                    next_g = bv;
+                }
+            }
+        }
+        float z = 0.f;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) z += expf(v[i] - m);
+        }
+        z = warp_sum(z);
+        const bool pick = lane < k;
+        const float ex = pick && !bad ? expf(my_g - m) : 0.f;
+        float wv = 0.f;
+        bool active = pick;
+        bool lat_bad = false;
+        float te = 1.f;
+        if (a.norm == MOE_NORM_WLR && pick && !bad) {
+            te = a.lat[t * E + my_e];
+            lat_bad = !(te > 0.f);  // NaN or non-positive latency
+        }
+        bad = __any_sync(0xffffffffu, bad || lat_bad);
+        if (bad) {
+            if (pick) {
+                a.ids[t * k + lane] = -1;
+                a.w[t * k + lane] = 0.f;
+            }
+            if (lane == 0) {
+                if (a.margin) a.margin[t] = NAN;
+                atomicAdd(a.counters + CNT_NONFINITE, 1ull);
+            }
+            continue;
+        }
+        if (a.norm == MOE_NORM_FULLPROB) {
+            wv = ex / z;
+        } else if (a.norm == MOE_NORM_RENORM) {
+            wv = ex / warp_sum(ex);
+        } else {
+            const float wlr = (ex / z) / te;  // p_e / t_e (0 when t_e = inf)
+            for (;;) {
+                const unsigned am = __ballot_sync(0xffffffffu, active);
+                if (__popc(am) < 2) break;
+                // smallest WLR (on equal WLR the higher expert index) and largest WLR
+                float mn = active ? wlr : INFINITY;
+                int mne = active ? my_e : -1;
+                float mx = active ? wlr : -INFINITY;
+#pragma unroll
+                for (int o = 16; o; o >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, mn, o);
+                    const int oe = __shfl_xor_sync(0xffffffffu, mne, o);
+                    if (ov < mn || (ov == mn && oe > mne)) {
+                        mn = ov;
+                        mne = oe;
+                    }
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                }
+                const float ratio = mn / (mn + mx);
+                if (ratio <= a.theta) {
+                    if (active && my_e == mne) active = false;
+                } else {
+                    break;
+                }
+            }
+            const float s = warp_sum(active ? ex : 0.f);
+            wv = active ? ex / s : 0.f;
+            if (active && isinf(te)) wv = 0.f;  // disconnected expert: weight 0
+        }
+        if (pick) {
+            a.ids[t * k + lane] = active ? my_e : -1;
+            a.w[t * k + lane] = wv;
+        }
+        const float kth = __shfl_sync(0xffffffffu, my_g, k - 1);
+        const float mg = k < E ? kth - next_g : INFINITY;
+        if (lane == 0) {
+            if (a.margin) a.margin[t] = mg;
+            if (mg < kNearTie) atomicAdd(a.counters + CNT_NEAR_TIE, 1ull);
+        }
+    }
+
+    if (a.Y_zero) {
+        const int64_t t_end = min64(a.N, t0 + kTok);
+        float4* Y4 = reinterpret_cast<float4*>(a.Y_zero + t0 * a.d);
+        const int64_t n4 = (t_end - t0) * a.d / 4;
+        for (int64_t i = tid; i < n4; i += kThreads) Y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+template <int TT, int TE, typename Tin>
+cudaError_t launch_one(const RouterArgs& a, cudaStream_t st) {
+    constexpr int EPAD = 8 * TT * TE;
+    const size_t smem = sizeof(float) * (kKC * kTok + kKC * EPAD);
+    auto kern = router_kernel<TT, TE, Tin>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = (a.N + kTok - 1) / kTok;
+    kern<<<(unsigned)blocks, kThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_typed(const RouterArgs& a, cudaStream_t st) {
+    if (a.E <= 8) return launch_one<1, 1, Tin>(a, st);
+    if (a.E <= 16) return launch_one<1, 2, Tin>(a, st);
+    if (a.E <= 32) return launch_one<2, 2, Tin>(a, st);
+    if (a.E <= 64) return launch_one<2, 4, Tin>(a, st);
+    if (a.E <= 128) return launch_one<4, 4, Tin>(a, st);
+    return launch_one<4, 8, Tin>(a, st);
+}
+
+}  // namespace
+
+cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, const float* b_r,
+                          const float* lat, int32_t* ids, float* w, float* margin,
+                          unsigned long long* counters, float* Y_zero, cudaStream_t st) {
+    RouterArgs a;
+    a.x = x;
+    a.W_r = W_r;
+    a.b_r = b_r;
+    a.lat = lat;
+    a.ids = ids;
+    a.w = w;
+    a.margin = margin;
+    a.counters = counters;
+    a.Y_zero = Y_zero;
+    a.N = p.N;
+    a.d = p.d;
+    a.E = p.E_r;
+    a.k = p.k;
+    a.norm = p.norm;
+    a.theta = p.theta;
+    if (p.N == 0) return cudaSuccess;
+    if (p.dtype == MOE_BF16) return launch_typed<__nv_bfloat16>(a, st);
+    return launch_typed<float>(a, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,124 @@
+"""Helpers for the GPU-vs-oracle parity tests (imported by tests only).
+
+Comparison rules (stated once, used by every parity test):
+  * routing ids are compared exactly for every token whose oracle score
+    margin g_(k) - g_(k+1) is >= 1e-5 (and, under WLR, whose every pruning
+    test has |ratio - theta| >= 1e-5); the others are near-ties: counted,
+    reported and excluded from id equality;
+  * dispatch is checked bit-exactly by running the oracle's dispatch on the
+    GPU's own ids (one flipped near-tie would shift later slots otherwise);
+  * weights: |a_gpu - a_oracle| <= 2e-6 + 2e-6 |a| (fp32 softmax vs double);
+  * outputs: max|Y_gpu - Y_ref| / max|Y_ref| <= 1e-4 (fp32 layers) or 2e-2
+    (bf16 layers, fp32 accumulation), with Y_ref the oracle's output
+    computed from the GPU's routing records; rows whose every path was
+    dropped must be exactly zero.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import seeded_inputs as si
+
+TOL = {si.DT_F32: 1e-4, si.DT_BF16: 2e-2}
+NEAR = 1e-5
+
+
+def torch_mod():
+    import torch
+    return torch
+
+
+def to_dev(a):
+    torch = torch_mod()
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def params_of(w: si.Workload):
+    import sparse_mixture_experts_25_b200 as moe
+    return moe.params(w.N, w.d, w.d_f, w.E, w.k, c=w.c, norm=w.norm, theta=w.theta,
+                      dtype=w.dtype, d_f_shared=w.d_f_shared)
+
+
+def gpu_forward(w: si.Workload, inp: dict, dev: dict | None = None):
+    """moe_forward through the C ABI; returns Y, routing records (host) and stats."""
+    import sparse_mixture_experts_25_b200 as moe
+    torch = torch_mod()
+    p = params_of(w)
+    if dev is None:
+        dev = {k: to_dev(v) for k, v in inp.items()}
+    ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+    Y = torch.full((w.N, w.d), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_forward(p, dev["x"], dev["W_r"], dev.get("b_r"), dev.get("lat"), dev["W_g"], dev["W_u"],
+                    dev["W_d"], dev.get("Ws_g"), dev.get("Ws_u"), dev.get("Ws_d"), Y, ws)
+    status, stats = moe.moe_get_stats(p, ws)
+    views = moe.workspace_views(p, ws)
+    rec = {k: v.cpu().numpy() for k, v in views.items()}
+    return {"Y": Y.cpu().numpy().astype(np.float64), "rec": rec, "stats": stats, "status": status,
+            "ws": ws, "p": p, "dev": dev}
+
+
+def check_routing(w: si.Workload, inp: dict, rec: dict):
+    """Oracle routing on the same inputs; returns (oracle route dict, near-tie mask)."""
+    r = oracle.route(inp["x"], inp["W_r"], k=w.k, norm=w.norm, theta=w.theta, b_r=inp.get("b_r"),
+                     lat=inp.get("lat"))
+    near = (r["margin"] < NEAR) | (r["wlr_gap"] < NEAR)
+    ok = ~near & ~r["invalid"]
+    assert (rec["ids"][ok] == r["ids"][ok]).all(), "routing ids differ on tokens that are not near-ties"
+    same = ok[:, None] & (rec["ids"] == r["ids"])
+    np.testing.assert_allclose(rec["w"][same], r["w"][same], rtol=2e-6, atol=2e-6)
+    assert (rec["ids"][r["invalid"]] == -1).all()
+    # margin reported by the GPU (fp32) agrees with the oracle's (double)
+    fin = ok & np.isfinite(r["margin"])
+    np.testing.assert_allclose(rec["margin"][fin], r["margin"][fin], rtol=1e-4, atol=2e-5)
+    return r, near
+
+
+def check_dispatch(w: si.Workload, rec: dict, stats: dict):
+    """Oracle dispatch on the GPU's own ids: slots, loads, offsets, records and
+    statistics must match bit for bit."""
+    C = oracle.capacity(w.c, w.N, w.k, w.E)
+    d = oracle.dispatch(rec["ids"], E=w.E, C=C)
+    np.testing.assert_array_equal(rec["slot"], d["slot"])
+    np.testing.assert_array_equal(rec["L"], d["L"])
+    np.testing.assert_array_equal(rec["acc"], d["acc"])
+    offs = np.concatenate([[0], np.cumsum(d["acc"])])
+    np.testing.assert_array_equal(rec["offsets"], offs)
+    # every accepted record sits at offsets[e] + slot with its token and weight
+    t_idx, j_idx = np.nonzero(d["slot"] >= 0)
+    pos = offs[rec["ids"][t_idx, j_idx]] + d["slot"][t_idx, j_idx]
+    np.testing.assert_array_equal(rec["slot_token"][pos], t_idx)
+    np.testing.assert_array_equal(rec["slot_w"][pos], rec["w"][t_idx, j_idx])
+    s = d["stats"]
+    for key in ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max"):
+        assert stats[key] == s[key], (key, stats[key], s[key])
+    assert stats["C"] == C
+    if w.N:
+        assert abs(stats["rho_max"] - oracle.rho_max(d["L"], w.N, w.k, w.E)) < 1e-12
+        for q, key in ((50, "L_p50"), (90, "L_p90"), (99, "L_p99")):
+            assert stats[key] == oracle.load_percentile(d["L"], q)
+    return d
+
+
+def rel_err(Y, Yref) -> float:
+    den = float(np.max(np.abs(Yref))) if Yref.size else 0.0
+    return float(np.max(np.abs(Y - Yref))) / (den if den > 0 else 1.0)
+
+
+def check_rows(w: si.Workload, inp: dict, rec: dict, Y: np.ndarray, tokens=None):
+    """Y rows against the oracle evaluated on the GPU's routing records."""
+    if tokens is None:
+        tokens = np.arange(w.N)
+    Ws = (inp.get("Ws_g"), inp.get("Ws_u"), inp.get("Ws_d")) if w.d_f_shared else None
+    ref = oracle.forward_rows(inp["x"], rec["ids"], rec["w"].astype(np.float64), rec["slot"], tokens,
+                              inp["W_g"], inp["W_u"], inp["W_d"], Ws=Ws)
+    err = rel_err(Y[tokens], ref)
+    assert err <= TOL[w.dtype], f"max-abs-rel error {err:.3e} above {TOL[w.dtype]:.0e}"
+    dropped = [i for i, t in enumerate(tokens) if not w.d_f_shared and (rec["slot"][t] < 0).all()]
+    for i in dropped:
+        assert (Y[tokens[i]] == 0).all()
+    return err

@@ -1,0 +1,106 @@
+"""The C-ABI library on a host without a GPU: it loads, exports every entry
+point the header declares, and its host-side logic (capacity, workspace
+layout, argument checks) behaves as documented.  No call here reaches a
+CUDA device."""
+import ctypes
+import math
+
+import pytest
+
+import oracle
+import sparse_mixture_experts_25_b200 as moe
+
+
+def test_library_exports_every_declared_symbol():
+    names = moe.declared_symbols()
+    assert {"moe_capacity", "moe_workspace_size", "moe_route", "moe_dispatch", "moe_expert_ffn",
+            "moe_combine", "moe_forward", "moe_get_stats", "moe_status_string"} <= set(names)
+    lib = moe.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_struct_sizes_match_the_header_layout():
+    assert ctypes.sizeof(moe.Params) == 48
+    assert ctypes.sizeof(moe.Stats) == 13 * 8 + 2 * 8 + 2 * 4
+    assert ctypes.sizeof(moe.WsLayout) == 15 * 8
+
+
+@pytest.mark.parametrize("c,N,k,E", [
+    (1.25, 1024, 1, 8), (1.25, 1000, 1, 8), (1.0, 4, 2, 3), (1.25, 8192, 8, 128),
+    (1.1, 1000, 1, 11), (1.25, 1001, 1, 8), (0.0, 4096, 2, 8), (-1.0, 77, 2, 8),
+    (2.0, 3, 1, 8), (0.3, 10, 1, 1000), (1.5, 4096, 8, 256), (0.9999999, 1000, 1, 10),
+    (1.0000000001, 1000, 1, 10), (3.7, 12345, 6, 97),
+])
+def test_capacity_matches_oracle(c, N, k, E):
+    p = moe.params(N, 64, 64, E, k, c=c)
+    assert moe.moe_capacity(p) == oracle.capacity(c, N, k, E)
+
+
+def test_capacity_printed_examples():
+    assert moe.moe_capacity(moe.params(1024, 64, 64, 8, 1, c=1.25)) == 160
+    assert moe.moe_capacity(moe.params(1000, 64, 64, 8, 1, c=1.25)) == 157
+    assert moe.moe_capacity(moe.params(4, 64, 64, 3, 2, c=1.0)) == 3
+
+
+def test_workspace_layout_regions():
+    p = moe.params(4096, 4096, 14336, 8, 2, dtype=moe.MOE_BF16)
+    L = moe.moe_workspace_layout(p)
+    assert moe.moe_workspace_size(p) == L["total"]
+    regions = sorted((v, k) for k, v in L.items() if k != "total")
+    for (o, _), (o2, _) in zip(regions, regions[1:]):
+        assert o % 256 == 0 and o2 >= o
+    assert L["h"] - L["x_perm"] >= 4096 * 2 * 4096 * 2
+    assert L["total"] - L["h"] >= 4096 * 2 * 14336 * 2
+    ps = moe.params(64, 4096, 2048, 8, 2, dtype=moe.MOE_BF16, d_f_shared=2048)
+    Ls = moe.moe_workspace_layout(ps)
+    assert Ls["scratch"] - Ls["h_shared"] >= 64 * 2048 * 2
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=9), moe.MOE_ERR_INVALID_ARG),
+    (dict(N=-1), moe.MOE_ERR_INVALID_ARG),
+    (dict(norm=7), moe.MOE_ERR_INVALID_ARG),
+    (dict(dtype=5), moe.MOE_ERR_INVALID_ARG),
+    (dict(norm=moe.MOE_NORM_WLR, theta=1.5), moe.MOE_ERR_INVALID_ARG),
+    (dict(d=100), moe.MOE_ERR_UNSUPPORTED),
+    (dict(d_f=36), moe.MOE_ERR_UNSUPPORTED),
+    (dict(E_r=2000, k=2), moe.MOE_ERR_UNSUPPORTED),
+    (dict(c=float("nan")), moe.MOE_ERR_INVALID_ARG),
+])
+def test_invalid_params_are_rejected_on_the_host(kw, status):
+    base = dict(N=16, d=64, d_f=64, E_r=8, k=2)
+    base.update(kw)
+    p = moe.params(**base)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_workspace_size(p)
+    assert ei.value.status == status
+
+
+def test_missing_workspace_is_reported_before_any_device_work():
+    p = moe.params(16, 64, 64, 8, 2)
+    r = moe.lib().moe_forward(ctypes.byref(p), None, None, None, None, None, None, None, None,
+                              None, None, None, None, None)
+    assert r == moe.MOE_ERR_WORKSPACE
+    r = moe.lib().moe_dispatch(ctypes.byref(p), None, None, 0, None, None, None, None, None, None,
+                               None, None)
+    assert r == moe.MOE_ERR_WORKSPACE
+    # router of more than 256 experts is not implemented by the fused router kernel
+    p = moe.params(16, 64, 64, 512, 2)
+    r = moe.lib().moe_route(ctypes.byref(p), None, None, None, None, None, None, None, None, None)
+    assert r == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_status_strings():
+    for s in range(7):
+        assert moe.moe_status_string(s)
+    assert "non-finite" in moe.moe_status_string(moe.MOE_ERR_NONFINITE)
+
+
+def test_host_tensors_are_refused_by_the_binding():
+    torch = pytest.importorskip("torch")
+    p = moe.params(4, 64, 64, 8, 2)
+    with pytest.raises(ValueError):
+        moe.moe_forward(p, torch.zeros(4, 64), None, None, None, None, None, None, None, None, None,
+                        None, None, stream=0)

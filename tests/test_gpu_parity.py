@@ -1,0 +1,293 @@
+"""CUDA path vs the CPU oracle, through the C ABI, on seeded inputs.
+
+Small cases span several tiles with ragged tails (rows per expert, output
+columns and K all end mid-tile); the full-size cases run the page-shaped
+layers in the launch configuration the benchmark times and check routing
+and dispatch on every token and outputs on sampled tokens.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import seeded_inputs as si
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover - GPU tests need a device
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import sparse_mixture_experts_25_b200 as moe  # noqa: E402
+
+W = si.WORKLOADS
+SMALL = {
+    # fp32 Switch-style top-1 with capacity: M tiles of 64, ragged d_f and d
+    "switch_small_f32": W["switch_top1_f32"].scaled("switch_small_f32", N=1000, d=72, d_f=96),
+    # Mixtral-shaped, bf16, k=2, uncapped: ragged N tile (d=320 -> 256 + 64)
+    "mixtral_small_bf16": W["mixtral_bf16"].scaled("mixtral_small_bf16", N=512, d=320, d_f=384),
+    # Qwen3-shaped with Zipf-biased hot experts and capacity drops
+    "qwen3_small_bf16": W["qwen3_skew_bf16"].scaled("qwen3_small_bf16", N=1024, d=256, d_f=192,
+                                                     E=32, k=4),
+    # DeepSeek-shaped with a shared expert of a different width
+    "deepseek_small_bf16": W["deepseek_shared_bf16"].scaled("deepseek_small_bf16", N=384, d=448,
+                                                             d_f=128, E=64, k=6, d_f_shared=192),
+    # WDMoE WLR pruning with per-token latencies
+    "wdmoe_small_bf16": W["wdmoe_decode_bf16"].scaled("wdmoe_small_bf16", N=64, d=512, d_f=640),
+    # bf16 Switch top-1 with capacity (full-probability weights)
+    "switch_small_bf16": W["switch_top1_f32"].scaled("switch_small_bf16", N=700, d=128, d_f=256,
+                                                      dtype=si.DT_BF16),
+    # all experts chosen (k = E_r), single expert group, fp32
+    "all_experts_f32": W["switch_top1_f32"].scaled("all_experts_f32", N=130, d=64, d_f=64, E=4, k=4,
+                                                   norm=si.NORM_RENORM, c=0.0),
+    "one_expert_bf16": W["mixtral_bf16"].scaled("one_expert_bf16", N=200, d=64, d_f=136, E=1, k=1),
+}
+
+
+def _end_to_end(w):
+    inp = si.inputs(w)
+    out = parity.gpu_forward(w, inp)
+    r, near = parity.check_routing(w, inp, out["rec"])
+    parity.check_dispatch(w, out["rec"], out["stats"])
+    err = parity.check_rows(w, inp, out["rec"], out["Y"])
+    flips = int((out["rec"]["ids"] != r["ids"]).any(axis=1).sum())
+    if flips == 0:
+        # routing identical: compare against the oracle's whole forward as well
+        full = oracle.forward(inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], k=w.k,
+                              norm=w.norm, c=w.c, theta=w.theta, b_r=inp.get("b_r"),
+                              lat=inp.get("lat"),
+                              Ws=(inp.get("Ws_g"), inp.get("Ws_u"), inp.get("Ws_d")) if w.d_f_shared else None)
+        assert parity.rel_err(out["Y"], full["Y"]) <= parity.TOL[w.dtype]
+    assert out["status"] == moe.MOE_OK
+    return out, err, int(near.sum())
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_small(name):
+    out, err, near = _end_to_end(SMALL[name])
+    print(f"{name}: max-abs-rel {err:.2e}, near-ties {near}, stats {out['stats']}")
+
+
+def test_switch_top1_f32_full():
+    """The Switch-shaped fp32 layer at its full size, every output row."""
+    out, err, near = _end_to_end(W["switch_top1_f32"])
+    assert out["stats"]["C"] == 160
+    print(f"switch_top1_f32: max-abs-rel {err:.2e}, near-ties {near}, stats {out['stats']}")
+
+
+def test_capacity_drops_give_zero_rows():
+    w = W["switch_top1_f32"].scaled("tight_capacity", N=256, d=64, d_f=64, c=0.25)
+    inp = si.inputs(w)
+    out = parity.gpu_forward(w, inp)
+    parity.check_dispatch(w, out["rec"], out["stats"])
+    dropped = (out["rec"]["slot"] < 0).all(axis=1)
+    assert dropped.sum() > 0
+    assert (out["Y"][dropped] == 0).all()
+    parity.check_rows(w, inp, out["rec"], out["Y"])
+
+
+def test_single_token_and_empty_batch():
+    w = W["mixtral_bf16"].scaled("one_token", N=1, d=64, d_f=64)
+    _end_to_end(w)
+    w0 = W["mixtral_bf16"].scaled("empty", N=0, d=64, d_f=64)
+    p = parity.params_of(w0)
+    ws = torch.zeros(max(moe.moe_workspace_size(p), 256), dtype=torch.uint8, device="cuda")
+    x = torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda")
+    Y = torch.zeros(8, 64, device="cuda")
+    moe.moe_forward(p, x, x, None, None, x, x, x, None, None, None, Y, ws)
+    status, stats = moe.moe_get_stats(p, ws)
+    assert status == moe.MOE_OK and stats["requested"] == 0
+
+
+def test_nonfinite_scores_are_reported():
+    w = W["mixtral_bf16"].scaled("nonfinite", N=100, d=64, d_f=64)
+    inp = si.inputs(w)
+    x = inp["x"].copy()
+    x[7, 3] = si.f32_to_bf16_bits(np.array([np.inf], np.float32))[0]
+    inp["x"] = x
+    out = parity.gpu_forward(w, inp)
+    assert out["status"] == moe.MOE_ERR_NONFINITE
+    assert out["stats"]["nonfinite"] == 1
+    assert (out["rec"]["ids"][7] == -1).all()
+    assert (out["Y"][7] == 0).all()
+    parity.check_dispatch(w, out["rec"], out["stats"])
+
+
+# ---------------------------------------------------------------------------
+# the page examples through the individual entry points
+# ---------------------------------------------------------------------------
+def _route_dispatch(p, x, W_r, C):
+    N, k, E = p.N, p.k, p.E_r
+    ws = torch.zeros(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+    ids = torch.empty(N, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(N, k, dtype=torch.float32, device="cuda")
+    margin = torch.empty(N, dtype=torch.float32, device="cuda")
+    moe.moe_route(p, x, W_r, None, None, ids, w, margin, ws)
+    slot = torch.empty(N, k, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    st = torch.empty(N * k, dtype=torch.int32, device="cuda")
+    sw = torch.empty(N * k, dtype=torch.float32, device="cuda")
+    moe.moe_dispatch(p, ids, w, C, slot, offsets, st, sw, None, None, ws)
+    return dict(ids=ids, w=w, slot=slot, offsets=offsets, st=st, sw=sw, ws=ws)
+
+
+def test_four_expert_example_through_route_and_combine():
+    # vegetog sec. 2-3: probabilities (0.12, 0.48, 0.08, 0.32), k = 2 -> weights 0.6/0.4,
+    # E1(x) = [2, 4], E3(x) = [8, 1] -> y = [4.4, 2.8]   (d padded to 8 with zeros)
+    p = moe.params(1, 8, 8, 4, 2, dtype=moe.MOE_F32)
+    x = torch.zeros(1, 8, device="cuda")
+    x[0, 0] = 1.0
+    W_r = torch.zeros(4, 8, device="cuda")
+    W_r[:, 0] = torch.log(torch.tensor([0.12, 0.48, 0.08, 0.32], device="cuda"))
+    r = _route_dispatch(p, x, W_r, C=1)
+    assert r["ids"].cpu().tolist() == [[1, 3]]
+    np.testing.assert_allclose(r["w"].cpu().numpy()[0], [0.6, 0.4], atol=1e-6)
+    H = torch.zeros(2, 8, device="cuda")
+    H[0, :2] = torch.tensor([2.0, 4.0])   # expert 1's row (offsets put expert 1 first)
+    H[1, :2] = torch.tensor([8.0, 1.0])   # expert 3's row
+    assert r["offsets"].cpu().tolist() == [0, 0, 1, 1, 2]
+    Y = torch.zeros(1, 8, device="cuda")
+    moe.moe_combine(p, H, r["offsets"], r["st"], r["sw"], Y)
+    np.testing.assert_allclose(Y.cpu().numpy()[0, :2], [4.4, 2.8], atol=1e-5)
+
+
+def test_n4_example_capacity_and_statistics():
+    # "LLM from scratch" ch. 36.4: N = 4, E_r = 3, k = 2, X = I_4, gamma = 1 -> C = 3,
+    # loads (3,4,1), accepted (3,3,1), token 4's path to expert 2 rejected, y_4 = 7/3 x_4
+    P = np.array([[0.7, 0.2, 0.1], [0.6, 0.3, 0.1], [0.55, 0.35, 0.1], [0.1, 0.2, 0.7]])
+    p = moe.params(4, 8, 8, 3, 2, c=1.0, dtype=moe.MOE_F32)
+    C = moe.moe_capacity(p)
+    assert C == 3
+    x = torch.zeros(4, 8, device="cuda")
+    x[:, :4] = torch.eye(4)
+    W_r = torch.zeros(3, 8, device="cuda")
+    W_r[:, :4] = torch.from_numpy(np.log(P).T.astype(np.float32)).cuda()
+    r = _route_dispatch(p, x, W_r, C)
+    status, s = moe.moe_get_stats(p, r["ws"])
+    assert s["requested"] == 8 and s["accepted"] == 7 and s["rejected"] == 1
+    assert s["tokens_affected"] == 1 and s["tokens_skipped"] == 0 and s["O"] == 1
+    assert s["rho_max"] == 1.5
+    views = moe.workspace_views(p, r["ws"])
+    assert views["L"].cpu().tolist() == [3, 4, 1]
+    assert views["acc"].cpu().tolist() == [3, 3, 1]
+    ids, slot = r["ids"].cpu().numpy(), r["slot"].cpu().numpy()
+    assert list(ids[3]) == [2, 1] and slot[3, 1] == -1
+    # linear experts F_e(x) = e x (1-based): H rows from the dispatched tokens
+    st = r["st"].cpu().numpy()
+    offs = r["offsets"].cpu().numpy()
+    H = np.zeros((7, 8), np.float32)
+    for e in range(3):
+        for row in range(offs[e], offs[e + 1]):
+            H[row, st[row]] = e + 1.0
+    Y = torch.zeros(4, 8, device="cuda")
+    moe.moe_combine(p, torch.from_numpy(H).cuda(), r["offsets"], r["st"], r["sw"], Y)
+    y = Y.cpu().numpy()
+    np.testing.assert_allclose(np.diag(y[:, :4]), [11 / 9, 4 / 3, 25 / 18, 7 / 3], atol=1e-5)
+
+
+# ---------------------------------------------------------------------------
+# the unfused entry points compose to the fused forward
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["mixtral_small_bf16", "switch_small_f32"])
+def test_unfused_path_matches_fused(name):
+    w = SMALL[name]
+    inp = si.inputs(w)
+    fused = parity.gpu_forward(w, inp)
+    dev = fused["dev"]
+    p = parity.params_of(w)
+    N, k, E, d = w.N, w.k, w.E, w.d
+    r = _route_dispatch_full(p, dev, w)
+    np.testing.assert_array_equal(r["ids"].cpu().numpy(), fused["rec"]["ids"])
+    H = torch.empty(N * k, d, dtype=torch.float32, device="cuda")
+    moe.moe_expert_ffn(p, r["x_perm"], r["offsets"], dev["W_g"], dev["W_u"], dev["W_d"], H, r["ws"])
+    # H rows against the oracle's expert on the gathered rows
+    offs = r["offsets"].cpu().numpy()
+    st = r["st"].cpu().numpy()
+    Hh = H.cpu().numpy().astype(np.float64)
+    for e in range(E):
+        lo, hi = offs[e], offs[e + 1]
+        if hi == lo:
+            continue
+        ref = oracle.swiglu_rows(inp["x"], st[lo:hi], inp["W_g"][e], inp["W_u"][e], inp["W_d"][e])
+        assert parity.rel_err(Hh[lo:hi], ref) <= parity.TOL[w.dtype]
+    Y = torch.zeros(N, d, device="cuda")
+    moe.moe_combine(p, H, r["offsets"], r["st"], r["sw"], Y)
+    assert parity.rel_err(Y.cpu().numpy().astype(np.float64), fused["Y"]) <= 1e-5
+
+
+def _route_dispatch_full(p, dev, w):
+    N, k, E, d = w.N, w.k, w.E, w.d
+    ws = torch.zeros(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+    ids = torch.empty(N, k, dtype=torch.int32, device="cuda")
+    wt = torch.empty(N, k, dtype=torch.float32, device="cuda")
+    moe.moe_route(p, dev["x"], dev["W_r"], dev.get("b_r"), dev.get("lat"), ids, wt, None, ws)
+    slot = torch.empty(N, k, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    st = torch.empty(N * k, dtype=torch.int32, device="cuda")
+    sw = torch.empty(N * k, dtype=torch.float32, device="cuda")
+    x_perm = torch.empty(N * k, d, dtype=dev["x"].dtype, device="cuda")
+    moe.moe_dispatch(p, ids, wt, moe.moe_capacity(p), slot, offsets, st, sw, dev["x"], x_perm, ws)
+    return dict(ids=ids, w=wt, slot=slot, offsets=offsets, st=st, sw=sw, x_perm=x_perm, ws=ws)
+
+
+# ---------------------------------------------------------------------------
+# full-size page-shaped layers: every token's routing and dispatch, sampled outputs
+# ---------------------------------------------------------------------------
+def _sample_tokens(N, n, seed):
+    rng = np.random.default_rng(seed)
+    pick = set(rng.choice(N, size=min(n, N), replace=False).tolist())
+    pick.update({0, N - 1})
+    return np.array(sorted(pick))
+
+
+@pytest.mark.parametrize("name,n_sample", [("mixtral_bf16", 12), ("qwen3_skew_bf16", 12),
+                                           ("wdmoe_decode_bf16", 16)])
+def test_full_size_sampled(name, n_sample):
+    w = W[name]
+    inp = si.inputs(w)
+    out = parity.gpu_forward(w, inp)
+    r, near = parity.check_routing(w, inp, out["rec"])
+    parity.check_dispatch(w, out["rec"], out["stats"])
+    toks = _sample_tokens(w.N, n_sample, 7)
+    err = parity.check_rows(w, inp, out["rec"], out["Y"], tokens=toks)
+    print(f"{name}: max-abs-rel {err:.2e} on {toks.size} tokens, near-ties {int(near.sum())}, "
+          f"stats {out['stats']}")
+    assert np.isfinite(out["Y"]).all()
+
+
+def test_full_size_deepseek_shared_sampled():
+    """DeepSeek-V3-shaped layer with the shared expert (22.6 GB of bf16 weights):
+    weights are generated and uploaded one expert at a time, and the oracle
+    regenerates only the experts its sampled tokens use."""
+    w = W["deepseek_shared_bf16"]
+    small = {n: si.tensor(w, n) for n in ("x", "W_r", "Ws_g", "Ws_u", "Ws_d")}
+    dev = {n: parity.to_dev(v) for n, v in small.items()}
+    for n in ("W_g", "W_u", "W_d"):
+        shp = si.shape(w, n)
+        t = torch.empty(shp, dtype=torch.bfloat16, device="cuda")
+        for e in range(w.E):
+            t[e].copy_(parity.to_dev(si.tensor(w, n, expert=e)))
+        dev[n] = t
+    out = parity.gpu_forward(w, small, dev=dev)
+    r, near = parity.check_routing(w, small, out["rec"])
+    parity.check_dispatch(w, out["rec"], out["stats"])
+    toks = _sample_tokens(w.N, 6, 11)
+    rec = out["rec"]
+    ref = np.zeros((toks.size, w.d))
+    cache = {}
+    for i, t in enumerate(toks):
+        for j in range(w.k):
+            e = int(rec["ids"][t, j])
+            if e < 0 or rec["slot"][t, j] < 0:
+                continue
+            if e not in cache:
+                cache.clear()
+                cache[e] = [si.tensor(w, n, expert=e) for n in ("W_g", "W_u", "W_d")]
+            g, u, dn = cache[e]
+            ref[i] += float(rec["w"][t, j]) * oracle.swiglu_rows(small["x"], [t], g, u, dn)[0]
+    ref += oracle.swiglu_rows(small["x"], toks, small["Ws_g"], small["Ws_u"], small["Ws_d"])
+    err = parity.rel_err(out["Y"][toks], ref)
+    print(f"deepseek_shared_bf16: max-abs-rel {err:.2e}, near-ties {int(near.sum())}, stats {out['stats']}")
+    assert err <= parity.TOL[w.dtype]
