@@ -48,12 +48,6 @@ def dist_env():
     return ws, rank, local
 
 
-def rank_workload(w: si.Workload, rank: int) -> si.Workload:
-    """Each rank draws its own token batch (seeded by rank); weights are the
-    same on every rank (tensor streams other than x keep the base seed)."""
-    return w
-
-
 def rank_x_seed(w: si.Workload, rank: int) -> int:
     return w.seed + 1000 * rank
 
@@ -109,7 +103,7 @@ def committed_traffic(kernel: str):
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
         ent = t.get(kernel)
-        if ent and ent.get("source_sha256_16") == kernel_source_hash() and ent.get("workload") == WORKLOAD:
+        if ent and ent.get("source_sha256_16") == kernel_source_hash():
             return ent.get("bytes_per_launch")
     except (OSError, ValueError):
         pass
@@ -387,7 +381,18 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(si.WORKLOADS))
     ap.add_argument("--ref-sample", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--override", action="append", default=[],
+                    help="key=value change of the workload shape (profiling of smaller cases)")
     args = ap.parse_args(argv)
+    if args.override:
+        w = si.WORKLOADS[args.workload]
+        kw = {}
+        for item in args.override:
+            key, val = item.split("=", 1)
+            kw[key] = type(getattr(w, key))(val)
+        name = w.name + "[" + ",".join(args.override) + "]"
+        si.WORKLOADS[name] = w.scaled(name, **kw)
+        args.workload = name
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -232,6 +232,10 @@ MOE_API moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats*
  */
 MOE_API moe_status moe_set_stage_events(void* const* events, int n);
 
+/* Text of the last CUDA failure seen by an entry point on the calling host
+ * thread ("" if none): the failing step and cudaGetErrorString's text. */
+MOE_API const char* moe_last_error(void);
+
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
 

@@ -19,7 +19,7 @@ __all__ = [
     "MoEError", "Params", "Stats", "WsLayout", "lib", "params", "moe_capacity",
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_dispatch",
     "moe_expert_ffn", "moe_combine", "moe_forward", "moe_get_stats",
-    "moe_set_stage_events", "moe_status_string", "workspace_views", "HEADER",
+    "moe_set_stage_events", "moe_status_string", "moe_last_error", "workspace_views", "HEADER",
 ]
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_NONFINITE = 0, 1, 2, 3
@@ -33,7 +33,10 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 class MoEError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {moe_status_string(status)} (status {status})")
+        detail = ""
+        if status == MOE_ERR_CUDA:
+            detail = f" [{moe_last_error()}]"
+        super().__init__(f"{where}: {moe_status_string(status)} (status {status}){detail}")
 
 
 class Params(ctypes.Structure):
@@ -83,6 +86,8 @@ def lib():
         L.moe_forward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_get_stats.argtypes = [pp, _P, ctypes.POINTER(Stats), _P]
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(_P), ctypes.c_int]
+        L.moe_last_error.argtypes = []
+        L.moe_last_error.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         for name in ("moe_capacity", "moe_workspace_size", "moe_workspace_layout", "moe_route",
@@ -130,6 +135,10 @@ def _stream(stream) -> Optional[int]:
 def _check(status: int, where: str):
     if status != MOE_OK:
         raise MoEError(status, where)
+
+
+def moe_last_error() -> str:
+    return lib().moe_last_error().decode()
 
 
 def moe_status_string(status: int) -> str:
@@ -191,8 +200,13 @@ def moe_get_stats(p, ws, stream=None):
 
 
 def moe_set_stage_events(events):
-    """events: list of torch.cuda.Event(enable_timing=True) (>= 5) or [] to stop."""
+    """events: list of torch.cuda.Event(enable_timing=True) (>= 5) or [] to stop.
+    torch creates the underlying CUDA event on its first record, so an event
+    without one is recorded once here to create it."""
     n = len(events)
+    for e in events:
+        if not e.cuda_event:
+            e.record()
     arr = (_P * max(n, 1))(*[e.cuda_event for e in events])
     _check(lib().moe_set_stage_events(arr if n else None, n), "moe_set_stage_events")
 

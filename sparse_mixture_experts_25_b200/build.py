@@ -19,7 +19,7 @@ NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",
     "--shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-    "-cudart", "static",
+    "-cudart", "shared",
     "--expt-relaxed-constexpr",
 ]
 

@@ -237,26 +237,35 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
                             const float* w, int32_t* slot, int32_t* offsets, int32_t* L,
                             int32_t* acc, int32_t* slot_token, float* slot_w, const void* x,
                             void* x_perm, unsigned long long* counters, const Scratch& sc,
-                            cudaStream_t st) {
+                            cudaStream_t st, const char** where) {
     const int E = p.E_r, k = p.k;
     const int n_tiles = sc.n_tiles;
+    cudaError_t e;
+    *where = "hist";
     hist_kernel<<<n_tiles, 256, sizeof(int) * E, st>>>(ids, p.N, k, E, sc.tile_tokens, n_tiles,
                                                         sc.hist, counters);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int threads = ((E + 31) / 32) * 32 < 64 ? 64 : ((E + 31) / 32) * 32;
+    *where = "scan";
     scan_kernel<<<1, threads, 0, st>>>(sc.hist, n_tiles, E, C, bm, L, acc, offsets, sc.mt_start,
                                        counters);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    *where = "assign";
     assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
                                                          n_tiles, sc.hist, offsets, slot,
                                                          slot_token, slot_w, counters);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (x && x_perm) {
+        *where = "gather";
         const int row_vec = (int)(p.d * esize(p.dtype) / 16);
         const int64_t rows = p.N * p.k;
         const int blocks = (int)min64(rows, (int64_t)num_sms() * 8);
         gather_kernel<<<blocks, 128, 0, st>>>(static_cast<const uint4*>(x),
                                               static_cast<uint4*>(x_perm), slot_token, offsets, E,
                                               row_vec);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    return cudaGetLastError();
+    return cudaSuccess;
 }
 
 cudaError_t launch_combine(const moe_params& p, const float* H, const int32_t* offsets,

@@ -2,6 +2,7 @@
 // stream-ordered launch sequence.  See include/moe.h for the contract of
 // every entry point.
 #include <math.h>
+#include <stdio.h>
 #include <string.h>
 
 #include <algorithm>
@@ -94,10 +95,17 @@ using namespace moe;
 namespace {
 
 thread_local cudaEvent_t g_stage_events[8];
+thread_local char g_last_error[256] = "";
+
+moe_status fail(cudaError_t e, const char* where) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e), (int)e);
+    return MOE_ERR_CUDA;
+}
 thread_local int g_stage_event_count = 0;
 
-inline void stage_mark(int i, cudaStream_t st) {
-    if (g_stage_event_count >= 5 && i < g_stage_event_count) cudaEventRecord(g_stage_events[i], st);
+inline cudaError_t stage_mark(int i, cudaStream_t st) {
+    if (g_stage_event_count >= 5 && i < g_stage_event_count) return cudaEventRecord(g_stage_events[i], st);
+    return cudaSuccess;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -117,7 +125,9 @@ moe_status check_params(const moe_params* p) {
     return MOE_OK;
 }
 
-moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+moe_status cuda_status(cudaError_t e, const char* where) {
+    return e == cudaSuccess ? MOE_OK : fail(e, where);
+}
 
 // exact capacity on the binary value of c (see moe.h)
 int64_t capacity_exact(double c, int64_t N, int k, int E) {
@@ -152,6 +162,8 @@ int64_t capacity_exact(double c, int64_t N, int k, int E) {
 }  // namespace
 
 extern "C" {
+
+const char* moe_last_error(void) { return g_last_error; }
 
 const char* moe_status_string(moe_status s) {
     switch (s) {
@@ -213,9 +225,11 @@ moe_status moe_route(const moe_params* p, const void* x, const void* W_r, const 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     WsView v;
     make_view(*p, ws, v);
-    if (cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st) != cudaSuccess) return MOE_ERR_CUDA;
+    (void)cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
+    if (e != cudaSuccess) return fail(e, "moe_route memset");
     return cuda_status(launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, ids,
-                                     w, margin, v.counters, nullptr, st));
+                                     w, margin, v.counters, nullptr, st), "moe_route router");
 }
 
 moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const float* w, int64_t C,
@@ -232,18 +246,26 @@ moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const float* w,
     WsView v;
     make_view(*p, ws, v);
     if (p->N == 0) {
-        if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p->E_r + 1), st) != cudaSuccess)
-            return MOE_ERR_CUDA;
+        cudaError_t e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p->E_r + 1), st);
+        if (e != cudaSuccess) return fail(e, "moe_dispatch memset");
         return MOE_OK;
     }
     if (!ids || !w || !slot || !slot_token || !slot_w) return MOE_ERR_INVALID_ARG;
+    (void)cudaGetLastError();
     // dispatch-side counters start from zero; router counters are kept
-    if (cudaMemsetAsync(v.counters + CNT_REQUESTED, 0, 6 * 8, st) != cudaSuccess ||
-        cudaMemsetAsync(v.counters + CNT_L_MAX, 0, 2 * 8, st) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    cudaError_t e = cudaMemsetAsync(v.counters + CNT_REQUESTED, 0, 6 * 8, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(v.counters + CNT_L_MAX, 0, 2 * 8, st);
+    if (e != cudaSuccess) return fail(e, "moe_dispatch memset");
     const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
-    return cuda_status(launch_dispatch(*p, C, bm, ids, w, slot, offsets, v.L, v.acc, slot_token,
-                                       slot_w, x, x_perm, v.counters, v.scratch, st));
+    const char* where = "";
+    e = launch_dispatch(*p, C, bm, ids, w, slot, offsets, v.L, v.acc, slot_token, slot_w, x, x_perm,
+                        v.counters, v.scratch, st, &where);
+    if (e != cudaSuccess) {
+        char buf[96];
+        snprintf(buf, sizeof(buf), "moe_dispatch %s", where);
+        return fail(e, buf);
+    }
+    return MOE_OK;
 }
 
 moe_status moe_expert_ffn(const moe_params* p, const void* x_perm, const int32_t* offsets,
@@ -263,23 +285,24 @@ moe_status moe_expert_ffn(const moe_params* p, const void* x_perm, const int32_t
     q.d_f_shared = 0;  // routed experts only
     ExpertWeights W{W_g, W_u, W_d, nullptr, nullptr, nullptr};
     const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
-    if (launch_mtile_prefix(p->E_r, bm, offsets, v.scratch.mt_start, st) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    (void)cudaGetLastError();
+    cudaError_t e0 = launch_mtile_prefix(p->E_r, bm, offsets, v.scratch.mt_start, st);
+    if (e0 != cudaSuccess) return fail(e0, "moe_expert_ffn prefix");
     int status = MOE_OK;
     cudaError_t e;
     if (p->dtype == MOE_BF16) {
         e = launch_tc_gate_up(q, x_perm, nullptr, offsets, v.scratch.mt_start, W, v.h, nullptr,
                               v.counters, st, &status);
-        if (e != cudaSuccess) return status != MOE_OK ? (moe_status)status : MOE_ERR_CUDA;
+        if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_expert_ffn gate/up: tensor map encode" : "moe_expert_ffn gate/up (tcgen05)");
         e = launch_tc_down(q, DOWN_STORE, v.h, nullptr, offsets, v.scratch.mt_start, W, nullptr,
                            nullptr, nullptr, H, v.counters, st, &status);
-        if (e != cudaSuccess) return status != MOE_OK ? (moe_status)status : MOE_ERR_CUDA;
+        if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_expert_ffn down: tensor map encode" : "moe_expert_ffn down (tcgen05)");
     } else {
         e = launch_simt_gate_up(q, x_perm, nullptr, offsets, v.scratch.mt_start, W, v.h, nullptr, st);
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        if (e != cudaSuccess) return fail(e, "moe_expert_ffn gate/up (fp32)");
         e = launch_simt_down(q, DOWN_STORE, v.h, nullptr, offsets, v.scratch.mt_start, W, nullptr,
                              nullptr, nullptr, H, st);
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        if (e != cudaSuccess) return fail(e, "moe_expert_ffn down (fp32)");
     }
     return MOE_OK;
 }
@@ -292,8 +315,9 @@ moe_status moe_combine(const moe_params* p, const float* H, const int32_t* offse
     if (p->N == 0) return MOE_OK;
     if (!H || !offsets || !slot_token || !slot_w || !Y || !aligned16(H) || !aligned16(Y))
         return MOE_ERR_INVALID_ARG;
+    (void)cudaGetLastError();
     return cuda_status(launch_combine(*p, H, offsets, slot_token, slot_w, Y,
-                                      reinterpret_cast<cudaStream_t>(stream)));
+                                      reinterpret_cast<cudaStream_t>(stream)), "moe_combine");
 }
 
 moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, const float* b_r,
@@ -307,7 +331,9 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     WsView v;
     make_view(*p, ws, v);
-    if (cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st) != cudaSuccess) return MOE_ERR_CUDA;
+    (void)cudaGetLastError();  // clear a stale non-sticky error left by earlier unrelated calls
+    cudaError_t e0 = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
+    if (e0 != cudaSuccess) return fail(e0, "moe_forward memset");
     if (p->N == 0) return MOE_OK;
     if (!x || !W_r || !W_g || !W_u || !W_d || !Y) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(W_r) || !aligned16(W_g) || !aligned16(W_u) || !aligned16(W_d) ||
@@ -320,34 +346,39 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     const int64_t C = capacity_exact(p->c, p->N, p->k, p->E_r);
     ExpertWeights W{W_g, W_u, W_d, sh ? Ws_g : nullptr, sh ? Ws_u : nullptr, sh ? Ws_d : nullptr};
 
-    stage_mark(0, st);
+    if ((e0 = stage_mark(0, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     cudaError_t e = launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, v.ids,
                                   v.w, v.margin, v.counters, Y, st);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    stage_mark(1, st);
+    if (e != cudaSuccess) return fail(e, "moe_forward router");
+    if ((e0 = stage_mark(1, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
+    const char* where = "";
     e = launch_dispatch(*p, C, bm, v.ids, v.w, v.slot, v.offsets, v.L, v.acc, v.slot_token, v.slot_w,
-                        x, v.x_perm, v.counters, v.scratch, st);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    stage_mark(2, st);
+                        x, v.x_perm, v.counters, v.scratch, st, &where);
+    if (e != cudaSuccess) {
+        char buf[96];
+        snprintf(buf, sizeof(buf), "moe_forward dispatch %s", where);
+        return fail(e, buf);
+    }
+    if ((e0 = stage_mark(2, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     int status = MOE_OK;
     if (p->dtype == MOE_BF16) {
         e = launch_tc_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared,
                               v.counters, st, &status);
-        if (e != cudaSuccess) return status != MOE_OK ? (moe_status)status : MOE_ERR_CUDA;
-        stage_mark(3, st);
+        if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_forward gate/up: tensor map encode" : "moe_forward gate/up (tcgen05)");
+        if ((e0 = stage_mark(3, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
         e = launch_tc_down(*p, DOWN_COMBINE, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
                            v.slot_token, v.slot_w, Y, nullptr, v.counters, st, &status);
-        if (e != cudaSuccess) return status != MOE_OK ? (moe_status)status : MOE_ERR_CUDA;
+        if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_forward down: tensor map encode" : "moe_forward down+combine (tcgen05)");
     } else {
         e = launch_simt_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, st);
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        stage_mark(3, st);
+        if (e != cudaSuccess) return fail(e, "moe_forward gate/up (fp32)");
+        if ((e0 = stage_mark(3, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
         e = launch_simt_down(*p, DOWN_COMBINE, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
                              v.slot_token, v.slot_w, Y, nullptr, st);
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        if (e != cudaSuccess) return fail(e, "moe_forward down+combine (fp32)");
     }
-    stage_mark(4, st);
+    if ((e0 = stage_mark(4, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     return MOE_OK;
 }
 
@@ -361,11 +392,11 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
     unsigned long long cnt[CNT_COUNT];
     std::vector<int32_t> L((size_t)p->E_r);
     memset(out, 0, sizeof(*out));
-    if (cudaMemcpyAsync(cnt, v.counters, sizeof(cnt), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-        cudaMemcpyAsync(L.data(), v.L, sizeof(int32_t) * L.size(), cudaMemcpyDeviceToHost, st) !=
-            cudaSuccess ||
-        cudaStreamSynchronize(st) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    cudaError_t e = cudaMemcpyAsync(cnt, v.counters, sizeof(cnt), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(L.data(), v.L, sizeof(int32_t) * L.size(), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(e, "moe_get_stats");
     out->C = (int64_t)cnt[CNT_C];
     out->requested = (int64_t)cnt[CNT_REQUESTED];
     out->accepted = (int64_t)cnt[CNT_ACCEPTED];

@@ -83,7 +83,7 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
                             const float* w, int32_t* slot, int32_t* offsets, int32_t* L,
                             int32_t* acc, int32_t* slot_token, float* slot_w, const void* x,
                             void* x_perm, unsigned long long* counters, const Scratch& sc,
-                            cudaStream_t st);
+                            cudaStream_t st, const char** where);
 cudaError_t launch_combine(const moe_params& p, const float* H, const int32_t* offsets,
                            const int32_t* slot_token, const float* slot_w, float* Y,
                            cudaStream_t st);

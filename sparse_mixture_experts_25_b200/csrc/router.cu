@@ -120,6 +120,13 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
             for (int j = 0; j < 8; ++j) wsm[(kc + j) * EPAD + e] = v[j];
         }
         __syncthreads();
+        // two-level fp32 summation: a fresh partial per 64-wide chunk, then
+        // added to the running score (error ~ (64 + d/64) ulp instead of d ulp)
+        float part[TT][TE];
+#pragma unroll
+        for (int i = 0; i < TT; ++i)
+#pragma unroll
+            for (int j = 0; j < TE; ++j) part[i][j] = 0.f;
 #pragma unroll 8
         for (int kk = 0; kk < kKC; ++kk) {
             float xv[TT], wv[TE];
@@ -130,8 +137,12 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
 #pragma unroll
             for (int i = 0; i < TT; ++i)
 #pragma unroll
-                for (int j = 0; j < TE; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+                for (int j = 0; j < TE; ++j) part[i][j] = fmaf(xv[i], wv[j], part[i][j]);
         }
+#pragma unroll
+        for (int i = 0; i < TT; ++i)
+#pragma unroll
+            for (int j = 0; j < TE; ++j) acc[i][j] += part[i][j];
         __syncthreads();
     }
 

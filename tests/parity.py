@@ -7,7 +7,10 @@ Comparison rules (stated once, used by every parity test):
     reported and excluded from id equality;
   * dispatch is checked bit-exactly by running the oracle's dispatch on the
     GPU's own ids (one flipped near-tie would shift later slots otherwise);
-  * weights: |a_gpu - a_oracle| <= 2e-6 + 2e-6 |a| (fp32 softmax vs double);
+  * weights: |a_gpu - a_oracle| <= 3e-5 (1 + |a|): the GPU accumulates router
+    scores in fp32 over d products (two-level, 64-wide chunks), an error of
+    order sqrt(d) 2^-24 |x||w| (~1e-6 .. 1e-5 at d = 4096..7168), and a
+    softmax weight moves by at most about twice the largest score error;
   * outputs: max|Y_gpu - Y_ref| / max|Y_ref| <= 1e-4 (fp32 layers) or 2e-2
     (bf16 layers, fp32 accumulation), with Y_ref the oracle's output
     computed from the GPU's routing records; rows whose every path was
@@ -70,7 +73,7 @@ def check_routing(w: si.Workload, inp: dict, rec: dict):
     ok = ~near & ~r["invalid"]
     assert (rec["ids"][ok] == r["ids"][ok]).all(), "routing ids differ on tokens that are not near-ties"
     same = ok[:, None] & (rec["ids"] == r["ids"])
-    np.testing.assert_allclose(rec["w"][same], r["w"][same], rtol=2e-6, atol=2e-6)
+    np.testing.assert_allclose(rec["w"][same], r["w"][same], rtol=3e-5, atol=3e-5)
     assert (rec["ids"][r["invalid"]] == -1).all()
     # margin reported by the GPU (fp32) agrees with the oracle's (double)
     fin = ok & np.isfinite(r["margin"])

@@ -291,3 +291,28 @@ def test_full_size_deepseek_shared_sampled():
     err = parity.rel_err(out["Y"][toks], ref)
     print(f"deepseek_shared_bf16: max-abs-rel {err:.2e}, near-ties {int(near.sum())}, stats {out['stats']}")
     assert err <= parity.TOL[w.dtype]
+
+
+def test_forward_on_a_side_stream_with_stage_events():
+    """Launches go to the caller's stream (a non-default torch stream here)
+    and the optional stage events are recorded on it."""
+    w = SMALL["mixtral_small_bf16"]
+    inp = si.inputs(w)
+    ref = parity.gpu_forward(w, inp)
+    dev = ref["dev"]
+    p = parity.params_of(w)
+    s = torch.cuda.Stream()
+    ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+    Y = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    with torch.cuda.stream(s):
+        moe.moe_set_stage_events(ev)
+        try:
+            moe.moe_forward(p, dev["x"], dev["W_r"], None, None, dev["W_g"], dev["W_u"], dev["W_d"],
+                            None, None, None, Y, ws, s)
+        finally:
+            moe.moe_set_stage_events([])
+    s.synchronize()
+    times = [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
+    assert all(t >= 0 for t in times)
+    np.testing.assert_allclose(Y.cpu().numpy(), ref["Y"], rtol=0, atol=1e-5)
