@@ -178,6 +178,36 @@ MOE_API moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const f
                         const void* x, void* x_perm, void* ws, moe_stream_t stream);
 
 /*
+ * moe_dispatch without a workspace, for callers that cannot allocate device
+ * memory where they dispatch: code running under a memory pool that may not
+ * grow, embedders whose allocator is not reachable from the call site, and
+ * call sites that must not call cudaMalloc because it can synchronise the
+ * device.  The pages have no counterpart of this entry point; it computes
+ * exactly what moe_dispatch computes (same arguments, minus ws) and fills
+ * the same outputs.
+ *
+ * Its scratch (per-tile request counts, per-expert loads, M-tile prefix,
+ * counters) lives in a 1 MiB array inside the library, which every GPU that
+ * loads the library holds until the process exits.  Limit:
+ * E_r * n_tiles + 3 E_r + 33 four-byte words must fit in 1 MiB, with
+ * n_tiles = ceil(N / max(8, floor(256 / k))) (for example N = 8192, k = 8,
+ * E_r = 128 needs 132 KB); larger sizes return MOE_ERR_UNSUPPORTED with the
+ * required size in moe_last_error.  The routing statistics of this call
+ * stay inside the array and are not readable through moe_get_stats.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call shares the array: a call clears the counters it accumulates and
+ * overwrites the rest, and the array keeps the last call's contents.  Calls
+ * that overlap on the GPU (unordered streams or threads) race on it.  The
+ * entry point allocates no memory, host or device.
+ */
+MOE_API moe_status moe_dispatch_noalloc(const moe_params* p, const int32_t* ids, const float* w,
+                                        int64_t C, int32_t* slot, int32_t* offsets,
+                                        int32_t* slot_token, float* slot_w, const void* x,
+                                        void* x_perm, moe_stream_t stream);
+
+/*
  * Routed SwiGLU experts on the dispatched rows (vegetog sec. 3:
  * E_i(x) = [SiLU(x W_gate,i) (.) (x W_up,i)] W_down,i; ch. 36.3: each expert
  * runs only on its accepted slots).

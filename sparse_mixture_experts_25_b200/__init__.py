@@ -18,6 +18,7 @@ from . import build as _build
 __all__ = [
     "MoEError", "Params", "Stats", "WsLayout", "lib", "params", "moe_capacity",
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_dispatch",
+    "moe_dispatch_noalloc",
     "moe_expert_ffn", "moe_combine", "moe_forward", "moe_get_stats",
     "moe_set_stage_events", "moe_status_string", "moe_last_error", "workspace_views", "HEADER",
 ]
@@ -34,7 +35,7 @@ class MoEError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         detail = ""
-        if status == MOE_ERR_CUDA:
+        if status in (MOE_ERR_CUDA, MOE_ERR_UNSUPPORTED) and moe_last_error():
             detail = f" [{moe_last_error()}]"
         super().__init__(f"{where}: {moe_status_string(status)} (status {status}){detail}")
 
@@ -81,6 +82,7 @@ def lib():
         L.moe_workspace_layout.argtypes = [pp, ctypes.POINTER(WsLayout)]
         L.moe_route.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_dispatch.argtypes = [pp, _P, _P, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_dispatch_noalloc.argtypes = [pp, _P, _P, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P]
         L.moe_expert_ffn.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_combine.argtypes = [pp, _P, _P, _P, _P, _P, _P]
         L.moe_forward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
@@ -91,7 +93,8 @@ def lib():
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         for name in ("moe_capacity", "moe_workspace_size", "moe_workspace_layout", "moe_route",
-                     "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
+                     "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine",
+                     "moe_forward",
                      "moe_get_stats", "moe_set_stage_events"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -172,6 +175,14 @@ def moe_dispatch(p, ids, w, C, slot, offsets, slot_token, slot_w, x, x_perm, ws,
     _check(lib().moe_dispatch(ctypes.byref(p), _ptr(ids), _ptr(w), int(C), _ptr(slot), _ptr(offsets),
                               _ptr(slot_token), _ptr(slot_w), _ptr(x), _ptr(x_perm), _ptr(ws),
                               _stream(stream)), "moe_dispatch")
+
+
+def moe_dispatch_noalloc(p, ids, w, C, slot, offsets, slot_token, slot_w, x, x_perm, stream=None):
+    """moe_dispatch with its scratch in the library's static device buffer
+    (for callers that cannot allocate device memory at the call site)."""
+    _check(lib().moe_dispatch_noalloc(ctypes.byref(p), _ptr(ids), _ptr(w), int(C), _ptr(slot),
+                                      _ptr(offsets), _ptr(slot_token), _ptr(slot_w), _ptr(x),
+                                      _ptr(x_perm), _stream(stream)), "moe_dispatch_noalloc")
 
 
 def moe_expert_ffn(p, x_perm, offsets, W_g, W_u, W_d, H, ws, stream=None):

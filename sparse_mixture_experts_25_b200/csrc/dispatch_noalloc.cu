@@ -1,0 +1,142 @@
+// moe_dispatch_noalloc: the dispatch step with its scratch memory in a fixed,
+// library-owned device buffer instead of a caller-provided workspace.
+//
+// Why it exists: some callers cannot allocate device memory at the point
+// where they dispatch.  Examples are code running inside a memory pool that
+// forbids growth, embedders whose allocator is not reachable from the call
+// site, and call sites that must not call cudaMalloc because it can
+// synchronise the device.  This variant takes only the inputs and outputs of
+// moe_dispatch; its per-tile histograms, per-expert counts, M-tile prefix and
+// counters live in a file-scope __device__ array of kScratchBytes (1 MiB).
+// Every GPU that loads the library holds that array until the process exits.
+//
+// The array is shared by every call: each call overwrites it and clears the
+// counters that must start at zero, and the buffer keeps the last call's
+// contents afterwards.  Calls that overlap on the GPU (different streams or
+// threads without ordering between them) race on it.
+#include <mutex>
+#include <stdio.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr size_t kScratchBytes = size_t(1) << 20;  // 1 MiB
+
+// Scratch layout (bytes from the start of the array):
+//   [0, 128)                          int64 counters[16]
+//   [128, 128 + 4 E)                  int32 L[E]
+//   next 4 E                          int32 acc[E]
+//   next 4 (E + 1)                    int32 M-tile prefix[E + 1]
+//   next 4 E n_tiles                  int32 per-tile histograms [E][n_tiles]
+static __device__ __align__(256) unsigned char g_dispatch_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices] = {nullptr};
+std::mutex g_setup_mutex;
+
+size_t scratch_needed(const moe_params& p, int n_tiles) {
+    const size_t E = (size_t)p.E_r;
+    return 128 + 4 * E + 4 * E + 4 * (E + 1) + 4 * E * (size_t)(n_tiles > 0 ? n_tiles : 1);
+}
+
+// Device address of the scratch array for the current device (set-up on the
+// first call per device: a symbol-address query with that device current).
+cudaError_t scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    if (!g_scratch_addr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_dispatch_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_addr[dev] = ptr;
+    }
+    *out = g_scratch_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_dispatch_noalloc(const moe_params* p, const int32_t* ids, const float* w, int64_t C,
+                                int32_t* slot, int32_t* offsets, int32_t* slot_token,
+                                float* slot_w, const void* x, void* x_perm, moe_stream_t stream) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    moe_ws_layout lay;
+    moe_status s = moe_workspace_layout(p, &lay);  // validates the parameters
+    if (s != MOE_OK) return s;
+    if (C < 1 || !offsets) return MOE_ERR_INVALID_ARG;
+    if ((x != nullptr) != (x_perm != nullptr)) return MOE_ERR_INVALID_ARG;
+    if (x && ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u)))
+        return MOE_ERR_INVALID_ARG;
+    const int tile_tokens = dispatch_tile_tokens(p->k);
+    const int n_tiles = (int)((p->N + tile_tokens - 1) / tile_tokens);
+    const size_t need = scratch_needed(*p, n_tiles);
+    if (need > kScratchBytes) {
+        char msg[256];
+        snprintf(msg, sizeof(msg),
+                 "moe_dispatch_noalloc: these sizes need %zu bytes of scratch, the static buffer "
+                 "holds %zu (E_r per-tile counts for each tile of max(8, 256/k) tokens); use moe_dispatch",
+                 need, kScratchBytes);
+        record_error(msg);
+        return MOE_ERR_UNSUPPORTED;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* base = nullptr;
+    cudaError_t e = scratch_address(&base);
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof(msg), "moe_dispatch_noalloc set-up: %s", cudaGetErrorString(e));
+        record_error(msg);
+        return MOE_ERR_CUDA;
+    }
+    if (p->N == 0) {
+        e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p->E_r + 1), st);
+        if (e != cudaSuccess) {
+            record_error("moe_dispatch_noalloc: memset of offsets failed");
+            return MOE_ERR_CUDA;
+        }
+        return MOE_OK;
+    }
+    if (!ids || !w || !slot || !slot_token || !slot_w) return MOE_ERR_INVALID_ARG;
+    char* b = static_cast<char*>(base);
+    const size_t E = (size_t)p->E_r;
+    unsigned long long* counters = reinterpret_cast<unsigned long long*>(b);
+    int32_t* L = reinterpret_cast<int32_t*>(b + 128);
+    int32_t* acc = L + E;
+    Scratch sc;
+    sc.mt_start = acc + E;
+    sc.hist = sc.mt_start + E + 1;
+    sc.n_tiles = n_tiles;
+    sc.tile_tokens = tile_tokens;
+    (void)cudaGetLastError();
+    // the counters are accumulated with atomics: start them at zero each call
+    e = cudaMemsetAsync(counters, 0, CNT_COUNT * sizeof(unsigned long long), st);
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof(msg), "moe_dispatch_noalloc: %s", cudaGetErrorString(e));
+        record_error(msg);
+        return MOE_ERR_CUDA;
+    }
+    const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
+    const char* where = "";
+    e = launch_dispatch(*p, C, bm, ids, w, slot, offsets, L, acc, slot_token, slot_w, x, x_perm,
+                        counters, sc, st, &where);
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof(msg), "moe_dispatch_noalloc %s: %s", where, cudaGetErrorString(e));
+        record_error(msg);
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -161,6 +161,10 @@ int64_t capacity_exact(double c, int64_t N, int k, int E) {
 
 }  // namespace
 
+namespace moe {
+void record_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+}  // namespace moe
+
 extern "C" {
 
 const char* moe_last_error(void) { return g_last_error; }

@@ -67,6 +67,7 @@ struct WsView {
 };
 
 // Host helpers (moe_api.cu)
+void record_error(const char* msg);  // text returned by moe_last_error on this thread
 int dispatch_tile_tokens(int k);
 size_t esize(int dtype);
 bool make_view(const moe_params& p, void* ws, WsView& v);
