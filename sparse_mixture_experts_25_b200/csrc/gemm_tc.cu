@@ -74,6 +74,8 @@ struct TcArgs {
     int ldY;
     int max_rows;             // rows of the routed A / output buffers (N k)
     int n_tokens;             // N
+    int has_routed;           // 0: only the second (dense) segment runs
+    int ks;                   // K splits per output tile (partial sums reduced with red.add)
     unsigned long long* counters;
 };
 
@@ -252,7 +254,7 @@ struct Tile {
     int a_row;      // first row of the A tile in its matrix
     int rows;       // valid rows (<= BM)
     int n_tile;     // output-column tile
-    int nkb;        // K blocks
+    int kb0, kb1;   // K blocks [kb0, kb1) of this tile
 };
 
 struct SchedSmem {
@@ -260,8 +262,11 @@ struct SchedSmem {
     int32_t off[kMaxExperts + 1];
 };
 
-__device__ __forceinline__ bool decode_tile(int t, const SchedSmem& s, const TcArgs& a, int routed_tiles,
-                                            Tile& ti) {
+__device__ __forceinline__ bool decode_tile(int t_in, const SchedSmem& s, const TcArgs& a,
+                                            int routed_tiles, Tile& ti) {
+    // K split fastest: consecutive tiles are the K slices of one output tile
+    const int kq = t_in % a.ks;
+    const int t = t_in / a.ks;
     if (t < routed_tiles) {
         const int q = t / a.nt_r;
         // last group g with mt[g] <= q (non-empty, since mt[g+1] > q)
@@ -275,7 +280,8 @@ __device__ __forceinline__ bool decode_tile(int t, const SchedSmem& s, const TcA
         const int mtiles = s.mt[g + 1] - s.mt[g];
         ti.shared = 0;
         ti.g = g;
-        ti.nkb = a.nkb_r;
+        ti.kb0 = (int)((int64_t)kq * a.nkb_r / a.ks);
+        ti.kb1 = (int)((int64_t)(kq + 1) * a.nkb_r / a.ks);
         if (mtiles <= 0) {  // inconsistent prefix (caller-supplied offsets): no rows
             ti.n_tile = 0;
             ti.a_row = 0;
@@ -299,7 +305,8 @@ __device__ __forceinline__ bool decode_tile(int t, const SchedSmem& s, const TcA
     ti.n_tile = local / mt_sh;
     ti.a_row = (local % mt_sh) * BM;
     ti.rows = min(BM, a.M_sh - ti.a_row);
-    ti.nkb = a.nkb_sh;
+    ti.kb0 = (int)((int64_t)kq * a.nkb_sh / a.ks);
+    ti.kb1 = (int)((int64_t)(kq + 1) * a.nkb_sh / a.ks);
     return true;
 }
 
@@ -333,9 +340,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    for (int i = threadIdx.x; i <= a.E; i += NUM_THREADS) {
-        sched->mt[i] = a.mt_start[i];
-        sched->off[i] = a.offsets[i];
+    if (a.has_routed) {
+        for (int i = threadIdx.x; i <= a.E; i += NUM_THREADS) {
+            sched->mt[i] = a.mt_start[i];
+            sched->off[i] = a.offsets[i];
+        }
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -366,8 +375,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_s;
 
-    const int routed_tiles = sched->mt[a.E] * a.nt_r;
-    const int total_tiles = routed_tiles + (a.M_sh > 0 ? ((a.M_sh + BM - 1) / BM) * a.nt_sh : 0);
+    const int routed_tiles = a.has_routed ? sched->mt[a.E] * a.nt_r : 0;
+    const int total_tiles =
+        (routed_tiles + (a.M_sh > 0 ? ((a.M_sh + BM - 1) / BM) * a.nt_sh : 0)) * a.ks;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -390,7 +400,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     b_row0 = (ti.shared ? 0 : ti.g * a.b_rows_r) + ti.n_tile * 256;
                     b_row1 = b_row0 + 128;
                 }
-                for (int kb = 0; kb < ti.nkb; ++kb) {
+                for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, a.counters)) {
                         ok = false;
                         break;
@@ -429,7 +439,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, a.counters)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < ti.nkb; ++kb) {
+                for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!wait_bounded(&full[stage], phase, abort_flag, a.counters)) {
                         ok = false;
                         break;
@@ -443,7 +453,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         // advance 16 elements (32 bytes) along K inside the swizzled row
                         umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2),
-                                  (kb | kk) ? 1u : 0u);
+                                  (kb > ti.kb0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&empty[stage]);
                     if (++stage == STAGES) {
@@ -540,7 +550,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                 const float x1 = __uint_as_float(v[q * 4 + 1]) * wgt;
                                 const float x2 = __uint_as_float(v[q * 4 + 2]) * wgt;
                                 const float x3 = __uint_as_float(v[q * 4 + 3]) * wgt;
-                                if (EPI == EPI_COMBINE) {
+                                if (EPI == EPI_COMBINE || a.ks > 1) {
                                     red_add_v4(p, x0, x1, x2, x3);
                                 } else {
                                     *reinterpret_cast<float4*>(p) = make_float4(x0, x1, x2, x3);
@@ -614,6 +624,34 @@ int64_t routed_mtile_bound(const moe_params& p) {
     return (p.N * p.k + BM - 1) / BM + p.E_r;
 }
 
+// Expected routed M tiles: each expert gets about mu = N k / E_r rows (at most
+// C); a group of r rows takes ceil(r / 128) tiles, about r / 128 + 1/2 on average.
+double routed_mtile_estimate(const moe_params& p, int64_t C) {
+    double mu = (double)p.N * p.k / p.E_r;
+    if (mu > (double)C) mu = (double)C;
+    if (mu <= 0) return 0;
+    const double per = mu / BM + 0.5;
+    return p.E_r * (per < 1.0 ? 1.0 : per);
+}
+
+// K splits for an output-tile count: minimise the number of full waves of
+// tile-time (ceil(tiles * ks / SMs) / ks), keeping >= 8 K blocks per slice.
+int choose_ksplit(double tiles, int nkb_min) {
+    const int sms = num_sms();
+    int best = 1;
+    double best_cost = 1e30;
+    for (int ks = 1; ks <= 8; ++ks) {
+        if (ks > 1 && nkb_min / ks < 8) break;
+        const double waves = ceil(tiles * ks / sms - 1e-9);
+        const double cost = waves / ks;
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = ks;
+        }
+    }
+    return best;
+}
+
 }  // namespace
 
 cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
@@ -658,13 +696,15 @@ cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const voi
     a.ld_out_sh = p.d_f_shared;
     a.max_rows = (int)(p.N * p.k);
     a.n_tokens = (int)p.N;
+    a.has_routed = 1;
+    a.ks = 1;  // the SwiGLU epilogue needs the whole K sum
     a.counters = counters;
     int64_t max_tiles = routed_mtile_bound(p) * a.nt_r + (sh ? ((p.N + BM - 1) / BM) * a.nt_sh : 0);
     return launch_tc<EPI_SWIGLU>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a, max_tiles, st);
 }
 
-cudaError_t launch_tc_down(const moe_params& p, int mode, const void* h, const void* h_shared,
-                           const int32_t* offsets, const int32_t* mt_start,
+cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void* h,
+                           const void* h_shared, const int32_t* offsets, const int32_t* mt_start,
                            const ExpertWeights& W, const int32_t* slot_token,
                            const float* slot_w, float* Y, float* H_out,
                            unsigned long long* counters, cudaStream_t st, int* status) {
@@ -704,11 +744,50 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, const void* h, const v
     a.ldY = p.d;
     a.max_rows = (int)(p.N * p.k);
     a.n_tokens = (int)p.N;
+    a.has_routed = 1;
+    a.ks = 1;
+    if (mode == DOWN_COMBINE) {
+        // the combine reduces with red.add into a zeroed Y, so K slices of one
+        // output tile can run on different SMs: split K to fill the last wave
+        const double tiles = routed_mtile_estimate(p, C) * a.nt_r +
+                             (sh ? (double)((p.N + BM - 1) / BM) * a.nt_sh : 0.0);
+        a.ks = choose_ksplit(tiles, sh ? std::min(a.nkb_r, a.nkb_sh) : a.nkb_r);
+    }
     a.counters = counters;
-    int64_t max_tiles = routed_mtile_bound(p) * a.nt_r + (sh ? ((p.N + BM - 1) / BM) * a.nt_sh : 0);
+    int64_t max_tiles =
+        (routed_mtile_bound(p) * a.nt_r + (sh ? ((p.N + BM - 1) / BM) * a.nt_sh : 0)) * a.ks;
     if (mode == DOWN_COMBINE)
         return launch_tc<EPI_COMBINE>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
     return launch_tc<EPI_STORE>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
+}
+
+cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,
+                             unsigned long long* counters, cudaStream_t st, int* status) {
+    *status = MOE_OK;
+    CUtensorMap mA, mB;
+    if (!make_map(&mA, x, (uint64_t)p.N, p.d) || !make_map(&mB, W_r, (uint64_t)p.E_r, p.d)) {
+        *status = MOE_ERR_CUDA;
+        return cudaErrorInvalidValue;
+    }
+    TcArgs a{};
+    a.E = 0;
+    a.has_routed = 0;
+    a.M_sh = (int)p.N;
+    a.nt_sh = (p.E_r + BN - 1) / BN;
+    a.nkb_sh = (p.d + BK - 1) / BK;
+    a.n_valid_sh = p.E_r;
+    a.out = logits;
+    a.ld_out = p.E_r;
+    a.max_rows = (int)p.N;
+    a.n_tokens = (int)p.N;
+    const int64_t tiles = ((p.N + BM - 1) / BM) * a.nt_sh;
+    a.ks = choose_ksplit((double)tiles, a.nkb_sh);
+    a.counters = counters;
+    if (a.ks > 1) {  // K slices add into the scores with red.add
+        cudaError_t e = cudaMemsetAsync(logits, 0, sizeof(float) * (size_t)p.N * p.E_r, st);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_tc<EPI_STORE>(mA, mB, mB, mA, mB, mB, a, tiles * a.ks, st);
 }
 
 }  // namespace moe

@@ -58,7 +58,9 @@ static bool layout(const moe_params& p, moe_ws_layout& L, int& n_tiles, int& til
     L.x_perm = take(Nk * (size_t)p.d * es);
     L.h = take(Nk * (size_t)p.d_f * es);
     L.h_shared = take((size_t)p.N * (size_t)(p.d_f_shared > 0 ? p.d_f_shared : 0) * es);
-    L.scratch = take(E * (size_t)std::max(n_tiles, 1) * 4 + (E + 1) * 4);
+    // scratch: per-tile histograms, M-tile prefix, then (16-byte aligned) router scores
+    L.scratch = take(align_up(E * (size_t)std::max(n_tiles, 1) * 4 + (E + 1) * 4, 256) +
+                     (size_t)p.N * E * 4);
     L.total = off;
     return true;
 }
@@ -83,6 +85,9 @@ bool make_view(const moe_params& p, void* ws, WsView& v) {
     v.h_shared = b + v.lay.h_shared;
     v.scratch.hist = reinterpret_cast<int32_t*>(b + v.lay.scratch);
     v.scratch.mt_start = v.scratch.hist + (size_t)p.E_r * std::max(n_tiles, 1);
+    v.scratch.logits = reinterpret_cast<float*>(
+        b + v.lay.scratch +
+        align_up((size_t)p.E_r * std::max(n_tiles, 1) * 4 + ((size_t)p.E_r + 1) * 4, 256));
     v.scratch.n_tiles = n_tiles;
     v.scratch.tile_tokens = tile_tokens;
     return true;
@@ -233,7 +238,8 @@ moe_status moe_route(const moe_params* p, const void* x, const void* W_r, const 
     cudaError_t e = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
     if (e != cudaSuccess) return fail(e, "moe_route memset");
     return cuda_status(launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, ids,
-                                     w, margin, v.counters, nullptr, st), "moe_route router");
+                                     w, margin, v.counters, nullptr, v.scratch.logits, st),
+                       "moe_route router");
 }
 
 moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const float* w, int64_t C,
@@ -298,7 +304,7 @@ moe_status moe_expert_ffn(const moe_params* p, const void* x_perm, const int32_t
         e = launch_tc_gate_up(q, x_perm, nullptr, offsets, v.scratch.mt_start, W, v.h, nullptr,
                               v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_expert_ffn gate/up: tensor map encode" : "moe_expert_ffn gate/up (tcgen05)");
-        e = launch_tc_down(q, DOWN_STORE, v.h, nullptr, offsets, v.scratch.mt_start, W, nullptr,
+        e = launch_tc_down(q, DOWN_STORE, p->N, v.h, nullptr, offsets, v.scratch.mt_start, W, nullptr,
                            nullptr, nullptr, H, v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_expert_ffn down: tensor map encode" : "moe_expert_ffn down (tcgen05)");
     } else {
@@ -352,7 +358,7 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
 
     if ((e0 = stage_mark(0, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     cudaError_t e = launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, v.ids,
-                                  v.w, v.margin, v.counters, Y, st);
+                                  v.w, v.margin, v.counters, Y, v.scratch.logits, st);
     if (e != cudaSuccess) return fail(e, "moe_forward router");
     if ((e0 = stage_mark(1, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
@@ -371,7 +377,7 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
                               v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_forward gate/up: tensor map encode" : "moe_forward gate/up (tcgen05)");
         if ((e0 = stage_mark(3, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
-        e = launch_tc_down(*p, DOWN_COMBINE, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
+        e = launch_tc_down(*p, DOWN_COMBINE, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
                            v.slot_token, v.slot_w, Y, nullptr, v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_forward down: tensor map encode" : "moe_forward down+combine (tcgen05)");
     } else {

@@ -43,6 +43,7 @@ constexpr float kNearTie = 1e-5f;
 struct Scratch {
     int32_t* hist;        // [E][n_tiles] per-tile request counts -> exclusive bases
     int32_t* mt_start;    // [E+1] prefix of M tiles (BM of the GEMM in use)
+    float* logits;        // [N][E] router scores (tensor-core score path)
     int n_tiles;          // dispatch tiles
     int tile_tokens;      // tokens per dispatch tile
 };
@@ -76,9 +77,11 @@ bool make_view(const moe_params& p, void* ws, WsView& v);
 // Launchers (each returns cudaGetLastError() of its launch)
 // ---------------------------------------------------------------------------
 // router.cu
+// logits: [N, E_r] fp32 scratch for the tensor-core score path (may be null)
 cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, const float* b_r,
                           const float* lat, int32_t* ids, float* w, float* margin,
-                          unsigned long long* counters, float* Y_zero, cudaStream_t st);
+                          unsigned long long* counters, float* Y_zero, float* logits,
+                          cudaStream_t st);
 // dispatch.cu
 cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_t* ids,
                             const float* w, int32_t* slot, int32_t* offsets, int32_t* L,
@@ -106,11 +109,14 @@ cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const voi
                               const int32_t* offsets, const int32_t* mt_start,
                               const ExpertWeights& W, void* h, void* h_shared,
                               unsigned long long* counters, cudaStream_t st, int* status);
-cudaError_t launch_tc_down(const moe_params& p, int mode, const void* h, const void* h_shared,
-                           const int32_t* offsets, const int32_t* mt_start,
+cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void* h,
+                           const void* h_shared, const int32_t* offsets, const int32_t* mt_start,
                            const ExpertWeights& W, const int32_t* slot_token,
                            const float* slot_w, float* Y, float* H_out,
                            unsigned long long* counters, cudaStream_t st, int* status);
+// router scores G = x W_r^T (bf16 in, fp32 out [N, E_r]) on the tensor cores
+cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,
+                             unsigned long long* counters, cudaStream_t st, int* status);
 
 // gemm_simt.cu (fp32 CUDA-core path)
 cudaError_t launch_simt_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,

@@ -71,6 +71,133 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Softmax, top-k in rank order (score descending, ties to the lower expert
+// index), weights and records for one token.  The calling warp holds the
+// token's scores (bias included) as v[i] = g[lane + 32 i], -inf past E_r.
+template <int PER>
+__device__ __forceinline__ void select_token(const RouterArgs& a, int64_t t, int lane, float (&v)[PER]) {
+    const int E = a.E, k = a.k;
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !isfinite(v[i])) bad = true;
+    }
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) m = fmaxf(m, v[i]);
+    m = warp_max(m);
+    unsigned taken = 0;
+    int my_e = -1;
+    float my_g = 0.f, next_g = -INFINITY;
+    const int rounds = k < E ? k + 1 : k;
+    if (!__any_sync(0xffffffffu, bad)) {
+        for (int r = 0; r < rounds; ++r) {
+            float bv = -INFINITY;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int e = lane + 32 * i;
+                if (!((taken >> i) & 1u) && e < E && (v[i] > bv || (v[i] == bv && e < be))) {
+                    bv = v[i];
+                    be = e;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                if (ov > bv || (ov == bv && oe < be)) {
+                    bv = ov;
+                    be = oe;
+                }
+            }
+            if (r < k) {
+                if (lane == r) {
+                    my_e = be;
+                    my_g = bv;
+                }
+                if ((be & 31) == lane) taken |= 1u << (be >> 5);
+            } else {
+                next_g = bv;
+            }
+        }
+    }
+    float z = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) z += expf(v[i] - m);
+    }
+    z = warp_sum(z);
+    const bool pick = lane < k;
+    const float ex = pick && !bad ? expf(my_g - m) : 0.f;
+    float wv = 0.f;
+    bool active = pick;
+    bool lat_bad = false;
+    float te = 1.f;
+    if (a.norm == MOE_NORM_WLR && pick && !bad) {
+        te = a.lat[t * E + my_e];
+        lat_bad = !(te > 0.f);  // NaN or non-positive latency
+    }
+    bad = __any_sync(0xffffffffu, bad || lat_bad);
+    if (bad) {
+        if (pick) {
+            a.ids[t * k + lane] = -1;
+            a.w[t * k + lane] = 0.f;
+        }
+        if (lane == 0) {
+            if (a.margin) a.margin[t] = NAN;
+            atomicAdd(a.counters + CNT_NONFINITE, 1ull);
+        }
+        return;
+    }
+    if (a.norm == MOE_NORM_FULLPROB) {
+        wv = ex / z;
+    } else if (a.norm == MOE_NORM_RENORM) {
+        wv = ex / warp_sum(ex);
+    } else {
+        const float wlr = (ex / z) / te;  // p_e / t_e (0 when t_e = inf)
+        for (;;) {
+            const unsigned am = __ballot_sync(0xffffffffu, active);
+            if (__popc(am) < 2) break;
+            // smallest WLR (on equal WLR the higher expert index) and largest WLR
+            float mn = active ? wlr : INFINITY;
+            int mne = active ? my_e : -1;
+            float mx = active ? wlr : -INFINITY;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, mn, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, mne, o);
+                if (ov < mn || (ov == mn && oe > mne)) {
+                    mn = ov;
+                    mne = oe;
+                }
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            const float ratio = mn / (mn + mx);
+            if (ratio <= a.theta) {
+                if (active && my_e == mne) active = false;
+            } else {
+                break;
+            }
+        }
+        const float s = warp_sum(active ? ex : 0.f);
+        wv = active ? ex / s : 0.f;
+        if (active && isinf(te)) wv = 0.f;  // disconnected expert: weight 0
+    }
+    if (pick) {
+        a.ids[t * k + lane] = active ? my_e : -1;
+        a.w[t * k + lane] = wv;
+    }
+    const float kth = __shfl_sync(0xffffffffu, my_g, k - 1);
+    const float mg = k < E ? kth - next_g : INFINITY;
+    if (lane == 0) {
+        if (a.margin) a.margin[t] = mg;
+        if (mg < kNearTie) atomicAdd(a.counters + CNT_NEAR_TIE, 1ull);
+    }
+}
+
 template <int TT, int TE, typename Tin>
 __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
     constexpr int EG = 8 * TT;       // expert groups across the CTA
@@ -159,134 +286,18 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
     __syncthreads();
 
     const int warp = tid >> 5, lane = tid & 31;
-    const int E = a.E, k = a.k;
     for (int q = 0; q < kTok / 8; ++q) {
         const int tt = warp * (kTok / 8) + q;
         const int64_t t = t0 + tt;
         if (t >= a.N) break;
         const float* g = lg + tt * LD;
         float v[PER];
-        bool bad = false;
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
             const int e = lane + 32 * i;
-            v[i] = e < E ? g[e] : -INFINITY;
-            if (e < E && !isfinite(v[i])) bad = true;
+            v[i] = e < a.E ? g[e] : -INFINITY;
         }
-        // selection in rank order: lane r keeps the r-th pick
-        float m = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < PER; ++i) m = fmaxf(m, v[i]);
-        m = warp_max(m);
-        unsigned taken = 0;
-        int my_e = -1;
-        float my_g = 0.f, next_g = -INFINITY;
-        const int rounds = k < E ? k + 1 : k;
-        if (!__any_sync(0xffffffffu, bad)) {
-            for (int r = 0; r < rounds; ++r) {
-                float bv = -INFINITY;
-                int be = 0x7fffffff;
-#pragma unroll
-                for (int i = 0; i < PER; ++i) {
-                    const int e = lane + 32 * i;
-                    if (!((taken >> i) & 1u) && e < E && (v[i] > bv || (v[i] == bv && e < be))) {
-                        bv = v[i];
-                        be = e;
-                    }
-                }
-#pragma unroll
-                for (int o = 16; o; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                    if (ov > bv || (ov == bv && oe < be)) {
-                        bv = ov;
-                        be = oe;
-                    }
-                }
-                if (r < k) {
-                    if (lane == r) {
-                        my_e = be;
-                        my_g = bv;
-                    }
-                    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-                } else {
-                    next_g = bv;
-                }
-            }
-        }
-        float z = 0.f;
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E) z += expf(v[i] - m);
-        }
-        z = warp_sum(z);
-        const bool pick = lane < k;
-        const float ex = pick && !bad ? expf(my_g - m) : 0.f;
-        float wv = 0.f;
-        bool active = pick;
-        bool lat_bad = false;
-        float te = 1.f;
-        if (a.norm == MOE_NORM_WLR && pick && !bad) {
-            te = a.lat[t * E + my_e];
-            lat_bad = !(te > 0.f);  // NaN or non-positive latency
-        }
-        bad = __any_sync(0xffffffffu, bad || lat_bad);
-        if (bad) {
-            if (pick) {
-                a.ids[t * k + lane] = -1;
-                a.w[t * k + lane] = 0.f;
-            }
-            if (lane == 0) {
-                if (a.margin) a.margin[t] = NAN;
-                atomicAdd(a.counters + CNT_NONFINITE, 1ull);
-            }
-            continue;
-        }
-        if (a.norm == MOE_NORM_FULLPROB) {
-            wv = ex / z;
-        } else if (a.norm == MOE_NORM_RENORM) {
-            wv = ex / warp_sum(ex);
-        } else {
-            const float wlr = (ex / z) / te;  // p_e / t_e (0 when t_e = inf)
-            for (;;) {
-                const unsigned am = __ballot_sync(0xffffffffu, active);
-                if (__popc(am) < 2) break;
-                // smallest WLR (on equal WLR the higher expert index) and largest WLR
-                float mn = active ? wlr : INFINITY;
-                int mne = active ? my_e : -1;
-                float mx = active ? wlr : -INFINITY;
-#pragma unroll
-                for (int o = 16; o; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, mn, o);
-                    const int oe = __shfl_xor_sync(0xffffffffu, mne, o);
-                    if (ov < mn || (ov == mn && oe > mne)) {
-                        mn = ov;
-                        mne = oe;
-                    }
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                }
-                const float ratio = mn / (mn + mx);
-                if (ratio <= a.theta) {
-                    if (active && my_e == mne) active = false;
-                } else {
-                    break;
-                }
-            }
-            const float s = warp_sum(active ? ex : 0.f);
-            wv = active ? ex / s : 0.f;
-            if (active && isinf(te)) wv = 0.f;  // disconnected expert: weight 0
-        }
-        if (pick) {
-            a.ids[t * k + lane] = active ? my_e : -1;
-            a.w[t * k + lane] = wv;
-        }
-        const float kth = __shfl_sync(0xffffffffu, my_g, k - 1);
-        const float mg = k < E ? kth - next_g : INFINITY;
-        if (lane == 0) {
-            if (a.margin) a.margin[t] = mg;
-            if (mg < kNearTie) atomicAdd(a.counters + CNT_NEAR_TIE, 1ull);
-        }
+        select_token<PER>(a, t, lane, v);
     }
 
     if (a.Y_zero) {
@@ -295,6 +306,104 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
         const int64_t n4 = (t_end - t0) * a.d / 4;
         for (int64_t i = tid; i < n4; i += kThreads) Y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+}
+
+// Read-only (L1-cached) loads of 8 weights; streaming loads of 8 activations.
+__device__ __forceinline__ void ldg8(const float* p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void ldg8(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void ldcs8(const float* p, float (&v)[8]) {
+    const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldcs(reinterpret_cast<const float4*>(p + 4));
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void ldcs8(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
+__device__ __forceinline__ void zero_row(float* Y, int64_t t, int d, int lane) {
+    float4* y4 = reinterpret_cast<float4*>(Y + t * d);
+    for (int i = lane; i < d / 4; i += 32) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// Narrow routers (E_r <= EMAX <= 32), one warp per token: the lanes stream the
+// token's row of x in 16-byte vectors (each lane a strided slice of d), keep
+// E_r partial scores, and a butterfly reduction gives every lane all scores.
+// W_r (E_r x d) is read through L1.  Bound by reading x once.
+template <int EMAX, typename Tin>
+__global__ void __launch_bounds__(256) router_narrow_kernel(RouterArgs a) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+    if (t >= a.N) return;
+    const Tin* X = static_cast<const Tin*>(a.x) + t * a.d;
+    const Tin* W = static_cast<const Tin*>(a.W_r);
+    float acc[EMAX];
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
+    for (int i = lane * 8; i < a.d; i += 256) {
+        float xv[8];
+        ldcs8(X + i, xv);
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) {
+            if (e < a.E) {
+                float wv[8];
+                ldg8(W + (int64_t)e * a.d + i, wv);
+                float part = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) part = fmaf(xv[j], wv[j], part);
+                acc[e] += part;
+            }
+        }
+    }
+    float v[1] = {-INFINITY};
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+        float s = acc[e];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == e && e < a.E) v[0] = s + (a.b_r ? a.b_r[e] : 0.f);
+    }
+    select_token<1>(a, t, lane, v);
+    if (a.Y_zero) zero_row(a.Y_zero, t, a.d, lane);
+}
+
+// Selection from precomputed scores [N, E_r] (tensor-core score path), one
+// warp per token.
+template <int PER>
+__global__ void __launch_bounds__(256) logits_topk_kernel(RouterArgs a, const float* __restrict__ logits) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+    if (t >= a.N) return;
+    const float* g = logits + t * a.E;
+    float v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < a.E ? g[e] + (a.b_r ? a.b_r[e] : 0.f) : -INFINITY;
+    }
+    select_token<PER>(a, t, lane, v);
+    if (a.Y_zero) zero_row(a.Y_zero, t, a.d, lane);
 }
 
 template <int TT, int TE, typename Tin>
@@ -323,7 +432,8 @@ cudaError_t launch_typed(const RouterArgs& a, cudaStream_t st) {
 
 cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, const float* b_r,
                           const float* lat, int32_t* ids, float* w, float* margin,
-                          unsigned long long* counters, float* Y_zero, cudaStream_t st) {
+                          unsigned long long* counters, float* Y_zero, float* logits,
+                          cudaStream_t st) {
     RouterArgs a;
     a.x = x;
     a.W_r = W_r;
@@ -341,7 +451,32 @@ cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, c
     a.norm = p.norm;
     a.theta = p.theta;
     if (p.N == 0) return cudaSuccess;
-    if (p.dtype == MOE_BF16) return launch_typed<__nv_bfloat16>(a, st);
+    const unsigned warps_blocks = (unsigned)((p.N + 7) / 8);
+    const bool bf16 = p.dtype == MOE_BF16;
+    if (p.E_r <= 32) {
+        if (p.E_r <= 8) {
+            if (bf16) router_narrow_kernel<8, __nv_bfloat16><<<warps_blocks, 256, 0, st>>>(a);
+            else router_narrow_kernel<8, float><<<warps_blocks, 256, 0, st>>>(a);
+        } else if (p.E_r <= 16) {
+            if (bf16) router_narrow_kernel<16, __nv_bfloat16><<<warps_blocks, 256, 0, st>>>(a);
+            else router_narrow_kernel<16, float><<<warps_blocks, 256, 0, st>>>(a);
+        } else {
+            if (bf16) router_narrow_kernel<32, __nv_bfloat16><<<warps_blocks, 256, 0, st>>>(a);
+            else router_narrow_kernel<32, float><<<warps_blocks, 256, 0, st>>>(a);
+        }
+        return cudaGetLastError();
+    }
+    if (bf16 && logits && p.E_r % 4 == 0) {
+        // wide routers: scores on the tensor cores, then one warp per token selects
+        int status = 0;
+        cudaError_t e = launch_tc_logits(p, x, W_r, logits, counters, st, &status);
+        if (e != cudaSuccess) return e;
+        if (p.E_r <= 64) logits_topk_kernel<2><<<warps_blocks, 256, 0, st>>>(a, logits);
+        else if (p.E_r <= 128) logits_topk_kernel<4><<<warps_blocks, 256, 0, st>>>(a, logits);
+        else logits_topk_kernel<8><<<warps_blocks, 256, 0, st>>>(a, logits);
+        return cudaGetLastError();
+    }
+    if (bf16) return launch_typed<__nv_bfloat16>(a, st);
     return launch_typed<float>(a, st);
 }
 

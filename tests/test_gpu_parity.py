@@ -43,6 +43,14 @@ SMALL = {
     "all_experts_f32": W["switch_top1_f32"].scaled("all_experts_f32", N=130, d=64, d_f=64, E=4, k=4,
                                                    norm=si.NORM_RENORM, c=0.0),
     "one_expert_bf16": W["mixtral_bf16"].scaled("one_expert_bf16", N=200, d=64, d_f=136, E=1, k=1),
+    # long K in the down projection: the combine runs with K split across SMs
+    "splitk_down_bf16": W["mixtral_bf16"].scaled("splitk_down_bf16", N=256, d=128, d_f=2048, E=4, k=1),
+    # 64 experts on d = 1024: router scores on the tensor cores with K split
+    "wide_router_bf16": W["mixtral_bf16"].scaled("wide_router_bf16", N=256, d=1024, d_f=128, E=64, k=4),
+    # fp32 with 48 experts and bf16 with 34 experts: the FFMA score kernel
+    "wide_router_f32": W["switch_top1_f32"].scaled("wide_router_f32", N=200, d=64, d_f=64, E=48, k=3,
+                                                   norm=si.NORM_RENORM, c=0.0),
+    "odd_experts_bf16": W["mixtral_bf16"].scaled("odd_experts_bf16", N=200, d=64, d_f=64, E=34, k=3),
 }
 
 
