@@ -75,6 +75,8 @@ struct TcArgs {
     int max_rows;             // rows of the routed A / output buffers (N k)
     int n_tokens;             // N
     int has_routed;           // 0: only the second (dense) segment runs
+    float* zero_ptr;          // optional fp32 buffer the epilogue warps zero first
+    int64_t zero_n4;          // its size in float4
     int ks;                   // K splits per output tile (partial sums reduced with red.add)
     unsigned long long* counters;
 };
@@ -168,6 +170,29 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
+}
+
+// Same with an L2 eviction-priority policy (createpolicy): activations that
+// many tiles re-read are kept (evict_last), weights streamed once go first.
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int c0, int c1, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
@@ -385,6 +410,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t phase = 0;
             int issued_parity[STAGES];
             for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+            const uint64_t pol_act = policy_evict_last();
+            const uint64_t pol_wgt = policy_evict_first();
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 Tile ti;
@@ -408,9 +435,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     uint8_t* sa = stage_base + stage * STAGE_BYTES;
                     uint8_t* sb = sa + A_BYTES;
                     mbar_expect_tx(&full[stage], STAGE_BYTES);
-                    tma_load_2d(sa, pa, &full[stage], kb * BK, ti.a_row);
-                    tma_load_2d(sb, pb0, &full[stage], kb * BK, b_row0);
-                    tma_load_2d(sb + B_HALF_BYTES, pb1, &full[stage], kb * BK, b_row1);
+                    tma_load_2d_hint(sa, pa, &full[stage], kb * BK, ti.a_row, pol_act);
+                    tma_load_2d_hint(sb, pb0, &full[stage], kb * BK, b_row0, pol_wgt);
+                    tma_load_2d_hint(sb + B_HALF_BYTES, pb1, &full[stage], kb * BK, b_row1, pol_wgt);
                     issued_parity[stage] = (int)phase;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -474,6 +501,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else {
         // epilogue warps 2..5: TMEM lane quarter = warp % 4
+        if (a.zero_ptr) {
+            // zero this CTA's share of the combine output while the first
+            // accumulator is being computed (the down projection adds into it)
+            const int64_t per = (a.zero_n4 + gridDim.x - 1) / gridDim.x;
+            const int64_t lo = per * blockIdx.x;
+            const int64_t hi = min64(a.zero_n4, lo + per);
+            float4* z = reinterpret_cast<float4*>(a.zero_ptr);
+            for (int64_t i = lo + (threadIdx.x - 64); i < hi; i += 128) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         int acc = 0;
@@ -634,10 +670,14 @@ double routed_mtile_estimate(const moe_params& p, int64_t C) {
     return p.E_r * (per < 1.0 ? 1.0 : per);
 }
 
-// K splits for an output-tile count: minimise the number of full waves of
-// tile-time (ceil(tiles * ks / SMs) / ks), keeping >= 8 K blocks per slice.
+// K splits for an output-tile count: only when the tiles fill less than one
+// wave of SMs (splitting a multi-wave launch measured slower on the
+// Mixtral-shaped down projection: the extra red.add traffic costs more than
+// the last partial wave), minimise ceil(tiles * ks / SMs) / ks, keeping >= 8 K
+// blocks per slice.
 int choose_ksplit(double tiles, int nkb_min) {
     const int sms = num_sms();
+    if (tiles >= sms) return 1;
     int best = 1;
     double best_cost = 1e30;
     for (int ks = 1; ks <= 8; ++ks) {
@@ -656,7 +696,7 @@ int choose_ksplit(double tiles, int nkb_min) {
 
 cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
                               const int32_t* offsets, const int32_t* mt_start,
-                              const ExpertWeights& W, void* h, void* h_shared,
+                              const ExpertWeights& W, void* h, void* h_shared, float* Y_zero,
                               unsigned long long* counters, cudaStream_t st, int* status) {
     *status = MOE_OK;
     CUtensorMap mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh;
@@ -698,8 +738,11 @@ cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const voi
     a.n_tokens = (int)p.N;
     a.has_routed = 1;
     a.ks = 1;  // the SwiGLU epilogue needs the whole K sum
+    a.zero_ptr = Y_zero;
+    a.zero_n4 = Y_zero ? p.N * (int64_t)p.d / 4 : 0;
     a.counters = counters;
     int64_t max_tiles = routed_mtile_bound(p) * a.nt_r + (sh ? ((p.N + BM - 1) / BM) * a.nt_sh : 0);
+    if (Y_zero && max_tiles < num_sms()) max_tiles = num_sms();  // every CTA zeroes a share
     return launch_tc<EPI_SWIGLU>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a, max_tiles, st);
 }
 

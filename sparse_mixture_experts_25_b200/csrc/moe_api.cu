@@ -302,7 +302,7 @@ moe_status moe_expert_ffn(const moe_params* p, const void* x_perm, const int32_t
     cudaError_t e;
     if (p->dtype == MOE_BF16) {
         e = launch_tc_gate_up(q, x_perm, nullptr, offsets, v.scratch.mt_start, W, v.h, nullptr,
-                              v.counters, st, &status);
+                              nullptr, v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_expert_ffn gate/up: tensor map encode" : "moe_expert_ffn gate/up (tcgen05)");
         e = launch_tc_down(q, DOWN_STORE, p->N, v.h, nullptr, offsets, v.scratch.mt_start, W, nullptr,
                            nullptr, nullptr, H, v.counters, st, &status);
@@ -357,8 +357,11 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     ExpertWeights W{W_g, W_u, W_d, sh ? Ws_g : nullptr, sh ? Ws_u : nullptr, sh ? Ws_d : nullptr};
 
     if ((e0 = stage_mark(0, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
+    // bf16 layers zero Y inside the gate/up kernel (hidden behind its first
+    // tile); fp32 layers zero it in the router
+    const bool bf16 = p->dtype == MOE_BF16;
     cudaError_t e = launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, v.ids,
-                                  v.w, v.margin, v.counters, Y, v.scratch.logits, st);
+                                  v.w, v.margin, v.counters, bf16 ? nullptr : Y, v.scratch.logits, st);
     if (e != cudaSuccess) return fail(e, "moe_forward router");
     if ((e0 = stage_mark(1, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
@@ -374,7 +377,7 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     int status = MOE_OK;
     if (p->dtype == MOE_BF16) {
         e = launch_tc_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared,
-                              v.counters, st, &status);
+                              Y, v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_forward gate/up: tensor map encode" : "moe_forward gate/up (tcgen05)");
         if ((e0 = stage_mark(3, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
         e = launch_tc_down(*p, DOWN_COMBINE, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,

@@ -105,9 +105,10 @@ struct ExpertWeights {
     const void* Ws_d;
 };
 enum DownMode { DOWN_COMBINE = 0, DOWN_STORE = 1 };
+// Y_zero (nullable): fp32 [N, d] that the kernel zeroes before the down projection adds into it
 cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
                               const int32_t* offsets, const int32_t* mt_start,
-                              const ExpertWeights& W, void* h, void* h_shared,
+                              const ExpertWeights& W, void* h, void* h_shared, float* Y_zero,
                               unsigned long long* counters, cudaStream_t st, int* status);
 cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void* h,
                            const void* h_shared, const int32_t* offsets, const int32_t* mt_start,

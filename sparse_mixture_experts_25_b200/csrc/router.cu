@@ -347,10 +347,47 @@ __device__ __forceinline__ void zero_row(float* Y, int64_t t, int d, int lane) {
     for (int i = lane; i < d / 4; i += 32) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
+// Eight consecutive inputs kept in their storage format until used (bf16
+// stays packed in one 16-byte register quad, halving register pressure).
+template <typename Tin>
+struct Vec8;
+template <>
+struct Vec8<__nv_bfloat16> {
+    uint4 u;
+    __device__ __forceinline__ void ldg(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+    __device__ __forceinline__ void ldcs(const __nv_bfloat16* p) { u = __ldcs(reinterpret_cast<const uint4*>(p)); }
+    __device__ __forceinline__ void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ float get(int j) const {
+        const uint32_t w = j < 2 ? u.x : j < 4 ? u.y : j < 6 ? u.z : u.w;
+        return (j & 1) ? __uint_as_float(w & 0xffff0000u) : __uint_as_float(w << 16);
+    }
+};
+template <>
+struct Vec8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void ldg(const float* p) {
+        a = __ldg(reinterpret_cast<const float4*>(p));
+        b = __ldg(reinterpret_cast<const float4*>(p + 4));
+    }
+    __device__ __forceinline__ void ldcs(const float* p) {
+        a = __ldcs(reinterpret_cast<const float4*>(p));
+        b = __ldcs(reinterpret_cast<const float4*>(p + 4));
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ float get(int j) const {
+        const float4& q = j < 4 ? a : b;
+        const int i = j & 3;
+        return i == 0 ? q.x : i == 1 ? q.y : i == 2 ? q.z : q.w;
+    }
+};
+
 // Narrow routers (E_r <= EMAX <= 32), one warp per token: the lanes stream the
 // token's row of x in 16-byte vectors (each lane a strided slice of d), keep
 // E_r partial scores, and a butterfly reduction gives every lane all scores.
-// W_r (E_r x d) is read through L1.  Bound by reading x once.
+// W_r (E_r x d) is read through L1.  All loads of one step (x and eight
+// experts' weights, two steps per iteration) are issued before their FMAs so
+// that the warp waits for memory once per iteration rather than once per
+// expert.  Bound by reading x once.
 template <int EMAX, typename Tin>
 __global__ void __launch_bounds__(256) router_narrow_kernel(RouterArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -358,21 +395,36 @@ __global__ void __launch_bounds__(256) router_narrow_kernel(RouterArgs a) {
     if (t >= a.N) return;
     const Tin* X = static_cast<const Tin*>(a.x) + t * a.d;
     const Tin* W = static_cast<const Tin*>(a.W_r);
+    const int E = a.E;
     float acc[EMAX];
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
-    for (int i = lane * 8; i < a.d; i += 256) {
-        float xv[8];
-        ldcs8(X + i, xv);
+    for (int i0 = lane * 8; i0 < a.d; i0 += 512) {
+        const int i1 = i0 + 256;
+        const bool has1 = i1 < a.d;
+        Vec8<Tin> x0, x1;
+        x0.ldcs(X + i0);
+        if (has1) x1.ldcs(X + i1);
+        else x1.zero();
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-            if (e < a.E) {
-                float wv[8];
-                ldg8(W + (int64_t)e * a.d + i, wv);
+        for (int g = 0; g < EMAX; g += 8) {
+            Vec8<Tin> w0[8], w1[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int ee = min(g + e, E - 1);  // clamped: loads are unconditional
+                const Tin* row = W + (int64_t)ee * a.d;
+                w0[e].ldg(row + i0);
+                if (has1) w1[e].ldg(row + i1);
+                else w1[e].zero();
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
                 float part = 0.f;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) part = fmaf(xv[j], wv[j], part);
-                acc[e] += part;
+                for (int j = 0; j < 8; ++j) part = fmaf(x0.get(j), w0[e].get(j), part);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) part = fmaf(x1.get(j), w1[e].get(j), part);
+                acc[g + e] += part;
             }
         }
     }
@@ -382,7 +434,7 @@ __global__ void __launch_bounds__(256) router_narrow_kernel(RouterArgs a) {
         float s = acc[e];
 #pragma unroll
         for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == e && e < a.E) v[0] = s + (a.b_r ? a.b_r[e] : 0.f);
+        if (lane == e && e < E) v[0] = s + (a.b_r ? a.b_r[e] : 0.f);
     }
     select_token<1>(a, t, lane, v);
     if (a.Y_zero) zero_row(a.Y_zero, t, a.d, lane);
@@ -453,7 +505,7 @@ cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, c
     if (p.N == 0) return cudaSuccess;
     const unsigned warps_blocks = (unsigned)((p.N + 7) / 8);
     const bool bf16 = p.dtype == MOE_BF16;
-    if (p.E_r <= 32) {
+    if (p.E_r <= 32 && !(bf16 && logits && p.E_r % 4 == 0)) {
         if (p.E_r <= 8) {
             if (bf16) router_narrow_kernel<8, __nv_bfloat16><<<warps_blocks, 256, 0, st>>>(a);
             else router_narrow_kernel<8, float><<<warps_blocks, 256, 0, st>>>(a);
@@ -467,11 +519,13 @@ cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, c
         return cudaGetLastError();
     }
     if (bf16 && logits && p.E_r % 4 == 0) {
-        // wide routers: scores on the tensor cores, then one warp per token selects
+        // bf16 routers: scores on the tensor cores (K split over SMs for small
+        // batches), then one warp per token selects
         int status = 0;
         cudaError_t e = launch_tc_logits(p, x, W_r, logits, counters, st, &status);
         if (e != cudaSuccess) return e;
-        if (p.E_r <= 64) logits_topk_kernel<2><<<warps_blocks, 256, 0, st>>>(a, logits);
+        if (p.E_r <= 32) logits_topk_kernel<1><<<warps_blocks, 256, 0, st>>>(a, logits);
+        else if (p.E_r <= 64) logits_topk_kernel<2><<<warps_blocks, 256, 0, st>>>(a, logits);
         else if (p.E_r <= 128) logits_topk_kernel<4><<<warps_blocks, 256, 0, st>>>(a, logits);
         else logits_topk_kernel<8><<<warps_blocks, 256, 0, st>>>(a, logits);
         return cudaGetLastError();
