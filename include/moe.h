@@ -246,6 +246,40 @@ MOE_API moe_status moe_forward(const moe_params* p, const void* x, const void* W
                        moe_stream_t stream);
 
 /*
+ * A routing group split over ranks (data parallel: each GPU holds a shard of
+ * the group's tokens, ranks in token order, weights replicated).  Capacity
+ * competition is defined over the whole routing group ("LLM from scratch"
+ * ch. 36.3-36.4 and Algorithm 36.1; auturnal review: C from the group's token
+ * count), so the shards exchange one small table: each rank's per-expert
+ * request counts.  Two calls around that exchange give exactly the routing,
+ * slots and outputs of one GPU running the concatenated batch:
+ *
+ * moe_forward_begin: route this rank's N = params.N tokens (as moe_route) and
+ * count its requests per expert: counts [E_r] int32 (device, nullable; also
+ * kept in the workspace).  The caller then all-gathers the counts of every
+ * rank into counts_all [n_ranks][E_r] (for example with NCCL on the same
+ * stream).
+ *
+ * moe_forward_end: with counts_all, this rank's requests for expert e are the
+ * requests base_e .. base_e + L_e - 1 of the whole group (base_e = sum of the
+ * counts of earlier ranks); the first C of the group are accepted.  Then it
+ * dispatches, runs the experts and the combine as moe_forward does (same
+ * x, weights, workspace; Y [N, d] overwritten).  C is the group's capacity
+ * (moe_capacity with N = N_group, the group's token count).  slot records
+ * hold group-wide slots.  moe_get_stats then reports this rank's request
+ * counts (requested, accepted, rejected, tokens_affected, tokens_skipped) and
+ * the group's loads (O, L_max, percentiles, rho_max over N_group).
+ */
+MOE_API moe_status moe_forward_begin(const moe_params* p, const void* x, const void* W_r,
+                                     const float* b_r, const float* lat, int32_t* counts,
+                                     void* ws, moe_stream_t stream);
+MOE_API moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32_t rank,
+                                   int32_t n_ranks, int64_t N_group, int64_t C, const void* x,
+                                   const void* W_g, const void* W_u, const void* W_d,
+                                   const void* Ws_g, const void* Ws_u, const void* Ws_d, float* Y,
+                                   void* ws, moe_stream_t stream);
+
+/*
  * Reads the routing statistics of the last dispatch on this workspace into
  * *out (host memory); waits for `stream`.  Returns MOE_ERR_NONFINITE when a
  * token had non-finite scores, MOE_ERR_TIMEOUT when a device wait gave up,

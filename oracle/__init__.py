@@ -61,6 +61,7 @@ def _load():
         i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
         lib.oracle_route.argtypes = [i64, i32, i32, i32, i32, dbl, i32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         lib.oracle_dispatch.argtypes = [i64, i32, i32, i64, _P, _P, _P, _P, _P]
+        lib.oracle_dispatch_ranked.argtypes = [i64, i32, i32, i64, _P, _P, _P, _P, _P, _P]
         lib.oracle_swiglu_rows.argtypes = [i32, i32, i32, i32, _P, _P, i64, _P, _P, _P, _P]
         lib.oracle_combine.argtypes = [i64, i32, i32, _P, _P, _P, _P, _P]
         lib.oracle_forward_rows.argtypes = [i32, i32, i32, i32, i32, i32, _P, _P, _P, _P, _P, i64,
@@ -70,7 +71,7 @@ def _load():
                                        _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         lib.oracle_round_bf16.argtypes = [dbl]
         lib.oracle_round_bf16.restype = dbl
-        for f in ("oracle_route", "oracle_dispatch", "oracle_swiglu_rows", "oracle_combine",
+        for f in ("oracle_route", "oracle_dispatch", "oracle_dispatch_ranked", "oracle_swiglu_rows", "oracle_combine",
                   "oracle_forward_rows", "oracle_forward"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
@@ -184,6 +185,26 @@ def dispatch(ids, E: int, C: int):
     names = ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max")
     stats = {n: int(v) for n, v in zip(names, cnt)}
     return {"slot": slot, "L": L, "acc": acc, "stats": stats}
+
+
+def dispatch_ranked(ids, E: int, C: int, base):
+    """Acceptance for one rank's shard of a routing group split over ranks
+    in token order; base[e] = requests for e by earlier ranks (see oracle.c).
+    Returns slot (group-wide slot or -1), this shard's L and acc, and the
+    shard's counters."""
+    ids = _c(ids, np.int32)
+    N, k = ids.shape
+    b = _c(np.asarray(base), np.int64)
+    slot = np.empty((N, k), np.int32)
+    L = np.empty(E, np.int64)
+    acc = np.empty(E, np.int64)
+    cnt = np.empty(7, np.int64)
+    rc = _load().oracle_dispatch_ranked(N, k, E, C, _ptr(ids), _ptr(b), _ptr(slot), _ptr(L), _ptr(acc),
+                                        _ptr(cnt))
+    if rc:
+        raise ValueError("oracle_dispatch_ranked: invalid arguments")
+    names = ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max")
+    return {"slot": slot, "L": L, "acc": acc, "stats": {n: int(v) for n, v in zip(names, cnt)}}
 
 
 def swiglu_rows(x, rows, Wg, Wu, Wd, round_h=None):

@@ -234,6 +234,42 @@ int oracle_dispatch(int64_t N, int k, int E, int64_t C, const int32_t* ids, int3
 }
 
 /*
+ * Token-order acceptance for one shard of a routing group split over ranks in
+ * token order (rank 0's tokens first).  base[e] = requests for expert e made
+ * by the tokens of earlier ranks.  A request is the base[e] + j-th request for
+ * e in the whole group (j = earlier requests for e in this shard) and is
+ * accepted iff that number is < C, exactly as Algorithm 36.1 decides on the
+ * concatenated batch.  slot[] receives that group-wide slot (or -1); L and
+ * acc are this shard's requested and accepted counts; cnt as oracle_dispatch
+ * but for this shard's requests, except cnt[3] (O) and cnt[6] (max load),
+ * which are left 0 (they need the group-wide loads).
+ */
+int oracle_dispatch_ranked(int64_t N, int k, int E, int64_t C, const int32_t* ids,
+                           const int64_t* base, int32_t* slot, int64_t* L, int64_t* acc,
+                           int64_t* cnt) {
+    if (N < 0 || k < 1 || E < 1 || C < 1) return 1;
+    for (int e = 0; e < E; ++e) { L[e] = 0; acc[e] = 0; }
+    for (int i = 0; i < 7; ++i) cnt[i] = 0;
+    for (int64_t t = 0; t < N; ++t) {
+        int req = 0, rej = 0;
+        for (int j = 0; j < k; ++j) {
+            int e = ids[t * k + j];
+            if (e < 0) { slot[t * k + j] = -1; continue; }
+            ++req;
+            int64_t c = base[e] + L[e];
+            L[e] += 1;
+            if (c < C) { slot[t * k + j] = (int32_t)c; acc[e] += 1; }
+            else { slot[t * k + j] = -1; ++rej; }
+        }
+        if (rej > 0) cnt[4] += 1;
+        if (req > 0 && rej == req) cnt[5] += 1;
+    }
+    for (int e = 0; e < E; ++e) { cnt[0] += L[e]; cnt[1] += acc[e]; }
+    cnt[2] = cnt[0] - cnt[1];
+    return 0;
+}
+
+/*
  * One SwiGLU expert on a list of token rows (vegetog sec. 3):
  *   E(x) = [SiLU(x W_gate) (.) (x W_up)] W_down
  * with W_gate, W_up stored [d_f, d] and W_down stored [d, d_f].  When

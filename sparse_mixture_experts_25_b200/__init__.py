@@ -19,7 +19,8 @@ __all__ = [
     "MoEError", "Params", "Stats", "WsLayout", "lib", "params", "moe_capacity",
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_dispatch",
     "moe_dispatch_noalloc",
-    "moe_expert_ffn", "moe_combine", "moe_forward", "moe_get_stats",
+    "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_begin", "moe_forward_end",
+    "moe_get_stats",
     "moe_set_stage_events", "moe_status_string", "moe_last_error", "workspace_views", "HEADER",
 ]
 
@@ -87,6 +88,9 @@ def lib():
         L.moe_combine.argtypes = [pp, _P, _P, _P, _P, _P, _P]
         L.moe_forward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_get_stats.argtypes = [pp, _P, ctypes.POINTER(Stats), _P]
+        L.moe_forward_begin.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_forward_end.argtypes = [pp, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
+                                      ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(_P), ctypes.c_int]
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
@@ -95,7 +99,8 @@ def lib():
         for name in ("moe_capacity", "moe_workspace_size", "moe_workspace_layout", "moe_route",
                      "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine",
                      "moe_forward",
-                     "moe_get_stats", "moe_set_stage_events"):
+                     "moe_get_stats", "moe_set_stage_events", "moe_forward_begin",
+                     "moe_forward_end"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -199,6 +204,19 @@ def moe_forward(p, x, W_r, b_r, lat, W_g, W_u, W_d, Ws_g, Ws_u, Ws_d, Y, ws, str
     _check(lib().moe_forward(ctypes.byref(p), _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(lat), _ptr(W_g),
                              _ptr(W_u), _ptr(W_d), _ptr(Ws_g), _ptr(Ws_u), _ptr(Ws_d), _ptr(Y),
                              _ptr(ws), _stream(stream)), "moe_forward")
+
+
+def moe_forward_begin(p, x, W_r, b_r, lat, counts, ws, stream=None):
+    _check(lib().moe_forward_begin(ctypes.byref(p), _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(lat),
+                                   _ptr(counts), _ptr(ws), _stream(stream)), "moe_forward_begin")
+
+
+def moe_forward_end(p, counts_all, rank, n_ranks, N_group, C, x, W_g, W_u, W_d, Ws_g, Ws_u, Ws_d, Y, ws,
+                    stream=None):
+    _check(lib().moe_forward_end(ctypes.byref(p), _ptr(counts_all), int(rank), int(n_ranks),
+                                 int(N_group), int(C), _ptr(x), _ptr(W_g), _ptr(W_u), _ptr(W_d),
+                                 _ptr(Ws_g), _ptr(Ws_u), _ptr(Ws_d), _ptr(Y), _ptr(ws),
+                                 _stream(stream)), "moe_forward_end")
 
 
 def moe_get_stats(p, ws, stream=None):

@@ -72,12 +72,9 @@ __global__ void hist_kernel(const int32_t* __restrict__ ids, int64_t N, int k, i
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)e * n_tiles + blockIdx.x] = h[e];
 }
 
-__global__ void scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int64_t C, int bm,
-                            int32_t* __restrict__ L, int32_t* __restrict__ acc,
-                            int32_t* __restrict__ offsets, int32_t* __restrict__ mt_start,
-                            unsigned long long* counters) {
-    __shared__ int sL[kMaxExperts];
-    __shared__ int warp_tot[33];
+// Per expert (one warp each), the per-tile request counts become exclusive
+// bases in place; sL[e] receives the expert's total.
+__device__ void tile_scan(int32_t* __restrict__ hist, int n_tiles, int E, int* sL) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     for (int e = warp; e < E; e += nw) {
         int run = 0;
@@ -91,6 +88,15 @@ __global__ void scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int6
         }
         if (lane == 0) sL[e] = run;
     }
+}
+
+__global__ void scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int64_t C, int bm,
+                            int32_t* __restrict__ L, int32_t* __restrict__ acc,
+                            int32_t* __restrict__ offsets, int32_t* __restrict__ mt_start,
+                            unsigned long long* counters) {
+    __shared__ int sL[kMaxExperts];
+    __shared__ int warp_tot[33];
+    tile_scan(hist, n_tiles, E, sL);
     __syncthreads();
     // one thread per expert (blockDim.x >= E)
     const int e = threadIdx.x;
@@ -120,9 +126,80 @@ __global__ void scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int6
     }
 }
 
+// Sharded routing group, first half: this rank's per-tile bases and its
+// per-expert request counts (written to L and, when given, counts_out for the
+// exchange between ranks).
+__global__ void count_scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E,
+                                  int32_t* __restrict__ L, int32_t* __restrict__ counts_out) {
+    __shared__ int sL[kMaxExperts];
+    tile_scan(hist, n_tiles, E, sL);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        L[e] = sL[e];
+        if (counts_out) counts_out[e] = sL[e];
+    }
+}
+
+// Sharded routing group, second half: from the gathered request counts of
+// every rank ([n_ranks][E], ranks in token order) this rank's requests for e
+// are requests base_e .. base_e + L_e - 1 of the whole group, base_e = sum of
+// the earlier ranks' counts; the first C of the group are accepted, so this
+// rank keeps acc_e = clamp(C - base_e, 0, L_e) of them.  Statistics: counts
+// of this rank's requests, plus O, the maximum load and (in L) the loads of
+// the whole group.
+__global__ void expert_scan_ranked_kernel(int E, int64_t C, int bm, const int32_t* __restrict__ table,
+                                          int rank, int n_ranks, int64_t n_group,
+                                          int32_t* __restrict__ L, int32_t* __restrict__ acc,
+                                          int32_t* __restrict__ offsets,
+                                          int32_t* __restrict__ mt_start,
+                                          int32_t* __restrict__ base_out,
+                                          unsigned long long* counters) {
+    __shared__ int warp_tot[33];
+    const int e = threadIdx.x;
+    int64_t base = 0, Lg = 0, Le = 0;
+    if (e < E) {
+        for (int r = 0; r < n_ranks; ++r) {
+            const int64_t v = table[(int64_t)r * E + e];
+            if (r < rank) base += v;
+            if (r == rank) Le = v;
+            Lg += v;
+        }
+    }
+    int64_t a64 = C - base;
+    a64 = a64 < 0 ? 0 : (a64 > Le ? Le : a64);
+    const int a = (int)a64;
+    const int mt = (a + bm - 1) / bm;
+    int tot_a, tot_mt, tot_L, tot_O;
+    const int ex_a = block_excl_scan(a, warp_tot, &tot_a);
+    const int ex_mt = block_excl_scan(mt, warp_tot, &tot_mt);
+    block_excl_scan((int)Le, warp_tot, &tot_L);
+    block_excl_scan(Lg > C ? (int)(Lg - C) : 0, warp_tot, &tot_O);
+    if (e < E) {
+        L[e] = (int32_t)Lg;
+        acc[e] = a;
+        offsets[e] = ex_a;
+        mt_start[e] = ex_mt;
+        base_out[e] = (int32_t)base;
+        atomicMax(counters + CNT_L_MAX, (unsigned long long)Lg);
+    }
+    if (threadIdx.x == 0) {
+        offsets[E] = tot_a;
+        mt_start[E] = tot_mt;
+        counters[CNT_REQUESTED] = (unsigned long long)tot_L;
+        counters[CNT_ACCEPTED] = (unsigned long long)tot_a;
+        counters[CNT_REJECTED] = (unsigned long long)(tot_L - tot_a);
+        counters[CNT_O] = (unsigned long long)tot_O;
+        counters[CNT_C] = (unsigned long long)C;
+        counters[CNT_N_GROUP] = (unsigned long long)n_group;
+    }
+}
+
+// rank_base (nullable): per-expert requests of earlier ranks of a sharded group;
+// a request's group-wide slot is base + its slot among this rank's requests.
 __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w,
                               int64_t N, int k, int E, int64_t C, int tile_tokens, int n_tiles,
                               const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets,
+                              const int32_t* __restrict__ rank_base,
                               int32_t* __restrict__ slot, int32_t* __restrict__ slot_token,
                               float* __restrict__ slot_w, unsigned long long* counters) {
     extern __shared__ int run[];
@@ -145,11 +222,12 @@ __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __re
         if (e >= 0 && lane == 31 - __clz(peers)) run[e] += __popc(peers);
         __syncwarp();
         if (valid) {
-            if (e >= 0 && s < C) {
+            const int64_t sg = e >= 0 ? (rank_base ? (int64_t)rank_base[e] + s : (int64_t)s) : -1;
+            if (e >= 0 && sg < C) {
                 const int64_t pos = (int64_t)offsets[e] + s;
                 slot_token[pos] = (int32_t)(i / k);
                 slot_w[pos] = w[i];
-                slot[i] = s;
+                slot[i] = (int32_t)sg;
             } else {
                 slot[i] = -1;
             }
@@ -252,8 +330,51 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     *where = "assign";
     assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
-                                                         n_tiles, sc.hist, offsets, slot,
+                                                         n_tiles, sc.hist, offsets, nullptr, slot,
                                                          slot_token, slot_w, counters);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (x && x_perm) {
+        *where = "gather";
+        const int row_vec = (int)(p.d * esize(p.dtype) / 16);
+        const int64_t rows = p.N * p.k;
+        const int blocks = (int)min64(rows, (int64_t)num_sms() * 8);
+        gather_kernel<<<blocks, 128, 0, st>>>(static_cast<const uint4*>(x),
+                                              static_cast<uint4*>(x_perm), slot_token, offsets, E,
+                                              row_vec);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_count(const moe_params& p, const int32_t* ids, int32_t* L, int32_t* counts_out,
+                         unsigned long long* counters, const Scratch& sc, cudaStream_t st) {
+    const int E = p.E_r;
+    hist_kernel<<<sc.n_tiles, 256, sizeof(int) * E, st>>>(ids, p.N, p.k, E, sc.tile_tokens,
+                                                           sc.n_tiles, sc.hist, counters);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int threads = ((E + 31) / 32) * 32 < 64 ? 64 : ((E + 31) / 32) * 32;
+    count_scan_kernel<<<1, threads, 0, st>>>(sc.hist, sc.n_tiles, E, L, counts_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_ranked(const moe_params& p, int64_t C, int bm, const int32_t* table,
+                                   int rank, int n_ranks, int64_t n_group, const int32_t* ids,
+                                   const float* w, int32_t* slot, int32_t* offsets, int32_t* L,
+                                   int32_t* acc, int32_t* slot_token, float* slot_w,
+                                   const void* x, void* x_perm, unsigned long long* counters,
+                                   const Scratch& sc, cudaStream_t st, const char** where) {
+    const int E = p.E_r, k = p.k;
+    cudaError_t e;
+    *where = "expert scan";
+    const int threads = ((E + 31) / 32) * 32 < 64 ? 64 : ((E + 31) / 32) * 32;
+    expert_scan_ranked_kernel<<<1, threads, 0, st>>>(E, C, bm, table, rank, n_ranks, n_group, L, acc,
+                                                     offsets, sc.mt_start, sc.base, counters);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    *where = "assign";
+    assign_kernel<<<sc.n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
+                                                            sc.n_tiles, sc.hist, offsets, sc.base,
+                                                            slot, slot_token, slot_w, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (x && x_perm) {
         *where = "gather";

@@ -112,7 +112,7 @@ moe_status moe_dispatch_noalloc(const moe_params* p, const int32_t* ids, const f
     unsigned long long* counters = reinterpret_cast<unsigned long long*>(b);
     int32_t* L = reinterpret_cast<int32_t*>(b + 128);
     int32_t* acc = L + E;
-    Scratch sc;
+    Scratch sc{};
     sc.mt_start = acc + E;
     sc.hist = sc.mt_start + E + 1;
     sc.n_tiles = n_tiles;

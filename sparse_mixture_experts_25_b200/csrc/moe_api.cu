@@ -58,8 +58,9 @@ static bool layout(const moe_params& p, moe_ws_layout& L, int& n_tiles, int& til
     L.x_perm = take(Nk * (size_t)p.d * es);
     L.h = take(Nk * (size_t)p.d_f * es);
     L.h_shared = take((size_t)p.N * (size_t)(p.d_f_shared > 0 ? p.d_f_shared : 0) * es);
-    // scratch: per-tile histograms, M-tile prefix, then (16-byte aligned) router scores
-    L.scratch = take(align_up(E * (size_t)std::max(n_tiles, 1) * 4 + (E + 1) * 4, 256) +
+    // scratch: per-tile histograms, M-tile prefix, earlier ranks' requests,
+    // then (256-byte aligned) router scores
+    L.scratch = take(align_up(E * (size_t)std::max(n_tiles, 1) * 4 + (E + 1) * 4 + E * 4, 256) +
                      (size_t)p.N * E * 4);
     L.total = off;
     return true;
@@ -85,9 +86,11 @@ bool make_view(const moe_params& p, void* ws, WsView& v) {
     v.h_shared = b + v.lay.h_shared;
     v.scratch.hist = reinterpret_cast<int32_t*>(b + v.lay.scratch);
     v.scratch.mt_start = v.scratch.hist + (size_t)p.E_r * std::max(n_tiles, 1);
+    v.scratch.base = v.scratch.mt_start + p.E_r + 1;
     v.scratch.logits = reinterpret_cast<float*>(
         b + v.lay.scratch +
-        align_up((size_t)p.E_r * std::max(n_tiles, 1) * 4 + ((size_t)p.E_r + 1) * 4, 256));
+        align_up((size_t)p.E_r * std::max(n_tiles, 1) * 4 + ((size_t)p.E_r + 1) * 4 +
+                     (size_t)p.E_r * 4, 256));
     v.scratch.n_tiles = n_tiles;
     v.scratch.tile_tokens = tile_tokens;
     return true;
@@ -395,6 +398,91 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     return MOE_OK;
 }
 
+moe_status moe_forward_begin(const moe_params* p, const void* x, const void* W_r, const float* b_r,
+                             const float* lat, int32_t* counts, void* ws, moe_stream_t stream) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (p->E_r > kMaxRouterExperts) return MOE_ERR_UNSUPPORTED;
+    if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    WsView v;
+    make_view(*p, ws, v);
+    (void)cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
+    if (e != cudaSuccess) return fail(e, "moe_forward_begin memset");
+    if (p->N == 0) {
+        if (counts) {
+            e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * p->E_r, st);
+            if (e != cudaSuccess) return fail(e, "moe_forward_begin memset");
+        }
+        return MOE_OK;
+    }
+    if (!x || !W_r || !aligned16(x) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
+    if (p->norm == MOE_NORM_WLR && !lat) return MOE_ERR_INVALID_ARG;
+    e = launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, v.ids, v.w, v.margin,
+                      v.counters, nullptr, v.scratch.logits, st);
+    if (e != cudaSuccess) return fail(e, "moe_forward_begin router");
+    e = launch_count(*p, v.ids, v.L, counts, v.counters, v.scratch, st);
+    if (e != cudaSuccess) return fail(e, "moe_forward_begin counts");
+    return MOE_OK;
+}
+
+moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32_t rank,
+                           int32_t n_ranks, int64_t N_group, int64_t C, const void* x,
+                           const void* W_g, const void* W_u, const void* W_d, const void* Ws_g,
+                           const void* Ws_u, const void* Ws_d, float* Y, void* ws,
+                           moe_stream_t stream) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (n_ranks < 1 || rank < 0 || rank >= n_ranks || !counts_all || C < 1 || N_group < p->N)
+        return MOE_ERR_INVALID_ARG;
+    if (p->N == 0) return MOE_OK;
+    if (!x || !W_g || !W_u || !W_d || !Y) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W_g) || !aligned16(W_u) || !aligned16(W_d) || !aligned16(Y))
+        return MOE_ERR_INVALID_ARG;
+    const bool sh = p->d_f_shared > 0;
+    if (sh && (!Ws_g || !Ws_u || !Ws_d || !aligned16(Ws_g) || !aligned16(Ws_u) || !aligned16(Ws_d)))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    WsView v;
+    make_view(*p, ws, v);
+    (void)cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(v.counters + CNT_REQUESTED, 0, 6 * 8, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(v.counters + CNT_L_MAX, 0, 2 * 8, st);
+    if (e != cudaSuccess) return fail(e, "moe_forward_end memset");
+    const bool bf16 = p->dtype == MOE_BF16;
+    const int bm = bf16 ? kTcBM : kSimtBM;
+    const char* where = "";
+    e = launch_dispatch_ranked(*p, C, bm, counts_all, rank, n_ranks, N_group, v.ids, v.w, v.slot,
+                               v.offsets, v.L, v.acc, v.slot_token, v.slot_w, x, v.x_perm,
+                               v.counters, v.scratch, st, &where);
+    if (e != cudaSuccess) {
+        char buf[96];
+        snprintf(buf, sizeof(buf), "moe_forward_end dispatch %s", where);
+        return fail(e, buf);
+    }
+    ExpertWeights W{W_g, W_u, W_d, sh ? Ws_g : nullptr, sh ? Ws_u : nullptr, sh ? Ws_d : nullptr};
+    int status = MOE_OK;
+    if (bf16) {
+        e = launch_tc_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, Y,
+                              v.counters, st, &status);
+        if (e != cudaSuccess) return fail(e, "moe_forward_end gate/up (tcgen05)");
+        e = launch_tc_down(*p, DOWN_COMBINE, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
+                           v.slot_token, v.slot_w, Y, nullptr, v.counters, st, &status);
+        if (e != cudaSuccess) return fail(e, "moe_forward_end down+combine (tcgen05)");
+    } else {
+        e = launch_zero_f32(Y, p->N * (int64_t)p->d, st);
+        if (e != cudaSuccess) return fail(e, "moe_forward_end zero");
+        e = launch_simt_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, st);
+        if (e != cudaSuccess) return fail(e, "moe_forward_end gate/up (fp32)");
+        e = launch_simt_down(*p, DOWN_COMBINE, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
+                             v.slot_token, v.slot_w, Y, nullptr, st);
+        if (e != cudaSuccess) return fail(e, "moe_forward_end down+combine (fp32)");
+    }
+    return MOE_OK;
+}
+
 moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, moe_stream_t stream) {
     moe_status s = check_params(p);
     if (s != MOE_OK) return s;
@@ -432,7 +520,8 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
         out->L_p50 = pct(50);
         out->L_p90 = pct(90);
         out->L_p99 = pct(99);
-        out->rho_max = (double)out->L_max * (double)p->E_r / ((double)p->N * (double)p->k);
+        const double n_group = cnt[CNT_N_GROUP] ? (double)cnt[CNT_N_GROUP] : (double)p->N;
+        out->rho_max = (double)out->L_max * (double)p->E_r / (n_group * (double)p->k);
         out->reject_rate = out->requested ? (double)out->rejected / (double)out->requested : 0.0;
     }
     if (cnt[CNT_DEVICE_ERROR] & DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;

@@ -32,6 +32,7 @@ enum Counter {
     CNT_L_MAX = 8,
     CNT_C = 9,
     CNT_DEVICE_ERROR = 10,  // bit flags, see DevErr
+    CNT_N_GROUP = 11,       // tokens of the whole routing group (sharded runs; 0 = N)
     CNT_COUNT = 16
 };
 
@@ -44,6 +45,7 @@ struct Scratch {
     int32_t* hist;        // [E][n_tiles] per-tile request counts -> exclusive bases
     int32_t* mt_start;    // [E+1] prefix of M tiles (BM of the GEMM in use)
     float* logits;        // [N][E] router scores (tensor-core score path)
+    int32_t* base;        // [E] requests of earlier ranks (sharded routing group)
     int n_tiles;          // dispatch tiles
     int tile_tokens;      // tokens per dispatch tile
 };
@@ -88,6 +90,16 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
                             int32_t* acc, int32_t* slot_token, float* slot_w, const void* x,
                             void* x_perm, unsigned long long* counters, const Scratch& sc,
                             cudaStream_t st, const char** where);
+// sharded routing group: per-rank request counts, then dispatch against the
+// gathered counts of all ranks
+cudaError_t launch_count(const moe_params& p, const int32_t* ids, int32_t* L, int32_t* counts_out,
+                         unsigned long long* counters, const Scratch& sc, cudaStream_t st);
+cudaError_t launch_dispatch_ranked(const moe_params& p, int64_t C, int bm, const int32_t* table,
+                                   int rank, int n_ranks, int64_t n_group, const int32_t* ids,
+                                   const float* w, int32_t* slot, int32_t* offsets, int32_t* L,
+                                   int32_t* acc, int32_t* slot_token, float* slot_w,
+                                   const void* x, void* x_perm, unsigned long long* counters,
+                                   const Scratch& sc, cudaStream_t st, const char** where);
 cudaError_t launch_combine(const moe_params& p, const float* H, const int32_t* offsets,
                            const int32_t* slot_token, const float* slot_w, float* Y,
                            cudaStream_t st);

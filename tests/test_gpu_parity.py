@@ -324,3 +324,44 @@ def test_forward_on_a_side_stream_with_stage_events():
     times = [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
     assert all(t >= 0 for t in times)
     np.testing.assert_allclose(Y.cpu().numpy(), ref["Y"], rtol=0, atol=1e-5)
+
+
+@pytest.mark.parametrize("name", ["qwen3_small_bf16", "switch_small_f32", "deepseek_small_bf16"])
+def test_sharded_group_two_ranks_on_one_gpu(name):
+    """moe_forward_begin / moe_forward_end for a routing group split over two
+    ranks, run one rank after the other on one GPU (the exchange is a stack of
+    the two count vectors): group-wide slots and outputs equal the single-GPU
+    forward of the whole batch."""
+    w = SMALL[name]
+    inp = si.inputs(w)
+    full = parity.gpu_forward(w, inp)
+    dev = full["dev"]
+    C = moe.moe_capacity(parity.params_of(w))
+    half = (w.N + 1) // 2
+    shards = [(0, half), (half, w.N)]
+    params, wss, counts = [], [], []
+    for lo, hi in shards:
+        p = parity.params_of(w.scaled(w.name, N=hi - lo))
+        ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+        cnt = torch.empty(w.E, dtype=torch.int32, device="cuda")
+        moe.moe_forward_begin(p, dev["x"][lo:hi].contiguous(), dev["W_r"], dev.get("b_r"),
+                              dev.get("lat"), cnt, ws)
+        params.append(p)
+        wss.append(ws)
+        counts.append(cnt)
+    counts_all = torch.stack(counts)
+    assert int(counts_all.sum()) == int(full["stats"]["requested"])
+    Ys, slots = [], []
+    for r, (lo, hi) in enumerate(shards):
+        Y = torch.full((hi - lo, w.d), float("nan"), device="cuda")
+        moe.moe_forward_end(params[r], counts_all, r, 2, w.N, C, dev["x"][lo:hi].contiguous(),
+                            dev["W_g"], dev["W_u"], dev["W_d"], dev.get("Ws_g"), dev.get("Ws_u"),
+                            dev.get("Ws_d"), Y, wss[r])
+        status, stats = moe.moe_get_stats(params[r], wss[r])
+        assert status == moe.MOE_OK
+        assert stats["O"] == full["stats"]["O"] and stats["L_max"] == full["stats"]["L_max"]
+        assert abs(stats["rho_max"] - full["stats"]["rho_max"]) < 1e-12
+        Ys.append(Y.cpu().numpy().astype(np.float64))
+        slots.append(moe.workspace_views(params[r], wss[r])["slot"].cpu().numpy())
+    np.testing.assert_array_equal(np.concatenate(slots), full["rec"]["slot"])
+    assert parity.rel_err(np.concatenate(Ys), full["Y"]) <= 1e-6
