@@ -32,7 +32,6 @@ import seeded_inputs as si  # noqa: E402
 
 METRIC = "MoE-layer fwd tokens/s; achieved TFLOP/s or HBM GB/s as fraction of B200 peak"
 WORKLOAD = "mixtral_bf16"
-KERNELS_PER_STEP = 7  # router, hist, scan, assign, gather, gate/up GEMM, down GEMM + combine
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -48,8 +47,17 @@ def dist_env():
     return ws, rank, local
 
 
-def rank_x_seed(w: si.Workload, rank: int) -> int:
-    return w.seed + 1000 * rank
+def kernels_per_step(w: si.Workload, sharded: bool) -> int:
+    """libmoe kernels one forward launches for this workload."""
+    if w.dtype == si.DT_BF16 and w.E % 4 == 0:
+        router = 2                      # score GEMM (tensor cores) + warp top-k
+    else:
+        router = 1                      # fused FFMA router
+    dispatch = 5 if sharded else 4      # hist, scan(s), assign, gather
+    experts = 2 if w.dtype == si.DT_BF16 else 3   # fp32 layers zero Y in the router or a kernel
+    if w.dtype != si.DT_BF16 and not sharded:
+        experts = 2
+    return router + dispatch + experts
 
 
 def max_over_ranks(value: float, device=None) -> float:
@@ -219,7 +227,9 @@ def config_of(w: si.Workload, args):
             "T": w.N, "d": w.d, "d_f": w.d_f, "E_r": w.E, "k": w.k,
             "norm": ["renorm", "fullprob", "wlr"][w.norm], "capacity_factor": w.c or None,
             "d_f_shared": w.d_f_shared, "seed": w.seed,
-            "parallelism": f"dp{args.gpus} (independent token batches per GPU)",
+            "parallelism": (f"dp{args.gpus}: one routing group of {w.N} x {args.gpus} tokens, "
+                            "per-expert request counts all-gathered once per step"
+                            if args.gpus > 1 else "dp1"),
             "l2": "inputs larger than L2 (expert weights 2.8 GB stream from HBM every step)"}
 
 
@@ -235,8 +245,10 @@ def run_gpu(args):
     # host-side inputs (generated before any CUDA call; the oracle leg below
     # uses the same buffers)
     inp = si.inputs(w)
-    if rank:
-        inp["x"] = si.fill(rank_x_seed(w, rank), si.TID["x"], w.N * w.d, dtype=w.dt).reshape(w.N, w.d)
+    if ws_n > 1:
+        # rank r holds rows [r N, (r+1) N) of one routing group of N * ranks tokens
+        inp["x"] = si.fill(w.seed, si.TID["x"], w.N * w.d, start=rank * w.N * w.d,
+                           dtype=w.dt).reshape(w.N, w.d)
     cpu_base = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         cpu_base = oracle_sample(w, inp, sample_tokens=args.ref_sample)
@@ -261,9 +273,23 @@ def run_gpu(args):
     Y = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
+    sharded_group = ws_n > 1
+    if sharded_group:
+        from sparse_mixture_experts_25_b200 import sharded
+        N_group = w.N * ws_n
+        C_group = moe.moe_capacity(moe.params(N_group, w.d, w.d_f, w.E, w.k, c=w.c, norm=w.norm,
+                                              theta=w.theta, dtype=w.dtype, d_f_shared=w.d_f_shared))
+        counts = torch.empty(w.E, dtype=torch.int32, device="cuda")
+
     def step(x_dev, y_dev):
-        moe.moe_forward(p, x_dev, d["W_r"], d["b_r"], d["lat"], d["W_g"], d["W_u"], d["W_d"],
-                        d["Ws_g"], d["Ws_u"], d["Ws_d"], y_dev, wsb, stream)
+        if sharded_group:
+            # one routing group over all ranks: exchange per-expert request counts
+            sharded.forward_sharded(p, N_group, C_group, x_dev, d["W_r"], d["b_r"], d["lat"], d["W_g"],
+                                    d["W_u"], d["W_d"], d["Ws_g"], d["Ws_u"], d["Ws_d"], y_dev, wsb,
+                                    counts=counts, stream=stream)
+        else:
+            moe.moe_forward(p, x_dev, d["W_r"], d["b_r"], d["lat"], d["W_g"], d["W_u"], d["W_d"],
+                            d["Ws_g"], d["Ws_u"], d["Ws_d"], y_dev, wsb, stream)
 
     for _ in range(args.warmup):
         step(d["x"], Y)
@@ -358,7 +384,7 @@ def run_gpu(args):
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
                 "ms_per_step": e_ms},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": kernels_per_step(w, sharded_group) * args.steps,
         "clocks": clk.summary(),
         "routing": {k: stats[k] for k in ("accepted", "rejected", "near_tie", "L_max", "rho_max")},
     }

@@ -292,7 +292,8 @@ MOE_API moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats*
  * n >= 5 events (cudaEvent_t handles created by the caller), the next
  * moe_forward calls record events[0] before the router, [1] after routing,
  * [2] after dispatch, [3] after the gate/up expert GEMM and [4] after the
- * down-projection + combine, on the call's stream.  n = 0 turns it off.
+ * down-projection + combine, on the call's stream (moe_forward_begin records
+ * [0] and [1], moe_forward_end [2] to [4]).  n = 0 turns it off.
  */
 MOE_API moe_status moe_set_stage_events(void* const* events, int n);
 

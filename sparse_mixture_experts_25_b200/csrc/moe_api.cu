@@ -419,9 +419,11 @@ moe_status moe_forward_begin(const moe_params* p, const void* x, const void* W_r
     }
     if (!x || !W_r || !aligned16(x) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
     if (p->norm == MOE_NORM_WLR && !lat) return MOE_ERR_INVALID_ARG;
+    if ((e = stage_mark(0, st)) != cudaSuccess) return fail(e, "moe_forward_begin stage event");
     e = launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, v.ids, v.w, v.margin,
                       v.counters, nullptr, v.scratch.logits, st);
     if (e != cudaSuccess) return fail(e, "moe_forward_begin router");
+    if ((e = stage_mark(1, st)) != cudaSuccess) return fail(e, "moe_forward_begin stage event");
     e = launch_count(*p, v.ids, v.L, counts, v.counters, v.scratch, st);
     if (e != cudaSuccess) return fail(e, "moe_forward_begin counts");
     return MOE_OK;
@@ -463,11 +465,13 @@ moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32
         return fail(e, buf);
     }
     ExpertWeights W{W_g, W_u, W_d, sh ? Ws_g : nullptr, sh ? Ws_u : nullptr, sh ? Ws_d : nullptr};
+    if ((e = stage_mark(2, st)) != cudaSuccess) return fail(e, "moe_forward_end stage event");
     int status = MOE_OK;
     if (bf16) {
         e = launch_tc_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, Y,
                               v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, "moe_forward_end gate/up (tcgen05)");
+        if ((e = stage_mark(3, st)) != cudaSuccess) return fail(e, "moe_forward_end stage event");
         e = launch_tc_down(*p, DOWN_COMBINE, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
                            v.slot_token, v.slot_w, Y, nullptr, v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, "moe_forward_end down+combine (tcgen05)");
@@ -476,10 +480,12 @@ moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32
         if (e != cudaSuccess) return fail(e, "moe_forward_end zero");
         e = launch_simt_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, st);
         if (e != cudaSuccess) return fail(e, "moe_forward_end gate/up (fp32)");
+        if ((e = stage_mark(3, st)) != cudaSuccess) return fail(e, "moe_forward_end stage event");
         e = launch_simt_down(*p, DOWN_COMBINE, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
                              v.slot_token, v.slot_w, Y, nullptr, st);
         if (e != cudaSuccess) return fail(e, "moe_forward_end down+combine (fp32)");
     }
+    if ((e = stage_mark(4, st)) != cudaSuccess) return fail(e, "moe_forward_end stage event");
     return MOE_OK;
 }
 

@@ -87,3 +87,29 @@ def test_rank_bases_and_ranges():
     assert sharded.rank_bases(counts_all, 0).tolist() == [0, 0, 0]
     assert sharded.rank_bases(counts_all, 2).tolist() == [4, 4, 2]
     assert [sharded.shard_range(10, r, 3) for r in range(3)] == [(0, 4), (4, 8), (8, 10)]
+
+
+def _max_worker(rank, world, port, out_q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        import bench
+        out_q.put((rank, bench.max_over_ranks(1.5 + rank, device="cpu")))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_time_is_the_max_over_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_max_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got == [(0, 2.5), (1, 2.5)]
