@@ -72,10 +72,11 @@ _lib = None
 
 
 def lib():
-    """Load (building first if missing or stale) the in-tree libmoe.so."""
+    """Load (building first if missing or stale) the in-tree libmoe.so, or the
+    library file named by the MOE_LIB_PATH environment variable."""
     global _lib
     if _lib is None:
-        path = _build.build()
+        path = os.environ.get("MOE_LIB_PATH") or _build.build()
         L = ctypes.CDLL(path)
         pp = ctypes.POINTER(Params)
         L.moe_capacity.argtypes = [pp, ctypes.POINTER(ctypes.c_int64)]

@@ -172,29 +172,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
-// Same with an L2 eviction-priority policy (createpolicy): activations that
-// many tiles re-read are kept (evict_last), weights streamed once go first.
-__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                                 int c0, int c1, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
-        : "memory");
-}
-
-__device__ __forceinline__ uint64_t policy_evict_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
-__device__ __forceinline__ uint64_t policy_evict_first() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -410,16 +387,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t phase = 0;
             int issued_parity[STAGES];
             for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
-            const uint64_t pol_act = policy_evict_last();
-            const uint64_t pol_wgt = policy_evict_first();
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                Tile ti;
-                decode_tile(t, *sched, a, routed_tiles, ti);
-                const CUtensorMap* pa = ti.shared ? &mA_sh : &mA;
-                const CUtensorMap* pb0 = ti.shared ? &mB0_sh : &mB0;
-                const CUtensorMap* pb1 = ti.shared ? &mB1_sh : &mB1;
-                int b_row0, b_row1;
+            // operand coordinates of a tile: A row, B rows of the two halves, maps
+            auto coords = [&](const Tile& ti, const CUtensorMap*& pa, const CUtensorMap*& pb0,
+                              const CUtensorMap*& pb1, int& b_row0, int& b_row1) {
+                pa = ti.shared ? &mA_sh : &mA;
+                pb0 = ti.shared ? &mB0_sh : &mB0;
+                pb1 = ti.shared ? &mB1_sh : &mB1;
                 if (EPI == EPI_SWIGLU) {
                     b_row0 = (ti.shared ? 0 : ti.g * a.b_rows_r) + ti.n_tile * 128;
                     b_row1 = b_row0;
@@ -427,6 +401,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     b_row0 = (ti.shared ? 0 : ti.g * a.b_rows_r) + ti.n_tile * 256;
                     b_row1 = b_row0 + 128;
                 }
+            };
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                Tile ti;
+                decode_tile(t, *sched, a, routed_tiles, ti);
+                const CUtensorMap *pa, *pb0, *pb1;
+                int b_row0, b_row1;
+                coords(ti, pa, pb0, pb1, b_row0, b_row1);
                 for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, a.counters)) {
                         ok = false;
@@ -435,9 +416,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     uint8_t* sa = stage_base + stage * STAGE_BYTES;
                     uint8_t* sb = sa + A_BYTES;
                     mbar_expect_tx(&full[stage], STAGE_BYTES);
-                    tma_load_2d_hint(sa, pa, &full[stage], kb * BK, ti.a_row, pol_act);
-                    tma_load_2d_hint(sb, pb0, &full[stage], kb * BK, b_row0, pol_wgt);
-                    tma_load_2d_hint(sb + B_HALF_BYTES, pb1, &full[stage], kb * BK, b_row1, pol_wgt);
+                    tma_load_2d(sa, pa, &full[stage], kb * BK, ti.a_row);
+                    tma_load_2d(sb, pb0, &full[stage], kb * BK, b_row0);
+                    tma_load_2d(sb + B_HALF_BYTES, pb1, &full[stage], kb * BK, b_row1);
                     issued_parity[stage] = (int)phase;
                     if (++stage == STAGES) {
                         stage = 0;

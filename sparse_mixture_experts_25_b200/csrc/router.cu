@@ -308,40 +308,6 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
     }
 }
 
-// Read-only (L1-cached) loads of 8 weights; streaming loads of 8 activations.
-__device__ __forceinline__ void ldg8(const float* p, float (&v)[8]) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ void ldg8(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(h[i]);
-        v[2 * i] = f.x;
-        v[2 * i + 1] = f.y;
-    }
-}
-__device__ __forceinline__ void ldcs8(const float* p, float (&v)[8]) {
-    const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
-    const float4 b = __ldcs(reinterpret_cast<const float4*>(p + 4));
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ void ldcs8(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(h[i]);
-        v[2 * i] = f.x;
-        v[2 * i + 1] = f.y;
-    }
-}
-
 __device__ __forceinline__ void zero_row(float* Y, int64_t t, int d, int lane) {
     float4* y4 = reinterpret_cast<float4*>(Y + t * d);
     for (int i = lane; i < d / 4; i += 32) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
