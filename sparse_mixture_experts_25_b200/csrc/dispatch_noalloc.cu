@@ -126,7 +126,7 @@ moe_status moe_dispatch_noalloc(const moe_params* p, const int32_t* ids, const f
         record_error(msg);
         return MOE_ERR_CUDA;
     }
-    const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
+    const int bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
     const char* where = "";
     e = launch_dispatch(*p, C, bm, ids, w, slot, offsets, L, acc, slot_token, slot_w, x, x_perm,
                         counters, sc, st, &where);

@@ -51,6 +51,8 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_HALF_BYTES = 128 * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + 2 * B_HALF_BYTES;
+constexpr int STAGES_PAIR = 6;                            // CTA pair: A + one B half per CTA
+constexpr int STAGE_BYTES_PAIR = A_BYTES + B_HALF_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
@@ -230,6 +232,84 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                  : "memory");
 }
 
+// --- CTA-pair (cta_group::2) forms -------------------------------------------
+// M = 256 across the pair (128 A rows in each CTA), N = 256 (128 B rows in each).
+constexpr uint32_t kIdescPair = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on an
+// mbarrier that may live in the peer CTA of the pair (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(kIdescPair), "r"(accumulate)
+        : "memory");
+}
+
+// arrive on the same barrier in both CTAs of the pair once the MMAs issued
+// so far complete
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((uint16_t)3)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -253,8 +333,8 @@ __device__ __forceinline__ void tmem_ld_wait() {
 struct Tile {
     int shared;     // 0 routed, 1 shared expert
     int g;          // expert
-    int a_row;      // first row of the A tile in its matrix
-    int rows;       // valid rows (<= BM)
+    int a_row;      // first row of the tile's rows in its A matrix
+    int rows;       // valid rows of the tile (<= TM)
     int n_tile;     // output-column tile
     int kb0, kb1;   // K blocks [kb0, kb1) of this tile
 };
@@ -264,6 +344,9 @@ struct SchedSmem {
     int32_t off[kMaxExperts + 1];
 };
 
+// TM: rows of one output tile (128 for one CTA, 256 for a CTA pair); the
+// M-tile prefix in `s.mt` counts tiles of TM rows.
+template <int TM>
 __device__ __forceinline__ bool decode_tile(int t_in, const SchedSmem& s, const TcArgs& a,
                                             int routed_tiles, Tile& ti) {
     // K split fastest: consecutive tiles are the K slices of one output tile
@@ -293,20 +376,20 @@ __device__ __forceinline__ bool decode_tile(int t_in, const SchedSmem& s, const 
         const int local = t - s.mt[g] * a.nt_r;
         const int m_tile = local % mtiles;
         ti.n_tile = local / mtiles;
-        ti.a_row = s.off[g] + m_tile * BM;
+        ti.a_row = s.off[g] + m_tile * TM;
         // rows of this tile inside the group and inside the row buffer
-        ti.rows = max(0, min(min(BM, s.off[g + 1] - ti.a_row), a.max_rows - ti.a_row));
+        ti.rows = max(0, min(min(TM, s.off[g + 1] - ti.a_row), a.max_rows - ti.a_row));
         if (ti.a_row < 0) ti.rows = 0;
         return true;
     }
-    const int mt_sh = (a.M_sh + BM - 1) / BM;
+    const int mt_sh = (a.M_sh + TM - 1) / TM;
     const int local = t - routed_tiles;
     if (a.M_sh <= 0 || local >= mt_sh * a.nt_sh) return false;
     ti.shared = 1;
     ti.g = 0;
     ti.n_tile = local / mt_sh;
-    ti.a_row = (local % mt_sh) * BM;
-    ti.rows = min(BM, a.M_sh - ti.a_row);
+    ti.a_row = (local % mt_sh) * TM;
+    ti.rows = min(TM, a.M_sh - ti.a_row);
     ti.kb0 = (int)((int64_t)kq * a.nkb_sh / a.ks);
     ti.kb1 = (int)((int64_t)(kq + 1) * a.nkb_sh / a.ks);
     return true;
@@ -319,28 +402,127 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Epilogue of one accumulator for the 128 rows this CTA owns (thread = row r
+// of the CTA's slice, which starts at global row `row0`; `rows` valid).
 template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const TcArgs& a, const Tile& ti, uint32_t t_row, int r,
+                                              int row0, int rows) {
+    const bool row_ok = r < rows;
+    const int grow = row0 + r;
+    if (EPI == EPI_SWIGLU) {
+        const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
+        const int ld = ti.shared ? a.ld_out_sh : a.ld_out;
+        __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(ti.shared ? a.out_sh : a.out);
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+            uint32_t g[32], u[32];
+            tmem_ld32(t_row + (uint32_t)c, g);
+            tmem_ld32(t_row + 128u + (uint32_t)c, u);
+            tmem_ld_wait();
+            const int col0 = ti.n_tile * 128 + c;
+            if (row_ok) {
+                uint4* dst = reinterpret_cast<uint4*>(outp + (int64_t)grow * ld + col0);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    if (col0 + v * 8 < n_valid) {
+                        uint4 pk;
+                        float h[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            h[j] = silu_f(__uint_as_float(g[v * 8 + j])) * __uint_as_float(u[v * 8 + j]);
+                        pk.x = pack_bf16(h[0], h[1]);
+                        pk.y = pack_bf16(h[2], h[3]);
+                        pk.z = pack_bf16(h[4], h[5]);
+                        pk.w = pack_bf16(h[6], h[7]);
+                        dst[v] = pk;
+                    }
+                }
+            }
+        }
+    } else {
+        const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
+        float wgt = 1.f;
+        float* dst_row = nullptr;
+        if (row_ok) {
+            if (EPI == EPI_COMBINE) {
+                int tok;
+                if (ti.shared) {
+                    tok = grow;
+                } else {
+                    tok = a.slot_token[grow];
+                    wgt = a.slot_w[grow];
+                }
+                if (tok < 0 || tok >= a.n_tokens) tok = -1;
+                dst_row = tok >= 0 ? a.Y + (int64_t)tok * a.ldY : nullptr;
+            } else {
+                dst_row = static_cast<float*>(a.out) + (int64_t)grow * a.ld_out;
+            }
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(t_row + (uint32_t)c, v);
+            tmem_ld_wait();
+            const int col0 = ti.n_tile * BN + c;
+            if (row_ok && dst_row) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    if (col0 + q * 4 < n_valid) {
+                        float* p = dst_row + col0 + q * 4;
+                        const float x0 = __uint_as_float(v[q * 4 + 0]) * wgt;
+                        const float x1 = __uint_as_float(v[q * 4 + 1]) * wgt;
+                        const float x2 = __uint_as_float(v[q * 4 + 2]) * wgt;
+                        const float x3 = __uint_as_float(v[q * 4 + 3]) * wgt;
+                        if (EPI == EPI_COMBINE || a.ks > 1) {
+                            red_add_v4(p, x0, x1, x2, x3);
+                        } else {
+                            *reinterpret_cast<float4*>(p) = make_float4(x0, x1, x2, x3);
+                        }
+                    }
+                }
+            }
+        }
+    }
+}
+
+// PAIR = false: one CTA computes a 128 x 256 tile (A 128 rows, B 256 rows:
+//   4 stages of 48 KB).
+// PAIR = true: a cluster of two CTAs computes a 256 x 256 tile with
+//   cta_group::2 MMAs issued by the leader (cluster rank 0): each CTA loads
+//   its 128 A rows and its 128-row half of B (6 stages of 32 KB), the
+//   leader's full barrier counts both CTAs' bytes, and the leader's commits
+//   arrive on the empty / accumulator-full barriers of both CTAs.  Each CTA
+//   drains its own TMEM rows; the leader's accumulator-empty barrier counts
+//   the epilogue warps of both CTAs.
+template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_grouped_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
                       const __grid_constant__ CUtensorMap mB1,
                       const __grid_constant__ CUtensorMap mA_sh,
                       const __grid_constant__ CUtensorMap mB0_sh,
                       const __grid_constant__ CUtensorMap mB1_sh, const TcArgs a) {
+    constexpr int NST = PAIR ? STAGES_PAIR : STAGES;
+    constexpr int SBYTES = PAIR ? STAGE_BYTES_PAIR : STAGE_BYTES;
+    constexpr int TM = PAIR ? 256 : 128;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned stage buffers (the 128-byte swizzle atom spans 8 rows)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* stage_base = smem;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-    uint64_t* empty = full + STAGES;
-    uint64_t* tfull = empty + STAGES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + NST * SBYTES);
+    uint64_t* empty = full + NST;
+    uint64_t* tfull = empty + NST;
     uint64_t* tempty = tfull + 2;
     uint64_t* done = tempty + 2;
     uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
-    SchedSmem* sched = reinterpret_cast<SchedSmem*>(smem + STAGES * STAGE_BYTES + 256);
+    SchedSmem* sched = reinterpret_cast<SchedSmem*>(smem + NST * SBYTES + 256);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
+    const bool leader = crank == 0;
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;   // tile-processing unit
+    const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     if (a.has_routed) {
         for (int i = threadIdx.x; i <= a.E; i += NUM_THREADS) {
@@ -349,19 +531,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 128);
+            mbar_init(&tempty[b], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
         }
         mbar_init(done, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) tmem_alloc(tmem_base_s, TMEM_COLS);
+    if (warp == 1) {
+        if (PAIR) tmem_alloc_pair(tmem_base_s, TMEM_COLS);
+        else tmem_alloc(tmem_base_s, TMEM_COLS);
+    }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&mA);
         tma_prefetch_desc(&mB0);
@@ -373,77 +558,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR) cluster_sync_all();  // the peer's barriers exist before any remote arrival
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_s;
 
     const int routed_tiles = a.has_routed ? sched->mt[a.E] * a.nt_r : 0;
     const int total_tiles =
-        (routed_tiles + (a.M_sh > 0 ? ((a.M_sh + BM - 1) / BM) * a.nt_sh : 0)) * a.ks;
+        (routed_tiles + (a.M_sh > 0 ? ((a.M_sh + TM - 1) / TM) * a.nt_sh : 0)) * a.ks;
 
     if (warp == 0) {
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int issued_parity[STAGES];
-            for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+            int issued_parity[NST];
+            for (int s = 0; s < NST; ++s) issued_parity[s] = -1;
             bool ok = true;
-            // operand coordinates of a tile: A row, B rows of the two halves, maps
-            auto coords = [&](const Tile& ti, const CUtensorMap*& pa, const CUtensorMap*& pb0,
-                              const CUtensorMap*& pb1, int& b_row0, int& b_row1) {
-                pa = ti.shared ? &mA_sh : &mA;
-                pb0 = ti.shared ? &mB0_sh : &mB0;
-                pb1 = ti.shared ? &mB1_sh : &mB1;
-                if (EPI == EPI_SWIGLU) {
+            for (int t = unit; t < total_tiles && ok; t += n_units) {
+                Tile ti;
+                decode_tile<TM>(t, *sched, a, routed_tiles, ti);
+                const CUtensorMap* pa = ti.shared ? &mA_sh : &mA;
+                const CUtensorMap* pb0 = ti.shared ? &mB0_sh : &mB0;
+                const CUtensorMap* pb1 = ti.shared ? &mB1_sh : &mB1;
+                int b_row0, b_row1;
+                if (EPI == EPI_SWIGLU) {  // gate rows and up rows of the same 128 columns
                     b_row0 = (ti.shared ? 0 : ti.g * a.b_rows_r) + ti.n_tile * 128;
                     b_row1 = b_row0;
-                } else {
+                } else {                  // two 128-column halves of a 256-column tile
                     b_row0 = (ti.shared ? 0 : ti.g * a.b_rows_r) + ti.n_tile * 256;
                     b_row1 = b_row0 + 128;
                 }
-            };
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                Tile ti;
-                decode_tile(t, *sched, a, routed_tiles, ti);
-                const CUtensorMap *pa, *pb0, *pb1;
-                int b_row0, b_row1;
-                coords(ti, pa, pb0, pb1, b_row0, b_row1);
+                const int a_row = ti.a_row + (PAIR ? (int)crank * 128 : 0);
                 for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, a.counters)) {
                         ok = false;
                         break;
                     }
-                    uint8_t* sa = stage_base + stage * STAGE_BYTES;
+                    uint8_t* sa = stage_base + stage * SBYTES;
                     uint8_t* sb = sa + A_BYTES;
-                    mbar_expect_tx(&full[stage], STAGE_BYTES);
-                    tma_load_2d(sa, pa, &full[stage], kb * BK, ti.a_row);
-                    tma_load_2d(sb, pb0, &full[stage], kb * BK, b_row0);
-                    tma_load_2d(sb + B_HALF_BYTES, pb1, &full[stage], kb * BK, b_row1);
+                    if (PAIR) {
+                        // both CTAs' bytes complete on the leader's full barrier
+                        const uint32_t fb = map_shared_rank(smem_u32(&full[stage]), 0);
+                        if (leader) mbar_expect_tx(&full[stage], 2 * SBYTES);
+                        tma_load_2d_pair(sa, pa, fb, kb * BK, a_row);
+                        if (crank == 0) tma_load_2d_pair(sb, pb0, fb, kb * BK, b_row0);
+                        else tma_load_2d_pair(sb, pb1, fb, kb * BK, b_row1);
+                    } else {
+                        mbar_expect_tx(&full[stage], SBYTES);
+                        tma_load_2d(sa, pa, &full[stage], kb * BK, a_row);
+                        tma_load_2d(sb, pb0, &full[stage], kb * BK, b_row0);
+                        tma_load_2d(sb + B_HALF_BYTES, pb1, &full[stage], kb * BK, b_row1);
+                    }
                     issued_parity[stage] = (int)phase;
-                    if (++stage == STAGES) {
+                    if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            if (*abort_flag) {
-                // drain copies still in flight into this CTA's shared memory
-                for (int s = 0; s < STAGES; ++s)
+            if (*abort_flag && (!PAIR || leader)) {
+                // drain copies still in flight into shared memory
+                for (int s = 0; s < NST; ++s)
                     if (issued_parity[s] >= 0)
                         wait_bounded(&full[s], (uint32_t)issued_parity[s], abort_flag, a.counters,
                                      kTimeoutNs / 4);
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && (!PAIR || leader)) {
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int t = unit; t < total_tiles && ok; t += n_units) {
                 Tile ti;
-                decode_tile(t, *sched, a, routed_tiles, ti);
+                decode_tile<TM>(t, *sched, a, routed_tiles, ti);
                 if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, a.counters)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -453,31 +643,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+                    const uint32_t sa = smem_u32(stage_base + stage * SBYTES);
                     const uint32_t sb = sa + A_BYTES;
                     const uint64_t ad = smem_desc_sw128(sa);
                     const uint64_t bd = smem_desc_sw128(sb);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         // advance 16 elements (32 bytes) along K inside the swizzled row
-                        umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2),
-                                  (kb > ti.kb0 || kk > 0) ? 1u : 0u);
+                        const uint32_t accum = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
+                        if (PAIR) umma_bf16_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), accum);
+                        else umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), accum);
                     }
-                    umma_commit(&empty[stage]);
-                    if (++stage == STAGES) {
+                    if (PAIR) umma_commit_pair_both(&empty[stage]);
+                    else umma_commit(&empty[stage]);
+                    if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                umma_commit(&tfull[acc]);
+                if (PAIR) umma_commit_pair_both(&tfull[acc]);
+                else umma_commit(&tfull[acc]);
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
             }
             // all MMAs issued by this thread have completed once `done` fires
-            umma_commit(done);
+            if (PAIR) umma_commit_pair_local(done);
+            else umma_commit(done);
             wait_bounded(done, 0, abort_flag, a.counters, kTimeoutNs / 4);
         }
     } else {
@@ -495,90 +689,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int r = quarter * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        for (int t = unit; t < total_tiles; t += n_units) {
             Tile ti;
-            decode_tile(t, *sched, a, routed_tiles, ti);
+            decode_tile<TM>(t, *sched, a, routed_tiles, ti);
             if (!warp_wait_bounded(&tfull[acc], acc_phase, abort_flag, a.counters)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-            const bool row_ok = r < ti.rows;
-            const int grow = ti.a_row + r;
-            if (EPI == EPI_SWIGLU) {
-                const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
-                const int ld = ti.shared ? a.ld_out_sh : a.ld_out;
-                __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(ti.shared ? a.out_sh : a.out);
-#pragma unroll 1
-                for (int c = 0; c < 128; c += 32) {
-                    uint32_t g[32], u[32];
-                    tmem_ld32(t_row + (uint32_t)c, g);
-                    tmem_ld32(t_row + 128u + (uint32_t)c, u);
-                    tmem_ld_wait();
-                    const int col0 = ti.n_tile * 128 + c;
-                    if (row_ok) {
-                        uint4* dst = reinterpret_cast<uint4*>(outp + (int64_t)grow * ld + col0);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            if (col0 + v * 8 < n_valid) {
-                                uint4 pk;
-                                float h[8];
-#pragma unroll
-                                for (int j = 0; j < 8; ++j)
-                                    h[j] = silu_f(__uint_as_float(g[v * 8 + j])) * __uint_as_float(u[v * 8 + j]);
-                                pk.x = pack_bf16(h[0], h[1]);
-                                pk.y = pack_bf16(h[2], h[3]);
-                                pk.z = pack_bf16(h[4], h[5]);
-                                pk.w = pack_bf16(h[6], h[7]);
-                                dst[v] = pk;
-                            }
-                        }
-                    }
-                }
-            } else {
-                const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
-                float wgt = 1.f;
-                float* dst_row = nullptr;
-                if (row_ok) {
-                    if (EPI == EPI_COMBINE) {
-                        int tok;
-                        if (ti.shared) {
-                            tok = grow;
-                        } else {
-                            tok = a.slot_token[grow];
-                            wgt = a.slot_w[grow];
-                        }
-                        if (tok < 0 || tok >= a.n_tokens) tok = -1;
-                        dst_row = tok >= 0 ? a.Y + (int64_t)tok * a.ldY : nullptr;
-                    } else {
-                        dst_row = static_cast<float*>(a.out) + (int64_t)grow * a.ld_out;
-                    }
-                }
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(t_row + (uint32_t)c, v);
-                    tmem_ld_wait();
-                    const int col0 = ti.n_tile * BN + c;
-                    if (row_ok && dst_row) {
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            if (col0 + q * 4 < n_valid) {
-                                float* p = dst_row + col0 + q * 4;
-                                const float x0 = __uint_as_float(v[q * 4 + 0]) * wgt;
-                                const float x1 = __uint_as_float(v[q * 4 + 1]) * wgt;
-                                const float x2 = __uint_as_float(v[q * 4 + 2]) * wgt;
-                                const float x3 = __uint_as_float(v[q * 4 + 3]) * wgt;
-                                if (EPI == EPI_COMBINE || a.ks > 1) {
-                                    red_add_v4(p, x0, x1, x2, x3);
-                                } else {
-                                    *reinterpret_cast<float4*>(p) = make_float4(x0, x1, x2, x3);
-                                }
-                            }
-                        }
-                    }
-                }
-            }
+            const int row0 = ti.a_row + (PAIR ? (int)crank * 128 : 0);
+            const int rows = PAIR ? max(0, min(128, ti.rows - (int)crank * 128)) : ti.rows;
+            epilogue_tile<EPI>(a, ti, t_row, r, row0, rows);
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);
+            __syncwarp();
+            if (lane == 0) {
+                if (PAIR) mbar_arrive_cluster(map_shared_rank(smem_u32(&tempty[acc]), 0));
+                else mbar_arrive(&tempty[acc]);
+            }
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
@@ -587,10 +712,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 
     __syncwarp();
+    if (PAIR && *abort_flag) {
+        // copies of the peer CTA complete on the leader's barriers: give any
+        // still in flight time to land before the pair leaves
+        const unsigned long long t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 2000000ull) {
+        }
+    }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR) cluster_sync_all();  // the leader's MMAs into the peer's TMEM are complete
+    else __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+    if (warp == 1) {
+        if (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        else tmem_dealloc(tmem_base, TMEM_COLS);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -623,31 +759,53 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
 }
 
 constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + sizeof(SchedSmem);
+constexpr size_t kSmemBytesPair = 1024 + (size_t)STAGES_PAIR * STAGE_BYTES_PAIR + 256 + sizeof(SchedSmem);
 
-template <int EPI>
+template <int EPI, bool PAIR>
 cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mB0, const CUtensorMap& mB1,
                       const CUtensorMap& mA_sh, const CUtensorMap& mB0_sh, const CUtensorMap& mB1_sh,
                       const TcArgs& a, int64_t max_tiles, cudaStream_t st) {
-    auto kern = tc_grouped_kernel<EPI>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    auto kern = tc_grouped_kernel<EPI, PAIR>;
+    const size_t smem = PAIR ? kSmemBytesPair : kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int grid = (int)min64(max_tiles, num_sms());
-    if (grid <= 0) return cudaSuccess;
-    kern<<<grid, NUM_THREADS, kSmemBytes, st>>>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a);
+    if (!PAIR) {
+        const int grid = (int)min64(max_tiles, num_sms());
+        if (grid <= 0) return cudaSuccess;
+        kern<<<grid, NUM_THREADS, smem, st>>>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a);
+        return cudaGetLastError();
+    }
+    // clusters of two CTAs, one tile per cluster at a time
+    const int pairs = (int)min64(max_tiles, num_sms() / 2);
+    if (pairs <= 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-int64_t routed_mtile_bound(const moe_params& p) {
-    return (p.N * p.k + BM - 1) / BM + p.E_r;
+int64_t routed_mtile_bound(const moe_params& p, int tm) {
+    return (p.N * p.k + tm - 1) / tm + p.E_r;
 }
 
 // Expected routed M tiles: each expert gets about mu = N k / E_r rows (at most
 // C); a group of r rows takes ceil(r / 128) tiles, about r / 128 + 1/2 on average.
-double routed_mtile_estimate(const moe_params& p, int64_t C) {
+double routed_mtile_estimate(const moe_params& p, int64_t C, int tm) {
     double mu = (double)p.N * p.k / p.E_r;
     if (mu > (double)C) mu = (double)C;
     if (mu <= 0) return 0;
-    const double per = mu / BM + 0.5;
+    const double per = mu / tm + 0.5;
     return p.E_r * (per < 1.0 ? 1.0 : per);
 }
 
@@ -674,6 +832,12 @@ int choose_ksplit(double tiles, int nkb_min) {
 }
 
 }  // namespace
+
+int tc_tile_rows(const moe_params& p) {
+    // CTA pairs (256-row tiles) when experts average enough rows to fill them
+    const double mu = (double)p.N * p.k / p.E_r;
+    return (p.dtype == MOE_BF16 && mu >= 768.0) ? 256 : 128;
+}
 
 cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
                               const int32_t* offsets, const int32_t* mt_start,
@@ -722,9 +886,14 @@ cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const voi
     a.zero_ptr = Y_zero;
     a.zero_n4 = Y_zero ? p.N * (int64_t)p.d / 4 : 0;
     a.counters = counters;
-    int64_t max_tiles = routed_mtile_bound(p) * a.nt_r + (sh ? ((p.N + BM - 1) / BM) * a.nt_sh : 0);
-    if (Y_zero && max_tiles < num_sms()) max_tiles = num_sms();  // every CTA zeroes a share
-    return launch_tc<EPI_SWIGLU>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a, max_tiles, st);
+    const bool pair = tc_tile_rows(p) == 256;
+    const int tm = pair ? 256 : 128;
+    int64_t max_tiles =
+        routed_mtile_bound(p, tm) * a.nt_r + (sh ? ((p.N + tm - 1) / tm) * a.nt_sh : 0);
+    const int units = pair ? num_sms() / 2 : num_sms();
+    if (Y_zero && max_tiles < units) max_tiles = units;  // every CTA zeroes a share
+    if (pair) return launch_tc<EPI_SWIGLU, true>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a, max_tiles, st);
+    return launch_tc<EPI_SWIGLU, false>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a, max_tiles, st);
 }
 
 cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void* h,
@@ -770,19 +939,24 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
     a.n_tokens = (int)p.N;
     a.has_routed = 1;
     a.ks = 1;
+    const bool pair = tc_tile_rows(p) == 256;
+    const int tm = pair ? 256 : 128;
     if (mode == DOWN_COMBINE) {
         // the combine reduces with red.add into a zeroed Y, so K slices of one
         // output tile can run on different SMs: split K to fill the last wave
-        const double tiles = routed_mtile_estimate(p, C) * a.nt_r +
-                             (sh ? (double)((p.N + BM - 1) / BM) * a.nt_sh : 0.0);
-        a.ks = choose_ksplit(tiles, sh ? std::min(a.nkb_r, a.nkb_sh) : a.nkb_r);
+        const double tiles = routed_mtile_estimate(p, C, tm) * a.nt_r +
+                             (sh ? (double)((p.N + tm - 1) / tm) * a.nt_sh : 0.0);
+        a.ks = choose_ksplit(pair ? 2.0 * tiles : tiles, sh ? std::min(a.nkb_r, a.nkb_sh) : a.nkb_r);
     }
     a.counters = counters;
     int64_t max_tiles =
-        (routed_mtile_bound(p) * a.nt_r + (sh ? ((p.N + BM - 1) / BM) * a.nt_sh : 0)) * a.ks;
-    if (mode == DOWN_COMBINE)
-        return launch_tc<EPI_COMBINE>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
-    return launch_tc<EPI_STORE>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
+        (routed_mtile_bound(p, tm) * a.nt_r + (sh ? ((p.N + tm - 1) / tm) * a.nt_sh : 0)) * a.ks;
+    if (mode == DOWN_COMBINE) {
+        if (pair) return launch_tc<EPI_COMBINE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
+        return launch_tc<EPI_COMBINE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
+    }
+    if (pair) return launch_tc<EPI_STORE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
+    return launch_tc<EPI_STORE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
 }
 
 cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,
@@ -804,14 +978,14 @@ cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r
     a.ld_out = p.E_r;
     a.max_rows = (int)p.N;
     a.n_tokens = (int)p.N;
-    const int64_t tiles = ((p.N + BM - 1) / BM) * a.nt_sh;
+    const int64_t tiles = ((p.N + 127) / 128) * a.nt_sh;
     a.ks = choose_ksplit((double)tiles, a.nkb_sh);
     a.counters = counters;
     if (a.ks > 1) {  // K slices add into the scores with red.add
         cudaError_t e = cudaMemsetAsync(logits, 0, sizeof(float) * (size_t)p.N * p.E_r, st);
         if (e != cudaSuccess) return e;
     }
-    return launch_tc<EPI_STORE>(mA, mB, mB, mA, mB, mB, a, tiles * a.ks, st);
+    return launch_tc<EPI_STORE, false>(mA, mB, mB, mA, mB, mB, a, tiles * a.ks, st);
 }
 
 }  // namespace moe

@@ -269,7 +269,7 @@ moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const float* w,
     cudaError_t e = cudaMemsetAsync(v.counters + CNT_REQUESTED, 0, 6 * 8, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(v.counters + CNT_L_MAX, 0, 2 * 8, st);
     if (e != cudaSuccess) return fail(e, "moe_dispatch memset");
-    const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
+    const int bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
     const char* where = "";
     e = launch_dispatch(*p, C, bm, ids, w, slot, offsets, v.L, v.acc, slot_token, slot_w, x, x_perm,
                         v.counters, v.scratch, st, &where);
@@ -297,7 +297,7 @@ moe_status moe_expert_ffn(const moe_params* p, const void* x_perm, const int32_t
     moe_params q = *p;
     q.d_f_shared = 0;  // routed experts only
     ExpertWeights W{W_g, W_u, W_d, nullptr, nullptr, nullptr};
-    const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
+    const int bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
     (void)cudaGetLastError();
     cudaError_t e0 = launch_mtile_prefix(p->E_r, bm, offsets, v.scratch.mt_start, st);
     if (e0 != cudaSuccess) return fail(e0, "moe_expert_ffn prefix");
@@ -367,7 +367,7 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
                                   v.w, v.margin, v.counters, bf16 ? nullptr : Y, v.scratch.logits, st);
     if (e != cudaSuccess) return fail(e, "moe_forward router");
     if ((e0 = stage_mark(1, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
-    const int bm = p->dtype == MOE_BF16 ? kTcBM : kSimtBM;
+    const int bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
     const char* where = "";
     e = launch_dispatch(*p, C, bm, v.ids, v.w, v.slot, v.offsets, v.L, v.acc, v.slot_token, v.slot_w,
                         x, v.x_perm, v.counters, v.scratch, st, &where);
@@ -454,7 +454,7 @@ moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32
     if (e == cudaSuccess) e = cudaMemsetAsync(v.counters + CNT_L_MAX, 0, 2 * 8, st);
     if (e != cudaSuccess) return fail(e, "moe_forward_end memset");
     const bool bf16 = p->dtype == MOE_BF16;
-    const int bm = bf16 ? kTcBM : kSimtBM;
+    const int bm = bf16 ? tc_tile_rows(*p) : kSimtBM;
     const char* where = "";
     e = launch_dispatch_ranked(*p, C, bm, counts_all, rank, n_ranks, N_group, v.ids, v.w, v.slot,
                                v.offsets, v.L, v.acc, v.slot_token, v.slot_w, x, v.x_perm,

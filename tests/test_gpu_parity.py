@@ -51,6 +51,12 @@ SMALL = {
     "wide_router_f32": W["switch_top1_f32"].scaled("wide_router_f32", N=200, d=64, d_f=64, E=48, k=3,
                                                    norm=si.NORM_RENORM, c=0.0),
     "odd_experts_bf16": W["mixtral_bf16"].scaled("odd_experts_bf16", N=200, d=64, d_f=64, E=34, k=3),
+    # >= 768 rows per expert: 256-row tiles on CTA pairs (ragged last pair tile)
+    "pair_bf16": W["mixtral_bf16"].scaled("pair_bf16", N=1600, d=320, d_f=384, E=2, k=1),
+    "pair_shared_bf16": W["mixtral_bf16"].scaled("pair_shared_bf16", N=1700, d=256, d_f=256, E=2, k=1,
+                                                 d_f_shared=128),
+    "pair_capped_bf16": W["mixtral_bf16"].scaled("pair_capped_bf16", N=2000, d=128, d_f=256, E=2, k=1,
+                                                 c=0.9),
 }
 
 
@@ -198,7 +204,7 @@ def test_n4_example_capacity_and_statistics():
 # ---------------------------------------------------------------------------
 # the unfused entry points compose to the fused forward
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("name", ["mixtral_small_bf16", "switch_small_f32"])
+@pytest.mark.parametrize("name", ["mixtral_small_bf16", "switch_small_f32", "pair_bf16"])
 def test_unfused_path_matches_fused(name):
     w = SMALL[name]
     inp = si.inputs(w)
@@ -326,7 +332,8 @@ def test_forward_on_a_side_stream_with_stage_events():
     np.testing.assert_allclose(Y.cpu().numpy(), ref["Y"], rtol=0, atol=1e-5)
 
 
-@pytest.mark.parametrize("name", ["qwen3_small_bf16", "switch_small_f32", "deepseek_small_bf16"])
+@pytest.mark.parametrize("name", ["qwen3_small_bf16", "switch_small_f32", "deepseek_small_bf16",
+                                  "pair_capped_bf16"])
 def test_sharded_group_two_ranks_on_one_gpu(name):
     """moe_forward_begin / moe_forward_end for a routing group split over two
     ranks, run one rank after the other on one GPU (the exchange is a stack of
