@@ -372,3 +372,29 @@ def test_sharded_group_two_ranks_on_one_gpu(name):
         slots.append(moe.workspace_views(params[r], wss[r])["slot"].cpu().numpy())
     np.testing.assert_array_equal(np.concatenate(slots), full["rec"]["slot"])
     assert parity.rel_err(np.concatenate(Ys), full["Y"]) <= 1e-6
+
+
+def test_host_pipeline_matches_direct_forward():
+    """Batches streamed from pinned host memory through HostPipeline give the
+    outputs of direct moe_forward calls, batch by batch."""
+    from sparse_mixture_experts_25_b200.pipeline import HostPipeline
+    w = SMALL["mixtral_small_bf16"]
+    batches = [w.scaled(w.name, seed=w.seed + i) for i in range(5)]
+    ref = [parity.gpu_forward(b, si.inputs(b)) for b in batches]
+    dev = ref[0]["dev"]
+    p = parity.params_of(w)
+    pipe = HostPipeline(p, dev)
+    hosts = [torch.from_numpy(si.tensor(b, "x").view(np.int16)).view(torch.bfloat16).pin_memory()
+             for b in batches]
+    outs = [torch.empty(w.N, w.d, dtype=torch.float32).pin_memory() for _ in batches]
+    for xh, yh in zip(hosts, outs):
+        pipe.submit(xh, yh)
+    pipe.synchronize()
+    # same weights for every batch: compare against the direct path on those weights
+    for b, yh in zip(batches, outs):
+        x = parity.to_dev(si.tensor(b, "x"))
+        Y = torch.empty(w.N, w.d, device="cuda")
+        ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+        moe.moe_forward(p, x, dev["W_r"], None, None, dev["W_g"], dev["W_u"], dev["W_d"], None, None, None, Y, ws)
+        torch.cuda.synchronize()
+        np.testing.assert_allclose(yh.numpy(), Y.cpu().numpy(), rtol=0, atol=1e-5)
