@@ -71,6 +71,15 @@ typedef enum moe_norm {
 
 typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
+/* What a path rejected by the capacity limit does to the token's other paths
+ * ("LLM from scratch" ch. 36.3-36.4: the overflow policy is part of the
+ * function; the worked example prints both outcomes). */
+typedef enum moe_reject_policy {
+    MOE_REJECT_ZERO = 0,   /* rejected path adds 0, the others keep their weights
+                              (Algorithm 36.1)                                     */
+    MOE_REJECT_RENORM = 1  /* the token's accepted paths are rescaled to sum to 1  */
+} moe_reject_policy;
+
 typedef struct moe_params {
     int64_t N;          /* tokens in the routing group, N >= 0                      */
     int32_t d;          /* model width                                               */
@@ -82,6 +91,7 @@ typedef struct moe_params {
     float theta;        /* WLR threshold in [0, 1) (MOE_NORM_WLR only)               */
     int32_t dtype;      /* moe_dtype of x and of every weight                        */
     int32_t d_f_shared; /* hidden width of the always-on shared expert; 0 = none     */
+    int32_t reject_policy; /* moe_reject_policy                                      */
 } moe_params;
 
 /* Routing statistics of the last moe_dispatch / moe_forward on a workspace
@@ -168,7 +178,9 @@ MOE_API moe_status moe_route(const moe_params* p, const void* x, const void* W_r
  *   offsets    [E_r + 1] int32 out: accepted rows of expert e are rows
  *              offsets[e] .. offsets[e+1]-1 of the expert buffers, in slot order
  *   slot_token [N k] int32 out: source token of each accepted row
- *   slot_w     [N k] fp32 out: weight a_te of each accepted row
+ *   slot_w     [N k] fp32 out: combine weight of each accepted row: a_te, or
+ *              under MOE_REJECT_RENORM a_te / (sum of the token's accepted a)
+ *              for tokens that lost a path
  *   x          [N, d] dtype, nullable; with x_perm [N k, d] dtype, gathers
  *              x_perm[r] = x[slot_token[r]] for every accepted row r
  * Statistics (L_e, accepted, O, ...) go to the workspace counters.

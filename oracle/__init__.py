@@ -66,12 +66,14 @@ def _load():
         lib.oracle_combine.argtypes = [i64, i32, i32, _P, _P, _P, _P, _P]
         lib.oracle_forward_rows.argtypes = [i32, i32, i32, i32, i32, i32, _P, _P, _P, _P, _P, i64,
                                             _P, _P, _P, _P, _P, _P, _P]
-        lib.oracle_forward.argtypes = [i64, i32, i32, i32, i32, i32, dbl, i32, i64, i32,
+        lib.oracle_reject_weights.argtypes = [i64, i32, i32, _P, _P, _P, _P]
+        lib.oracle_forward.argtypes = [i64, i32, i32, i32, i32, i32, dbl, i32, i64, i32, i32,
                                        _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                        _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         lib.oracle_round_bf16.argtypes = [dbl]
         lib.oracle_round_bf16.restype = dbl
-        for f in ("oracle_route", "oracle_dispatch", "oracle_dispatch_ranked", "oracle_swiglu_rows", "oracle_combine",
+        for f in ("oracle_route", "oracle_dispatch", "oracle_dispatch_ranked", "oracle_reject_weights",
+                  "oracle_swiglu_rows", "oracle_combine",
                   "oracle_forward_rows", "oracle_forward"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
@@ -262,8 +264,21 @@ def forward_rows(x, ids, w, slot, tokens, Wg, Wu, Wd, Ws=None):
     return Y
 
 
+def reject_weights(ids, w, slot, policy: int):
+    """Combine weights of the routing records under an overflow policy
+    (0: zero, no renormalisation; 1: accepted paths of a token that lost a
+    path rescaled to sum to one); see oracle.c."""
+    ids = _c(ids, np.int32)
+    N, k = ids.shape
+    w = _c(w, np.float64)
+    slot = _c(slot, np.int32)
+    wc = np.empty((N, k), np.float64)
+    _load().oracle_reject_weights(N, k, int(policy), _ptr(ids), _ptr(w), _ptr(slot), _ptr(wc))
+    return wc
+
+
 def forward(x, W_r, Wg, Wu, Wd, *, k: int, norm: int, c: float = 0.0, theta: float = 0.0,
-            b_r=None, lat=None, Ws=None):
+            b_r=None, lat=None, Ws=None, reject_policy: int = 0):
     """The whole layer (Algorithm 36.1 generalised by the weighting mode and a
     shared expert).  Returns a dict with Y [N,d] f64, the routing records,
     per-expert loads and the statistics."""
@@ -290,7 +305,8 @@ def forward(x, W_r, Wg, Wu, Wd, *, k: int, norm: int, c: float = 0.0, theta: flo
         dsh = 0
     b = _c(b_r, np.float32)
     la = _c(lat, np.float32)
-    rc = _load().oracle_forward(N, d, d_f, E, k, norm, theta, dt, max(C, 1), dsh, _ptr(x), _ptr(W_r),
+    rc = _load().oracle_forward(N, d, d_f, E, k, norm, theta, dt, max(C, 1), dsh, int(reject_policy),
+                                _ptr(x), _ptr(W_r),
                                 _ptr(b), _ptr(la), _ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(Wsg), _ptr(Wsu),
                                 _ptr(Wsd), _ptr(Y), _ptr(ids), _ptr(w), _ptr(slot), _ptr(margin),
                                 _ptr(gap), _ptr(inv), _ptr(L), _ptr(acc), _ptr(cnt))

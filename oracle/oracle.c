@@ -270,6 +270,35 @@ int oracle_dispatch_ranked(int64_t N, int k, int E, int64_t C, const int32_t* id
 }
 
 /*
+ * Combine weights under an overflow policy ("LLM from scratch" ch. 36.3: the
+ * handling of a rejected path is part of the model definition; ch. 36.4
+ * worked example, both outcomes).  policy 0: a rejected path contributes 0
+ * and the other paths keep a_te (Algorithm 36.1).  policy 1: for a token
+ * that lost some but not all paths, its accepted paths are rescaled to sum to
+ * one: wc = a_te / sum over its accepted paths of a.  wc is 0 for rejected or
+ * unrequested paths.
+ */
+int oracle_reject_weights(int64_t N, int k, int policy, const int32_t* ids, const double* w,
+                          const int32_t* slot, double* wc) {
+    for (int64_t t = 0; t < N; ++t) {
+        int req = 0, rej = 0;
+        double acc_sum = 0.0;
+        for (int j = 0; j < k; ++j) {
+            if (ids[t * k + j] < 0) continue;
+            ++req;
+            if (slot[t * k + j] < 0) ++rej;
+            else acc_sum += w[t * k + j];
+        }
+        for (int j = 0; j < k; ++j) {
+            int i = (int)(t * k + j);
+            if (ids[i] < 0 || slot[i] < 0) { wc[i] = 0.0; continue; }
+            wc[i] = (policy == 1 && rej > 0 && rej < req) ? w[i] / acc_sum : w[i];
+        }
+    }
+    return 0;
+}
+
+/*
  * One SwiGLU expert on a list of token rows (vegetog sec. 3):
  *   E(x) = [SiLU(x W_gate) (.) (x W_up)] W_down
  * with W_gate, W_up stored [d_f, d] and W_down stored [d, d_f].  When
@@ -365,13 +394,13 @@ int oracle_forward_rows(int d, int d_f, int E, int k, int dtype, int d_f_sh, con
 }
 
 /*
- * The whole layer (Algorithm 36.1, generalised by the normalisation mode and
- * an optional shared expert): route, token-order acceptance with capacity C,
+ * The whole layer (Algorithm 36.1, generalised by the normalisation mode, the
+ * overflow policy of oracle_reject_weights and an optional shared expert): route, token-order acceptance with capacity C,
  * each expert evaluated only on its accepted slots, weighted combine, plus
  * the shared expert.  Y is [N, d] in double.
  */
 int oracle_forward(int64_t N, int d, int d_f, int E, int k, int norm, double theta, int dtype,
-                   int64_t C, int d_f_sh, const void* x, const void* W_r, const float* b_r,
+                   int64_t C, int d_f_sh, int reject_policy, const void* x, const void* W_r, const float* b_r,
                    const float* lat, const void* Wg, const void* Wu, const void* Wd,
                    const void* Wsg, const void* Wsu, const void* Wsd, double* Y, int32_t* ids,
                    double* w, int32_t* slot, double* margin, double* wlr_gap, uint8_t* invalid,
@@ -402,7 +431,10 @@ int oracle_forward(int64_t N, int d, int d_f, int E, int k, int norm, double the
                            (const char*)Wd + (size_t)e * d * d_f * esz, Hs[e]);
         free(rows);
     }
-    oracle_combine(N, k, d, ids, w, slot, (const double* const*)Hs, Y);
+    double* wc = (double*)malloc(sizeof(double) * N * k);
+    oracle_reject_weights(N, k, reject_policy, ids, w, slot, wc);
+    oracle_combine(N, k, d, ids, wc, slot, (const double* const*)Hs, Y);
+    free(wc);
     for (int e = 0; e < E; ++e) free(Hs[e]);
     free(Hs);
     if (d_f_sh > 0 && Wsg) {

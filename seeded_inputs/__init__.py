@@ -167,6 +167,7 @@ class Workload:
     zipf_s: float = 0.0         # > 0: router bias b_e = 0.5 ln(Zipf(s) weight of rank e+1)
     latency: bool = False       # per-token per-expert latency t = t_up + t_comp + t_down
     seed: int = 25000
+    reject_policy: int = 0      # 0: rejected path adds 0; 1: accepted paths renormalised
 
     @property
     def dt(self) -> str:

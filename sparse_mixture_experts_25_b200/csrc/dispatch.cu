@@ -199,7 +199,7 @@ __global__ void expert_scan_ranked_kernel(int E, int64_t C, int bm, const int32_
 __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w,
                               int64_t N, int k, int E, int64_t C, int tile_tokens, int n_tiles,
                               const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets,
-                              const int32_t* __restrict__ rank_base,
+                              const int32_t* __restrict__ rank_base, int renorm_rejected,
                               int32_t* __restrict__ slot, int32_t* __restrict__ slot_token,
                               float* __restrict__ slot_w, unsigned long long* counters) {
     extern __shared__ int run[];
@@ -246,6 +246,19 @@ __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __re
         }
         affected += rej > 0;
         skipped += (req > 0 && rej == req);
+        if (renorm_rejected && rej > 0 && rej < req) {
+            // the token's accepted paths share its weight: rescale them to sum to one
+            float sum = 0.f;
+            for (int j = 0; j < k; ++j)
+                if (slot[t * k + j] >= 0) sum += w[t * k + j];
+            for (int j = 0; j < k; ++j) {
+                const int sg = slot[t * k + j];
+                if (sg < 0) continue;
+                const int e = ids[t * k + j];
+                const int64_t local = rank_base ? (int64_t)sg - rank_base[e] : (int64_t)sg;
+                slot_w[(int64_t)offsets[e] + local] = w[t * k + j] / sum;
+            }
+        }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
@@ -330,7 +343,8 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     *where = "assign";
     assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
-                                                         n_tiles, sc.hist, offsets, nullptr, slot,
+                                                         n_tiles, sc.hist, offsets, nullptr,
+                                                         p.reject_policy == MOE_REJECT_RENORM, slot,
                                                          slot_token, slot_w, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (x && x_perm) {
@@ -374,6 +388,7 @@ cudaError_t launch_dispatch_ranked(const moe_params& p, int64_t C, int bm, const
     *where = "assign";
     assign_kernel<<<sc.n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
                                                             sc.n_tiles, sc.hist, offsets, sc.base,
+                                                            p.reject_policy == MOE_REJECT_RENORM,
                                                             slot, slot_token, slot_w, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (x && x_perm) {

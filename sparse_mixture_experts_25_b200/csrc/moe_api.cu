@@ -125,6 +125,8 @@ moe_status check_params(const moe_params* p) {
     if (p->norm < MOE_NORM_RENORM || p->norm > MOE_NORM_WLR) return MOE_ERR_INVALID_ARG;
     if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (p->d_f_shared < 0) return MOE_ERR_INVALID_ARG;
+    if (p->reject_policy != MOE_REJECT_ZERO && p->reject_policy != MOE_REJECT_RENORM)
+        return MOE_ERR_INVALID_ARG;
     if (!(p->c == p->c) || p->c > 1e6) return MOE_ERR_INVALID_ARG;
     if (p->norm == MOE_NORM_WLR && !(p->theta >= 0.f && p->theta < 1.f)) return MOE_ERR_INVALID_ARG;
     if (p->E_r > kMaxExperts || p->k > kMaxK) return MOE_ERR_UNSUPPORTED;

@@ -44,7 +44,7 @@ def to_dev(a):
 def params_of(w: si.Workload):
     import sparse_mixture_experts_25_b200 as moe
     return moe.params(w.N, w.d, w.d_f, w.E, w.k, c=w.c, norm=w.norm, theta=w.theta,
-                      dtype=w.dtype, d_f_shared=w.d_f_shared)
+                      dtype=w.dtype, d_f_shared=w.d_f_shared, reject_policy=w.reject_policy)
 
 
 def gpu_forward(w: si.Workload, inp: dict, dev: dict | None = None):
@@ -95,7 +95,11 @@ def check_dispatch(w: si.Workload, rec: dict, stats: dict):
     t_idx, j_idx = np.nonzero(d["slot"] >= 0)
     pos = offs[rec["ids"][t_idx, j_idx]] + d["slot"][t_idx, j_idx]
     np.testing.assert_array_equal(rec["slot_token"][pos], t_idx)
-    np.testing.assert_array_equal(rec["slot_w"][pos], rec["w"][t_idx, j_idx])
+    wc = oracle.reject_weights(rec["ids"], rec["w"].astype(np.float64), rec["slot"], w.reject_policy)
+    if w.reject_policy == 0:
+        np.testing.assert_array_equal(rec["slot_w"][pos], rec["w"][t_idx, j_idx])
+    else:
+        np.testing.assert_allclose(rec["slot_w"][pos], wc[t_idx, j_idx], rtol=1e-6, atol=1e-7)
     s = d["stats"]
     for key in ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max"):
         assert stats[key] == s[key], (key, stats[key], s[key])
@@ -117,7 +121,8 @@ def check_rows(w: si.Workload, inp: dict, rec: dict, Y: np.ndarray, tokens=None)
     if tokens is None:
         tokens = np.arange(w.N)
     Ws = (inp.get("Ws_g"), inp.get("Ws_u"), inp.get("Ws_d")) if w.d_f_shared else None
-    ref = oracle.forward_rows(inp["x"], rec["ids"], rec["w"].astype(np.float64), rec["slot"], tokens,
+    wc = oracle.reject_weights(rec["ids"], rec["w"].astype(np.float64), rec["slot"], w.reject_policy)
+    ref = oracle.forward_rows(inp["x"], rec["ids"], wc, rec["slot"], tokens,
                               inp["W_g"], inp["W_u"], inp["W_d"], Ws=Ws)
     err = rel_err(Y[tokens], ref)
     assert err <= TOL[w.dtype], f"max-abs-rel error {err:.3e} above {TOL[w.dtype]:.0e}"

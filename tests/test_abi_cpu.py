@@ -21,7 +21,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_struct_sizes_match_the_header_layout():
-    assert ctypes.sizeof(moe.Params) == 48
+    assert ctypes.sizeof(moe.Params) == 56
     assert ctypes.sizeof(moe.Stats) == 13 * 8 + 2 * 8 + 2 * 4
     assert ctypes.sizeof(moe.WsLayout) == 15 * 8
 
@@ -68,6 +68,7 @@ def test_workspace_layout_regions():
     (dict(d_f=36), moe.MOE_ERR_UNSUPPORTED),
     (dict(E_r=2000, k=2), moe.MOE_ERR_UNSUPPORTED),
     (dict(c=float("nan")), moe.MOE_ERR_INVALID_ARG),
+    (dict(reject_policy=2), moe.MOE_ERR_INVALID_ARG),
 ])
 def test_invalid_params_are_rejected_on_the_host(kw, status):
     base = dict(N=16, d=64, d_f=64, E_r=8, k=2)

@@ -57,6 +57,11 @@ SMALL = {
                                                  d_f_shared=128),
     "pair_capped_bf16": W["mixtral_bf16"].scaled("pair_capped_bf16", N=2000, d=128, d_f=256, E=2, k=1,
                                                  c=0.9),
+    # overflow policy: a token that loses a path renormalises its accepted ones
+    "renorm_reject_bf16": W["qwen3_skew_bf16"].scaled("renorm_reject_bf16", N=1024, d=256, d_f=192,
+                                                     E=32, k=4, reject_policy=1),
+    "renorm_reject_f32": W["switch_top1_f32"].scaled("renorm_reject_f32", N=700, d=64, d_f=96, k=2,
+                                                    norm=si.NORM_RENORM, c=0.8, reject_policy=1),
 }
 
 
@@ -71,7 +76,7 @@ def _end_to_end(w):
         # routing identical: compare against the oracle's whole forward as well
         full = oracle.forward(inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], k=w.k,
                               norm=w.norm, c=w.c, theta=w.theta, b_r=inp.get("b_r"),
-                              lat=inp.get("lat"),
+                              lat=inp.get("lat"), reject_policy=w.reject_policy,
                               Ws=(inp.get("Ws_g"), inp.get("Ws_u"), inp.get("Ws_d")) if w.d_f_shared else None)
         assert parity.rel_err(out["Y"], full["Y"]) <= parity.TOL[w.dtype]
     assert out["status"] == moe.MOE_OK
@@ -199,6 +204,12 @@ def test_n4_example_capacity_and_statistics():
     moe.moe_combine(p, torch.from_numpy(H).cuda(), r["offsets"], r["st"], r["sw"], Y)
     y = Y.cpu().numpy()
     np.testing.assert_allclose(np.diag(y[:, :4]), [11 / 9, 4 / 3, 25 / 18, 7 / 3], atol=1e-5)
+    # renormalising the remaining path instead: expert 3's weight becomes one, y_4 = 3 x_4
+    p1 = moe.params(4, 8, 8, 3, 2, c=1.0, dtype=moe.MOE_F32, reject_policy=moe.MOE_REJECT_RENORM)
+    r1 = _route_dispatch(p1, x, W_r, C)
+    Y1 = torch.zeros(4, 8, device="cuda")
+    moe.moe_combine(p1, torch.from_numpy(H).cuda(), r1["offsets"], r1["st"], r1["sw"], Y1)
+    np.testing.assert_allclose(np.diag(Y1.cpu().numpy()[:, :4]), [11 / 9, 4 / 3, 25 / 18, 3.0], atol=1e-5)
 
 
 # ---------------------------------------------------------------------------

@@ -123,6 +123,12 @@ def test_n4_example_capacity_and_statistics():
     assert abs(Y[3, 3] - _frac(g["token4_output_coefficient_zero_reject"])) < 1e-6
     for t in range(3):
         assert abs(Y[t, t] - _frac(g["uncapped_output_coefficients"][t])) < 1e-6
+    # the other overflow policy the page works out: renormalise the remaining path
+    wc = oracle.reject_weights(r["ids"], r["w"], d["slot"], policy=1)
+    Y1 = oracle.combine(r["ids"], wc, d["slot"], H, d=4)
+    assert abs(Y1[3, 3] - _frac(g["token4_output_coefficient_renormalised_reject"])) < 1e-6
+    for t in range(3):
+        assert abs(Y1[t, t] - _frac(g["uncapped_output_coefficients"][t])) < 1e-6
 
 
 def test_capacity_printed_examples():
@@ -429,3 +435,26 @@ def test_parameter_counts():
     Pe, tot, act = oracle.param_counts(1024, 4096, 8, 2)
     assert (Pe, tot, act) == (12_582_912, 100_663_296, 25_165_824)
     assert tot * 2 == 201_326_592 and tot * 2 // 2 ** 20 == 192 and act * 2 // 2 ** 20 == 48
+
+
+@pytest.mark.parametrize("norm", [oracle.NORM_RENORM, oracle.NORM_FULLPROB])
+def test_renormalising_reject_policy_invariants(norm):
+    rng = np.random.default_rng(8)
+    N, d, E, k = 300, 8, 6, 3
+    x = rng.standard_normal((N, d)).astype(np.float32)
+    W_r = rng.standard_normal((E, d)).astype(np.float32)
+    r = oracle.route(x, W_r, k=k, norm=norm)
+    dsp = oracle.dispatch(r["ids"], E=E, C=oracle.capacity(0.7, N, k, E))
+    w0 = oracle.reject_weights(r["ids"], r["w"], dsp["slot"], policy=0)
+    w1 = oracle.reject_weights(r["ids"], r["w"], dsp["slot"], policy=1)
+    acc = dsp["slot"] >= 0
+    np.testing.assert_array_equal(w0, np.where(acc, r["w"], 0.0))
+    nacc = acc.sum(axis=1)
+    lost = (nacc < k) & (nacc > 0)
+    assert lost.any()
+    np.testing.assert_allclose(w1[lost].sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    # within a token, the accepted weights keep their ratios
+    t = int(np.nonzero(lost & (nacc >= 2))[0][0])
+    j = np.nonzero(acc[t])[0]
+    assert abs(w1[t, j[0]] / w1[t, j[1]] - r["w"][t, j[0]] / r["w"][t, j[1]]) < 1e-12
+    np.testing.assert_array_equal(w1[~lost], w0[~lost])
