@@ -54,6 +54,8 @@ constexpr int STAGE_BYTES = A_BYTES + 2 * B_HALF_BYTES;
 constexpr int STAGES_PAIR = 6;                            // CTA pair: A + one B half per CTA
 constexpr int STAGE_BYTES_PAIR = A_BYTES + B_HALF_BYTES;
 constexpr int NUM_THREADS = 192;
+constexpr int kStgLd = 36;  // floats per staging row (32 + 4: conflict-free 16-byte access)
+constexpr size_t kStgBytes = 4 * 32 * kStgLd * sizeof(float) + 128;  // + alignment slack
 constexpr int TMEM_COLS = 512;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
@@ -236,6 +238,12 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 // M = 256 across the pair (128 A rows in each CTA), N = 256 (128 B rows in each).
 constexpr uint32_t kIdescPair = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                 ((uint32_t)(256 >> 4) << 24);
+// M = 128 across the pair (64 A rows in each CTA), N = 256: for tiles of at
+// most 128 rows.  Each CTA's accumulator then holds its 64 rows twice as
+// wide: TMEM lanes 0-63 carry MMA columns 0-127, lanes 64-127 columns
+// 128-255, both at TMEM columns 0-127.
+constexpr uint32_t kIdescPairHalf = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                    ((uint32_t)(128 >> 4) << 24);
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -280,12 +288,12 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 }
 
 __device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                               uint32_t accumulate) {
+                                               uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(kIdescPair), "r"(accumulate)
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -402,24 +410,28 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Epilogue of one accumulator for the 128 rows this CTA owns (thread = row r
-// of the CTA's slice, which starts at global row `row0`; `rows` valid).
+// Epilogue of one accumulator segment.  The calling thread owns one output
+// row (`row_ok`, global row `grow`) in TMEM lane `t_row`'s quarter; the
+// segment spans TMEM columns [cb, cb + width) of that lane, which hold the
+// output columns starting at `ob`.
+//   SwiGLU: the gate value of output column ob + c sits at TMEM column
+//           cb + c and the up value at cb + up_off + c (c < width).
+//   fp32:   TMEM column cb + c is output column ob + c.
 template <int EPI>
-__device__ __forceinline__ void epilogue_tile(const TcArgs& a, const Tile& ti, uint32_t t_row, int r,
-                                              int row0, int rows) {
-    const bool row_ok = r < rows;
-    const int grow = row0 + r;
+__device__ __forceinline__ void epilogue_segment(const TcArgs& a, const Tile& ti, uint32_t t_row,
+                                                 int lane, bool row_ok, int grow, int cb, int ob,
+                                                 int width, int up_off, float* stg) {
+    const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
     if (EPI == EPI_SWIGLU) {
-        const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
         const int ld = ti.shared ? a.ld_out_sh : a.ld_out;
         __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(ti.shared ? a.out_sh : a.out);
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
+        for (int c = 0; c < width; c += 32) {
             uint32_t g[32], u[32];
-            tmem_ld32(t_row + (uint32_t)c, g);
-            tmem_ld32(t_row + 128u + (uint32_t)c, u);
+            tmem_ld32(t_row + (uint32_t)(cb + c), g);
+            tmem_ld32(t_row + (uint32_t)(cb + up_off + c), u);
             tmem_ld_wait();
-            const int col0 = ti.n_tile * 128 + c;
+            const int col0 = ob + c;
             if (row_ok) {
                 uint4* dst = reinterpret_cast<uint4*>(outp + (int64_t)grow * ld + col0);
 #pragma unroll
@@ -440,9 +452,13 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, const Tile& ti, u
             }
         }
     } else {
-        const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
+        // fp32 rows (combine into Y, or plain stores): each 32-column chunk is
+        // transposed through this warp's staging tile so that one warp
+        // instruction covers 4 rows x 128 contiguous bytes (8 lanes per row)
+        // instead of 32 rows x 16 bytes
         float wgt = 1.f;
-        float* dst_row = nullptr;
+        long long dst_off = -1;  // element offset of this row in the destination, -1: none
+        float* dst_base = EPI == EPI_COMBINE ? a.Y : static_cast<float*>(a.out);
         if (row_ok) {
             if (EPI == EPI_COMBINE) {
                 int tok;
@@ -452,35 +468,37 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& a, const Tile& ti, u
                     tok = a.slot_token[grow];
                     wgt = a.slot_w[grow];
                 }
-                if (tok < 0 || tok >= a.n_tokens) tok = -1;
-                dst_row = tok >= 0 ? a.Y + (int64_t)tok * a.ldY : nullptr;
+                if (tok >= 0 && tok < a.n_tokens) dst_off = (long long)tok * a.ldY;
             } else {
-                dst_row = static_cast<float*>(a.out) + (int64_t)grow * a.ld_out;
+                dst_off = (long long)grow * a.ld_out;
             }
         }
+        const bool reduce = EPI == EPI_COMBINE || a.ks > 1;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = 0; c < width; c += 32) {
             uint32_t v[32];
-            tmem_ld32(t_row + (uint32_t)c, v);
+            tmem_ld32(t_row + (uint32_t)(cb + c), v);
             tmem_ld_wait();
-            const int col0 = ti.n_tile * BN + c;
-            if (row_ok && dst_row) {
+            float4* my = reinterpret_cast<float4*>(stg + lane * kStgLd);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    if (col0 + q * 4 < n_valid) {
-                        float* p = dst_row + col0 + q * 4;
-                        const float x0 = __uint_as_float(v[q * 4 + 0]) * wgt;
-                        const float x1 = __uint_as_float(v[q * 4 + 1]) * wgt;
-                        const float x2 = __uint_as_float(v[q * 4 + 2]) * wgt;
-                        const float x3 = __uint_as_float(v[q * 4 + 3]) * wgt;
-                        if (EPI == EPI_COMBINE || a.ks > 1) {
-                            red_add_v4(p, x0, x1, x2, x3);
-                        } else {
-                            *reinterpret_cast<float4*>(p) = make_float4(x0, x1, x2, x3);
-                        }
-                    }
+            for (int q = 0; q < 8; ++q)
+                my[q] = make_float4(__uint_as_float(v[4 * q]) * wgt, __uint_as_float(v[4 * q + 1]) * wgt,
+                                    __uint_as_float(v[4 * q + 2]) * wgt, __uint_as_float(v[4 * q + 3]) * wgt);
+            __syncwarp();
+            const int col0 = ob + c;
+            const int cg = (lane & 7) * 4;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int rr = i * 4 + (lane >> 3);
+                const long long off = __shfl_sync(0xffffffffu, dst_off, rr);
+                if (off >= 0 && col0 + cg < n_valid) {
+                    const float4 val = *reinterpret_cast<const float4*>(stg + rr * kStgLd + cg);
+                    float* p = dst_base + off + col0 + cg;
+                    if (reduce) red_add_v4(p, val.x, val.y, val.z, val.w);
+                    else *reinterpret_cast<float4*>(p) = val;
                 }
             }
+            __syncwarp();
         }
     }
 }
@@ -500,7 +518,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       const __grid_constant__ CUtensorMap mB1,
                       const __grid_constant__ CUtensorMap mA_sh,
                       const __grid_constant__ CUtensorMap mB0_sh,
-                      const __grid_constant__ CUtensorMap mB1_sh, const TcArgs a) {
+                      const __grid_constant__ CUtensorMap mB1_sh,
+                      const __grid_constant__ CUtensorMap mA_h,
+                      const __grid_constant__ CUtensorMap mA_sh_h, const TcArgs a) {
     constexpr int NST = PAIR ? STAGES_PAIR : STAGES;
     constexpr int SBYTES = PAIR ? STAGE_BYTES_PAIR : STAGE_BYTES;
     constexpr int TM = PAIR ? 256 : 128;
@@ -517,6 +537,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
     SchedSmem* sched = reinterpret_cast<SchedSmem*>(smem + NST * SBYTES + 256);
+    // per-epilogue-warp staging tiles [32 rows][kStgLd floats]
+    float* stg_all = reinterpret_cast<float*>(
+        (reinterpret_cast<uintptr_t>(sched) + sizeof(SchedSmem) + 127) & ~static_cast<uintptr_t>(127));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
@@ -556,6 +579,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_prefetch_desc(&mB0_sh);
             tma_prefetch_desc(&mB1_sh);
         }
+        if (PAIR) {
+            tma_prefetch_desc(&mA_h);
+            if (a.M_sh > 0) tma_prefetch_desc(&mA_sh_h);
+        }
     }
     tc_fence_before();
     if (PAIR) cluster_sync_all();  // the peer's barriers exist before any remote arrival
@@ -577,7 +604,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int t = unit; t < total_tiles && ok; t += n_units) {
                 Tile ti;
                 decode_tile<TM>(t, *sched, a, routed_tiles, ti);
-                const CUtensorMap* pa = ti.shared ? &mA_sh : &mA;
+                // pair tiles of at most 128 rows load 64 A rows per CTA
+                const bool half = PAIR && ti.rows <= 128;
+                const CUtensorMap* pa = ti.shared ? (half ? &mA_sh_h : &mA_sh) : (half ? &mA_h : &mA);
                 const CUtensorMap* pb0 = ti.shared ? &mB0_sh : &mB0;
                 const CUtensorMap* pb1 = ti.shared ? &mB1_sh : &mB1;
                 int b_row0, b_row1;
@@ -588,7 +617,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     b_row0 = (ti.shared ? 0 : ti.g * a.b_rows_r) + ti.n_tile * 256;
                     b_row1 = b_row0 + 128;
                 }
-                const int a_row = ti.a_row + (PAIR ? (int)crank * 128 : 0);
+                const int a_row = ti.a_row + (PAIR ? (int)crank * (half ? 64 : 128) : 0);
+                const uint32_t a_bytes = half ? A_BYTES / 2 : A_BYTES;
                 for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, a.counters)) {
                         ok = false;
@@ -599,10 +629,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (PAIR) {
                         // both CTAs' bytes complete on the leader's full barrier
                         const uint32_t fb = map_shared_rank(smem_u32(&full[stage]), 0);
-                        if (leader) mbar_expect_tx(&full[stage], 2 * SBYTES);
+                        if (leader) mbar_expect_tx(&full[stage], 2 * (a_bytes + B_HALF_BYTES));
                         tma_load_2d_pair(sa, pa, fb, kb * BK, a_row);
-                        if (crank == 0) tma_load_2d_pair(sb, pb0, fb, kb * BK, b_row0);
-                        else tma_load_2d_pair(sb, pb1, fb, kb * BK, b_row1);
+                        if (EPI == EPI_SWIGLU) {
+                            // this CTA's B half: 64 gate rows, then the 64 up
+                            // rows of the same output columns
+                            const int br = b_row0 + (int)crank * 64;
+                            tma_load_2d_pair(sb, pb0, fb, kb * BK, br);
+                            tma_load_2d_pair(sb + B_HALF_BYTES / 2, pb1, fb, kb * BK, br);
+                        } else if (crank == 0) {
+                            tma_load_2d_pair(sb, pb0, fb, kb * BK, b_row0);
+                        } else {
+                            tma_load_2d_pair(sb, pb1, fb, kb * BK, b_row1);
+                        }
                     } else {
                         mbar_expect_tx(&full[stage], SBYTES);
                         tma_load_2d(sa, pa, &full[stage], kb * BK, a_row);
@@ -634,6 +673,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int t = unit; t < total_tiles && ok; t += n_units) {
                 Tile ti;
                 decode_tile<TM>(t, *sched, a, routed_tiles, ti);
+                const uint32_t idesc_pair = ti.rows <= 128 ? kIdescPairHalf : kIdescPair;
                 if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, a.counters)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -651,7 +691,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         // advance 16 elements (32 bytes) along K inside the swizzled row
                         const uint32_t accum = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
-                        if (PAIR) umma_bf16_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), accum);
+                        if (PAIR)
+                            umma_bf16_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc_pair,
+                                           accum);
                         else umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), accum);
                     }
                     if (PAIR) umma_commit_pair_both(&empty[stage]);
@@ -687,6 +729,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
+        float* stg = stg_all + (warp - 2) * 32 * kStgLd;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = unit; t < total_tiles; t += n_units) {
@@ -695,9 +738,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!warp_wait_bounded(&tfull[acc], acc_phase, abort_flag, a.counters)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-            const int row0 = ti.a_row + (PAIR ? (int)crank * 128 : 0);
-            const int rows = PAIR ? max(0, min(128, ti.rows - (int)crank * 128)) : ti.rows;
-            epilogue_tile<EPI>(a, ti, t_row, r, row0, rows);
+            if (!PAIR) {
+                // lane r = row r; gate/up: gate columns 0-127, up 128-255
+                const bool ok = r < ti.rows;
+                if (EPI == EPI_SWIGLU)
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + r, 0, ti.n_tile * 128, 128, 128, stg);
+                else
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + r, 0, ti.n_tile * BN, BN, 0, stg);
+            } else if (ti.rows > 128) {
+                // 256-row tile: lane r = row crank * 128 + r, all 256 columns
+                const int lr = (int)crank * 128 + r;
+                const bool ok = lr < ti.rows;
+                if (EPI == EPI_SWIGLU) {
+                    // each CTA's B half is 64 gate rows then 64 up rows
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 0, ti.n_tile * 128, 64, 64, stg);
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 128, ti.n_tile * 128 + 64, 64,
+                                          64, stg);
+                } else {
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 0, ti.n_tile * BN, BN, 0, stg);
+                }
+            } else {
+                // 128-row tile (64 rows per CTA): lanes 0-63 hold the first
+                // 128 MMA columns of rows 0-63, lanes 64-127 the last 128
+                const int lr = (int)crank * 64 + (quarter & 1) * 32 + lane;
+                const int hf = quarter >> 1;
+                const bool ok = lr < ti.rows;
+                if (EPI == EPI_SWIGLU)
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 0, ti.n_tile * 128 + hf * 64, 64,
+                                          64, stg);
+                else
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 0, ti.n_tile * BN + hf * 128, 128,
+                                          0, stg);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -744,13 +816,13 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// 2-D bf16 row-major matrix [rows, cols] read in boxes of 128 rows x 64 columns
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+// 2-D bf16 row-major matrix [rows, cols] read in boxes of box_rows rows x 64 columns
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows = 128) {
     auto enc = get_encode();
     if (!enc || rows == 0 || cols == 0) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {BK, 128};
+    cuuint32_t box[2] = {BK, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -758,21 +830,29 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
     return r == CUDA_SUCCESS;
 }
 
-constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + sizeof(SchedSmem);
-constexpr size_t kSmemBytesPair = 1024 + (size_t)STAGES_PAIR * STAGE_BYTES_PAIR + 256 + sizeof(SchedSmem);
+// the fp32 epilogues stage through shared memory; the SwiGLU epilogue does not
+constexpr size_t smem_bytes(int epi, bool pair) {
+    return 1024 + (pair ? (size_t)STAGES_PAIR * STAGE_BYTES_PAIR : (size_t)STAGES * STAGE_BYTES) + 256 +
+           sizeof(SchedSmem) + (epi == EPI_SWIGLU ? 0 : kStgBytes);
+}
+static_assert(smem_bytes(EPI_COMBINE, false) <= 232448 && smem_bytes(EPI_COMBINE, true) <= 232448,
+              "shared memory per CTA");
 
+// mA_h / mA_sh_h: the A matrices again in 64-row boxes (CTA-pair tiles of at
+// most 128 rows); unused by single-CTA launches.
 template <int EPI, bool PAIR>
 cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mB0, const CUtensorMap& mB1,
                       const CUtensorMap& mA_sh, const CUtensorMap& mB0_sh, const CUtensorMap& mB1_sh,
-                      const TcArgs& a, int64_t max_tiles, cudaStream_t st) {
+                      const CUtensorMap& mA_h, const CUtensorMap& mA_sh_h, const TcArgs& a,
+                      int64_t max_tiles, cudaStream_t st) {
     auto kern = tc_grouped_kernel<EPI, PAIR>;
-    const size_t smem = PAIR ? kSmemBytesPair : kSmemBytes;
+    const size_t smem = smem_bytes(EPI, PAIR);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (!PAIR) {
         const int grid = (int)min64(max_tiles, num_sms());
         if (grid <= 0) return cudaSuccess;
-        kern<<<grid, NUM_THREADS, smem, st>>>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a);
+        kern<<<grid, NUM_THREADS, smem, st>>>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, a);
         return cudaGetLastError();
     }
     // clusters of two CTAs, one tile per cluster at a time
@@ -790,7 +870,7 @@ cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mB0, const CUten
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a);
+    e = cudaLaunchKernelEx(&cfg, kern, mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -844,18 +924,23 @@ cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const voi
                               const ExpertWeights& W, void* h, void* h_shared, float* Y_zero,
                               unsigned long long* counters, cudaStream_t st, int* status) {
     *status = MOE_OK;
-    CUtensorMap mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh;
+    CUtensorMap mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h;
+    const bool pair = tc_tile_rows(p) == 256;
+    // CTA pairs: each CTA loads 64 gate rows and 64 up rows per 128 columns
+    const uint32_t b_box = pair ? 64 : 128;
     const uint64_t rows = (uint64_t)(p.N * p.k);
-    bool ok = make_map(&mA, x_perm, rows, p.d) &&
-              make_map(&mB0, W.W_g, (uint64_t)p.E_r * p.d_f, p.d) &&
-              make_map(&mB1, W.W_u, (uint64_t)p.E_r * p.d_f, p.d);
+    bool ok = make_map(&mA, x_perm, rows, p.d) && make_map(&mA_h, x_perm, rows, p.d, 64) &&
+              make_map(&mB0, W.W_g, (uint64_t)p.E_r * p.d_f, p.d, b_box) &&
+              make_map(&mB1, W.W_u, (uint64_t)p.E_r * p.d_f, p.d, b_box);
     const bool sh = p.d_f_shared > 0;
     if (ok && sh) {
         ok = make_map(&mA_sh, x_shared, (uint64_t)p.N, p.d) &&
-             make_map(&mB0_sh, W.Ws_g, (uint64_t)p.d_f_shared, p.d) &&
-             make_map(&mB1_sh, W.Ws_u, (uint64_t)p.d_f_shared, p.d);
+             make_map(&mA_sh_h, x_shared, (uint64_t)p.N, p.d, 64) &&
+             make_map(&mB0_sh, W.Ws_g, (uint64_t)p.d_f_shared, p.d, b_box) &&
+             make_map(&mB1_sh, W.Ws_u, (uint64_t)p.d_f_shared, p.d, b_box);
     } else {
         mA_sh = mA;
+        mA_sh_h = mA_h;
         mB0_sh = mB0;
         mB1_sh = mB1;
     }
@@ -886,14 +971,15 @@ cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const voi
     a.zero_ptr = Y_zero;
     a.zero_n4 = Y_zero ? p.N * (int64_t)p.d / 4 : 0;
     a.counters = counters;
-    const bool pair = tc_tile_rows(p) == 256;
     const int tm = pair ? 256 : 128;
     int64_t max_tiles =
         routed_mtile_bound(p, tm) * a.nt_r + (sh ? ((p.N + tm - 1) / tm) * a.nt_sh : 0);
     const int units = pair ? num_sms() / 2 : num_sms();
     if (Y_zero && max_tiles < units) max_tiles = units;  // every CTA zeroes a share
-    if (pair) return launch_tc<EPI_SWIGLU, true>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a, max_tiles, st);
-    return launch_tc<EPI_SWIGLU, false>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, a, max_tiles, st);
+    if (pair)
+        return launch_tc<EPI_SWIGLU, true>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, a, max_tiles,
+                                           st);
+    return launch_tc<EPI_SWIGLU, false>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, a, max_tiles, st);
 }
 
 cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void* h,
@@ -902,15 +988,18 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
                            const float* slot_w, float* Y, float* H_out,
                            unsigned long long* counters, cudaStream_t st, int* status) {
     *status = MOE_OK;
-    CUtensorMap mA, mB0, mA_sh, mB0_sh;
+    CUtensorMap mA, mB0, mA_sh, mB0_sh, mA_h, mA_sh_h;
     const uint64_t rows = (uint64_t)(p.N * p.k);
-    bool ok = make_map(&mA, h, rows, p.d_f) && make_map(&mB0, W.W_d, (uint64_t)p.E_r * p.d, p.d_f);
+    bool ok = make_map(&mA, h, rows, p.d_f) && make_map(&mA_h, h, rows, p.d_f, 64) &&
+              make_map(&mB0, W.W_d, (uint64_t)p.E_r * p.d, p.d_f);
     const bool sh = p.d_f_shared > 0 && mode == DOWN_COMBINE;
     if (ok && sh) {
         ok = make_map(&mA_sh, h_shared, (uint64_t)p.N, p.d_f_shared) &&
+             make_map(&mA_sh_h, h_shared, (uint64_t)p.N, p.d_f_shared, 64) &&
              make_map(&mB0_sh, W.Ws_d, (uint64_t)p.d, p.d_f_shared);
     } else {
         mA_sh = mA;
+        mA_sh_h = mA_h;
         mB0_sh = mB0;
     }
     if (!ok) {
@@ -952,11 +1041,15 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
     int64_t max_tiles =
         (routed_mtile_bound(p, tm) * a.nt_r + (sh ? ((p.N + tm - 1) / tm) * a.nt_sh : 0)) * a.ks;
     if (mode == DOWN_COMBINE) {
-        if (pair) return launch_tc<EPI_COMBINE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
-        return launch_tc<EPI_COMBINE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
+        if (pair)
+            return launch_tc<EPI_COMBINE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles,
+                                                st);
+        return launch_tc<EPI_COMBINE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles,
+                                             st);
     }
-    if (pair) return launch_tc<EPI_STORE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
-    return launch_tc<EPI_STORE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, a, max_tiles, st);
+    if (pair)
+        return launch_tc<EPI_STORE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles, st);
+    return launch_tc<EPI_STORE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles, st);
 }
 
 cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,
@@ -985,7 +1078,7 @@ cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r
         cudaError_t e = cudaMemsetAsync(logits, 0, sizeof(float) * (size_t)p.N * p.E_r, st);
         if (e != cudaSuccess) return e;
     }
-    return launch_tc<EPI_STORE, false>(mA, mB, mB, mA, mB, mB, a, tiles * a.ks, st);
+    return launch_tc<EPI_STORE, false>(mA, mB, mB, mA, mB, mB, mA, mA, a, tiles * a.ks, st);
 }
 
 }  // namespace moe
