@@ -19,11 +19,21 @@
 //              epilogue.
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator rows (one TMEM lane
 //              per row), then SwiGLU -> bf16 h (gate/up) or the weighted
-//              scatter-combine with 16-byte fp32 red.global.add (down).
+//              scatter-combine with 16-byte fp32 red.global.add (down), each
+//              32-column chunk transposed through a per-warp shared-memory
+//              tile so one warp instruction adds 4 rows x 128 contiguous bytes.
 // For gate/up the two B tiles are the gate and up rows of the same 128
 // output columns, so one N=256 MMA yields both and the SwiGLU is local to a
 // thread.  For the down projection they are two consecutive 128-row halves
 // of a 256-column output tile.
+//
+// Layers with many rows per expert run on CTA pairs instead (cluster of 2,
+// cta_group::2 MMAs issued by the leader): a 256 x 256 tile, each CTA loading
+// its 128 A rows and half of B (6 stages of 32 KB), so each SM reads half the
+// B bytes per MMA.  A pair tile of at most 128 rows uses the M=128 pair MMA
+// (64 A rows per CTA).  On pairs the gate/up B half of a CTA is 64 gate rows
+// followed by the 64 up rows of the same columns, which keeps gate and up of
+// one output column in one TMEM lane for both tile heights.
 //
 // Tiles are scheduled statically (tile = blockIdx.x + i * gridDim.x) over a
 // list ordered group by group, output-column tile by column tile, with the
