@@ -89,6 +89,23 @@ def step_flops(w: si.Workload, accepted: int) -> float:
     return f
 
 
+def gate_up_bytes(w: si.Workload, accepted: int, experts_touched: int) -> float:
+    """Algorithmic HBM bytes of the gate/up launch: W_g and W_u of every
+    expert with an accepted row, the gathered rows (A d) read and h (A d_f)
+    written, Y zeroed (N d fp32); the shared expert adds its two matrices, x
+    and h_shared."""
+    s = 2 if w.dtype == si.DT_BF16 else 4
+    b = experts_touched * 2.0 * w.d_f * w.d * s + accepted * (w.d + w.d_f) * s + w.N * w.d * 4.0
+    if w.d_f_shared:
+        b += 2.0 * w.d_f_shared * w.d * s + w.N * (w.d + w.d_f_shared) * s
+    return b
+
+
+# fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 FLOP (FFMA) x the maximum SM clock
+def ffma_peak_tflops(sm_mhz: float) -> float:
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
 def load_peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -222,6 +239,22 @@ def run_reference(args):
     return 0
 
 
+L2_BYTES = 126 * 2**20
+
+
+def input_bytes(w: si.Workload) -> int:
+    """Bytes of the layer's inputs read every step: expert and router weights and x."""
+    s = 2 if w.dtype == si.DT_BF16 else 4
+    b = w.E * 3 * w.d * w.d_f * s + w.E * w.d * s + w.N * w.d * s
+    if w.d_f_shared:
+        b += 3 * w.d * w.d_f_shared * s
+    return b
+
+
+def flushes_l2(w: si.Workload) -> bool:
+    return input_bytes(w) < 2 * L2_BYTES
+
+
 def config_of(w: si.Workload, args):
     return {"workload": f"{w.name}: T={w.N} d={w.d} d_f={w.d_f} E_r={w.E} k={w.k}",
             "T": w.N, "d": w.d, "d_f": w.d_f, "E_r": w.E, "k": w.k,
@@ -230,7 +263,9 @@ def config_of(w: si.Workload, args):
             "parallelism": (f"dp{args.gpus}: one routing group of {w.N} x {args.gpus} tokens, "
                             "per-expert request counts all-gathered once per step"
                             if args.gpus > 1 else "dp1"),
-            "l2": "inputs larger than L2 (expert weights 2.8 GB stream from HBM every step)"}
+            "l2": (f"L2 flushed between timed steps (256 MiB write outside the per-step events); "
+                   f"inputs {input_bytes(w) / 2**20:.1f} MiB" if flushes_l2(w) else
+                   f"inputs larger than L2 ({input_bytes(w) / 1e9:.2f} GB of weights and x read every step)")}
 
 
 # ---------------------------------------------------------------------------
@@ -305,10 +340,13 @@ def run_gpu(args):
     if ws_n > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    flush = torch.empty(256 * 2**20 // 4, dtype=torch.int32, device="cuda") if flushes_l2(w) else None
     with ClockSampler(local) as clk:
         time.sleep(0.3)
         start.record(stream)
         for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(i)   # evict the layer's inputs from L2; outside the step's events
             moe.moe_set_stage_events(ev[i])
             step(d["x"], Y)
         moe.moe_set_stage_events([])
@@ -317,7 +355,10 @@ def run_gpu(args):
         time.sleep(0.2)
     if ws_n > 1:
         dist.barrier()
-    ms_total = start.elapsed_time(end)
+    if flush is None:
+        ms_total = start.elapsed_time(end)
+    else:  # sum of the steps' own spans (first stage event to last)
+        ms_total = float(sum(ev[i][0].elapsed_time(ev[i][4]) for i in range(args.steps)))
     ms_total = max_over_ranks(ms_total, device="cuda")
     ms_step = ms_total / args.steps
     stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(4)] for i in range(args.steps)])
@@ -362,6 +403,34 @@ def run_gpu(args):
         peak_tf, peak_kind = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), "sustained"
     gu_flops = gate_up_flops(w, accepted)
     achieved = gu_flops / (gate_up_ms * 1e-3) / 1e12
+    touched = int((moe.workspace_views(p, wsb)["acc"] > 0).sum().item())
+    gu_bytes = gate_up_bytes(w, accepted, touched)
+    if w.dtype != si.DT_BF16:
+        # fp32 layers run the FFMA kernels: bound by CUDA-core arithmetic
+        peak_ffma = ffma_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
+        roof = {"kernel": "simt_grouped_kernel<SWIGLU> (gate/up GEMM + SwiGLU, fp32 FFMA)",
+                "bound": "alu", "achieved": achieved, "peak": peak_ffma, "unit": "TFLOP/s",
+                "frac": achieved / peak_ffma, "traffic": None,
+                "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock"}
+    elif gu_bytes / (peaks["hbm_gbs"] * 1e9) > gu_flops / (peak_tf * 1e12):
+        # streaming the touched weights takes longer than the MMAs: HBM-bound
+        gbs = gu_bytes / (gate_up_ms * 1e-3) / 1e9
+        roof = {"kernel": "tc_grouped_kernel<SWIGLU> (gate/up GEMM + SwiGLU)",
+                "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"],
+                "traffic": committed_traffic("gate_up") if w.name == "mixtral_bf16" else None,
+                "peak_source": f"{peak_src} HBM copy"}
+    else:
+        roof = {"kernel": "tc_grouped_kernel<SWIGLU> (gate/up GEMM + SwiGLU)",
+                "bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved / peak_tf,
+                "traffic": committed_traffic("gate_up") if w.name == "mixtral_bf16" else None,
+                "peak_source": f"{peak_src} bf16 {peak_kind}"}
+    gu_gbs = gu_bytes / (gate_up_ms * 1e-3) / 1e9
+    roof.update({"flops_per_launch": gu_flops, "bytes_per_launch": gu_bytes, "avg_launch_ms": gate_up_ms,
+                 "tflops": achieved, "gbs": gu_gbs, "hbm_frac": gu_gbs / peaks["hbm_gbs"]})
+    if w.dtype == si.DT_BF16:
+        roof["tensor_frac"] = achieved / peak_tf
     line = {
         "metric": METRIC,
         "value": ws_n * w.N / (ms_step * 1e-3),
@@ -376,13 +445,7 @@ def run_gpu(args):
         "dtype": "bf16" if w.dtype == si.DT_BF16 else "f32",
         "data": "synthetic (seeded SplitMix64/Box-Muller; x~N(0,1), W~N(0,1/fan_in)); no dataset or checkpoint",
         "config": config_of(w, args),
-        "roofline": {
-            "kernel": "tc_grouped_kernel<SWIGLU> (gate/up GEMM + SwiGLU)",
-            "bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
-            "frac": achieved / peak_tf, "traffic": committed_traffic("gate_up"),
-            "peak_source": f"{peak_src} bf16 {peak_kind}",
-            "flops_per_launch": gu_flops, "avg_launch_ms": gate_up_ms,
-        },
+        "roofline": roof,
         "stages_ms": {"route": float(stage_ms[:, 0].mean()), "dispatch": float(stage_ms[:, 1].mean()),
                       "gate_up": gate_up_ms, "down_combine": down_ms},
         "step_tflops": step_flops(w, accepted) / (ms_step * 1e-3) / 1e12,
@@ -392,7 +455,8 @@ def run_gpu(args):
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
                 "ms_per_step": e_ms,
                 "how": "pinned x upload, moe_forward, pinned Y download per step; copies of "
-                       "neighbouring steps overlap compute (HostPipeline, 2 device buffers)"},
+                       "neighbouring steps overlap compute (HostPipeline, 2 device buffers)"
+                       + ("; L2 not flushed between these steps" if flush is not None else "")},
         "gpu_launches": kernels_per_step(w, sharded_group) * args.steps,
         "clocks": clk.summary(),
         "routing": {k: stats[k] for k in ("accepted", "rejected", "near_tie", "L_max", "rho_max")},

@@ -302,7 +302,8 @@ MOE_API moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats*
 /*
  * Optional stage timing for moe_forward on the calling host thread: with
  * n >= 5 events (cudaEvent_t handles created by the caller), the next
- * moe_forward calls record events[0] before the router, [1] after routing,
+ * moe_forward calls record events[0] at the start of the call's device work
+ * (before the statistics counters are reset), [1] after routing,
  * [2] after dispatch, [3] after the gate/up expert GEMM and [4] after the
  * down-projection + combine, on the call's stream (moe_forward_begin records
  * [0] and [1], moe_forward_end [2] to [4]).  n = 0 turns it off.

@@ -11,7 +11,7 @@
 //   hist   one CTA per tile of tokens counts its requests per expert
 //          (shared-memory atomics; order does not matter for counts);
 //   scan   one CTA turns the [E][tiles] counts into exclusive per-tile bases
-//          (one warp per expert, warp-wide scans), then scans the accepted
+//          (a warp per expert, each lane a contiguous run of tiles), then scans the accepted
 //          counts min(L_e, C) over experts into row offsets and the M-tile
 //          prefix used by the grouped GEMMs, and writes the statistics;
 //   assign one warp per tile walks its requests in token order, 32 at a
@@ -73,20 +73,43 @@ __global__ void hist_kernel(const int32_t* __restrict__ ids, int64_t N, int k, i
 }
 
 // Per expert (one warp each), the per-tile request counts become exclusive
-// bases in place; sL[e] receives the expert's total.
+// bases in place; sL[e] receives the expert's total.  Each lane owns a
+// contiguous segment of the expert's tiles: it sums the segment (independent
+// loads), one warp scan turns the sums into segment bases, and the lane
+// rewrites its segment as running bases.  A warp takes its experts four at a
+// time so that the loads of all four are in flight together.
 __device__ void tile_scan(int32_t* __restrict__ hist, int n_tiles, int E, int* sL) {
+    constexpr int G = 4;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    for (int e = warp; e < E; e += nw) {
-        int run = 0;
-        int32_t* row = hist + (int64_t)e * n_tiles;
-        for (int b = 0; b < n_tiles; b += 32) {
-            const int i = b + lane;
-            const int v = i < n_tiles ? row[i] : 0;
-            const int inc = warp_incl_scan(v, lane);
-            if (i < n_tiles) row[i] = run + inc - v;
-            run += __shfl_sync(0xffffffffu, inc, 31);
+    const int seg = (n_tiles + 31) / 32;
+    const int i0 = min(n_tiles, lane * seg), i1 = min(n_tiles, i0 + seg);
+    for (int e0 = warp; e0 < E; e0 += G * nw) {
+        int sum[G];
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            sum[j] = 0;
+            const int e = e0 + j * nw;
+            if (e < E) {
+                const int32_t* row = hist + (int64_t)e * n_tiles;
+#pragma unroll 8
+                for (int i = i0; i < i1; ++i) sum[j] += row[i];
+            }
         }
-        if (lane == 0) sL[e] = run;
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            const int e = e0 + j * nw;  // warp-uniform
+            if (e >= E) break;
+            int32_t* row = hist + (int64_t)e * n_tiles;
+            const int inc = warp_incl_scan(sum[j], lane);
+            int run = inc - sum[j];
+#pragma unroll 8
+            for (int i = i0; i < i1; ++i) {
+                const int v = row[i];
+                row[i] = run;
+                run += v;
+            }
+            if (lane == 31) sL[e] = inc;
+        }
     }
 }
 
@@ -336,9 +359,10 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
     hist_kernel<<<n_tiles, 256, sizeof(int) * E, st>>>(ids, p.N, k, E, sc.tile_tokens, n_tiles,
                                                         sc.hist, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int threads = ((E + 31) / 32) * 32 < 64 ? 64 : ((E + 31) / 32) * 32;
+    // 32 warps share the per-expert tile scans; the expert-level scans need
+    // one thread per expert (E <= kMaxExperts = 1024)
     *where = "scan";
-    scan_kernel<<<1, threads, 0, st>>>(sc.hist, n_tiles, E, C, bm, L, acc, offsets, sc.mt_start,
+    scan_kernel<<<1, 1024, 0, st>>>(sc.hist, n_tiles, E, C, bm, L, acc, offsets, sc.mt_start,
                                        counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     *where = "assign";
@@ -367,8 +391,7 @@ cudaError_t launch_count(const moe_params& p, const int32_t* ids, int32_t* L, in
                                                            sc.n_tiles, sc.hist, counters);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int threads = ((E + 31) / 32) * 32 < 64 ? 64 : ((E + 31) / 32) * 32;
-    count_scan_kernel<<<1, threads, 0, st>>>(sc.hist, sc.n_tiles, E, L, counts_out);
+    count_scan_kernel<<<1, 1024, 0, st>>>(sc.hist, sc.n_tiles, E, L, counts_out);
     return cudaGetLastError();
 }
 

@@ -347,7 +347,9 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     WsView v;
     make_view(*p, ws, v);
     (void)cudaGetLastError();  // clear a stale non-sticky error left by earlier unrelated calls
-    cudaError_t e0 = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
+    cudaError_t e0;
+    if (p->N > 0 && (e0 = stage_mark(0, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
+    e0 = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
     if (e0 != cudaSuccess) return fail(e0, "moe_forward memset");
     if (p->N == 0) return MOE_OK;
     if (!x || !W_r || !W_g || !W_u || !W_d || !Y) return MOE_ERR_INVALID_ARG;
@@ -361,7 +363,6 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     const int64_t C = capacity_exact(p->c, p->N, p->k, p->E_r);
     ExpertWeights W{W_g, W_u, W_d, sh ? Ws_g : nullptr, sh ? Ws_u : nullptr, sh ? Ws_d : nullptr};
 
-    if ((e0 = stage_mark(0, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     // bf16 layers zero Y inside the gate/up kernel (hidden behind its first
     // tile); fp32 layers zero it in the router
     const bool bf16 = p->dtype == MOE_BF16;
@@ -410,7 +411,9 @@ moe_status moe_forward_begin(const moe_params* p, const void* x, const void* W_r
     WsView v;
     make_view(*p, ws, v);
     (void)cudaGetLastError();
-    cudaError_t e = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
+    cudaError_t e;
+    if (p->N > 0 && (e = stage_mark(0, st)) != cudaSuccess) return fail(e, "moe_forward_begin stage event");
+    e = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
     if (e != cudaSuccess) return fail(e, "moe_forward_begin memset");
     if (p->N == 0) {
         if (counts) {
@@ -421,7 +424,6 @@ moe_status moe_forward_begin(const moe_params* p, const void* x, const void* W_r
     }
     if (!x || !W_r || !aligned16(x) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
     if (p->norm == MOE_NORM_WLR && !lat) return MOE_ERR_INVALID_ARG;
-    if ((e = stage_mark(0, st)) != cudaSuccess) return fail(e, "moe_forward_begin stage event");
     e = launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, v.ids, v.w, v.margin,
                       v.counters, nullptr, v.scratch.logits, st);
     if (e != cudaSuccess) return fail(e, "moe_forward_begin router");

@@ -131,6 +131,53 @@ def test_n4_example_capacity_and_statistics():
         assert abs(Y1[t, t] - _frac(g["uncapped_output_coefficients"][t])) < 1e-6
 
 
+def _fcfs_slots(ids, E, C):
+    """First-come-first-served in token order, written out: slot = number of
+    earlier requests for the same expert, -1 when that number reaches C."""
+    seen = [0] * E
+    slot = np.full(ids.shape, -1, np.int64)
+    for t in range(ids.shape[0]):
+        for j in range(ids.shape[1]):
+            e = int(ids[t, j])
+            if e < 0:
+                continue
+            if seen[e] < C:
+                slot[t, j] = seen[e]
+            seen[e] += 1
+    return slot
+
+
+def _ranked_slots(ids, E, C, cuts):
+    """The group split at `cuts` into consecutive shards; each shard's base is
+    the request count of the shards before it."""
+    bounds = [0] + list(cuts) + [ids.shape[0]]
+    out, base = [], np.zeros(E, np.int64)
+    for lo, hi in zip(bounds, bounds[1:]):
+        part = ids[lo:hi]
+        out.append(oracle.dispatch_ranked(part, E=E, C=C, base=base)["slot"])
+        req = part[part >= 0]
+        base = base + np.bincount(req, minlength=E)
+    return np.concatenate(out)
+
+
+def test_ranked_dispatch_equals_one_batch_at_every_cut():
+    # the ch. 36.4 example (capacity 3): every split into two ranks
+    g, x, W_r = _n4_setup()
+    r = oracle.route(x, W_r, k=2, norm=oracle.NORM_RENORM)
+    want = _fcfs_slots(r["ids"], 3, g["capacity"])
+    for cut in range(0, 5):
+        np.testing.assert_array_equal(_ranked_slots(r["ids"], 3, g["capacity"], [cut]), want)
+    # random ids with pruned (-1) entries, three ranks, capacity binding
+    rng = np.random.default_rng(7)
+    N, E, k, C = 60, 5, 3, 20
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(N)]).astype(np.int32)
+    ids[rng.random((N, k)) < 0.1] = -1
+    want = _fcfs_slots(ids, E, C)
+    assert (want < 0).sum() > (ids < 0).sum()          # capacity rejects some requests
+    for cuts in ([10, 35], [0, 60], [1, 2], [59, 60]):
+        np.testing.assert_array_equal(_ranked_slots(ids, E, C, cuts), want)
+
+
 def test_capacity_printed_examples():
     for case in _golden("capacity_examples.json")["cases"]:
         assert oracle.capacity(case["c"], case["T"], case["k"], case["E"]) == case["C"], case
