@@ -110,8 +110,12 @@ typedef struct moe_stats {
     int64_t L_max, L_p50, L_p90, L_p99; /* requested load: max, nearest-rank pct  */
     double rho_max;          /* max_e L_e / (N k / E_r)                           */
     double reject_rate;      /* rejected / requested                              */
-    int32_t device_error;    /* nonzero: a bounded device wait timed out          */
+    int32_t device_error;    /* nonzero: a bounded device wait timed out (bit 0)
+                                or a routing id was out of range (bit 1)           */
     int32_t reserved;
+    int64_t padded_rows;     /* rows the routed expert GEMMs compute: each expert's
+                                accepted rows rounded up to the GEMM's row tile    */
+    double padding_ratio;    /* padded_rows / accepted (0 when nothing accepted)  */
 } moe_stats;
 
 /* Byte offsets of the regions inside the workspace (for inspection and
@@ -309,6 +313,21 @@ MOE_API moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats*
  * [0] and [1], moe_forward_end [2] to [4]).  n = 0 turns it off.
  */
 MOE_API moe_status moe_set_stage_events(void* const* events, int n);
+
+/*
+ * Self-test of the library's bounded device waits (no counterpart on the
+ * pages).  Launches one CTA that waits on a shared-memory mbarrier nothing
+ * ever arrives on, with the same bounded-wait routine the tensor-core GEMMs
+ * use but a limit of limit_ns nanoseconds (1e6 .. 5e9) instead of 2 s; on
+ * expiry the routine records the timeout in the counters of `ws` exactly as a
+ * GEMM would, and the CTA returns.  `ws` is a workspace laid out for `p`; its
+ * counters are reset first.  moe_get_stats then returns MOE_ERR_TIMEOUT with
+ * device_error bit 0 set, and the CUDA context stays usable.  Asynchronous on
+ * `stream`.  Errors: MOE_ERR_INVALID_ARG (limit out of range),
+ * MOE_ERR_WORKSPACE (ws missing or misaligned), MOE_ERR_CUDA (launch).
+ */
+MOE_API moe_status moe_selftest_wait_timeout(const moe_params* p, void* ws, int64_t limit_ns,
+                                             moe_stream_t stream);
 
 /* Text of the last CUDA failure seen by an entry point on the calling host
  * thread ("" if none): the failing step and cudaGetErrorString's text. */

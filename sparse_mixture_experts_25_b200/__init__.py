@@ -21,7 +21,8 @@ __all__ = [
     "moe_dispatch_noalloc",
     "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_begin", "moe_forward_end",
     "moe_get_stats",
-    "moe_set_stage_events", "moe_status_string", "moe_last_error", "workspace_views", "HEADER",
+    "moe_set_stage_events", "moe_selftest_wait_timeout", "moe_status_string", "moe_last_error",
+    "workspace_views", "HEADER",
 ]
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_NONFINITE = 0, 1, 2, 3
@@ -54,7 +55,8 @@ class Stats(ctypes.Structure):
         "C", "requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped",
         "nonfinite", "near_tie", "L_max", "L_p50", "L_p90", "L_p99")] + [
         ("rho_max", ctypes.c_double), ("reject_rate", ctypes.c_double),
-        ("device_error", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+        ("device_error", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("padded_rows", ctypes.c_int64), ("padding_ratio", ctypes.c_double)]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_ if n != "reserved"}
@@ -94,6 +96,7 @@ def lib():
         L.moe_forward_end.argtypes = [pp, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
                                       ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(_P), ctypes.c_int]
+        L.moe_selftest_wait_timeout.argtypes = [pp, _P, ctypes.c_int64, _P]
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [ctypes.c_int]
@@ -102,7 +105,7 @@ def lib():
                      "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine",
                      "moe_forward",
                      "moe_get_stats", "moe_set_stage_events", "moe_forward_begin",
-                     "moe_forward_end"):
+                     "moe_forward_end", "moe_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -228,6 +231,13 @@ def moe_get_stats(p, ws, stream=None):
     if status not in (MOE_OK, MOE_ERR_NONFINITE, MOE_ERR_TIMEOUT):
         raise MoEError(status, "moe_get_stats")
     return status, s.as_dict()
+
+
+def moe_selftest_wait_timeout(p, ws, limit_ns: int, stream=None):
+    """Run the bounded-wait self-test into ws's counters (see the header);
+    moe_get_stats afterwards reports MOE_ERR_TIMEOUT."""
+    _check(lib().moe_selftest_wait_timeout(ctypes.byref(p), _ptr(ws), int(limit_ns), _stream(stream)),
+           "moe_selftest_wait_timeout")
 
 
 def moe_set_stage_events(events):

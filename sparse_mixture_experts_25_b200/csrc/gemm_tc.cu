@@ -345,6 +345,18 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Self-test of the bounded wait: one thread waits on a barrier that nothing
+// arrives on; the wait gives up after limit_ns and records DEVERR_TIMEOUT.
+__global__ void wait_selftest_kernel(unsigned long long* counters, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        wait_bounded(&bar, 0u, &abort_flag, counters, limit_ns);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Tile schedule
 // ---------------------------------------------------------------------------
@@ -1089,6 +1101,11 @@ cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r
         if (e != cudaSuccess) return e;
     }
     return launch_tc<EPI_STORE, false>(mA, mB, mB, mA, mB, mB, mA, mA, a, tiles * a.ks, st);
+}
+
+cudaError_t launch_wait_selftest(unsigned long long* counters, unsigned long long limit_ns, cudaStream_t st) {
+    wait_selftest_kernel<<<1, 32, 0, st>>>(counters, limit_ns);
+    return cudaGetLastError();
 }
 
 }  // namespace moe

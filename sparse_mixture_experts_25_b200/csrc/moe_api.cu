@@ -8,6 +8,8 @@
 #include <algorithm>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -111,7 +113,21 @@ moe_status fail(cudaError_t e, const char* where) {
 }
 thread_local int g_stage_event_count = 0;
 
+// Stage boundaries of moe_forward / moe_forward_begin + moe_forward_end:
+// 0 before routing, 1 after routing, 2 after dispatch, 3 after gate/up,
+// 4 after down + combine.  Each boundary records the caller's stage event (if
+// any) and closes / opens an NVTX range named after the stage, so a timeline
+// profiler shows the host-side enqueue of each stage.
+thread_local nvtxRangeId_t g_nvtx_range = 0;
+
 inline cudaError_t stage_mark(int i, cudaStream_t st) {
+    static const char* const kStageNames[4] = {"moe route", "moe dispatch", "moe gate/up + SwiGLU",
+                                               "moe down + combine"};
+    if (g_nvtx_range) {
+        nvtxRangeEnd(g_nvtx_range);
+        g_nvtx_range = 0;
+    }
+    if (i < 4) g_nvtx_range = nvtxRangeStartA(kStageNames[i]);
     if (g_stage_event_count >= 5 && i < g_stage_event_count) return cudaEventRecord(g_stage_events[i], st);
     return cudaSuccess;
 }
@@ -493,6 +509,21 @@ moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32
     return MOE_OK;
 }
 
+moe_status moe_selftest_wait_timeout(const moe_params* p, void* ws, int64_t limit_ns, moe_stream_t stream) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (limit_ns < 1000000 || limit_ns > 5000000000LL) return MOE_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    WsView v;
+    make_view(*p, ws, v);
+    (void)cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
+    if (e == cudaSuccess) e = launch_wait_selftest(v.counters, (unsigned long long)limit_ns, st);
+    if (e != cudaSuccess) return fail(e, "moe_selftest_wait_timeout");
+    return MOE_OK;
+}
+
 moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, moe_stream_t stream) {
     moe_status s = check_params(p);
     if (s != MOE_OK) return s;
@@ -501,11 +532,13 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
     WsView v;
     make_view(*p, const_cast<void*>(ws), v);
     unsigned long long cnt[CNT_COUNT];
-    std::vector<int32_t> L((size_t)p->E_r);
+    std::vector<int32_t> L((size_t)p->E_r), acc((size_t)p->E_r);
     memset(out, 0, sizeof(*out));
     cudaError_t e = cudaMemcpyAsync(cnt, v.counters, sizeof(cnt), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(L.data(), v.L, sizeof(int32_t) * L.size(), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(acc.data(), v.acc, sizeof(int32_t) * acc.size(), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return fail(e, "moe_get_stats");
     out->C = (int64_t)cnt[CNT_C];
@@ -533,6 +566,16 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
         const double n_group = cnt[CNT_N_GROUP] ? (double)cnt[CNT_N_GROUP] : (double)p->N;
         out->rho_max = (double)out->L_max * (double)p->E_r / (n_group * (double)p->k);
         out->reject_rate = out->requested ? (double)out->rejected / (double)out->requested : 0.0;
+        // rows the routed GEMMs compute: accepted rows per expert rounded up
+        // to the row tile of the kernels that run them
+        const int64_t bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
+        int64_t padded = 0, accepted = 0;
+        for (int32_t a : acc) {
+            padded += (a + bm - 1) / bm * bm;
+            accepted += a;
+        }
+        out->padded_rows = padded;
+        out->padding_ratio = accepted ? (double)padded / (double)accepted : 0.0;
     }
     if (cnt[CNT_DEVICE_ERROR] & DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
     if (cnt[CNT_NONFINITE]) return MOE_ERR_NONFINITE;

@@ -130,6 +130,7 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
 // rows of one output tile of the tcgen05 grouped GEMMs for these params
 // (256 when CTA pairs are used, else 128): the dispatch's M-tile prefix unit
 int tc_tile_rows(const moe_params& p);
+cudaError_t launch_wait_selftest(unsigned long long* counters, unsigned long long limit_ns, cudaStream_t st);
 // router scores G = x W_r^T (bf16 in, fp32 out [N, E_r]) on the tensor cores
 cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,
                              unsigned long long* counters, cudaStream_t st, int* status);

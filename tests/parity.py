@@ -19,6 +19,7 @@ Comparison rules (stated once, used by every parity test):
 from __future__ import annotations
 
 import numpy as np
+import pytest
 
 import oracle
 import seeded_inputs as si
@@ -104,6 +105,13 @@ def check_dispatch(w: si.Workload, rec: dict, stats: dict):
     for key in ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max"):
         assert stats[key] == s[key], (key, stats[key], s[key])
     assert stats["C"] == C
+    # tile padding of the routed GEMMs: each expert's accepted rows rounded up
+    # to the row tile (64 rows for fp32 layers; 128, or 256 on CTA pairs when
+    # experts average >= 768 rows, for bf16 layers)
+    bm = 64 if w.dtype == si.DT_F32 else (256 if w.N * w.k >= 768 * w.E else 128)
+    padded = int(sum(-(-int(a) // bm) * bm for a in d["acc"]))
+    assert stats["padded_rows"] == padded
+    assert stats["padding_ratio"] == pytest.approx(padded / s["accepted"] if s["accepted"] else 0.0)
     if w.N:
         assert abs(stats["rho_max"] - oracle.rho_max(d["L"], w.N, w.k, w.E)) < 1e-12
         for q, key in ((50, "L_p50"), (90, "L_p90"), (99, "L_p99")):

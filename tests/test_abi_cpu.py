@@ -22,7 +22,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_struct_sizes_match_the_header_layout():
     assert ctypes.sizeof(moe.Params) == 56
-    assert ctypes.sizeof(moe.Stats) == 13 * 8 + 2 * 8 + 2 * 4
+    assert ctypes.sizeof(moe.Stats) == 13 * 8 + 2 * 8 + 2 * 4 + 8 + 8
     assert ctypes.sizeof(moe.WsLayout) == 15 * 8
 
 
@@ -91,6 +91,15 @@ def test_missing_workspace_is_reported_before_any_device_work():
     p = moe.params(16, 64, 64, 512, 2)
     r = moe.lib().moe_route(ctypes.byref(p), None, None, None, None, None, None, None, None, None)
     assert r == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_wait_selftest_limits_are_checked_on_the_host():
+    p = moe.params(16, 64, 64, 8, 2)
+    for bad in (0, 999_999, 5_000_000_001):
+        r = moe.lib().moe_selftest_wait_timeout(ctypes.byref(p), None, bad, None)
+        assert r == moe.MOE_ERR_INVALID_ARG
+    r = moe.lib().moe_selftest_wait_timeout(ctypes.byref(p), None, 50_000_000, None)
+    assert r == moe.MOE_ERR_WORKSPACE
 
 
 def test_status_strings():
