@@ -62,12 +62,13 @@ def _load():
         lib.oracle_route.argtypes = [i64, i32, i32, i32, i32, dbl, i32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         lib.oracle_dispatch.argtypes = [i64, i32, i32, i64, _P, _P, _P, _P, _P]
         lib.oracle_dispatch_ranked.argtypes = [i64, i32, i32, i64, _P, _P, _P, _P, _P, _P]
+        lib.oracle_dispatch_priority.argtypes = [i64, i32, i32, i64, _P, _P, _P, _P, _P, _P]
         lib.oracle_swiglu_rows.argtypes = [i32, i32, i32, i32, _P, _P, i64, _P, _P, _P, _P]
         lib.oracle_combine.argtypes = [i64, i32, i32, _P, _P, _P, _P, _P]
         lib.oracle_forward_rows.argtypes = [i32, i32, i32, i32, i32, i32, _P, _P, _P, _P, _P, i64,
                                             _P, _P, _P, _P, _P, _P, _P]
         lib.oracle_reject_weights.argtypes = [i64, i32, i32, _P, _P, _P, _P]
-        lib.oracle_forward.argtypes = [i64, i32, i32, i32, i32, i32, dbl, i32, i64, i32, i32,
+        lib.oracle_forward.argtypes = [i64, i32, i32, i32, i32, i32, dbl, i32, i64, i32, i32, i32,
                                        _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                        _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         lib.oracle_round_bf16.argtypes = [dbl]
@@ -189,6 +190,26 @@ def dispatch(ids, E: int, C: int):
     return {"slot": slot, "L": L, "acc": acc, "stats": stats}
 
 
+def dispatch_priority(ids, w, E: int, C: int):
+    """Acceptance by routing weight: each expert keeps the C requests with the
+    largest weight (equal weights: earlier token); accepted rows in token
+    order (see oracle.c).  Same return values as dispatch."""
+    ids = _c(ids, np.int32)
+    N, k = ids.shape
+    wd = _c(np.asarray(w, np.float64).reshape(N, k), np.float64)
+    slot = np.empty((N, k), np.int32)
+    L = np.empty(E, np.int64)
+    acc = np.empty(E, np.int64)
+    cnt = np.empty(7, np.int64)
+    rc = _load().oracle_dispatch_priority(N, k, E, C, _ptr(ids), _ptr(wd), _ptr(slot), _ptr(L), _ptr(acc),
+                                          _ptr(cnt))
+    if rc:
+        raise ValueError("oracle_dispatch_priority: invalid arguments")
+    names = ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max")
+    stats = {n: int(v) for n, v in zip(names, cnt)}
+    return {"slot": slot, "L": L, "acc": acc, "stats": stats}
+
+
 def dispatch_ranked(ids, E: int, C: int, base):
     """Acceptance for one rank's shard of a routing group split over ranks
     in token order; base[e] = requests for e by earlier ranks (see oracle.c).
@@ -278,7 +299,7 @@ def reject_weights(ids, w, slot, policy: int):
 
 
 def forward(x, W_r, Wg, Wu, Wd, *, k: int, norm: int, c: float = 0.0, theta: float = 0.0,
-            b_r=None, lat=None, Ws=None, reject_policy: int = 0):
+            b_r=None, lat=None, Ws=None, reject_policy: int = 0, accept_order: int = 0):
     """The whole layer (Algorithm 36.1 generalised by the weighting mode and a
     shared expert).  Returns a dict with Y [N,d] f64, the routing records,
     per-expert loads and the statistics."""
@@ -306,6 +327,7 @@ def forward(x, W_r, Wg, Wu, Wd, *, k: int, norm: int, c: float = 0.0, theta: flo
     b = _c(b_r, np.float32)
     la = _c(lat, np.float32)
     rc = _load().oracle_forward(N, d, d_f, E, k, norm, theta, dt, max(C, 1), dsh, int(reject_policy),
+                                int(accept_order),
                                 _ptr(x), _ptr(W_r),
                                 _ptr(b), _ptr(la), _ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(Wsg), _ptr(Wsu),
                                 _ptr(Wsd), _ptr(Y), _ptr(ids), _ptr(w), _ptr(slot), _ptr(margin),

@@ -234,6 +234,79 @@ int oracle_dispatch(int64_t N, int k, int E, int64_t C, const int32_t* ids, int3
 }
 
 /*
+ * Acceptance by gate weight ("LLM from scratch" ch. 36.3, on how the
+ * acceptance rule makes outputs depend on the batch: besides
+ * first-come-first-served the page names ordering by gate weight, under which
+ * the low-weight paths are the ones that lose their computation).  Read here
+ * as: among the paths that request expert e, the C with the largest routing
+ * weight w[t*k+j] (a_te) are accepted; equal weights go to the earlier token.
+ * Accepted paths take slots in token order (slot = number of accepted paths
+ * of e from earlier tokens), so only which paths are accepted differs from
+ * oracle_dispatch.  Outputs and counters as oracle_dispatch.
+ */
+typedef struct { int32_t e; int64_t t; int j; double w; } prio_req;
+
+static int prio_cmp(const void* pa, const void* pb) {
+    const prio_req* a = (const prio_req*)pa;
+    const prio_req* b = (const prio_req*)pb;
+    if (a->e != b->e) return a->e < b->e ? -1 : 1;
+    if (a->w != b->w) return a->w > b->w ? -1 : 1;  /* larger weight first */
+    if (a->t != b->t) return a->t < b->t ? -1 : 1;  /* then the earlier token */
+    return 0;
+}
+
+int oracle_dispatch_priority(int64_t N, int k, int E, int64_t C, const int32_t* ids, const double* w,
+                             int32_t* slot, int64_t* L, int64_t* acc, int64_t* cnt) {
+    if (N < 0 || k < 1 || E < 1 || C < 1) return 1;
+    for (int e = 0; e < E; ++e) { L[e] = 0; acc[e] = 0; }
+    for (int i = 0; i < 7; ++i) cnt[i] = 0;
+    int64_t nreq = 0;
+    for (int64_t i = 0; i < N * k; ++i)
+        if (ids[i] >= 0) ++nreq;
+    prio_req* r = (prio_req*)malloc(sizeof(prio_req) * (size_t)(nreq > 0 ? nreq : 1));
+    char* ok = (char*)calloc((size_t)(N * k > 0 ? N * k : 1), 1);
+    if (!r || !ok) { free(r); free(ok); return 2; }
+    int64_t n = 0;
+    for (int64_t t = 0; t < N; ++t)
+        for (int j = 0; j < k; ++j) {
+            const int e = ids[t * k + j];
+            if (e < 0) continue;
+            r[n].e = e; r[n].t = t; r[n].j = j; r[n].w = w[t * k + j];
+            ++n;
+            L[e] += 1;
+        }
+    qsort(r, (size_t)n, sizeof(prio_req), prio_cmp);
+    /* the first C entries of each expert's run are accepted */
+    int64_t run = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        run = (i > 0 && r[i].e == r[i - 1].e) ? run + 1 : 0;
+        if (run < C) ok[r[i].t * k + r[i].j] = 1;
+    }
+    for (int64_t t = 0; t < N; ++t) {
+        int req = 0, rej = 0;
+        for (int j = 0; j < k; ++j) {
+            const int e = ids[t * k + j];
+            if (e < 0) { slot[t * k + j] = -1; continue; }
+            ++req;
+            if (ok[t * k + j]) { slot[t * k + j] = (int32_t)acc[e]; acc[e] += 1; }
+            else { slot[t * k + j] = -1; ++rej; }
+        }
+        if (rej > 0) cnt[4] += 1;
+        if (req > 0 && rej == req) cnt[5] += 1;
+    }
+    for (int e = 0; e < E; ++e) {
+        cnt[0] += L[e];
+        cnt[1] += acc[e];
+        cnt[3] += L[e] > C ? L[e] - C : 0;
+        if (L[e] > cnt[6]) cnt[6] = L[e];
+    }
+    cnt[2] = cnt[0] - cnt[1];
+    free(r);
+    free(ok);
+    return 0;
+}
+
+/*
  * Token-order acceptance for one shard of a routing group split over ranks in
  * token order (rank 0's tokens first).  base[e] = requests for expert e made
  * by the tokens of earlier ranks.  A request is the base[e] + j-th request for
@@ -400,7 +473,8 @@ int oracle_forward_rows(int d, int d_f, int E, int k, int dtype, int d_f_sh, con
  * the shared expert.  Y is [N, d] in double.
  */
 int oracle_forward(int64_t N, int d, int d_f, int E, int k, int norm, double theta, int dtype,
-                   int64_t C, int d_f_sh, int reject_policy, const void* x, const void* W_r, const float* b_r,
+                   int64_t C, int d_f_sh, int reject_policy, int accept_order, const void* x,
+                   const void* W_r, const float* b_r,
                    const float* lat, const void* Wg, const void* Wu, const void* Wd,
                    const void* Wsg, const void* Wsu, const void* Wsd, double* Y, int32_t* ids,
                    double* w, int32_t* slot, double* margin, double* wlr_gap, uint8_t* invalid,
@@ -413,7 +487,8 @@ int oracle_forward(int64_t N, int d, int d_f, int E, int k, int norm, double the
     int rc = oracle_route(N, d, E, k, norm, theta, dtype, x, W_r, b_r, lat, 0, ids, w, margin,
                           wlr_gap, invalid);
     if (rc) return rc;
-    rc = oracle_dispatch(N, k, E, C, ids, slot, L, acc, cnt);
+    rc = accept_order == 1 ? oracle_dispatch_priority(N, k, E, C, ids, w, slot, L, acc, cnt)
+                           : oracle_dispatch(N, k, E, C, ids, slot, L, acc, cnt);
     if (rc) return rc;
     int round_h = dtype == DT_BF16;
     size_t esz = dtype == DT_BF16 ? 2 : 4;

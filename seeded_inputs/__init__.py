@@ -168,6 +168,7 @@ class Workload:
     latency: bool = False       # per-token per-expert latency t = t_up + t_comp + t_down
     seed: int = 25000
     reject_policy: int = 0      # 0: rejected path adds 0; 1: accepted paths renormalised
+    accept_order: int = 0       # 0: token order; 1: largest routing weight first
 
     @property
     def dt(self) -> str:

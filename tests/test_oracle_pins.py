@@ -178,6 +178,75 @@ def test_ranked_dispatch_equals_one_batch_at_every_cut():
         np.testing.assert_array_equal(_ranked_slots(ids, E, C, cuts), want)
 
 
+# ---------------------------------------------------------------------------
+# acceptance by gate weight ("LLM from scratch" ch. 36.3: the other acceptance
+# rule the page names besides first come first served)
+# ---------------------------------------------------------------------------
+def test_weight_order_hand_example():
+    # expert 1 is asked by all four tokens with weights 0.5, 0.9, 0.7, 0.2;
+    # C = 2 keeps tokens 1 and 2 (0.9, 0.7), where token order would keep 0, 1
+    ids = np.array([[0, 1], [1, 2], [0, 1], [1, 2]], np.int32)
+    w = np.array([[0.5, 0.5], [0.9, 0.1], [0.3, 0.7], [0.2, 0.8]])
+    d = oracle.dispatch_priority(ids, w, E=3, C=2)
+    # accepted rows keep token order: expert 1 -> token 1 at slot 0, token 2 at slot 1
+    np.testing.assert_array_equal(d["slot"], [[0, -1], [0, 0], [1, 1], [-1, 1]])
+    assert list(d["L"]) == [2, 4, 2] and list(d["acc"]) == [2, 2, 2]
+    s = d["stats"]
+    assert (s["rejected"], s["tokens_affected"], s["tokens_skipped"], s["O"]) == (2, 2, 0, 2)
+    # equal weights: the earlier token wins
+    ids2 = np.array([[0], [0], [0]], np.int32)
+    d2 = oracle.dispatch_priority(ids2, np.array([[0.5], [0.75], [0.5]]), E=1, C=2)
+    np.testing.assert_array_equal(d2["slot"].ravel(), [0, 1, -1])
+
+
+def test_weight_order_on_the_page_example():
+    # ch. 36.4 example with the printed weights as exact fractions: expert 2 is
+    # asked with 2/9, 1/3, 7/18, 2/9 (tokens 1-4); keeping the three largest
+    # drops one of the equal 2/9 paths, the later token's: the printed outcome
+    g, x, W_r = _n4_setup()
+    r = oracle.route(x, W_r, k=2, norm=oracle.NORM_RENORM)
+    # put the printed weights, exact, on the ids the oracle chose (its order
+    # within a token may differ from the printed one)
+    wk = np.zeros((4, 2))
+    for t in range(4):
+        by_expert = dict(zip(g["chosen_sets"][t], (_frac(v) for v in g["weights_by_expert_index"][t])))
+        for j in range(2):
+            wk[t, j] = by_expert[int(r["ids"][t, j]) + 1]
+    d = oracle.dispatch_priority(r["ids"], wk, E=3, C=g["capacity"])
+    assert list(d["acc"]) == g["accepted_loads"]
+    rt, re_ = g["rejected_path"]["token"] - 1, g["rejected_path"]["expert"] - 1
+    for t in range(4):
+        for j in range(2):
+            assert (d["slot"][t, j] < 0) == (t == rt and r["ids"][t, j] == re_)
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_weight_order_invariants(seed):
+    rng = np.random.default_rng(seed)
+    N, E, k = 200, 6, 3
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(N)]).astype(np.int32)
+    ids[rng.random((N, k)) < 0.05] = -1
+    # coarse weights so that equal weights meet at the capacity cut
+    w = rng.integers(1, 8, size=(N, k)) / 8.0
+    for C in (5, 40, 100, N * k):
+        d = oracle.dispatch_priority(ids, w, E=E, C=C)
+        for e in range(E):
+            t_idx, j_idx = np.nonzero(ids == e)
+            acc = d["slot"][t_idx, j_idx] >= 0
+            assert acc.sum() == min(len(t_idx), C) == d["acc"][e]
+            # every accepted request outranks every rejected one: (weight desc, token asc)
+            key = [(-w[t, j], t) for t, j in zip(t_idx, j_idx)]
+            if (~acc).any() and acc.any():
+                assert max(kk for kk, a in zip(key, acc) if a) < min(kk for kk, a in zip(key, acc) if not a)
+            # accepted requests are numbered in token order
+            order = np.argsort(t_idx[acc], kind="stable")
+            np.testing.assert_array_equal(d["slot"][t_idx, j_idx][acc][order], np.arange(acc.sum()))
+        if C >= N * k:
+            np.testing.assert_array_equal(d["slot"], oracle.dispatch(ids, E=E, C=C)["slot"])
+        s = d["stats"]
+        assert s["requested"] == s["accepted"] + s["rejected"] == (ids >= 0).sum()
+
+
 def test_capacity_printed_examples():
     for case in _golden("capacity_examples.json")["cases"]:
         assert oracle.capacity(case["c"], case["T"], case["k"], case["E"]) == case["C"], case
