@@ -54,6 +54,8 @@ def kernels_per_step(w: si.Workload, sharded: bool) -> int:
     else:
         router = 1                      # fused FFMA router
     dispatch = 5 if sharded else 4      # hist, scan(s), assign, gather
+    if w.accept_order == 1:
+        dispatch += 3                   # placement, rank, numbering, per-token pass replace assign
     experts = 2 if w.dtype == si.DT_BF16 else 3   # fp32 layers zero Y in the router or a kernel
     if w.dtype != si.DT_BF16 and not sharded:
         experts = 2
@@ -201,11 +203,15 @@ def oracle_sample(w: si.Workload, inp: dict, sample_tokens: int = 32):
     r = oracle.route(inp["x"], inp["W_r"], k=w.k, norm=w.norm, theta=w.theta, b_r=inp.get("b_r"),
                      lat=inp.get("lat"))
     C = oracle.capacity(w.c, w.N, w.k, w.E)
-    d = oracle.dispatch(r["ids"], E=w.E, C=C)
+    if w.accept_order == 1:
+        d = oracle.dispatch_priority(r["ids"], r["w"], E=w.E, C=C)
+    else:
+        d = oracle.dispatch(r["ids"], E=w.E, C=C)
+    wc = oracle.reject_weights(r["ids"], r["w"], d["slot"], w.reject_policy)
     t1 = time.perf_counter()
     toks = np.linspace(0, w.N - 1, sample_tokens).astype(np.int64)
     Ws = (inp.get("Ws_g"), inp.get("Ws_u"), inp.get("Ws_d")) if w.d_f_shared else None
-    oracle.forward_rows(inp["x"], r["ids"], r["w"], d["slot"], toks, inp["W_g"], inp["W_u"], inp["W_d"], Ws=Ws)
+    oracle.forward_rows(inp["x"], r["ids"], wc, d["slot"], toks, inp["W_g"], inp["W_u"], inp["W_d"], Ws=Ws)
     t2 = time.perf_counter()
     per_batch = (t1 - t0) + (t2 - t1) * w.N / sample_tokens
     cores = si.host_threads()
@@ -260,6 +266,8 @@ def config_of(w: si.Workload, args):
             "T": w.N, "d": w.d, "d_f": w.d_f, "E_r": w.E, "k": w.k,
             "norm": ["renorm", "fullprob", "wlr"][w.norm], "capacity_factor": w.c or None,
             "d_f_shared": w.d_f_shared, "seed": w.seed,
+            "overflow": {"reject": ["zero", "renormalise"][w.reject_policy],
+                         "accept": ["token order", "largest weight"][w.accept_order]},
             "parallelism": (f"dp{args.gpus}: one routing group of {w.N} x {args.gpus} tokens, "
                             "per-expert request counts all-gathered once per step"
                             if args.gpus > 1 else "dp1"),
@@ -303,7 +311,7 @@ def run_gpu(args):
 
     d = {k: dev(v) for k, v in inp.items()}
     p = moe.params(w.N, w.d, w.d_f, w.E, w.k, c=w.c, norm=w.norm, theta=w.theta, dtype=w.dtype,
-                   d_f_shared=w.d_f_shared)
+                   d_f_shared=w.d_f_shared, reject_policy=w.reject_policy, accept_order=w.accept_order)
     wsb = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
     Y = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()

@@ -80,6 +80,19 @@ typedef enum moe_reject_policy {
     MOE_REJECT_RENORM = 1  /* the token's accepted paths are rescaled to sum to 1  */
 } moe_reject_policy;
 
+/* Which requests an over-full expert accepts ("LLM from scratch" ch. 36.3,
+ * on how the acceptance rule makes outputs depend on the batch: first come
+ * first served in token order, or ordering by gate weight, under which the
+ * low-weight paths lose their computation). */
+typedef enum moe_accept_order {
+    MOE_ACCEPT_TOKEN = 0,  /* the first C requests in token order (Algorithm 36.1) */
+    MOE_ACCEPT_WEIGHT = 1  /* the C requests with the largest routing weight a_te,
+                              equal weights to the earlier token; accepted rows
+                              keep token order in the expert's buffer.  Single
+                              routing group only (moe_forward_begin/end and
+                              moe_dispatch_noalloc return MOE_ERR_UNSUPPORTED). */
+} moe_accept_order;
+
 typedef struct moe_params {
     int64_t N;          /* tokens in the routing group, N >= 0                      */
     int32_t d;          /* model width                                               */
@@ -92,6 +105,7 @@ typedef struct moe_params {
     int32_t dtype;      /* moe_dtype of x and of every weight                        */
     int32_t d_f_shared; /* hidden width of the always-on shared expert; 0 = none     */
     int32_t reject_policy; /* moe_reject_policy                                      */
+    int32_t accept_order;  /* moe_accept_order                                       */
 } moe_params;
 
 /* Routing statistics of the last moe_dispatch / moe_forward on a workspace

@@ -30,6 +30,7 @@ MOE_ERR_CUDA, MOE_ERR_WORKSPACE, MOE_ERR_TIMEOUT = 4, 5, 6
 MOE_NORM_RENORM, MOE_NORM_FULLPROB, MOE_NORM_WLR = 0, 1, 2
 MOE_F32, MOE_BF16 = 0, 1
 MOE_REJECT_ZERO, MOE_REJECT_RENORM = 0, 1
+MOE_ACCEPT_TOKEN, MOE_ACCEPT_WEIGHT = 0, 1
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
 
@@ -47,7 +48,8 @@ class Params(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("d", ctypes.c_int32), ("d_f", ctypes.c_int32),
                 ("E_r", ctypes.c_int32), ("k", ctypes.c_int32), ("c", ctypes.c_double),
                 ("norm", ctypes.c_int32), ("theta", ctypes.c_float), ("dtype", ctypes.c_int32),
-                ("d_f_shared", ctypes.c_int32), ("reject_policy", ctypes.c_int32)]
+                ("d_f_shared", ctypes.c_int32), ("reject_policy", ctypes.c_int32),
+                ("accept_order", ctypes.c_int32)]
 
 
 class Stats(ctypes.Structure):
@@ -119,9 +121,9 @@ def declared_symbols():
 
 
 def params(N, d, d_f, E_r, k, c=0.0, norm=MOE_NORM_RENORM, theta=0.0, dtype=MOE_BF16,
-           d_f_shared=0, reject_policy=MOE_REJECT_ZERO) -> Params:
+           d_f_shared=0, reject_policy=MOE_REJECT_ZERO, accept_order=MOE_ACCEPT_TOKEN) -> Params:
     return Params(int(N), int(d), int(d_f), int(E_r), int(k), float(c), int(norm), float(theta),
-                  int(dtype), int(d_f_shared), int(reject_policy))
+                  int(dtype), int(d_f_shared), int(reject_policy), int(accept_order))
 
 
 def _ptr(t) -> Optional[int]:

@@ -116,7 +116,7 @@ __device__ void tile_scan(int32_t* __restrict__ hist, int n_tiles, int E, int* s
 __global__ void scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int64_t C, int bm,
                             int32_t* __restrict__ L, int32_t* __restrict__ acc,
                             int32_t* __restrict__ offsets, int32_t* __restrict__ mt_start,
-                            unsigned long long* counters) {
+                            int32_t* __restrict__ all_offsets, unsigned long long* counters) {
     __shared__ int sL[kMaxExperts];
     __shared__ int warp_tot[33];
     tile_scan(hist, n_tiles, E, sL);
@@ -129,16 +129,18 @@ __global__ void scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int6
     int tot_a, tot_mt, tot_L, tot_O;
     const int ex_a = block_excl_scan(a, warp_tot, &tot_a);
     const int ex_mt = block_excl_scan(mt, warp_tot, &tot_mt);
-    block_excl_scan(Le, warp_tot, &tot_L);
+    const int ex_L = block_excl_scan(Le, warp_tot, &tot_L);
     block_excl_scan(Le > C ? (int)(Le - C) : 0, warp_tot, &tot_O);
     if (e < E) {
         L[e] = Le;
         acc[e] = a;
         offsets[e] = ex_a;
         mt_start[e] = ex_mt;
+        if (all_offsets) all_offsets[e] = ex_L;
         atomicMax(counters + CNT_L_MAX, (unsigned long long)Le);
     }
     if (threadIdx.x == 0) {
+        if (all_offsets) all_offsets[E] = tot_L;
         offsets[E] = tot_a;
         mt_start[E] = tot_mt;
         counters[CNT_REQUESTED] = (unsigned long long)tot_L;
@@ -219,12 +221,19 @@ __global__ void expert_scan_ranked_kernel(int E, int64_t C, int bm, const int32_
 
 // rank_base (nullable): per-expert requests of earlier ranks of a sharded group;
 // a request's group-wide slot is base + its slot among this rank's requests.
+__device__ void token_pass(const int32_t* __restrict__ ids, const float* __restrict__ w, int k, int E,
+                           int64_t tb, int64_t te, const int32_t* __restrict__ offsets,
+                           const int32_t* __restrict__ rank_base, int renorm_rejected,
+                           const int32_t* __restrict__ slot, float* __restrict__ slot_w,
+                           unsigned long long* counters);
+
 __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w,
                               int64_t N, int k, int E, int64_t C, int tile_tokens, int n_tiles,
                               const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets,
                               const int32_t* __restrict__ rank_base, int renorm_rejected,
-                              int32_t* __restrict__ slot, int32_t* __restrict__ slot_token,
-                              float* __restrict__ slot_w, unsigned long long* counters) {
+                              int store_request, int32_t* __restrict__ slot,
+                              int32_t* __restrict__ slot_token, float* __restrict__ slot_w,
+                              unsigned long long* counters) {
     extern __shared__ int run[];
     const int lane = threadIdx.x;
     const int tile = blockIdx.x;
@@ -248,7 +257,7 @@ __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __re
             const int64_t sg = e >= 0 ? (rank_base ? (int64_t)rank_base[e] + s : (int64_t)s) : -1;
             if (e >= 0 && sg < C) {
                 const int64_t pos = (int64_t)offsets[e] + s;
-                slot_token[pos] = (int32_t)(i / k);
+                slot_token[pos] = store_request ? (int32_t)i : (int32_t)(i / k);
                 slot_w[pos] = w[i];
                 slot[i] = (int32_t)sg;
             } else {
@@ -257,6 +266,19 @@ __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __re
         }
     }
     __syncwarp();
+    if (store_request) return;  // placement pass of acceptance by weight: no statistics yet
+    token_pass(ids, w, k, E, tb, te, offsets, rank_base, renorm_rejected, slot, slot_w, counters);
+}
+
+// Per token of [tb, te) (one warp): tokens with a rejected path, tokens with
+// every path rejected, and (reject policy 1) the rescaling of the accepted
+// paths' combine weights to sum to one.
+__device__ void token_pass(const int32_t* __restrict__ ids, const float* __restrict__ w, int k, int E,
+                           int64_t tb, int64_t te, const int32_t* __restrict__ offsets,
+                           const int32_t* __restrict__ rank_base, int renorm_rejected,
+                           const int32_t* __restrict__ slot, float* __restrict__ slot_w,
+                           unsigned long long* counters) {
+    const int lane = threadIdx.x & 31;
     unsigned long long affected = 0, skipped = 0;
     for (int64_t t = tb + lane; t < te; t += 32) {
         int req = 0, rej = 0;
@@ -292,6 +314,133 @@ __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __re
         if (affected) atomicAdd(counters + CNT_AFFECTED, affected);
         if (skipped) atomicAdd(counters + CNT_SKIPPED, skipped);
     }
+}
+
+// --- acceptance by routing weight ------------------------------------------
+// After the placement pass (assign_kernel with no capacity, storing request
+// indices), expert e's requests sit in token order at seg_req / seg_w
+// [all_offsets[e], all_offsets[e+1]).  An expert with more than C requests
+// accepts the C with the largest weight, equal weights to the earlier
+// request.  prio_select_kernel finds, per such expert, the C-th largest
+// weight W* by a radix select over the order-preserving bit pattern of the
+// fp32 weights (four passes of 8-bit digits, 256-bin shared-memory
+// histograms) and how many of the requests equal to W* are taken; requests
+// above W* are all accepted, and those equal to W* in token order up to that
+// count.
+
+// fp32 bits -> unsigned integer with the same order as the floats
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__global__ void prio_select_kernel(int64_t C, const int32_t* __restrict__ all_offsets,
+                                   const float* __restrict__ seg_w, uint32_t* __restrict__ sel_key,
+                                   int32_t* __restrict__ sel_take) {
+    __shared__ int hist[256];
+    __shared__ uint32_t s_prefix, s_mask;
+    __shared__ int s_rem;
+    const int e = blockIdx.x;
+    const int s0 = all_offsets[e], Le = all_offsets[e + 1] - s0;
+    if (Le <= C) return;  // every request accepted; nothing to select
+    if (threadIdx.x == 0) {
+        s_prefix = 0;
+        s_mask = 0;
+        s_rem = (int)C;  // rank (1-based, from the top) of the wanted key among the candidates
+    }
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0;
+        __syncthreads();
+        const uint32_t prefix = s_prefix, mask = s_mask;
+        for (int i = threadIdx.x; i < Le; i += blockDim.x) {
+            const uint32_t key = order_key(seg_w[s0 + i]);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            // the digit holding the s_rem-th largest candidate, counting from digit 255 down
+            int cum = 0, rem = s_rem, d = 255;
+            for (; d > 0; --d) {
+                if (cum + hist[d] >= rem) break;
+                cum += hist[d];
+            }
+            s_rem = rem - cum;
+            s_prefix = prefix | ((uint32_t)d << shift);
+            s_mask = mask | (255u << shift);
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        sel_key[e] = s_prefix;  // key of the C-th largest weight
+        sel_take[e] = s_rem;    // requests with exactly that key to accept, earliest first
+    }
+}
+
+// One block per expert: walks its requests in token order, decides which are
+// accepted (all of them for an expert with at most C requests), numbers the
+// accepted ones (block-wide scans) and writes the routing records: slot of
+// each request (-1 if rejected) and the token / weight of each accepted row.
+__global__ void prio_scatter_kernel(int k, int64_t C, const int32_t* __restrict__ all_offsets,
+                                    const int32_t* __restrict__ offsets,
+                                    const int32_t* __restrict__ seg_req, const float* __restrict__ seg_w,
+                                    const uint32_t* __restrict__ sel_key,
+                                    const int32_t* __restrict__ sel_take, const float* __restrict__ w,
+                                    int32_t* __restrict__ slot, int32_t* __restrict__ slot_token,
+                                    float* __restrict__ slot_w) {
+    __shared__ int warp_tot[33];
+    const int e = blockIdx.x;
+    const int s0 = all_offsets[e], Le = all_offsets[e + 1] - s0;
+    const bool all_in = Le <= C;
+    // accepted rows of e: Le or C (the cap also keeps a caller's NaN weight,
+    // whose key is arbitrary, from numbering a row past the expert's block)
+    const int cap = all_in ? Le : (int)C;
+    const uint32_t T = all_in ? 0u : sel_key[e];
+    const int take = all_in ? 0 : sel_take[e];
+    int run = 0, run_eq = 0;
+    for (int b = 0; b < Le; b += blockDim.x) {
+        const int i = b + threadIdx.x;
+        const bool in = i < Le;
+        int f = in ? 1 : 0;
+        if (!all_in) {
+            const uint32_t key = in ? order_key(seg_w[s0 + i]) : 0u;
+            const int eq = (in && key == T) ? 1 : 0;
+            int tot_eq;
+            const int ex_eq = block_excl_scan(eq, warp_tot, &tot_eq);
+            f = in && (key > T || (eq && run_eq + ex_eq < take)) ? 1 : 0;
+            run_eq += tot_eq;
+        }
+        int tot;
+        const int ex = block_excl_scan(f, warp_tot, &tot);
+        if (in) {
+            const int req = seg_req[s0 + i];
+            if (f && run + ex < cap) {
+                const int sl = run + ex;
+                slot[req] = sl;
+                slot_token[(int64_t)offsets[e] + sl] = req / k;
+                slot_w[(int64_t)offsets[e] + sl] = w[req];
+            } else {
+                slot[req] = -1;
+            }
+        }
+        run += tot;
+    }
+}
+
+// Unrequested paths (-1 ids) get slot -1, then the per-token statistics and
+// the reject policy; one warp per tile of tokens.
+__global__ void prio_token_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w,
+                                  int64_t N, int k, int E, int tile_tokens,
+                                  const int32_t* __restrict__ offsets, int renorm_rejected,
+                                  int32_t* __restrict__ slot, float* __restrict__ slot_w,
+                                  unsigned long long* counters) {
+    const int64_t tb = (int64_t)blockIdx.x * tile_tokens;
+    const int64_t te = min64(N, tb + tile_tokens);
+    for (int64_t i = tb * k + threadIdx.x; i < te * k; i += 32) {
+        const int e = ids[i];
+        if (e < 0 || e >= E) slot[i] = -1;
+    }
+    __syncwarp();
+    token_pass(ids, w, k, E, tb, te, offsets, nullptr, renorm_rejected, slot, slot_w, counters);
 }
 
 __global__ void gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ x_perm,
@@ -362,15 +511,38 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
     // 32 warps share the per-expert tile scans; the expert-level scans need
     // one thread per expert (E <= kMaxExperts = 1024)
     *where = "scan";
+    const bool by_weight = p.accept_order == MOE_ACCEPT_WEIGHT;
     scan_kernel<<<1, 1024, 0, st>>>(sc.hist, n_tiles, E, C, bm, L, acc, offsets, sc.mt_start,
-                                       counters);
+                                    by_weight ? sc.all_offsets : nullptr, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    *where = "assign";
-    assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
-                                                         n_tiles, sc.hist, offsets, nullptr,
-                                                         p.reject_policy == MOE_REJECT_RENORM, slot,
-                                                         slot_token, slot_w, counters);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int renorm = p.reject_policy == MOE_REJECT_RENORM;
+    if (!by_weight) {
+        *where = "assign";
+        assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
+                                                             n_tiles, sc.hist, offsets, nullptr, renorm, 0,
+                                                             slot, slot_token, slot_w, counters);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else {
+        // every request placed in its expert's segment in token order, then
+        // the C-th largest weight of each over-full expert selected, then the
+        // accepted requests numbered and scattered
+        *where = "place";
+        assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, INT64_MAX, sc.tile_tokens,
+                                                             n_tiles, sc.hist, sc.all_offsets, nullptr, 0, 1,
+                                                             slot, sc.seg_req, sc.seg_w, counters);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        *where = "select";
+        prio_select_kernel<<<E, 256, 0, st>>>(C, sc.all_offsets, sc.seg_w, sc.sel_key, sc.sel_take);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        *where = "number";
+        prio_scatter_kernel<<<E, 256, 0, st>>>(k, C, sc.all_offsets, offsets, sc.seg_req, sc.seg_w, sc.sel_key,
+                                              sc.sel_take, w, slot, slot_token, slot_w);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        *where = "tokens";
+        prio_token_kernel<<<n_tiles, 32, 0, st>>>(ids, w, p.N, k, E, sc.tile_tokens, offsets, renorm, slot,
+                                                  slot_w, counters);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (x && x_perm) {
         *where = "gather";
         const int row_vec = (int)(p.d * esize(p.dtype) / 16);
@@ -411,7 +583,7 @@ cudaError_t launch_dispatch_ranked(const moe_params& p, int64_t C, int bm, const
     *where = "assign";
     assign_kernel<<<sc.n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
                                                             sc.n_tiles, sc.hist, offsets, sc.base,
-                                                            p.reject_policy == MOE_REJECT_RENORM,
+                                                            p.reject_policy == MOE_REJECT_RENORM, 0,
                                                             slot, slot_token, slot_w, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (x && x_perm) {

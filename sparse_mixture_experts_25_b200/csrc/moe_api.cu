@@ -61,9 +61,10 @@ static bool layout(const moe_params& p, moe_ws_layout& L, int& n_tiles, int& til
     L.h = take(Nk * (size_t)p.d_f * es);
     L.h_shared = take((size_t)p.N * (size_t)(p.d_f_shared > 0 ? p.d_f_shared : 0) * es);
     // scratch: per-tile histograms, M-tile prefix, earlier ranks' requests,
-    // then (256-byte aligned) router scores
+    // then (256-byte aligned) router scores, then the acceptance-by-weight
+    // arrays (all-request offsets, selected keys and counts, requests, weights)
     L.scratch = take(align_up(E * (size_t)std::max(n_tiles, 1) * 4 + (E + 1) * 4 + E * 4, 256) +
-                     (size_t)p.N * E * 4);
+                     align_up((size_t)p.N * E * 4, 256) + align_up((3 * E + 1) * 4, 256) + 2 * Nk * 4);
     L.total = off;
     return true;
 }
@@ -93,6 +94,16 @@ bool make_view(const moe_params& p, void* ws, WsView& v) {
         b + v.lay.scratch +
         align_up((size_t)p.E_r * std::max(n_tiles, 1) * 4 + ((size_t)p.E_r + 1) * 4 +
                      (size_t)p.E_r * 4, 256));
+    {
+        const size_t Nk = (size_t)p.N * p.k;
+        char* pr = reinterpret_cast<char*>(v.scratch.logits) + align_up((size_t)p.N * p.E_r * 4, 256);
+        v.scratch.all_offsets = reinterpret_cast<int32_t*>(pr);
+        v.scratch.sel_key = reinterpret_cast<uint32_t*>(v.scratch.all_offsets + p.E_r + 1);
+        v.scratch.sel_take = reinterpret_cast<int32_t*>(v.scratch.sel_key + p.E_r);
+        pr += align_up((3 * (size_t)p.E_r + 1) * 4, 256);
+        v.scratch.seg_req = reinterpret_cast<int32_t*>(pr);
+        v.scratch.seg_w = reinterpret_cast<float*>(pr + Nk * 4);
+    }
     v.scratch.n_tiles = n_tiles;
     v.scratch.tile_tokens = tile_tokens;
     return true;
@@ -142,6 +153,8 @@ moe_status check_params(const moe_params* p) {
     if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (p->d_f_shared < 0) return MOE_ERR_INVALID_ARG;
     if (p->reject_policy != MOE_REJECT_ZERO && p->reject_policy != MOE_REJECT_RENORM)
+        return MOE_ERR_INVALID_ARG;
+    if (p->accept_order != MOE_ACCEPT_TOKEN && p->accept_order != MOE_ACCEPT_WEIGHT)
         return MOE_ERR_INVALID_ARG;
     if (!(p->c == p->c) || p->c > 1e6) return MOE_ERR_INVALID_ARG;
     if (p->norm == MOE_NORM_WLR && !(p->theta >= 0.f && p->theta < 1.f)) return MOE_ERR_INVALID_ARG;
@@ -421,6 +434,7 @@ moe_status moe_forward_begin(const moe_params* p, const void* x, const void* W_r
                              const float* lat, int32_t* counts, void* ws, moe_stream_t stream) {
     moe_status s = check_params(p);
     if (s != MOE_OK) return s;
+    if (p->accept_order == MOE_ACCEPT_WEIGHT) return MOE_ERR_UNSUPPORTED;  // needs every rank's weights
     if (p->E_r > kMaxRouterExperts) return MOE_ERR_UNSUPPORTED;
     if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -456,6 +470,7 @@ moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32
                            moe_stream_t stream) {
     moe_status s = check_params(p);
     if (s != MOE_OK) return s;
+    if (p->accept_order == MOE_ACCEPT_WEIGHT) return MOE_ERR_UNSUPPORTED;  // needs every rank's weights
     if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     if (n_ranks < 1 || rank < 0 || rank >= n_ranks || !counts_all || C < 1 || N_group < p->N)
         return MOE_ERR_INVALID_ARG;

@@ -46,6 +46,11 @@ struct Scratch {
     int32_t* mt_start;    // [E+1] prefix of M tiles (BM of the GEMM in use)
     float* logits;        // [N][E] router scores (tensor-core score path)
     int32_t* base;        // [E] requests of earlier ranks (sharded routing group)
+    int32_t* all_offsets; // [E+1] start of each expert's requests (acceptance by weight)
+    uint32_t* sel_key;    // [E] order key of the C-th largest weight of an over-full expert
+    int32_t* sel_take;    // [E] requests with exactly that key to accept
+    int32_t* seg_req;     // [N k] requests grouped by expert, token order (acceptance by weight)
+    float* seg_w;         // [N k] their routing weights
     int n_tiles;          // dispatch tiles
     int tile_tokens;      // tokens per dispatch tile
 };

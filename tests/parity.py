@@ -45,7 +45,8 @@ def to_dev(a):
 def params_of(w: si.Workload):
     import sparse_mixture_experts_25_b200 as moe
     return moe.params(w.N, w.d, w.d_f, w.E, w.k, c=w.c, norm=w.norm, theta=w.theta,
-                      dtype=w.dtype, d_f_shared=w.d_f_shared, reject_policy=w.reject_policy)
+                      dtype=w.dtype, d_f_shared=w.d_f_shared, reject_policy=w.reject_policy,
+                      accept_order=w.accept_order)
 
 
 def gpu_forward(w: si.Workload, inp: dict, dev: dict | None = None):
@@ -83,10 +84,15 @@ def check_routing(w: si.Workload, inp: dict, rec: dict):
 
 
 def check_dispatch(w: si.Workload, rec: dict, stats: dict):
-    """Oracle dispatch on the GPU's own ids: slots, loads, offsets, records and
-    statistics must match bit for bit."""
+    """Oracle dispatch on the GPU's own ids (and, for acceptance by weight, on
+    its own fp32 weights, so both sides order the requests by the same
+    numbers): slots, loads, offsets, records and statistics must match bit
+    for bit."""
     C = oracle.capacity(w.c, w.N, w.k, w.E)
-    d = oracle.dispatch(rec["ids"], E=w.E, C=C)
+    if w.accept_order == 1:
+        d = oracle.dispatch_priority(rec["ids"], rec["w"].astype(np.float64), E=w.E, C=C)
+    else:
+        d = oracle.dispatch(rec["ids"], E=w.E, C=C)
     np.testing.assert_array_equal(rec["slot"], d["slot"])
     np.testing.assert_array_equal(rec["L"], d["L"])
     np.testing.assert_array_equal(rec["acc"], d["acc"])

@@ -69,6 +69,7 @@ def test_workspace_layout_regions():
     (dict(E_r=2000, k=2), moe.MOE_ERR_UNSUPPORTED),
     (dict(c=float("nan")), moe.MOE_ERR_INVALID_ARG),
     (dict(reject_policy=2), moe.MOE_ERR_INVALID_ARG),
+    (dict(accept_order=2), moe.MOE_ERR_INVALID_ARG),
 ])
 def test_invalid_params_are_rejected_on_the_host(kw, status):
     base = dict(N=16, d=64, d_f=64, E_r=8, k=2)
@@ -100,6 +101,17 @@ def test_wait_selftest_limits_are_checked_on_the_host():
         assert r == moe.MOE_ERR_INVALID_ARG
     r = moe.lib().moe_selftest_wait_timeout(ctypes.byref(p), None, 50_000_000, None)
     assert r == moe.MOE_ERR_WORKSPACE
+
+
+def test_acceptance_by_weight_is_refused_where_it_is_not_built():
+    # one routing group over ranks would need every rank's weights, and the
+    # no-allocation dispatch has no room for the ranking arrays
+    p = moe.params(16, 64, 64, 8, 2, c=1.0, accept_order=moe.MOE_ACCEPT_WEIGHT)
+    L = moe.lib()
+    assert L.moe_forward_begin(ctypes.byref(p), None, None, None, None, None, None, None) == \
+        moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_dispatch_noalloc(ctypes.byref(p), None, None, 1, None, 16, None, None, None, None,
+                                  None) == moe.MOE_ERR_UNSUPPORTED
 
 
 def test_status_strings():

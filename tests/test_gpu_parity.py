@@ -62,6 +62,14 @@ SMALL = {
                                                      E=32, k=4, reject_policy=1),
     "renorm_reject_f32": W["switch_top1_f32"].scaled("renorm_reject_f32", N=700, d=64, d_f=96, k=2,
                                                     norm=si.NORM_RENORM, c=0.8, reject_policy=1),
+    # acceptance by routing weight: over-full experts keep their largest-weight requests
+    "weight_order_bf16": W["qwen3_skew_bf16"].scaled("weight_order_bf16", N=1024, d=256, d_f=192,
+                                                    E=32, k=4, accept_order=1),
+    "weight_order_f32": W["switch_top1_f32"].scaled("weight_order_f32", N=1000, d=72, d_f=96, c=0.6,
+                                                   accept_order=1),
+    "weight_order_renorm_bf16": W["qwen3_skew_bf16"].scaled("weight_order_renorm_bf16", N=700, d=128,
+                                                           d_f=64, E=16, k=4, reject_policy=1,
+                                                           accept_order=1),
 }
 
 
@@ -77,8 +85,13 @@ def _end_to_end(w):
         full = oracle.forward(inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], k=w.k,
                               norm=w.norm, c=w.c, theta=w.theta, b_r=inp.get("b_r"),
                               lat=inp.get("lat"), reject_policy=w.reject_policy,
+                              accept_order=w.accept_order,
                               Ws=(inp.get("Ws_g"), inp.get("Ws_u"), inp.get("Ws_d")) if w.d_f_shared else None)
-        assert parity.rel_err(out["Y"], full["Y"]) <= parity.TOL[w.dtype]
+        # acceptance by weight orders by the weights each side computed (fp32 on
+        # the GPU, double in the oracle): compare the whole forward when both
+        # accepted the same paths (the oracle-on-GPU-weights check above is exact)
+        if w.accept_order == 0 or np.array_equal(full["slot"], out["rec"]["slot"]):
+            assert parity.rel_err(out["Y"], full["Y"]) <= parity.TOL[w.dtype]
     assert out["status"] == moe.MOE_OK
     return out, err, int(near.sum())
 
@@ -268,9 +281,10 @@ def _sample_tokens(N, n, seed):
 
 
 @pytest.mark.parametrize("name,n_sample", [("mixtral_bf16", 12), ("qwen3_skew_bf16", 12),
-                                           ("wdmoe_decode_bf16", 16)])
+                                           ("wdmoe_decode_bf16", 16), ("qwen3_skew_bf16:weight", 8)])
 def test_full_size_sampled(name, n_sample):
-    w = W[name]
+    base, _, order = name.partition(":")
+    w = W[base] if not order else W[base].scaled(name, accept_order=1)
     inp = si.inputs(w)
     out = parity.gpu_forward(w, inp)
     r, near = parity.check_routing(w, inp, out["rec"])
