@@ -342,5 +342,38 @@ def forward(x, W_r, Wg, Wu, Wd, *, k: int, norm: int, c: float = 0.0, theta: flo
             "invalid": inv.astype(bool), "L": L, "acc": acc, "stats": stats, "C": C}
 
 
+def expert_choice(x, W_r, Wg, Wu, Wd, C: int, b_r=None, P=None):
+    """Expert-choice routing ("LLM from scratch" ch. 36.6, table of routing
+    styles: each expert picks a limited number of tokens by its column of
+    scores; a token may be picked by several experts or by none), written out
+    from that definition: P = softmax over experts of x W_r^T + b; expert e
+    takes the C tokens with the largest P[t, e] (equal scores: the lower token
+    index); Y_t = sum over the experts that took t of P[t, e] E_e(x_t).
+    P may be given (for example the scores another implementation computed)
+    so that both sides pick by the same numbers.  Returns Y [N, d] float64,
+    the picks [E, C'] (token indices, C' = min(C, N)) and P."""
+    x = _c(x)
+    dt = _dtype_of(x)
+    N, d = x.shape
+    E = Wg.shape[0]
+    if P is None:
+        r = route(x, W_r, k=E, norm=NORM_FULLPROB, b_r=b_r)
+        G = r["logits"]
+        G = G - G.max(axis=1, keepdims=True)
+        P = np.exp(G)
+        P /= P.sum(axis=1, keepdims=True)
+    P = np.asarray(P, np.float64)
+    Y = np.zeros((N, d), np.float64)
+    picks = []
+    for e in range(E):
+        order = sorted(range(N), key=lambda t: (-P[t, e], t))[:min(C, N)]
+        picks.append(order)
+        if order:
+            out = swiglu_rows(x, order, Wg[e], Wu[e], Wd[e])
+            for row, t in zip(out, order):
+                Y[t] += P[t, e] * row
+    return {"Y": Y, "picks": np.array(picks, np.int64), "P": P}
+
+
 def round_bf16(v: float) -> float:
     return _load().oracle_round_bf16(float(v))

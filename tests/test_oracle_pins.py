@@ -247,6 +247,59 @@ def test_weight_order_invariants(seed):
         assert s["requested"] == s["accepted"] + s["rejected"] == (ids >= 0).sum()
 
 
+# ---------------------------------------------------------------------------
+# expert-choice routing (ch. 36.6 table: each expert picks tokens by its score
+# column; a token may get several experts or none)
+# ---------------------------------------------------------------------------
+def _swiglu_np(xr, Wg, Wu, Wd):
+    g = xr @ Wg.T
+    u = xr @ Wu.T
+    return ((g / (1.0 + np.exp(-g))) * u) @ Wd.T
+
+
+def test_expert_choice_brute_force():
+    rng = np.random.default_rng(11)
+    N, d, d_f, E, C = 7, 4, 6, 3, 2
+    x = rng.standard_normal((N, d)).astype(np.float32)
+    W_r = rng.standard_normal((E, d)).astype(np.float32)
+    Wg = (rng.standard_normal((E, d_f, d)) / 2).astype(np.float32)
+    Wu = (rng.standard_normal((E, d_f, d)) / 2).astype(np.float32)
+    Wd = (rng.standard_normal((E, d, d_f)) / 2).astype(np.float32)
+    out = oracle.expert_choice(x, W_r, Wg, Wu, Wd, C)
+    G = x.astype(np.float64) @ W_r.astype(np.float64).T
+    P = np.exp(G - G.max(axis=1, keepdims=True))
+    P /= P.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(out["P"], P, rtol=1e-12, atol=1e-15)
+    Y = np.zeros((N, d))
+    for e in range(E):
+        top = np.argsort(-P[:, e], kind="stable")[:C]        # ties: lower index first
+        assert sorted(top.tolist()) == sorted(out["picks"][e].tolist())
+        for t in top:
+            Y[t] += P[t, e] * _swiglu_np(x[t].astype(np.float64), Wg[e].astype(np.float64),
+                                         Wu[e].astype(np.float64), Wd[e].astype(np.float64))
+    np.testing.assert_allclose(out["Y"], Y, rtol=1e-10, atol=1e-12)
+    # with C = N every expert takes every token: the dense softmax mixture
+    full = oracle.expert_choice(x, W_r, Wg, Wu, Wd, N)
+    dense = sum(P[:, [e]] * np.stack([_swiglu_np(x[t].astype(np.float64), Wg[e].astype(np.float64),
+                                                 Wu[e].astype(np.float64), Wd[e].astype(np.float64))
+                                      for t in range(N)]) for e in range(E))
+    np.testing.assert_allclose(full["Y"], dense, rtol=1e-10, atol=1e-12)
+
+
+def test_expert_choice_ties_and_unpicked_tokens():
+    # all scores equal: every expert picks the lowest token indices, the other
+    # tokens get no expert and an exactly zero output
+    N, d, E, C = 5, 2, 3, 2
+    x = np.ones((N, d), np.float32)
+    W_r = np.zeros((E, d), np.float32)
+    Wg = np.ones((E, 2, d), np.float32)
+    Wu = np.ones((E, 2, d), np.float32)
+    Wd = np.ones((E, d, 2), np.float32)
+    out = oracle.expert_choice(x, W_r, Wg, Wu, Wd, C)
+    np.testing.assert_array_equal(out["picks"], [[0, 1]] * E)
+    assert (out["Y"][2:] == 0).all() and (out["Y"][:2] != 0).all()
+
+
 def test_capacity_printed_examples():
     for case in _golden("capacity_examples.json")["cases"]:
         assert oracle.capacity(case["c"], case["T"], case["k"], case["E"]) == case["C"], case
