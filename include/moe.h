@@ -83,7 +83,13 @@ typedef enum moe_reject_policy {
 /* Which requests an over-full expert accepts ("LLM from scratch" ch. 36.3,
  * on how the acceptance rule makes outputs depend on the batch: first come
  * first served in token order, or ordering by gate weight, under which the
- * low-weight paths lose their computation). */
+ * low-weight paths lose their computation).
+ *
+ * Expert-choice routing (ch. 36.6 table of routing styles: each expert picks
+ * a limited number of tokens by its column of scores; a token may get several
+ * experts or none) is this library with k = E_r, MOE_NORM_FULLPROB and
+ * MOE_ACCEPT_WEIGHT: every token requests every expert with weight p_te and
+ * each expert keeps the C largest, C = ceil(c N) (c = C / N). */
 typedef enum moe_accept_order {
     MOE_ACCEPT_TOKEN = 0,  /* the first C requests in token order (Algorithm 36.1) */
     MOE_ACCEPT_WEIGHT = 1  /* the C requests with the largest routing weight a_te,

@@ -22,6 +22,7 @@ __all__ = [
     "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_begin", "moe_forward_end",
     "moe_get_stats",
     "moe_set_stage_events", "moe_selftest_wait_timeout", "moe_status_string", "moe_last_error",
+    "expert_choice_params",
     "workspace_views", "HEADER",
 ]
 
@@ -124,6 +125,19 @@ def params(N, d, d_f, E_r, k, c=0.0, norm=MOE_NORM_RENORM, theta=0.0, dtype=MOE_
            d_f_shared=0, reject_policy=MOE_REJECT_ZERO, accept_order=MOE_ACCEPT_TOKEN) -> Params:
     return Params(int(N), int(d), int(d_f), int(E_r), int(k), float(c), int(norm), float(theta),
                   int(dtype), int(d_f_shared), int(reject_policy), int(accept_order))
+
+
+def expert_choice_params(N, d, d_f, E_r, C, dtype=MOE_BF16, d_f_shared=0) -> Params:
+    """Parameters under which moe_forward computes expert-choice routing: every
+    token requests every expert (k = E_r) with its full-softmax probability as
+    the weight, and each expert accepts the C requests with the largest weight
+    (acceptance by weight), i.e. picks its C tokens by its score column.  The
+    capacity C = ceil(c N k / E_r) = ceil(c N) is reached with c = C / N.
+    E_r <= 32 (the library's limit on k)."""
+    if not (1 <= int(C) <= max(int(N), 1)):
+        raise ValueError("expert choice needs 1 <= C <= N")
+    return params(N, d, d_f, E_r, E_r, c=float(C) / max(int(N), 1), norm=MOE_NORM_FULLPROB, dtype=dtype,
+                  d_f_shared=d_f_shared, accept_order=MOE_ACCEPT_WEIGHT)
 
 
 def _ptr(t) -> Optional[int]:

@@ -271,6 +271,42 @@ def _route_dispatch_full(p, dev, w):
 
 
 # ---------------------------------------------------------------------------
+# expert-choice routing: k = E_r, full-softmax weights, acceptance by weight
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype,N,d,d_f,E,C", [(si.DT_BF16, 512, 256, 192, 8, 96),
+                                              (si.DT_F32, 300, 64, 96, 4, 50),
+                                              (si.DT_BF16, 1000, 128, 64, 16, 40)])
+def test_expert_choice(dtype, N, d, d_f, E, C):
+    base = W["mixtral_bf16"] if dtype == si.DT_BF16 else W["switch_top1_f32"]
+    w = base.scaled(f"expert_choice_{dtype}_{E}_{C}", N=N, d=d, d_f=d_f, E=E, k=E, norm=si.NORM_FULLPROB,
+                    c=C / N, accept_order=1, dtype=dtype)
+    p = moe.expert_choice_params(N, d, d_f, E, C, dtype=dtype)
+    q = parity.params_of(w)
+    assert [getattr(p, f) for f, _ in p._fields_] == [getattr(q, f) for f, _ in q._fields_]
+    assert moe.moe_capacity(p) == C
+    inp = si.inputs(w)
+    out = parity.gpu_forward(w, inp)
+    assert out["status"] == moe.MOE_OK
+    rec = out["rec"]
+    # the GPU's scores as an [N, E] table (k = E lists every expert once per token)
+    P = np.zeros((N, E))
+    P[np.arange(N)[:, None], rec["ids"]] = rec["w"]
+    ref = oracle.expert_choice(inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], C)
+    assert (np.abs(P - ref["P"]) <= 3e-5 * (1 + np.abs(ref["P"]))).all()
+    # picks by the GPU's own scores, so both sides decide on the same numbers
+    ec = oracle.expert_choice(inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], C, P=P)
+    got = {(int(t), int(rec["ids"][t, j])) for t, j in zip(*np.nonzero(rec["slot"] >= 0))}
+    want = {(int(t), e) for e in range(E) for t in ec["picks"][e]}
+    assert got == want
+    assert (np.bincount([e for _, e in got], minlength=E) == C).all()
+    err = parity.rel_err(out["Y"], ec["Y"])
+    assert err <= parity.TOL[dtype], err
+    unpicked = np.setdiff1d(np.arange(N), [t for t, _ in got])
+    assert (out["Y"][unpicked] == 0).all()
+    print(f"expert choice E={E} C={C}: max-abs-rel {err:.2e}, tokens with no expert {unpicked.size}")
+
+
+# ---------------------------------------------------------------------------
 # full-size page-shaped layers: every token's routing and dispatch, sampled outputs
 # ---------------------------------------------------------------------------
 def _sample_tokens(N, n, seed):
