@@ -63,6 +63,7 @@ def _load():
         lib.oracle_dispatch.argtypes = [i64, i32, i32, i64, _P, _P, _P, _P, _P]
         lib.oracle_dispatch_ranked.argtypes = [i64, i32, i32, i64, _P, _P, _P, _P, _P, _P]
         lib.oracle_dispatch_priority.argtypes = [i64, i32, i32, i64, _P, _P, _P, _P, _P, _P]
+        lib.oracle_swiglu_dense.argtypes = [i32, i32, i32, i32, _P, i64, _P, _P, _P, _P]
         lib.oracle_swiglu_rows.argtypes = [i32, i32, i32, i32, _P, _P, i64, _P, _P, _P, _P]
         lib.oracle_combine.argtypes = [i64, i32, i32, _P, _P, _P, _P, _P]
         lib.oracle_forward_rows.argtypes = [i32, i32, i32, i32, i32, i32, _P, _P, _P, _P, _P, i64,
@@ -373,6 +374,46 @@ def expert_choice(x, W_r, Wg, Wu, Wd, C: int, b_r=None, P=None):
             for row, t in zip(out, order):
                 Y[t] += P[t, e] * row
     return {"Y": Y, "picks": np.array(picks, np.int64), "P": P}
+
+
+def soft_moe(x, Phi, Wg, Wu, Wd, p: int):
+    """Soft MoE ("LLM from scratch" ch. 36.6, Soft Mixture of Experts), written
+    out from its definition: S = E_r p slots, slot e p + i belongs to expert e;
+    scores Z = X Phi^T [N, S] (Phi stored [S, d]); dispatch weights D =
+    softmax of Z over the tokens (each column sums to one); combine weights
+    C = softmax of Z over the slots (each row sums to one); slot inputs
+    Xs = D^T X [S, d]; slot outputs Ys_s = E_{e(s)}(Xs_s) (h rounded to bf16
+    for bf16 weights, as in the other layers); Y = C Ys [N, d].  Returns Y,
+    D, C, Xs and Ys in float64."""
+    x, Phi, Wg, Wu, Wd = _c(x), _c(Phi), _c(Wg), _c(Wu), _c(Wd)
+    dt = _dtype_of(x)
+    X = _as_f64(x)
+    F = _as_f64(Phi)
+    N, d = X.shape
+    E, d_f = Wg.shape[0], Wg.shape[1]
+    S = E * p
+    assert F.shape == (S, d)
+    Z = X @ F.T
+    D = np.exp(Z - Z.max(axis=0, keepdims=True))
+    D /= D.sum(axis=0, keepdims=True)
+    Cw = np.exp(Z - Z.max(axis=1, keepdims=True))
+    Cw /= Cw.sum(axis=1, keepdims=True)
+    Xs = D.T @ X
+    Ys = np.empty((S, d), np.float64)
+    for e in range(E):
+        blk = np.ascontiguousarray(Xs[e * p:(e + 1) * p])
+        out = np.empty((p, d), np.float64)
+        _load().oracle_swiglu_dense(d, d_f, dt, int(dt == DT_BF16), _ptr(blk), p, _ptr(_c(Wg[e])),
+                                    _ptr(_c(Wu[e])), _ptr(_c(Wd[e])), _ptr(out))
+        Ys[e * p:(e + 1) * p] = out
+    return {"Y": Cw @ Ys, "D": D, "C": Cw, "Xs": Xs, "Ys": Ys}
+
+
+def _as_f64(a):
+    """fp32 or bf16 (uint16 bit patterns) array -> float64, exactly."""
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
 
 
 def round_bf16(v: float) -> float:

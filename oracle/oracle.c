@@ -408,6 +408,36 @@ int oracle_swiglu_rows(int d, int d_f, int dtype, int round_h, const void* x, co
 }
 
 /*
+ * The same SwiGLU expert on M input rows given directly in double (for Soft
+ * MoE, whose expert inputs are mixtures of token rows, not token rows):
+ * out[r*d + o] = E(X_r)_o.
+ */
+int oracle_swiglu_dense(int d, int d_f, int dtype, int round_h, const double* X, int64_t M, const void* Wg,
+                        const void* Wu, const void* Wd, double* out) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < M; ++r) {
+        const double* xt = X + r * d;
+        double* h = (double*)malloc(sizeof(double) * d_f);
+        for (int j = 0; j < d_f; ++j) {
+            double gs = 0.0, us = 0.0;
+            for (int i = 0; i < d; ++i) {
+                gs += xt[i] * load(Wg, dtype, (size_t)j * d + i);
+                us += xt[i] * load(Wu, dtype, (size_t)j * d + i);
+            }
+            double hv = silu(gs) * us;
+            h[j] = round_h ? oracle_round_bf16(hv) : hv;
+        }
+        for (int o = 0; o < d; ++o) {
+            double s = 0.0;
+            for (int j = 0; j < d_f; ++j) s += h[j] * load(Wd, dtype, (size_t)o * d_f + j);
+            out[r * d + o] = s;
+        }
+        free(h);
+    }
+    return 0;
+}
+
+/*
  * Combine (ch. 36.3, Algorithm 36.1 step 6): for every accepted record
  * (t, e, slot c, a_te), Y_t += a_te * H_e[c].  H is given per expert as a
  * pointer table Hs[e] -> [rows, d] with row c = slot c.  Y is overwritten

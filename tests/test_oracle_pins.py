@@ -300,6 +300,59 @@ def test_expert_choice_ties_and_unpicked_tokens():
     assert (out["Y"][2:] == 0).all() and (out["Y"][:2] != 0).all()
 
 
+# ---------------------------------------------------------------------------
+# Soft MoE (ch. 36.6: tokens mixed into slots, experts on slots, slots mixed
+# back; dispatch normalised over tokens, combine over slots)
+# ---------------------------------------------------------------------------
+def _soft_case(seed, N, d, d_f, E, p):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((N, d)).astype(np.float32)
+    Wg = (rng.standard_normal((E, d_f, d)) / 2).astype(np.float32)
+    Wu = (rng.standard_normal((E, d_f, d)) / 2).astype(np.float32)
+    Wd = (rng.standard_normal((E, d, d_f)) / 2).astype(np.float32)
+    return rng, x, Wg, Wu, Wd
+
+
+def test_soft_moe_uniform_scores_closed_form():
+    # Phi = 0: every slot averages all tokens, every token averages all slots,
+    # so every output row is the mean over experts of E_e(mean of x)
+    N, d, d_f, E, p = 9, 5, 7, 3, 2
+    _, x, Wg, Wu, Wd = _soft_case(5, N, d, d_f, E, p)
+    out = oracle.soft_moe(x, np.zeros((E * p, d), np.float32), Wg, Wu, Wd, p)
+    xbar = x.astype(np.float64).mean(axis=0)
+    want = np.mean([_swiglu_np(xbar, Wg[e].astype(np.float64), Wu[e].astype(np.float64),
+                               Wd[e].astype(np.float64)) for e in range(E)], axis=0)
+    np.testing.assert_allclose(out["Y"], np.tile(want, (N, 1)), rtol=1e-12, atol=1e-13)
+
+
+def test_soft_moe_one_token_per_slot_limit():
+    # N = S slots, x_t = e_t and Phi_s = 60 e_s: Z = 60 I, so D and C are the
+    # identity up to e^-60 and token t is processed alone by slot t's expert
+    E, p = 3, 2
+    N = d = E * p
+    _, _, Wg, Wu, Wd = _soft_case(6, N, d, 4, E, p)
+    x = np.eye(N, d, dtype=np.float32)
+    Phi = (60.0 * np.eye(N, d)).astype(np.float32)
+    out = oracle.soft_moe(x, Phi, Wg, Wu, Wd, p)
+    want = np.stack([_swiglu_np(x[t].astype(np.float64), Wg[t // p].astype(np.float64),
+                                Wu[t // p].astype(np.float64), Wd[t // p].astype(np.float64))
+                     for t in range(N)])
+    np.testing.assert_allclose(out["Y"], want, rtol=1e-12, atol=1e-20)
+
+
+def test_soft_moe_normalisations():
+    N, d, d_f, E, p = 11, 6, 5, 4, 3
+    rng, x, Wg, Wu, Wd = _soft_case(7, N, d, d_f, E, p)
+    Phi = rng.standard_normal((E * p, d)).astype(np.float32)
+    out = oracle.soft_moe(x, Phi, Wg, Wu, Wd, p)
+    np.testing.assert_allclose(out["D"].sum(axis=0), 1.0, rtol=1e-13)   # each slot: weights over tokens
+    np.testing.assert_allclose(out["C"].sum(axis=1), 1.0, rtol=1e-13)   # each token: weights over slots
+    assert (out["D"] > 0).all() and (out["C"] > 0).all()
+    # slot inputs are convex combinations of the tokens
+    assert (out["Xs"].min(axis=0) >= x.min(axis=0) - 1e-12).all()
+    assert (out["Xs"].max(axis=0) <= x.max(axis=0) + 1e-12).all()
+
+
 def test_capacity_printed_examples():
     for case in _golden("capacity_examples.json")["cases"]:
         assert oracle.capacity(case["c"], case["T"], case["k"], case["E"]) == case["C"], case
