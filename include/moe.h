@@ -335,6 +335,51 @@ MOE_API moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats*
 MOE_API moe_status moe_set_stage_events(void* const* events, int n);
 
 /*
+ * Soft MoE ("LLM from scratch" ch. 36.6, Soft Mixture of Experts): tokens are
+ * mixed into S = E_r p slots, each expert processes its p slots, and the slot
+ * outputs are mixed back into the tokens.
+ *   Z  = X Phi^T [N, S]; D = softmax of Z over the tokens (each slot's column
+ *   sums to one); C = softmax of Z over the slots (each token's row sums to
+ *   one); Xs = D^T X [S, d]; Ys_s = E_{e(s)}(Xs_s) with e(s) = s / p (SwiGLU
+ *   expert as in moe_forward); Y = C Ys [N, d].
+ * Layouts: x [N, d] bf16; Phi [S, d] bf16 (slot s's score vector, slots of
+ * expert e at rows e p .. e p + p - 1); W_g, W_u [E_r, d_f, d], W_d
+ * [E_r, d, d_f] bf16 as in moe_forward; Y [N, d] fp32, overwritten.
+ * Precision: scores, softmax statistics and all accumulations fp32; D, C, the
+ * slot inputs and the slot outputs are bf16 operands of the tensor-core
+ * contractions; the experts' hidden activations are bf16.
+ * Constraints: dtype MOE_BF16 (fp32 soft layers are not built:
+ * MOE_ERR_UNSUPPORTED); N, d, d_f and S multiples of 8 (16-byte operand rows;
+ * else MOE_ERR_UNSUPPORTED).  Every token mixes into every slot, so this is
+ * not causal across the batch.  Non-finite scores are not detected (they
+ * propagate into Y).
+ */
+typedef struct moe_soft_params {
+    int64_t N;          /* tokens                                                   */
+    int32_t d;          /* model width                                              */
+    int32_t d_f;        /* expert hidden width                                      */
+    int32_t E_r;        /* experts, 1..1024                                         */
+    int32_t p;          /* slots per expert (S = E_r p)                             */
+    int32_t dtype;      /* MOE_BF16                                                 */
+    int32_t reserved;
+} moe_soft_params;
+
+/* Workspace bytes of moe_soft_forward (caller-allocated, 16-byte aligned). */
+MOE_API moe_status moe_soft_workspace_size(const moe_soft_params* p, size_t* bytes);
+
+/* The Soft MoE forward pass above, asynchronous on `stream`; the library
+ * allocates nothing.  Errors: MOE_ERR_INVALID_ARG (null or misaligned
+ * pointers), MOE_ERR_WORKSPACE, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA (with
+ * moe_last_error).  N = 0 returns MOE_OK with nothing launched. */
+MOE_API moe_status moe_soft_forward(const moe_soft_params* p, const void* x, const void* Phi,
+                                    const void* W_g, const void* W_u, const void* W_d, float* Y, void* ws,
+                                    moe_stream_t stream);
+
+/* Waits for `stream` and reports MOE_ERR_TIMEOUT if a device wait of the
+ * last moe_soft_forward on `ws` gave up, else MOE_OK. */
+MOE_API moe_status moe_soft_check(const moe_soft_params* p, const void* ws, moe_stream_t stream);
+
+/*
  * Self-test of the library's bounded device waits (no counterpart on the
  * pages).  Launches one CTA that waits on a shared-memory mbarrier nothing
  * ever arrives on, with the same bounded-wait routine the tensor-core GEMMs

@@ -33,7 +33,7 @@ DT_F32, DT_BF16 = 0, 1
 
 # tensor ids of the counter-based streams
 TID = {"x": 1, "W_r": 2, "W_g": 3, "W_u": 4, "W_d": 5, "Ws_g": 6, "Ws_u": 7, "Ws_d": 8,
-       "lat_up": 9, "lat_comp": 10, "lat_down": 11}
+       "lat_up": 9, "lat_comp": 10, "lat_down": 11, "Phi": 12}
 
 
 def build(force: bool = False) -> str:
@@ -169,6 +169,7 @@ class Workload:
     seed: int = 25000
     reject_policy: int = 0      # 0: rejected path adds 0; 1: accepted paths renormalised
     accept_order: int = 0       # 0: token order; 1: largest routing weight first
+    soft_p: int = 0             # > 0: Soft MoE layer with soft_p slots per expert (Phi [E soft_p, d])
 
     @property
     def dt(self) -> str:
@@ -197,13 +198,14 @@ def shape(w: Workload, name: str):
         "x": (w.N, w.d), "W_r": (w.E, w.d), "b_r": (w.E,), "lat": (w.N, w.E),
         "W_g": (w.E, w.d_f, w.d), "W_u": (w.E, w.d_f, w.d), "W_d": (w.E, w.d, w.d_f),
         "Ws_g": (w.d_f_shared, w.d), "Ws_u": (w.d_f_shared, w.d), "Ws_d": (w.d, w.d_f_shared),
+        "Phi": (w.E * w.soft_p, w.d),
     }[name]
 
 
 def _std(w: Workload, name: str) -> float:
     if name in ("x",):
         return 1.0
-    if name in ("W_r", "W_g", "W_u", "Ws_g", "Ws_u"):
+    if name in ("W_r", "W_g", "W_u", "Ws_g", "Ws_u", "Phi"):
         return 1.0 / math.sqrt(w.d)
     if name == "W_d":
         return 1.0 / math.sqrt(w.d_f)
@@ -232,6 +234,8 @@ def tensor(w: Workload, name: str, expert: Optional[int] = None) -> Optional[np.
                 for part in ("lat_up", "lat_comp", "lat_down"))
         return t.astype(np.float32).reshape(w.N, w.E)
     if name.startswith("Ws_") and w.d_f_shared <= 0:
+        return None
+    if name == "Phi" and w.soft_p <= 0:
         return None
     shp = shape(w, name)
     if expert is not None:

@@ -22,7 +22,8 @@ __all__ = [
     "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_begin", "moe_forward_end",
     "moe_get_stats",
     "moe_set_stage_events", "moe_selftest_wait_timeout", "moe_status_string", "moe_last_error",
-    "expert_choice_params",
+    "expert_choice_params", "SoftParams", "soft_params", "moe_soft_workspace_size", "moe_soft_forward",
+    "moe_soft_check",
     "workspace_views", "HEADER",
 ]
 
@@ -51,6 +52,17 @@ class Params(ctypes.Structure):
                 ("norm", ctypes.c_int32), ("theta", ctypes.c_float), ("dtype", ctypes.c_int32),
                 ("d_f_shared", ctypes.c_int32), ("reject_policy", ctypes.c_int32),
                 ("accept_order", ctypes.c_int32)]
+
+
+class SoftParams(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("d", ctypes.c_int32), ("d_f", ctypes.c_int32),
+                ("E_r", ctypes.c_int32), ("p", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+def soft_params(N, d, d_f, E_r, p, dtype=None) -> SoftParams:
+    """Soft MoE layer: S = E_r p slots (see moe_soft_forward in the header)."""
+    return SoftParams(int(N), int(d), int(d_f), int(E_r), int(p), int(MOE_BF16 if dtype is None else dtype), 0)
 
 
 class Stats(ctypes.Structure):
@@ -100,6 +112,10 @@ def lib():
                                       ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(_P), ctypes.c_int]
         L.moe_selftest_wait_timeout.argtypes = [pp, _P, ctypes.c_int64, _P]
+        sp = ctypes.POINTER(SoftParams)
+        L.moe_soft_workspace_size.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t)]
+        L.moe_soft_forward.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_soft_check.argtypes = [sp, _P, _P]
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [ctypes.c_int]
@@ -108,7 +124,8 @@ def lib():
                      "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_combine",
                      "moe_forward",
                      "moe_get_stats", "moe_set_stage_events", "moe_forward_begin",
-                     "moe_forward_end", "moe_selftest_wait_timeout"):
+                     "moe_forward_end", "moe_selftest_wait_timeout", "moe_soft_workspace_size",
+                     "moe_soft_forward", "moe_soft_check"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -247,6 +264,23 @@ def moe_get_stats(p, ws, stream=None):
     if status not in (MOE_OK, MOE_ERR_NONFINITE, MOE_ERR_TIMEOUT):
         raise MoEError(status, "moe_get_stats")
     return status, s.as_dict()
+
+
+def moe_soft_workspace_size(sp) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_soft_workspace_size(ctypes.byref(sp), ctypes.byref(n)), "moe_soft_workspace_size")
+    return n.value
+
+
+def moe_soft_forward(sp, x, Phi, W_g, W_u, W_d, Y, ws, stream=None):
+    """Soft MoE forward on device tensors (asynchronous)."""
+    _check(lib().moe_soft_forward(ctypes.byref(sp), _ptr(x), _ptr(Phi), _ptr(W_g), _ptr(W_u), _ptr(W_d),
+                                  _ptr(Y), _ptr(ws), _stream(stream)), "moe_soft_forward")
+
+
+def moe_soft_check(sp, ws, stream=None) -> int:
+    """Waits for the stream; MOE_OK or MOE_ERR_TIMEOUT."""
+    return lib().moe_soft_check(ctypes.byref(sp), _ptr(ws), _stream(stream))
 
 
 def moe_selftest_wait_timeout(p, ws, limit_ns: int, stream=None):

@@ -1074,33 +1074,39 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
     return launch_tc<EPI_STORE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles, st);
 }
 
-cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,
-                             unsigned long long* counters, cudaStream_t st, int* status) {
+cudaError_t launch_tc_dense(int64_t M, int64_t Nc, int64_t K, const void* A, const void* B, float* out,
+                            unsigned long long* counters, cudaStream_t st, int* status) {
     *status = MOE_OK;
+    if (M <= 0 || Nc <= 0) return cudaSuccess;
     CUtensorMap mA, mB;
-    if (!make_map(&mA, x, (uint64_t)p.N, p.d) || !make_map(&mB, W_r, (uint64_t)p.E_r, p.d)) {
+    if (!make_map(&mA, A, (uint64_t)M, (uint64_t)K) || !make_map(&mB, B, (uint64_t)Nc, (uint64_t)K)) {
         *status = MOE_ERR_CUDA;
         return cudaErrorInvalidValue;
     }
     TcArgs a{};
     a.E = 0;
     a.has_routed = 0;
-    a.M_sh = (int)p.N;
-    a.nt_sh = (p.E_r + BN - 1) / BN;
-    a.nkb_sh = (p.d + BK - 1) / BK;
-    a.n_valid_sh = p.E_r;
-    a.out = logits;
-    a.ld_out = p.E_r;
-    a.max_rows = (int)p.N;
-    a.n_tokens = (int)p.N;
-    const int64_t tiles = ((p.N + 127) / 128) * a.nt_sh;
+    a.M_sh = (int)M;
+    a.nt_sh = (int)((Nc + BN - 1) / BN);
+    a.nkb_sh = (int)((K + BK - 1) / BK);
+    a.n_valid_sh = (int)Nc;
+    a.out = out;
+    a.ld_out = (int)Nc;
+    a.max_rows = (int)M;
+    a.n_tokens = (int)M;
+    const int64_t tiles = ((M + 127) / 128) * a.nt_sh;
     a.ks = choose_ksplit((double)tiles, a.nkb_sh);
     a.counters = counters;
-    if (a.ks > 1) {  // K slices add into the scores with red.add
-        cudaError_t e = cudaMemsetAsync(logits, 0, sizeof(float) * (size_t)p.N * p.E_r, st);
+    if (a.ks > 1) {  // K slices add into the output with red.add
+        cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)M * (size_t)Nc, st);
         if (e != cudaSuccess) return e;
     }
     return launch_tc<EPI_STORE, false>(mA, mB, mB, mA, mB, mB, mA, mA, a, tiles * a.ks, st);
+}
+
+cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,
+                             unsigned long long* counters, cudaStream_t st, int* status) {
+    return launch_tc_dense(p.N, p.E_r, p.d, x, W_r, logits, counters, st, status);
 }
 
 cudaError_t launch_wait_selftest(unsigned long long* counters, unsigned long long limit_ns, cudaStream_t st) {

@@ -1,0 +1,319 @@
+// Soft MoE forward ("LLM from scratch" ch. 36.6, Soft Mixture of Experts).
+//
+// What it computes: S = E_r p slots, slot s = e p + i belongs to expert e;
+//   Z  = X Phi^T                      [N, S]  slot scores
+//   D  = softmax of Z over tokens     (each slot's column sums to one)
+//   C  = softmax of Z over slots      (each token's row sums to one)
+//   Xs = D^T X                        [S, d]  slot inputs (token mixtures)
+//   Ys_s = E_{e(s)}(Xs_s)             SwiGLU expert of the slot's owner
+//   Y  = C Ys                         [N, d]
+//
+// Design: the three contractions run on the tcgen05 dense GEMM
+// (out = A B^T with both operands K-major), so the operands are laid out for
+// it: D is written transposed ([S, N], K = tokens), X is transposed once
+// ([d, N]), and the slot outputs are transposed ([d, S], K = slots).  The
+// experts run on the grouped tcgen05 GEMMs with p rows per expert (the slot
+// rows are already grouped by expert).  D, C, Xs and Ys enter the tensor cores
+// as bf16; scores, softmax statistics and every accumulation are fp32.
+// Small kernels: column statistics of Z (online max / sum per slot), the
+// transposed dispatch weights, the row softmax, bf16 transposes in 32 x 32
+// shared-memory tiles, an fp32 -> bf16 conversion.
+#include <cuda_bf16.h>
+#include <stdio.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kT = 32;  // transpose tile
+
+// per slot s: m_s = max_t Z[t, s], l_s = sum_t exp(Z[t, s] - m_s); one block
+// per 32 slots, lane = slot, the 8 warps stride over the tokens
+__global__ void soft_colstat_kernel(const float* __restrict__ Z, int64_t N, int S, float* __restrict__ colmax,
+                                    float* __restrict__ colsum) {
+    __shared__ float sm[8][32], sl[8][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int s = blockIdx.x * 32 + lane;
+    float m = -INFINITY, l = 0.f;
+    if (s < S) {
+        for (int64_t t = warp; t < N; t += 8) {
+            const float z = Z[t * S + s];
+            if (l == 0.f) {
+                m = z;
+                l = 1.f;
+            } else if (z > m) {
+                l = l * expf(m - z) + 1.f;
+                m = z;
+            } else {
+                l += expf(z - m);
+            }
+        }
+    }
+    sm[warp][lane] = m;
+    sl[warp][lane] = l;
+    __syncthreads();
+    if (warp == 0 && s < S) {
+        float M = -INFINITY;
+        for (int w = 0; w < 8; ++w)
+            if (sl[w][lane] > 0.f) M = fmaxf(M, sm[w][lane]);
+        float L = 0.f;
+        for (int w = 0; w < 8; ++w)
+            if (sl[w][lane] > 0.f) L += sl[w][lane] * expf(sm[w][lane] - M);
+        colmax[s] = M;
+        colsum[s] = L;
+    }
+}
+
+// Dt[s, t] = exp(Z[t, s] - m_s) / l_s in bf16, written transposed through a
+// 32 x 32 shared-memory tile (reads and writes coalesced)
+__global__ void soft_dispatch_t_kernel(const float* __restrict__ Z, int64_t N, int S,
+                                       const float* __restrict__ colmax, const float* __restrict__ colsum,
+                                       __nv_bfloat16* __restrict__ Dt) {
+    __shared__ float tile[kT][kT + 1];
+    const int64_t t0 = (int64_t)blockIdx.x * kT;
+    const int s0 = blockIdx.y * kT;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    for (int r = ty; r < kT; r += blockDim.y) {
+        const int64_t t = t0 + r;
+        const int s = s0 + tx;
+        float v = 0.f;
+        if (t < N && s < S) v = expf(Z[t * S + s] - colmax[s]) / colsum[s];
+        tile[r][tx] = v;
+    }
+    __syncthreads();
+    for (int r = ty; r < kT; r += blockDim.y) {
+        const int s = s0 + r;
+        const int64_t t = t0 + tx;
+        if (s < S && t < N) Dt[(int64_t)s * N + t] = __float2bfloat16_rn(tile[tx][r]);
+    }
+}
+
+// C[t, s] = exp(Z[t, s] - m_t) / l_t in bf16; one warp per token
+__global__ void soft_combine_w_kernel(const float* __restrict__ Z, int64_t N, int S,
+                                      __nv_bfloat16* __restrict__ Cw) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= N) return;
+    const float* z = Z + t * S;
+    float m = -INFINITY, l = 0.f;
+    for (int s = lane; s < S; s += 32) {
+        const float v = z[s];
+        if (l == 0.f) {
+            m = v;
+            l = 1.f;
+        } else if (v > m) {
+            l = l * expf(m - v) + 1.f;
+            m = v;
+        } else {
+            l += expf(v - m);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
+        const float M = l2 > 0.f ? (l > 0.f ? fmaxf(m, m2) : m2) : m;
+        l = (l > 0.f ? l * expf(m - M) : 0.f) + (l2 > 0.f ? l2 * expf(m2 - M) : 0.f);
+        m = M;
+    }
+    for (int s = lane; s < S; s += 32) Cw[t * S + s] = __float2bfloat16_rn(expf(z[s] - m) / l);
+}
+
+// out[c, r] = in[r, c] for a row-major [R, Cc] input; bf16 -> bf16 or fp32 -> bf16
+template <typename Tin>
+__global__ void soft_transpose_kernel(const Tin* __restrict__ in, int64_t R, int64_t Cc,
+                                      __nv_bfloat16* __restrict__ out) {
+    __shared__ float tile[kT][kT + 1];
+    const int64_t r0 = (int64_t)blockIdx.x * kT, c0 = (int64_t)blockIdx.y * kT;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    for (int i = ty; i < kT; i += blockDim.y) {
+        const int64_t r = r0 + i, c = c0 + tx;
+        float v = 0.f;
+        if (r < R && c < Cc) {
+            if constexpr (sizeof(Tin) == 2) v = __bfloat162float(in[r * Cc + c]);
+            else v = in[r * Cc + c];
+        }
+        tile[i][tx] = v;
+    }
+    __syncthreads();
+    for (int i = ty; i < kT; i += blockDim.y) {
+        const int64_t c = c0 + i, r = r0 + tx;
+        if (c < Cc && r < R) out[c * R + r] = __float2bfloat16_rn(tile[tx][i]);
+    }
+}
+
+__global__ void soft_to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out, int64_t n4) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 v = in[i];
+        __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+        out[i] = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+    }
+}
+
+__global__ void soft_offsets_kernel(int E, int p, int32_t* __restrict__ offsets) {
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = e * p;
+}
+
+struct SoftLayout {
+    size_t counters, offsets, mt_start, Z, colmax, colsum, Dt, Cw, Xt, S32, Xs, h, Yst, total;
+};
+
+size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+SoftLayout soft_layout(const moe_soft_params& p) {
+    const size_t N = (size_t)p.N, S = (size_t)p.E_r * p.p, d = (size_t)p.d, df = (size_t)p.d_f;
+    const size_t E = (size_t)p.E_r;
+    SoftLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = up256(off + bytes);
+        return o;
+    };
+    L.counters = take(CNT_COUNT * 8);
+    L.offsets = take((E + 1) * 4);
+    L.mt_start = take((E + 1) * 4);
+    L.Z = take(N * S * 4);
+    L.colmax = take(S * 4);
+    L.colsum = take(S * 4);
+    L.Dt = take(S * N * 2);
+    L.Cw = take(N * S * 2);
+    L.Xt = take(d * N * 2);
+    L.S32 = take(S * d * 4);  // slot inputs, then slot outputs, fp32
+    L.Xs = take(S * d * 2);
+    L.h = take(S * df * 2);
+    L.Yst = take(d * S * 2);
+    L.total = off;
+    return L;
+}
+
+moe_status soft_check(const moe_soft_params* p) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (p->N < 0 || p->d <= 0 || p->d_f <= 0 || p->E_r <= 0 || p->p <= 0) return MOE_ERR_INVALID_ARG;
+    if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (p->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;  // the slot contractions are bf16 tcgen05 GEMMs
+    if (p->E_r > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    const int64_t S = (int64_t)p->E_r * p->p;
+    // 16-byte rows for every tensor-core operand (K = d, tokens, slots)
+    if (p->d % 8 || p->d_f % 8 || p->N % 8 || S % 8) return MOE_ERR_UNSUPPORTED;
+    if (p->N > (int64_t)1 << 30 || S > (int64_t)1 << 30) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+thread_local char g_soft_error[256] = "";
+
+moe_status soft_fail(cudaError_t e, const char* where) {
+    snprintf(g_soft_error, sizeof(g_soft_error), "%s: %s (%d)", where, cudaGetErrorString(e), (int)e);
+    record_error(g_soft_error);
+    return MOE_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_soft_workspace_size(const moe_soft_params* p, size_t* bytes) {
+    moe_status s = soft_check(p);
+    if (s != MOE_OK) return s;
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    *bytes = soft_layout(*p).total;
+    return MOE_OK;
+}
+
+moe_status moe_soft_forward(const moe_soft_params* p, const void* x, const void* Phi, const void* W_g,
+                            const void* W_u, const void* W_d, float* Y, void* ws, moe_stream_t stream) {
+    moe_status s = soft_check(p);
+    if (s != MOE_OK) return s;
+    auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+    if (!ws || !al16(ws)) return MOE_ERR_WORKSPACE;
+    if (p->N == 0) return MOE_OK;
+    if (!x || !Phi || !W_g || !W_u || !W_d || !Y) return MOE_ERR_INVALID_ARG;
+    if (!al16(x) || !al16(Phi) || !al16(W_g) || !al16(W_u) || !al16(W_d) || !al16(Y)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const SoftLayout L = soft_layout(*p);
+    char* b = static_cast<char*>(ws);
+    auto* counters = reinterpret_cast<unsigned long long*>(b + L.counters);
+    auto* offsets = reinterpret_cast<int32_t*>(b + L.offsets);
+    auto* mt_start = reinterpret_cast<int32_t*>(b + L.mt_start);
+    auto* Z = reinterpret_cast<float*>(b + L.Z);
+    auto* colmax = reinterpret_cast<float*>(b + L.colmax);
+    auto* colsum = reinterpret_cast<float*>(b + L.colsum);
+    auto* Dt = reinterpret_cast<__nv_bfloat16*>(b + L.Dt);
+    auto* Cw = reinterpret_cast<__nv_bfloat16*>(b + L.Cw);
+    auto* Xt = reinterpret_cast<__nv_bfloat16*>(b + L.Xt);
+    auto* S32 = reinterpret_cast<float*>(b + L.S32);
+    auto* Xs = reinterpret_cast<__nv_bfloat16*>(b + L.Xs);
+    auto* h = b + L.h;
+    auto* Yst = reinterpret_cast<__nv_bfloat16*>(b + L.Yst);
+    const int64_t N = p->N;
+    const int S = p->E_r * p->p;
+    const int d = p->d;
+    (void)cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(counters, 0, CNT_COUNT * 8, st);
+    if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward memset");
+    int status = MOE_OK;
+    // slot scores
+    e = launch_tc_dense(N, S, d, x, Phi, Z, counters, st, &status);
+    if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward scores (tcgen05)");
+    // dispatch weights (transposed) and combine weights
+    soft_colstat_kernel<<<(S + 31) / 32, 256, 0, st>>>(Z, N, S, colmax, colsum);
+    const dim3 tb(kT, 8);
+    soft_dispatch_t_kernel<<<dim3((unsigned)((N + kT - 1) / kT), (unsigned)((S + kT - 1) / kT)), tb, 0, st>>>(
+        Z, N, S, colmax, colsum, Dt);
+    soft_combine_w_kernel<<<(unsigned)((N + 7) / 8), 256, 0, st>>>(Z, N, S, Cw);
+    // slot inputs Xs = D^T X: X transposed so that K = tokens is contiguous
+    soft_transpose_kernel<__nv_bfloat16><<<dim3((unsigned)((N + kT - 1) / kT), (unsigned)((d + kT - 1) / kT)), tb,
+                                           0, st>>>(static_cast<const __nv_bfloat16*>(x), N, d, Xt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return soft_fail(e, "moe_soft_forward weights");
+    e = launch_tc_dense(S, d, N, Dt, Xt, S32, counters, st, &status);
+    if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward slot inputs (tcgen05)");
+    const int64_t n4 = (int64_t)S * d / 4;
+    soft_to_bf16_kernel<<<(unsigned)min64((n4 + 255) / 256, (int64_t)num_sms() * 8), 256, 0, st>>>(
+        reinterpret_cast<const float4*>(S32), reinterpret_cast<uint2*>(Xs), n4);
+    // experts on their slots: p consecutive slot rows per expert
+    moe_params q{};
+    q.N = S;
+    q.d = d;
+    q.d_f = p->d_f;
+    q.E_r = p->E_r;
+    q.k = 1;
+    q.dtype = MOE_BF16;
+    soft_offsets_kernel<<<1, 256, 0, st>>>(p->E_r, p->p, offsets);
+    if ((e = cudaGetLastError()) != cudaSuccess) return soft_fail(e, "moe_soft_forward slots");
+    e = launch_mtile_prefix(p->E_r, tc_tile_rows(q), offsets, mt_start, st);
+    if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward prefix");
+    ExpertWeights W{W_g, W_u, W_d, nullptr, nullptr, nullptr};
+    e = launch_tc_gate_up(q, Xs, nullptr, offsets, mt_start, W, h, nullptr, nullptr, counters, st, &status);
+    if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward gate/up (tcgen05)");
+    e = launch_tc_down(q, DOWN_STORE, S, h, nullptr, offsets, mt_start, W, nullptr, nullptr, nullptr, S32,
+                       counters, st, &status);
+    if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward down (tcgen05)");
+    // Y = C Ys: slot outputs transposed so that K = slots is contiguous
+    soft_transpose_kernel<float><<<dim3((unsigned)((S + kT - 1) / kT), (unsigned)((d + kT - 1) / kT)), tb, 0, st>>>(
+        S32, S, d, Yst);
+    if ((e = cudaGetLastError()) != cudaSuccess) return soft_fail(e, "moe_soft_forward transpose");
+    e = launch_tc_dense(N, d, S, Cw, Yst, Y, counters, st, &status);
+    if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward combine (tcgen05)");
+    return MOE_OK;
+}
+
+moe_status moe_soft_check(const moe_soft_params* p, const void* ws, moe_stream_t stream) {
+    moe_status s = soft_check(p);
+    if (s != MOE_OK) return s;
+    if (!ws) return MOE_ERR_WORKSPACE;
+    const SoftLayout L = soft_layout(*p);
+    unsigned long long cnt[CNT_COUNT];
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(cnt, static_cast<const char*>(ws) + L.counters, sizeof(cnt),
+                                    cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return soft_fail(e, "moe_soft_check");
+    if (cnt[CNT_DEVICE_ERROR] & DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -114,6 +114,25 @@ def test_acceptance_by_weight_is_refused_where_it_is_not_built():
                                   None) == moe.MOE_ERR_UNSUPPORTED
 
 
+def test_soft_moe_params_are_checked_on_the_host():
+    assert ctypes.sizeof(moe.SoftParams) == 32
+    L = moe.lib()
+    n = ctypes.c_size_t(0)
+    for kw, status in ((dict(dtype=moe.MOE_F32), moe.MOE_ERR_UNSUPPORTED),   # bf16 contractions only
+                       (dict(N=100), moe.MOE_ERR_UNSUPPORTED),                # 16-byte operand rows
+                       (dict(E_r=3, p=3), moe.MOE_ERR_UNSUPPORTED),           # S = 9 slots
+                       (dict(p=0), moe.MOE_ERR_INVALID_ARG),
+                       (dict(d=0), moe.MOE_ERR_INVALID_ARG)):
+        args = dict(N=64, d=64, d_f=32, E_r=8, p=2)
+        args.update(kw)
+        sp = moe.soft_params(**args)
+        assert L.moe_soft_workspace_size(ctypes.byref(sp), ctypes.byref(n)) == status, kw
+    sp = moe.soft_params(64, 64, 32, 8, 2)
+    assert L.moe_soft_workspace_size(ctypes.byref(sp), ctypes.byref(n)) == moe.MOE_OK and n.value > 0
+    assert L.moe_soft_forward(ctypes.byref(sp), None, None, None, None, None, None, None, None) == \
+        moe.MOE_ERR_WORKSPACE
+
+
 def test_status_strings():
     for s in range(7):
         assert moe.moe_status_string(s)

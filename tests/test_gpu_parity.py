@@ -307,6 +307,28 @@ def test_expert_choice(dtype, N, d, d_f, E, C):
 
 
 # ---------------------------------------------------------------------------
+# Soft MoE: slot mixing on the tensor cores, experts on their slots
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N,d,d_f,E,p", [(256, 128, 64, 4, 4), (512, 320, 192, 8, 16),
+                                         (1000, 256, 128, 3, 8), (1536, 128, 128, 2, 768)])
+def test_soft_moe(N, d, d_f, E, p):
+    w = W["mixtral_bf16"].scaled(f"soft_{N}_{E}_{p}", N=N, d=d, d_f=d_f, E=E, soft_p=p)
+    inp = {n: si.tensor(w, n) for n in ("x", "Phi", "W_g", "W_u", "W_d")}
+    dev = {n: parity.to_dev(v) for n, v in inp.items()}
+    sp = moe.soft_params(N, d, d_f, E, p)
+    ws = torch.empty(moe.moe_soft_workspace_size(sp), dtype=torch.uint8, device="cuda")
+    Y = torch.full((N, d), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_soft_forward(sp, dev["x"], dev["Phi"], dev["W_g"], dev["W_u"], dev["W_d"], Y, ws)
+    assert moe.moe_soft_check(sp, ws) == moe.MOE_OK
+    ref = oracle.soft_moe(inp["x"], inp["Phi"], inp["W_g"], inp["W_u"], inp["W_d"], p)
+    Yg = Y.cpu().numpy().astype(np.float64)
+    assert np.isfinite(Yg).all()
+    err = parity.rel_err(Yg, ref["Y"])
+    assert err <= parity.TOL[si.DT_BF16], err
+    print(f"soft MoE N={N} S={E * p}: max-abs-rel {err:.2e}")
+
+
+# ---------------------------------------------------------------------------
 # full-size page-shaped layers: every token's routing and dispatch, sampled outputs
 # ---------------------------------------------------------------------------
 def _sample_tokens(N, n, seed):
