@@ -279,6 +279,88 @@ def config_of(w: si.Workload, args):
 # ---------------------------------------------------------------------------
 # GPU leg
 # ---------------------------------------------------------------------------
+def run_gpu_soft(args):
+    """Soft MoE layer (one GPU): one step = moe_soft_forward over the batch."""
+    import torch
+    ws_n, rank, local = dist_env()
+    if ws_n > 1:
+        raise SystemExit("the Soft MoE layer mixes every token into every slot: one GPU only")
+    w = si.WORKLOADS[args.workload]
+    names = ("x", "Phi", "W_g", "W_u", "W_d")
+    inp = {n: si.tensor(w, n) for n in names}
+    torch.cuda.set_device(local)
+    import sparse_mixture_experts_25_b200 as moe
+    d = {n: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).cuda().view(torch.bfloat16)
+         for n, v in inp.items()}
+    sp = moe.soft_params(w.N, w.d, w.d_f, w.E, w.soft_p)
+    wsb = torch.empty(moe.moe_soft_workspace_size(sp), dtype=torch.uint8, device="cuda")
+    Y = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(x_dev, y_dev, ws_dev=wsb, st=stream):
+        moe.moe_soft_forward(sp, x_dev, d["Phi"], d["W_g"], d["W_u"], d["W_d"], y_dev, ws_dev, st)
+
+    for _ in range(args.warmup):
+        step(d["x"], Y)
+    if moe.moe_soft_check(sp, wsb) != moe.MOE_OK:
+        raise RuntimeError("moe_soft_forward: a device wait gave up")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        start.record(stream)
+        for _ in range(args.steps):
+            step(d["x"], Y)
+        end.record(stream)
+        torch.cuda.synchronize()
+        time.sleep(0.2)
+    ms_step = start.elapsed_time(end) / args.steps
+    # end to end with host buffers
+    from sparse_mixture_experts_25_b200.pipeline import HostPipeline
+    x_host = torch.from_numpy(np.ascontiguousarray(inp["x"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty(w.N, w.d, dtype=torch.float32).pin_memory()
+    pipe = HostPipeline(None, d, forward=lambda xd, yd, wsd, st: step(xd, yd, wsd, st),
+                        ws_bytes=moe.moe_soft_workspace_size(sp), shape=(w.N, w.d))
+    for _ in range(3):
+        pipe.submit(x_host, y_host)
+    pipe.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(pipe.h2d)
+    for _ in range(args.steps):
+        pipe.submit(x_host, y_host)
+    pipe.compute.wait_stream(pipe.d2h)
+    pipe.d2h.wait_stream(pipe.compute)
+    e1.record(pipe.d2h)
+    pipe.synchronize()
+    e_ms = e0.elapsed_time(e1) / args.steps
+    S = w.E * w.soft_p
+    flops = 2.0 * w.N * S * w.d * 3 + 2.0 * S * 3 * w.d * w.d_f   # scores, D^T X, C Ys; experts
+    peaks, peak_src = load_peaks()
+    peak_tf = peaks["bf16_tflops"] if ms_step * args.steps < 1000 else peaks.get("bf16_tflops_sustained",
+                                                                                   peaks["bf16_tflops"])
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": w.N / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64/Box-Muller; x~N(0,1), W~N(0,1/fan_in)); no dataset or checkpoint",
+        "config": {"workload": f"{w.name}: Soft MoE T={w.N} d={w.d} d_f={w.d_f} E_r={w.E} slots={S}",
+                   "T": w.N, "d": w.d, "d_f": w.d_f, "E_r": w.E, "slots_per_expert": w.soft_p,
+                   "seed": w.seed, "parallelism": "dp1",
+                   "l2": f"inputs larger than L2 ({input_bytes(w) / 1e9:.2f} GB of weights and x read every step)"},
+        "roofline": {"kernel": "whole Soft MoE step (three slot contractions + slot experts)", "bound": "tensor",
+                     "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                     "traffic": None, "peak_source": f"{peak_src} bf16", "flops_per_step": flops},
+        "e2e": {"value": w.N / (e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()), "ms_per_step": e_ms},
+        "gpu_launches": 13 * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -504,6 +586,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if si.WORKLOADS[args.workload].soft_p > 0:
+        return run_gpu_soft(args)
     return run_gpu(args)
 
 

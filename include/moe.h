@@ -349,8 +349,8 @@ MOE_API moe_status moe_set_stage_events(void* const* events, int n);
  * slot inputs and the slot outputs are bf16 operands of the tensor-core
  * contractions; the experts' hidden activations are bf16.
  * Constraints: dtype MOE_BF16 (fp32 soft layers are not built:
- * MOE_ERR_UNSUPPORTED); N, d, d_f and S multiples of 8 (16-byte operand rows;
- * else MOE_ERR_UNSUPPORTED).  Every token mixes into every slot, so this is
+ * MOE_ERR_UNSUPPORTED); N, d, d_f and S multiples of 8 (16-byte operand rows),
+ * N <= 65535 * 256 and S <= 65535 * 32 (else MOE_ERR_UNSUPPORTED).  Every token mixes into every slot, so this is
  * not causal across the batch.  Non-finite scores are not detected (they
  * propagate into Y).
  */

@@ -190,6 +190,12 @@ WORKLOADS = {
                                      norm=NORM_RENORM, d_f_shared=2048, seed=25003),
     "wdmoe_decode_bf16": Workload("wdmoe_decode_bf16", N=64, d=4096, d_f=14336, E=8, k=2,
                                   norm=NORM_WLR, theta=0.3, latency=True, seed=25004),
+    # routing variants on the Mixtral shape (the pages give no configuration for them):
+    # expert choice with C = N k / E_r for k = 2, and Soft MoE with S = N slots
+    "expert_choice_bf16": Workload("expert_choice_bf16", N=4096, d=4096, d_f=14336, E=8, k=8,
+                                   norm=NORM_FULLPROB, c=0.25, accept_order=1, seed=25005),
+    "soft_moe_bf16": Workload("soft_moe_bf16", N=4096, d=4096, d_f=14336, E=8, k=1, soft_p=512,
+                              seed=25006),
 }
 
 

@@ -15,7 +15,7 @@
 // experts run on the grouped tcgen05 GEMMs with p rows per expert (the slot
 // rows are already grouped by expert).  D, C, Xs and Ys enter the tensor cores
 // as bf16; scores, softmax statistics and every accumulation are fp32.
-// Small kernels: column statistics of Z (online max / sum per slot), the
+// Small kernels: column statistics of Z (per-chunk max / sum, merged), the
 // transposed dispatch weights, the row softmax, bf16 transposes in 32 x 32
 // shared-memory tiles, an fp32 -> bf16 conversion.
 #include <cuda_bf16.h>
@@ -28,41 +28,62 @@ namespace {
 
 constexpr int kT = 32;  // transpose tile
 
-// per slot s: m_s = max_t Z[t, s], l_s = sum_t exp(Z[t, s] - m_s); one block
-// per 32 slots, lane = slot, the 8 warps stride over the tokens
-__global__ void soft_colstat_kernel(const float* __restrict__ Z, int64_t N, int S, float* __restrict__ colmax,
-                                    float* __restrict__ colsum) {
+// Column statistics of Z in two steps.  Partial: one block per 32 slots x
+// 256 tokens; each warp takes 32 tokens (independent loads, lane = slot),
+// computes their max and sum of exp, and the 8 warps merge into one partial
+// (max, sum) per slot and chunk.  Merge: one thread per slot combines its
+// chunks into m_s = max_t Z[t, s] and l_s = sum_t exp(Z[t, s] - m_s).
+constexpr int kColChunk = 256;
+
+__global__ void soft_colstat_partial_kernel(const float* __restrict__ Z, int64_t N, int S,
+                                            float* __restrict__ pmax, float* __restrict__ psum) {
     __shared__ float sm[8][32], sl[8][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int s = blockIdx.x * 32 + lane;
-    float m = -INFINITY, l = 0.f;
-    if (s < S) {
-        for (int64_t t = warp; t < N; t += 8) {
-            const float z = Z[t * S + s];
-            if (l == 0.f) {
-                m = z;
-                l = 1.f;
-            } else if (z > m) {
-                l = l * expf(m - z) + 1.f;
-                m = z;
-            } else {
-                l += expf(z - m);
-            }
-        }
+    const int64_t t0 = (int64_t)blockIdx.y * kColChunk + warp * 32;
+    float v[32];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int64_t t = t0 + i;
+        v[i] = (s < S && t < N) ? Z[t * S + s] : -INFINITY;
+        m = fmaxf(m, v[i]);
+    }
+    float l = 0.f;
+    if (m != -INFINITY) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) l += expf(v[i] - m);
     }
     sm[warp][lane] = m;
     sl[warp][lane] = l;
     __syncthreads();
     if (warp == 0 && s < S) {
         float M = -INFINITY;
-        for (int w = 0; w < 8; ++w)
-            if (sl[w][lane] > 0.f) M = fmaxf(M, sm[w][lane]);
+        for (int w = 0; w < 8; ++w) M = fmaxf(M, sm[w][lane]);
         float L = 0.f;
-        for (int w = 0; w < 8; ++w)
-            if (sl[w][lane] > 0.f) L += sl[w][lane] * expf(sm[w][lane] - M);
-        colmax[s] = M;
-        colsum[s] = L;
+        if (M != -INFINITY)
+            for (int w = 0; w < 8; ++w)
+                if (sl[w][lane] > 0.f) L += sl[w][lane] * expf(sm[w][lane] - M);
+        pmax[(int64_t)blockIdx.y * S + s] = M;
+        psum[(int64_t)blockIdx.y * S + s] = L;
     }
+}
+
+__global__ void soft_colstat_merge_kernel(const float* __restrict__ pmax, const float* __restrict__ psum,
+                                          int n_chunks, int S, float* __restrict__ colmax,
+                                          float* __restrict__ colsum) {
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= S) return;
+    float M = -INFINITY;
+    for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, pmax[(int64_t)c * S + s]);
+    float L = 0.f;
+    if (M != -INFINITY)
+        for (int c = 0; c < n_chunks; ++c) {
+            const float l = psum[(int64_t)c * S + s];
+            if (l > 0.f) L += l * expf(pmax[(int64_t)c * S + s] - M);
+        }
+    colmax[s] = M;
+    colsum[s] = L;
 }
 
 // Dt[s, t] = exp(Z[t, s] - m_s) / l_s in bf16, written transposed through a
@@ -89,35 +110,40 @@ __global__ void soft_dispatch_t_kernel(const float* __restrict__ Z, int64_t N, i
     }
 }
 
-// C[t, s] = exp(Z[t, s] - m_t) / l_t in bf16; one warp per token
+// C[t, s] = exp(Z[t, s] - m_t) / l_t in bf16; one warp per token, three
+// passes over the token's row in 16-byte loads (max, sum of exp, write)
 __global__ void soft_combine_w_kernel(const float* __restrict__ Z, int64_t N, int S,
                                       __nv_bfloat16* __restrict__ Cw) {
     const int lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= N) return;
-    const float* z = Z + t * S;
-    float m = -INFINITY, l = 0.f;
-    for (int s = lane; s < S; s += 32) {
-        const float v = z[s];
-        if (l == 0.f) {
-            m = v;
-            l = 1.f;
-        } else if (v > m) {
-            l = l * expf(m - v) + 1.f;
-            m = v;
-        } else {
-            l += expf(v - m);
-        }
+    const float4* z = reinterpret_cast<const float4*>(Z + t * S);
+    const int S4 = S / 4;
+    float m = -INFINITY;
+#pragma unroll 4
+    for (int i = lane; i < S4; i += 32) {
+        const float4 v = z[i];
+        m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
     }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-        const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-        const float M = l2 > 0.f ? (l > 0.f ? fmaxf(m, m2) : m2) : m;
-        l = (l > 0.f ? l * expf(m - M) : 0.f) + (l2 > 0.f ? l2 * expf(m2 - M) : 0.f);
-        m = M;
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+#pragma unroll 4
+    for (int i = lane; i < S4; i += 32) {
+        const float4 v = z[i];
+        l += expf(v.x - m) + expf(v.y - m) + expf(v.z - m) + expf(v.w - m);
     }
-    for (int s = lane; s < S; s += 32) Cw[t * S + s] = __float2bfloat16_rn(expf(z[s] - m) / l);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    const float inv = 1.f / l;
+    uint2* out = reinterpret_cast<uint2*>(Cw + t * S);
+#pragma unroll 4
+    for (int i = lane; i < S4; i += 32) {
+        const float4 v = z[i];
+        __nv_bfloat162 a = __floats2bfloat162_rn(expf(v.x - m) * inv, expf(v.y - m) * inv);
+        __nv_bfloat162 b = __floats2bfloat162_rn(expf(v.z - m) * inv, expf(v.w - m) * inv);
+        out[i] = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+    }
 }
 
 // out[c, r] = in[r, c] for a row-major [R, Cc] input; bf16 -> bf16 or fp32 -> bf16
@@ -156,7 +182,7 @@ __global__ void soft_offsets_kernel(int E, int p, int32_t* __restrict__ offsets)
 }
 
 struct SoftLayout {
-    size_t counters, offsets, mt_start, Z, colmax, colsum, Dt, Cw, Xt, S32, Xs, h, Yst, total;
+    size_t counters, offsets, mt_start, Z, colmax, colsum, pmax, psum, Dt, Cw, Xt, S32, Xs, h, Yst, total;
 };
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -177,6 +203,8 @@ SoftLayout soft_layout(const moe_soft_params& p) {
     L.Z = take(N * S * 4);
     L.colmax = take(S * 4);
     L.colsum = take(S * 4);
+    L.pmax = take((N + kColChunk - 1) / kColChunk * S * 4);
+    L.psum = take((N + kColChunk - 1) / kColChunk * S * 4);
     L.Dt = take(S * N * 2);
     L.Cw = take(N * S * 2);
     L.Xt = take(d * N * 2);
@@ -197,7 +225,8 @@ moe_status soft_check(const moe_soft_params* p) {
     const int64_t S = (int64_t)p->E_r * p->p;
     // 16-byte rows for every tensor-core operand (K = d, tokens, slots)
     if (p->d % 8 || p->d_f % 8 || p->N % 8 || S % 8) return MOE_ERR_UNSUPPORTED;
-    if (p->N > (int64_t)1 << 30 || S > (int64_t)1 << 30) return MOE_ERR_UNSUPPORTED;
+    // grid limits of the column-statistics and transposition launches
+    if (p->N > (int64_t)65535 * kColChunk || S > (int64_t)65535 * kT) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 
@@ -260,7 +289,12 @@ moe_status moe_soft_forward(const moe_soft_params* p, const void* x, const void*
     e = launch_tc_dense(N, S, d, x, Phi, Z, counters, st, &status);
     if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward scores (tcgen05)");
     // dispatch weights (transposed) and combine weights
-    soft_colstat_kernel<<<(S + 31) / 32, 256, 0, st>>>(Z, N, S, colmax, colsum);
+    const int n_chunks = (int)((N + kColChunk - 1) / kColChunk);
+    soft_colstat_partial_kernel<<<dim3((unsigned)((S + 31) / 32), (unsigned)n_chunks), 256, 0, st>>>(
+        Z, N, S, reinterpret_cast<float*>(b + L.pmax), reinterpret_cast<float*>(b + L.psum));
+    soft_colstat_merge_kernel<<<(S + 255) / 256, 256, 0, st>>>(reinterpret_cast<const float*>(b + L.pmax),
+                                                                reinterpret_cast<const float*>(b + L.psum),
+                                                                n_chunks, S, colmax, colsum);
     const dim3 tb(kT, 8);
     soft_dispatch_t_kernel<<<dim3((unsigned)((N + kT - 1) / kT), (unsigned)((S + kT - 1) / kT)), tb, 0, st>>>(
         Z, N, S, colmax, colsum, Dt);

@@ -16,22 +16,26 @@ import sparse_mixture_experts_25_b200 as moe
 
 class HostPipeline:
     def __init__(self, p: "moe.Params", weights: dict, depth: int = 2, x_dtype=None, device="cuda",
-                 forward=None):
+                 forward=None, ws_bytes=None, shape=None):
         """weights: device tensors W_r, W_g, W_u, W_d and optionally b_r, lat,
         Ws_g, Ws_u, Ws_d (held fixed across batches).  forward(x, y, ws,
         stream), if given, replaces moe_forward (for example the sharded
-        forward of a multi-GPU routing group)."""
+        forward of a multi-GPU routing group, or the Soft MoE forward, which
+        passes p = None with its workspace bytes and the (N, d) shape)."""
         import torch
         self.torch = torch
         self.p = p
         self.w = weights
         self.forward = forward
         self.depth = depth
-        x_dtype = x_dtype or (torch.bfloat16 if p.dtype == moe.MOE_BF16 else torch.float32)
-        self.x = [torch.empty(p.N, p.d, dtype=x_dtype, device=device) for _ in range(depth)]
-        self.y = [torch.empty(p.N, p.d, dtype=torch.float32, device=device) for _ in range(depth)]
+        N, d = shape if shape is not None else (p.N, p.d)
+        bf16 = p is None or p.dtype == moe.MOE_BF16
+        x_dtype = x_dtype or (torch.bfloat16 if bf16 else torch.float32)
+        self.x = [torch.empty(N, d, dtype=x_dtype, device=device) for _ in range(depth)]
+        self.y = [torch.empty(N, d, dtype=torch.float32, device=device) for _ in range(depth)]
         # batches compute one after another on one stream, so one workspace serves all
-        self.ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device=device)
+        nbytes = ws_bytes if ws_bytes is not None else moe.moe_workspace_size(p)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.compute = torch.cuda.Stream(device=device)
         self.h2d = torch.cuda.Stream(device=device)
         self.d2h = torch.cuda.Stream(device=device)
