@@ -149,7 +149,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
     }
 }
 
-// Warp-collective bounded wait: every lane returns the same verdict, so the
+// Warp-collective bounded wait: every lane returns the same result, so the
 // .sync.aligned tcgen05 loads that follow are executed by the whole warp.
 __device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort_flag,
@@ -274,7 +274,8 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 
 // TMA load into this CTA's shared memory whose completion is counted on an
-// mbarrier that may live in the peer CTA of the pair (no multicast).
+// mbarrier that may live in the peer CTA of the pair (each CTA fetches only
+// the tiles it stores itself).
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
                                                  int c0, int c1) {
     asm volatile(
