@@ -271,6 +271,69 @@ def _route_dispatch_full(p, dev, w):
 
 
 # ---------------------------------------------------------------------------
+# the largest supported routing shapes
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("order", [0, 1])
+def test_dispatch_at_1024_experts_and_k_32(order):
+    """moe_dispatch with caller-given routing records at E_r = 1024 (the
+    dispatch limit) and k = 32 (the k limit), with pruned (-1) entries and a
+    binding capacity: records bit-exact against the oracle."""
+    N, k, E = 3000, 32, 1024
+    rng = np.random.default_rng(123 + order)
+    # skewed expert choice: low expert indices far more popular
+    pool = rng.zipf(1.3, size=(N, 4 * k)) % E
+    ids = np.full((N, k), -1, np.int32)
+    for t in range(N):
+        _, first = np.unique(pool[t], return_index=True)
+        uniq = pool[t][np.sort(first)][:k]
+        ids[t, :len(uniq)] = uniq
+    ids[rng.random((N, k)) < 0.1] = -1
+    w = rng.integers(1, 16, size=(N, k)).astype(np.float32) / 16.0   # coarse: many equal weights
+    p = moe.params(N, 64, 64, E, k, c=1.0, dtype=moe.MOE_BF16, accept_order=order)
+    C = moe.moe_capacity(p)
+    ws = torch.zeros(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+    d_ids, d_w = torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda()
+    slot = torch.empty(N, k, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    st = torch.empty(N * k, dtype=torch.int32, device="cuda")
+    sw = torch.empty(N * k, dtype=torch.float32, device="cuda")
+    moe.moe_dispatch(p, d_ids, d_w, C, slot, offsets, st, sw, None, None, ws)
+    status, stats = moe.moe_get_stats(p, ws)
+    assert status == moe.MOE_OK
+    if order:
+        ref = oracle.dispatch_priority(ids, w.astype(np.float64), E=E, C=C)
+    else:
+        ref = oracle.dispatch(ids, E=E, C=C)
+    assert ref["stats"]["rejected"] > 0
+    np.testing.assert_array_equal(slot.cpu().numpy(), ref["slot"])
+    offs = np.concatenate([[0], np.cumsum(ref["acc"])])
+    np.testing.assert_array_equal(offsets.cpu().numpy(), offs)
+    t_idx, j_idx = np.nonzero(ref["slot"] >= 0)
+    pos = offs[ids[t_idx, j_idx]] + ref["slot"][t_idx, j_idx]
+    np.testing.assert_array_equal(st.cpu().numpy()[pos], t_idx)
+    np.testing.assert_array_equal(sw.cpu().numpy()[pos], w[t_idx, j_idx])
+    for key in ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max"):
+        assert stats[key] == ref["stats"][key], key
+
+
+def test_router_at_256_experts_and_k_32():
+    """moe_route at E_r = 256 (the router limit) and k = 32, bf16 scores on
+    the tensor cores: ids exact off near-ties, weights within 3e-5."""
+    w = W["deepseek_shared_bf16"].scaled("router_256_k32", N=512, d=512, d_f=64, E=256, k=32, d_f_shared=0)
+    inp = si.inputs(w)
+    p = parity.params_of(w)
+    dev = {n: parity.to_dev(inp[n]) for n in ("x", "W_r")}
+    ws = torch.zeros(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+    ids = torch.empty(w.N, w.k, dtype=torch.int32, device="cuda")
+    wt = torch.empty(w.N, w.k, dtype=torch.float32, device="cuda")
+    margin = torch.empty(w.N, dtype=torch.float32, device="cuda")
+    moe.moe_route(p, dev["x"], dev["W_r"], None, None, ids, wt, margin, ws)
+    rec = {"ids": ids.cpu().numpy(), "w": wt.cpu().numpy(), "margin": margin.cpu().numpy()}
+    r, near = parity.check_routing(w, inp, rec)
+    assert near.sum() < w.N // 4
+
+
+# ---------------------------------------------------------------------------
 # expert-choice routing: k = E_r, full-softmax weights, acceptance by weight
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("dtype,N,d,d_f,E,C", [(si.DT_BF16, 512, 256, 192, 8, 96),
