@@ -44,7 +44,15 @@ def forward_sharded(p_local: "moe.Params", N_group: int, C: int, x, W_r, b_r, la
     if counts is None:
         counts = torch.empty(p_local.E_r, dtype=torch.int32, device=x.device)
     moe.moe_forward_begin(p_local, x, W_r, b_r, lat, counts, ws, stream)
-    counts_all = exchange_counts(counts, group)
+    # the exchange runs on the layer's stream, after the counts are written
+    if stream is None:
+        st = torch.cuda.current_stream(x.device)
+    elif isinstance(stream, int):
+        st = torch.cuda.ExternalStream(stream, device=x.device)
+    else:
+        st = stream
+    with torch.cuda.stream(st):
+        counts_all = exchange_counts(counts, group)
     moe.moe_forward_end(p_local, counts_all, dist.get_rank(group), dist.get_world_size(group),
                         N_group, C, x, W_g, W_u, W_d, Ws_g, Ws_u, Ws_d, Y, ws, stream)
     return counts_all

@@ -520,6 +520,46 @@ def test_sharded_group_two_ranks_on_one_gpu(name):
     assert parity.rel_err(np.concatenate(Ys), full["Y"]) <= 1e-6
 
 
+def test_forward_sharded_on_a_side_stream_one_rank():
+    """sharded.forward_sharded through a one-rank NCCL group, on a stream that
+    is not the current one: the count exchange is ordered after the counts
+    are written, and the result equals moe_forward."""
+    import os
+    import socket
+    import torch.distributed as dist
+    from sparse_mixture_experts_25_b200 import sharded
+    w = SMALL["qwen3_small_bf16"]
+    inp = si.inputs(w)
+    full = parity.gpu_forward(w, inp)
+    dev = full["dev"]
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("nccl", rank=0, world_size=1,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        p = parity.params_of(w)
+        C = moe.moe_capacity(p)
+        ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+        Y = torch.full((w.N, w.d), float("nan"), device="cuda")
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        counts_all = sharded.forward_sharded(p, w.N, C, dev["x"], dev["W_r"], dev.get("b_r"), dev.get("lat"),
+                                             dev["W_g"], dev["W_u"], dev["W_d"], None, None, None, Y, ws,
+                                             stream=side)
+        side.synchronize()
+        assert counts_all.shape == (1, w.E)
+        assert int(counts_all.sum()) == int(full["stats"]["requested"])
+        slot = moe.workspace_views(p, ws)["slot"].cpu().numpy()
+        np.testing.assert_array_equal(slot, full["rec"]["slot"])
+        assert parity.rel_err(Y.cpu().numpy().astype(np.float64), full["Y"]) <= 1e-6
+    finally:
+        dist.destroy_process_group()
+
+
 def test_host_pipeline_matches_direct_forward():
     """Batches streamed from pinned host memory through HostPipeline give the
     outputs of direct moe_forward calls, batch by batch."""
