@@ -271,6 +271,7 @@ def config_of(w: si.Workload, args):
             "parallelism": (f"dp{args.gpus}: one routing group of {w.N} x {args.gpus} tokens, "
                             "per-expert request counts all-gathered once per step"
                             if args.gpus > 1 else "dp1"),
+            "cuda_graph": bool(getattr(args, "graph", False)),
             "l2": (f"L2 flushed between timed steps (256 MiB write outside the per-step events); "
                    f"inputs {input_bytes(w) / 2**20:.1f} MiB" if flushes_l2(w) else
                    f"inputs larger than L2 ({input_bytes(w) / 1e9:.2f} GB of weights and x read every step)")}
@@ -431,12 +432,31 @@ def run_gpu(args):
         dist.barrier()
     torch.cuda.synchronize()
     flush = torch.empty(256 * 2**20 // 4, dtype=torch.int32, device="cuda") if flushes_l2(w) else None
+    graph = None
+    if args.graph and sharded_group:
+        raise SystemExit("--graph times one GPU's step; the sharded group exchanges counts between ranks")
+    if args.graph:
+        # one step captured into a CUDA graph and replayed (fewer launch gaps)
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            moe.moe_forward(p, d["x"], d["W_r"], d["b_r"], d["lat"], d["W_g"], d["W_u"], d["W_d"],
+                            d["Ws_g"], d["Ws_u"], d["Ws_d"], Y, wsb, cap)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         time.sleep(0.3)
         start.record(stream)
         for i in range(args.steps):
             if flush is not None:
                 flush.fill_(i)   # evict the layer's inputs from L2; outside the step's events
+            if graph is not None:
+                ev[i][0].record(stream)
+                graph.replay()
+                ev[i][4].record(stream)
+                continue
             moe.moe_set_stage_events(ev[i])
             step(d["x"], Y)
         moe.moe_set_stage_events([])
@@ -451,6 +471,13 @@ def run_gpu(args):
         ms_total = float(sum(ev[i][0].elapsed_time(ev[i][4]) for i in range(args.steps)))
     ms_total = max_over_ranks(ms_total, device="cuda")
     ms_step = ms_total / args.steps
+    if graph is not None:
+        # stage times from eager steps (a replay records no stage events)
+        for i in range(args.steps):
+            moe.moe_set_stage_events(ev[i])
+            step(d["x"], Y)
+        moe.moe_set_stage_events([])
+        torch.cuda.synchronize()
     stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(4)] for i in range(args.steps)])
     gate_up_ms = float(stage_ms[:, 2].mean())
     down_ms = float(stage_ms[:, 3].mean())
@@ -570,6 +597,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(si.WORKLOADS))
     ap.add_argument("--ref-sample", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of one step captured into a CUDA graph (one GPU)")
     ap.add_argument("--override", action="append", default=[],
                     help="key=value change of the workload shape (profiling of smaller cases)")
     args = ap.parse_args(argv)

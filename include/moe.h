@@ -275,6 +275,10 @@ MOE_API moe_status moe_combine(const moe_params* p, const float* H, const int32_
  * params.d_f_shared > 0.  Y [N, d] fp32 is overwritten.  Routing records
  * and statistics stay in the workspace (moe_workspace_layout, moe_get_stats).
  * Ws_g/Ws_u/Ws_d are required when d_f_shared > 0 and ignored otherwise.
+ * The call only enqueues kernels and memsets on `stream` (no host wait, no
+ * allocation), so it can be captured into a CUDA graph and replayed with new
+ * contents of the same buffers; make the first call on a device outside a
+ * capture (it sets the kernels' shared-memory attributes).
  */
 MOE_API moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, const float* b_r,
                        const float* lat, const void* W_g, const void* W_u, const void* W_d,

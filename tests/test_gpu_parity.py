@@ -560,6 +560,40 @@ def test_forward_sharded_on_a_side_stream_one_rank():
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("name", ["switch_small_f32", "mixtral_small_bf16", "pair_bf16", "weight_order_bf16"])
+def test_forward_replays_from_a_cuda_graph(name):
+    """moe_forward neither synchronises nor allocates, so a step can be
+    captured once into a CUDA graph and replayed: each replay on new inputs
+    equals the eager forward on them."""
+    w = SMALL[name]
+    inp = si.inputs(w)
+    ref = parity.gpu_forward(w, inp)
+    dev = ref["dev"]
+    p = parity.params_of(w)
+    ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+    x = dev["x"].clone()
+    Y = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):   # warm-up outside the capture (kernel attributes, tensor maps)
+        moe.moe_forward(p, x, dev["W_r"], dev.get("b_r"), dev.get("lat"), dev["W_g"], dev["W_u"], dev["W_d"],
+                        dev.get("Ws_g"), dev.get("Ws_u"), dev.get("Ws_d"), Y, ws, side)
+    side.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        moe.moe_forward(p, x, dev["W_r"], dev.get("b_r"), dev.get("lat"), dev["W_g"], dev["W_u"], dev["W_d"],
+                        dev.get("Ws_g"), dev.get("Ws_u"), dev.get("Ws_d"), Y, ws, side)
+    for shift in (0, 1):
+        x.copy_(torch.roll(dev["x"], shifts=shift, dims=0))
+        Y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        want = parity.gpu_forward(w, inp, dev=dict(dev, x=x.clone()))
+        np.testing.assert_array_equal(moe.workspace_views(p, ws)["slot"].cpu().numpy(), want["rec"]["slot"])
+        assert parity.rel_err(Y.cpu().numpy().astype(np.float64), want["Y"]) <= 1e-6
+    del g
+
+
 def test_host_pipeline_matches_direct_forward():
     """Batches streamed from pinned host memory through HostPipeline give the
     outputs of direct moe_forward calls, batch by batch."""
