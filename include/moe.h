@@ -339,6 +339,32 @@ MOE_API moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats*
 MOE_API moe_status moe_set_stage_events(void* const* events, int n);
 
 /*
+ * Dispatch step of a routing group sharded over ranks, on its own (the first
+ * half of moe_forward_end): after moe_forward_begin on this workspace and
+ * the exchange of the per-expert request counts (counts_all [n_ranks, E_r],
+ * ranks in token order), accepts this rank's requests by their group-wide
+ * token order, writes the routing records (slot, offsets, L, acc, slot_token,
+ * slot_w in the workspace) and gathers the accepted rows of x into x_perm
+ * (moe_workspace_layout), grouped by expert.  Used by expert parallelism
+ * ("LLM from scratch" ch. 36.7: experts placed on different devices, token
+ * rows sent to the device of their expert and the outputs sent back), where
+ * x_perm's expert blocks are what each rank sends.  Token-order acceptance
+ * only (MOE_ERR_UNSUPPORTED for MOE_ACCEPT_WEIGHT).
+ */
+MOE_API moe_status moe_dispatch_ranked(const moe_params* p, const int32_t* counts_all, int32_t rank,
+                                       int32_t n_ranks, int64_t N_group, int64_t C, const void* x, void* ws,
+                                       moe_stream_t stream);
+
+/*
+ * dst[i] = src[index[i]] for i < n_rows, rows of row_bytes bytes (a multiple
+ * of 16; 16-byte aligned src and dst): the regrouping of rows exchanged
+ * between ranks under expert parallelism (ch. 36.7).  No bounds checks on
+ * index beyond the caller's contract (0 <= index[i] < rows of src).
+ */
+MOE_API moe_status moe_gather_rows(const void* src, const int32_t* index, int64_t n_rows, int64_t row_bytes,
+                                   void* dst, moe_stream_t stream);
+
+/*
  * Soft MoE ("LLM from scratch" ch. 36.6, Soft Mixture of Experts): tokens are
  * mixed into S = E_r p slots, each expert processes its p slots, and the slot
  * outputs are mixed back into the tokens.

@@ -23,6 +23,7 @@ __all__ = [
     "moe_get_stats",
     "moe_set_stage_events", "moe_selftest_wait_timeout", "moe_status_string", "moe_last_error",
     "expert_choice_params", "SoftParams", "soft_params", "moe_soft_workspace_size", "moe_soft_forward",
+    "moe_dispatch_ranked", "moe_gather_rows", "workspace_x_perm",
     "moe_soft_check",
     "workspace_views", "HEADER",
 ]
@@ -112,6 +113,9 @@ def lib():
                                       ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(_P), ctypes.c_int]
         L.moe_selftest_wait_timeout.argtypes = [pp, _P, ctypes.c_int64, _P]
+        L.moe_dispatch_ranked.argtypes = [pp, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
+                                          ctypes.c_int64, _P, _P, _P]
+        L.moe_gather_rows.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int64, _P, _P]
         sp = ctypes.POINTER(SoftParams)
         L.moe_soft_workspace_size.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t)]
         L.moe_soft_forward.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P]
@@ -125,7 +129,7 @@ def lib():
                      "moe_forward",
                      "moe_get_stats", "moe_set_stage_events", "moe_forward_begin",
                      "moe_forward_end", "moe_selftest_wait_timeout", "moe_soft_workspace_size",
-                     "moe_soft_forward", "moe_soft_check"):
+                     "moe_soft_forward", "moe_soft_check", "moe_dispatch_ranked", "moe_gather_rows"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -266,6 +270,21 @@ def moe_get_stats(p, ws, stream=None):
     return status, s.as_dict()
 
 
+def moe_dispatch_ranked(p, counts_all, rank: int, n_ranks: int, N_group: int, C: int, x, ws, stream=None):
+    """Dispatch of a sharded routing group into the workspace (after
+    moe_forward_begin and the count exchange)."""
+    _check(lib().moe_dispatch_ranked(ctypes.byref(p), _ptr(counts_all), int(rank), int(n_ranks), int(N_group),
+                                     int(C), _ptr(x), _ptr(ws), _stream(stream)), "moe_dispatch_ranked")
+
+
+def moe_gather_rows(src, index, dst, stream=None):
+    """dst[i] = src[index[i]] for the rows of index (device tensors)."""
+    n = int(index.numel())
+    row_bytes = src[0].numel() * src.element_size() if src.dim() > 1 else src.element_size()
+    _check(lib().moe_gather_rows(_ptr(src), _ptr(index), n, int(row_bytes), _ptr(dst), _stream(stream)),
+           "moe_gather_rows")
+
+
 def moe_soft_workspace_size(sp) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().moe_soft_workspace_size(ctypes.byref(sp), ctypes.byref(n)), "moe_soft_workspace_size")
@@ -323,3 +342,14 @@ def workspace_views(p: Params, ws):
         "slot_token": view("slot_token", N * k, torch.int32, (N * k,)),
         "slot_w": view("slot_w", N * k, torch.float32, (N * k,)),
     }
+
+
+def workspace_x_perm(p: Params, ws):
+    """The gathered rows x_perm [N k, d] inside a workspace tensor (accepted
+    rows first, grouped by expert as offsets says)."""
+    import torch
+    L = moe_workspace_layout(p)
+    dt = torch.bfloat16 if p.dtype == MOE_BF16 else torch.float32
+    n = p.N * p.k * p.d
+    nbytes = n * torch.empty((), dtype=dt).element_size()
+    return ws[L["x_perm"]:L["x_perm"] + nbytes].view(dt).view(p.N * p.k, p.d)

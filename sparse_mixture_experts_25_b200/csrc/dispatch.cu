@@ -455,6 +455,17 @@ __global__ void gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ x
     }
 }
 
+// dst[i] = src[index[i]], rows of row_vec 16-byte words (expert-parallel
+// regrouping of exchanged rows)
+__global__ void gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ index, int64_t n,
+                                   int row_vec, uint4* __restrict__ dst) {
+    for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
+        const uint4* a = src + (int64_t)index[r] * row_vec;
+        uint4* b = dst + r * row_vec;
+        for (int i = threadIdx.x; i < row_vec; i += blockDim.x) b[i] = a[i];
+    }
+}
+
 __global__ void combine_kernel(const float* __restrict__ H, const int32_t* __restrict__ offsets,
                                int E, const int32_t* __restrict__ slot_token,
                                const float* __restrict__ slot_w, float* Y, int d, int64_t N,
@@ -597,6 +608,14 @@ cudaError_t launch_dispatch_ranked(const moe_params& p, int64_t C, int bm, const
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+cudaError_t launch_gather_rows(const void* src, const int32_t* index, int64_t n_rows, int64_t row_bytes, void* dst,
+                               cudaStream_t st) {
+    const int blocks = (int)min64(n_rows, (int64_t)num_sms() * 8);
+    gather_rows_kernel<<<blocks, 128, 0, st>>>(static_cast<const uint4*>(src), index, n_rows, (int)(row_bytes / 16),
+                                               static_cast<uint4*>(dst));
+    return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const moe_params& p, const float* H, const int32_t* offsets,

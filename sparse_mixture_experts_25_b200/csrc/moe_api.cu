@@ -463,6 +463,46 @@ moe_status moe_forward_begin(const moe_params* p, const void* x, const void* W_r
     return MOE_OK;
 }
 
+moe_status moe_dispatch_ranked(const moe_params* p, const int32_t* counts_all, int32_t rank, int32_t n_ranks,
+                               int64_t N_group, int64_t C, const void* x, void* ws, moe_stream_t stream) {
+    moe_status s = check_params(p);
+    if (s != MOE_OK) return s;
+    if (p->accept_order == MOE_ACCEPT_WEIGHT) return MOE_ERR_UNSUPPORTED;  // needs every rank's weights
+    if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (n_ranks < 1 || rank < 0 || rank >= n_ranks || !counts_all || C < 1 || N_group < p->N)
+        return MOE_ERR_INVALID_ARG;
+    if (p->N == 0) return MOE_OK;
+    if (!x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    WsView v;
+    make_view(*p, ws, v);
+    (void)cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(v.counters + CNT_REQUESTED, 0, 6 * 8, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(v.counters + CNT_L_MAX, 0, 2 * 8, st);
+    if (e != cudaSuccess) return fail(e, "moe_dispatch_ranked memset");
+    const int bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
+    const char* where = "";
+    e = launch_dispatch_ranked(*p, C, bm, counts_all, rank, n_ranks, N_group, v.ids, v.w, v.slot, v.offsets, v.L,
+                               v.acc, v.slot_token, v.slot_w, x, v.x_perm, v.counters, v.scratch, st, &where);
+    if (e != cudaSuccess) {
+        char buf[96];
+        snprintf(buf, sizeof(buf), "moe_dispatch_ranked %s", where);
+        return fail(e, buf);
+    }
+    return MOE_OK;
+}
+
+moe_status moe_gather_rows(const void* src, const int32_t* index, int64_t n_rows, int64_t row_bytes, void* dst,
+                           moe_stream_t stream) {
+    if (n_rows < 0 || row_bytes <= 0 || row_bytes % 16) return MOE_ERR_INVALID_ARG;
+    if (n_rows == 0) return MOE_OK;
+    if (!src || !index || !dst || !aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID_ARG;
+    (void)cudaGetLastError();
+    cudaError_t e = launch_gather_rows(src, index, n_rows, row_bytes, dst, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(e, "moe_gather_rows");
+    return MOE_OK;
+}
+
 moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32_t rank,
                            int32_t n_ranks, int64_t N_group, int64_t C, const void* x,
                            const void* W_g, const void* W_u, const void* W_d, const void* Ws_g,

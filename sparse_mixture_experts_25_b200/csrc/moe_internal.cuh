@@ -139,6 +139,8 @@ int tc_tile_rows(const moe_params& p);
 // of K elements (K % 8 == 0, 16-byte aligned bases), tcgen05 tiles of 128 x 256
 cudaError_t launch_tc_dense(int64_t M, int64_t Nc, int64_t K, const void* A, const void* B, float* out,
                             unsigned long long* counters, cudaStream_t st, int* status);
+cudaError_t launch_gather_rows(const void* src, const int32_t* index, int64_t n_rows, int64_t row_bytes, void* dst,
+                               cudaStream_t st);
 cudaError_t launch_wait_selftest(unsigned long long* counters, unsigned long long limit_ns, cudaStream_t st);
 // router scores G = x W_r^T (bf16 in, fp32 out [N, E_r]) on the tensor cores
 cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,
