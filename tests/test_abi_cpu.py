@@ -133,6 +133,23 @@ def test_soft_moe_params_are_checked_on_the_host():
         moe.MOE_ERR_WORKSPACE
 
 
+def test_ranked_dispatch_and_row_gather_check_arguments_on_the_host():
+    L = moe.lib()
+    p = moe.params(16, 64, 64, 8, 2, c=1.0)
+    # rank out of range, missing counts, C < 1, a group smaller than the shard
+    for rank, n_ranks, counts, N_group, C in ((2, 2, 16, 32, 4), (0, 2, None, 32, 4), (0, 2, 16, 32, 0),
+                                              (0, 2, 16, 8, 4)):
+        r = L.moe_dispatch_ranked(ctypes.byref(p), counts, rank, n_ranks, N_group, C, 16, 256, None)
+        assert r == moe.MOE_ERR_INVALID_ARG, (rank, n_ranks, counts, N_group, C)
+    assert L.moe_dispatch_ranked(ctypes.byref(p), 16, 0, 2, 32, 4, 16, None, None) == moe.MOE_ERR_WORKSPACE
+    pw = moe.params(16, 64, 64, 8, 2, c=1.0, accept_order=moe.MOE_ACCEPT_WEIGHT)
+    assert L.moe_dispatch_ranked(ctypes.byref(pw), 16, 0, 2, 32, 4, 16, 256, None) == moe.MOE_ERR_UNSUPPORTED
+    # row sizes must be whole 16-byte words; nothing to do for zero rows
+    assert L.moe_gather_rows(16, 16, 4, 24, 16, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_gather_rows(16, 16, -1, 32, 16, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_gather_rows(None, None, 0, 32, None, None) == moe.MOE_OK
+
+
 def test_status_strings():
     for s in range(7):
         assert moe.moe_status_string(s)
