@@ -16,7 +16,7 @@
 // rows are already grouped by expert).  D, C, Xs and Ys enter the tensor cores
 // as bf16; scores, softmax statistics and every accumulation are fp32.
 // Small kernels: column statistics of Z (per-chunk max / sum, merged), the
-// transposed dispatch weights, the row softmax, bf16 transposes in 32 x 32
+// transposed dispatch weights, the row softmax, bf16 transposes in 64 x 64
 // shared-memory tiles, an fp32 -> bf16 conversion.
 #include <cuda_bf16.h>
 #include <stdio.h>
@@ -26,7 +26,7 @@
 namespace moe {
 namespace {
 
-constexpr int kT = 32;  // transpose tile
+constexpr int kT = 32;  // grid limit unit of the slot dimension
 
 // Column statistics of Z in two steps.  Partial: one block per 32 slots x
 // 256 tokens; each warp takes 32 tokens (independent loads, lane = slot),
@@ -86,30 +86,6 @@ __global__ void soft_colstat_merge_kernel(const float* __restrict__ pmax, const 
     colsum[s] = L;
 }
 
-// Dt[s, t] = exp(Z[t, s] - m_s) / l_s in bf16, written transposed through a
-// 32 x 32 shared-memory tile (reads and writes coalesced)
-__global__ void soft_dispatch_t_kernel(const float* __restrict__ Z, int64_t N, int S,
-                                       const float* __restrict__ colmax, const float* __restrict__ colsum,
-                                       __nv_bfloat16* __restrict__ Dt) {
-    __shared__ float tile[kT][kT + 1];
-    const int64_t t0 = (int64_t)blockIdx.x * kT;
-    const int s0 = blockIdx.y * kT;
-    const int tx = threadIdx.x, ty = threadIdx.y;
-    for (int r = ty; r < kT; r += blockDim.y) {
-        const int64_t t = t0 + r;
-        const int s = s0 + tx;
-        float v = 0.f;
-        if (t < N && s < S) v = expf(Z[t * S + s] - colmax[s]) / colsum[s];
-        tile[r][tx] = v;
-    }
-    __syncthreads();
-    for (int r = ty; r < kT; r += blockDim.y) {
-        const int s = s0 + r;
-        const int64_t t = t0 + tx;
-        if (s < S && t < N) Dt[(int64_t)s * N + t] = __float2bfloat16_rn(tile[tx][r]);
-    }
-}
-
 // C[t, s] = exp(Z[t, s] - m_t) / l_t in bf16; one warp per token, three
 // passes over the token's row in 16-byte loads (max, sum of exp, write)
 __global__ void soft_combine_w_kernel(const float* __restrict__ Z, int64_t N, int S,
@@ -146,26 +122,69 @@ __global__ void soft_combine_w_kernel(const float* __restrict__ Z, int64_t N, in
     }
 }
 
-// out[c, r] = in[r, c] for a row-major [R, Cc] input; bf16 -> bf16 or fp32 -> bf16
-template <typename Tin>
-__global__ void soft_transpose_kernel(const Tin* __restrict__ in, int64_t R, int64_t Cc,
-                                      __nv_bfloat16* __restrict__ out) {
-    __shared__ float tile[kT][kT + 1];
-    const int64_t r0 = (int64_t)blockIdx.x * kT, c0 = (int64_t)blockIdx.y * kT;
-    const int tx = threadIdx.x, ty = threadIdx.y;
-    for (int i = ty; i < kT; i += blockDim.y) {
-        const int64_t r = r0 + i, c = c0 + tx;
-        float v = 0.f;
+// out[c, r] = f(in[r, c]) in bf16 for a row-major [R, Cc] input (R, Cc
+// multiples of 8): 64 x 64 tiles through shared memory, every global access a
+// 16-byte chunk of 8 elements (a warp covers four 128-byte row segments).
+// SOFTMAX: f(z) = exp(z - colmax[c]) / colsum[c] (the dispatch weights, read
+// from the scores), else the identity.
+constexpr int kTT = 64;
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+template <typename Tin, bool SOFTMAX>
+__global__ void __launch_bounds__(256) soft_transpose_kernel(const Tin* __restrict__ in, int64_t R, int64_t Cc,
+                                                             const float* __restrict__ colmax,
+                                                             const float* __restrict__ colsum,
+                                                             __nv_bfloat16* __restrict__ out) {
+    __shared__ float tile[kTT][kTT + 1];
+    const int64_t r0 = (int64_t)blockIdx.x * kTT, c0 = (int64_t)blockIdx.y * kTT;
+    const int t = threadIdx.x;
+    const int cc = (t & 7) * 8;  // chunk column inside the tile
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int rr = (t >> 3) + h * 32;
+        const int64_t r = r0 + rr, c = c0 + cc;
+        float v[8];
         if (r < R && c < Cc) {
-            if constexpr (sizeof(Tin) == 2) v = __bfloat162float(in[r * Cc + c]);
-            else v = in[r * Cc + c];
+            load8(in + r * Cc + c, v);
+            if (SOFTMAX) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = expf(v[i] - colmax[c + i]) / colsum[c + i];
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = 0.f;
         }
-        tile[i][tx] = v;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tile[rr][cc + i] = v[i];
     }
     __syncthreads();
-    for (int i = ty; i < kT; i += blockDim.y) {
-        const int64_t c = c0 + i, r = r0 + tx;
-        if (c < Cc && r < R) out[c * R + r] = __float2bfloat16_rn(tile[tx][i]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int oc = (t >> 3) + h * 32;   // output row = input column
+        const int64_t c = c0 + oc, r = r0 + cc;
+        if (c < Cc && r < R) {
+            uint4 q;
+            __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(&q);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = __floats2bfloat162_rn(tile[cc + 2 * i][oc], tile[cc + 2 * i + 1][oc]);
+            *reinterpret_cast<uint4*>(out + c * R + r) = q;
+        }
     }
 }
 
@@ -295,13 +314,13 @@ moe_status moe_soft_forward(const moe_soft_params* p, const void* x, const void*
     soft_colstat_merge_kernel<<<(S + 255) / 256, 256, 0, st>>>(reinterpret_cast<const float*>(b + L.pmax),
                                                                 reinterpret_cast<const float*>(b + L.psum),
                                                                 n_chunks, S, colmax, colsum);
-    const dim3 tb(kT, 8);
-    soft_dispatch_t_kernel<<<dim3((unsigned)((N + kT - 1) / kT), (unsigned)((S + kT - 1) / kT)), tb, 0, st>>>(
-        Z, N, S, colmax, colsum, Dt);
+    soft_transpose_kernel<float, true><<<dim3((unsigned)((N + kTT - 1) / kTT), (unsigned)((S + kTT - 1) / kTT)),
+                                         256, 0, st>>>(Z, N, S, colmax, colsum, Dt);
     soft_combine_w_kernel<<<(unsigned)((N + 7) / 8), 256, 0, st>>>(Z, N, S, Cw);
     // slot inputs Xs = D^T X: X transposed so that K = tokens is contiguous
-    soft_transpose_kernel<__nv_bfloat16><<<dim3((unsigned)((N + kT - 1) / kT), (unsigned)((d + kT - 1) / kT)), tb,
-                                           0, st>>>(static_cast<const __nv_bfloat16*>(x), N, d, Xt);
+    soft_transpose_kernel<__nv_bfloat16, false><<<dim3((unsigned)((N + kTT - 1) / kTT),
+                                                        (unsigned)((d + kTT - 1) / kTT)), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), N, d, nullptr, nullptr, Xt);
     if ((e = cudaGetLastError()) != cudaSuccess) return soft_fail(e, "moe_soft_forward weights");
     e = launch_tc_dense(S, d, N, Dt, Xt, S32, counters, st, &status);
     if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward slot inputs (tcgen05)");
@@ -327,8 +346,8 @@ moe_status moe_soft_forward(const moe_soft_params* p, const void* x, const void*
                        counters, st, &status);
     if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward down (tcgen05)");
     // Y = C Ys: slot outputs transposed so that K = slots is contiguous
-    soft_transpose_kernel<float><<<dim3((unsigned)((S + kT - 1) / kT), (unsigned)((d + kT - 1) / kT)), tb, 0, st>>>(
-        S32, S, d, Yst);
+    soft_transpose_kernel<float, false><<<dim3((unsigned)((S + kTT - 1) / kTT), (unsigned)((d + kTT - 1) / kTT)),
+                                          256, 0, st>>>(S32, S, d, nullptr, nullptr, Yst);
     if ((e = cudaGetLastError()) != cudaSuccess) return soft_fail(e, "moe_soft_forward transpose");
     e = launch_tc_dense(N, d, S, Cw, Yst, Y, counters, st, &status);
     if (e != cudaSuccess) return soft_fail(e, "moe_soft_forward combine (tcgen05)");
