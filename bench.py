@@ -355,7 +355,7 @@ def run_gpu_soft(args):
         "e2e": {"value": w.N / (e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()), "ms_per_step": e_ms},
-        "gpu_launches": 13 * args.steps,
+        "gpu_launches": 14 * args.steps,   # scores, 2 column-statistics, dispatch weights, combine weights, x transpose, slot inputs, bf16, offsets, prefix, gate/up, down, transpose, combine
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
