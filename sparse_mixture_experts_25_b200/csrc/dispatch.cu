@@ -543,10 +543,10 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
                                                              slot, sc.seg_req, sc.seg_w, counters);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         *where = "select";
-        prio_select_kernel<<<E, 256, 0, st>>>(C, sc.all_offsets, sc.seg_w, sc.sel_key, sc.sel_take);
+        prio_select_kernel<<<E, 1024, 0, st>>>(C, sc.all_offsets, sc.seg_w, sc.sel_key, sc.sel_take);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         *where = "number";
-        prio_scatter_kernel<<<E, 256, 0, st>>>(k, C, sc.all_offsets, offsets, sc.seg_req, sc.seg_w, sc.sel_key,
+        prio_scatter_kernel<<<E, 1024, 0, st>>>(k, C, sc.all_offsets, offsets, sc.seg_req, sc.seg_w, sc.sel_key,
                                               sc.sel_take, w, slot, slot_token, slot_w);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         *where = "tokens";
