@@ -136,6 +136,12 @@ typedef struct moe_stats {
     int64_t padded_rows;     /* rows the routed expert GEMMs compute: each expert's
                                 accepted rows rounded up to the GEMM's row tile    */
     double padding_ratio;    /* padded_rows / accepted (0 when nothing accepted)  */
+    double aux_balance;      /* E_r sum_e f_e pbar_e ("LLM from scratch" ch. 36.4
+                                balance objective, value only): f_e = L_e / sum L,
+                                the requests' shares before capacity; pbar_e = the
+                                mean full-softmax probability over the tokens with
+                                finite scores (this rank's tokens in a sharded
+                                group); 1 when both are uniform                    */
 } moe_stats;
 
 /* Byte offsets of the regions inside the workspace (for inspection and

@@ -416,5 +416,27 @@ def _as_f64(a):
     return a.astype(np.float64)
 
 
+def aux_balance(logits, ids, E: int, invalid=None) -> float:
+    """The balance objective's value ("LLM from scratch" ch. 36.4, Switch's
+    product of hard assignment shares and mean probabilities, top-k form):
+    E_r sum_e f_e pbar_e with f_e = n_e / sum n (requests per expert before
+    capacity; both f and pbar sum to one) and pbar_e the mean over the tokens
+    with finite scores of the full-softmax probability p_te.  It equals one
+    when both are uniform."""
+    G = np.asarray(logits, np.float64)
+    ok = ~np.asarray(invalid, bool) if invalid is not None else np.isfinite(G).all(axis=1)
+    if not ok.any():
+        return 0.0
+    Gv = G[ok]
+    P = np.exp(Gv - Gv.max(axis=1, keepdims=True))
+    P /= P.sum(axis=1, keepdims=True)
+    pbar = P.sum(axis=0) / ok.sum()
+    ids = np.asarray(ids)
+    n = np.bincount(ids[ids >= 0], minlength=E).astype(np.float64)
+    if n.sum() == 0:
+        return 0.0
+    return float(E * ((n / n.sum()) * pbar).sum())
+
+
 def round_bf16(v: float) -> float:
     return _load().oracle_round_bf16(float(v))

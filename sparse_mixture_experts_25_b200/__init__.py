@@ -72,7 +72,8 @@ class Stats(ctypes.Structure):
         "nonfinite", "near_tie", "L_max", "L_p50", "L_p90", "L_p99")] + [
         ("rho_max", ctypes.c_double), ("reject_rate", ctypes.c_double),
         ("device_error", ctypes.c_int32), ("reserved", ctypes.c_int32),
-        ("padded_rows", ctypes.c_int64), ("padding_ratio", ctypes.c_double)]
+        ("padded_rows", ctypes.c_int64), ("padding_ratio", ctypes.c_double),
+        ("aux_balance", ctypes.c_double)]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_ if n != "reserved"}

@@ -64,7 +64,8 @@ static bool layout(const moe_params& p, moe_ws_layout& L, int& n_tiles, int& til
     // then (256-byte aligned) router scores, then the acceptance-by-weight
     // arrays (all-request offsets, selected keys and counts, requests, weights)
     L.scratch = take(align_up(E * (size_t)std::max(n_tiles, 1) * 4 + (E + 1) * 4 + E * 4, 256) +
-                     align_up((size_t)p.N * E * 4, 256) + align_up((3 * E + 1) * 4, 256) + 2 * Nk * 4);
+                     align_up((size_t)p.N * E * 4, 256) + align_up((3 * E + 1) * 4, 256) + align_up(2 * Nk * 4, 256) +
+                     E * 4);
     L.total = off;
     return true;
 }
@@ -103,6 +104,7 @@ bool make_view(const moe_params& p, void* ws, WsView& v) {
         pr += align_up((3 * (size_t)p.E_r + 1) * 4, 256);
         v.scratch.seg_req = reinterpret_cast<int32_t*>(pr);
         v.scratch.seg_w = reinterpret_cast<float*>(pr + Nk * 4);
+        v.scratch.psum = reinterpret_cast<float*>(pr + align_up(2 * Nk * 4, 256));
     }
     v.scratch.n_tiles = n_tiles;
     v.scratch.tile_tokens = tile_tokens;
@@ -270,9 +272,10 @@ moe_status moe_route(const moe_params* p, const void* x, const void* W_r, const 
     make_view(*p, ws, v);
     (void)cudaGetLastError();
     cudaError_t e = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(v.scratch.psum, 0, sizeof(float) * p->E_r, st);
     if (e != cudaSuccess) return fail(e, "moe_route memset");
     return cuda_status(launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, ids,
-                                     w, margin, v.counters, nullptr, v.scratch.logits, st),
+                                     w, margin, v.counters, nullptr, v.scratch.logits, v.scratch.psum, st),
                        "moe_route router");
 }
 
@@ -379,6 +382,7 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     cudaError_t e0;
     if (p->N > 0 && (e0 = stage_mark(0, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     e0 = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
+    if (e0 == cudaSuccess) e0 = cudaMemsetAsync(v.scratch.psum, 0, sizeof(float) * p->E_r, st);
     if (e0 != cudaSuccess) return fail(e0, "moe_forward memset");
     if (p->N == 0) return MOE_OK;
     if (!x || !W_r || !W_g || !W_u || !W_d || !Y) return MOE_ERR_INVALID_ARG;
@@ -396,7 +400,8 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     // tile); fp32 layers zero it in the router
     const bool bf16 = p->dtype == MOE_BF16;
     cudaError_t e = launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, v.ids,
-                                  v.w, v.margin, v.counters, bf16 ? nullptr : Y, v.scratch.logits, st);
+                                  v.w, v.margin, v.counters, bf16 ? nullptr : Y, v.scratch.logits,
+                                  v.scratch.psum, st);
     if (e != cudaSuccess) return fail(e, "moe_forward router");
     if ((e0 = stage_mark(1, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     const int bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
@@ -444,6 +449,7 @@ moe_status moe_forward_begin(const moe_params* p, const void* x, const void* W_r
     cudaError_t e;
     if (p->N > 0 && (e = stage_mark(0, st)) != cudaSuccess) return fail(e, "moe_forward_begin stage event");
     e = cudaMemsetAsync(v.counters, 0, CNT_COUNT * 8, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(v.scratch.psum, 0, sizeof(float) * p->E_r, st);
     if (e != cudaSuccess) return fail(e, "moe_forward_begin memset");
     if (p->N == 0) {
         if (counts) {
@@ -455,7 +461,7 @@ moe_status moe_forward_begin(const moe_params* p, const void* x, const void* W_r
     if (!x || !W_r || !aligned16(x) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
     if (p->norm == MOE_NORM_WLR && !lat) return MOE_ERR_INVALID_ARG;
     e = launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, v.ids, v.w, v.margin,
-                      v.counters, nullptr, v.scratch.logits, st);
+                      v.counters, nullptr, v.scratch.logits, v.scratch.psum, st);
     if (e != cudaSuccess) return fail(e, "moe_forward_begin router");
     if ((e = stage_mark(1, st)) != cudaSuccess) return fail(e, "moe_forward_begin stage event");
     e = launch_count(*p, v.ids, v.L, counts, v.counters, v.scratch, st);
@@ -588,12 +594,15 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
     make_view(*p, const_cast<void*>(ws), v);
     unsigned long long cnt[CNT_COUNT];
     std::vector<int32_t> L((size_t)p->E_r), acc((size_t)p->E_r);
+    std::vector<float> psum((size_t)p->E_r);
     memset(out, 0, sizeof(*out));
     cudaError_t e = cudaMemcpyAsync(cnt, v.counters, sizeof(cnt), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(L.data(), v.L, sizeof(int32_t) * L.size(), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(acc.data(), v.acc, sizeof(int32_t) * acc.size(), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(psum.data(), v.scratch.psum, sizeof(float) * psum.size(), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return fail(e, "moe_get_stats");
     out->C = (int64_t)cnt[CNT_C];
@@ -631,6 +640,16 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
         }
         out->padded_rows = padded;
         out->padding_ratio = accepted ? (double)padded / (double)accepted : 0.0;
+        // balance statistic: E_r sum_e f_e pbar_e, f_e = L_e / sum L (requests
+        // before capacity), pbar_e = mean full-softmax probability over the
+        // tokens with finite scores
+        const double n_valid = (double)(p->N - (int64_t)cnt[CNT_NONFINITE]);
+        double req = 0.0;
+        for (int32_t l : L) req += l;
+        double aux = 0.0;
+        if (req > 0 && n_valid > 0)
+            for (int e2 = 0; e2 < p->E_r; ++e2) aux += ((double)L[e2] / req) * ((double)psum[e2] / n_valid);
+        out->aux_balance = aux * p->E_r;
     }
     if (cnt[CNT_DEVICE_ERROR] & DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
     if (cnt[CNT_NONFINITE]) return MOE_ERR_NONFINITE;

@@ -51,6 +51,7 @@ struct Scratch {
     int32_t* sel_take;    // [E] requests with exactly that key to accept
     int32_t* seg_req;     // [N k] requests grouped by expert, token order (acceptance by weight)
     float* seg_w;         // [N k] their routing weights
+    float* psum;          // [E] sum over tokens of the full-softmax probabilities
     int n_tiles;          // dispatch tiles
     int tile_tokens;      // tokens per dispatch tile
 };
@@ -85,9 +86,10 @@ bool make_view(const moe_params& p, void* ws, WsView& v);
 // ---------------------------------------------------------------------------
 // router.cu
 // logits: [N, E_r] fp32 scratch for the tensor-core score path (may be null)
+// psum: [E_r] fp32 sums of the full-softmax probabilities, accumulated (may be null)
 cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, const float* b_r,
                           const float* lat, int32_t* ids, float* w, float* margin,
-                          unsigned long long* counters, float* Y_zero, float* logits,
+                          unsigned long long* counters, float* Y_zero, float* logits, float* psum,
                           cudaStream_t st);
 // dispatch.cu
 cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_t* ids,

@@ -36,6 +36,7 @@ struct RouterArgs {
     float* margin;
     unsigned long long* counters;
     float* Y_zero;
+    float* psum;  // [E] sum over tokens of the full-softmax probabilities (nullable)
     int64_t N;
     int d, E, k, norm;
     float theta;
@@ -74,8 +75,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Softmax, top-k in rank order (score descending, ties to the lower expert
 // index), weights and records for one token.  The calling warp holds the
 // token's scores (bias included) as v[i] = g[lane + 32 i], -inf past E_r.
+// ps (shared memory, nullable) accumulates the token's full-softmax
+// probabilities per expert, for the mean router probability of the batch.
 template <int PER>
-__device__ __forceinline__ void select_token(const RouterArgs& a, int64_t t, int lane, float (&v)[PER]) {
+__device__ __forceinline__ void select_token(const RouterArgs& a, int64_t t, int lane, float (&v)[PER],
+                                             float* ps) {
     const int E = a.E, k = a.k;
     bool bad = false;
 #pragma unroll
@@ -124,10 +128,12 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int64_t t, int
         }
     }
     float z = 0.f;
+    float ev[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
         const int e = lane + 32 * i;
-        if (e < E) z += expf(v[i] - m);
+        ev[i] = e < E ? expf(v[i] - m) : 0.f;
+        z += ev[i];
     }
     z = warp_sum(z);
     const bool pick = lane < k;
@@ -151,6 +157,14 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int64_t t, int
             atomicAdd(a.counters + CNT_NONFINITE, 1ull);
         }
         return;
+    }
+    if (ps) {
+        const float iz = 1.f / z;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) atomicAdd(&ps[e], ev[i] * iz);
+        }
     }
     if (a.norm == MOE_NORM_FULLPROB) {
         wv = ex / z;
@@ -208,9 +222,11 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
     float* xs = smem;                 // [kKC][kTok]
     float* wsm = smem + kKC * kTok;   // [kKC][EPAD]
 
+    __shared__ float ps[kMaxRouterExperts];
     const int tid = threadIdx.x;
     const int tg = tid / EG, eg = tid % EG;
     const int64_t t0 = (int64_t)blockIdx.x * kTok;
+    for (int e = tid; e < a.E; e += kThreads) ps[e] = 0.f;
     const Tin* X = static_cast<const Tin*>(a.x);
     const Tin* W = static_cast<const Tin*>(a.W_r);
 
@@ -297,7 +313,12 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
             const int e = lane + 32 * i;
             v[i] = e < a.E ? g[e] : -INFINITY;
         }
-        select_token<PER>(a, t, lane, v);
+        select_token<PER>(a, t, lane, v, a.psum ? ps : nullptr);
+    }
+    if (a.psum) {
+        __syncthreads();
+        for (int e = tid; e < a.E; e += kThreads)
+            if (ps[e] != 0.f) atomicAdd(&a.psum[e], ps[e]);
     }
 
     if (a.Y_zero) {
@@ -355,10 +376,7 @@ struct Vec8<float> {
 // that the warp waits for memory once per iteration rather than once per
 // expert.  Bound by reading x once.
 template <int EMAX, typename Tin>
-__global__ void __launch_bounds__(256) router_narrow_kernel(RouterArgs a) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * 8 + warp;
-    if (t >= a.N) return;
+__device__ __forceinline__ void narrow_token(const RouterArgs& a, int64_t t, int lane, float* ps) {
     const Tin* X = static_cast<const Tin*>(a.x) + t * a.d;
     const Tin* W = static_cast<const Tin*>(a.W_r);
     const int E = a.E;
@@ -402,26 +420,49 @@ __global__ void __launch_bounds__(256) router_narrow_kernel(RouterArgs a) {
         for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
         if (lane == e && e < E) v[0] = s + (a.b_r ? a.b_r[e] : 0.f);
     }
-    select_token<1>(a, t, lane, v);
+    select_token<1>(a, t, lane, v, ps);
     if (a.Y_zero) zero_row(a.Y_zero, t, a.d, lane);
+}
+
+template <int EMAX, typename Tin>
+__global__ void __launch_bounds__(256) router_narrow_kernel(RouterArgs a) {
+    __shared__ float ps[EMAX];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+    if (threadIdx.x < EMAX) ps[threadIdx.x] = 0.f;
+    __syncthreads();
+    if (t < a.N) narrow_token<EMAX, Tin>(a, t, lane, a.psum ? ps : nullptr);
+    if (a.psum) {
+        __syncthreads();
+        if (threadIdx.x < a.E && ps[threadIdx.x] != 0.f) atomicAdd(&a.psum[threadIdx.x], ps[threadIdx.x]);
+    }
 }
 
 // Selection from precomputed scores [N, E_r] (tensor-core score path), one
 // warp per token.
 template <int PER>
 __global__ void __launch_bounds__(256) logits_topk_kernel(RouterArgs a, const float* __restrict__ logits) {
+    __shared__ float ps[32 * PER];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * 8 + warp;
-    if (t >= a.N) return;
-    const float* g = logits + t * a.E;
-    float v[PER];
+    for (int e = threadIdx.x; e < 32 * PER; e += blockDim.x) ps[e] = 0.f;
+    __syncthreads();
+    if (t < a.N) {
+        const float* g = logits + t * a.E;
+        float v[PER];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int e = lane + 32 * i;
-        v[i] = e < a.E ? g[e] + (a.b_r ? a.b_r[e] : 0.f) : -INFINITY;
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane + 32 * i;
+            v[i] = e < a.E ? g[e] + (a.b_r ? a.b_r[e] : 0.f) : -INFINITY;
+        }
+        select_token<PER>(a, t, lane, v, a.psum ? ps : nullptr);
+        if (a.Y_zero) zero_row(a.Y_zero, t, a.d, lane);
     }
-    select_token<PER>(a, t, lane, v);
-    if (a.Y_zero) zero_row(a.Y_zero, t, a.d, lane);
+    if (a.psum) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+            if (ps[e] != 0.f) atomicAdd(&a.psum[e], ps[e]);
+    }
 }
 
 template <int TT, int TE, typename Tin>
@@ -450,7 +491,7 @@ cudaError_t launch_typed(const RouterArgs& a, cudaStream_t st) {
 
 cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, const float* b_r,
                           const float* lat, int32_t* ids, float* w, float* margin,
-                          unsigned long long* counters, float* Y_zero, float* logits,
+                          unsigned long long* counters, float* Y_zero, float* logits, float* psum,
                           cudaStream_t st) {
     RouterArgs a;
     a.x = x;
@@ -462,6 +503,7 @@ cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, c
     a.margin = margin;
     a.counters = counters;
     a.Y_zero = Y_zero;
+    a.psum = psum;
     a.N = p.N;
     a.d = p.d;
     a.E = p.E_r;

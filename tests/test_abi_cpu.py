@@ -22,7 +22,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_struct_sizes_match_the_header_layout():
     assert ctypes.sizeof(moe.Params) == 56
-    assert ctypes.sizeof(moe.Stats) == 13 * 8 + 2 * 8 + 2 * 4 + 8 + 8
+    assert ctypes.sizeof(moe.Stats) == 13 * 8 + 2 * 8 + 2 * 4 + 8 + 8 + 8
     assert ctypes.sizeof(moe.WsLayout) == 15 * 8
 
 

@@ -78,6 +78,8 @@ def _end_to_end(w):
     out = parity.gpu_forward(w, inp)
     r, near = parity.check_routing(w, inp, out["rec"])
     parity.check_dispatch(w, out["rec"], out["stats"])
+    aux = oracle.aux_balance(r["logits"], out["rec"]["ids"], w.E, r["invalid"])
+    assert abs(out["stats"]["aux_balance"] - aux) <= 1e-4 * max(1.0, aux)
     err = parity.check_rows(w, inp, out["rec"], out["Y"])
     flips = int((out["rec"]["ids"] != r["ids"]).any(axis=1).sum())
     if flips == 0:

@@ -353,6 +353,24 @@ def test_soft_moe_normalisations():
     assert (out["Xs"].max(axis=0) <= x.max(axis=0) + 1e-12).all()
 
 
+def test_aux_balance_on_the_page_example_and_uniform():
+    # ch. 36.4: the example's probability table and requested loads (3, 4, 1)
+    # give pbar = (0.4875, 0.2625, 0.25), f = (3/8, 1/2, 1/8), so
+    # E_r sum f pbar = 3 (3/8 0.4875 + 1/2 0.2625 + 1/8 0.25) = 1.0359375
+    g, x, W_r = _n4_setup()
+    r = oracle.route(x, W_r, k=2, norm=oracle.NORM_RENORM)
+    # the example's router matrix holds ln P rounded to fp32: probabilities to ~1e-8
+    assert abs(oracle.aux_balance(r["logits"], r["ids"], 3) - 1.0359375) < 1e-7
+    # uniform shares and probabilities: exactly one
+    E = 4
+    logits = np.zeros((8, E))
+    ids = np.array([[e] for e in range(E)] * 2)
+    assert abs(oracle.aux_balance(logits, ids, E) - 1.0) < 1e-15
+    # all requests on one expert whose probability dominates: close to E_r
+    logits = np.tile([20.0, 0.0, 0.0, 0.0], (8, 1))
+    assert abs(oracle.aux_balance(logits, np.zeros((8, 1), int), E) - E) < 1e-6
+
+
 def test_capacity_printed_examples():
     for case in _golden("capacity_examples.json")["cases"]:
         assert oracle.capacity(case["c"], case["T"], case["k"], case["E"]) == case["C"], case
