@@ -440,3 +440,7 @@ def aux_balance(logits, ids, E: int, invalid=None) -> float:
 
 def round_bf16(v: float) -> float:
     return _load().oracle_round_bf16(float(v))
+
+
+# gradients of the layer (numpy, float64): oracle/backward.py
+from oracle.backward import backward, bf16_round, score_gradient  # noqa: E402,F401
