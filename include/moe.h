@@ -416,6 +416,76 @@ MOE_API moe_status moe_soft_forward(const moe_soft_params* p, const void* x, con
 MOE_API moe_status moe_soft_check(const moe_soft_params* p, const void* ws, moe_stream_t stream);
 
 /*
+ * Backward pass: gradients of
+ *     L = sum_{t,o} dY[t,o] Y[t,o] + aux_coef * aux
+ * for the forward pass that moe_forward last ran on `ws` (single routing
+ * group, bf16 layer).  Y is the layer output ("LLM from scratch" ch. 36.3,
+ * Algorithm 36.1; ch. 36.6 shared expert; vegetog "MoE token routing" sec. 3
+ * SwiGLU expert) and aux the balance objective E_r sum_e f_e pbar_e of
+ * ch. 36.4 (the value moe_stats.aux_balance reports).  The routing decisions
+ * (top-k sets, WLR pruning, capacity acceptance) are held fixed: they are
+ * piecewise constant in the inputs.  The objective's gradient reaches the
+ * router only through the mean probabilities pbar_e (the hard shares f_e are
+ * constants, ch. 36.4), via the softmax Jacobian.
+ *
+ * Chain (per accepted path j of token t with expert e, combine weight wc):
+ *   dwc = <dY_t, o>, o = W_d h;  dh = wc W_d^T dY_t;  dW_d += wc dY_t h^T;
+ *   dz = dh u SiLU'(z), du = dh SiLU(z);  dx_t += W_g^T dz + W_u^T du;
+ *   dW_g += dz x_t^T, dW_u += du x_t^T;  combine weight -> routing weight
+ *   (overflow policy, renormalisation over the chosen or surviving experts)
+ *   -> probability -> score (softmax Jacobian) -> dx_t += W_r^T dg_t,
+ *   dW_r = dg^T X, db_r = sum_t dg_t; the shared expert as an expert with
+ *   weight 1 on every token.
+ * Precision: dY enters rounded to bf16; the forward's bf16 h is used as
+ * stored (its rounding passes the gradient through); wc dY, dz and du are
+ * rounded to bf16 as tensor-core operands; every accumulation and all router
+ * arithmetic are fp32.  Gradients are fp32.
+ *
+ * Arguments: p, x, W_r, b_r and the weights exactly as given to that
+ * moe_forward (b_r nullable); dY [N, d] fp32 (device); ws the forward's
+ * workspace, unchanged since (its routing records, gathered rows x_perm and
+ * hidden activations are read); offsets_host a HOST copy of the forward's
+ * offsets [E_r + 1] (ws's "offsets" array, read after the forward finished:
+ * the per-expert weight-gradient launches are sized by it); grads the output
+ * buffers (device, fp32, overwritten; see moe_grads); bws the backward
+ * workspace (moe_backward_workspace_size bytes, 256-byte aligned
+ * recommended); aux_coef the objective's coefficient (0: none).
+ * Constraints: dtype MOE_BF16 (MOE_ERR_UNSUPPORTED for fp32 layers), E_r <=
+ * 256, k <= 32, N <= 65535 * 64; single routing group (not after
+ * moe_forward_end).
+ * Errors: MOE_ERR_INVALID_ARG (null or misaligned pointers, offsets_host not
+ * a non-decreasing prefix from 0 to at most N k), MOE_ERR_WORKSPACE,
+ * MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA (with moe_last_error).  Asynchronous on
+ * `stream`; the library allocates nothing.  N = 0 zeroes the weight
+ * gradients and returns.
+ */
+typedef struct moe_grads {
+    float* dx;      /* [N, d]                       required (may be null when N = 0) */
+    float* dW_r;    /* [E_r, d]                                        required */
+    float* db_r;    /* [E_r]                                           nullable */
+    float* dW_g;    /* [E_r, d_f, d]                                   required */
+    float* dW_u;    /* [E_r, d_f, d]                                   required */
+    float* dW_d;    /* [E_r, d, d_f]                                   required */
+    float* dWs_g;   /* [d_f_shared, d]     required when d_f_shared > 0          */
+    float* dWs_u;   /* [d_f_shared, d]     required when d_f_shared > 0          */
+    float* dWs_d;   /* [d, d_f_shared]     required when d_f_shared > 0          */
+} moe_grads;
+
+/* Bytes of the backward workspace for p (the worst case over routings). */
+MOE_API moe_status moe_backward_workspace_size(const moe_params* p, size_t* bytes);
+
+MOE_API moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offsets_host,
+                                const void* x, const void* W_r, const float* b_r, const void* W_g,
+                                const void* W_u, const void* W_d, const void* Ws_g, const void* Ws_u,
+                                const void* Ws_d, const float* dY, const void* ws, const moe_grads* grads,
+                                void* bws, moe_stream_t stream);
+
+/* Waits for `stream` and reports MOE_ERR_TIMEOUT if a bounded device wait of
+ * the last moe_backward on `bws` gave up (its tensor-core GEMMs record that in
+ * the backward workspace), else MOE_OK. */
+MOE_API moe_status moe_backward_check(const moe_params* p, const void* bws, moe_stream_t stream);
+
+/*
  * Self-test of the library's bounded device waits (no counterpart on the
  * pages).  Launches one CTA that waits on a shared-memory mbarrier nothing
  * ever arrives on, with the same bounded-wait routine the tensor-core GEMMs

@@ -33,7 +33,7 @@ DT_F32, DT_BF16 = 0, 1
 
 # tensor ids of the counter-based streams
 TID = {"x": 1, "W_r": 2, "W_g": 3, "W_u": 4, "W_d": 5, "Ws_g": 6, "Ws_u": 7, "Ws_d": 8,
-       "lat_up": 9, "lat_comp": 10, "lat_down": 11, "Phi": 12}
+       "lat_up": 9, "lat_comp": 10, "lat_down": 11, "Phi": 12, "dY": 13}
 
 
 def build(force: bool = False) -> str:
@@ -251,6 +251,13 @@ def tensor(w: Workload, name: str, expert: Optional[int] = None) -> Optional[np.
         return a.reshape(shp[1], shp[2])
     n = int(np.prod(shp))
     return fill(w.seed, TID[name], n, std=_std(w, name), dtype=w.dt).reshape(shp)
+
+
+def upstream_gradient(w: Workload, seed_offset: int = 0) -> np.ndarray:
+    """The gradient dL/dY [N, d] fed to the layer's backward pass: standard
+    normals in fp32 (the backward rounds it to its own precision)."""
+    n = w.N * w.d
+    return fill(w.seed + seed_offset, TID["dY"], n, std=1.0, dtype="f32").reshape(w.N, w.d)
 
 
 def inputs(w: Workload, names=("x", "W_r", "b_r", "lat", "W_g", "W_u", "W_d", "Ws_g", "Ws_u", "Ws_d")):

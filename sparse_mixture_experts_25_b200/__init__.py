@@ -91,6 +91,14 @@ _P = ctypes.c_void_p
 _lib = None
 
 
+GRAD_NAMES = ("dx", "dW_r", "db_r", "dW_g", "dW_u", "dW_d", "dWs_g", "dWs_u", "dWs_d")
+
+
+class Grads(ctypes.Structure):
+    """moe_grads: device pointers of the gradient buffers (fp32)."""
+    _fields_ = [(n, _P) for n in GRAD_NAMES]
+
+
 def lib():
     """Load (building first if missing or stale) the in-tree libmoe.so, or the
     library file named by the MOE_LIB_PATH environment variable."""
@@ -121,6 +129,10 @@ def lib():
         L.moe_soft_workspace_size.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t)]
         L.moe_soft_forward.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_soft_check.argtypes = [sp, _P, _P]
+        L.moe_backward_workspace_size.argtypes = [pp, ctypes.POINTER(ctypes.c_size_t)]
+        L.moe_backward.argtypes = [pp, ctypes.c_float, ctypes.POINTER(ctypes.c_int32), _P, _P, _P, _P, _P, _P,
+                                   _P, _P, _P, _P, _P, ctypes.POINTER(Grads), _P, _P]
+        L.moe_backward_check.argtypes = [pp, _P, _P]
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [ctypes.c_int]
@@ -130,7 +142,8 @@ def lib():
                      "moe_forward",
                      "moe_get_stats", "moe_set_stage_events", "moe_forward_begin",
                      "moe_forward_end", "moe_selftest_wait_timeout", "moe_soft_workspace_size",
-                     "moe_soft_forward", "moe_soft_check", "moe_dispatch_ranked", "moe_gather_rows"):
+                     "moe_soft_forward", "moe_soft_check", "moe_dispatch_ranked", "moe_gather_rows",
+                     "moe_backward_workspace_size", "moe_backward", "moe_backward_check"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -354,3 +367,33 @@ def workspace_x_perm(p: Params, ws):
     n = p.N * p.k * p.d
     nbytes = n * torch.empty((), dtype=dt).element_size()
     return ws[L["x_perm"]:L["x_perm"] + nbytes].view(dt).view(p.N * p.k, p.d)
+
+
+def moe_backward_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().moe_backward_workspace_size(ctypes.byref(p), ctypes.byref(n)), "moe_backward_workspace_size")
+    return n.value
+
+
+def moe_backward(p, offsets_host, x, W_r, b_r, W_g, W_u, W_d, Ws_g, Ws_u, Ws_d, dY, ws, grads, bws,
+                 aux_coef: float = 0.0, stream=None):
+    """Gradients of sum(dY * Y) + aux_coef * aux for the forward last run on
+    ws (see moe_backward in include/moe.h).  offsets_host: the forward's
+    offsets [E_r + 1] on the host (a numpy array or CPU tensor); grads: dict
+    of device fp32 tensors keyed by GRAD_NAMES (db_r and the shared-expert
+    entries may be missing or None)."""
+    import numpy as np
+    off = np.ascontiguousarray(np.asarray(offsets_host), dtype=np.int32)
+    if off.shape != (p.E_r + 1,):
+        raise ValueError("offsets_host must hold E_r + 1 entries")
+    g = Grads(*[_ptr(grads.get(n)) for n in GRAD_NAMES])
+    _check(lib().moe_backward(ctypes.byref(p), float(aux_coef), off.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                              _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W_g), _ptr(W_u), _ptr(W_d), _ptr(Ws_g), _ptr(Ws_u),
+                              _ptr(Ws_d), _ptr(dY), _ptr(ws), ctypes.byref(g), _ptr(bws), _stream(stream)),
+           "moe_backward")
+
+
+def moe_backward_check(p, bws, stream=None) -> int:
+    """Waits for the stream; MOE_ERR_TIMEOUT if a bounded wait of the last
+    moe_backward on bws gave up, else MOE_OK."""
+    return lib().moe_backward_check(ctypes.byref(p), _ptr(bws), _stream(stream))

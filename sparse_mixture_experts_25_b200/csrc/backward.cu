@@ -1,0 +1,894 @@
+// Backward pass of the sparse-MoE layer: gradients of
+//   L = sum dY (.) Y + aux_coef * aux
+// with the routing decisions of the forward held fixed ("LLM from scratch"
+// ch. 36.3 combine, ch. 36.4 balance objective whose gradient reaches the
+// router through the mean probabilities and the softmax Jacobian, ch. 36.6
+// shared expert; vegetog "MoE token routing" sec. 3 SwiGLU expert).
+//
+// Per accepted path (row r of expert e, token t, combine weight wc):
+//   z = W_g x, u = W_u x        recomputed on the tensor cores (fp32)
+//   Gd = W_d^T dY_t             one grouped GEMM on the bf16 dY rows
+//   dwc = <Gd, h>               = <dY_t, W_d h>, the combine-weight gradient
+//   dh = wc Gd; dz = dh u SiLU'(z), du = dh SiLU(z)   (bf16 operands)
+//   dx_perm = [dz | du] [W_g ; W_u]                   one grouped GEMM
+//   dW_d = (wc dY)^T h, dW_g = dz^T x, dW_u = du^T x  per-expert GEMMs over
+//                                                     the expert's rows (K)
+// Router (one warp per token): dwc -> routing-weight gradient (overflow
+// policy, renormalisation) -> probability gradient -> score gradient dG
+// (softmax Jacobian) + the balance objective's term; dx += dG W_r,
+// dW_r = dG^T X, db = column sums of dG (fp32 CUDA-core kernels: E_r is
+// small).  dx gathers the expert rows' dx_perm in token order.
+//
+// Layout choices for the tcgen05 GEMM (out = A B^T, both operands K-major):
+// the row-grouped contractions run on the grouped kernel in store mode with
+// the dimensions relabelled (its "d_f" is K, its "d" the output width), which
+// needs W_d^T [E, d_f, d] and [W_g^T | W_u^T] [E, d, 2 d_f]: both are written
+// once per call by a batched transpose.  The weight gradients contract over an
+// expert's rows, so their operands are transposed per expert into column
+// blocks padded to a multiple of 8 rows with zeros (16-byte TMA rows); the
+// host launches one dense GEMM per expert with the row counts it was given.
+#include <cuda_bf16.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <vector>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+using bf16 = __nv_bfloat16;
+constexpr int kTT = 64;  // transposition tile
+
+__device__ __forceinline__ void ld8(const bf16* p, float (&v)[8]) {
+    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
+__device__ __forceinline__ uint32_t pk2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// padoff[g]: first column of group g's transposed block (groups padded to a
+// multiple of 8 rows); tstart[g]: first 64-row transposition tile of group g.
+// One thread: G <= 1024.
+__global__ void bwd_tables_kernel(int G, const int32_t* __restrict__ offsets, int32_t* __restrict__ padoff,
+                                  int32_t* __restrict__ tstart) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    int32_t p = 0, t = 0;
+    for (int g = 0; g < G; ++g) {
+        padoff[g] = p;
+        tstart[g] = t;
+        int32_t R = offsets[g + 1] - offsets[g];
+        if (R < 0) R = 0;
+        p += (R + 7) & ~7;
+        t += (R + kTT - 1) / kTT;
+    }
+    padoff[G] = p;
+    tstart[G] = t;
+}
+
+__global__ void bwd_single_group_kernel(int32_t n, int32_t* __restrict__ off) {
+    if (threadIdx.x == 0) {
+        off[0] = 0;
+        off[1] = n;
+    }
+}
+
+// Group-wise transposition: for group g (rows offsets[g] .. offsets[g+1]-1 of
+// src [*, ld], columns 0..C-1), dst block g = dst + C padoff[g] is [C, Rp_g]
+// row-major with dst[c, r] = bf16(scale[row] src[row, c]) (scale optional) and
+// zeros in the padding columns r in [R_g, Rp_g).  64 x 64 tiles through shared
+// memory, 16-byte global accesses.  C, ld multiples of 8.
+template <bool SCALE>
+__global__ void __launch_bounds__(256)
+    bwd_group_transpose_kernel(const bf16* __restrict__ src, int64_t ld, int64_t C, const int32_t* __restrict__ offsets,
+                               const int32_t* __restrict__ padoff, const int32_t* __restrict__ tstart, int G,
+                               const float* __restrict__ scale, bf16* __restrict__ dst) {
+    __shared__ float tile[kTT][kTT + 1];
+    const int bx = blockIdx.x;
+    int lo = 0, hi = G - 1;  // last group whose first tile is <= bx
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tstart[mid] <= bx) lo = mid;
+        else hi = mid - 1;
+    }
+    const int g = lo;
+    const int64_t R = offsets[g + 1] - offsets[g];
+    const int64_t Rp = padoff[g + 1] - padoff[g];
+    const int64_t lr0 = (int64_t)(bx - tstart[g]) * kTT;
+    const int64_t c0 = (int64_t)blockIdx.y * kTT;
+    const int t = threadIdx.x, cc = (t & 7) * 8;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int rr = (t >> 3) + h * 32;
+        const int64_t lr = lr0 + rr, c = c0 + cc;
+        float v[8];
+        if (lr < R && c < C) {
+            const int64_t row = offsets[g] + lr;
+            ld8(src + row * ld + c, v);
+            if (SCALE) {
+                const float s = scale[row];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] *= s;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tile[rr][cc + i] = v[i];
+    }
+    __syncthreads();
+    bf16* base = dst + C * (int64_t)padoff[g];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int oc = (t >> 3) + h * 32;
+        const int64_t c = c0 + oc, lr = lr0 + cc;
+        if (c < C && lr < Rp) {
+            uint4 q;
+            q.x = pk2(tile[cc][oc], tile[cc + 1][oc]);
+            q.y = pk2(tile[cc + 2][oc], tile[cc + 3][oc]);
+            q.z = pk2(tile[cc + 4][oc], tile[cc + 5][oc]);
+            q.w = pk2(tile[cc + 6][oc], tile[cc + 7][oc]);
+            *reinterpret_cast<uint4*>(base + c * Rp + lr) = q;
+        }
+    }
+}
+
+// dst[b][c][r] (row stride ld_dst, batch stride bs_dst) = src[b][r][c] for a
+// contiguous batch of [R, C] matrices; R, C, ld_dst multiples of 8.
+__global__ void __launch_bounds__(256)
+    bwd_batched_transpose_kernel(const bf16* __restrict__ src, int64_t R, int64_t C, bf16* __restrict__ dst,
+                                 int64_t ld_dst, int64_t bs_dst) {
+    __shared__ float tile[kTT][kTT + 1];
+    const int64_t b = blockIdx.z;
+    const bf16* s = src + b * R * C;
+    bf16* o = dst + b * bs_dst;
+    const int64_t r0 = (int64_t)blockIdx.x * kTT, c0 = (int64_t)blockIdx.y * kTT;
+    const int t = threadIdx.x, cc = (t & 7) * 8;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int rr = (t >> 3) + h * 32;
+        const int64_t r = r0 + rr, c = c0 + cc;
+        float v[8];
+        if (r < R && c < C) {
+            ld8(s + r * C + c, v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tile[rr][cc + i] = v[i];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int oc = (t >> 3) + h * 32;
+        const int64_t c = c0 + oc, r = r0 + cc;
+        if (c < C && r < R) {
+            uint4 q;
+            q.x = pk2(tile[cc][oc], tile[cc + 1][oc]);
+            q.y = pk2(tile[cc + 2][oc], tile[cc + 3][oc]);
+            q.z = pk2(tile[cc + 4][oc], tile[cc + 5][oc]);
+            q.w = pk2(tile[cc + 6][oc], tile[cc + 7][oc]);
+            *reinterpret_cast<uint4*>(o + c * ld_dst + r) = q;
+        }
+    }
+}
+
+// out[r, :] = bf16(dY[tok(r), :]) for r < n (tok = slot_token[r], or r when
+// slot_token is null; n = *n_dev clamped to max_rows, or n_fixed).  One warp
+// per row, 4 columns per lane step.
+__global__ void __launch_bounds__(256)
+    bwd_gather_dy_kernel(const float* __restrict__ dY, int64_t d, const int32_t* __restrict__ slot_token,
+                         const int32_t* __restrict__ n_dev, int64_t n_fixed, int64_t max_rows, int64_t n_tokens,
+                         bf16* __restrict__ out) {
+    int64_t n = n_fixed;
+    if (n_dev) {
+        n = *n_dev;
+        if (n > max_rows) n = max_rows;
+    }
+    const int lane = threadIdx.x & 31;
+    const int64_t wpb = blockDim.x >> 5;
+    for (int64_t r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += (int64_t)gridDim.x * wpb) {
+        const int64_t tok = slot_token ? (int64_t)slot_token[r] : r;
+        const bool ok = tok >= 0 && tok < n_tokens;
+        uint2* o = reinterpret_cast<uint2*>(out + r * d);
+        const float4* src = reinterpret_cast<const float4*>(dY + (ok ? tok : 0) * d);
+        for (int64_t c = lane; c < d / 4; c += 32) {
+            float4 v = ok ? src[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+            o[c] = make_uint2(pk2(v.x, v.y), pk2(v.z, v.w));
+        }
+    }
+}
+
+// SwiGLU backward of routed (or shared) rows r < n: with dh = wc[r] Gd[r],
+//   dz = dh u SiLU'(z), du = dh SiLU(z)  ->  dzu[r] = [dz | du] (bf16, 2 d_f)
+//   dwc[r] = <Gd[r], h[r]>                  (fp32; skipped when dwc is null)
+// SiLU(z) = z s(z), SiLU'(z) = s(z) (1 + z (1 - s(z))), s the logistic
+// function.  wc null: weight 1.  One warp per row.
+__global__ void __launch_bounds__(256)
+    bwd_swiglu_kernel(const float* __restrict__ Z, const float* __restrict__ U, const float* __restrict__ Gd,
+                      const bf16* __restrict__ H, int64_t d_f, const float* __restrict__ wc,
+                      const int32_t* __restrict__ n_dev, int64_t n_fixed, int64_t max_rows, bf16* __restrict__ dzu,
+                      float* __restrict__ dwc) {
+    int64_t n = n_fixed;
+    if (n_dev) {
+        n = *n_dev;
+        if (n > max_rows) n = max_rows;
+    }
+    const int lane = threadIdx.x & 31;
+    const int64_t wpb = blockDim.x >> 5;
+    for (int64_t r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += (int64_t)gridDim.x * wpb) {
+        const float w = wc ? wc[r] : 1.f;
+        const float4* z4 = reinterpret_cast<const float4*>(Z + r * d_f);
+        const float4* u4 = reinterpret_cast<const float4*>(U + r * d_f);
+        const float4* g4 = reinterpret_cast<const float4*>(Gd + r * d_f);
+        const uint2* h4 = reinterpret_cast<const uint2*>(H + r * d_f);
+        uint2* dz4 = reinterpret_cast<uint2*>(dzu + r * 2 * d_f);
+        uint2* du4 = reinterpret_cast<uint2*>(dzu + r * 2 * d_f + d_f);
+        float acc = 0.f;
+        for (int64_t c = lane; c < d_f / 4; c += 32) {
+            const float4 z = z4[c], u = u4[c], g = g4[c];
+            const uint2 hq = h4[c];
+            const float2 h01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hq.x));
+            const float2 h23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hq.y));
+            acc += g.x * h01.x + g.y * h01.y + g.z * h23.x + g.w * h23.y;
+            const float zz[4] = {z.x, z.y, z.z, z.w}, uu[4] = {u.x, u.y, u.z, u.w}, gg[4] = {g.x, g.y, g.z, g.w};
+            float dz[4], du[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float s = 1.f / (1.f + expf(-zz[i]));
+                const float dh = w * gg[i];
+                du[i] = dh * (zz[i] * s);
+                dz[i] = dh * uu[i] * (s * (1.f + zz[i] * (1.f - s)));
+            }
+            dz4[c] = make_uint2(pk2(dz[0], dz[1]), pk2(dz[2], dz[3]));
+            du4[c] = make_uint2(pk2(du[0], du[1]), pk2(du[2], du[3]));
+        }
+        acc = warp_sum(acc);
+        if (dwc && lane == 0) dwc[r] = acc;
+    }
+}
+
+// Score gradient, one warp per token (see moe_backward in moe.h):
+//   da_j  = dwc_j                     (policy 0, or no partial rejection)
+//         = (dwc_j - sum_i dwc_i wc_i) / A,  wc = a / A,  A = sum_acc a   (policy 1)
+//   RENORM / WLR: a_j = m_j p_j / s (s = sum over the chosen experts of p,
+//                 m_j = 0 where the forward's weight is 0);
+//                 dp_j = (m_j da_j - sum_i da_i a_i) / s
+//   FULLPROB:     a_j = p_j, dp_j = da_j
+//   dg_e = p_e (dp_e - sum_i p_i dp_i)
+//        + aux_coef (E_r / N_valid) p_e (f_e - sum_i f_i p_i),  f = L / sum L
+// Tokens with a non-finite score get dg = 0.
+struct RouterBwd {
+    const float* logits;  // [N, E] scores without bias
+    const float* b_r;     // [E] or null
+    const int32_t* ids;
+    const float* w;
+    const int32_t* slot;
+    const int32_t* offsets;
+    const float* dwc;     // [rows] per routed row
+    const int32_t* L;     // [E] requests per expert
+    const unsigned long long* counters;
+    float* dG;            // [N, E]
+    int64_t N;
+    int E, k, norm, policy;
+    float aux_coef;
+    int64_t max_rows;
+};
+
+__global__ void __launch_bounds__(256) bwd_router_kernel(RouterBwd a) {
+    __shared__ float sp[8][kMaxRouterExperts];
+    __shared__ float sdp[8][kMaxRouterExperts];
+    __shared__ float sf[kMaxRouterExperts];
+    __shared__ float s_coef;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int E = a.E;
+    const bool aux = a.aux_coef != 0.f;
+    if (threadIdx.x == 0) {
+        const double req = (double)a.counters[CNT_REQUESTED];
+        const double nv = (double)(a.N - (int64_t)a.counters[CNT_NONFINITE]);
+        s_coef = (aux && req > 0 && nv > 0) ? (float)(a.aux_coef * E / nv) : 0.f;
+    }
+    __syncthreads();
+    if (aux) {
+        const double req = (double)a.counters[CNT_REQUESTED];
+        for (int e = threadIdx.x; e < E; e += blockDim.x) sf[e] = req > 0 ? (float)(a.L[e] / req) : 0.f;
+    }
+    __syncthreads();
+    const float coef = s_coef;
+    float* p = sp[warp];
+    float* dp = sdp[warp];
+    for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < a.N; t += (int64_t)gridDim.x * 8) {
+        float m = -INFINITY;
+        bool bad = false;
+        for (int e = lane; e < E; e += 32) {
+            const float g = a.logits[t * E + e] + (a.b_r ? a.b_r[e] : 0.f);
+            p[e] = g;
+            bad |= !isfinite(g);
+            m = fmaxf(m, g);
+        }
+        bad = __any_sync(0xffffffffu, bad);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (bad) {
+            for (int e = lane; e < E; e += 32) a.dG[t * E + e] = 0.f;
+            __syncwarp();
+            continue;
+        }
+        float z = 0.f;
+        for (int e = lane; e < E; e += 32) {
+            const float v = expf(p[e] - m);
+            p[e] = v;
+            dp[e] = 0.f;
+            z += v;
+        }
+        z = warp_sum(z);
+        const float inv = 1.f / z;
+        for (int e = lane; e < E; e += 32) p[e] *= inv;
+        __syncwarp();
+        // this lane's routing record
+        int ej = -1;
+        float aj = 0.f, dw = 0.f;
+        bool acc = false;
+        if (lane < a.k) {
+            ej = a.ids[t * a.k + lane];
+            if (ej >= E) ej = -1;
+            if (ej >= 0) {
+                aj = a.w[t * a.k + lane];
+                const int s = a.slot[t * a.k + lane];
+                if (s >= 0) {
+                    const int64_t row = (int64_t)a.offsets[ej] + s;
+                    if (row < a.max_rows) {
+                        acc = true;
+                        dw = a.dwc[row];
+                    }
+                }
+            }
+        }
+        const bool chosen = ej >= 0;
+        const float pj = chosen ? p[ej] : 0.f;
+        const float ssel = warp_sum(pj);
+        const float mj = (chosen && aj != 0.f) ? 1.f : 0.f;
+        const float ap = a.norm == MOE_NORM_FULLPROB ? pj : (ssel > 0.f ? mj * pj / ssel : 0.f);
+        const int req = __popc(__ballot_sync(0xffffffffu, chosen));
+        const int rej = __popc(__ballot_sync(0xffffffffu, chosen && !acc));
+        float da = acc ? dw : 0.f;
+        if (a.policy == MOE_REJECT_RENORM && rej > 0 && rej < req) {
+            const float A = warp_sum(acc ? ap : 0.f);
+            const float S = warp_sum(acc && A > 0.f ? dw * (ap / A) : 0.f);
+            da = (acc && A > 0.f) ? (dw - S) / A : 0.f;
+        }
+        float dpj;
+        if (a.norm == MOE_NORM_FULLPROB) {
+            dpj = da;
+        } else {
+            const float T = warp_sum(da * ap);
+            dpj = ssel > 0.f ? (mj * da - T) / ssel : 0.f;
+        }
+        if (chosen) dp[ej] = dpj;
+        __syncwarp();
+        float spd = 0.f, sfp = 0.f;
+        for (int e = lane; e < E; e += 32) {
+            spd += p[e] * dp[e];
+            if (aux) sfp += sf[e] * p[e];
+        }
+        spd = warp_sum(spd);
+        if (aux) sfp = warp_sum(sfp);
+        for (int e = lane; e < E; e += 32) {
+            float g = p[e] * (dp[e] - spd);
+            if (aux) g += coef * p[e] * (sf[e] - sfp);
+            a.dG[t * E + e] = g;
+        }
+        __syncwarp();
+    }
+}
+
+// db[e] = sum_t dG[t, e]: one block per 32 columns, 8 warps over the rows
+__global__ void __launch_bounds__(256) bwd_colsum_kernel(const float* __restrict__ dG, int64_t N, int E,
+                                                         float* __restrict__ db) {
+    __shared__ float part[8][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int e = blockIdx.x * 32 + lane;
+    float s = 0.f;
+    if (e < E)
+        for (int64_t t = warp; t < N; t += 8) s += dG[t * E + e];
+    part[warp][lane] = s;
+    __syncthreads();
+    if (warp == 0 && e < E) {
+        float v = 0.f;
+        for (int i = 0; i < 8; ++i) v += part[i][lane];
+        db[e] = v;
+    }
+}
+
+// dx[t] += sum over the token's accepted paths (rank order) of
+// dxp[offsets[e] + slot] (+ dxs[t] when the shared expert ran).  One warp
+// per token, float4 columns.
+__global__ void __launch_bounds__(256)
+    bwd_dx_kernel(float* __restrict__ dx, const float* __restrict__ dxp, const float* __restrict__ dxs,
+                  const int32_t* __restrict__ ids, const int32_t* __restrict__ slot, const int32_t* __restrict__ offsets,
+                  int64_t N, int64_t d, int k, int E, int64_t max_rows) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wpb = blockDim.x >> 5;
+    for (int64_t t = blockIdx.x * wpb + (threadIdx.x >> 5); t < N; t += (int64_t)gridDim.x * wpb) {
+        float4* o = reinterpret_cast<float4*>(dx + t * d);
+        for (int64_t c = lane; c < d / 4; c += 32) {
+            float4 v = o[c];
+            if (dxs) {
+                const float4 s = reinterpret_cast<const float4*>(dxs + t * d)[c];
+                v.x += s.x; v.y += s.y; v.z += s.z; v.w += s.w;
+            }
+            for (int j = 0; j < k; ++j) {
+                const int e = ids[t * k + j];
+                const int s = slot[t * k + j];
+                if (e < 0 || e >= E || s < 0) continue;
+                const int64_t row = (int64_t)offsets[e] + s;
+                if (row >= max_rows) continue;
+                const float4 q = reinterpret_cast<const float4*>(dxp + row * d)[c];
+                v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
+            }
+            o[c] = v;
+        }
+    }
+}
+
+// C[m, n] = sum_k A(m, k) B(n, k) with A(m, k) = A[m sam + k sak] and
+// B(n, k) = B[n sbn + k sbk] (fp32 accumulate, C row-major with ldc): 64 x 64
+// tiles, K steps of 16 through shared memory, 4 x 4 outputs per thread.  For
+// the router's small contractions (one side is E_r wide).
+__device__ __forceinline__ float as_f32(float v) { return v; }
+__device__ __forceinline__ float as_f32(bf16 v) { return __bfloat162float(v); }
+
+template <typename TA, typename TB>
+__global__ void __launch_bounds__(256)
+    bwd_simt_gemm_kernel(int64_t M, int64_t N, int64_t K, const TA* __restrict__ A, int64_t sam, int64_t sak,
+                         const TB* __restrict__ B, int64_t sbn, int64_t sbk, float* __restrict__ C, int64_t ldc) {
+    __shared__ float As[16][64 + 4];
+    __shared__ float Bs[16][64 + 4];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int64_t m0 = (int64_t)blockIdx.y * 64, n0 = (int64_t)blockIdx.x * 64;
+    float acc[4][4] = {};
+    for (int64_t k0 = 0; k0 < K; k0 += 16) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int idx = tid + i * 256;
+            int mm, kk;
+            if (sak == 1) { kk = idx & 15; mm = idx >> 4; }
+            else { mm = idx & 63; kk = idx >> 6; }
+            const int64_t m = m0 + mm, kq = k0 + kk;
+            As[kk][mm] = (m < M && kq < K) ? as_f32(A[m * sam + kq * sak]) : 0.f;
+            int nn, kb;
+            if (sbk == 1) { kb = idx & 15; nn = idx >> 4; }
+            else { nn = idx & 63; kb = idx >> 6; }
+            const int64_t n = n0 + nn, kr = k0 + kb;
+            Bs[kb][nn] = (n < N && kr < K) ? as_f32(B[n * sbn + kr * sbk]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            float av[4], bv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                av[i] = As[kk][ty * 4 + i];
+                bv[i] = Bs[kk][tx * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] += av[i] * bv[j];
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t m = m0 + ty * 4 + i;
+        if (m >= M) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t n = n0 + tx * 4 + j;
+            if (n < N) C[m * ldc + n] = acc[i][j];
+        }
+    }
+}
+
+template <typename TA, typename TB>
+cudaError_t simt_gemm(int64_t M, int64_t N, int64_t K, const TA* A, int64_t sam, int64_t sak, const TB* B,
+                      int64_t sbn, int64_t sbk, float* C, int64_t ldc, cudaStream_t st) {
+    if (M <= 0 || N <= 0) return cudaSuccess;
+    const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + 63) / 64));
+    bwd_simt_gemm_kernel<TA, TB><<<grid, 256, 0, st>>>(M, N, K, A, sam, sak, B, sbn, sbk, C, ldc);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Workspace
+// ---------------------------------------------------------------------------
+struct BwdLayout {
+    size_t padoff, tstart, mt_start, sh_off, sh_padoff, sh_tstart, counters;
+    size_t logits, dG, dwc, Wt_d, Wt_gu, dYp, Z, U, Gd, dzu, dxp, doT, xT, hT, dzT, duT;
+    size_t dYs, Zs, Us, Gs, dzus, dxs, WsT_d, WsT_gu, dYsT, xsT, hsT, dzsT, dusT;
+    size_t total;
+};
+
+size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+BwdLayout bwd_layout(const moe_params& p) {
+    const size_t N = (size_t)p.N, d = (size_t)p.d, df = (size_t)p.d_f, E = (size_t)p.E_r;
+    const size_t rows = N * (size_t)p.k;
+    const size_t Rp = rows + 7 * E;  // padded columns of the per-expert transposed blocks
+    const size_t ds = p.d_f_shared > 0 ? (size_t)p.d_f_shared : 0;
+    const size_t Np = (N + 7) & ~(size_t)7;
+    BwdLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = up256(off + bytes);
+        return o;
+    };
+    L.padoff = take((E + 1) * 4);
+    L.tstart = take((E + 1) * 4);
+    L.mt_start = take((E + 1) * 4);
+    L.sh_off = take(2 * 4);
+    L.sh_padoff = take(2 * 4);
+    L.sh_tstart = take(2 * 4);
+    L.counters = take(CNT_COUNT * 8);
+    L.logits = take(N * E * 4);
+    L.dG = take(N * E * 4);
+    L.dwc = take(rows * 4);
+    L.Wt_d = take(E * df * d * 2);
+    L.Wt_gu = take(E * d * 2 * df * 2);
+    L.dYp = take(rows * d * 2);
+    L.Z = take(rows * df * 4);
+    L.U = take(rows * df * 4);
+    L.Gd = take(rows * df * 4);
+    L.dzu = take(rows * 2 * df * 2);
+    L.dxp = take(rows * d * 4);
+    L.doT = take(d * Rp * 2);
+    L.xT = take(d * Rp * 2);
+    L.hT = take(df * Rp * 2);
+    L.dzT = take(df * Rp * 2);
+    L.duT = take(df * Rp * 2);
+    if (ds) {
+        L.dYs = take(N * d * 2);
+        L.Zs = take(N * ds * 4);
+        L.Us = take(N * ds * 4);
+        L.Gs = take(N * ds * 4);
+        L.dzus = take(N * 2 * ds * 2);
+        L.dxs = take(N * d * 4);
+        L.WsT_d = take(ds * d * 2);
+        L.WsT_gu = take(d * 2 * ds * 2);
+        L.dYsT = take(d * Np * 2);
+        L.xsT = take(d * Np * 2);
+        L.hsT = take(ds * Np * 2);
+        L.dzsT = take(ds * Np * 2);
+        L.dusT = take(ds * Np * 2);
+    }
+    L.total = off;
+    return L;
+}
+
+thread_local char g_bwd_error[256] = "";
+
+moe_status bwd_fail(cudaError_t e, const char* where) {
+    snprintf(g_bwd_error, sizeof(g_bwd_error), "moe_backward %s: %s (%d)", where, cudaGetErrorString(e), (int)e);
+    record_error(g_bwd_error);
+    return MOE_ERR_CUDA;
+}
+
+bool al16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
+
+moe_status bwd_check(const moe_params* p) {
+    size_t ws = 0;
+    const moe_status s = moe_workspace_size(p, &ws);  // the forward's parameter checks
+    if (s != MOE_OK) return s;
+    if (p->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (p->E_r > kMaxRouterExperts || p->k > kMaxK) return MOE_ERR_UNSUPPORTED;
+    if (p->N > (int64_t)65535 * 64) return MOE_ERR_UNSUPPORTED;  // grid rows of the router contractions
+    return MOE_OK;
+}
+
+unsigned grid_for(int64_t items_per_block_units, int64_t n) {
+    int64_t b = (n + items_per_block_units - 1) / items_per_block_units;
+    const int64_t cap = (int64_t)num_sms() * 16;
+    if (b > cap) b = cap;
+    if (b < 1) b = 1;
+    return (unsigned)b;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_backward_workspace_size(const moe_params* p, size_t* bytes) {
+    const moe_status s = bwd_check(p);
+    if (s != MOE_OK) return s;
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    *bytes = bwd_layout(*p).total;
+    return MOE_OK;
+}
+
+moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offsets_host, const void* x,
+                        const void* W_r, const float* b_r, const void* W_g, const void* W_u, const void* W_d,
+                        const void* Ws_g, const void* Ws_u, const void* Ws_d, const float* dY, const void* ws,
+                        const moe_grads* gr, void* bws, moe_stream_t stream) {
+    moe_status s = bwd_check(p);
+    if (s != MOE_OK) return s;
+    if (!ws || !al16(ws) || !bws || !al16(bws)) return MOE_ERR_WORKSPACE;
+    if (!gr || !offsets_host) return MOE_ERR_INVALID_ARG;
+    const bool sh = p->d_f_shared > 0;
+    if ((p->N > 0 && !gr->dx) || !gr->dW_r || !gr->dW_g || !gr->dW_u || !gr->dW_d) return MOE_ERR_INVALID_ARG;
+    if (sh && (!gr->dWs_g || !gr->dWs_u || !gr->dWs_d)) return MOE_ERR_INVALID_ARG;
+    if (!(aux_coef == aux_coef)) return MOE_ERR_INVALID_ARG;
+    const int64_t N = p->N, d = p->d, df = p->d_f, E = p->E_r, k = p->k;
+    const int64_t rows = N * k;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    const int64_t dfs = sh ? p->d_f_shared : 0;
+    if (N == 0) {  // no tokens: every weight gradient is zero
+        (void)cudaGetLastError();
+        e = cudaMemsetAsync(gr->dW_r, 0, sizeof(float) * E * d, st);
+        if (e == cudaSuccess && gr->db_r) e = cudaMemsetAsync(gr->db_r, 0, sizeof(float) * E, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW_g, 0, sizeof(float) * E * df * d, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW_u, 0, sizeof(float) * E * df * d, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW_d, 0, sizeof(float) * E * df * d, st);
+        if (e == cudaSuccess && sh) e = cudaMemsetAsync(gr->dWs_g, 0, sizeof(float) * dfs * d, st);
+        if (e == cudaSuccess && sh) e = cudaMemsetAsync(gr->dWs_u, 0, sizeof(float) * dfs * d, st);
+        if (e == cudaSuccess && sh) e = cudaMemsetAsync(gr->dWs_d, 0, sizeof(float) * dfs * d, st);
+        return e == cudaSuccess ? MOE_OK : bwd_fail(e, "memset");
+    }
+    // (an empty forward writes no offsets, so they are checked only now)
+    if (offsets_host[0] != 0) return MOE_ERR_INVALID_ARG;
+    for (int64_t e = 0; e < E; ++e)
+        if (offsets_host[e + 1] < offsets_host[e]) return MOE_ERR_INVALID_ARG;
+    if (offsets_host[E] > rows) return MOE_ERR_INVALID_ARG;
+    (void)cudaGetLastError();  // clear a stale non-sticky error left by earlier unrelated calls
+    if (!x || !W_r || !W_g || !W_u || !W_d || !dY) return MOE_ERR_INVALID_ARG;
+    if (!al16(x) || !al16(W_r) || !al16(W_g) || !al16(W_u) || !al16(W_d) || !al16(dY) || !al16(gr->dx) ||
+        !al16(gr->dW_g) || !al16(gr->dW_u) || !al16(gr->dW_d))
+        return MOE_ERR_INVALID_ARG;
+    if (sh && (!Ws_g || !Ws_u || !Ws_d || !al16(Ws_g) || !al16(Ws_u) || !al16(Ws_d) || !al16(gr->dWs_g) ||
+               !al16(gr->dWs_u) || !al16(gr->dWs_d)))
+        return MOE_ERR_INVALID_ARG;
+
+    WsView v;
+    make_view(*p, const_cast<void*>(ws), v);
+    const BwdLayout L = bwd_layout(*p);
+    char* b = static_cast<char*>(bws);
+    auto I32 = [&](size_t o) { return reinterpret_cast<int32_t*>(b + o); };
+    auto F32 = [&](size_t o) { return reinterpret_cast<float*>(b + o); };
+    auto B16 = [&](size_t o) { return reinterpret_cast<bf16*>(b + o); };
+    int32_t* padoff = I32(L.padoff);
+    int32_t* tstart = I32(L.tstart);
+    int32_t* mt_start = I32(L.mt_start);
+    auto* counters = reinterpret_cast<unsigned long long*>(b + L.counters);
+    float* logits = F32(L.logits);
+    float* dG = F32(L.dG);
+    float* dwc = F32(L.dwc);
+    bf16 *Wt_d = B16(L.Wt_d), *Wt_gu = B16(L.Wt_gu), *dYp = B16(L.dYp), *dzu = B16(L.dzu);
+    float *Z = F32(L.Z), *U = F32(L.U), *Gd = F32(L.Gd), *dxp = F32(L.dxp);
+    bf16 *doT = B16(L.doT), *xT = B16(L.xT), *hT = B16(L.hT), *dzT = B16(L.dzT), *duT = B16(L.duT);
+    const bf16* xp = static_cast<const bf16*>(v.x_perm);
+    const bf16* hp = static_cast<const bf16*>(v.h);
+    const int32_t* n_rows = v.offsets + E;  // accepted rows, on the device
+    int status = MOE_OK;
+
+    e = cudaMemsetAsync(counters, 0, CNT_COUNT * 8, st);
+    if (e != cudaSuccess) return bwd_fail(e, "memset");
+    // host copy of the per-expert padded column offsets (same rule as bwd_tables_kernel)
+    std::vector<int64_t> hpad(E + 1);
+    int64_t n_tiles = 0;
+    hpad[0] = 0;
+    for (int64_t g = 0; g < E; ++g) {
+        const int64_t R = offsets_host[g + 1] - offsets_host[g];
+        hpad[g + 1] = hpad[g] + ((R + 7) & ~(int64_t)7);
+        n_tiles += (R + kTT - 1) / kTT;
+    }
+
+    bwd_tables_kernel<<<1, 32, 0, st>>>((int)E, v.offsets, padoff, tstart);
+    e = launch_mtile_prefix((int)E, tc_tile_rows(*p), v.offsets, mt_start, st);
+    if (e != cudaSuccess) return bwd_fail(e, "tables");
+    // router scores (bias added in the router kernel): tensor cores when the
+    // fp32 epilogue's 4-column groups tile E_r, else the CUDA-core GEMM
+    if (E % 4 == 0)
+        e = launch_tc_dense(N, E, d, x, W_r, logits, counters, st, &status);
+    else
+        e = simt_gemm<bf16, bf16>(N, E, d, static_cast<const bf16*>(x), d, 1, static_cast<const bf16*>(W_r), d, 1,
+                                  logits, E, st);
+    if (e != cudaSuccess) return bwd_fail(e, "scores");
+    // W_d^T [E, d_f, d] and [W_g^T | W_u^T] [E, d, 2 d_f]
+    bwd_batched_transpose_kernel<<<dim3((unsigned)((d + kTT - 1) / kTT), (unsigned)((df + kTT - 1) / kTT), (unsigned)E),
+                                   256, 0, st>>>(static_cast<const bf16*>(W_d), d, df, Wt_d, d, df * d);
+    bwd_batched_transpose_kernel<<<dim3((unsigned)((df + kTT - 1) / kTT), (unsigned)((d + kTT - 1) / kTT), (unsigned)E),
+                                   256, 0, st>>>(static_cast<const bf16*>(W_g), df, d, Wt_gu, 2 * df, d * 2 * df);
+    bwd_batched_transpose_kernel<<<dim3((unsigned)((df + kTT - 1) / kTT), (unsigned)((d + kTT - 1) / kTT), (unsigned)E),
+                                   256, 0, st>>>(static_cast<const bf16*>(W_u), df, d, Wt_gu + df, 2 * df, d * 2 * df);
+    // dY rows of the accepted paths, bf16
+    bwd_gather_dy_kernel<<<grid_for(8, rows), 256, 0, st>>>(dY, d, v.slot_token, n_rows, 0, rows, N, dYp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "transposes");
+
+    // row-grouped contractions on the grouped tcgen05 kernel (store mode):
+    // its output width is q.d and its K is q.d_f
+    ExpertWeights W0{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+    moe_params q = *p;
+    q.d_f_shared = 0;
+    q.d = (int32_t)df;
+    q.d_f = (int32_t)d;
+    W0.W_d = W_g;
+    e = launch_tc_down(q, DOWN_STORE, N, xp, nullptr, v.offsets, mt_start, W0, nullptr, nullptr, nullptr, Z, counters,
+                       st, &status);
+    if (e != cudaSuccess) return bwd_fail(e, "z (tcgen05)");
+    W0.W_d = W_u;
+    e = launch_tc_down(q, DOWN_STORE, N, xp, nullptr, v.offsets, mt_start, W0, nullptr, nullptr, nullptr, U, counters,
+                       st, &status);
+    if (e != cudaSuccess) return bwd_fail(e, "u (tcgen05)");
+    W0.W_d = Wt_d;
+    e = launch_tc_down(q, DOWN_STORE, N, dYp, nullptr, v.offsets, mt_start, W0, nullptr, nullptr, nullptr, Gd,
+                       counters, st, &status);
+    if (e != cudaSuccess) return bwd_fail(e, "W_d^T dY (tcgen05)");
+    bwd_swiglu_kernel<<<grid_for(8, rows), 256, 0, st>>>(Z, U, Gd, hp, df, v.slot_w, n_rows, 0, rows, dzu, dwc);
+    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "SwiGLU backward");
+    moe_params q2 = *p;
+    q2.d_f_shared = 0;
+    q2.d = (int32_t)d;
+    q2.d_f = (int32_t)(2 * df);
+    W0.W_d = Wt_gu;
+    e = launch_tc_down(q2, DOWN_STORE, N, dzu, nullptr, v.offsets, mt_start, W0, nullptr, nullptr, nullptr, dxp,
+                       counters, st, &status);
+    if (e != cudaSuccess) return bwd_fail(e, "dx rows (tcgen05)");
+
+    // router: score gradient, then dx = dG W_r, dW_r = dG^T X, db = colsum dG
+    RouterBwd ra{};
+    ra.logits = logits;
+    ra.b_r = b_r;
+    ra.ids = v.ids;
+    ra.w = v.w;
+    ra.slot = v.slot;
+    ra.offsets = v.offsets;
+    ra.dwc = dwc;
+    ra.L = v.L;
+    ra.counters = v.counters;
+    ra.dG = dG;
+    ra.N = N;
+    ra.E = (int)E;
+    ra.k = (int)k;
+    ra.norm = p->norm;
+    ra.policy = p->reject_policy;
+    ra.aux_coef = aux_coef;
+    ra.max_rows = rows;
+    bwd_router_kernel<<<grid_for(8, N), 256, 0, st>>>(ra);
+    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "router");
+    const bf16* xb = static_cast<const bf16*>(x);
+    const bf16* Wrb = static_cast<const bf16*>(W_r);
+    e = simt_gemm<float, bf16>(N, d, E, dG, E, 1, Wrb, 1, d, gr->dx, d, st);
+    if (e == cudaSuccess) e = simt_gemm<float, bf16>(E, d, N, dG, 1, E, xb, 1, d, gr->dW_r, d, st);
+    if (e != cudaSuccess) return bwd_fail(e, "router contractions");
+    if (gr->db_r) {
+        bwd_colsum_kernel<<<(unsigned)((E + 31) / 32), 256, 0, st>>>(dG, N, (int)E, gr->db_r);
+        if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "db");
+    }
+
+    // shared expert: weight 1 on every token
+    float* dxs = nullptr;
+    if (sh) {
+        const int64_t Np = (N + 7) & ~(int64_t)7;
+        bf16 *dYs = B16(L.dYs), *dzus = B16(L.dzus), *WsT_d = B16(L.WsT_d), *WsT_gu = B16(L.WsT_gu);
+        float *Zs = F32(L.Zs), *Us = F32(L.Us), *Gs = F32(L.Gs);
+        dxs = F32(L.dxs);
+        int32_t *sh_off = I32(L.sh_off), *sh_pad = I32(L.sh_padoff), *sh_ts = I32(L.sh_tstart);
+        bwd_single_group_kernel<<<1, 32, 0, st>>>((int32_t)N, sh_off);
+        bwd_tables_kernel<<<1, 32, 0, st>>>(1, sh_off, sh_pad, sh_ts);
+        bwd_gather_dy_kernel<<<grid_for(8, N), 256, 0, st>>>(dY, d, nullptr, nullptr, N, N, N, dYs);
+        bwd_batched_transpose_kernel<<<dim3((unsigned)((d + kTT - 1) / kTT), (unsigned)((dfs + kTT - 1) / kTT), 1), 256,
+                                       0, st>>>(static_cast<const bf16*>(Ws_d), d, dfs, WsT_d, d, 0);
+        bwd_batched_transpose_kernel<<<dim3((unsigned)((dfs + kTT - 1) / kTT), (unsigned)((d + kTT - 1) / kTT), 1), 256,
+                                       0, st>>>(static_cast<const bf16*>(Ws_g), dfs, d, WsT_gu, 2 * dfs, 0);
+        bwd_batched_transpose_kernel<<<dim3((unsigned)((dfs + kTT - 1) / kTT), (unsigned)((d + kTT - 1) / kTT), 1), 256,
+                                       0, st>>>(static_cast<const bf16*>(Ws_u), dfs, d, WsT_gu + dfs, 2 * dfs, 0);
+        if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "shared transposes");
+        e = launch_tc_dense(N, dfs, d, x, Ws_g, Zs, counters, st, &status);
+        if (e == cudaSuccess) e = launch_tc_dense(N, dfs, d, x, Ws_u, Us, counters, st, &status);
+        if (e == cudaSuccess) e = launch_tc_dense(N, dfs, d, dYs, WsT_d, Gs, counters, st, &status);
+        if (e != cudaSuccess) return bwd_fail(e, "shared z, u, W_d^T dY (tcgen05)");
+        bwd_swiglu_kernel<<<grid_for(8, N), 256, 0, st>>>(Zs, Us, Gs, static_cast<const bf16*>(v.h_shared), dfs,
+                                                          nullptr, nullptr, N, N, dzus, nullptr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "shared SwiGLU backward");
+        e = launch_tc_dense(N, d, 2 * dfs, dzus, WsT_gu, dxs, counters, st, &status);
+        if (e != cudaSuccess) return bwd_fail(e, "shared dx (tcgen05)");
+        // weight gradients over all tokens (K = N, padded to a multiple of 8)
+        bf16 *dYsT = B16(L.dYsT), *xsT = B16(L.xsT), *hsT = B16(L.hsT), *dzsT = B16(L.dzsT), *dusT = B16(L.dusT);
+        const unsigned tiles_sh = (unsigned)((N + kTT - 1) / kTT);
+        bwd_group_transpose_kernel<false><<<dim3(tiles_sh, (unsigned)((d + kTT - 1) / kTT)), 256, 0, st>>>(
+            dYs, d, d, sh_off, sh_pad, sh_ts, 1, nullptr, dYsT);
+        bwd_group_transpose_kernel<false><<<dim3(tiles_sh, (unsigned)((d + kTT - 1) / kTT)), 256, 0, st>>>(
+            xb, d, d, sh_off, sh_pad, sh_ts, 1, nullptr, xsT);
+        bwd_group_transpose_kernel<false><<<dim3(tiles_sh, (unsigned)((dfs + kTT - 1) / kTT)), 256, 0, st>>>(
+            static_cast<const bf16*>(v.h_shared), dfs, dfs, sh_off, sh_pad, sh_ts, 1, nullptr, hsT);
+        bwd_group_transpose_kernel<false><<<dim3(tiles_sh, (unsigned)((dfs + kTT - 1) / kTT)), 256, 0, st>>>(
+            dzus, 2 * dfs, dfs, sh_off, sh_pad, sh_ts, 1, nullptr, dzsT);
+        bwd_group_transpose_kernel<false><<<dim3(tiles_sh, (unsigned)((dfs + kTT - 1) / kTT)), 256, 0, st>>>(
+            dzus + dfs, 2 * dfs, dfs, sh_off, sh_pad, sh_ts, 1, nullptr, dusT);
+        if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "shared row transposes");
+        e = launch_tc_dense(d, dfs, Np, dYsT, hsT, gr->dWs_d, counters, st, &status);
+        if (e == cudaSuccess) e = launch_tc_dense(dfs, d, Np, dzsT, xsT, gr->dWs_g, counters, st, &status);
+        if (e == cudaSuccess) e = launch_tc_dense(dfs, d, Np, dusT, xsT, gr->dWs_u, counters, st, &status);
+        if (e != cudaSuccess) return bwd_fail(e, "shared weight gradients (tcgen05)");
+    }
+
+    // dx: router part (written above) + expert rows + shared expert
+    bwd_dx_kernel<<<grid_for(8, N), 256, 0, st>>>(gr->dx, dxp, dxs, v.ids, v.slot, v.offsets, N, d, (int)k, (int)E,
+                                                  rows);
+    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "dx");
+
+    // weight gradients: per-expert column blocks of the transposed operands
+    if (n_tiles > 0) {
+        const dim3 gd((unsigned)n_tiles, (unsigned)((d + kTT - 1) / kTT));
+        const dim3 gf((unsigned)n_tiles, (unsigned)((df + kTT - 1) / kTT));
+        bwd_group_transpose_kernel<true><<<gd, 256, 0, st>>>(dYp, d, d, v.offsets, padoff, tstart, (int)E, v.slot_w,
+                                                             doT);
+        bwd_group_transpose_kernel<false><<<gd, 256, 0, st>>>(xp, d, d, v.offsets, padoff, tstart, (int)E, nullptr,
+                                                              xT);
+        bwd_group_transpose_kernel<false><<<gf, 256, 0, st>>>(hp, df, df, v.offsets, padoff, tstart, (int)E, nullptr,
+                                                              hT);
+        bwd_group_transpose_kernel<false><<<gf, 256, 0, st>>>(dzu, 2 * df, df, v.offsets, padoff, tstart, (int)E,
+                                                              nullptr, dzT);
+        bwd_group_transpose_kernel<false><<<gf, 256, 0, st>>>(dzu + df, 2 * df, df, v.offsets, padoff, tstart, (int)E,
+                                                              nullptr, duT);
+        if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "row transposes");
+    }
+    for (int64_t g = 0; g < E; ++g) {
+        const int64_t Kp = hpad[g + 1] - hpad[g];
+        float* gWd = gr->dW_d + g * d * df;
+        float* gWg = gr->dW_g + g * df * d;
+        float* gWu = gr->dW_u + g * df * d;
+        if (Kp == 0) {
+            e = cudaMemsetAsync(gWd, 0, sizeof(float) * d * df, st);
+            if (e == cudaSuccess) e = cudaMemsetAsync(gWg, 0, sizeof(float) * d * df, st);
+            if (e == cudaSuccess) e = cudaMemsetAsync(gWu, 0, sizeof(float) * d * df, st);
+            if (e != cudaSuccess) return bwd_fail(e, "memset");
+            continue;
+        }
+        e = launch_tc_dense(d, df, Kp, doT + d * hpad[g], hT + df * hpad[g], gWd, counters, st, &status);
+        if (e == cudaSuccess)
+            e = launch_tc_dense(df, d, Kp, dzT + df * hpad[g], xT + d * hpad[g], gWg, counters, st, &status);
+        if (e == cudaSuccess)
+            e = launch_tc_dense(df, d, Kp, duT + df * hpad[g], xT + d * hpad[g], gWu, counters, st, &status);
+        if (e != cudaSuccess) return bwd_fail(e, "weight gradients (tcgen05)");
+    }
+    return MOE_OK;
+}
+
+moe_status moe_backward_check(const moe_params* p, const void* bws, moe_stream_t stream) {
+    const moe_status s = bwd_check(p);
+    if (s != MOE_OK) return s;
+    if (!bws || !al16(bws)) return MOE_ERR_WORKSPACE;
+    unsigned long long cnt[CNT_COUNT];
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(cnt, static_cast<const char*>(bws) + bwd_layout(*p).counters, sizeof(cnt),
+                                    cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return bwd_fail(e, "check");
+    if (cnt[CNT_DEVICE_ERROR] & DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+    return MOE_OK;
+}
+
+}  // extern "C"

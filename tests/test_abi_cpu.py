@@ -162,3 +162,58 @@ def test_host_tensors_are_refused_by_the_binding():
     with pytest.raises(ValueError):
         moe.moe_forward(p, torch.zeros(4, 64), None, None, None, None, None, None, None, None, None,
                         None, None, stream=0)
+
+
+def test_backward_checks_arguments_on_the_host():
+    L = moe.lib()
+    assert ctypes.sizeof(moe.Grads) == 9 * 8
+    p = moe.params(16, 64, 64, 8, 2, c=1.0)
+    # fp32 layers have no backward; E_r above the router kernel's limit neither
+    assert L.moe_backward_workspace_size(ctypes.byref(moe.params(16, 64, 64, 8, 2, dtype=moe.MOE_F32)),
+                                         ctypes.byref(ctypes.c_size_t())) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_backward_workspace_size(ctypes.byref(moe.params(16, 64, 64, 300, 2)),
+                                         ctypes.byref(ctypes.c_size_t())) == moe.MOE_ERR_UNSUPPORTED
+    n = moe.moe_backward_workspace_size(p)
+    assert n >= 8 * 64 * 64 * 2 * 3            # the transposed expert weights alone
+    # the worst case grows with the routed rows N k
+    assert moe.moe_backward_workspace_size(moe.params(32, 64, 64, 8, 2, c=1.0)) > n
+    fake = 4096                                  # aligned, never dereferenced: the checks come first
+    g = moe.Grads(*([fake] * 9))
+
+    def call(offsets, ws=fake, bws=fake, grads=g, aux=0.0):
+        arr = (ctypes.c_int32 * len(offsets))(*offsets)
+        return L.moe_backward(ctypes.byref(p), aux, arr, fake, fake, None, fake, fake, fake, None, None, None,
+                              fake, ws, ctypes.byref(grads) if grads is not None else None, bws, None)
+
+    good = [0, 4, 4, 8, 12, 16, 20, 24, 28]
+    assert call(good, ws=None) == moe.MOE_ERR_WORKSPACE
+    assert call(good, bws=fake + 8) == moe.MOE_ERR_WORKSPACE
+    assert call(good, grads=None) == moe.MOE_ERR_INVALID_ARG
+    assert call(good, aux=float("nan")) == moe.MOE_ERR_INVALID_ARG
+    assert call([1] + good[1:]) == moe.MOE_ERR_INVALID_ARG             # does not start at 0
+    assert call([0, 4, 3] + good[3:]) == moe.MOE_ERR_INVALID_ARG       # decreasing
+    assert call(good[:-1] + [33]) == moe.MOE_ERR_INVALID_ARG           # more rows than N k
+    missing = moe.Grads(*([fake] * 3 + [None] + [fake] * 5))          # dW_g missing
+    assert call(good, grads=missing) == moe.MOE_ERR_INVALID_ARG
+    ps = moe.params(16, 64, 64, 8, 2, d_f_shared=64)
+    arr = (ctypes.c_int32 * 9)(*good)
+    no_shared = moe.Grads(*([fake] * 6 + [None] * 3))
+    assert L.moe_backward(ctypes.byref(ps), 0.0, arr, fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
+                          fake, ctypes.byref(no_shared), fake, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_backward_of_an_empty_batch_needs_no_dx():
+    # an empty dx tensor has no storage (a null pointer): N = 0 must pass the
+    # argument checks without it (on a host without a GPU the call then fails
+    # in CUDA; with a GPU it would write to the fake addresses, so it is skipped)
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("fake device addresses are only safe without a GPU")
+    L = moe.lib()
+    p = moe.params(0, 64, 64, 8, 2)
+    fake = 4096
+    g = moe.Grads(None, *([fake] * 8))
+    arr = (ctypes.c_int32 * 9)(*([0] * 9))
+    r = L.moe_backward(ctypes.byref(p), 0.0, arr, None, None, None, None, None, None, None, None, None, None,
+                       fake, ctypes.byref(g), fake, None)
+    assert r not in (moe.MOE_ERR_INVALID_ARG, moe.MOE_ERR_WORKSPACE)

@@ -1,0 +1,143 @@
+"""Backward pass on the GPU (moe_backward through the C ABI) against the
+gradient oracle, on seeded inputs.
+
+The oracle runs on the GPU forward's own routing records (ids, weights,
+slots), so both sides differentiate the same piecewise-smooth function.
+Tolerances (max-abs error over max-abs reference, per gradient):
+  * expert and shared-expert weight gradients and dx: 5e-3.  The tensor-core
+    operands (dY, wc dY, dz, du and the forward's h) are bf16 on both sides,
+    but the GPU rounds values it accumulated in fp32, so an operand can land
+    one bf16 step (2^-8 = 3.9e-3 relative) away from the oracle's where the
+    fp32 value sits near a rounding boundary; such a flip moves one term of
+    a sum, so an output element moves by less than 2^-8 of the largest
+    output, plus fp32 accumulation error;
+  * router gradients dW_r and db_r: 2e-3.  They come from the combine-weight
+    gradients <W_d^T dY_t, h>, fp32 sums over d_f of bf16-exact products,
+    and fp32 router arithmetic; a missing term of the chain (an overflow
+    policy, the renormalisation, the balance objective) moves them by far
+    more;
+  * the balance objective's gradient alone (dY = 0): 1e-4.
+Cases span single-CTA and CTA-pair tiles, ragged row, column and K tails,
+capacity rejection under both overflow policies, acceptance by weight, WLR
+pruning, a shared expert, an expert count that is not a multiple of 4 (score
+recomputation on the CUDA cores) and the empty batch.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import seeded_inputs as si
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover - GPU tests need a device
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import sparse_mixture_experts_25_b200 as moe  # noqa: E402
+
+W = si.WORKLOADS
+CASES = {
+    "mixtral_small": W["mixtral_bf16"].scaled("bwd_mixtral_small", N=512, d=320, d_f=384),
+    "pair_tiles": W["mixtral_bf16"].scaled("bwd_pair", N=1600, d=320, d_f=384, E=2, k=1),
+    "qwen3_capped_aux": W["qwen3_skew_bf16"].scaled("bwd_qwen3", N=1024, d=256, d_f=192, E=32, k=4),
+    "deepseek_shared": W["deepseek_shared_bf16"].scaled("bwd_deepseek", N=384, d=448, d_f=128, E=64, k=6,
+                                                        d_f_shared=192),
+    "wdmoe_wlr": W["wdmoe_decode_bf16"].scaled("bwd_wdmoe", N=64, d=512, d_f=640),
+    "renorm_reject": W["qwen3_skew_bf16"].scaled("bwd_renorm_reject", N=1024, d=256, d_f=192, E=16, k=2,
+                                                 reject_policy=1),
+    "weight_order": W["qwen3_skew_bf16"].scaled("bwd_weight_order", N=700, d=128, d_f=192, E=16, k=2, c=0.8,
+                                                accept_order=1, reject_policy=1),
+    "odd_experts": W["mixtral_bf16"].scaled("bwd_odd_experts", N=200, d=64, d_f=64, E=34, k=3, c=1.0),
+    "one_expert_ragged": W["mixtral_bf16"].scaled("bwd_one_expert", N=200, d=64, d_f=136, E=1, k=1),
+}
+AUX = {"qwen3_capped_aux": 0.5, "weight_order": 0.3, "odd_experts": 1.0}
+
+
+def _grads(w, device="cuda"):
+    shapes = {"dx": (w.N, w.d), "dW_r": (w.E, w.d), "db_r": (w.E,), "dW_g": (w.E, w.d_f, w.d),
+              "dW_u": (w.E, w.d_f, w.d), "dW_d": (w.E, w.d, w.d_f)}
+    if w.d_f_shared:
+        shapes.update({"dWs_g": (w.d_f_shared, w.d), "dWs_u": (w.d_f_shared, w.d), "dWs_d": (w.d, w.d_f_shared)})
+    return {n: torch.full(s, float("nan"), dtype=torch.float32, device=device) for n, s in shapes.items()}
+
+
+def _backward(w, inp, full, dY, aux):
+    p, dev, ws = full["p"], full["dev"], full["ws"]
+    g = _grads(w)
+    bws = torch.empty(moe.moe_backward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    moe.moe_backward(p, full["rec"]["offsets"], dev["x"], dev["W_r"], dev.get("b_r"), dev["W_g"], dev["W_u"],
+                     dev["W_d"], dev.get("Ws_g"), dev.get("Ws_u"), dev.get("Ws_d"),
+                     torch.from_numpy(dY).cuda(), ws, g, bws, aux_coef=aux)
+    assert moe.moe_backward_check(p, bws) == moe.MOE_OK
+    return {n: t.cpu().numpy().astype(np.float64) for n, t in g.items()}
+
+
+def _reference(w, inp, rec, dY, aux):
+    Ws = (inp["Ws_g"], inp["Ws_u"], inp["Ws_d"]) if w.d_f_shared else None
+    return oracle.backward(inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], dY, rec["ids"], rec["w"],
+                           rec["slot"], norm=w.norm, reject_policy=w.reject_policy, b_r=inp.get("b_r"), Ws=Ws,
+                           aux_coef=aux)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_backward_matches_oracle(name):
+    w = CASES[name]
+    inp = si.inputs(w)
+    full = parity.gpu_forward(w, inp)
+    assert full["status"] == moe.MOE_OK
+    if w.c > 0:
+        assert full["stats"]["rejected"] > 0       # the capacity binds
+    dY = si.upstream_gradient(w)
+    aux = AUX.get(name, 0.0)
+    got = _backward(w, inp, full, dY, aux)
+    ref = _reference(w, inp, full["rec"], dY, aux)
+    errs = {}
+    for n, g in got.items():
+        assert np.isfinite(g).all(), n
+        errs[n] = parity.rel_err(g, ref[n])
+        tol = 2e-3 if n in ("dW_r", "db_r") else 5e-3
+        assert errs[n] <= tol, (n, errs[n], errs)
+    # experts that received no rows have exactly zero weight gradients
+    empty = np.nonzero(full["rec"]["acc"] == 0)[0]
+    for e in empty:
+        assert not got["dW_g"][e].any() and not got["dW_u"][e].any() and not got["dW_d"][e].any()
+
+
+def test_balance_objective_gradient_alone():
+    w = CASES["qwen3_capped_aux"]
+    inp = si.inputs(w)
+    full = parity.gpu_forward(w, inp)
+    dY = np.zeros((w.N, w.d), np.float32)
+    got = _backward(w, inp, full, dY, 1.0)
+    ref = _reference(w, inp, full["rec"], dY, 1.0)
+    for n in ("dW_g", "dW_u", "dW_d"):
+        assert not got[n].any(), n
+    for n in ("dx", "dW_r", "db_r"):
+        assert np.abs(ref[n]).max() > 0
+        assert parity.rel_err(got[n], ref[n]) <= 1e-4, n
+
+
+def test_backward_empty_batch():
+    w = CASES["mixtral_small"].scaled("bwd_empty", N=0)
+    inp = si.inputs(w)
+    full = parity.gpu_forward(w, inp)
+    got = _backward(w, inp, full, np.zeros((0, w.d), np.float32), 0.0)
+    for n, g in got.items():
+        assert not g.any(), n
+
+
+def test_backward_rejects_bad_offsets():
+    w = CASES["mixtral_small"]
+    inp = si.inputs(w)
+    full = parity.gpu_forward(w, inp)
+    p, dev = full["p"], full["dev"]
+    g = _grads(w)
+    bws = torch.empty(moe.moe_backward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    bad = full["rec"]["offsets"].copy()
+    bad[-1] = w.N * w.k + 1
+    dY = torch.zeros(w.N, w.d, device="cuda")
+    with pytest.raises(moe.MoEError):
+        moe.moe_backward(p, bad, dev["x"], dev["W_r"], None, dev["W_g"], dev["W_u"], dev["W_d"], None, None, None,
+                         dY, full["ws"], g, bws)
