@@ -447,14 +447,16 @@ MOE_API moe_status moe_soft_check(const moe_soft_params* p, const void* ws, moe_
  * hidden activations are read); offsets_host a HOST copy of the forward's
  * offsets [E_r + 1] (ws's "offsets" array, read after the forward finished:
  * the per-expert weight-gradient launches are sized by it); grads the output
- * buffers (device, fp32, overwritten; see moe_grads); bws the backward
- * workspace (moe_backward_workspace_size bytes, 256-byte aligned
- * recommended); aux_coef the objective's coefficient (0: none).
+ * buffers (device, fp32, overwritten; see moe_grads); bws, bws_bytes the
+ * backward workspace (at least moe_backward_workspace_size bytes for these
+ * offsets, 256-byte aligned recommended); aux_coef the objective's
+ * coefficient (0: none).
  * Constraints: dtype MOE_BF16 (MOE_ERR_UNSUPPORTED for fp32 layers), E_r <=
  * 256, k <= 32, N <= 65535 * 64; single routing group (not after
  * moe_forward_end).
  * Errors: MOE_ERR_INVALID_ARG (null or misaligned pointers, offsets_host not
- * a non-decreasing prefix from 0 to at most N k), MOE_ERR_WORKSPACE,
+ * a non-decreasing prefix from 0 to at most N k), MOE_ERR_WORKSPACE (missing,
+ * misaligned or smaller than needed),
  * MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA (with moe_last_error).  Asynchronous on
  * `stream`; the library allocates nothing.  N = 0 zeroes the weight
  * gradients and returns.
@@ -471,14 +473,19 @@ typedef struct moe_grads {
     float* dWs_d;   /* [d, d_f_shared]     required when d_f_shared > 0          */
 } moe_grads;
 
-/* Bytes of the backward workspace for p (the worst case over routings). */
-MOE_API moe_status moe_backward_workspace_size(const moe_params* p, size_t* bytes);
+/* Bytes of the backward workspace for p and the forward's offsets (host,
+ * [E_r + 1]; the weight-gradient operands take E_r x max_e ceil64(rows of
+ * expert e) columns).  offsets_host NULL: the bound for any routing (every
+ * expert at min(capacity, N) rows).  MOE_ERR_INVALID_ARG for invalid
+ * offsets. */
+MOE_API moe_status moe_backward_workspace_size(const moe_params* p, const int32_t* offsets_host,
+                                               size_t* bytes);
 
 MOE_API moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offsets_host,
                                 const void* x, const void* W_r, const float* b_r, const void* W_g,
                                 const void* W_u, const void* W_d, const void* Ws_g, const void* Ws_u,
                                 const void* Ws_d, const float* dY, const void* ws, const moe_grads* grads,
-                                void* bws, moe_stream_t stream);
+                                void* bws, size_t bws_bytes, moe_stream_t stream);
 
 /* Waits for `stream` and reports MOE_ERR_TIMEOUT if a bounded device wait of
  * the last moe_backward on `bws` gave up (its tensor-core GEMMs record that in

@@ -129,9 +129,9 @@ def lib():
         L.moe_soft_workspace_size.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t)]
         L.moe_soft_forward.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_soft_check.argtypes = [sp, _P, _P]
-        L.moe_backward_workspace_size.argtypes = [pp, ctypes.POINTER(ctypes.c_size_t)]
+        L.moe_backward_workspace_size.argtypes = [pp, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_size_t)]
         L.moe_backward.argtypes = [pp, ctypes.c_float, ctypes.POINTER(ctypes.c_int32), _P, _P, _P, _P, _P, _P,
-                                   _P, _P, _P, _P, _P, ctypes.POINTER(Grads), _P, _P]
+                                   _P, _P, _P, _P, _P, ctypes.POINTER(Grads), _P, ctypes.c_size_t, _P]
         L.moe_backward_check.argtypes = [pp, _P, _P]
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
@@ -369,9 +369,21 @@ def workspace_x_perm(p: Params, ws):
     return ws[L["x_perm"]:L["x_perm"] + nbytes].view(dt).view(p.N * p.k, p.d)
 
 
-def moe_backward_workspace_size(p: Params) -> int:
+def _offsets_arg(p, offsets_host):
+    import numpy as np
+    off = np.ascontiguousarray(np.asarray(offsets_host), dtype=np.int32)
+    if off.shape != (p.E_r + 1,):
+        raise ValueError("offsets_host must hold E_r + 1 entries")
+    return off
+
+
+def moe_backward_workspace_size(p: Params, offsets_host=None) -> int:
+    """Backward workspace bytes for the forward's offsets (host array), or
+    the bound for any routing when offsets_host is None."""
     n = ctypes.c_size_t()
-    _check(lib().moe_backward_workspace_size(ctypes.byref(p), ctypes.byref(n)), "moe_backward_workspace_size")
+    off = None if offsets_host is None else _offsets_arg(p, offsets_host)
+    ptr = None if off is None else off.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    _check(lib().moe_backward_workspace_size(ctypes.byref(p), ptr, ctypes.byref(n)), "moe_backward_workspace_size")
     return n.value
 
 
@@ -381,15 +393,14 @@ def moe_backward(p, offsets_host, x, W_r, b_r, W_g, W_u, W_d, Ws_g, Ws_u, Ws_d, 
     ws (see moe_backward in include/moe.h).  offsets_host: the forward's
     offsets [E_r + 1] on the host (a numpy array or CPU tensor); grads: dict
     of device fp32 tensors keyed by GRAD_NAMES (db_r and the shared-expert
-    entries may be missing or None)."""
-    import numpy as np
-    off = np.ascontiguousarray(np.asarray(offsets_host), dtype=np.int32)
-    if off.shape != (p.E_r + 1,):
-        raise ValueError("offsets_host must hold E_r + 1 entries")
+    entries may be missing or None); bws: a uint8 device tensor of at least
+    moe_backward_workspace_size(p, offsets_host) bytes."""
+    off = _offsets_arg(p, offsets_host)
     g = Grads(*[_ptr(grads.get(n)) for n in GRAD_NAMES])
     _check(lib().moe_backward(ctypes.byref(p), float(aux_coef), off.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                               _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W_g), _ptr(W_u), _ptr(W_d), _ptr(Ws_g), _ptr(Ws_u),
-                              _ptr(Ws_d), _ptr(dY), _ptr(ws), ctypes.byref(g), _ptr(bws), _stream(stream)),
+                              _ptr(Ws_d), _ptr(dY), _ptr(ws), ctypes.byref(g), _ptr(bws), int(bws.numel()),
+                              _stream(stream)),
            "moe_backward")
 
 

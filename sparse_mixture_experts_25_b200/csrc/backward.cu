@@ -24,13 +24,17 @@
 // the dimensions relabelled (its "d_f" is K, its "d" the output width), which
 // needs W_d^T [E, d_f, d] and [W_g^T | W_u^T] [E, d, 2 d_f]: both are written
 // once per call by a batched transpose.  The weight gradients contract over an
-// expert's rows, so their operands are transposed per expert into column
-// blocks padded to a multiple of 8 rows with zeros (16-byte TMA rows); the
-// host launches one dense GEMM per expert with the row counts it was given.
+// expert's rows, so their operands are transposed into blocks [E][C][Kmax]
+// (expert e's C rows hold its R_e row values as columns, zero-padded to whole
+// 64-wide K blocks; Kmax = the largest padded R_e, from the host offsets).
+// Read as a grouped GEMM whose group e owns rows e C .. e C + C - 1, one
+// launch per gradient computes every expert's dW_e = A_e B_e^T, each group
+// contracting over its own K blocks only.
 #include <cuda_bf16.h>
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <vector>
 
 #include "moe_internal.cuh"
@@ -63,23 +67,27 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// padoff[g]: first column of group g's transposed block (groups padded to a
-// multiple of 8 rows); tstart[g]: first 64-row transposition tile of group g.
-// One thread: G <= 1024.
-__global__ void bwd_tables_kernel(int G, const int32_t* __restrict__ offsets, int32_t* __restrict__ padoff,
-                                  int32_t* __restrict__ tstart) {
+// tstart[g]: first 64-row transposition tile of group g; nkb[g]: its 64-wide
+// K blocks, max(1, ceil(R_g / 64)) (an empty group still gets one block of
+// zeros, so its gradient tile is written).  One thread: G <= 1024.
+__global__ void bwd_tables_kernel(int G, const int32_t* __restrict__ offsets, int32_t* __restrict__ tstart,
+                                  int32_t* __restrict__ nkb) {
     if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    int32_t p = 0, t = 0;
+    int32_t t = 0;
     for (int g = 0; g < G; ++g) {
-        padoff[g] = p;
-        tstart[g] = t;
         int32_t R = offsets[g + 1] - offsets[g];
         if (R < 0) R = 0;
-        p += (R + 7) & ~7;
-        t += (R + kTT - 1) / kTT;
+        const int32_t n = R > 0 ? (R + kTT - 1) / kTT : 1;
+        tstart[g] = t;
+        nkb[g] = n;
+        t += n;
     }
-    padoff[G] = p;
     tstart[G] = t;
+}
+
+// off[e] = e C for e = 0..E: groups of C consecutive rows
+__global__ void bwd_strided_offsets_kernel(int E, int32_t C, int32_t* __restrict__ off) {
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) off[e] = e * C;
 }
 
 __global__ void bwd_single_group_kernel(int32_t n, int32_t* __restrict__ off) {
@@ -90,17 +98,19 @@ __global__ void bwd_single_group_kernel(int32_t n, int32_t* __restrict__ off) {
 }
 
 // Group-wise transposition: for group g (rows offsets[g] .. offsets[g+1]-1 of
-// src [*, ld], columns 0..C-1), dst block g = dst + C padoff[g] is [C, Rp_g]
-// row-major with dst[c, r] = bf16(scale[row] src[row, c]) (scale optional) and
-// zeros in the padding columns r in [R_g, Rp_g).  64 x 64 tiles through shared
-// memory, 16-byte global accesses.  C, ld multiples of 8.
+// src [*, ld], columns 0..C-1), block g = dst + g gstride is [C, kstride]
+// row-major with dst[c, r] = bf16(scale[row] src[row, c]) (scale optional)
+// for r < R_g and zeros for r in [R_g, 64 nkb_g) (the group's K blocks).
+// 64 x 64 tiles through shared memory, 16-byte global accesses; C, ld and
+// kstride multiples of 8.
 template <bool SCALE>
 __global__ void __launch_bounds__(256)
     bwd_group_transpose_kernel(const bf16* __restrict__ src, int64_t ld, int64_t C, const int32_t* __restrict__ offsets,
-                               const int32_t* __restrict__ padoff, const int32_t* __restrict__ tstart, int G,
-                               const float* __restrict__ scale, bf16* __restrict__ dst) {
+                               const int32_t* __restrict__ tstart, int G, const float* __restrict__ scale,
+                               bf16* __restrict__ dst, int64_t kstride, int64_t gstride) {
     __shared__ float tile[kTT][kTT + 1];
     const int bx = blockIdx.x;
+    if (bx >= tstart[G]) return;
     int lo = 0, hi = G - 1;  // last group whose first tile is <= bx
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -109,7 +119,6 @@ __global__ void __launch_bounds__(256)
     }
     const int g = lo;
     const int64_t R = offsets[g + 1] - offsets[g];
-    const int64_t Rp = padoff[g + 1] - padoff[g];
     const int64_t lr0 = (int64_t)(bx - tstart[g]) * kTT;
     const int64_t c0 = (int64_t)blockIdx.y * kTT;
     const int t = threadIdx.x, cc = (t & 7) * 8;
@@ -134,18 +143,18 @@ __global__ void __launch_bounds__(256)
         for (int i = 0; i < 8; ++i) tile[rr][cc + i] = v[i];
     }
     __syncthreads();
-    bf16* base = dst + C * (int64_t)padoff[g];
+    bf16* base = dst + (int64_t)g * gstride;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int oc = (t >> 3) + h * 32;
         const int64_t c = c0 + oc, lr = lr0 + cc;
-        if (c < C && lr < Rp) {
+        if (c < C && lr + 8 <= kstride) {
             uint4 q;
             q.x = pk2(tile[cc][oc], tile[cc + 1][oc]);
             q.y = pk2(tile[cc + 2][oc], tile[cc + 3][oc]);
             q.z = pk2(tile[cc + 4][oc], tile[cc + 5][oc]);
             q.w = pk2(tile[cc + 6][oc], tile[cc + 7][oc]);
-            *reinterpret_cast<uint4*>(base + c * Rp + lr) = q;
+            *reinterpret_cast<uint4*>(base + c * kstride + lr) = q;
         }
     }
 }
@@ -521,33 +530,54 @@ cudaError_t simt_gemm(int64_t M, int64_t N, int64_t K, const TA* A, int64_t sam,
 // Workspace
 // ---------------------------------------------------------------------------
 struct BwdLayout {
-    size_t padoff, tstart, mt_start, sh_off, sh_padoff, sh_tstart, counters;
+    size_t tstart, nkb, mt_start, offs_d, offs_f, mt_d, mt_f, sh_off, sh_tstart, sh_nkb, counters;
     size_t logits, dG, dwc, Wt_d, Wt_gu, dYp, Z, U, Gd, dzu, dxp, doT, xT, hT, dzT, duT;
     size_t dYs, Zs, Us, Gs, dzus, dxs, WsT_d, WsT_gu, dYsT, xsT, hsT, dzsT, dusT;
+    int64_t Kmax, Kmax_sh;
     size_t total;
 };
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-BwdLayout bwd_layout(const moe_params& p) {
+int64_t up64(int64_t v) { return (v + kTT - 1) / kTT * kTT; }
+
+// Kmax: the widest expert block of the weight-gradient operands (64 times the
+// largest nkb), from the host offsets, else the bound min(capacity, N).
+int64_t kmax_of(const moe_params& p, const int32_t* offsets_host) {
+    int64_t m = kTT;
+    if (offsets_host) {
+        for (int64_t g = 0; g < p.E_r; ++g) m = std::max(m, up64((int64_t)offsets_host[g + 1] - offsets_host[g]));
+        return m;
+    }
+    int64_t C = p.N;
+    moe_capacity(&p, &C);
+    return std::max(m, up64(std::min<int64_t>(C, p.N)));
+}
+
+BwdLayout bwd_layout(const moe_params& p, int64_t Kmax) {
     const size_t N = (size_t)p.N, d = (size_t)p.d, df = (size_t)p.d_f, E = (size_t)p.E_r;
     const size_t rows = N * (size_t)p.k;
-    const size_t Rp = rows + 7 * E;  // padded columns of the per-expert transposed blocks
     const size_t ds = p.d_f_shared > 0 ? (size_t)p.d_f_shared : 0;
-    const size_t Np = (N + 7) & ~(size_t)7;
     BwdLayout L{};
+    L.Kmax = Kmax;
+    L.Kmax_sh = std::max<int64_t>(kTT, up64(p.N));
+    const size_t K = (size_t)Kmax, Ks = (size_t)L.Kmax_sh;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;
         off = up256(off + bytes);
         return o;
     };
-    L.padoff = take((E + 1) * 4);
     L.tstart = take((E + 1) * 4);
+    L.nkb = take(E * 4);
     L.mt_start = take((E + 1) * 4);
+    L.offs_d = take((E + 1) * 4);
+    L.offs_f = take((E + 1) * 4);
+    L.mt_d = take((E + 1) * 4);
+    L.mt_f = take((E + 1) * 4);
     L.sh_off = take(2 * 4);
-    L.sh_padoff = take(2 * 4);
     L.sh_tstart = take(2 * 4);
+    L.sh_nkb = take(4);
     L.counters = take(CNT_COUNT * 8);
     L.logits = take(N * E * 4);
     L.dG = take(N * E * 4);
@@ -560,11 +590,11 @@ BwdLayout bwd_layout(const moe_params& p) {
     L.Gd = take(rows * df * 4);
     L.dzu = take(rows * 2 * df * 2);
     L.dxp = take(rows * d * 4);
-    L.doT = take(d * Rp * 2);
-    L.xT = take(d * Rp * 2);
-    L.hT = take(df * Rp * 2);
-    L.dzT = take(df * Rp * 2);
-    L.duT = take(df * Rp * 2);
+    L.doT = take(E * d * K * 2);
+    L.xT = take(E * d * K * 2);
+    L.hT = take(E * df * K * 2);
+    L.dzT = take(E * df * K * 2);
+    L.duT = take(E * df * K * 2);
     if (ds) {
         L.dYs = take(N * d * 2);
         L.Zs = take(N * ds * 4);
@@ -574,11 +604,11 @@ BwdLayout bwd_layout(const moe_params& p) {
         L.dxs = take(N * d * 4);
         L.WsT_d = take(ds * d * 2);
         L.WsT_gu = take(d * 2 * ds * 2);
-        L.dYsT = take(d * Np * 2);
-        L.xsT = take(d * Np * 2);
-        L.hsT = take(ds * Np * 2);
-        L.dzsT = take(ds * Np * 2);
-        L.dusT = take(ds * Np * 2);
+        L.dYsT = take(d * Ks * 2);
+        L.xsT = take(d * Ks * 2);
+        L.hsT = take(ds * Ks * 2);
+        L.dzsT = take(ds * Ks * 2);
+        L.dusT = take(ds * Ks * 2);
     }
     L.total = off;
     return L;
@@ -601,7 +631,17 @@ moe_status bwd_check(const moe_params* p) {
     if (p->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
     if (p->E_r > kMaxRouterExperts || p->k > kMaxK) return MOE_ERR_UNSUPPORTED;
     if (p->N > (int64_t)65535 * 64) return MOE_ERR_UNSUPPORTED;  // grid rows of the router contractions
+    // rows of the grouped weight-gradient GEMMs (E_r groups of d or d_f rows)
+    if ((int64_t)p->E_r * std::max(p->d, p->d_f) >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
+}
+
+// offsets_host: a non-decreasing prefix from 0 to at most N k
+bool offsets_valid(const moe_params& p, const int32_t* o) {
+    if (o[0] != 0) return false;
+    for (int64_t e = 0; e < p.E_r; ++e)
+        if (o[e + 1] < o[e]) return false;
+    return (int64_t)o[p.E_r] <= p.N * p.k;
 }
 
 unsigned grid_for(int64_t items_per_block_units, int64_t n) {
@@ -619,18 +659,19 @@ using namespace moe;
 
 extern "C" {
 
-moe_status moe_backward_workspace_size(const moe_params* p, size_t* bytes) {
+moe_status moe_backward_workspace_size(const moe_params* p, const int32_t* offsets_host, size_t* bytes) {
     const moe_status s = bwd_check(p);
     if (s != MOE_OK) return s;
     if (!bytes) return MOE_ERR_INVALID_ARG;
-    *bytes = bwd_layout(*p).total;
+    if (offsets_host && p->N > 0 && !offsets_valid(*p, offsets_host)) return MOE_ERR_INVALID_ARG;
+    *bytes = bwd_layout(*p, kmax_of(*p, p->N > 0 ? offsets_host : nullptr)).total;
     return MOE_OK;
 }
 
 moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offsets_host, const void* x,
                         const void* W_r, const float* b_r, const void* W_g, const void* W_u, const void* W_d,
                         const void* Ws_g, const void* Ws_u, const void* Ws_d, const float* dY, const void* ws,
-                        const moe_grads* gr, void* bws, moe_stream_t stream) {
+                        const moe_grads* gr, void* bws, size_t bws_bytes, moe_stream_t stream) {
     moe_status s = bwd_check(p);
     if (s != MOE_OK) return s;
     if (!ws || !al16(ws) || !bws || !al16(bws)) return MOE_ERR_WORKSPACE;
@@ -656,12 +697,6 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
         if (e == cudaSuccess && sh) e = cudaMemsetAsync(gr->dWs_d, 0, sizeof(float) * dfs * d, st);
         return e == cudaSuccess ? MOE_OK : bwd_fail(e, "memset");
     }
-    // (an empty forward writes no offsets, so they are checked only now)
-    if (offsets_host[0] != 0) return MOE_ERR_INVALID_ARG;
-    for (int64_t e = 0; e < E; ++e)
-        if (offsets_host[e + 1] < offsets_host[e]) return MOE_ERR_INVALID_ARG;
-    if (offsets_host[E] > rows) return MOE_ERR_INVALID_ARG;
-    (void)cudaGetLastError();  // clear a stale non-sticky error left by earlier unrelated calls
     if (!x || !W_r || !W_g || !W_u || !W_d || !dY) return MOE_ERR_INVALID_ARG;
     if (!al16(x) || !al16(W_r) || !al16(W_g) || !al16(W_u) || !al16(W_d) || !al16(dY) || !al16(gr->dx) ||
         !al16(gr->dW_g) || !al16(gr->dW_u) || !al16(gr->dW_d))
@@ -669,17 +704,20 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     if (sh && (!Ws_g || !Ws_u || !Ws_d || !al16(Ws_g) || !al16(Ws_u) || !al16(Ws_d) || !al16(gr->dWs_g) ||
                !al16(gr->dWs_u) || !al16(gr->dWs_d)))
         return MOE_ERR_INVALID_ARG;
+    // (an empty forward writes no offsets, so they are checked only now)
+    if (!offsets_valid(*p, offsets_host)) return MOE_ERR_INVALID_ARG;
+    const BwdLayout L = bwd_layout(*p, kmax_of(*p, offsets_host));
+    if (bws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    (void)cudaGetLastError();  // clear a stale non-sticky error left by earlier unrelated calls
 
     WsView v;
     make_view(*p, const_cast<void*>(ws), v);
-    const BwdLayout L = bwd_layout(*p);
     char* b = static_cast<char*>(bws);
     auto I32 = [&](size_t o) { return reinterpret_cast<int32_t*>(b + o); };
     auto F32 = [&](size_t o) { return reinterpret_cast<float*>(b + o); };
     auto B16 = [&](size_t o) { return reinterpret_cast<bf16*>(b + o); };
-    int32_t* padoff = I32(L.padoff);
-    int32_t* tstart = I32(L.tstart);
-    int32_t* mt_start = I32(L.mt_start);
+    int32_t *tstart = I32(L.tstart), *nkb = I32(L.nkb), *mt_start = I32(L.mt_start);
+    int32_t *offs_d = I32(L.offs_d), *offs_f = I32(L.offs_f), *mt_d = I32(L.mt_d), *mt_f = I32(L.mt_f);
     auto* counters = reinterpret_cast<unsigned long long*>(b + L.counters);
     float* logits = F32(L.logits);
     float* dG = F32(L.dG);
@@ -690,21 +728,21 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     const bf16* xp = static_cast<const bf16*>(v.x_perm);
     const bf16* hp = static_cast<const bf16*>(v.h);
     const int32_t* n_rows = v.offsets + E;  // accepted rows, on the device
+    const int64_t Kmax = L.Kmax;
     int status = MOE_OK;
+    // transposition tiles of the routed rows (host count, same rule as bwd_tables_kernel)
+    int64_t n_tiles = 0;
+    for (int64_t g = 0; g < E; ++g) {
+        const int64_t R = offsets_host[g + 1] - offsets_host[g];
+        n_tiles += R > 0 ? (R + kTT - 1) / kTT : 1;
+    }
 
     e = cudaMemsetAsync(counters, 0, CNT_COUNT * 8, st);
     if (e != cudaSuccess) return bwd_fail(e, "memset");
-    // host copy of the per-expert padded column offsets (same rule as bwd_tables_kernel)
-    std::vector<int64_t> hpad(E + 1);
-    int64_t n_tiles = 0;
-    hpad[0] = 0;
-    for (int64_t g = 0; g < E; ++g) {
-        const int64_t R = offsets_host[g + 1] - offsets_host[g];
-        hpad[g + 1] = hpad[g] + ((R + 7) & ~(int64_t)7);
-        n_tiles += (R + kTT - 1) / kTT;
-    }
-
-    bwd_tables_kernel<<<1, 32, 0, st>>>((int)E, v.offsets, padoff, tstart);
+    bwd_tables_kernel<<<1, 32, 0, st>>>((int)E, v.offsets, tstart, nkb);
+    bwd_strided_offsets_kernel<<<1, 256, 0, st>>>((int)E, (int32_t)d, offs_d);
+    bwd_strided_offsets_kernel<<<1, 256, 0, st>>>((int)E, (int32_t)df, offs_f);
+    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "tables");
     e = launch_mtile_prefix((int)E, tc_tile_rows(*p), v.offsets, mt_start, st);
     if (e != cudaSuccess) return bwd_fail(e, "tables");
     // router scores (bias added in the router kernel): tensor cores when the
@@ -790,13 +828,13 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     // shared expert: weight 1 on every token
     float* dxs = nullptr;
     if (sh) {
-        const int64_t Np = (N + 7) & ~(int64_t)7;
+        const int64_t Ks = L.Kmax_sh;
         bf16 *dYs = B16(L.dYs), *dzus = B16(L.dzus), *WsT_d = B16(L.WsT_d), *WsT_gu = B16(L.WsT_gu);
         float *Zs = F32(L.Zs), *Us = F32(L.Us), *Gs = F32(L.Gs);
         dxs = F32(L.dxs);
-        int32_t *sh_off = I32(L.sh_off), *sh_pad = I32(L.sh_padoff), *sh_ts = I32(L.sh_tstart);
+        int32_t *sh_off = I32(L.sh_off), *sh_ts = I32(L.sh_tstart), *sh_nkb = I32(L.sh_nkb);
         bwd_single_group_kernel<<<1, 32, 0, st>>>((int32_t)N, sh_off);
-        bwd_tables_kernel<<<1, 32, 0, st>>>(1, sh_off, sh_pad, sh_ts);
+        bwd_tables_kernel<<<1, 32, 0, st>>>(1, sh_off, sh_ts, sh_nkb);
         bwd_gather_dy_kernel<<<grid_for(8, N), 256, 0, st>>>(dY, d, nullptr, nullptr, N, N, N, dYs);
         bwd_batched_transpose_kernel<<<dim3((unsigned)((d + kTT - 1) / kTT), (unsigned)((dfs + kTT - 1) / kTT), 1), 256,
                                        0, st>>>(static_cast<const bf16*>(Ws_d), d, dfs, WsT_d, d, 0);
@@ -814,23 +852,23 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
         if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "shared SwiGLU backward");
         e = launch_tc_dense(N, d, 2 * dfs, dzus, WsT_gu, dxs, counters, st, &status);
         if (e != cudaSuccess) return bwd_fail(e, "shared dx (tcgen05)");
-        // weight gradients over all tokens (K = N, padded to a multiple of 8)
+        // weight gradients over all tokens (K = N, zero-padded to whole 64-wide blocks)
         bf16 *dYsT = B16(L.dYsT), *xsT = B16(L.xsT), *hsT = B16(L.hsT), *dzsT = B16(L.dzsT), *dusT = B16(L.dusT);
-        const unsigned tiles_sh = (unsigned)((N + kTT - 1) / kTT);
+        const unsigned tiles_sh = (unsigned)(Ks / kTT);
         bwd_group_transpose_kernel<false><<<dim3(tiles_sh, (unsigned)((d + kTT - 1) / kTT)), 256, 0, st>>>(
-            dYs, d, d, sh_off, sh_pad, sh_ts, 1, nullptr, dYsT);
+            dYs, d, d, sh_off, sh_ts, 1, nullptr, dYsT, Ks, 0);
         bwd_group_transpose_kernel<false><<<dim3(tiles_sh, (unsigned)((d + kTT - 1) / kTT)), 256, 0, st>>>(
-            xb, d, d, sh_off, sh_pad, sh_ts, 1, nullptr, xsT);
+            xb, d, d, sh_off, sh_ts, 1, nullptr, xsT, Ks, 0);
         bwd_group_transpose_kernel<false><<<dim3(tiles_sh, (unsigned)((dfs + kTT - 1) / kTT)), 256, 0, st>>>(
-            static_cast<const bf16*>(v.h_shared), dfs, dfs, sh_off, sh_pad, sh_ts, 1, nullptr, hsT);
+            static_cast<const bf16*>(v.h_shared), dfs, dfs, sh_off, sh_ts, 1, nullptr, hsT, Ks, 0);
         bwd_group_transpose_kernel<false><<<dim3(tiles_sh, (unsigned)((dfs + kTT - 1) / kTT)), 256, 0, st>>>(
-            dzus, 2 * dfs, dfs, sh_off, sh_pad, sh_ts, 1, nullptr, dzsT);
+            dzus, 2 * dfs, dfs, sh_off, sh_ts, 1, nullptr, dzsT, Ks, 0);
         bwd_group_transpose_kernel<false><<<dim3(tiles_sh, (unsigned)((dfs + kTT - 1) / kTT)), 256, 0, st>>>(
-            dzus + dfs, 2 * dfs, dfs, sh_off, sh_pad, sh_ts, 1, nullptr, dusT);
+            dzus + dfs, 2 * dfs, dfs, sh_off, sh_ts, 1, nullptr, dusT, Ks, 0);
         if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "shared row transposes");
-        e = launch_tc_dense(d, dfs, Np, dYsT, hsT, gr->dWs_d, counters, st, &status);
-        if (e == cudaSuccess) e = launch_tc_dense(dfs, d, Np, dzsT, xsT, gr->dWs_g, counters, st, &status);
-        if (e == cudaSuccess) e = launch_tc_dense(dfs, d, Np, dusT, xsT, gr->dWs_u, counters, st, &status);
+        e = launch_tc_dense(d, dfs, Ks, dYsT, hsT, gr->dWs_d, counters, st, &status);
+        if (e == cudaSuccess) e = launch_tc_dense(dfs, d, Ks, dzsT, xsT, gr->dWs_g, counters, st, &status);
+        if (e == cudaSuccess) e = launch_tc_dense(dfs, d, Ks, dusT, xsT, gr->dWs_u, counters, st, &status);
         if (e != cudaSuccess) return bwd_fail(e, "shared weight gradients (tcgen05)");
     }
 
@@ -839,41 +877,47 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
                                                   rows);
     if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "dx");
 
-    // weight gradients: per-expert column blocks of the transposed operands
-    if (n_tiles > 0) {
+    // weight gradients: operands transposed into [E][C][Kmax] blocks (expert
+    // e's rows as columns, zeros up to its last K block), then one grouped
+    // GEMM per gradient whose group e is the expert's C rows
+    {
         const dim3 gd((unsigned)n_tiles, (unsigned)((d + kTT - 1) / kTT));
         const dim3 gf((unsigned)n_tiles, (unsigned)((df + kTT - 1) / kTT));
-        bwd_group_transpose_kernel<true><<<gd, 256, 0, st>>>(dYp, d, d, v.offsets, padoff, tstart, (int)E, v.slot_w,
-                                                             doT);
-        bwd_group_transpose_kernel<false><<<gd, 256, 0, st>>>(xp, d, d, v.offsets, padoff, tstart, (int)E, nullptr,
-                                                              xT);
-        bwd_group_transpose_kernel<false><<<gf, 256, 0, st>>>(hp, df, df, v.offsets, padoff, tstart, (int)E, nullptr,
-                                                              hT);
-        bwd_group_transpose_kernel<false><<<gf, 256, 0, st>>>(dzu, 2 * df, df, v.offsets, padoff, tstart, (int)E,
-                                                              nullptr, dzT);
-        bwd_group_transpose_kernel<false><<<gf, 256, 0, st>>>(dzu + df, 2 * df, df, v.offsets, padoff, tstart, (int)E,
-                                                              nullptr, duT);
+        bwd_group_transpose_kernel<true><<<gd, 256, 0, st>>>(dYp, d, d, v.offsets, tstart, (int)E, v.slot_w, doT, Kmax,
+                                                             d * Kmax);
+        bwd_group_transpose_kernel<false><<<gd, 256, 0, st>>>(xp, d, d, v.offsets, tstart, (int)E, nullptr, xT, Kmax,
+                                                              d * Kmax);
+        bwd_group_transpose_kernel<false><<<gf, 256, 0, st>>>(hp, df, df, v.offsets, tstart, (int)E, nullptr, hT, Kmax,
+                                                              df * Kmax);
+        bwd_group_transpose_kernel<false><<<gf, 256, 0, st>>>(dzu, 2 * df, df, v.offsets, tstart, (int)E, nullptr, dzT,
+                                                              Kmax, df * Kmax);
+        bwd_group_transpose_kernel<false><<<gf, 256, 0, st>>>(dzu + df, 2 * df, df, v.offsets, tstart, (int)E, nullptr,
+                                                              duT, Kmax, df * Kmax);
         if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "row transposes");
     }
-    for (int64_t g = 0; g < E; ++g) {
-        const int64_t Kp = hpad[g + 1] - hpad[g];
-        float* gWd = gr->dW_d + g * d * df;
-        float* gWg = gr->dW_g + g * df * d;
-        float* gWu = gr->dW_u + g * df * d;
-        if (Kp == 0) {
-            e = cudaMemsetAsync(gWd, 0, sizeof(float) * d * df, st);
-            if (e == cudaSuccess) e = cudaMemsetAsync(gWg, 0, sizeof(float) * d * df, st);
-            if (e == cudaSuccess) e = cudaMemsetAsync(gWu, 0, sizeof(float) * d * df, st);
-            if (e != cudaSuccess) return bwd_fail(e, "memset");
-            continue;
-        }
-        e = launch_tc_dense(d, df, Kp, doT + d * hpad[g], hT + df * hpad[g], gWd, counters, st, &status);
-        if (e == cudaSuccess)
-            e = launch_tc_dense(df, d, Kp, dzT + df * hpad[g], xT + d * hpad[g], gWg, counters, st, &status);
-        if (e == cudaSuccess)
-            e = launch_tc_dense(df, d, Kp, duT + df * hpad[g], xT + d * hpad[g], gWu, counters, st, &status);
-        if (e != cudaSuccess) return bwd_fail(e, "weight gradients (tcgen05)");
-    }
+    moe_params qw = *p;  // groups of d rows (dW_d) or d_f rows (dW_g, dW_u), K = Kmax
+    qw.d_f_shared = 0;
+    qw.k = 1;
+    qw.d_f = (int32_t)Kmax;
+    qw.N = E * d;
+    qw.d = (int32_t)df;
+    e = launch_mtile_prefix((int)E, tc_tile_rows(qw), offs_d, mt_d, st);
+    if (e != cudaSuccess) return bwd_fail(e, "tables");
+    W0.W_d = hT;
+    e = launch_tc_down(qw, DOWN_STORE, qw.N, doT, nullptr, offs_d, mt_d, W0, nullptr, nullptr, nullptr, gr->dW_d,
+                       counters, st, &status, nkb);
+    if (e != cudaSuccess) return bwd_fail(e, "dW_d (tcgen05)");
+    qw.N = E * df;
+    qw.d = (int32_t)d;
+    e = launch_mtile_prefix((int)E, tc_tile_rows(qw), offs_f, mt_f, st);
+    if (e != cudaSuccess) return bwd_fail(e, "tables");
+    W0.W_d = xT;
+    e = launch_tc_down(qw, DOWN_STORE, qw.N, dzT, nullptr, offs_f, mt_f, W0, nullptr, nullptr, nullptr, gr->dW_g,
+                       counters, st, &status, nkb);
+    if (e == cudaSuccess)
+        e = launch_tc_down(qw, DOWN_STORE, qw.N, duT, nullptr, offs_f, mt_f, W0, nullptr, nullptr, nullptr, gr->dW_u,
+                           counters, st, &status, nkb);
+    if (e != cudaSuccess) return bwd_fail(e, "dW_g, dW_u (tcgen05)");
     return MOE_OK;
 }
 
@@ -883,7 +927,8 @@ moe_status moe_backward_check(const moe_params* p, const void* bws, moe_stream_t
     if (!bws || !al16(bws)) return MOE_ERR_WORKSPACE;
     unsigned long long cnt[CNT_COUNT];
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(cnt, static_cast<const char*>(bws) + bwd_layout(*p).counters, sizeof(cnt),
+    // the counters sit at the same offset whatever Kmax is
+    cudaError_t e = cudaMemcpyAsync(cnt, static_cast<const char*>(bws) + bwd_layout(*p, kTT).counters, sizeof(cnt),
                                     cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return bwd_fail(e, "check");

@@ -92,6 +92,7 @@ struct TcArgs {
     float* zero_ptr;          // optional fp32 buffer the epilogue warps zero first
     int64_t zero_n4;          // its size in float4
     int ks;                   // K splits per output tile (partial sums reduced with red.add)
+    const int32_t* grp_nkb;   // [E] K blocks of each routed group (null: nkb_r for all; ks must be 1)
     unsigned long long* counters;
 };
 
@@ -398,6 +399,10 @@ __device__ __forceinline__ bool decode_tile(int t_in, const SchedSmem& s, const 
         ti.g = g;
         ti.kb0 = (int)((int64_t)kq * a.nkb_r / a.ks);
         ti.kb1 = (int)((int64_t)(kq + 1) * a.nkb_r / a.ks);
+        if (a.grp_nkb) {  // a group's own K extent (at least one block: its tiles are always written)
+            const int nk = min(max(a.grp_nkb[g], 1), a.nkb_r);
+            if (ti.kb1 > nk) ti.kb1 = nk;
+        }
         if (mtiles <= 0) {  // inconsistent prefix (caller-supplied offsets): no rows
             ti.n_tile = 0;
             ti.a_row = 0;
@@ -1009,8 +1014,10 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
                            const void* h_shared, const int32_t* offsets, const int32_t* mt_start,
                            const ExpertWeights& W, const int32_t* slot_token,
                            const float* slot_w, float* Y, float* H_out,
-                           unsigned long long* counters, cudaStream_t st, int* status) {
+                           unsigned long long* counters, cudaStream_t st, int* status,
+                           const int32_t* grp_nkb) {
     *status = MOE_OK;
+    if (grp_nkb && mode != DOWN_STORE) return cudaErrorInvalidValue;
     CUtensorMap mA, mB0, mA_sh, mB0_sh, mA_h, mA_sh_h;
     const uint64_t rows = (uint64_t)(p.N * p.k);
     bool ok = make_map(&mA, h, rows, p.d_f) && make_map(&mA_h, h, rows, p.d_f, 64) &&
@@ -1051,6 +1058,7 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
     a.n_tokens = (int)p.N;
     a.has_routed = 1;
     a.ks = 1;
+    a.grp_nkb = grp_nkb;
     const bool pair = tc_tile_rows(p) == 256;
     const int tm = pair ? 256 : 128;
     if (mode == DOWN_COMBINE) {

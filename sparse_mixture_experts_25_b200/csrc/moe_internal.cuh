@@ -129,11 +129,14 @@ cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const voi
                               const int32_t* offsets, const int32_t* mt_start,
                               const ExpertWeights& W, void* h, void* h_shared, float* Y_zero,
                               unsigned long long* counters, cudaStream_t st, int* status);
+// grp_nkb (DOWN_STORE only, nullable): [E] K blocks of 64 that each group
+// contracts over (at least 1); the rest of K is skipped for that group
 cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void* h,
                            const void* h_shared, const int32_t* offsets, const int32_t* mt_start,
                            const ExpertWeights& W, const int32_t* slot_token,
                            const float* slot_w, float* Y, float* H_out,
-                           unsigned long long* counters, cudaStream_t st, int* status);
+                           unsigned long long* counters, cudaStream_t st, int* status,
+                           const int32_t* grp_nkb = nullptr);
 // rows of one output tile of the tcgen05 grouped GEMMs for these params
 // (256 when CTA pairs are used, else 128): the dispatch's M-tile prefix unit
 int tc_tile_rows(const moe_params& p);

@@ -168,26 +168,37 @@ def test_backward_checks_arguments_on_the_host():
     L = moe.lib()
     assert ctypes.sizeof(moe.Grads) == 9 * 8
     p = moe.params(16, 64, 64, 8, 2, c=1.0)
+    sz = ctypes.c_size_t()
     # fp32 layers have no backward; E_r above the router kernel's limit neither
-    assert L.moe_backward_workspace_size(ctypes.byref(moe.params(16, 64, 64, 8, 2, dtype=moe.MOE_F32)),
-                                         ctypes.byref(ctypes.c_size_t())) == moe.MOE_ERR_UNSUPPORTED
-    assert L.moe_backward_workspace_size(ctypes.byref(moe.params(16, 64, 64, 300, 2)),
-                                         ctypes.byref(ctypes.c_size_t())) == moe.MOE_ERR_UNSUPPORTED
-    n = moe.moe_backward_workspace_size(p)
+    assert L.moe_backward_workspace_size(ctypes.byref(moe.params(16, 64, 64, 8, 2, dtype=moe.MOE_F32)), None,
+                                         ctypes.byref(sz)) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_backward_workspace_size(ctypes.byref(moe.params(16, 64, 64, 300, 2)), None,
+                                         ctypes.byref(sz)) == moe.MOE_ERR_UNSUPPORTED
+    good = [0, 4, 4, 8, 12, 16, 20, 24, 28]
+    n_any = moe.moe_backward_workspace_size(p)
+    n = moe.moe_backward_workspace_size(p, good)
     assert n >= 8 * 64 * 64 * 2 * 3            # the transposed expert weights alone
-    # the worst case grows with the routed rows N k
-    assert moe.moe_backward_workspace_size(moe.params(32, 64, 64, 8, 2, c=1.0)) > n
+    # C = 4 rows per expert at most: one 64-wide K block either way
+    assert n == n_any
+    # the bound grows with the capacity; a routing with a long expert needs more
+    big = moe.params(256, 64, 64, 8, 2)
+    skew = [0, 200, 200, 200, 200, 200, 200, 200, 200]
+    even = [0, 25, 50, 75, 100, 125, 150, 175, 200]
+    assert moe.moe_backward_workspace_size(big, skew) > moe.moe_backward_workspace_size(big, even)
+    assert moe.moe_backward_workspace_size(big) >= moe.moe_backward_workspace_size(big, skew)
+    arr_bad = (ctypes.c_int32 * 9)(*([0, 5, 3] + good[3:]))
+    assert L.moe_backward_workspace_size(ctypes.byref(p), arr_bad, ctypes.byref(sz)) == moe.MOE_ERR_INVALID_ARG
     fake = 4096                                  # aligned, never dereferenced: the checks come first
     g = moe.Grads(*([fake] * 9))
 
-    def call(offsets, ws=fake, bws=fake, grads=g, aux=0.0):
+    def call(offsets, ws=fake, bws=fake, grads=g, aux=0.0, nbytes=n):
         arr = (ctypes.c_int32 * len(offsets))(*offsets)
         return L.moe_backward(ctypes.byref(p), aux, arr, fake, fake, None, fake, fake, fake, None, None, None,
-                              fake, ws, ctypes.byref(grads) if grads is not None else None, bws, None)
+                              fake, ws, ctypes.byref(grads) if grads is not None else None, bws, nbytes, None)
 
-    good = [0, 4, 4, 8, 12, 16, 20, 24, 28]
     assert call(good, ws=None) == moe.MOE_ERR_WORKSPACE
     assert call(good, bws=fake + 8) == moe.MOE_ERR_WORKSPACE
+    assert call(good, nbytes=n - 1) == moe.MOE_ERR_WORKSPACE
     assert call(good, grads=None) == moe.MOE_ERR_INVALID_ARG
     assert call(good, aux=float("nan")) == moe.MOE_ERR_INVALID_ARG
     assert call([1] + good[1:]) == moe.MOE_ERR_INVALID_ARG             # does not start at 0
@@ -199,7 +210,7 @@ def test_backward_checks_arguments_on_the_host():
     arr = (ctypes.c_int32 * 9)(*good)
     no_shared = moe.Grads(*([fake] * 6 + [None] * 3))
     assert L.moe_backward(ctypes.byref(ps), 0.0, arr, fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
-                          fake, ctypes.byref(no_shared), fake, None) == moe.MOE_ERR_INVALID_ARG
+                          fake, ctypes.byref(no_shared), fake, 1 << 40, None) == moe.MOE_ERR_INVALID_ARG
 
 
 def test_backward_of_an_empty_batch_needs_no_dx():
@@ -215,5 +226,5 @@ def test_backward_of_an_empty_batch_needs_no_dx():
     g = moe.Grads(None, *([fake] * 8))
     arr = (ctypes.c_int32 * 9)(*([0] * 9))
     r = L.moe_backward(ctypes.byref(p), 0.0, arr, None, None, None, None, None, None, None, None, None, None,
-                       fake, ctypes.byref(g), fake, None)
+                       fake, ctypes.byref(g), fake, 0, None)
     assert r not in (moe.MOE_ERR_INVALID_ARG, moe.MOE_ERR_WORKSPACE)

@@ -66,7 +66,8 @@ def _grads(w, device="cuda"):
 def _backward(w, inp, full, dY, aux):
     p, dev, ws = full["p"], full["dev"], full["ws"]
     g = _grads(w)
-    bws = torch.empty(moe.moe_backward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    bws = torch.empty(moe.moe_backward_workspace_size(p, full["rec"]["offsets"] if w.N else None),
+                      dtype=torch.uint8, device="cuda")
     moe.moe_backward(p, full["rec"]["offsets"], dev["x"], dev["W_r"], dev.get("b_r"), dev["W_g"], dev["W_u"],
                      dev["W_d"], dev.get("Ws_g"), dev.get("Ws_u"), dev.get("Ws_d"),
                      torch.from_numpy(dY).cuda(), ws, g, bws, aux_coef=aux)
