@@ -588,6 +588,122 @@ def run_gpu(args):
     return 0
 
 
+def backward_kernels(w: si.Workload) -> int:
+    """Kernels one moe_backward launches: tables (4), scores (1), weight
+    transposes (3), dY gather (1), z / u / W_d^T dY / dx-row GEMMs (4),
+    SwiGLU backward (1), router (1), router contractions (2, plus the slice
+    sum when dW_r = dG^T X is split over the tokens), db (2), dx (1), row
+    transposes (5), weight-gradient prefixes (2) and GEMMs (3); the shared
+    expert adds 19."""
+    tiles = ((w.E + 63) // 64) * ((w.d + 63) // 64)
+    sms = 148
+    slices = max(1, min(-(-2 * sms // tiles), max(1, w.N // 256), 16))
+    return 30 + (1 if slices > 1 else 0) + (19 if w.d_f_shared else 0)
+
+
+def run_gpu_backward(args):
+    """--backward: one GPU; the forward runs once (routing records, x_perm,
+    h), then moe_backward is timed: gradients of sum(dY * Y) + 0.01 aux with
+    respect to x, W_r, b_r, the experts and the shared expert."""
+    import torch
+    import sparse_mixture_experts_25_b200 as moe
+    if dist_env()[0] > 1:
+        raise SystemExit("--backward runs on one GPU")
+    w = si.WORKLOADS[args.workload]
+    if w.dtype != si.DT_BF16:
+        raise SystemExit("the backward pass is built for bf16 layers")
+    inp = si.inputs(w)
+    dY_host = si.upstream_gradient(w)
+    torch.cuda.set_device(0)
+
+    def dev(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+    d = {k: dev(v) for k, v in inp.items()}
+    p = moe.params(w.N, w.d, w.d_f, w.E, w.k, c=w.c, norm=w.norm, theta=w.theta, dtype=w.dtype,
+                   d_f_shared=w.d_f_shared, reject_policy=w.reject_policy, accept_order=w.accept_order)
+    wsb = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+    Y = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
+    moe.moe_forward(p, d["x"], d["W_r"], d["b_r"], d["lat"], d["W_g"], d["W_u"], d["W_d"], d["Ws_g"], d["Ws_u"],
+                    d["Ws_d"], Y, wsb)
+    status, stats = moe.moe_get_stats(p, wsb)
+    if status != moe.MOE_OK:
+        raise RuntimeError(f"moe_forward status: {moe.moe_status_string(status)}")
+    offsets = moe.workspace_views(p, wsb)["offsets"].cpu().numpy()
+    dY = torch.from_numpy(dY_host).cuda()
+    shapes = {"dx": (w.N, w.d), "dW_r": (w.E, w.d), "db_r": (w.E,), "dW_g": (w.E, w.d_f, w.d),
+              "dW_u": (w.E, w.d_f, w.d), "dW_d": (w.E, w.d, w.d_f)}
+    if w.d_f_shared:
+        shapes.update({"dWs_g": (w.d_f_shared, w.d), "dWs_u": (w.d_f_shared, w.d), "dWs_d": (w.d, w.d_f_shared)})
+    g = {n: torch.empty(sh, dtype=torch.float32, device="cuda") for n, sh in shapes.items()}
+    bws = torch.empty(moe.moe_backward_workspace_size(p, offsets), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moe.moe_backward(p, offsets, d["x"], d["W_r"], d["b_r"], d["W_g"], d["W_u"], d["W_d"], d["Ws_g"],
+                         d["Ws_u"], d["Ws_d"], dY, wsb, g, bws, aux_coef=0.01, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if moe.moe_backward_check(p, bws) != moe.MOE_OK:
+        raise RuntimeError("moe_backward: a bounded device wait timed out")
+    flush = torch.empty(256 * 2**20 // 4, dtype=torch.int32, device="cuda")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(0) as clk:
+        time.sleep(0.3)
+        for i in range(args.steps):
+            flush.fill_(i)   # evict the layer's data from L2; outside the step's events
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        time.sleep(0.2)
+    ms_step = float(sum(a.elapsed_time(b) for a, b in ev)) / args.steps
+    R = int(stats["accepted"])
+    touched = int((moe.workspace_views(p, wsb)["acc"] > 0).sum().item())
+    ds = w.d_f_shared
+    # 8 contractions of the expert size per routed row: z, u (recomputed), W_d^T dY,
+    # dx rows (two), dW_d, dW_g, dW_u; the same over every token for the shared
+    # expert; the router's three E_r-wide contractions
+    flops = 16.0 * R * w.d * w.d_f + 16.0 * w.N * w.d * ds + 6.0 * w.N * w.E * w.d
+    # least HBM traffic: bf16 weights read, fp32 weight gradients written, x and
+    # dY read, dx written
+    nbytes = (3.0 * touched * w.d * w.d_f * (2 + 4) + 3.0 * w.d * ds * (2 + 4)
+              + w.N * w.d * (2 + 4 + 4) + w.E * w.d * (2 + 4))
+    peaks, peak_src = load_peaks()
+    timed_s = ms_step * args.steps / 1000.0
+    peak_tf = peaks["bf16_tflops"] if timed_s < 1.0 else peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    t_tensor = flops / (peak_tf * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    tflops = flops / (ms_step * 1e-3) / 1e12
+    gbs = nbytes / (ms_step * 1e-3) / 1e9
+    if t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s", "frac": tflops / peak_tf}
+    else:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"]}
+    roof.update({"kernel": "moe_backward, all launches of one call", "traffic": None,
+                 "flops_per_launch": flops, "bytes_per_launch": nbytes, "avg_launch_ms": ms_step,
+                 "peak_source": f"{peak_src} bf16 {'burst' if timed_s < 1.0 else 'sustained'} / HBM copy"})
+    line = {
+        "metric": "MoE-layer backward tokens/s (gradients of x, W_r, b_r, experts, shared expert)",
+        "value": w.N / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; dY ~ N(0,1)); no dataset or checkpoint",
+        "config": dict(config_of(w, args), l2="flushed between steps (256 MiB write)"),
+        "roofline": roof, "gpu_launches": backward_kernels(w) * args.steps, "clocks": clk.summary(),
+        "routing": {k: stats[k] for k in ("accepted", "rejected", "L_max")},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -599,6 +715,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of one step captured into a CUDA graph (one GPU)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (one GPU, bf16 layers) instead of the forward")
     ap.add_argument("--override", action="append", default=[],
                     help="key=value change of the workload shape (profiling of smaller cases)")
     args = ap.parse_args(argv)
@@ -615,6 +733,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.backward:
+        return run_gpu_backward(args)
     if si.WORKLOADS[args.workload].soft_p > 0:
         return run_gpu_soft(args)
     return run_gpu(args)

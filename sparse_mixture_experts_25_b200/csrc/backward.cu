@@ -61,6 +61,11 @@ __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+unsigned grid_blocks(int64_t n) {  // 256-thread blocks for a grid-stride loop over n items
+    const int64_t b = std::min<int64_t>((n + 255) / 256, (int64_t)num_sms() * 8);
+    return (unsigned)std::max<int64_t>(b, 1);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -409,21 +414,34 @@ __global__ void __launch_bounds__(256) bwd_router_kernel(RouterBwd a) {
     }
 }
 
-// db[e] = sum_t dG[t, e]: one block per 32 columns, 8 warps over the rows
+// db[e] = sum_t dG[t, e] in two deterministic phases: block (x, y) sums the
+// rows of chunk y for 32 columns (8 warps over the rows, then shared memory)
+// into part[y][e]; bwd_reduce_kernel then adds the chunks in order.
 __global__ void __launch_bounds__(256) bwd_colsum_kernel(const float* __restrict__ dG, int64_t N, int E,
-                                                         float* __restrict__ db) {
-    __shared__ float part[8][32];
+                                                         int64_t chunk, float* __restrict__ part) {
+    __shared__ float sm[8][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int e = blockIdx.x * 32 + lane;
+    const int64_t t0 = (int64_t)blockIdx.y * chunk;
+    const int64_t t1 = min64(N, t0 + chunk);
     float s = 0.f;
     if (e < E)
-        for (int64_t t = warp; t < N; t += 8) s += dG[t * E + e];
-    part[warp][lane] = s;
+        for (int64_t t = t0 + warp; t < t1; t += 8) s += dG[t * E + e];
+    sm[warp][lane] = s;
     __syncthreads();
     if (warp == 0 && e < E) {
         float v = 0.f;
-        for (int i = 0; i < 8; ++i) v += part[i][lane];
-        db[e] = v;
+        for (int i = 0; i < 8; ++i) v += sm[i][lane];
+        part[(int64_t)blockIdx.y * E + e] = v;
+    }
+}
+
+// out[i] = sum_{z < S} part[z n + i], z in order
+__global__ void bwd_reduce_kernel(const float* __restrict__ part, int S, int64_t n, float* __restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        float v = 0.f;
+        for (int z = 0; z < S; ++z) v += part[(int64_t)z * n + i];
+        out[i] = v;
     }
 }
 
@@ -465,16 +483,22 @@ __global__ void __launch_bounds__(256)
 __device__ __forceinline__ float as_f32(float v) { return v; }
 __device__ __forceinline__ float as_f32(bf16 v) { return __bfloat162float(v); }
 
+// blockIdx.z = K slice: slice z sums k in [z kchunk, (z+1) kchunk) into
+// C + z cz (kchunk a multiple of 16; one slice: kchunk >= K, cz unused).
 template <typename TA, typename TB>
 __global__ void __launch_bounds__(256)
     bwd_simt_gemm_kernel(int64_t M, int64_t N, int64_t K, const TA* __restrict__ A, int64_t sam, int64_t sak,
-                         const TB* __restrict__ B, int64_t sbn, int64_t sbk, float* __restrict__ C, int64_t ldc) {
+                         const TB* __restrict__ B, int64_t sbn, int64_t sbk, float* __restrict__ C, int64_t ldc,
+                         int64_t kchunk, int64_t cz) {
     __shared__ float As[16][64 + 4];
     __shared__ float Bs[16][64 + 4];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int64_t m0 = (int64_t)blockIdx.y * 64, n0 = (int64_t)blockIdx.x * 64;
+    const int64_t kbeg = (int64_t)blockIdx.z * kchunk;
+    K = min64(K, kbeg + kchunk);
+    C += (int64_t)blockIdx.z * cz;
     float acc[4][4] = {};
-    for (int64_t k0 = 0; k0 < K; k0 += 16) {
+    for (int64_t k0 = kbeg; k0 < K; k0 += 16) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int idx = tid + i * 256;
@@ -521,8 +545,36 @@ template <typename TA, typename TB>
 cudaError_t simt_gemm(int64_t M, int64_t N, int64_t K, const TA* A, int64_t sam, int64_t sak, const TB* B,
                       int64_t sbn, int64_t sbk, float* C, int64_t ldc, cudaStream_t st) {
     if (M <= 0 || N <= 0) return cudaSuccess;
-    const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + 63) / 64));
-    bwd_simt_gemm_kernel<TA, TB><<<grid, 256, 0, st>>>(M, N, K, A, sam, sak, B, sbn, sbk, C, ldc);
+    const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + 63) / 64), 1);
+    bwd_simt_gemm_kernel<TA, TB><<<grid, 256, 0, st>>>(M, N, K, A, sam, sak, B, sbn, sbk, C, ldc, K + 16, 0);
+    return cudaGetLastError();
+}
+
+// K slices of a long contraction with few output tiles: enough slices for
+// about two waves, at least 256 K per slice, at most kMaxSlices
+constexpr int kMaxSlices = 16;
+
+int k_slices(int64_t M, int64_t N, int64_t K) {
+    const int64_t tiles = ((M + 63) / 64) * ((N + 63) / 64);
+    int64_t s = (2 * (int64_t)num_sms() + tiles - 1) / tiles;
+    s = std::min<int64_t>(s, std::max<int64_t>(1, K / 256));
+    return (int)std::max<int64_t>(1, std::min<int64_t>(s, kMaxSlices));
+}
+
+// C [M, N] (row-major, ldc = N) = the K-sliced contraction: slices into
+// part [S, M, N], then added in slice order (deterministic)
+template <typename TA, typename TB>
+cudaError_t simt_gemm_sliced(int64_t M, int64_t N, int64_t K, const TA* A, int64_t sam, int64_t sak, const TB* B,
+                             int64_t sbn, int64_t sbk, float* C, float* part, cudaStream_t st) {
+    if (M <= 0 || N <= 0) return cudaSuccess;
+    const int S = k_slices(M, N, K);
+    if (S == 1) return simt_gemm(M, N, K, A, sam, sak, B, sbn, sbk, C, N, st);
+    const int64_t kchunk = ((K + S - 1) / S + 15) / 16 * 16;
+    const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + 63) / 64), (unsigned)S);
+    bwd_simt_gemm_kernel<TA, TB><<<grid, 256, 0, st>>>(M, N, K, A, sam, sak, B, sbn, sbk, part, N, kchunk, M * N);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bwd_reduce_kernel<<<grid_blocks(M * N), 256, 0, st>>>(part, S, M * N, C);
     return cudaGetLastError();
 }
 
@@ -531,7 +583,7 @@ cudaError_t simt_gemm(int64_t M, int64_t N, int64_t K, const TA* A, int64_t sam,
 // ---------------------------------------------------------------------------
 struct BwdLayout {
     size_t tstart, nkb, mt_start, offs_d, offs_f, mt_d, mt_f, sh_off, sh_tstart, sh_nkb, counters;
-    size_t logits, dG, dwc, Wt_d, Wt_gu, dYp, Z, U, Gd, dzu, dxp, doT, xT, hT, dzT, duT;
+    size_t logits, dG, part, part_db, dwc, Wt_d, Wt_gu, dYp, Z, U, Gd, dzu, dxp, doT, xT, hT, dzT, duT;
     size_t dYs, Zs, Us, Gs, dzus, dxs, WsT_d, WsT_gu, dYsT, xsT, hsT, dzsT, dusT;
     int64_t Kmax, Kmax_sh;
     size_t total;
@@ -581,6 +633,8 @@ BwdLayout bwd_layout(const moe_params& p, int64_t Kmax) {
     L.counters = take(CNT_COUNT * 8);
     L.logits = take(N * E * 4);
     L.dG = take(N * E * 4);
+    L.part = take((size_t)kMaxSlices * E * d * 4);
+    L.part_db = take((size_t)kMaxSlices * E * 4);
     L.dwc = take(rows * 4);
     L.Wt_d = take(E * df * d * 2);
     L.Wt_gu = take(E * d * 2 * df * 2);
@@ -818,10 +872,14 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     const bf16* xb = static_cast<const bf16*>(x);
     const bf16* Wrb = static_cast<const bf16*>(W_r);
     e = simt_gemm<float, bf16>(N, d, E, dG, E, 1, Wrb, 1, d, gr->dx, d, st);
-    if (e == cudaSuccess) e = simt_gemm<float, bf16>(E, d, N, dG, 1, E, xb, 1, d, gr->dW_r, d, st);
+    if (e == cudaSuccess)  // K = N tokens, few output tiles: sliced over the tokens
+        e = simt_gemm_sliced<float, bf16>(E, d, N, dG, 1, E, xb, 1, d, gr->dW_r, F32(L.part), st);
     if (e != cudaSuccess) return bwd_fail(e, "router contractions");
     if (gr->db_r) {
-        bwd_colsum_kernel<<<(unsigned)((E + 31) / 32), 256, 0, st>>>(dG, N, (int)E, gr->db_r);
+        const int64_t chunk = (N + kMaxSlices - 1) / kMaxSlices;
+        bwd_colsum_kernel<<<dim3((unsigned)((E + 31) / 32), (unsigned)kMaxSlices), 256, 0, st>>>(dG, N, (int)E, chunk,
+                                                                                                 F32(L.part_db));
+        bwd_reduce_kernel<<<grid_blocks(E), 256, 0, st>>>(F32(L.part_db), kMaxSlices, E, gr->db_r);
         if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "db");
     }
 
