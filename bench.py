@@ -598,6 +598,10 @@ def backward_kernels(w: si.Workload) -> int:
     tiles = ((w.E + 63) // 64) * ((w.d + 63) // 64)
     sms = 148
     slices = max(1, min(-(-2 * sms // tiles), max(1, w.N // 256), 16))
+    if w.dtype != si.DT_BF16:
+        # fp32: scores, two gathers, SwiGLU, router chain, dx; per touched expert
+        # z, u, W_d^T dY, two dx-row and three weight-gradient contractions
+        return 1 + 2 + 1 + (3 + 2 + (1 if slices > 1 else 0)) + 1 + 8 * w.E + (8 if w.d_f_shared else 0)
     return 30 + (1 if slices > 1 else 0) + (19 if w.d_f_shared else 0)
 
 
@@ -610,8 +614,6 @@ def run_gpu_backward(args):
     if dist_env()[0] > 1:
         raise SystemExit("--backward runs on one GPU")
     w = si.WORKLOADS[args.workload]
-    if w.dtype != si.DT_BF16:
-        raise SystemExit("the backward pass is built for bf16 layers")
     inp = si.inputs(w)
     dY_host = si.upstream_gradient(w)
     torch.cuda.set_device(0)
@@ -673,8 +675,9 @@ def run_gpu_backward(args):
     flops = 16.0 * R * w.d * w.d_f + 16.0 * w.N * w.d * ds + 6.0 * w.N * w.E * w.d
     # least HBM traffic: bf16 weights read, fp32 weight gradients written, x and
     # dY read, dx written
-    nbytes = (3.0 * touched * w.d * w.d_f * (2 + 4) + 3.0 * w.d * ds * (2 + 4)
-              + w.N * w.d * (2 + 4 + 4) + w.E * w.d * (2 + 4))
+    es = 2 if w.dtype == si.DT_BF16 else 4
+    nbytes = (3.0 * touched * w.d * w.d_f * (es + 4) + 3.0 * w.d * ds * (es + 4)
+              + w.N * w.d * (es + 4 + 4) + w.E * w.d * (es + 4))
     peaks, peak_src = load_peaks()
     timed_s = ms_step * args.steps / 1000.0
     peak_tf = peaks["bf16_tflops"] if timed_s < 1.0 else peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -682,7 +685,12 @@ def run_gpu_backward(args):
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     tflops = flops / (ms_step * 1e-3) / 1e12
     gbs = nbytes / (ms_step * 1e-3) / 1e9
-    if t_tensor >= t_hbm:
+    if w.dtype != si.DT_BF16:
+        # fp32 layers contract on the CUDA cores: bound by FP32 arithmetic
+        peak_ffma = ffma_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
+        roof = {"bound": "alu", "achieved": tflops, "peak": peak_ffma, "unit": "TFLOP/s",
+                "frac": tflops / peak_ffma}
+    elif t_tensor >= t_hbm:
         roof = {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s", "frac": tflops / peak_tf}
     else:
         roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -694,7 +702,7 @@ def run_gpu_backward(args):
         "metric": "MoE-layer backward tokens/s (gradients of x, W_r, b_r, experts, shared expert)",
         "value": w.N / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == si.DT_BF16 else "f32",
         "data": "synthetic (seeded; dY ~ N(0,1)); no dataset or checkpoint",
         "config": dict(config_of(w, args), l2="flushed between steps (256 MiB write)"),
         "roofline": roof, "gpu_launches": backward_kernels(w) * args.steps, "clocks": clk.summary(),

@@ -436,7 +436,7 @@ MOE_API moe_status moe_soft_check(const moe_soft_params* p, const void* ws, moe_
  *   -> probability -> score (softmax Jacobian) -> dx_t += W_r^T dg_t,
  *   dW_r = dg^T X, db_r = sum_t dg_t; the shared expert as an expert with
  *   weight 1 on every token.
- * Precision: dY enters rounded to bf16; the forward's bf16 h is used as
+ * Precision (bf16 layers): dY enters rounded to bf16; the forward's bf16 h is used as
  * stored (its rounding passes the gradient through); wc dY, dz and du are
  * rounded to bf16 as tensor-core operands; every accumulation and all router
  * arithmetic are fp32.  Gradients are fp32.
@@ -451,7 +451,8 @@ MOE_API moe_status moe_soft_check(const moe_soft_params* p, const void* ws, moe_
  * backward workspace (at least moe_backward_workspace_size bytes for these
  * offsets, 256-byte aligned recommended); aux_coef the objective's
  * coefficient (0: none).
- * Constraints: dtype MOE_BF16 (MOE_ERR_UNSUPPORTED for fp32 layers), E_r <=
+ * fp32 layers: the same chain on the CUDA cores, nothing rounded.
+ * Constraints: E_r <=
  * 256, k <= 32, N <= 65535 * 64; single routing group (not after
  * moe_forward_end).
  * Errors: MOE_ERR_INVALID_ARG (null or misaligned pointers, offsets_host not

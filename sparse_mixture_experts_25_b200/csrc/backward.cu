@@ -66,6 +66,19 @@ unsigned grid_blocks(int64_t n) {  // 256-thread blocks for a grid-stride loop o
     return (unsigned)std::max<int64_t>(b, 1);
 }
 
+// four consecutive elements as fp32 (8-byte bf16 or 16-byte fp32 accesses)
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 ld4(const bf16* p) {
+    const uint2 q = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void st4(bf16* p, float4 v) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pk2(v.x, v.y), pk2(v.z, v.w));
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -205,13 +218,14 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// out[r, :] = bf16(dY[tok(r), :]) for r < n (tok = slot_token[r], or r when
-// slot_token is null; n = *n_dev clamped to max_rows, or n_fixed).  One warp
-// per row, 4 columns per lane step.
+// out[r, :] = scale[r] dY[tok(r), :] in T (bf16: rounded) for r < n (tok =
+// slot_token[r], or r when slot_token is null; scale null: 1; n = *n_dev
+// clamped to max_rows, or n_fixed).  One warp per row, 4 columns per step.
+template <typename T>
 __global__ void __launch_bounds__(256)
     bwd_gather_dy_kernel(const float* __restrict__ dY, int64_t d, const int32_t* __restrict__ slot_token,
                          const int32_t* __restrict__ n_dev, int64_t n_fixed, int64_t max_rows, int64_t n_tokens,
-                         bf16* __restrict__ out) {
+                         const float* __restrict__ scale, T* __restrict__ out) {
     int64_t n = n_fixed;
     if (n_dev) {
         n = *n_dev;
@@ -222,24 +236,27 @@ __global__ void __launch_bounds__(256)
     for (int64_t r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += (int64_t)gridDim.x * wpb) {
         const int64_t tok = slot_token ? (int64_t)slot_token[r] : r;
         const bool ok = tok >= 0 && tok < n_tokens;
-        uint2* o = reinterpret_cast<uint2*>(out + r * d);
-        const float4* src = reinterpret_cast<const float4*>(dY + (ok ? tok : 0) * d);
+        const float s = scale ? scale[r] : 1.f;
+        const float* src = dY + (ok ? tok : 0) * d;
         for (int64_t c = lane; c < d / 4; c += 32) {
-            float4 v = ok ? src[c] : make_float4(0.f, 0.f, 0.f, 0.f);
-            o[c] = make_uint2(pk2(v.x, v.y), pk2(v.z, v.w));
+            float4 v = ok ? ld4(src + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v.x *= s; v.y *= s; v.z *= s; v.w *= s;
+            st4(out + r * d + 4 * c, v);
         }
     }
 }
 
 // SwiGLU backward of routed (or shared) rows r < n: with dh = wc[r] Gd[r],
-//   dz = dh u SiLU'(z), du = dh SiLU(z)  ->  dzu[r] = [dz | du] (bf16, 2 d_f)
+//   dz = dh u SiLU'(z), du = dh SiLU(z)  ->  dzu[r] = [dz | du] (TO, 2 d_f)
 //   dwc[r] = <Gd[r], h[r]>                  (fp32; skipped when dwc is null)
 // SiLU(z) = z s(z), SiLU'(z) = s(z) (1 + z (1 - s(z))), s the logistic
-// function.  wc null: weight 1.  One warp per row.
+// function.  wc null: weight 1.  TH: the forward's h type; TO: bf16 (rounded
+// tensor-core operands) or fp32.  One warp per row.
+template <typename TH, typename TO>
 __global__ void __launch_bounds__(256)
     bwd_swiglu_kernel(const float* __restrict__ Z, const float* __restrict__ U, const float* __restrict__ Gd,
-                      const bf16* __restrict__ H, int64_t d_f, const float* __restrict__ wc,
-                      const int32_t* __restrict__ n_dev, int64_t n_fixed, int64_t max_rows, bf16* __restrict__ dzu,
+                      const TH* __restrict__ H, int64_t d_f, const float* __restrict__ wc,
+                      const int32_t* __restrict__ n_dev, int64_t n_fixed, int64_t max_rows, TO* __restrict__ dzu,
                       float* __restrict__ dwc) {
     int64_t n = n_fixed;
     if (n_dev) {
@@ -250,19 +267,11 @@ __global__ void __launch_bounds__(256)
     const int64_t wpb = blockDim.x >> 5;
     for (int64_t r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += (int64_t)gridDim.x * wpb) {
         const float w = wc ? wc[r] : 1.f;
-        const float4* z4 = reinterpret_cast<const float4*>(Z + r * d_f);
-        const float4* u4 = reinterpret_cast<const float4*>(U + r * d_f);
-        const float4* g4 = reinterpret_cast<const float4*>(Gd + r * d_f);
-        const uint2* h4 = reinterpret_cast<const uint2*>(H + r * d_f);
-        uint2* dz4 = reinterpret_cast<uint2*>(dzu + r * 2 * d_f);
-        uint2* du4 = reinterpret_cast<uint2*>(dzu + r * 2 * d_f + d_f);
         float acc = 0.f;
-        for (int64_t c = lane; c < d_f / 4; c += 32) {
-            const float4 z = z4[c], u = u4[c], g = g4[c];
-            const uint2 hq = h4[c];
-            const float2 h01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hq.x));
-            const float2 h23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hq.y));
-            acc += g.x * h01.x + g.y * h01.y + g.z * h23.x + g.w * h23.y;
+        for (int64_t c = 4 * lane; c < d_f; c += 128) {
+            const float4 z = ld4(Z + r * d_f + c), u = ld4(U + r * d_f + c), g = ld4(Gd + r * d_f + c);
+            const float4 h = ld4(H + r * d_f + c);
+            acc += g.x * h.x + g.y * h.y + g.z * h.z + g.w * h.w;
             const float zz[4] = {z.x, z.y, z.z, z.w}, uu[4] = {u.x, u.y, u.z, u.w}, gg[4] = {g.x, g.y, g.z, g.w};
             float dz[4], du[4];
 #pragma unroll
@@ -272,8 +281,8 @@ __global__ void __launch_bounds__(256)
                 du[i] = dh * (zz[i] * s);
                 dz[i] = dh * uu[i] * (s * (1.f + zz[i] * (1.f - s)));
             }
-            dz4[c] = make_uint2(pk2(dz[0], dz[1]), pk2(dz[2], dz[3]));
-            du4[c] = make_uint2(pk2(du[0], du[1]), pk2(du[2], du[3]));
+            st4(dzu + r * 2 * d_f + c, make_float4(dz[0], dz[1], dz[2], dz[3]));
+            st4(dzu + r * 2 * d_f + d_f + c, make_float4(du[0], du[1], du[2], du[3]));
         }
         acc = warp_sum(acc);
         if (dwc && lane == 0) dwc[r] = acc;
@@ -489,7 +498,7 @@ template <typename TA, typename TB>
 __global__ void __launch_bounds__(256)
     bwd_simt_gemm_kernel(int64_t M, int64_t N, int64_t K, const TA* __restrict__ A, int64_t sam, int64_t sak,
                          const TB* __restrict__ B, int64_t sbn, int64_t sbk, float* __restrict__ C, int64_t ldc,
-                         int64_t kchunk, int64_t cz) {
+                         int64_t kchunk, int64_t cz, int accumulate) {
     __shared__ float As[16][64 + 4];
     __shared__ float Bs[16][64 + 4];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -536,17 +545,19 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int64_t n = n0 + tx * 4 + j;
-            if (n < N) C[m * ldc + n] = acc[i][j];
+            if (n < N) C[m * ldc + n] = accumulate ? C[m * ldc + n] + acc[i][j] : acc[i][j];
         }
     }
 }
 
+// accumulate: C += the product instead of C = the product
 template <typename TA, typename TB>
 cudaError_t simt_gemm(int64_t M, int64_t N, int64_t K, const TA* A, int64_t sam, int64_t sak, const TB* B,
-                      int64_t sbn, int64_t sbk, float* C, int64_t ldc, cudaStream_t st) {
+                      int64_t sbn, int64_t sbk, float* C, int64_t ldc, cudaStream_t st, int accumulate = 0) {
     if (M <= 0 || N <= 0) return cudaSuccess;
     const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + 63) / 64), 1);
-    bwd_simt_gemm_kernel<TA, TB><<<grid, 256, 0, st>>>(M, N, K, A, sam, sak, B, sbn, sbk, C, ldc, K + 16, 0);
+    bwd_simt_gemm_kernel<TA, TB><<<grid, 256, 0, st>>>(M, N, K, A, sam, sak, B, sbn, sbk, C, ldc, K + 16, 0,
+                                                       accumulate);
     return cudaGetLastError();
 }
 
@@ -571,7 +582,7 @@ cudaError_t simt_gemm_sliced(int64_t M, int64_t N, int64_t K, const TA* A, int64
     if (S == 1) return simt_gemm(M, N, K, A, sam, sak, B, sbn, sbk, C, N, st);
     const int64_t kchunk = ((K + S - 1) / S + 15) / 16 * 16;
     const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + 63) / 64), (unsigned)S);
-    bwd_simt_gemm_kernel<TA, TB><<<grid, 256, 0, st>>>(M, N, K, A, sam, sak, B, sbn, sbk, part, N, kchunk, M * N);
+    bwd_simt_gemm_kernel<TA, TB><<<grid, 256, 0, st>>>(M, N, K, A, sam, sak, B, sbn, sbk, part, N, kchunk, M * N, 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     bwd_reduce_kernel<<<grid_blocks(M * N), 256, 0, st>>>(part, S, M * N, C);
@@ -583,7 +594,7 @@ cudaError_t simt_gemm_sliced(int64_t M, int64_t N, int64_t K, const TA* A, int64
 // ---------------------------------------------------------------------------
 struct BwdLayout {
     size_t tstart, nkb, mt_start, offs_d, offs_f, mt_d, mt_f, sh_off, sh_tstart, sh_nkb, counters;
-    size_t logits, dG, part, part_db, dwc, Wt_d, Wt_gu, dYp, Z, U, Gd, dzu, dxp, doT, xT, hT, dzT, duT;
+    size_t logits, dG, part, part_db, dwc, doP, Wt_d, Wt_gu, dYp, Z, U, Gd, dzu, dxp, doT, xT, hT, dzT, duT;
     size_t dYs, Zs, Us, Gs, dzus, dxs, WsT_d, WsT_gu, dYsT, xsT, hsT, dzsT, dusT;
     int64_t Kmax, Kmax_sh;
     size_t total;
@@ -597,6 +608,7 @@ int64_t up64(int64_t v) { return (v + kTT - 1) / kTT * kTT; }
 // largest nkb), from the host offsets, else the bound min(capacity, N).
 int64_t kmax_of(const moe_params& p, const int32_t* offsets_host) {
     int64_t m = kTT;
+    if (p.dtype != MOE_BF16) return m;  // no transposed operands
     if (offsets_host) {
         for (int64_t g = 0; g < p.E_r; ++g) m = std::max(m, up64((int64_t)offsets_host[g + 1] - offsets_host[g]));
         return m;
@@ -606,10 +618,16 @@ int64_t kmax_of(const moe_params& p, const int32_t* offsets_host) {
     return std::max(m, up64(std::min<int64_t>(C, p.N)));
 }
 
+// bf16 layers: tensor-core operands in bf16, transposed weights and the
+// [E][C][Kmax] weight-gradient operands.  fp32 layers: fp32 rows only (their
+// CUDA-core contractions read any layout through strides).
 BwdLayout bwd_layout(const moe_params& p, int64_t Kmax) {
+    const bool b16 = p.dtype == MOE_BF16;
     const size_t N = (size_t)p.N, d = (size_t)p.d, df = (size_t)p.d_f, E = (size_t)p.E_r;
     const size_t rows = N * (size_t)p.k;
     const size_t ds = p.d_f_shared > 0 ? (size_t)p.d_f_shared : 0;
+    const size_t es = b16 ? 2 : 4;     // element size of the operand buffers
+    const size_t tb = b16 ? 1 : 0;     // bf16-only buffers
     BwdLayout L{};
     L.Kmax = Kmax;
     L.Kmax_sh = std::max<int64_t>(kTT, up64(p.N));
@@ -636,33 +654,34 @@ BwdLayout bwd_layout(const moe_params& p, int64_t Kmax) {
     L.part = take((size_t)kMaxSlices * E * d * 4);
     L.part_db = take((size_t)kMaxSlices * E * 4);
     L.dwc = take(rows * 4);
-    L.Wt_d = take(E * df * d * 2);
-    L.Wt_gu = take(E * d * 2 * df * 2);
-    L.dYp = take(rows * d * 2);
+    L.doP = take((1 - tb) * rows * d * 4);
+    L.Wt_d = take(tb * E * df * d * 2);
+    L.Wt_gu = take(tb * E * d * 2 * df * 2);
+    L.dYp = take(rows * d * es);
     L.Z = take(rows * df * 4);
     L.U = take(rows * df * 4);
     L.Gd = take(rows * df * 4);
-    L.dzu = take(rows * 2 * df * 2);
+    L.dzu = take(rows * 2 * df * es);
     L.dxp = take(rows * d * 4);
-    L.doT = take(E * d * K * 2);
-    L.xT = take(E * d * K * 2);
-    L.hT = take(E * df * K * 2);
-    L.dzT = take(E * df * K * 2);
-    L.duT = take(E * df * K * 2);
+    L.doT = take(tb * E * d * K * 2);
+    L.xT = take(tb * E * d * K * 2);
+    L.hT = take(tb * E * df * K * 2);
+    L.dzT = take(tb * E * df * K * 2);
+    L.duT = take(tb * E * df * K * 2);
     if (ds) {
-        L.dYs = take(N * d * 2);
+        L.dYs = take(tb * N * d * 2);
         L.Zs = take(N * ds * 4);
         L.Us = take(N * ds * 4);
         L.Gs = take(N * ds * 4);
-        L.dzus = take(N * 2 * ds * 2);
+        L.dzus = take(N * 2 * ds * es);
         L.dxs = take(N * d * 4);
-        L.WsT_d = take(ds * d * 2);
-        L.WsT_gu = take(d * 2 * ds * 2);
-        L.dYsT = take(d * Ks * 2);
-        L.xsT = take(d * Ks * 2);
-        L.hsT = take(ds * Ks * 2);
-        L.dzsT = take(ds * Ks * 2);
-        L.dusT = take(ds * Ks * 2);
+        L.WsT_d = take(tb * ds * d * 2);
+        L.WsT_gu = take(tb * d * 2 * ds * 2);
+        L.dYsT = take(tb * d * Ks * 2);
+        L.xsT = take(tb * d * Ks * 2);
+        L.hsT = take(tb * ds * Ks * 2);
+        L.dzsT = take(tb * ds * Ks * 2);
+        L.dusT = take(tb * ds * Ks * 2);
     }
     L.total = off;
     return L;
@@ -682,11 +701,154 @@ moe_status bwd_check(const moe_params* p) {
     size_t ws = 0;
     const moe_status s = moe_workspace_size(p, &ws);  // the forward's parameter checks
     if (s != MOE_OK) return s;
-    if (p->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
     if (p->E_r > kMaxRouterExperts || p->k > kMaxK) return MOE_ERR_UNSUPPORTED;
     if (p->N > (int64_t)65535 * 64) return MOE_ERR_UNSUPPORTED;  // grid rows of the router contractions
     // rows of the grouped weight-gradient GEMMs (E_r groups of d or d_f rows)
     if ((int64_t)p->E_r * std::max(p->d, p->d_f) >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+// blocks of 8 warps for one warp per item, at most 16 per SM (grid-stride)
+unsigned grid_for(int64_t items_per_block_units, int64_t n) {
+    int64_t b = (n + items_per_block_units - 1) / items_per_block_units;
+    const int64_t cap = (int64_t)num_sms() * 16;
+    if (b > cap) b = cap;
+    if (b < 1) b = 1;
+    return (unsigned)b;
+}
+
+// Router chain of the backward: score gradient dG (bwd_router_kernel), then
+// dx = dG W_r (written), dW_r = dG^T X (sliced over the tokens) and db_r.
+template <typename T>
+moe_status router_backward(const moe_params& p, float aux_coef, const T* x, const T* W_r, const float* b_r,
+                           const WsView& v, const float* logits, const float* dwc, float* dG, float* part,
+                           float* part_db, const moe_grads* gr, cudaStream_t st) {
+    const int64_t N = p.N, d = p.d, E = p.E_r;
+    RouterBwd ra{};
+    ra.logits = logits;
+    ra.b_r = b_r;
+    ra.ids = v.ids;
+    ra.w = v.w;
+    ra.slot = v.slot;
+    ra.offsets = v.offsets;
+    ra.dwc = dwc;
+    ra.L = v.L;
+    ra.counters = v.counters;
+    ra.dG = dG;
+    ra.N = N;
+    ra.E = (int)E;
+    ra.k = p.k;
+    ra.norm = p.norm;
+    ra.policy = p.reject_policy;
+    ra.aux_coef = aux_coef;
+    ra.max_rows = N * p.k;
+    bwd_router_kernel<<<grid_for(8, N), 256, 0, st>>>(ra);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return bwd_fail(e, "router");
+    e = simt_gemm<float, T>(N, d, E, dG, E, 1, W_r, 1, d, gr->dx, d, st);
+    if (e == cudaSuccess)  // K = N tokens, few output tiles: sliced over the tokens
+        e = simt_gemm_sliced<float, T>(E, d, N, dG, 1, E, x, 1, d, gr->dW_r, part, st);
+    if (e != cudaSuccess) return bwd_fail(e, "router contractions");
+    if (gr->db_r) {
+        const int64_t chunk = (N + kMaxSlices - 1) / kMaxSlices;
+        bwd_colsum_kernel<<<dim3((unsigned)((E + 31) / 32), (unsigned)kMaxSlices), 256, 0, st>>>(dG, N, (int)E, chunk,
+                                                                                                 part_db);
+        bwd_reduce_kernel<<<grid_blocks(E), 256, 0, st>>>(part_db, kMaxSlices, E, gr->db_r);
+        if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "db");
+    }
+    return MOE_OK;
+}
+
+// The fp32 layer: every contraction on the CUDA cores (bwd_simt_gemm_kernel
+// reads the weights and rows in place through strides), one launch per expert
+// and contraction; nothing is rounded.
+moe_status backward_f32(const moe_params& p, float aux_coef, const int32_t* off_h, const float* x, const float* W_r,
+                        const float* b_r, const float* W_g, const float* W_u, const float* W_d, const float* Ws_g,
+                        const float* Ws_u, const float* Ws_d, const float* dY, const WsView& v, const moe_grads* gr,
+                        char* b, const BwdLayout& L, cudaStream_t st) {
+    const int64_t N = p.N, d = p.d, df = p.d_f, E = p.E_r, rows = N * p.k;
+    auto F32 = [&](size_t o) { return reinterpret_cast<float*>(b + o); };
+    float *logits = F32(L.logits), *dG = F32(L.dG), *dwc = F32(L.dwc), *dYp = F32(L.dYp), *doP = F32(L.doP);
+    float *Z = F32(L.Z), *U = F32(L.U), *Gd = F32(L.Gd), *dzu = F32(L.dzu), *dxp = F32(L.dxp);
+    const float* xp = static_cast<const float*>(v.x_perm);
+    const float* hp = static_cast<const float*>(v.h);
+    const int32_t* n_rows = v.offsets + E;
+    cudaError_t e = simt_gemm<float, float>(N, E, d, x, d, 1, W_r, d, 1, logits, E, st);
+    if (e != cudaSuccess) return bwd_fail(e, "scores");
+    // dY rows of the accepted paths, and wc dY for dW_d
+    bwd_gather_dy_kernel<float><<<grid_for(8, rows), 256, 0, st>>>(dY, d, v.slot_token, n_rows, 0, rows, N, nullptr,
+                                                                   dYp);
+    bwd_gather_dy_kernel<float><<<grid_for(8, rows), 256, 0, st>>>(dY, d, v.slot_token, n_rows, 0, rows, N, v.slot_w,
+                                                                   doP);
+    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "dY rows");
+    for (int64_t g = 0; g < E; ++g) {
+        const int64_t o = off_h[g], R = off_h[g + 1] - off_h[g];
+        if (R == 0) continue;
+        const float* Wg = W_g + g * df * d;
+        const float* Wu = W_u + g * df * d;
+        const float* Wd = W_d + g * d * df;
+        e = simt_gemm<float, float>(R, df, d, xp + o * d, d, 1, Wg, d, 1, Z + o * df, df, st);
+        if (e == cudaSuccess) e = simt_gemm<float, float>(R, df, d, xp + o * d, d, 1, Wu, d, 1, U + o * df, df, st);
+        // W_d^T dY: B(j, i) = W_d[i, j]
+        if (e == cudaSuccess) e = simt_gemm<float, float>(R, df, d, dYp + o * d, d, 1, Wd, 1, df, Gd + o * df, df, st);
+        if (e != cudaSuccess) return bwd_fail(e, "z, u, W_d^T dY");
+    }
+    bwd_swiglu_kernel<float, float><<<grid_for(8, rows), 256, 0, st>>>(Z, U, Gd, hp, df, v.slot_w, n_rows, 0, rows,
+                                                                       dzu, dwc);
+    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "SwiGLU backward");
+    for (int64_t g = 0; g < E; ++g) {  // dx rows = dz W_g + du W_u: B(i, j) = W[j, i]
+        const int64_t o = off_h[g], R = off_h[g + 1] - off_h[g];
+        if (R == 0) continue;
+        e = simt_gemm<float, float>(R, d, df, dzu + o * 2 * df, 2 * df, 1, W_g + g * df * d, 1, d, dxp + o * d, d, st);
+        if (e == cudaSuccess)
+            e = simt_gemm<float, float>(R, d, df, dzu + o * 2 * df + df, 2 * df, 1, W_u + g * df * d, 1, d,
+                                        dxp + o * d, d, st, 1);
+        if (e != cudaSuccess) return bwd_fail(e, "dx rows");
+    }
+    moe_status s = router_backward<float>(p, aux_coef, x, W_r, b_r, v, logits, dwc, dG, F32(L.part), F32(L.part_db),
+                                          gr, st);
+    if (s != MOE_OK) return s;
+    float* dxs = nullptr;
+    if (p.d_f_shared > 0) {
+        const int64_t ds = p.d_f_shared;
+        const float* hs = static_cast<const float*>(v.h_shared);
+        float *Zs = F32(L.Zs), *Us = F32(L.Us), *Gs = F32(L.Gs), *dzus = F32(L.dzus);
+        dxs = F32(L.dxs);
+        e = simt_gemm<float, float>(N, ds, d, x, d, 1, Ws_g, d, 1, Zs, ds, st);
+        if (e == cudaSuccess) e = simt_gemm<float, float>(N, ds, d, x, d, 1, Ws_u, d, 1, Us, ds, st);
+        if (e == cudaSuccess) e = simt_gemm<float, float>(N, ds, d, dY, d, 1, Ws_d, 1, ds, Gs, ds, st);
+        if (e != cudaSuccess) return bwd_fail(e, "shared z, u, W_d^T dY");
+        bwd_swiglu_kernel<float, float><<<grid_for(8, N), 256, 0, st>>>(Zs, Us, Gs, hs, ds, nullptr, nullptr, N, N,
+                                                                        dzus, nullptr);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = simt_gemm<float, float>(N, d, ds, dzus, 2 * ds, 1, Ws_g, 1, d, dxs, d, st);
+        if (e == cudaSuccess) e = simt_gemm<float, float>(N, d, ds, dzus + ds, 2 * ds, 1, Ws_u, 1, d, dxs, d, st, 1);
+        // weight gradients over the tokens: A(m, t) and B(n, t) read column-wise
+        if (e == cudaSuccess) e = simt_gemm<float, float>(d, ds, N, dY, 1, d, hs, 1, ds, gr->dWs_d, ds, st);
+        if (e == cudaSuccess) e = simt_gemm<float, float>(ds, d, N, dzus, 1, 2 * ds, x, 1, d, gr->dWs_g, d, st);
+        if (e == cudaSuccess) e = simt_gemm<float, float>(ds, d, N, dzus + ds, 1, 2 * ds, x, 1, d, gr->dWs_u, d, st);
+        if (e != cudaSuccess) return bwd_fail(e, "shared expert");
+    }
+    bwd_dx_kernel<<<grid_for(8, N), 256, 0, st>>>(gr->dx, dxp, dxs, v.ids, v.slot, v.offsets, N, d, p.k, (int)E, rows);
+    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "dx");
+    for (int64_t g = 0; g < E; ++g) {  // weight gradients over the expert's rows
+        const int64_t o = off_h[g], R = off_h[g + 1] - off_h[g];
+        float* gWd = gr->dW_d + g * d * df;
+        float* gWg = gr->dW_g + g * df * d;
+        float* gWu = gr->dW_u + g * df * d;
+        if (R == 0) {
+            e = cudaMemsetAsync(gWd, 0, sizeof(float) * d * df, st);
+            if (e == cudaSuccess) e = cudaMemsetAsync(gWg, 0, sizeof(float) * d * df, st);
+            if (e == cudaSuccess) e = cudaMemsetAsync(gWu, 0, sizeof(float) * d * df, st);
+        } else {
+            e = simt_gemm<float, float>(d, df, R, doP + o * d, 1, d, hp + o * df, 1, df, gWd, df, st);
+            if (e == cudaSuccess)
+                e = simt_gemm<float, float>(df, d, R, dzu + o * 2 * df, 1, 2 * df, xp + o * d, 1, d, gWg, d, st);
+            if (e == cudaSuccess)
+                e = simt_gemm<float, float>(df, d, R, dzu + o * 2 * df + df, 1, 2 * df, xp + o * d, 1, d, gWu, d, st);
+        }
+        if (e != cudaSuccess) return bwd_fail(e, "weight gradients");
+    }
     return MOE_OK;
 }
 
@@ -696,14 +858,6 @@ bool offsets_valid(const moe_params& p, const int32_t* o) {
     for (int64_t e = 0; e < p.E_r; ++e)
         if (o[e + 1] < o[e]) return false;
     return (int64_t)o[p.E_r] <= p.N * p.k;
-}
-
-unsigned grid_for(int64_t items_per_block_units, int64_t n) {
-    int64_t b = (n + items_per_block_units - 1) / items_per_block_units;
-    const int64_t cap = (int64_t)num_sms() * 16;
-    if (b > cap) b = cap;
-    if (b < 1) b = 1;
-    return (unsigned)b;
 }
 
 }  // namespace
@@ -767,6 +921,13 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     WsView v;
     make_view(*p, const_cast<void*>(ws), v);
     char* b = static_cast<char*>(bws);
+    e = cudaMemsetAsync(b + L.counters, 0, CNT_COUNT * 8, st);
+    if (e != cudaSuccess) return bwd_fail(e, "memset");
+    if (p->dtype == MOE_F32)
+        return backward_f32(*p, aux_coef, offsets_host, static_cast<const float*>(x), static_cast<const float*>(W_r),
+                            b_r, static_cast<const float*>(W_g), static_cast<const float*>(W_u),
+                            static_cast<const float*>(W_d), static_cast<const float*>(Ws_g),
+                            static_cast<const float*>(Ws_u), static_cast<const float*>(Ws_d), dY, v, gr, b, L, st);
     auto I32 = [&](size_t o) { return reinterpret_cast<int32_t*>(b + o); };
     auto F32 = [&](size_t o) { return reinterpret_cast<float*>(b + o); };
     auto B16 = [&](size_t o) { return reinterpret_cast<bf16*>(b + o); };
@@ -791,8 +952,6 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
         n_tiles += R > 0 ? (R + kTT - 1) / kTT : 1;
     }
 
-    e = cudaMemsetAsync(counters, 0, CNT_COUNT * 8, st);
-    if (e != cudaSuccess) return bwd_fail(e, "memset");
     bwd_tables_kernel<<<1, 32, 0, st>>>((int)E, v.offsets, tstart, nkb);
     bwd_strided_offsets_kernel<<<1, 256, 0, st>>>((int)E, (int32_t)d, offs_d);
     bwd_strided_offsets_kernel<<<1, 256, 0, st>>>((int)E, (int32_t)df, offs_f);
@@ -815,7 +974,8 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     bwd_batched_transpose_kernel<<<dim3((unsigned)((df + kTT - 1) / kTT), (unsigned)((d + kTT - 1) / kTT), (unsigned)E),
                                    256, 0, st>>>(static_cast<const bf16*>(W_u), df, d, Wt_gu + df, 2 * df, d * 2 * df);
     // dY rows of the accepted paths, bf16
-    bwd_gather_dy_kernel<<<grid_for(8, rows), 256, 0, st>>>(dY, d, v.slot_token, n_rows, 0, rows, N, dYp);
+    bwd_gather_dy_kernel<bf16><<<grid_for(8, rows), 256, 0, st>>>(dY, d, v.slot_token, n_rows, 0, rows, N, nullptr,
+                                                                  dYp);
     if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "transposes");
 
     // row-grouped contractions on the grouped tcgen05 kernel (store mode):
@@ -837,7 +997,8 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     e = launch_tc_down(q, DOWN_STORE, N, dYp, nullptr, v.offsets, mt_start, W0, nullptr, nullptr, nullptr, Gd,
                        counters, st, &status);
     if (e != cudaSuccess) return bwd_fail(e, "W_d^T dY (tcgen05)");
-    bwd_swiglu_kernel<<<grid_for(8, rows), 256, 0, st>>>(Z, U, Gd, hp, df, v.slot_w, n_rows, 0, rows, dzu, dwc);
+    bwd_swiglu_kernel<bf16, bf16><<<grid_for(8, rows), 256, 0, st>>>(Z, U, Gd, hp, df, v.slot_w, n_rows, 0, rows, dzu,
+                                                                     dwc);
     if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "SwiGLU backward");
     moe_params q2 = *p;
     q2.d_f_shared = 0;
@@ -848,40 +1009,10 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
                        counters, st, &status);
     if (e != cudaSuccess) return bwd_fail(e, "dx rows (tcgen05)");
 
-    // router: score gradient, then dx = dG W_r, dW_r = dG^T X, db = colsum dG
-    RouterBwd ra{};
-    ra.logits = logits;
-    ra.b_r = b_r;
-    ra.ids = v.ids;
-    ra.w = v.w;
-    ra.slot = v.slot;
-    ra.offsets = v.offsets;
-    ra.dwc = dwc;
-    ra.L = v.L;
-    ra.counters = v.counters;
-    ra.dG = dG;
-    ra.N = N;
-    ra.E = (int)E;
-    ra.k = (int)k;
-    ra.norm = p->norm;
-    ra.policy = p->reject_policy;
-    ra.aux_coef = aux_coef;
-    ra.max_rows = rows;
-    bwd_router_kernel<<<grid_for(8, N), 256, 0, st>>>(ra);
-    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "router");
     const bf16* xb = static_cast<const bf16*>(x);
-    const bf16* Wrb = static_cast<const bf16*>(W_r);
-    e = simt_gemm<float, bf16>(N, d, E, dG, E, 1, Wrb, 1, d, gr->dx, d, st);
-    if (e == cudaSuccess)  // K = N tokens, few output tiles: sliced over the tokens
-        e = simt_gemm_sliced<float, bf16>(E, d, N, dG, 1, E, xb, 1, d, gr->dW_r, F32(L.part), st);
-    if (e != cudaSuccess) return bwd_fail(e, "router contractions");
-    if (gr->db_r) {
-        const int64_t chunk = (N + kMaxSlices - 1) / kMaxSlices;
-        bwd_colsum_kernel<<<dim3((unsigned)((E + 31) / 32), (unsigned)kMaxSlices), 256, 0, st>>>(dG, N, (int)E, chunk,
-                                                                                                 F32(L.part_db));
-        bwd_reduce_kernel<<<grid_blocks(E), 256, 0, st>>>(F32(L.part_db), kMaxSlices, E, gr->db_r);
-        if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "db");
-    }
+    if ((s = router_backward<bf16>(*p, aux_coef, xb, static_cast<const bf16*>(W_r), b_r, v, logits, dwc, dG,
+                                   F32(L.part), F32(L.part_db), gr, st)) != MOE_OK)
+        return s;
 
     // shared expert: weight 1 on every token
     float* dxs = nullptr;
@@ -893,7 +1024,7 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
         int32_t *sh_off = I32(L.sh_off), *sh_ts = I32(L.sh_tstart), *sh_nkb = I32(L.sh_nkb);
         bwd_single_group_kernel<<<1, 32, 0, st>>>((int32_t)N, sh_off);
         bwd_tables_kernel<<<1, 32, 0, st>>>(1, sh_off, sh_ts, sh_nkb);
-        bwd_gather_dy_kernel<<<grid_for(8, N), 256, 0, st>>>(dY, d, nullptr, nullptr, N, N, N, dYs);
+        bwd_gather_dy_kernel<bf16><<<grid_for(8, N), 256, 0, st>>>(dY, d, nullptr, nullptr, N, N, N, nullptr, dYs);
         bwd_batched_transpose_kernel<<<dim3((unsigned)((d + kTT - 1) / kTT), (unsigned)((dfs + kTT - 1) / kTT), 1), 256,
                                        0, st>>>(static_cast<const bf16*>(Ws_d), d, dfs, WsT_d, d, 0);
         bwd_batched_transpose_kernel<<<dim3((unsigned)((dfs + kTT - 1) / kTT), (unsigned)((d + kTT - 1) / kTT), 1), 256,
@@ -905,8 +1036,8 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
         if (e == cudaSuccess) e = launch_tc_dense(N, dfs, d, x, Ws_u, Us, counters, st, &status);
         if (e == cudaSuccess) e = launch_tc_dense(N, dfs, d, dYs, WsT_d, Gs, counters, st, &status);
         if (e != cudaSuccess) return bwd_fail(e, "shared z, u, W_d^T dY (tcgen05)");
-        bwd_swiglu_kernel<<<grid_for(8, N), 256, 0, st>>>(Zs, Us, Gs, static_cast<const bf16*>(v.h_shared), dfs,
-                                                          nullptr, nullptr, N, N, dzus, nullptr);
+        bwd_swiglu_kernel<bf16, bf16><<<grid_for(8, N), 256, 0, st>>>(Zs, Us, Gs, static_cast<const bf16*>(v.h_shared),
+                                                                      dfs, nullptr, nullptr, N, N, dzus, nullptr);
         if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "shared SwiGLU backward");
         e = launch_tc_dense(N, d, 2 * dfs, dzus, WsT_gu, dxs, counters, st, &status);
         if (e != cudaSuccess) return bwd_fail(e, "shared dx (tcgen05)");

@@ -169,9 +169,10 @@ def test_backward_checks_arguments_on_the_host():
     assert ctypes.sizeof(moe.Grads) == 9 * 8
     p = moe.params(16, 64, 64, 8, 2, c=1.0)
     sz = ctypes.c_size_t()
-    # fp32 layers have no backward; E_r above the router kernel's limit neither
-    assert L.moe_backward_workspace_size(ctypes.byref(moe.params(16, 64, 64, 8, 2, dtype=moe.MOE_F32)), None,
-                                         ctypes.byref(sz)) == moe.MOE_ERR_UNSUPPORTED
+    # fp32 layers keep fp32 rows only (no transposed operands); E_r above the
+    # router kernel's limit has no backward
+    p32 = moe.params(16, 64, 64, 8, 2, c=1.0, dtype=moe.MOE_F32)
+    assert 0 < moe.moe_backward_workspace_size(p32) < moe.moe_backward_workspace_size(p)
     assert L.moe_backward_workspace_size(ctypes.byref(moe.params(16, 64, 64, 300, 2)), None,
                                          ctypes.byref(sz)) == moe.MOE_ERR_UNSUPPORTED
     good = [0, 4, 4, 8, 12, 16, 20, 24, 28]

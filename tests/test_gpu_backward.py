@@ -17,10 +17,12 @@ Tolerances (max-abs error over max-abs reference, per gradient):
     policy, the renormalisation, the balance objective) moves them by far
     more;
   * the balance objective's gradient alone (dY = 0): 1e-4.
+  * fp32 layers (CUDA-core contractions, nothing rounded): 1e-4, the forward's
+    fp32 bound.
 Cases span single-CTA and CTA-pair tiles, ragged row, column and K tails,
 capacity rejection under both overflow policies, acceptance by weight, WLR
 pruning, a shared expert, an expert count that is not a multiple of 4 (score
-recomputation on the CUDA cores) and the empty batch.
+recomputation on the CUDA cores), fp32 layers and the empty batch.
 """
 import numpy as np
 import pytest
@@ -51,8 +53,13 @@ CASES = {
                                                 accept_order=1, reject_policy=1),
     "odd_experts": W["mixtral_bf16"].scaled("bwd_odd_experts", N=200, d=64, d_f=64, E=34, k=3, c=1.0),
     "one_expert_ragged": W["mixtral_bf16"].scaled("bwd_one_expert", N=200, d=64, d_f=136, E=1, k=1),
+    # fp32 layers (every contraction on the CUDA cores, nothing rounded)
+    "switch_f32_capped": W["switch_top1_f32"].scaled("bwd_switch_f32", N=1000, d=72, d_f=96, c=0.9),
+    "renorm_f32_shared_policy1": W["switch_top1_f32"].scaled("bwd_f32_shared", N=500, d=64, d_f=80, E=6, k=2,
+                                                            norm=si.NORM_RENORM, c=0.8, d_f_shared=40,
+                                                            reject_policy=1),
 }
-AUX = {"qwen3_capped_aux": 0.5, "weight_order": 0.3, "odd_experts": 1.0}
+AUX = {"qwen3_capped_aux": 0.5, "weight_order": 0.3, "odd_experts": 1.0, "switch_f32_capped": 0.5}
 
 
 def _grads(w, device="cuda"):
@@ -99,6 +106,8 @@ def test_backward_matches_oracle(name):
         assert np.isfinite(g).all(), n
         errs[n] = parity.rel_err(g, ref[n])
         tol = 2e-3 if n in ("dW_r", "db_r") else 5e-3
+        if w.dtype == si.DT_F32:
+            tol = 1e-4       # fp32 accumulation against float64, nothing rounded
         assert errs[n] <= tol, (n, errs[n], errs)
     # experts that received no rows have exactly zero weight gradients
     empty = np.nonzero(full["rec"]["acc"] == 0)[0]
