@@ -229,3 +229,11 @@ def test_backward_of_an_empty_batch_needs_no_dx():
     r = L.moe_backward(ctypes.byref(p), 0.0, arr, None, None, None, None, None, None, None, None, None, None,
                        fake, ctypes.byref(g), fake, 0, None)
     assert r not in (moe.MOE_ERR_INVALID_ARG, moe.MOE_ERR_WORKSPACE)
+
+
+def test_backward_binding_checks_the_offsets_shape():
+    p = moe.params(16, 64, 64, 8, 2)
+    with pytest.raises(ValueError):
+        moe.moe_backward_workspace_size(p, [0, 1, 2])
+    with pytest.raises(ValueError):
+        moe.moe_backward(p, [0] * 8, None, None, None, None, None, None, None, None, None, None, None, {}, None)
