@@ -239,10 +239,16 @@ MOE_API moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const f
  *
  * The first call on each device looks up the array's device address (with
  * that device current); make that first call before any stream capture.
+ * With lazy module loading (the CUDA 12 default) that first lookup may be
+ * what loads the library onto the device: a one-time reservation of the
+ * 1 MiB array that can synchronise the device.  Make the first call early
+ * (for example at start-up, with N = 0), outside any region that must not
+ * allocate.  The address is looked up again after the device's context was
+ * destroyed and re-created (cudaDeviceReset).
  * Every call shares the array: a call clears the counters it accumulates and
  * overwrites the rest, and the array keeps the last call's contents.  Calls
- * that overlap on the GPU (unordered streams or threads) race on it.  The
- * entry point allocates no memory, host or device.
+ * that overlap on the GPU (unordered streams or threads) race on it.  After
+ * that first call the entry point allocates no memory, host or device.
  */
 MOE_API moe_status moe_dispatch_noalloc(const moe_params* p, const int32_t* ids, const float* w,
                                         int64_t C, int32_t* slot, int32_t* offsets,
@@ -490,7 +496,10 @@ MOE_API moe_status moe_backward(const moe_params* p, float aux_coef, const int32
 
 /* Waits for `stream` and reports MOE_ERR_TIMEOUT if a bounded device wait of
  * the last moe_backward on `bws` gave up (its tensor-core GEMMs record that in
- * the backward workspace), else MOE_OK. */
+ * the backward workspace), MOE_ERR_INVALID_ARG if the offsets_host given to
+ * that call differed from the forward's offsets on the device (a stale or
+ * foreign host copy: the launches were sized from it, so the gradients are
+ * not valid), else MOE_OK. */
 MOE_API moe_status moe_backward_check(const moe_params* p, const void* bws, moe_stream_t stream);
 
 /*

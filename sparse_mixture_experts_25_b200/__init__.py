@@ -399,12 +399,14 @@ def moe_backward(p, offsets_host, x, W_r, b_r, W_g, W_u, W_d, Ws_g, Ws_u, Ws_d, 
     g = Grads(*[_ptr(grads.get(n)) for n in GRAD_NAMES])
     _check(lib().moe_backward(ctypes.byref(p), float(aux_coef), off.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                               _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W_g), _ptr(W_u), _ptr(W_d), _ptr(Ws_g), _ptr(Ws_u),
-                              _ptr(Ws_d), _ptr(dY), _ptr(ws), ctypes.byref(g), _ptr(bws), int(bws.numel()),
+                              _ptr(Ws_d), _ptr(dY), _ptr(ws), ctypes.byref(g), _ptr(bws),
+                              int(bws.numel()) * int(bws.element_size()),
                               _stream(stream)),
            "moe_backward")
 
 
 def moe_backward_check(p, bws, stream=None) -> int:
     """Waits for the stream; MOE_ERR_TIMEOUT if a bounded wait of the last
-    moe_backward on bws gave up, else MOE_OK."""
+    moe_backward on bws gave up, MOE_ERR_INVALID_ARG if its offsets_host
+    differed from the forward's device offsets, else MOE_OK."""
     return lib().moe_backward_check(ctypes.byref(p), _ptr(bws), _stream(stream))

@@ -103,6 +103,23 @@ __global__ void bwd_tables_kernel(int G, const int32_t* __restrict__ offsets, in
     tstart[G] = t;
 }
 
+// The caller's host copy of the forward's offsets, passed by value.
+struct HostOffsets {
+    int32_t v[kMaxRouterExperts + 1];
+};
+
+// The launches, the operand blocks and the fp32 per-expert contractions are
+// sized from the caller's host copy of the offsets; the kernels read the
+// device copy.  A copy that differs (stale, or from another forward) would
+// give wrong gradients without any fault: record it as DEVERR_BOUNDS, which
+// moe_backward_check reports.
+__global__ void bwd_offsets_check_kernel(int G, const int32_t* __restrict__ offsets, HostOffsets host,
+                                         unsigned long long* counters) {
+    bool bad = false;
+    for (int g = threadIdx.x; g <= G; g += blockDim.x) bad |= offsets[g] != host.v[g];
+    if (__syncthreads_or(bad) && threadIdx.x == 0)
+        atomicOr(counters + CNT_DEVICE_ERROR, (unsigned long long)DEVERR_BOUNDS);
+}
 // off[e] = e C for e = 0..E: groups of C consecutive rows
 __global__ void bwd_strided_offsets_kernel(int E, int32_t C, int32_t* __restrict__ off) {
     for (int e = threadIdx.x; e <= E; e += blockDim.x) off[e] = e * C;
@@ -923,6 +940,13 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     char* b = static_cast<char*>(bws);
     e = cudaMemsetAsync(b + L.counters, 0, CNT_COUNT * 8, st);
     if (e != cudaSuccess) return bwd_fail(e, "memset");
+    {
+        HostOffsets ho;
+        for (int64_t g = 0; g <= p->E_r; ++g) ho.v[g] = offsets_host[g];
+        bwd_offsets_check_kernel<<<1, 256, 0, st>>>(p->E_r, v.offsets,
+                                                    ho, reinterpret_cast<unsigned long long*>(b + L.counters));
+        if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "offsets check");
+    }
     if (p->dtype == MOE_F32)
         return backward_f32(*p, aux_coef, offsets_host, static_cast<const float*>(x), static_cast<const float*>(W_r),
                             b_r, static_cast<const float*>(W_g), static_cast<const float*>(W_u),
@@ -1122,6 +1146,7 @@ moe_status moe_backward_check(const moe_params* p, const void* bws, moe_stream_t
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return bwd_fail(e, "check");
     if (cnt[CNT_DEVICE_ERROR] & DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+    if (cnt[CNT_DEVICE_ERROR] & DEVERR_BOUNDS) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
 

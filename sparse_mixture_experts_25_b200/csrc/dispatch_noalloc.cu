@@ -14,6 +14,14 @@
 // counters that must start at zero, and the buffer keeps the last call's
 // contents afterwards.  Calls that overlap on the GPU (different streams or
 // threads without ordering between them) race on it.
+//
+// The array's device address is looked up once per device and context: the
+// first call on a device (and the first after that device's context was
+// destroyed and re-created, e.g. by cudaDeviceReset) queries it with the
+// device current.  With lazy module loading (the CUDA 12 default) that first
+// query can be what loads the library's kernels onto the device, which
+// reserves the 1 MiB array and may synchronise; later calls do neither.
+#include <cudaTypedefs.h>
 #include <mutex>
 #include <stdio.h>
 
@@ -34,7 +42,33 @@ static __device__ __align__(256) unsigned char g_dispatch_scratch[kScratchBytes]
 
 constexpr int kMaxDevices = 64;
 void* g_scratch_addr[kMaxDevices] = {nullptr};
+unsigned long long g_scratch_ctx[kMaxDevices] = {0};  // id of the context the address belongs to
 std::mutex g_setup_mutex;
+
+// Unique id of the calling thread's current context (0 if it cannot be read,
+// in which case the address is looked up again on every call).
+unsigned long long current_context_id() {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static bool looked_up = false;
+    if (!looked_up) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+        looked_up = true;
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
 
 size_t scratch_needed(const moe_params& p, int n_tiles) {
     const size_t E = (size_t)p.E_r;
@@ -42,18 +76,22 @@ size_t scratch_needed(const moe_params& p, int n_tiles) {
 }
 
 // Device address of the scratch array for the current device (set-up on the
-// first call per device: a symbol-address query with that device current).
+// first call per device and context: a symbol-address query with that device
+// current).  A cached address is dropped when the device's context changed
+// since it was taken (a reset frees the array with the old context).
 cudaError_t scratch_address(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
+    const unsigned long long ctx = current_context_id();  // 0 before the runtime made one current
+    if (!g_scratch_addr[dev] || ctx == 0 || g_scratch_ctx[dev] != ctx) {
         void* ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_dispatch_scratch);
+        e = cudaGetSymbolAddress(&ptr, g_dispatch_scratch);  // makes the primary context current
         if (e != cudaSuccess) return e;
         g_scratch_addr[dev] = ptr;
+        g_scratch_ctx[dev] = current_context_id();
     }
     *out = g_scratch_addr[dev];
     return cudaSuccess;

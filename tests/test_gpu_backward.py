@@ -151,3 +151,23 @@ def test_backward_rejects_bad_offsets():
     with pytest.raises(moe.MoEError):
         moe.moe_backward(p, bad, dev["x"], dev["W_r"], None, dev["W_g"], dev["W_u"], dev["W_d"], None, None, None,
                          dY, full["ws"], g, bws)
+
+
+def test_backward_check_reports_stale_host_offsets():
+    """Host offsets that pass the host checks (a non-decreasing prefix from 0)
+    but are not the forward's: the backward sizes its launches from them, so
+    moe_backward_check must report the mismatch instead of MOE_OK."""
+    w = CASES["mixtral_small"]
+    inp = si.inputs(w)
+    full = parity.gpu_forward(w, inp)
+    p, dev = full["p"], full["dev"]
+    g = _grads(w)
+    good = full["rec"]["offsets"].astype(np.int32)
+    stale = (good // 2).astype(np.int32)          # every expert with about half its rows
+    assert (np.diff(stale) >= 0).all() and stale[0] == 0 and (stale != good).any()
+    dY = torch.zeros(w.N, w.d, device="cuda")
+    for offs, want in ((stale, moe.MOE_ERR_INVALID_ARG), (good, moe.MOE_OK)):
+        bws = torch.empty(moe.moe_backward_workspace_size(p, offs), dtype=torch.uint8, device="cuda")
+        moe.moe_backward(p, offs, dev["x"], dev["W_r"], None, dev["W_g"], dev["W_u"], dev["W_d"], None, None, None,
+                         dY, full["ws"], g, bws)
+        assert moe.moe_backward_check(p, bws) == want

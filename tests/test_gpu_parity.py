@@ -80,7 +80,7 @@ def _end_to_end(w):
     parity.check_dispatch(w, out["rec"], out["stats"])
     aux = oracle.aux_balance(r["logits"], out["rec"]["ids"], w.E, r["invalid"])
     assert abs(out["stats"]["aux_balance"] - aux) <= 1e-4 * max(1.0, aux)
-    err = parity.check_rows(w, inp, out["rec"], out["Y"])
+    err, row = parity.check_rows(w, inp, out["rec"], out["Y"])
     flips = int((out["rec"]["ids"] != r["ids"]).any(axis=1).sum())
     if flips == 0:
         # routing identical: compare against the oracle's whole forward as well
@@ -93,22 +93,23 @@ def _end_to_end(w):
         # the GPU, double in the oracle): compare the whole forward when both
         # accepted the same paths (the oracle-on-GPU-weights check above is exact)
         if w.accept_order == 0 or np.array_equal(full["slot"], out["rec"]["slot"]):
-            assert parity.rel_err(out["Y"], full["Y"]) <= parity.TOL[w.dtype]
+            parity.assert_rows_close(out["Y"], full["Y"], parity.TOL[w.dtype])
     assert out["status"] == moe.MOE_OK
-    return out, err, int(near.sum())
+    return out, (err, row), int(near.sum())
 
 
 @pytest.mark.parametrize("name", list(SMALL))
 def test_forward_small(name):
-    out, err, near = _end_to_end(SMALL[name])
-    print(f"{name}: max-abs-rel {err:.2e}, near-ties {near}, stats {out['stats']}")
+    out, (err, row), near = _end_to_end(SMALL[name])
+    print(f"{name}: max-abs-rel {err:.2e} (largest per row {row:.2e}), near-ties {near}, stats {out['stats']}")
 
 
 def test_switch_top1_f32_full():
     """The Switch-shaped fp32 layer at its full size, every output row."""
-    out, err, near = _end_to_end(W["switch_top1_f32"])
+    out, (err, row), near = _end_to_end(W["switch_top1_f32"])
     assert out["stats"]["C"] == 160
-    print(f"switch_top1_f32: max-abs-rel {err:.2e}, near-ties {near}, stats {out['stats']}")
+    print(f"switch_top1_f32: max-abs-rel {err:.2e} (largest per row {row:.2e}), near-ties {near}, "
+          f"stats {out['stats']}")
 
 
 def test_capacity_drops_give_zero_rows():
@@ -251,7 +252,7 @@ def test_unfused_path_matches_fused(name):
         if hi == lo:
             continue
         ref = oracle.swiglu_rows(inp["x"], st[lo:hi], inp["W_g"][e], inp["W_u"][e], inp["W_d"][e])
-        assert parity.rel_err(Hh[lo:hi], ref) <= parity.TOL[w.dtype]
+        parity.assert_rows_close(Hh[lo:hi], ref, parity.TOL[w.dtype])
     Y = torch.zeros(N, d, device="cuda")
     moe.moe_combine(p, H, r["offsets"], r["st"], r["sw"], Y)
     assert parity.rel_err(Y.cpu().numpy().astype(np.float64), fused["Y"]) <= 1e-5
@@ -364,8 +365,7 @@ def test_expert_choice(dtype, N, d, d_f, E, C):
     want = {(int(t), e) for e in range(E) for t in ec["picks"][e]}
     assert got == want
     assert (np.bincount([e for _, e in got], minlength=E) == C).all()
-    err = parity.rel_err(out["Y"], ec["Y"])
-    assert err <= parity.TOL[dtype], err
+    err, row = parity.assert_rows_close(out["Y"], ec["Y"], parity.TOL[dtype])
     unpicked = np.setdiff1d(np.arange(N), [t for t, _ in got])
     assert (out["Y"][unpicked] == 0).all()
     print(f"expert choice E={E} C={C}: max-abs-rel {err:.2e}, tokens with no expert {unpicked.size}")
@@ -388,9 +388,8 @@ def test_soft_moe(N, d, d_f, E, p):
     ref = oracle.soft_moe(inp["x"], inp["Phi"], inp["W_g"], inp["W_u"], inp["W_d"], p)
     Yg = Y.cpu().numpy().astype(np.float64)
     assert np.isfinite(Yg).all()
-    err = parity.rel_err(Yg, ref["Y"])
-    assert err <= parity.TOL[si.DT_BF16], err
-    print(f"soft MoE N={N} S={E * p}: max-abs-rel {err:.2e}")
+    err, row = parity.assert_rows_close(Yg, ref["Y"], parity.TOL[si.DT_BF16])
+    print(f"soft MoE N={N} S={E * p}: max-abs-rel {err:.2e}, largest per-row {row:.2e}")
 
 
 # ---------------------------------------------------------------------------
@@ -403,56 +402,69 @@ def _sample_tokens(N, n, seed):
     return np.array(sorted(pick))
 
 
-@pytest.mark.parametrize("name,n_sample", [("mixtral_bf16", 12), ("qwen3_skew_bf16", 12),
-                                           ("wdmoe_decode_bf16", 16), ("qwen3_skew_bf16:weight", 8)])
-def test_full_size_sampled(name, n_sample):
+@pytest.mark.parametrize("name,n_sample", [("mixtral_bf16", 256), ("qwen3_skew_bf16", 256),
+                                           ("wdmoe_decode_bf16", 64), ("qwen3_skew_bf16:weight", 256)])
+def test_full_size_dense(name, n_sample):
+    """The page-shaped layers at full size in the benchmark's launch
+    configuration: routing and dispatch on every token; outputs on every
+    token that owns a row in some expert's last (ragged) row tile, plus
+    n_sample seeded random tokens, each row within the tolerance on its own
+    (ch. 36.3: every accepted record is combined exactly once)."""
     base, _, order = name.partition(":")
     w = W[base] if not order else W[base].scaled(name, accept_order=1)
     inp = si.inputs(w)
     out = parity.gpu_forward(w, inp)
     r, near = parity.check_routing(w, inp, out["rec"])
     parity.check_dispatch(w, out["rec"], out["stats"])
-    toks = _sample_tokens(w.N, n_sample, 7)
-    err = parity.check_rows(w, inp, out["rec"], out["Y"], tokens=toks)
-    print(f"{name}: max-abs-rel {err:.2e} on {toks.size} tokens, near-ties {int(near.sum())}, "
-          f"stats {out['stats']}")
+    tail = parity.last_tile_tokens(out["rec"])
+    toks = np.union1d(tail, _sample_tokens(w.N, n_sample, 7))
+    err, row = parity.check_rows(w, inp, out["rec"], out["Y"], tokens=toks)
+    print(f"{name}: max-abs-rel {err:.2e}, largest per-row {row:.2e} on {toks.size} tokens "
+          f"({tail.size} with a row in a last tile), near-ties {int(near.sum())}, stats {out['stats']}")
     assert np.isfinite(out["Y"]).all()
 
 
-def test_full_size_deepseek_shared_sampled():
-    """DeepSeek-V3-shaped layer with the shared expert (22.6 GB of bf16 weights):
-    weights are generated and uploaded one expert at a time, and the oracle
-    regenerates only the experts its sampled tokens use."""
+def test_full_size_deepseek_shared_dense():
+    """DeepSeek-V3-shaped layer with the shared expert (22.6 GB of bf16 weights).
+    The weights are generated and uploaded one expert at a time; 96 seeded
+    tokens whose routing is not a near-tie are chosen from the oracle's
+    routing before the upload, and each expert's oracle rows for them are
+    computed while that expert's weights are on the host."""
     w = W["deepseek_shared_bf16"]
     small = {n: si.tensor(w, n) for n in ("x", "W_r", "Ws_g", "Ws_u", "Ws_d")}
+    r = oracle.route(small["x"], small["W_r"], k=w.k, norm=w.norm)
+    clear = np.nonzero((r["margin"] >= parity.NEAR) & ~r["invalid"])[0]
+    rng = np.random.default_rng(11)
+    toks = np.sort(rng.choice(clear, size=96, replace=False))
+    touched = np.unique(r["ids"][toks])
+    assert touched.size >= 32
     dev = {n: parity.to_dev(v) for n, v in small.items()}
+    rows = {}   # (token, expert) -> oracle E_e(x_t)
     for n in ("W_g", "W_u", "W_d"):
-        shp = si.shape(w, n)
-        t = torch.empty(shp, dtype=torch.bfloat16, device="cuda")
-        for e in range(w.E):
-            t[e].copy_(parity.to_dev(si.tensor(w, n, expert=e)))
-        dev[n] = t
+        dev[n] = torch.empty(si.shape(w, n), dtype=torch.bfloat16, device="cuda")
+    for e in range(w.E):
+        We = [si.tensor(w, n, expert=e) for n in ("W_g", "W_u", "W_d")]
+        for n, a in zip(("W_g", "W_u", "W_d"), We):
+            dev[n][e].copy_(parity.to_dev(a))
+        mine = [t for t in toks if e in r["ids"][t]]
+        if mine:
+            out_e = oracle.swiglu_rows(small["x"], mine, *We)
+            for t, v in zip(mine, out_e):
+                rows[(int(t), e)] = v
     out = parity.gpu_forward(w, small, dev=dev)
-    r, near = parity.check_routing(w, small, out["rec"])
+    rr, near = parity.check_routing(w, small, out["rec"])
     parity.check_dispatch(w, out["rec"], out["stats"])
-    toks = _sample_tokens(w.N, 6, 11)
     rec = out["rec"]
-    ref = np.zeros((toks.size, w.d))
-    cache = {}
+    assert (rec["ids"][toks] == r["ids"][toks]).all()
+    ref = oracle.swiglu_rows(small["x"], toks, small["Ws_g"], small["Ws_u"], small["Ws_d"])
     for i, t in enumerate(toks):
         for j in range(w.k):
             e = int(rec["ids"][t, j])
-            if e < 0 or rec["slot"][t, j] < 0:
-                continue
-            if e not in cache:
-                cache.clear()
-                cache[e] = [si.tensor(w, n, expert=e) for n in ("W_g", "W_u", "W_d")]
-            g, u, dn = cache[e]
-            ref[i] += float(rec["w"][t, j]) * oracle.swiglu_rows(small["x"], [t], g, u, dn)[0]
-    ref += oracle.swiglu_rows(small["x"], toks, small["Ws_g"], small["Ws_u"], small["Ws_d"])
-    err = parity.rel_err(out["Y"][toks], ref)
-    print(f"deepseek_shared_bf16: max-abs-rel {err:.2e}, near-ties {int(near.sum())}, stats {out['stats']}")
-    assert err <= parity.TOL[w.dtype]
+            assert rec["slot"][t, j] >= 0   # no capacity limit: every path is accepted
+            ref[i] += float(rec["w"][t, j]) * rows[(int(t), e)]
+    err, row = parity.assert_rows_close(out["Y"][toks], ref, parity.TOL[w.dtype])
+    print(f"deepseek_shared_bf16: max-abs-rel {err:.2e}, largest per-row {row:.2e} on {toks.size} tokens "
+          f"over {touched.size} experts, near-ties {int(near.sum())}, stats {out['stats']}")
 
 
 def test_forward_on_a_side_stream_with_stage_events():

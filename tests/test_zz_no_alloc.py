@@ -73,6 +73,24 @@ def test_noalloc_dispatch_matches_workspace_dispatch_on_two_calls_in_a_row():
             assert (ref["slot"] < 0).any()
 
 
+def test_noalloc_dispatch_leaves_free_device_memory_unchanged():
+    """After a first call (which may load the library and reserve its static
+    array), further calls change nothing in the device's free memory."""
+    w = si.WORKLOADS["qwen3_skew_bf16"].scaled("noalloc_mem", N=2048, d=128, d_f=64, E=64, k=8)
+    p, dev, ids, wt, ws = _routed(w)
+    C = moe.moe_capacity(p)
+    out = _outputs(w, dev["x"].dtype)
+    args = (p, ids, wt, C, out["slot"], out["offsets"], out["st"], out["sw"], dev["x"], out["x_perm"])
+    moe.moe_dispatch_noalloc(*args)           # warm-up: the one-time set-up happens here at the latest
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        moe.moe_dispatch_noalloc(*args)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+
+
 def test_noalloc_dispatch_rejects_sizes_beyond_its_buffer():
     p = moe.params(1 << 20, 64, 64, 1024, 1)
     dummy = torch.zeros(8, dtype=torch.int32, device="cuda")
