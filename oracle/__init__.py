@@ -72,9 +72,12 @@ def _load():
         lib.oracle_forward.argtypes = [i64, i32, i32, i32, i32, i32, dbl, i32, i64, i32, i32, i32,
                                        _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                        _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+        lib.oracle_reroute_candidates.argtypes = [i64, i32, i32, i32, i32, _P, _P, _P, _P, _P]
+        lib.oracle_dispatch_reroute.argtypes = [i64, i32, i32, i64, i32, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         lib.oracle_round_bf16.argtypes = [dbl]
         lib.oracle_round_bf16.restype = dbl
         for f in ("oracle_route", "oracle_dispatch", "oracle_dispatch_ranked", "oracle_reject_weights",
+                  "oracle_reroute_candidates", "oracle_dispatch_reroute",
                   "oracle_swiglu_rows", "oracle_combine",
                   "oracle_forward_rows", "oracle_forward"):
             getattr(lib, f).restype = ctypes.c_int
@@ -231,6 +234,65 @@ def dispatch_ranked(ids, E: int, C: int, base):
     return {"slot": slot, "L": L, "acc": acc, "stats": {n: int(v) for n, v in zip(names, cnt)}}
 
 
+def reroute_candidates(logits, ids, invalid, k: int, X: int, norm: int):
+    """Each token's next-ranked experts (ranks k .. k+X-1, -1 past E_r) and
+    their weights under the layer's normalisation against the token's chosen
+    set (see oracle.c, rerouting as an overflow policy).  logits [N, E] f64,
+    ids [N, k], invalid [N] bool.  Returns (cand [N, X] int32, cand_w [N, X] f64)."""
+    lg = _c(np.asarray(logits, np.float64))
+    N, E = lg.shape
+    ids = _c(ids, np.int32)
+    inv = _c(np.asarray(invalid, np.uint8))
+    cand = np.empty((N, X), np.int32)
+    cw = np.empty((N, X), np.float64)
+    rc = _load().oracle_reroute_candidates(N, E, k, X, norm, _ptr(lg), _ptr(ids), _ptr(inv), _ptr(cand), _ptr(cw))
+    if rc:
+        raise ValueError("oracle_reroute_candidates: invalid arguments")
+    return cand, cw
+
+
+def dispatch_reroute(ids, cand, E: int, C: int):
+    """Token-order acceptance with rerouting of rejected paths to each token's
+    next-ranked experts with free slots, in rounds (see oracle.c).  Returns
+    slot (first choice), rr_e, rr_slot, rr_q [N, k], L (first-choice loads),
+    acc (rows per expert, rerouted included) and the statistics."""
+    ids = _c(ids, np.int32)
+    cand = _c(cand, np.int32)
+    N, k = ids.shape
+    X = cand.shape[1]
+    slot = np.empty((N, k), np.int32)
+    rr_e = np.empty((N, k), np.int32)
+    rr_slot = np.empty((N, k), np.int32)
+    rr_q = np.empty((N, k), np.int32)
+    L = np.empty(E, np.int64)
+    acc = np.empty(E, np.int64)
+    cnt = np.empty(9, np.int64)
+    rc = _load().oracle_dispatch_reroute(N, k, E, C, X, _ptr(ids), _ptr(cand), _ptr(slot), _ptr(rr_e),
+                                         _ptr(rr_slot), _ptr(rr_q), _ptr(L), _ptr(acc), _ptr(cnt))
+    if rc:
+        raise ValueError("oracle_dispatch_reroute: invalid arguments")
+    names = ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max",
+             "rerouted", "rounds")
+    return {"slot": slot, "rr_e": rr_e, "rr_slot": rr_slot, "rr_q": rr_q, "L": L, "acc": acc,
+            "stats": {n: int(v) for n, v in zip(names, cnt)}}
+
+
+def served_records(ids, w, slot, rr_e, rr_slot, rr_q, cand_w):
+    """The paths that run an expert, as [N, 2k] records for forward_rows:
+    columns 0..k-1 the first-choice paths (weight a_te, slot or -1), columns
+    k..2k-1 the rerouted paths (their candidate's weight, slot or -1)."""
+    ids = np.asarray(ids, np.int32)
+    N, k = ids.shape
+    rr_e = np.asarray(rr_e, np.int32)
+    rq = np.asarray(rr_q)
+    cw = np.asarray(cand_w, np.float64)
+    w_rr = np.where(rq >= 0, cw[np.arange(N)[:, None], np.maximum(rq, 0)], 0.0)
+    ids2 = np.concatenate([ids, rr_e], axis=1).astype(np.int32)
+    w2 = np.concatenate([np.asarray(w, np.float64), w_rr], axis=1)
+    slot2 = np.concatenate([np.asarray(slot, np.int32), np.asarray(rr_slot, np.int32)], axis=1)
+    return ids2, w2, slot2
+
+
 def swiglu_rows(x, rows, Wg, Wu, Wd, round_h=None):
     """E(x_t) for t in rows, for one expert with weights Wg, Wu [d_f, d] and
     Wd [d, d_f].  Returns [len(rows), d] float64."""
@@ -300,15 +362,21 @@ def reject_weights(ids, w, slot, policy: int):
 
 
 def forward(x, W_r, Wg, Wu, Wd, *, k: int, norm: int, c: float = 0.0, theta: float = 0.0,
-            b_r=None, lat=None, Ws=None, reject_policy: int = 0, accept_order: int = 0):
+            b_r=None, lat=None, Ws=None, reject_policy: int = 0, accept_order: int = 0,
+            reroute_depth: int = 0):
     """The whole layer (Algorithm 36.1 generalised by the weighting mode and a
     shared expert).  Returns a dict with Y [N,d] f64, the routing records,
-    per-expert loads and the statistics."""
+    per-expert loads and the statistics.  reject_policy 2 reroutes rejected
+    paths to up to reroute_depth next-ranked experts per token (token-order
+    acceptance only)."""
     x, W_r, Wg, Wu, Wd = _c(x), _c(W_r), _c(Wg), _c(Wu), _c(Wd)
     dt = _dtype_of(x)
     N, d = x.shape
     E, d_f = Wg.shape[0], Wg.shape[1]
     C = capacity(c, N, k, E)
+    if reject_policy == 2:
+        return _forward_reroute(x, W_r, Wg, Wu, Wd, k=k, norm=norm, C=C, b_r=b_r, Ws=Ws,
+                                depth=reroute_depth)
     Y = np.zeros((N, d), np.float64)
     ids = np.empty((N, k), np.int32)
     w = np.empty((N, k), np.float64)
@@ -341,6 +409,25 @@ def forward(x, W_r, Wg, Wu, Wd, *, k: int, norm: int, c: float = 0.0, theta: flo
     stats["rho_max"] = rho_max(L, N, k, E) if N else 0.0
     return {"Y": Y, "ids": ids, "w": w, "slot": slot, "margin": margin, "wlr_gap": gap,
             "invalid": inv.astype(bool), "L": L, "acc": acc, "stats": stats, "C": C}
+
+
+def _forward_reroute(x, W_r, Wg, Wu, Wd, *, k, norm, C, b_r, Ws, depth):
+    """forward() under rerouting: route, each token's candidates, token-order
+    acceptance with rerouting rounds, then every served path's expert output
+    weighted and summed per token (plus the shared expert)."""
+    N, d = x.shape
+    E = Wg.shape[0]
+    r = route(x, W_r, k=k, norm=norm, b_r=b_r)
+    cand, cw = reroute_candidates(r["logits"], r["ids"], r["invalid"], k, depth, norm)
+    dr = dispatch_reroute(r["ids"], cand, E, C)
+    ids2, w2, slot2 = served_records(r["ids"], r["w"], dr["slot"], dr["rr_e"], dr["rr_slot"], dr["rr_q"], cw)
+    Y = forward_rows(x, ids2, w2, slot2, np.arange(N), Wg, Wu, Wd, Ws=Ws) if N else np.zeros((0, d))
+    stats = dict(dr["stats"])
+    stats["C"] = C
+    stats["rho_max"] = rho_max(dr["L"], N, k, E) if N else 0.0
+    return {"Y": Y, "ids": r["ids"], "w": r["w"], "slot": dr["slot"], "margin": r["margin"],
+            "wlr_gap": r["wlr_gap"], "invalid": r["invalid"], "L": dr["L"], "acc": dr["acc"], "stats": stats,
+            "C": C, "cand": cand, "cand_w": cw, "rr_e": dr["rr_e"], "rr_slot": dr["rr_slot"], "rr_q": dr["rr_q"]}
 
 
 def expert_choice(x, W_r, Wg, Wu, Wd, C: int, b_r=None, P=None):

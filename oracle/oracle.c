@@ -372,6 +372,159 @@ int oracle_reject_weights(int64_t N, int k, int policy, const int32_t* ids, cons
 }
 
 /*
+ * Rerouting as an overflow policy ("LLM from scratch" ch. 36.3, capacity and
+ * overflow: handling a path past capacity is part of the model definition;
+ * besides zeroing it, a rejected path may be rerouted, which calls another
+ * expert's parameters; the same section notes that other experts' free slots
+ * do not stand in for the full expert's function; vegetog "MoE token routing"
+ * sec. 5: an over-capacity token is dropped from that expert's branch or
+ * rerouted, depending on the implementation).  The pages do not say to which
+ * expert or with what weight.  Reading taken here:
+ *
+ *  - A token's rerouting candidates are its experts of ranks k, k+1, ...,
+ *    k+X-1 in the router's order (score descending, ties to the lower index),
+ *    i.e. the experts it would have chosen next.
+ *  - A candidate carries the weight the router's normalisation gives it
+ *    against the token's chosen set S (the same factor as the token's other
+ *    paths): p_e / sum_{S} p under renormalisation, p_e under the full
+ *    probability.  (WLR pruning is not combined with rerouting.)
+ *  - Round 0 is Algorithm 36.1: first-choice requests in token order, the
+ *    first C per expert accepted.  Rerouting then fills the slots left free,
+ *    in rounds r = 1, 2, ...: each path still without an expert takes its
+ *    token's next unused candidate whose expert was not full at the start of
+ *    the round (a token's paths in rank order take consecutive candidates);
+ *    the round's offers are accepted in token order while the expert has a
+ *    free slot (slot = rows already accepted by that expert).  A path that is
+ *    refused tries its token's next candidate in the next round; rounds stop
+ *    when no path makes an offer.  A path that finds no free expert adds 0.
+ *  - An expert's rows are its first-choice rows in token order, then each
+ *    round's rerouted rows in token order.
+ */
+
+/* cand[t*X+q] = the token's expert of rank k+q (-1 past E_r or for an
+ * invalid token), cand_w its weight as above.  logits [N, E] in double (the
+ * router scores); ids/w the router's records.  norm: renorm or full
+ * probability only. */
+int oracle_reroute_candidates(int64_t N, int E, int k, int X, int norm, const double* logits,
+                              const int32_t* ids, const uint8_t* invalid, int32_t* cand, double* cand_w) {
+    if (N < 0 || E < 1 || k < 1 || k > E || X < 1) return 1;
+    if (norm != NORM_RENORM && norm != NORM_FULLPROB) return 1;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t t = 0; t < N; ++t) {
+        const double* g = logits + t * E;
+        for (int q = 0; q < X; ++q) { cand[t * X + q] = -1; cand_w[t * X + q] = 0.0; }
+        if (invalid[t]) continue;
+        int* order = (int*)malloc(sizeof(int) * E);
+        double* p = (double*)malloc(sizeof(double) * E);
+        for (int e = 0; e < E; ++e) order[e] = e;
+        for (int a = 1; a < E; ++a) {
+            int cur = order[a], b = a - 1;
+            while (b >= 0 && (g[order[b]] < g[cur] || (g[order[b]] == g[cur] && order[b] > cur))) {
+                order[b + 1] = order[b];
+                --b;
+            }
+            order[b + 1] = cur;
+        }
+        double gmax = g[order[0]], z = 0.0;
+        for (int e = 0; e < E; ++e) { p[e] = exp(g[e] - gmax); z += p[e]; }
+        for (int e = 0; e < E; ++e) p[e] /= z;
+        double ssel = 0.0;
+        for (int j = 0; j < k; ++j)
+            if (ids[t * k + j] >= 0) ssel += p[ids[t * k + j]];
+        for (int q = 0; q < X && k + q < E; ++q) {
+            int e = order[k + q];
+            cand[t * X + q] = e;
+            cand_w[t * X + q] = norm == NORM_FULLPROB ? p[e] : p[e] / ssel;
+        }
+        free(order);
+        free(p);
+    }
+    return 0;
+}
+
+/* Token-order acceptance with rerouting of the rejected paths (rounds as
+ * above).  Outputs: slot [N,k] first-choice slot (-1 if rejected or not
+ * requested), as oracle_dispatch; rr_e [N,k] expert a rejected path was
+ * rerouted to (-1: none), rr_slot [N,k] its slot there, rr_q [N,k] the
+ * candidate index used; L [E] first-choice requested loads; acc [E] rows per
+ * expert (first-choice plus rerouted); counters
+ *  cnt[0] requested   cnt[1] paths given a slot (first choice or rerouted)
+ *  cnt[2] requested - cnt[1]   cnt[3] O = sum_e max(0, L_e - C)
+ *  cnt[4] tokens with >= 1 requested path left without an expert
+ *  cnt[5] tokens with >= 1 request and every requested path without an expert
+ *  cnt[6] max_e L_e   cnt[7] rerouted paths  cnt[8] rounds that made offers */
+int oracle_dispatch_reroute(int64_t N, int k, int E, int64_t C, int X, const int32_t* ids,
+                            const int32_t* cand, int32_t* slot, int32_t* rr_e, int32_t* rr_slot,
+                            int32_t* rr_q, int64_t* L, int64_t* acc, int64_t* cnt) {
+    if (N < 0 || k < 1 || E < 1 || C < 1 || X < 1) return 1;
+    int64_t base_cnt[7];
+    int rc = oracle_dispatch(N, k, E, C, ids, slot, L, acc, base_cnt);
+    if (rc) return rc;
+    for (int64_t i = 0; i < N * k; ++i) { rr_e[i] = -1; rr_slot[i] = -1; rr_q[i] = -1; }
+    int* next = (int*)calloc((size_t)(N > 0 ? N : 1), sizeof(int));     /* next unused candidate per token */
+    int64_t* full_at_start = (int64_t*)malloc(sizeof(int64_t) * E);
+    int32_t* offer = (int32_t*)malloc(sizeof(int32_t) * (size_t)(N * k > 0 ? N * k : 1));
+    int rounds = 0;
+    for (;;) {
+        for (int e = 0; e < E; ++e) full_at_start[e] = acc[e] >= C;
+        int64_t n_offers = 0;
+        for (int64_t t = 0; t < N; ++t) {
+            for (int j = 0; j < k; ++j) {
+                int64_t i = t * k + j;
+                offer[i] = -1;
+                if (ids[i] < 0 || slot[i] >= 0 || rr_e[i] >= 0) continue;
+                while (next[t] < X && cand[t * X + next[t]] >= 0 && full_at_start[cand[t * X + next[t]]]) ++next[t];
+                if (next[t] < X && cand[t * X + next[t]] >= 0) {
+                    offer[i] = next[t];
+                    ++next[t];
+                    ++n_offers;
+                }
+            }
+        }
+        if (n_offers == 0) break;
+        ++rounds;
+        for (int64_t t = 0; t < N; ++t) {
+            for (int j = 0; j < k; ++j) {
+                int64_t i = t * k + j;
+                if (offer[i] < 0) continue;
+                int e = cand[t * X + offer[i]];
+                if (acc[e] < C) {
+                    rr_e[i] = e;
+                    rr_slot[i] = (int32_t)acc[e];
+                    rr_q[i] = offer[i];
+                    acc[e] += 1;
+                }
+            }
+        }
+    }
+    for (int i = 0; i < 9; ++i) cnt[i] = 0;
+    for (int64_t t = 0; t < N; ++t) {
+        int req = 0, lost = 0;
+        for (int j = 0; j < k; ++j) {
+            int64_t i = t * k + j;
+            if (ids[i] < 0) continue;
+            ++req;
+            if (slot[i] < 0 && rr_e[i] < 0) ++lost;
+            if (rr_e[i] >= 0) cnt[7] += 1;
+        }
+        if (lost > 0) cnt[4] += 1;
+        if (req > 0 && lost == req) cnt[5] += 1;
+    }
+    for (int e = 0; e < E; ++e) {
+        cnt[0] += L[e];
+        cnt[1] += acc[e];
+        cnt[3] += L[e] > C ? L[e] - C : 0;
+        if (L[e] > cnt[6]) cnt[6] = L[e];
+    }
+    cnt[2] = cnt[0] - cnt[1];
+    cnt[8] = rounds;
+    free(next);
+    free(full_at_start);
+    free(offer);
+    return 0;
+}
+
+/*
  * One SwiGLU expert on a list of token rows (vegetog sec. 3):
  *   E(x) = [SiLU(x W_gate) (.) (x W_up)] W_down
  * with W_gate, W_up stored [d_f, d] and W_down stored [d, d_f].  When
