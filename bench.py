@@ -56,6 +56,8 @@ def kernels_per_step(w: si.Workload, sharded: bool) -> int:
     dispatch = 5 if sharded else 4      # hist, scan(s), assign, gather
     if w.accept_order == 1:
         dispatch += 3                   # placement, rank, numbering, per-token pass replace assign
+    if w.reject_policy == 2:
+        dispatch += 3 * w.reroute_depth + 2   # offer, scan, assign per round; final offsets; rows
     experts = 2 if w.dtype == si.DT_BF16 else 3   # fp32 layers zero Y in the router or a kernel
     if w.dtype != si.DT_BF16 and not sharded:
         experts = 2
@@ -123,13 +125,14 @@ def kernel_source_hash() -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def committed_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
-    None when the kernel source changed since the counters were taken."""
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary, or None when there is none for that workload or the kernel source
+    changed since the counters were taken."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
-        ent = t.get(kernel)
+        ent = t.get(f"{kernel}:{workload}")
         if ent and ent.get("source_sha256_16") == kernel_source_hash():
             return ent.get("bytes_per_launch")
     except (OSError, ValueError):
@@ -222,6 +225,10 @@ def oracle_sample(w: si.Workload, inp: dict, sample_tokens: int = 32):
 
 
 def run_reference(args):
+    """The CPU oracle on the host cores: each step is one bounded sample of the
+    workload (routing and dispatch of the whole batch, expert outputs of
+    --ref-sample tokens).  steps / warmup / ms_per_step describe those samples
+    as run; value is the whole-batch tokens/s extrapolated from them."""
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
@@ -233,9 +240,14 @@ def run_reference(args):
         if i >= args.warmup:
             steps.append(s)
     val = statistics.median([s["value"] for s in steps])
+    sample_ms = statistics.median([1000.0 * s["seconds"] for s in steps])
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * w.N / val,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sample_ms,
+        "step": (f"one bounded sample of the workload: routing and dispatch of all {w.N} tokens and the expert "
+                 f"outputs of {args.ref_sample} tokens"),
+        "extrapolated": True,
+        "extrapolated_ms_per_full_batch": 1000.0 * w.N / val,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w, args),
         "cpu_baseline": {k: steps[-1][k] for k in ("kind", "cores", "sample")} | {"value": val, "unit": "tokens/s"},
@@ -266,7 +278,7 @@ def config_of(w: si.Workload, args):
             "T": w.N, "d": w.d, "d_f": w.d_f, "E_r": w.E, "k": w.k,
             "norm": ["renorm", "fullprob", "wlr"][w.norm], "capacity_factor": w.c or None,
             "d_f_shared": w.d_f_shared, "seed": w.seed,
-            "overflow": {"reject": ["zero", "renormalise"][w.reject_policy],
+            "overflow": {"reject": ["zero", "renormalise", f"reroute (depth {w.reroute_depth})"][w.reject_policy],
                          "accept": ["token order", "largest weight"][w.accept_order]},
             "parallelism": (f"dp{args.gpus}: one routing group of {w.N} x {args.gpus} tokens, "
                             "per-expert request counts all-gathered once per step"
@@ -362,28 +374,23 @@ def run_gpu_soft(args):
     return 0
 
 
-def run_gpu(args):
-    import torch
-    import torch.distributed as dist
+PER_CONFIG = ("switch_top1_f32", "qwen3_skew_bf16", "deepseek_shared_bf16", "wdmoe_decode_bf16")
+EXPERT_TENSORS = ("W_g", "W_u", "W_d")
 
-    ws_n, rank, local = dist_env()
-    w = si.WORKLOADS[args.workload]
-    # host-side inputs (generated before any CUDA call; the oracle leg below
-    # uses the same buffers)
-    inp = si.inputs(w)
+
+def device_inputs(w: si.Workload, rank: int, ws_n: int):
+    """Host inputs of the layer's small tensors (x, router, bias, latencies,
+    shared expert) and the same seeded expert weights generated one expert at
+    a time straight into device tensors (a 22.6 GB layer never sits in host
+    memory whole).  Returns (host dict of the small tensors, device dict)."""
+    import torch
+
+    small = ("x", "W_r", "b_r", "lat", "Ws_g", "Ws_u", "Ws_d")
+    inp = si.inputs(w, names=small)
     if ws_n > 1:
         # rank r holds rows [r N, (r+1) N) of one routing group of N * ranks tokens
         inp["x"] = si.fill(w.seed, si.TID["x"], w.N * w.d, start=rank * w.N * w.d,
                            dtype=w.dt).reshape(w.N, w.d)
-    cpu_base = None
-    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
-        cpu_base = oracle_sample(w, inp, sample_tokens=args.ref_sample)
-
-    torch.cuda.set_device(local)
-    if ws_n > 1:
-        dist.init_process_group("nccl", init_method="env://",
-                                timeout=__import__("datetime").timedelta(seconds=120))
-    import sparse_mixture_experts_25_b200 as moe
 
     def dev(a):
         if a is None:
@@ -393,8 +400,28 @@ def run_gpu(args):
         return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
     d = {k: dev(v) for k, v in inp.items()}
+    tdt = torch.bfloat16 if w.dtype == si.DT_BF16 else torch.float32
+    for n in EXPERT_TENSORS:
+        t = torch.empty(si.shape(w, n), dtype=tdt, device="cuda")
+        for e in range(w.E):
+            t[e].copy_(dev(si.tensor(w, n, expert=e)))
+        d[n] = t
+    return inp, d
+
+
+def measure_forward(w: si.Workload, args, steps: int, warmup: int, cpu_base=None):
+    """Device-timed moe_forward steps (inputs resident in HBM), stage times,
+    the gate/up roofline and the end-to-end host-buffer leg for one workload;
+    returns the JSON line (without printing)."""
+    import torch
+    import torch.distributed as dist
+    import sparse_mixture_experts_25_b200 as moe
+
+    ws_n, rank, local = dist_env()
+    inp, d = device_inputs(w, rank, ws_n)
     p = moe.params(w.N, w.d, w.d_f, w.E, w.k, c=w.c, norm=w.norm, theta=w.theta, dtype=w.dtype,
-                   d_f_shared=w.d_f_shared, reject_policy=w.reject_policy, accept_order=w.accept_order)
+                   d_f_shared=w.d_f_shared, reject_policy=w.reject_policy, accept_order=w.accept_order,
+                   reroute_depth=w.reroute_depth)
     wsb = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
     Y = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
@@ -417,7 +444,7 @@ def run_gpu(args):
             moe.moe_forward(p, x_dev, d["W_r"], d["b_r"], d["lat"], d["W_g"], d["W_u"], d["W_d"],
                             d["Ws_g"], d["Ws_u"], d["Ws_d"], y_dev, wsb, stream)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step(d["x"], Y)
     torch.cuda.synchronize()
     status, stats = moe.moe_get_stats(p, wsb)
@@ -426,7 +453,7 @@ def run_gpu(args):
     accepted = int(stats["accepted"])
 
     # device-timed steps, inputs resident in HBM; stage events around each kernel group
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if ws_n > 1:
         dist.barrier()
@@ -449,7 +476,7 @@ def run_gpu(args):
     with ClockSampler(local) as clk:
         time.sleep(0.3)
         start.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             if flush is not None:
                 flush.fill_(i)   # evict the layer's inputs from L2; outside the step's events
             if graph is not None:
@@ -468,17 +495,18 @@ def run_gpu(args):
     if flush is None:
         ms_total = start.elapsed_time(end)
     else:  # sum of the steps' own spans (first stage event to last)
-        ms_total = float(sum(ev[i][0].elapsed_time(ev[i][4]) for i in range(args.steps)))
+        ms_total = float(sum(ev[i][0].elapsed_time(ev[i][4]) for i in range(steps)))
     ms_total = max_over_ranks(ms_total, device="cuda")
-    ms_step = ms_total / args.steps
+    ms_step = ms_total / steps
     if graph is not None:
         # stage times from eager steps (a replay records no stage events)
-        for i in range(args.steps):
+        for i in range(steps):
             moe.moe_set_stage_events(ev[i])
             step(d["x"], Y)
         moe.moe_set_stage_events([])
         torch.cuda.synchronize()
-    stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(4)] for i in range(args.steps)])
+        del graph
+    stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(4)] for i in range(steps)])
     gate_up_ms = float(stage_ms[:, 2].mean())
     down_ms = float(stage_ms[:, 3].mean())
 
@@ -504,13 +532,13 @@ def run_gpu(args):
     if ws_n > 1:
         dist.barrier()
     e_start.record(pipe.h2d)
-    for _ in range(args.steps):
+    for _ in range(steps):
         pipe.submit(x_host, y_host)
     pipe.compute.wait_stream(pipe.d2h)
     pipe.d2h.wait_stream(pipe.compute)
     e_end.record(pipe.d2h)
     pipe.synchronize()
-    e_ms = max_over_ranks(e_start.elapsed_time(e_end), device="cuda") / args.steps
+    e_ms = max_over_ranks(e_start.elapsed_time(e_end), device="cuda") / steps
 
     peaks, peak_src = load_peaks()
     timed_s = ms_total / 1000.0
@@ -535,13 +563,13 @@ def run_gpu(args):
         roof = {"kernel": "tc_grouped_kernel<SWIGLU> (gate/up GEMM + SwiGLU)",
                 "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / peaks["hbm_gbs"],
-                "traffic": committed_traffic("gate_up") if w.name == "mixtral_bf16" else None,
+                "traffic": committed_traffic("gate_up", w.name),
                 "peak_source": f"{peak_src} HBM copy"}
     else:
         roof = {"kernel": "tc_grouped_kernel<SWIGLU> (gate/up GEMM + SwiGLU)",
                 "bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                 "frac": achieved / peak_tf,
-                "traffic": committed_traffic("gate_up") if w.name == "mixtral_bf16" else None,
+                "traffic": committed_traffic("gate_up", w.name),
                 "peak_source": f"{peak_src} bf16 {peak_kind}"}
     gu_gbs = gu_bytes / (gate_up_ms * 1e-3) / 1e9
     roof.update({"flops_per_launch": gu_flops, "bytes_per_launch": gu_bytes, "avg_launch_ms": gate_up_ms,
@@ -553,8 +581,8 @@ def run_gpu(args):
         "value": ws_n * w.N / (ms_step * 1e-3),
         "unit": "tokens/s",
         "n_gpus": ws_n,
-        "steps": args.steps,
-        "warmup": args.warmup,
+        "steps": steps,
+        "warmup": warmup,
         "ms_per_step": ms_step,
         "higher_is_better": True,
         "scaling": "weak",
@@ -574,12 +602,55 @@ def run_gpu(args):
                 "how": "pinned x upload, moe_forward, pinned Y download per step; copies of "
                        "neighbouring steps overlap compute (HostPipeline, 2 device buffers)"
                        + ("; L2 not flushed between these steps" if flush is not None else "")},
-        "gpu_launches": kernels_per_step(w, sharded_group) * args.steps,
+        "gpu_launches": kernels_per_step(w, sharded_group) * steps,
         "clocks": clk.summary(),
         "routing": {k: stats[k] for k in ("accepted", "rejected", "near_tie", "L_max", "rho_max")},
     }
     if cpu_base is not None:
         line["cpu_baseline"] = {k: cpu_base[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    return line
+
+
+def per_config_summary(line: dict) -> dict:
+    """The keys of one workload's line that the headline's per_config object carries."""
+    keep = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config", "roofline", "stages_ms",
+            "e2e", "gpu_launches", "clocks", "routing")
+    out = {k: line[k] for k in keep}
+    out["roofline"] = {k: line["roofline"][k] for k in ("kernel", "bound", "achieved", "peak", "unit", "frac",
+                                                         "traffic", "peak_source", "avg_launch_ms", "hbm_frac")
+                       if k in line["roofline"]}
+    if "tensor_frac" in line["roofline"]:
+        out["roofline"]["tensor_frac"] = line["roofline"]["tensor_frac"]
+    out["e2e"] = {k: line["e2e"][k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step",
+                                              "ms_per_step")}
+    return out
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    ws_n, rank, local = dist_env()
+    w = si.WORKLOADS[args.workload]
+    cpu_base = None
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        # the oracle on a bounded sample of the same seeded inputs (host cores,
+        # before any CUDA call)
+        cpu_base = oracle_sample(w, si.inputs(w), sample_tokens=args.ref_sample)
+
+    torch.cuda.set_device(local)
+    if ws_n > 1:
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    line = measure_forward(w, args, args.steps, args.warmup, cpu_base=cpu_base)
+    if ws_n == 1 and args.per_config and args.workload == WORKLOAD and not args.graph:
+        # the other page-shaped layers, each measured the same way in this run
+        per = {}
+        for name in PER_CONFIG:
+            torch.cuda.empty_cache()
+            per[name] = per_config_summary(measure_forward(si.WORKLOADS[name], args, args.steps, args.warmup))
+        line["per_config"] = per
+        line["gpu_launches"] += sum(v["gpu_launches"] for v in per.values())
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_n > 1:
@@ -721,6 +792,10 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(si.WORKLOADS))
     ap.add_argument("--ref-sample", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-config", dest="per_config", action="store_true", default=True,
+                    help="with the default workload on one GPU, also measure the other page-shaped layers "
+                         "(per_config object; default on)")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of one step captured into a CUDA graph (one GPU)")
     ap.add_argument("--backward", action="store_true",

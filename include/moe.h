@@ -75,10 +75,33 @@ typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * ("LLM from scratch" ch. 36.3-36.4: the overflow policy is part of the
  * function; the worked example prints both outcomes). */
 typedef enum moe_reject_policy {
-    MOE_REJECT_ZERO = 0,   /* rejected path adds 0, the others keep their weights
-                              (Algorithm 36.1)                                     */
-    MOE_REJECT_RENORM = 1  /* the token's accepted paths are rescaled to sum to 1  */
+    MOE_REJECT_ZERO = 0,    /* rejected path adds 0, the others keep their weights
+                               (Algorithm 36.1)                                     */
+    MOE_REJECT_RENORM = 1,  /* the token's accepted paths are rescaled to sum to 1  */
+    MOE_REJECT_REROUTE = 2  /* a rejected path is rerouted to the token's next-ranked
+                               expert with a free slot (below); a path that finds
+                               none adds 0                                          */
 } moe_reject_policy;
+
+/* Rerouting (MOE_REJECT_REROUTE; "LLM from scratch" ch. 36.3: a rejected path
+ * may be rerouted, which calls another expert's parameters; vegetog "MoE
+ * token routing" sec. 5).  The pages leave the target open; this library
+ * reads it as follows.  A token's candidates are its experts of ranks k .. k
+ * + reroute_depth - 1 in the router's order (score descending, ties to the
+ * lower index), each weighted as the router's normalisation weights it
+ * against the token's chosen set S (p_e / sum_S p under MOE_NORM_RENORM, p_e
+ * under MOE_NORM_FULLPROB).  After Algorithm 36.1's token-order acceptance of
+ * the first choices, the rejected paths fill the slots left free in rounds:
+ * each path still without an expert takes its token's next unused candidate
+ * whose expert was not full at the start of the round (a token's paths in
+ * rank order take consecutive candidates), and the round's offers are
+ * accepted in token order while the expert has a free slot.  A refused path
+ * tries the next candidate in the next round.  An expert's rows are its
+ * first-choice rows in token order, then each round's rerouted rows in token
+ * order.  Requires MOE_NORM_RENORM or MOE_NORM_FULLPROB and
+ * MOE_ACCEPT_TOKEN, a single routing group (not moe_forward_begin/end,
+ * moe_dispatch_ranked or moe_dispatch_noalloc: MOE_ERR_UNSUPPORTED), and no
+ * backward pass (moe_backward returns MOE_ERR_UNSUPPORTED). */
 
 /* Which requests an over-full expert accepts ("LLM from scratch" ch. 36.3,
  * on how the acceptance rule makes outputs depend on the batch: first come
@@ -112,6 +135,9 @@ typedef struct moe_params {
     int32_t d_f_shared; /* hidden width of the always-on shared expert; 0 = none     */
     int32_t reject_policy; /* moe_reject_policy                                      */
     int32_t accept_order;  /* moe_accept_order                                       */
+    int32_t reroute_depth; /* MOE_REJECT_REROUTE: candidates per token, 1 ..
+                              min(E_r - k, 32 - k); ignored by the other policies   */
+    int32_t reserved;      /* 0                                                      */
 } moe_params;
 
 /* Routing statistics of the last moe_dispatch / moe_forward on a workspace
@@ -132,9 +158,14 @@ typedef struct moe_stats {
     double reject_rate;      /* rejected / requested                              */
     int32_t device_error;    /* nonzero: a bounded device wait timed out (bit 0)
                                 or a routing id was out of range (bit 1)           */
-    int32_t reserved;
-    int64_t padded_rows;     /* rows the routed expert GEMMs compute: each expert's
-                                accepted rows rounded up to the GEMM's row tile    */
+    int32_t rerouted;        /* MOE_REJECT_REROUTE: rejected paths served by a
+                                rerouted expert (included in accepted; rejected and
+                                tokens_affected / tokens_skipped then count the
+                                paths left without any expert); 0 otherwise       */
+    int64_t padded_rows;     /* rows the forward's routed expert GEMMs compute: fp32
+                                layers round each expert's accepted rows up to 64;
+                                bf16 layers run tiles of 256 tokens and round an
+                                expert's last tile up to 32 tokens               */
     double padding_ratio;    /* padded_rows / accepted (0 when nothing accepted)  */
     double aux_balance;      /* E_r sum_e f_e pbar_e ("LLM from scratch" ch. 36.4
                                 balance objective, value only): f_e = L_e / sum L,
@@ -160,6 +191,11 @@ typedef struct moe_ws_layout {
     size_t x_perm;     /* dtype [N k, d] gathered expert inputs                    */
     size_t h;          /* dtype [N k, d_f] expert hidden activations               */
     size_t h_shared;   /* dtype [N, d_f_shared]                                    */
+    size_t cand;       /* int32 [N, reroute_depth] rerouting candidates (rank k + q),
+                          -1 past E_r or for an invalid token (MOE_REJECT_REROUTE)  */
+    size_t cand_w;     /* fp32  [N, reroute_depth] their weights                    */
+    size_t rr_e;       /* int32 [N, k] expert a rejected path was rerouted to, -1   */
+    size_t rr_slot;    /* int32 [N, k] its slot in that expert's buffer, -1        */
     size_t scratch;    /* internal                                                 */
     size_t total;      /* bytes required                                           */
 } moe_ws_layout;
@@ -191,7 +227,10 @@ MOE_API moe_status moe_workspace_layout(const moe_params* p, moe_ws_layout* out)
  * Scores are accumulated in fp32.  A token with a non-finite score (or,
  * under WLR, a chosen expert whose latency is not a positive number) gets no
  * paths and is counted in the workspace counters (MOE_ERR_NONFINITE from
- * moe_get_stats).  ws: workspace of moe_workspace_size bytes.
+ * moe_get_stats).  ws: workspace of moe_workspace_size bytes.  Under
+ * MOE_REJECT_REROUTE the call also writes each token's rerouting candidates
+ * and their weights into ws (moe_ws_layout.cand, cand_w), which
+ * moe_dispatch on the same workspace reads.
  */
 MOE_API moe_status moe_route(const moe_params* p, const void* x, const void* W_r, const float* b_r,
                      const float* lat, int32_t* ids, float* w, float* margin, void* ws,
@@ -214,6 +253,12 @@ MOE_API moe_status moe_route(const moe_params* p, const void* x, const void* W_r
  *   x          [N, d] dtype, nullable; with x_perm [N k, d] dtype, gathers
  *              x_perm[r] = x[slot_token[r]] for every accepted row r
  * Statistics (L_e, accepted, O, ...) go to the workspace counters.
+ * MOE_REJECT_REROUTE: the rejected paths are then rerouted (see
+ * moe_reject_policy) to the candidates moe_route wrote into ws; slot keeps the
+ * first-choice slots (-1 for a rejected path), the rerouted paths' experts and
+ * slots go to ws (moe_ws_layout.rr_e, rr_slot), and the rows, offsets,
+ * slot_token and slot_w cover both (a rerouted row's weight is its
+ * candidate's weight).  The rounds are launched reroute_depth times.
  */
 MOE_API moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const float* w, int64_t C,
                         int32_t* slot, int32_t* offsets, int32_t* slot_token, float* slot_w,
@@ -361,11 +406,62 @@ MOE_API moe_status moe_set_stage_events(void* const* events, int n);
  * ("LLM from scratch" ch. 36.7: experts placed on different devices, token
  * rows sent to the device of their expert and the outputs sent back), where
  * x_perm's expert blocks are what each rank sends.  Token-order acceptance
- * only (MOE_ERR_UNSUPPORTED for MOE_ACCEPT_WEIGHT).
+ * only (MOE_ERR_UNSUPPORTED for MOE_ACCEPT_WEIGHT).  x may be NULL: the
+ * routing records are written and no rows are gathered (the fused exchange,
+ * moe_ep_dispatch, reads x itself).
  */
 MOE_API moe_status moe_dispatch_ranked(const moe_params* p, const int32_t* counts_all, int32_t rank,
                                        int32_t n_ranks, int64_t N_group, int64_t C, const void* x, void* ws,
                                        moe_stream_t stream);
+
+/*
+ * Expert parallelism ("LLM from scratch" ch. 36.7: experts on different
+ * devices; token rows go to their expert's device and the outputs come back).
+ * Rank r of n_ranks owns experts [r El, (r+1) El), El = E_r / n_ranks; the
+ * routing group's tokens are sharded over the ranks in token order.  Every
+ * rank derives the same plan from the all-gathered request counts
+ * counts_all [n_ranks][E_r] (moe_forward_begin): rank s's accepted requests for
+ * expert e are acc[s][e] = min(C, cum_s[e]) - min(C, cum_{s-1}[e]), cum_s the
+ * requests of ranks 0..s (token-order acceptance over the group).  An owner
+ * keeps its rows expert-major: owned expert j's rows from rank 0, then rank 1,
+ * ..., token order within a rank.
+ *
+ * moe_ep_plan: after moe_dispatch_ranked on this workspace.  Writes (device,
+ * caller-owned) local_offsets [El + 1] (the owned experts' rows in this rank's
+ * expert-major buffer), send_rows [n_ranks] and recv_rows [n_ranks] (the
+ * split sizes of an all-to-all of x_perm's expert blocks), and, when given,
+ * regroup / regroup_inv [rows received] (row i of the expert-major buffer is
+ * received row regroup[i] of a source-major all-to-all; regroup_inv is the
+ * inverse, for the return trip).  It also stores, in ws, where each of this
+ * rank's expert blocks lands in its owner's expert-major buffer.
+ *
+ * moe_ep_dispatch: the exchange fused into the dispatch.  Copies each of this
+ * rank's accepted rows of x [N, d] straight to its place in its owner's
+ * expert-major buffer: recv_bufs is a DEVICE array of n_ranks device pointers
+ * (rank r's buffer, of at least El C rows of d elements; another GPU's memory
+ * reachable by peer access, or this GPU's own).  The kernel ends with a
+ * system-scope fence; the caller orders the owners' expert computation
+ * (moe_expert_ffn on their buffer with local_offsets) after every rank's
+ * dispatch (a barrier across the ranks).
+ *
+ * moe_ep_combine: the return trip fused into the combine.  After the owners'
+ * outputs are complete (a barrier across the ranks), Y[t] += a_te out[row] for
+ * each of this rank's accepted rows, reading the output row from its owner's
+ * buffer out_bufs[owner] (DEVICE array of n_ranks pointers to fp32 [rows, d]
+ * expert-major outputs, peer or local).  Y is accumulated into (zero it
+ * first); the shared expert, if any, is the caller's (replicated per rank).
+ *
+ * Token-order acceptance, overflow policies 0 and 1; n_ranks <= 64 dividing
+ * E_r.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE,
+ * MOE_ERR_CUDA (moe_last_error).  All three are asynchronous on `stream`.
+ */
+MOE_API moe_status moe_ep_plan(const moe_params* p, const int32_t* counts_all, int32_t rank, int32_t n_ranks,
+                               int64_t C, int32_t* local_offsets, int32_t* send_rows, int32_t* recv_rows,
+                               int32_t* regroup, int32_t* regroup_inv, void* ws, moe_stream_t stream);
+MOE_API moe_status moe_ep_dispatch(const moe_params* p, int32_t n_ranks, const void* x, void* const* recv_bufs,
+                                   const void* ws, moe_stream_t stream);
+MOE_API moe_status moe_ep_combine(const moe_params* p, int32_t n_ranks, const float* const* out_bufs, float* Y,
+                                  const void* ws, moe_stream_t stream);
 
 /*
  * dst[i] = src[index[i]] for i < n_rows, rows of row_bytes bytes (a multiple

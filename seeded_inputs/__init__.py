@@ -167,8 +167,9 @@ class Workload:
     zipf_s: float = 0.0         # > 0: router bias b_e = 0.5 ln(Zipf(s) weight of rank e+1)
     latency: bool = False       # per-token per-expert latency t = t_up + t_comp + t_down
     seed: int = 25000
-    reject_policy: int = 0      # 0: rejected path adds 0; 1: accepted paths renormalised
+    reject_policy: int = 0      # 0: rejected path adds 0; 1: accepted paths renormalised; 2: rerouted
     accept_order: int = 0       # 0: token order; 1: largest routing weight first
+    reroute_depth: int = 0      # reject_policy 2: next-ranked experts a token may try
     soft_p: int = 0             # > 0: Soft MoE layer with soft_p slots per expert (Phi [E soft_p, d])
 
     @property

@@ -24,6 +24,7 @@ __all__ = [
     "moe_set_stage_events", "moe_selftest_wait_timeout", "moe_status_string", "moe_last_error",
     "expert_choice_params", "SoftParams", "soft_params", "moe_soft_workspace_size", "moe_soft_forward",
     "moe_dispatch_ranked", "moe_gather_rows", "workspace_x_perm",
+    "moe_ep_plan", "moe_ep_dispatch", "moe_ep_combine", "pointer_table",
     "moe_soft_check",
     "workspace_views", "HEADER",
 ]
@@ -32,7 +33,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_NONFINITE = 0, 1, 2, 3
 MOE_ERR_CUDA, MOE_ERR_WORKSPACE, MOE_ERR_TIMEOUT = 4, 5, 6
 MOE_NORM_RENORM, MOE_NORM_FULLPROB, MOE_NORM_WLR = 0, 1, 2
 MOE_F32, MOE_BF16 = 0, 1
-MOE_REJECT_ZERO, MOE_REJECT_RENORM = 0, 1
+MOE_REJECT_ZERO, MOE_REJECT_RENORM, MOE_REJECT_REROUTE = 0, 1, 2
 MOE_ACCEPT_TOKEN, MOE_ACCEPT_WEIGHT = 0, 1
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
@@ -52,7 +53,8 @@ class Params(ctypes.Structure):
                 ("E_r", ctypes.c_int32), ("k", ctypes.c_int32), ("c", ctypes.c_double),
                 ("norm", ctypes.c_int32), ("theta", ctypes.c_float), ("dtype", ctypes.c_int32),
                 ("d_f_shared", ctypes.c_int32), ("reject_policy", ctypes.c_int32),
-                ("accept_order", ctypes.c_int32)]
+                ("accept_order", ctypes.c_int32), ("reroute_depth", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class SoftParams(ctypes.Structure):
@@ -71,16 +73,16 @@ class Stats(ctypes.Structure):
         "C", "requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped",
         "nonfinite", "near_tie", "L_max", "L_p50", "L_p90", "L_p99")] + [
         ("rho_max", ctypes.c_double), ("reject_rate", ctypes.c_double),
-        ("device_error", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("device_error", ctypes.c_int32), ("rerouted", ctypes.c_int32),
         ("padded_rows", ctypes.c_int64), ("padding_ratio", ctypes.c_double),
         ("aux_balance", ctypes.c_double)]
 
     def as_dict(self):
-        return {n: getattr(self, n) for n, _ in self._fields_ if n != "reserved"}
+        return {n: getattr(self, n) for n, _ in self._fields_}
 
 
 _LAYOUT_FIELDS = ("ids", "w", "margin", "slot", "offsets", "L", "acc", "slot_token", "slot_w",
-                  "counters", "x_perm", "h", "h_shared", "scratch", "total")
+                  "counters", "x_perm", "h", "h_shared", "cand", "cand_w", "rr_e", "rr_slot", "scratch", "total")
 
 
 class WsLayout(ctypes.Structure):
@@ -125,6 +127,9 @@ def lib():
         L.moe_dispatch_ranked.argtypes = [pp, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
                                           ctypes.c_int64, _P, _P, _P]
         L.moe_gather_rows.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int64, _P, _P]
+        L.moe_ep_plan.argtypes = [pp, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_ep_dispatch.argtypes = [pp, ctypes.c_int32, _P, _P, _P, _P]
+        L.moe_ep_combine.argtypes = [pp, ctypes.c_int32, _P, _P, _P, _P]
         sp = ctypes.POINTER(SoftParams)
         L.moe_soft_workspace_size.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t)]
         L.moe_soft_forward.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P]
@@ -157,9 +162,12 @@ def declared_symbols():
 
 
 def params(N, d, d_f, E_r, k, c=0.0, norm=MOE_NORM_RENORM, theta=0.0, dtype=MOE_BF16,
-           d_f_shared=0, reject_policy=MOE_REJECT_ZERO, accept_order=MOE_ACCEPT_TOKEN) -> Params:
+           d_f_shared=0, reject_policy=MOE_REJECT_ZERO, accept_order=MOE_ACCEPT_TOKEN,
+           reroute_depth=0) -> Params:
+    """moe_params; reroute_depth is the number of next-ranked experts a token
+    may try under MOE_REJECT_REROUTE (ignored by the other policies)."""
     return Params(int(N), int(d), int(d_f), int(E_r), int(k), float(c), int(norm), float(theta),
-                  int(dtype), int(d_f_shared), int(reject_policy), int(accept_order))
+                  int(dtype), int(d_f_shared), int(reject_policy), int(accept_order), int(reroute_depth), 0)
 
 
 def expert_choice_params(N, d, d_f, E_r, C, dtype=MOE_BF16, d_f_shared=0) -> Params:
@@ -291,6 +299,37 @@ def moe_dispatch_ranked(p, counts_all, rank: int, n_ranks: int, N_group: int, C:
                                      int(C), _ptr(x), _ptr(ws), _stream(stream)), "moe_dispatch_ranked")
 
 
+def moe_ep_plan(p, counts_all, rank: int, n_ranks: int, C: int, local_offsets, send_rows, recv_rows, ws,
+                regroup=None, regroup_inv=None, stream=None):
+    """Plan of an expert-parallel step from the exchanged counts (device
+    tensors; see moe_ep_plan in include/moe.h)."""
+    _check(lib().moe_ep_plan(ctypes.byref(p), _ptr(counts_all), int(rank), int(n_ranks), int(C), _ptr(local_offsets),
+                             _ptr(send_rows), _ptr(recv_rows), _ptr(regroup), _ptr(regroup_inv), _ptr(ws),
+                             _stream(stream)), "moe_ep_plan")
+
+
+def pointer_table(buffers, device="cuda"):
+    """A device int64 tensor holding the device addresses of `buffers`
+    (tensors or integer addresses), for moe_ep_dispatch / moe_ep_combine."""
+    import torch
+    addrs = [b if isinstance(b, int) else b.data_ptr() for b in buffers]
+    return torch.tensor(addrs, dtype=torch.int64, device=device)
+
+
+def moe_ep_dispatch(p, n_ranks: int, x, recv_table, ws, stream=None):
+    """This rank's accepted rows of x into their owners' buffers (recv_table:
+    pointer_table of the ranks' receive buffers)."""
+    _check(lib().moe_ep_dispatch(ctypes.byref(p), int(n_ranks), _ptr(x), _ptr(recv_table), _ptr(ws),
+                                 _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_combine(p, n_ranks: int, out_table, Y, ws, stream=None):
+    """Y += weighted expert outputs read from their owners' output buffers
+    (out_table: pointer_table of the ranks' fp32 output buffers)."""
+    _check(lib().moe_ep_combine(ctypes.byref(p), int(n_ranks), _ptr(out_table), _ptr(Y), _ptr(ws),
+                                _stream(stream)), "moe_ep_combine")
+
+
 def moe_gather_rows(src, index, dst, stream=None):
     """dst[i] = src[index[i]] for the rows of index (device tensors)."""
     n = int(index.numel())
@@ -345,7 +384,7 @@ def workspace_views(p: Params, ws):
         nbytes = count * torch.empty((), dtype=dtype).element_size()
         return ws[L[name]:L[name] + nbytes].view(dtype).view(*shape)
 
-    return {
+    out = {
         "ids": view("ids", N * k, torch.int32, (N, k)),
         "w": view("w", N * k, torch.float32, (N, k)),
         "margin": view("margin", N, torch.float32, (N,)),
@@ -356,6 +395,15 @@ def workspace_views(p: Params, ws):
         "slot_token": view("slot_token", N * k, torch.int32, (N * k,)),
         "slot_w": view("slot_w", N * k, torch.float32, (N * k,)),
     }
+    if p.reject_policy == MOE_REJECT_REROUTE:
+        X = p.reroute_depth
+        out.update({
+            "cand": view("cand", N * X, torch.int32, (N, X)),
+            "cand_w": view("cand_w", N * X, torch.float32, (N, X)),
+            "rr_e": view("rr_e", N * k, torch.int32, (N, k)),
+            "rr_slot": view("rr_slot", N * k, torch.int32, (N, k)),
+        })
+    return out
 
 
 def workspace_x_perm(p: Params, ws):

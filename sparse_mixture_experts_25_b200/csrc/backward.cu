@@ -719,6 +719,7 @@ moe_status bwd_check(const moe_params* p) {
     const moe_status s = moe_workspace_size(p, &ws);  // the forward's parameter checks
     if (s != MOE_OK) return s;
     if (p->E_r > kMaxRouterExperts || p->k > kMaxK) return MOE_ERR_UNSUPPORTED;
+    if (p->reject_policy == MOE_REJECT_REROUTE) return MOE_ERR_UNSUPPORTED;  // rerouted weights: no backward
     if (p->N > (int64_t)65535 * 64) return MOE_ERR_UNSUPPORTED;  // grid rows of the router contractions
     // rows of the grouped weight-gradient GEMMs (E_r groups of d or d_f rows)
     if ((int64_t)p->E_r * std::max(p->d, p->d_f) >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;

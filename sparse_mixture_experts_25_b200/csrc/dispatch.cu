@@ -227,11 +227,13 @@ __device__ void token_pass(const int32_t* __restrict__ ids, const float* __restr
                            const int32_t* __restrict__ slot, float* __restrict__ slot_w,
                            unsigned long long* counters);
 
+// slots_only: write slot[] only (first round of rerouting: the rows and the
+// per-token statistics are written once every round is done)
 __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w,
                               int64_t N, int k, int E, int64_t C, int tile_tokens, int n_tiles,
                               const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets,
                               const int32_t* __restrict__ rank_base, int renorm_rejected,
-                              int store_request, int32_t* __restrict__ slot,
+                              int store_request, int slots_only, int32_t* __restrict__ slot,
                               int32_t* __restrict__ slot_token, float* __restrict__ slot_w,
                               unsigned long long* counters) {
     extern __shared__ int run[];
@@ -256,9 +258,11 @@ __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __re
         if (valid) {
             const int64_t sg = e >= 0 ? (rank_base ? (int64_t)rank_base[e] + s : (int64_t)s) : -1;
             if (e >= 0 && sg < C) {
-                const int64_t pos = (int64_t)offsets[e] + s;
-                slot_token[pos] = store_request ? (int32_t)i : (int32_t)(i / k);
-                slot_w[pos] = w[i];
+                if (!slots_only) {
+                    const int64_t pos = (int64_t)offsets[e] + s;
+                    slot_token[pos] = store_request ? (int32_t)i : (int32_t)(i / k);
+                    slot_w[pos] = w[i];
+                }
                 slot[i] = (int32_t)sg;
             } else {
                 slot[i] = -1;
@@ -266,7 +270,7 @@ __global__ void assign_kernel(const int32_t* __restrict__ ids, const float* __re
         }
     }
     __syncwarp();
-    if (store_request) return;  // placement pass of acceptance by weight: no statistics yet
+    if (store_request || slots_only) return;  // no statistics yet
     token_pass(ids, w, k, E, tb, te, offsets, rank_base, renorm_rejected, slot, slot_w, counters);
 }
 
@@ -443,6 +447,193 @@ __global__ void prio_token_kernel(const int32_t* __restrict__ ids, const float* 
     token_pass(ids, w, k, E, tb, te, offsets, nullptr, renorm_rejected, slot, slot_w, counters);
 }
 
+// --- rerouting of rejected paths (MOE_REJECT_REROUTE) ----------------------
+// After the first-choice acceptance (assign_kernel, slots only), each round:
+//   offer   per token (one thread each): every path still without an expert
+//           takes the token's next unused candidate whose expert was not full
+//           at the start of the round (acc[] as the previous round left it);
+//           offers are counted per tile and expert, like first choices;
+//   scan    per-tile bases of the offers, base[e] = acc[e], and acc[e] grows
+//           by the offers it can take (at most C in all);
+//   assign  one warp per tile walks the offers in token order: an offer for e
+//           gets slot base[e] + (earlier offers for e) and is accepted iff
+//           that is < C.
+// Then the final offsets (prefix of acc), and the rows of every served path
+// (first choices at offsets[e] + slot, rerouted ones at offsets[e] + rr_slot)
+// with the per-token statistics.
+__global__ void reroute_offer_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ slot,
+                                     const int32_t* __restrict__ cand, int X, const int32_t* __restrict__ acc,
+                                     int64_t C, int64_t N, int k, int E, int tile_tokens, int n_tiles,
+                                     const int32_t* __restrict__ rr_e, int32_t* __restrict__ rr_next,
+                                     int32_t* __restrict__ rr_offer, int32_t* __restrict__ hist) {
+    extern __shared__ int h[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    __syncthreads();
+    const int64_t t0 = (int64_t)blockIdx.x * tile_tokens;
+    const int64_t t1 = min64(N, t0 + tile_tokens);
+    for (int64_t t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
+        int q = rr_next[t];
+        for (int j = 0; j < k; ++j) {
+            const int64_t i = t * k + j;
+            int off = -1;
+            const int e0 = ids[i];
+            if (e0 >= 0 && e0 < E && slot[i] < 0 && rr_e[i] < 0) {
+                while (q < X) {
+                    const int c = cand[t * X + q];
+                    if (c < 0 || c >= E) {  // no further candidate
+                        q = X;
+                        break;
+                    }
+                    if (acc[c] < C) break;
+                    ++q;
+                }
+                if (q < X) {
+                    off = q;
+                    atomicAdd(&h[cand[t * X + q]], 1);
+                    ++q;
+                }
+            }
+            rr_offer[i] = off;
+        }
+        rr_next[t] = q;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)e * n_tiles + blockIdx.x] = h[e];
+}
+
+__global__ void reroute_scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int64_t C,
+                                    int32_t* __restrict__ acc, int32_t* __restrict__ base) {
+    __shared__ int sL[kMaxExperts];
+    tile_scan(hist, n_tiles, E, sL);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int a = acc[e];
+        base[e] = a;
+        acc[e] = (int)min64((int64_t)a + sL[e], C);
+    }
+}
+
+__global__ void reroute_assign_kernel(const int32_t* __restrict__ rr_offer, const int32_t* __restrict__ cand,
+                                      int X, int64_t N, int k, int E, int64_t C, int tile_tokens, int n_tiles,
+                                      const int32_t* __restrict__ hist, const int32_t* __restrict__ base,
+                                      int32_t* __restrict__ rr_e, int32_t* __restrict__ rr_slot,
+                                      int32_t* __restrict__ rr_q) {
+    extern __shared__ int run[];
+    const int lane = threadIdx.x;
+    const int tile = blockIdx.x;
+    for (int e = lane; e < E; e += 32) run[e] = hist[(int64_t)e * n_tiles + tile];
+    __syncwarp();
+    const int64_t tb = (int64_t)tile * tile_tokens;
+    const int64_t te = min64(N, tb + tile_tokens);
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int64_t b = tb * k; b < te * k; b += 32) {
+        const int64_t i = b + lane;
+        const bool valid = i < te * k;
+        const int q = valid ? rr_offer[i] : -1;
+        int e = q >= 0 ? cand[(i / k) * X + q] : -1;
+        if (e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(peers & lt_mask);
+        const int s = e >= 0 ? run[e] + rank : -1;
+        __syncwarp();
+        if (e >= 0 && lane == 31 - __clz(peers)) run[e] += __popc(peers);
+        __syncwarp();
+        if (e >= 0) {
+            const int64_t sg = (int64_t)base[e] + s;
+            if (sg < C) {
+                rr_e[i] = e;
+                rr_slot[i] = (int32_t)sg;
+                rr_q[i] = q;
+            }
+        }
+    }
+}
+
+// Offsets and M-tile prefix from the final rows per expert; accepted and
+// rejected counters (requested, O, the maximum load and C were written by the
+// first-choice scan).
+__global__ void reroute_final_scan_kernel(int E, int bm, const int32_t* __restrict__ acc,
+                                          int32_t* __restrict__ offsets, int32_t* __restrict__ mt_start,
+                                          unsigned long long* counters) {
+    __shared__ int warp_tot[33];
+    const int e = threadIdx.x;  // blockDim.x >= E
+    const int a = e < E ? acc[e] : 0;
+    const int mt = (a + bm - 1) / bm;
+    int tot_a, tot_mt;
+    const int ex_a = block_excl_scan(a, warp_tot, &tot_a);
+    const int ex_mt = block_excl_scan(mt, warp_tot, &tot_mt);
+    if (e < E) {
+        offsets[e] = ex_a;
+        mt_start[e] = ex_mt;
+    }
+    if (threadIdx.x == 0) {
+        offsets[E] = tot_a;
+        mt_start[E] = tot_mt;
+        const unsigned long long req = counters[CNT_REQUESTED];
+        counters[CNT_ACCEPTED] = (unsigned long long)tot_a;
+        counters[CNT_REJECTED] = req - (unsigned long long)tot_a;
+    }
+}
+
+// Rows of every served path and the per-token statistics (one warp per tile):
+// tokens with a requested path left without an expert, tokens with every
+// requested path left without one, and the rerouted paths.
+__global__ void reroute_rows_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w,
+                                    const int32_t* __restrict__ slot, const int32_t* __restrict__ rr_e,
+                                    const int32_t* __restrict__ rr_slot, const int32_t* __restrict__ rr_q,
+                                    const float* __restrict__ cand_w, int X, int64_t N, int k, int E,
+                                    int tile_tokens, const int32_t* __restrict__ offsets,
+                                    int32_t* __restrict__ slot_token, float* __restrict__ slot_w,
+                                    unsigned long long* counters) {
+    const int lane = threadIdx.x & 31;
+    const int64_t tb = (int64_t)blockIdx.x * tile_tokens;
+    const int64_t te = min64(N, tb + tile_tokens);
+    const int total = offsets[E];
+    for (int64_t i = tb * k + lane; i < te * k; i += 32) {
+        const int64_t t = i / k;
+        const int e0 = ids[i];
+        if (e0 < 0 || e0 >= E) continue;
+        int64_t row = -1;
+        float wr = 0.f;
+        if (slot[i] >= 0) {
+            row = (int64_t)offsets[e0] + slot[i];
+            wr = w[i];
+        } else if (rr_e[i] >= 0) {
+            row = (int64_t)offsets[rr_e[i]] + rr_slot[i];
+            wr = cand_w[t * X + rr_q[i]];
+        }
+        if (row >= 0 && row < total) {
+            slot_token[row] = (int32_t)t;
+            slot_w[row] = wr;
+        }
+    }
+    unsigned long long affected = 0, skipped = 0, moved = 0;
+    for (int64_t t = tb + lane; t < te; t += 32) {
+        int req = 0, lost = 0;
+        for (int j = 0; j < k; ++j) {
+            const int64_t i = t * k + j;
+            const int e0 = ids[i];
+            if (e0 < 0 || e0 >= E) continue;
+            ++req;
+            if (rr_e[i] >= 0) ++moved;
+            else if (slot[i] < 0) ++lost;
+        }
+        affected += lost > 0;
+        skipped += (req > 0 && lost == req);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        affected += __shfl_xor_sync(0xffffffffu, affected, o);
+        skipped += __shfl_xor_sync(0xffffffffu, skipped, o);
+        moved += __shfl_xor_sync(0xffffffffu, moved, o);
+    }
+    if (lane == 0) {
+        if (affected) atomicAdd(counters + CNT_AFFECTED, affected);
+        if (skipped) atomicAdd(counters + CNT_SKIPPED, skipped);
+        if (moved) atomicAdd(counters + CNT_REROUTED, moved);
+    }
+}
+
 __global__ void gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ x_perm,
                               const int32_t* __restrict__ slot_token,
                               const int32_t* __restrict__ offsets, int E, int row_vec) {
@@ -527,10 +718,48 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
                                     by_weight ? sc.all_offsets : nullptr, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int renorm = p.reject_policy == MOE_REJECT_RENORM;
-    if (!by_weight) {
+    const bool reroute = p.reject_policy == MOE_REJECT_REROUTE;
+    if (reroute) {
+        // first choices (slots only), then reroute_depth rounds of offers for
+        // the slots left free, then the final offsets, rows and statistics
+        const int X = p.reroute_depth;
+        *where = "assign";
+        assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens, n_tiles, sc.hist,
+                                                             offsets, nullptr, 0, 0, 1, slot, slot_token, slot_w,
+                                                             counters);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        *where = "reroute init";
+        const size_t nk = (size_t)p.N * k;
+        if ((e = cudaMemsetAsync(sc.rr_e, 0xff, nk * 4, st)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(sc.rr_slot, 0xff, nk * 4, st)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(sc.rr_q, 0xff, nk * 4, st)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(sc.rr_next, 0, (size_t)p.N * 4, st)) != cudaSuccess) return e;
+        for (int r = 0; r < X; ++r) {
+            *where = "reroute offer";
+            reroute_offer_kernel<<<n_tiles, 256, sizeof(int) * E, st>>>(ids, slot, sc.cand, X, acc, C, p.N, k, E,
+                                                                         sc.tile_tokens, n_tiles, sc.rr_e,
+                                                                         sc.rr_next, sc.rr_offer, sc.hist);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            *where = "reroute scan";
+            reroute_scan_kernel<<<1, 1024, 0, st>>>(sc.hist, n_tiles, E, C, acc, sc.base);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            *where = "reroute assign";
+            reroute_assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(sc.rr_offer, sc.cand, X, p.N, k, E, C,
+                                                                         sc.tile_tokens, n_tiles, sc.hist, sc.base,
+                                                                         sc.rr_e, sc.rr_slot, sc.rr_q);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        *where = "reroute offsets";
+        reroute_final_scan_kernel<<<1, 1024, 0, st>>>(E, bm, acc, offsets, sc.mt_start, counters);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        *where = "reroute rows";
+        reroute_rows_kernel<<<n_tiles, 32, 0, st>>>(ids, w, slot, sc.rr_e, sc.rr_slot, sc.rr_q, sc.cand_w, X, p.N,
+                                                    k, E, sc.tile_tokens, offsets, slot_token, slot_w, counters);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else if (!by_weight) {
         *where = "assign";
         assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
-                                                             n_tiles, sc.hist, offsets, nullptr, renorm, 0,
+                                                             n_tiles, sc.hist, offsets, nullptr, renorm, 0, 0,
                                                              slot, slot_token, slot_w, counters);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     } else {
@@ -539,7 +768,7 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
         // accepted requests numbered and scattered
         *where = "place";
         assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, INT64_MAX, sc.tile_tokens,
-                                                             n_tiles, sc.hist, sc.all_offsets, nullptr, 0, 1,
+                                                             n_tiles, sc.hist, sc.all_offsets, nullptr, 0, 1, 0,
                                                              slot, sc.seg_req, sc.seg_w, counters);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         *where = "select";
@@ -594,7 +823,7 @@ cudaError_t launch_dispatch_ranked(const moe_params& p, int64_t C, int bm, const
     *where = "assign";
     assign_kernel<<<sc.n_tiles, 32, sizeof(int) * E, st>>>(ids, w, p.N, k, E, C, sc.tile_tokens,
                                                             sc.n_tiles, sc.hist, offsets, sc.base,
-                                                            p.reject_policy == MOE_REJECT_RENORM, 0,
+                                                            p.reject_policy == MOE_REJECT_RENORM, 0, 0,
                                                             slot, slot_token, slot_w, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (x && x_perm) {

@@ -113,6 +113,7 @@ moe_status moe_dispatch_noalloc(const moe_params* p, const int32_t* ids, const f
     if (s != MOE_OK) return s;
     if (C < 1 || !offsets) return MOE_ERR_INVALID_ARG;
     if (p->accept_order == MOE_ACCEPT_WEIGHT) return MOE_ERR_UNSUPPORTED;  // token order only
+    if (p->reject_policy == MOE_REJECT_REROUTE) return MOE_ERR_UNSUPPORTED;  // needs the workspace's candidates
     if ((x != nullptr) != (x_perm != nullptr)) return MOE_ERR_INVALID_ARG;
     if (x && ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u)))
         return MOE_ERR_INVALID_ARG;

@@ -60,12 +60,20 @@ static bool layout(const moe_params& p, moe_ws_layout& L, int& n_tiles, int& til
     L.x_perm = take(Nk * (size_t)p.d * es);
     L.h = take(Nk * (size_t)p.d_f * es);
     L.h_shared = take((size_t)p.N * (size_t)(p.d_f_shared > 0 ? p.d_f_shared : 0) * es);
+    const bool rr = p.reject_policy == MOE_REJECT_REROUTE;
+    const size_t X = rr ? (size_t)p.reroute_depth : 0;
+    L.cand = take((size_t)p.N * X * 4);
+    L.cand_w = take((size_t)p.N * X * 4);
+    L.rr_e = take(rr ? Nk * 4 : 0);
+    L.rr_slot = take(rr ? Nk * 4 : 0);
     // scratch: per-tile histograms, M-tile prefix, earlier ranks' requests,
     // then (256-byte aligned) router scores, then the acceptance-by-weight
-    // arrays (all-request offsets, selected keys and counts, requests, weights)
+    // arrays (all-request offsets, selected keys and counts, requests, weights),
+    // the per-expert probability sums and (rerouting) the rounds' state
     L.scratch = take(align_up(E * (size_t)std::max(n_tiles, 1) * 4 + (E + 1) * 4 + E * 4, 256) +
                      align_up((size_t)p.N * E * 4, 256) + align_up((3 * E + 1) * 4, 256) + align_up(2 * Nk * 4, 256) +
-                     E * 4);
+                     align_up(E * 4, 256) + (rr ? align_up(2 * Nk * 4 + (size_t)p.N * 4, 256) : 0) +
+                     align_up(2 * E * 4, 256));
     L.total = off;
     return true;
 }
@@ -105,7 +113,23 @@ bool make_view(const moe_params& p, void* ws, WsView& v) {
         v.scratch.seg_req = reinterpret_cast<int32_t*>(pr);
         v.scratch.seg_w = reinterpret_cast<float*>(pr + Nk * 4);
         v.scratch.psum = reinterpret_cast<float*>(pr + align_up(2 * Nk * 4, 256));
+        char* rq = reinterpret_cast<char*>(v.scratch.psum) + align_up((size_t)p.E_r * 4, 256);
+        v.scratch.rr_q = reinterpret_cast<int32_t*>(rq);
+        v.scratch.rr_offer = v.scratch.rr_q + Nk;
+        v.scratch.rr_next = v.scratch.rr_offer + Nk;
+        const bool rr = p.reject_policy == MOE_REJECT_REROUTE;
+        char* ep = rq + (rr ? align_up(2 * Nk * 4 + (size_t)p.N * 4, 256) : 0);
+        v.scratch.ep_dest = reinterpret_cast<int32_t*>(ep);
+        v.scratch.ep_recv_base = v.scratch.ep_dest + p.E_r;
     }
+    v.cand = reinterpret_cast<int32_t*>(b + v.lay.cand);
+    v.cand_w = reinterpret_cast<float*>(b + v.lay.cand_w);
+    v.rr_e = reinterpret_cast<int32_t*>(b + v.lay.rr_e);
+    v.rr_slot = reinterpret_cast<int32_t*>(b + v.lay.rr_slot);
+    v.scratch.cand = v.cand;
+    v.scratch.cand_w = v.cand_w;
+    v.scratch.rr_e = v.rr_e;
+    v.scratch.rr_slot = v.rr_slot;
     v.scratch.n_tiles = n_tiles;
     v.scratch.tile_tokens = tile_tokens;
     return true;
@@ -154,8 +178,15 @@ moe_status check_params(const moe_params* p) {
     if (p->norm < MOE_NORM_RENORM || p->norm > MOE_NORM_WLR) return MOE_ERR_INVALID_ARG;
     if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (p->d_f_shared < 0) return MOE_ERR_INVALID_ARG;
-    if (p->reject_policy != MOE_REJECT_ZERO && p->reject_policy != MOE_REJECT_RENORM)
+    if (p->reject_policy != MOE_REJECT_ZERO && p->reject_policy != MOE_REJECT_RENORM &&
+        p->reject_policy != MOE_REJECT_REROUTE)
         return MOE_ERR_INVALID_ARG;
+    if (p->reject_policy == MOE_REJECT_REROUTE) {
+        // candidates are ranks k .. k + depth - 1, held one per lane of a warp
+        if (p->reroute_depth < 1 || p->reroute_depth > p->E_r - p->k || p->k + p->reroute_depth > kMaxK)
+            return MOE_ERR_INVALID_ARG;
+        if (p->norm == MOE_NORM_WLR || p->accept_order != MOE_ACCEPT_TOKEN) return MOE_ERR_UNSUPPORTED;
+    }
     if (p->accept_order != MOE_ACCEPT_TOKEN && p->accept_order != MOE_ACCEPT_WEIGHT)
         return MOE_ERR_INVALID_ARG;
     if (!(p->c == p->c) || p->c > 1e6) return MOE_ERR_INVALID_ARG;
@@ -275,7 +306,8 @@ moe_status moe_route(const moe_params* p, const void* x, const void* W_r, const 
     if (e == cudaSuccess) e = cudaMemsetAsync(v.scratch.psum, 0, sizeof(float) * p->E_r, st);
     if (e != cudaSuccess) return fail(e, "moe_route memset");
     return cuda_status(launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, ids,
-                                     w, margin, v.counters, nullptr, v.scratch.logits, v.scratch.psum, st),
+                                     w, margin, v.counters, nullptr, v.scratch.logits, v.scratch.psum, st,
+                                     v.cand, v.cand_w),
                        "moe_route router");
 }
 
@@ -302,6 +334,7 @@ moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const float* w,
     // dispatch-side counters start from zero; router counters are kept
     cudaError_t e = cudaMemsetAsync(v.counters + CNT_REQUESTED, 0, 6 * 8, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(v.counters + CNT_L_MAX, 0, 2 * 8, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(v.counters + CNT_REROUTED, 0, 8, st);
     if (e != cudaSuccess) return fail(e, "moe_dispatch memset");
     const int bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
     const char* where = "";
@@ -401,10 +434,10 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     const bool bf16 = p->dtype == MOE_BF16;
     cudaError_t e = launch_router(*p, x, W_r, b_r, p->norm == MOE_NORM_WLR ? lat : nullptr, v.ids,
                                   v.w, v.margin, v.counters, bf16 ? nullptr : Y, v.scratch.logits,
-                                  v.scratch.psum, st);
+                                  v.scratch.psum, st, v.cand, v.cand_w);
     if (e != cudaSuccess) return fail(e, "moe_forward router");
     if ((e0 = stage_mark(1, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
-    const int bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
+    const int bm = p->dtype == MOE_BF16 ? kSwapTok : kSimtBM;
     const char* where = "";
     e = launch_dispatch(*p, C, bm, v.ids, v.w, v.slot, v.offsets, v.L, v.acc, v.slot_token, v.slot_w,
                         x, v.x_perm, v.counters, v.scratch, st, &where);
@@ -416,12 +449,12 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     if ((e0 = stage_mark(2, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     int status = MOE_OK;
     if (p->dtype == MOE_BF16) {
-        e = launch_tc_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared,
-                              Y, v.counters, st, &status);
+        e = launch_swap_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, Y, v.counters,
+                                st, &status);
         if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_forward gate/up: tensor map encode" : "moe_forward gate/up (tcgen05)");
         if ((e0 = stage_mark(3, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
-        e = launch_tc_down(*p, DOWN_COMBINE, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
-                           v.slot_token, v.slot_w, Y, nullptr, v.counters, st, &status);
+        e = launch_swap_down(*p, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W, v.slot_token, v.slot_w, Y,
+                             v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_forward down: tensor map encode" : "moe_forward down+combine (tcgen05)");
     } else {
         e = launch_simt_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, st);
@@ -440,6 +473,7 @@ moe_status moe_forward_begin(const moe_params* p, const void* x, const void* W_r
     moe_status s = check_params(p);
     if (s != MOE_OK) return s;
     if (p->accept_order == MOE_ACCEPT_WEIGHT) return MOE_ERR_UNSUPPORTED;  // needs every rank's weights
+    if (p->reject_policy == MOE_REJECT_REROUTE) return MOE_ERR_UNSUPPORTED;  // single routing group only
     if (p->E_r > kMaxRouterExperts) return MOE_ERR_UNSUPPORTED;
     if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -474,11 +508,12 @@ moe_status moe_dispatch_ranked(const moe_params* p, const int32_t* counts_all, i
     moe_status s = check_params(p);
     if (s != MOE_OK) return s;
     if (p->accept_order == MOE_ACCEPT_WEIGHT) return MOE_ERR_UNSUPPORTED;  // needs every rank's weights
+    if (p->reject_policy == MOE_REJECT_REROUTE) return MOE_ERR_UNSUPPORTED;  // single routing group only
     if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     if (n_ranks < 1 || rank < 0 || rank >= n_ranks || !counts_all || C < 1 || N_group < p->N)
         return MOE_ERR_INVALID_ARG;
     if (p->N == 0) return MOE_OK;
-    if (!x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+    if (x && !aligned16(x)) return MOE_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     WsView v;
     make_view(*p, ws, v);
@@ -489,7 +524,8 @@ moe_status moe_dispatch_ranked(const moe_params* p, const int32_t* counts_all, i
     const int bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
     const char* where = "";
     e = launch_dispatch_ranked(*p, C, bm, counts_all, rank, n_ranks, N_group, v.ids, v.w, v.slot, v.offsets, v.L,
-                               v.acc, v.slot_token, v.slot_w, x, v.x_perm, v.counters, v.scratch, st, &where);
+                               v.acc, v.slot_token, v.slot_w, x, x ? v.x_perm : nullptr, v.counters, v.scratch, st,
+                               &where);
     if (e != cudaSuccess) {
         char buf[96];
         snprintf(buf, sizeof(buf), "moe_dispatch_ranked %s", where);
@@ -517,6 +553,7 @@ moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32
     moe_status s = check_params(p);
     if (s != MOE_OK) return s;
     if (p->accept_order == MOE_ACCEPT_WEIGHT) return MOE_ERR_UNSUPPORTED;  // needs every rank's weights
+    if (p->reject_policy == MOE_REJECT_REROUTE) return MOE_ERR_UNSUPPORTED;  // single routing group only
     if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     if (n_ranks < 1 || rank < 0 || rank >= n_ranks || !counts_all || C < 1 || N_group < p->N)
         return MOE_ERR_INVALID_ARG;
@@ -535,7 +572,7 @@ moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32
     if (e == cudaSuccess) e = cudaMemsetAsync(v.counters + CNT_L_MAX, 0, 2 * 8, st);
     if (e != cudaSuccess) return fail(e, "moe_forward_end memset");
     const bool bf16 = p->dtype == MOE_BF16;
-    const int bm = bf16 ? tc_tile_rows(*p) : kSimtBM;
+    const int bm = bf16 ? kSwapTok : kSimtBM;
     const char* where = "";
     e = launch_dispatch_ranked(*p, C, bm, counts_all, rank, n_ranks, N_group, v.ids, v.w, v.slot,
                                v.offsets, v.L, v.acc, v.slot_token, v.slot_w, x, v.x_perm,
@@ -549,12 +586,12 @@ moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32
     if ((e = stage_mark(2, st)) != cudaSuccess) return fail(e, "moe_forward_end stage event");
     int status = MOE_OK;
     if (bf16) {
-        e = launch_tc_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, Y,
-                              v.counters, st, &status);
+        e = launch_swap_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, Y, v.counters,
+                                st, &status);
         if (e != cudaSuccess) return fail(e, "moe_forward_end gate/up (tcgen05)");
         if ((e = stage_mark(3, st)) != cudaSuccess) return fail(e, "moe_forward_end stage event");
-        e = launch_tc_down(*p, DOWN_COMBINE, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
-                           v.slot_token, v.slot_w, Y, nullptr, v.counters, st, &status);
+        e = launch_swap_down(*p, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W, v.slot_token, v.slot_w, Y,
+                             v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, "moe_forward_end down+combine (tcgen05)");
     } else {
         e = launch_zero_f32(Y, p->N * (int64_t)p->d, st);
@@ -616,6 +653,7 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
     out->near_tie = (int64_t)cnt[CNT_NEAR_TIE];
     out->L_max = (int64_t)cnt[CNT_L_MAX];
     out->device_error = (int32_t)cnt[CNT_DEVICE_ERROR];
+    out->rerouted = (int32_t)cnt[CNT_REROUTED];
     if (p->N > 0) {
         std::vector<int32_t> srt(L);
         std::sort(srt.begin(), srt.end());
@@ -630,12 +668,17 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
         const double n_group = cnt[CNT_N_GROUP] ? (double)cnt[CNT_N_GROUP] : (double)p->N;
         out->rho_max = (double)out->L_max * (double)p->E_r / (n_group * (double)p->k);
         out->reject_rate = out->requested ? (double)out->rejected / (double)out->requested : 0.0;
-        // rows the routed GEMMs compute: accepted rows per expert rounded up
-        // to the row tile of the kernels that run them
-        const int64_t bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
+        // rows the forward's routed GEMMs compute: fp32 layers round each
+        // expert's accepted rows up to the 64-row tile; bf16 layers run full
+        // token tiles of kSwapTok plus a last tile rounded up to kSwapGran
         int64_t padded = 0, accepted = 0;
         for (int32_t a : acc) {
-            padded += (a + bm - 1) / bm * bm;
+            if (p->dtype == MOE_BF16) {
+                const int64_t full = a / kSwapTok * kSwapTok, tail = a - full;
+                padded += full + (tail + kSwapGran - 1) / kSwapGran * kSwapGran;
+            } else {
+                padded += (a + kSimtBM - 1) / kSimtBM * kSimtBM;
+            }
             accepted += a;
         }
         out->padded_rows = padded;

@@ -33,6 +33,7 @@ enum Counter {
     CNT_C = 9,
     CNT_DEVICE_ERROR = 10,  // bit flags, see DevErr
     CNT_N_GROUP = 11,       // tokens of the whole routing group (sharded runs; 0 = N)
+    CNT_REROUTED = 12,      // rejected paths served by a rerouted expert
     CNT_COUNT = 16
 };
 
@@ -52,6 +53,19 @@ struct Scratch {
     int32_t* seg_req;     // [N k] requests grouped by expert, token order (acceptance by weight)
     float* seg_w;         // [N k] their routing weights
     float* psum;          // [E] sum over tokens of the full-softmax probabilities
+    // rerouting (MOE_REJECT_REROUTE): candidates and results (workspace
+    // records), then the rounds' state
+    const int32_t* cand;  // [N, X] candidate experts (rank k + q), -1 none
+    const float* cand_w;  // [N, X] their weights
+    int32_t* rr_e;        // [N k] expert a rejected path was rerouted to, -1
+    int32_t* rr_slot;     // [N k] its slot
+    int32_t* rr_q;        // [N k] candidate index used
+    int32_t* rr_offer;    // [N k] candidate index offered in the current round, -1
+    int32_t* rr_next;     // [N] next unused candidate of each token
+    // expert parallelism: position of this rank's first row of each expert in
+    // its owner's buffer, and (receiving side) source-major row starts [R][El]
+    int32_t* ep_dest;     // [E]
+    int32_t* ep_recv_base;  // [E]
     int n_tiles;          // dispatch tiles
     int tile_tokens;      // tokens per dispatch tile
 };
@@ -72,6 +86,10 @@ struct WsView {
     void* x_perm;
     void* h;
     void* h_shared;
+    int32_t* cand;
+    float* cand_w;
+    int32_t* rr_e;
+    int32_t* rr_slot;
     Scratch scratch;
 };
 
@@ -87,10 +105,11 @@ bool make_view(const moe_params& p, void* ws, WsView& v);
 // router.cu
 // logits: [N, E_r] fp32 scratch for the tensor-core score path (may be null)
 // psum: [E_r] fp32 sums of the full-softmax probabilities, accumulated (may be null)
+// cand / cand_w (MOE_REJECT_REROUTE, nullable): [N, reroute_depth] rerouting candidates
 cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, const float* b_r,
                           const float* lat, int32_t* ids, float* w, float* margin,
                           unsigned long long* counters, float* Y_zero, float* logits, float* psum,
-                          cudaStream_t st);
+                          cudaStream_t st, int32_t* cand = nullptr, float* cand_w = nullptr);
 // dispatch.cu
 cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_t* ids,
                             const float* w, int32_t* slot, int32_t* offsets, int32_t* L,
@@ -140,12 +159,37 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
 // rows of one output tile of the tcgen05 grouped GEMMs for these params
 // (256 when CTA pairs are used, else 128): the dispatch's M-tile prefix unit
 int tc_tile_rows(const moe_params& p);
+// The forward's routed GEMMs of bf16 layers: weight-stationary tiles on CTA
+// pairs (expert weight rows on the MMA's M side, up to kSwapTok tokens on its
+// N side); mt_start is the prefix of ceil(rows / kSwapTok) per expert.
+constexpr int kSwapTok = 256;
+constexpr int kSwapGran = 32;   // a tile's tokens are rounded up to a multiple of this
+cudaError_t launch_swap_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
+                                const int32_t* offsets, const int32_t* mt_start, const ExpertWeights& W, void* h,
+                                void* h_shared, float* Y_zero, unsigned long long* counters, cudaStream_t st,
+                                int* status);
+cudaError_t launch_swap_down(const moe_params& p, int64_t C, const void* h, const void* h_shared,
+                             const int32_t* offsets, const int32_t* mt_start, const ExpertWeights& W,
+                             const int32_t* slot_token, const float* slot_w, float* Y, unsigned long long* counters,
+                             cudaStream_t st, int* status);
 // out[M, Nc] (fp32, row-major) = A[M, K] B[Nc, K]^T, bf16 operands with rows
 // of K elements (K % 8 == 0, 16-byte aligned bases), tcgen05 tiles of 128 x 256
 cudaError_t launch_tc_dense(int64_t M, int64_t Nc, int64_t K, const void* A, const void* B, float* out,
                             unsigned long long* counters, cudaStream_t st, int* status);
 cudaError_t launch_gather_rows(const void* src, const int32_t* index, int64_t n_rows, int64_t row_bytes, void* dst,
                                cudaStream_t st);
+// expert_parallel.cu: plan of an expert-parallel step from the exchanged
+// request counts, and the exchange fused into the dispatch and the combine
+constexpr int kMaxEpRanks = 64;
+cudaError_t launch_ep_plan(const moe_params& p, const int32_t* counts_all, int R, int rank, int64_t C,
+                           int32_t* dest_base, int32_t* local_offsets, int32_t* send_rows, int32_t* recv_rows,
+                           int32_t* recv_base, int32_t* regroup, int32_t* regroup_inv, cudaStream_t st);
+cudaError_t launch_ep_dispatch(const moe_params& p, int R, const void* x, const int32_t* offsets,
+                               const int32_t* slot_token, const int32_t* dest_base, void* const* recv_bufs,
+                               cudaStream_t st);
+cudaError_t launch_ep_combine(const moe_params& p, int R, const int32_t* offsets, const int32_t* slot_token,
+                              const float* slot_w, const int32_t* dest_base, const float* const* out_bufs, float* Y,
+                              cudaStream_t st);
 cudaError_t launch_wait_selftest(unsigned long long* counters, unsigned long long limit_ns, cudaStream_t st);
 // router scores G = x W_r^T (bf16 in, fp32 out [N, E_r]) on the tensor cores
 cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,

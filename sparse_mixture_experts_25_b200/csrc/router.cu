@@ -37,8 +37,11 @@ struct RouterArgs {
     unsigned long long* counters;
     float* Y_zero;
     float* psum;  // [E] sum over tokens of the full-softmax probabilities (nullable)
+    int32_t* cand;  // [N, X] rerouting candidates: experts of rank k .. k+X-1 (X > 0 only)
+    float* cand_w;  // [N, X] their weights under the layer's normalisation
     int64_t N;
     int d, E, k, norm;
+    int X;          // rerouting candidates per token (0: none)
     float theta;
 };
 
@@ -94,7 +97,10 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int64_t t, int
     unsigned taken = 0;
     int my_e = -1;
     float my_g = 0.f, next_g = -INFINITY;
-    const int rounds = k < E ? k + 1 : k;
+    // ranks 0..k-1 are the chosen experts; rank k gives the margin; ranks
+    // k..k+X-1 are the rerouting candidates (lane r holds rank r)
+    const int want = k + (a.X > 1 ? a.X : 1);
+    const int rounds = want < E ? want : E;
     if (!__any_sync(0xffffffffu, bad)) {
         for (int r = 0; r < rounds; ++r) {
             float bv = -INFINITY;
@@ -116,15 +122,12 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int64_t t, int
                     be = oe;
                 }
             }
-            if (r < k) {
-                if (lane == r) {
-                    my_e = be;
-                    my_g = bv;
-                }
-                if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            } else {
-                next_g = bv;
+            if (lane == r) {
+                my_e = be;
+                my_g = bv;
             }
+            if (r == k) next_g = bv;
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
         }
     }
     float z = 0.f;
@@ -147,10 +150,15 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int64_t t, int
         lat_bad = !(te > 0.f);  // NaN or non-positive latency
     }
     bad = __any_sync(0xffffffffu, bad || lat_bad);
+    const bool is_cand = lane >= k && lane < k + a.X;
     if (bad) {
         if (pick) {
             a.ids[t * k + lane] = -1;
             a.w[t * k + lane] = 0.f;
+        }
+        if (is_cand) {
+            a.cand[t * a.X + (lane - k)] = -1;
+            a.cand_w[t * a.X + (lane - k)] = 0.f;
         }
         if (lane == 0) {
             if (a.margin) a.margin[t] = NAN;
@@ -166,10 +174,12 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int64_t t, int
             if (e < E) atomicAdd(&ps[e], ev[i] * iz);
         }
     }
+    float sel_sum = 1.f;  // sum of the chosen experts' exp(g - m) (renormalisation)
     if (a.norm == MOE_NORM_FULLPROB) {
         wv = ex / z;
     } else if (a.norm == MOE_NORM_RENORM) {
-        wv = ex / warp_sum(ex);
+        sel_sum = warp_sum(ex);
+        wv = ex / sel_sum;
     } else {
         const float wlr = (ex / z) / te;  // p_e / t_e (0 when t_e = inf)
         for (;;) {
@@ -203,6 +213,14 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int64_t t, int
     if (pick) {
         a.ids[t * k + lane] = active ? my_e : -1;
         a.w[t * k + lane] = wv;
+    }
+    if (is_cand) {
+        // the expert of rank `lane`, weighted against the chosen set as the
+        // chosen experts are (full probability: p; renormalised: p / sum_S p)
+        const bool have = lane < E;
+        const float exc = have ? expf(my_g - m) : 0.f;
+        a.cand[t * a.X + (lane - k)] = have ? my_e : -1;
+        a.cand_w[t * a.X + (lane - k)] = have ? (a.norm == MOE_NORM_FULLPROB ? exc / z : exc / sel_sum) : 0.f;
     }
     const float kth = __shfl_sync(0xffffffffu, my_g, k - 1);
     const float mg = k < E ? kth - next_g : INFINITY;
@@ -492,7 +510,7 @@ cudaError_t launch_typed(const RouterArgs& a, cudaStream_t st) {
 cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, const float* b_r,
                           const float* lat, int32_t* ids, float* w, float* margin,
                           unsigned long long* counters, float* Y_zero, float* logits, float* psum,
-                          cudaStream_t st) {
+                          cudaStream_t st, int32_t* cand, float* cand_w) {
     RouterArgs a;
     a.x = x;
     a.W_r = W_r;
@@ -510,6 +528,9 @@ cudaError_t launch_router(const moe_params& p, const void* x, const void* W_r, c
     a.k = p.k;
     a.norm = p.norm;
     a.theta = p.theta;
+    a.X = (p.reject_policy == MOE_REJECT_REROUTE && cand && cand_w) ? p.reroute_depth : 0;
+    a.cand = cand;
+    a.cand_w = cand_w;
     if (p.N == 0) return cudaSuccess;
     const unsigned warps_blocks = (unsigned)((p.N + 7) / 8);
     const bool bf16 = p.dtype == MOE_BF16;

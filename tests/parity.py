@@ -49,7 +49,7 @@ def params_of(w: si.Workload):
     import sparse_mixture_experts_25_b200 as moe
     return moe.params(w.N, w.d, w.d_f, w.E, w.k, c=w.c, norm=w.norm, theta=w.theta,
                       dtype=w.dtype, d_f_shared=w.d_f_shared, reject_policy=w.reject_policy,
-                      accept_order=w.accept_order)
+                      accept_order=w.accept_order, reroute_depth=w.reroute_depth)
 
 
 def gpu_forward(w: si.Workload, inp: dict, dev: dict | None = None):
@@ -86,11 +86,58 @@ def check_routing(w: si.Workload, inp: dict, rec: dict):
     return r, near
 
 
+def check_candidates(w: si.Workload, r: dict, rec: dict):
+    """Rerouting candidates (ranks k .. k+X-1) against the oracle's, on the
+    tokens whose scores around those ranks are not near-ties (every gap
+    between consecutive ranks k-1 .. k+X at least 1e-5); weights within the
+    routing-weight bound.  Returns the mask of compared tokens."""
+    X = w.reroute_depth
+    cand, cw = oracle.reroute_candidates(r["logits"], r["ids"], r["invalid"], w.k, X, w.norm)
+    g = -np.sort(-r["logits"], axis=1)
+    hi = min(w.E - 1, w.k + X)
+    gaps = g[:, w.k - 1:hi] - g[:, w.k:hi + 1]
+    clear = ~r["invalid"] & (gaps.min(axis=1) >= NEAR if gaps.shape[1] else True) & (r["margin"] >= NEAR)
+    np.testing.assert_array_equal(rec["cand"][clear], cand[clear])
+    np.testing.assert_allclose(rec["cand_w"][clear], cw[clear], rtol=3e-5, atol=3e-5)
+    assert (rec["cand"][r["invalid"]] == -1).all()
+    return clear
+
+
+def check_dispatch_reroute(w: si.Workload, rec: dict, stats: dict):
+    """Rerouting dispatch: the oracle's rounds on the GPU's own ids and
+    candidates; first-choice slots, rerouted experts and slots, rows per
+    expert, offsets, row records and statistics bit for bit."""
+    C = oracle.capacity(w.c, w.N, w.k, w.E)
+    d = oracle.dispatch_reroute(rec["ids"], rec["cand"], E=w.E, C=C)
+    np.testing.assert_array_equal(rec["slot"], d["slot"])
+    np.testing.assert_array_equal(rec["rr_e"], d["rr_e"])
+    np.testing.assert_array_equal(rec["rr_slot"], d["rr_slot"])
+    np.testing.assert_array_equal(rec["L"], d["L"])
+    np.testing.assert_array_equal(rec["acc"], d["acc"])
+    offs = np.concatenate([[0], np.cumsum(d["acc"])])
+    np.testing.assert_array_equal(rec["offsets"], offs)
+    ids2, w2, slot2 = oracle.served_records(rec["ids"], rec["w"].astype(np.float64), d["slot"], d["rr_e"],
+                                            d["rr_slot"], d["rr_q"], rec["cand_w"].astype(np.float64))
+    t_idx, j_idx = np.nonzero(slot2 >= 0)
+    pos = offs[ids2[t_idx, j_idx]] + slot2[t_idx, j_idx]
+    assert pos.size == offs[-1] and np.unique(pos).size == pos.size
+    np.testing.assert_array_equal(rec["slot_token"][pos], t_idx)
+    np.testing.assert_array_equal(rec["slot_w"][pos], w2[t_idx, j_idx].astype(np.float32))
+    s = d["stats"]
+    for key in ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max",
+                "rerouted"):
+        assert stats[key] == s[key], (key, stats[key], s[key])
+    assert stats["C"] == C
+    return d
+
+
 def check_dispatch(w: si.Workload, rec: dict, stats: dict):
     """Oracle dispatch on the GPU's own ids (and, for acceptance by weight, on
     its own fp32 weights, so both sides order the requests by the same
     numbers): slots, loads, offsets, records and statistics must match bit
     for bit."""
+    if w.reject_policy == 2:
+        return check_dispatch_reroute(w, rec, stats)
     C = oracle.capacity(w.c, w.N, w.k, w.E)
     if w.accept_order == 1:
         d = oracle.dispatch_priority(rec["ids"], rec["w"].astype(np.float64), E=w.E, C=C)
@@ -114,11 +161,13 @@ def check_dispatch(w: si.Workload, rec: dict, stats: dict):
     for key in ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max"):
         assert stats[key] == s[key], (key, stats[key], s[key])
     assert stats["C"] == C
-    # tile padding of the routed GEMMs: each expert's accepted rows rounded up
-    # to the row tile (64 rows for fp32 layers; 128, or 256 on CTA pairs when
-    # experts average >= 768 rows, for bf16 layers)
-    bm = 64 if w.dtype == si.DT_F32 else (256 if w.N * w.k >= 768 * w.E else 128)
-    padded = int(sum(-(-int(a) // bm) * bm for a in d["acc"]))
+    # tile padding of the forward's routed GEMMs: fp32 layers round each
+    # expert's accepted rows up to 64; bf16 layers run 256-token tiles and a
+    # last tile rounded up to 32 tokens
+    if w.dtype == si.DT_F32:
+        padded = int(sum(-(-int(a) // 64) * 64 for a in d["acc"]))
+    else:
+        padded = int(sum(int(a) // 256 * 256 + -(-(int(a) % 256) // 32) * 32 for a in d["acc"]))
     assert stats["padded_rows"] == padded
     assert stats["padding_ratio"] == pytest.approx(padded / s["accepted"] if s["accepted"] else 0.0)
     if w.N:
@@ -183,11 +232,19 @@ def check_rows(w: si.Workload, inp: dict, rec: dict, Y: np.ndarray, tokens=None)
     if tokens is None:
         tokens = np.arange(w.N)
     Ws = (inp.get("Ws_g"), inp.get("Ws_u"), inp.get("Ws_d")) if w.d_f_shared else None
-    wc = oracle.reject_weights(rec["ids"], rec["w"].astype(np.float64), rec["slot"], w.reject_policy)
-    ref = oracle.forward_rows(inp["x"], rec["ids"], wc, rec["slot"], tokens,
+    if w.reject_policy == 2:
+        # every served path: first choices and rerouted ones, from the GPU's records
+        C = oracle.capacity(w.c, w.N, w.k, w.E)
+        d = oracle.dispatch_reroute(rec["ids"], rec["cand"], E=w.E, C=C)
+        ids2, wc, slot2 = oracle.served_records(rec["ids"], rec["w"].astype(np.float64), d["slot"], d["rr_e"],
+                                                d["rr_slot"], d["rr_q"], rec["cand_w"].astype(np.float64))
+    else:
+        ids2, slot2 = rec["ids"], rec["slot"]
+        wc = oracle.reject_weights(rec["ids"], rec["w"].astype(np.float64), rec["slot"], w.reject_policy)
+    ref = oracle.forward_rows(inp["x"], ids2, wc, slot2, tokens,
                               inp["W_g"], inp["W_u"], inp["W_d"], Ws=Ws)
     err, row = assert_rows_close(Y[tokens], ref, TOL[w.dtype])
-    dropped = [i for i, t in enumerate(tokens) if not w.d_f_shared and (rec["slot"][t] < 0).all()]
+    dropped = [i for i, t in enumerate(tokens) if not w.d_f_shared and (slot2[t] < 0).all()]
     for i in dropped:
         assert (Y[tokens[i]] == 0).all()
     return err, row

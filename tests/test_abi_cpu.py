@@ -21,9 +21,9 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_struct_sizes_match_the_header_layout():
-    assert ctypes.sizeof(moe.Params) == 56
+    assert ctypes.sizeof(moe.Params) == 64
     assert ctypes.sizeof(moe.Stats) == 13 * 8 + 2 * 8 + 2 * 4 + 8 + 8 + 8
-    assert ctypes.sizeof(moe.WsLayout) == 15 * 8
+    assert ctypes.sizeof(moe.WsLayout) == 19 * 8
 
 
 @pytest.mark.parametrize("c,N,k,E", [
@@ -68,8 +68,14 @@ def test_workspace_layout_regions():
     (dict(d_f=36), moe.MOE_ERR_UNSUPPORTED),
     (dict(E_r=2000, k=2), moe.MOE_ERR_UNSUPPORTED),
     (dict(c=float("nan")), moe.MOE_ERR_INVALID_ARG),
-    (dict(reject_policy=2), moe.MOE_ERR_INVALID_ARG),
+    (dict(reject_policy=3), moe.MOE_ERR_INVALID_ARG),
     (dict(accept_order=2), moe.MOE_ERR_INVALID_ARG),
+    # rerouting: 1 <= depth <= min(E_r - k, 32 - k); not with WLR or acceptance by weight
+    (dict(reject_policy=2), moe.MOE_ERR_INVALID_ARG),
+    (dict(reject_policy=2, reroute_depth=7), moe.MOE_ERR_INVALID_ARG),
+    (dict(reject_policy=2, E_r=64, k=30, reroute_depth=3), moe.MOE_ERR_INVALID_ARG),
+    (dict(reject_policy=2, reroute_depth=2, norm=moe.MOE_NORM_WLR, theta=0.3), moe.MOE_ERR_UNSUPPORTED),
+    (dict(reject_policy=2, reroute_depth=2, accept_order=1), moe.MOE_ERR_UNSUPPORTED),
 ])
 def test_invalid_params_are_rejected_on_the_host(kw, status):
     base = dict(N=16, d=64, d_f=64, E_r=8, k=2)
@@ -101,6 +107,24 @@ def test_wait_selftest_limits_are_checked_on_the_host():
         assert r == moe.MOE_ERR_INVALID_ARG
     r = moe.lib().moe_selftest_wait_timeout(ctypes.byref(p), None, 50_000_000, None)
     assert r == moe.MOE_ERR_WORKSPACE
+
+
+def test_reroute_workspace_regions_and_refusals():
+    p = moe.params(1000, 64, 64, 16, 4, c=1.0, reject_policy=moe.MOE_REJECT_REROUTE, reroute_depth=5)
+    L = moe.moe_workspace_layout(p)
+    assert L["cand_w"] - L["cand"] >= 1000 * 5 * 4 and L["rr_e"] - L["cand_w"] >= 1000 * 5 * 4
+    assert L["rr_slot"] - L["rr_e"] >= 1000 * 4 * 4 and L["scratch"] - L["rr_slot"] >= 1000 * 4 * 4
+    p0 = moe.params(1000, 64, 64, 16, 4, c=1.0)
+    L0 = moe.moe_workspace_layout(p0)
+    assert L0["cand"] == L0["cand_w"] == L0["rr_e"] == L0["rr_slot"] == L0["scratch"]
+    assert moe.moe_workspace_size(p) > moe.moe_workspace_size(p0)
+    lib = moe.lib()
+    fake = ctypes.c_void_p(256)
+    assert lib.moe_forward_begin(ctypes.byref(p), fake, fake, None, None, None, fake, None) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_dispatch_noalloc(ctypes.byref(p), fake, fake, 1, fake, fake, fake, fake, None, None,
+                                    None) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_backward_workspace_size(ctypes.byref(p), None, ctypes.byref(ctypes.c_size_t())) == \
+        moe.MOE_ERR_UNSUPPORTED
 
 
 def test_acceptance_by_weight_is_refused_where_it_is_not_built():

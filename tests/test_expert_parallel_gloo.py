@@ -15,7 +15,7 @@ import torch.multiprocessing as mp
 
 import oracle
 import seeded_inputs as si
-from sparse_mixture_experts_25_b200 import expert_parallel as ep
+from tests import ep_host_plan as ep
 from sparse_mixture_experts_25_b200 import sharded
 
 CASE = si.WORKLOADS["qwen3_skew_bf16"].scaled("ep_gloo", N=400, d=64, d_f=32, E=8, k=2, dtype=si.DT_F32)

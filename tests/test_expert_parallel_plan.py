@@ -4,7 +4,7 @@ checked against a brute-force replay of group-wide token-order acceptance."""
 import numpy as np
 import pytest
 
-from sparse_mixture_experts_25_b200 import expert_parallel as ep
+from tests import ep_host_plan as ep
 
 
 def _brute(counts_all, C):
@@ -45,3 +45,29 @@ def test_plan_matches_brute_force(R, E, C, seed):
         got = [src[i] for i in index]
         want = [(s, j) for j in range(El) for s in range(R) for _ in range(int(acc[s, r * El + j]))]
         assert got == want
+
+
+@pytest.mark.parametrize("R,E,C,seed", [(2, 8, 5, 0), (4, 8, 3, 1), (4, 16, 40, 2), (8, 64, 7, 3)])
+def test_fused_exchange_positions_are_the_owners_expert_major_order(R, E, C, seed):
+    """Where the fused exchange writes each accepted row: source s's i-th row
+    for expert e lands at dest_base[e] + i in the owner's buffer, which must be
+    exactly that row's place in expert-major order (owned expert, then source,
+    then token order), built here by brute force."""
+    rng = np.random.default_rng(seed)
+    counts = rng.integers(0, 12, size=(R, E))
+    acc = _brute(counts, C)
+    El = E // R
+    for owner in range(R):
+        order = [(s, e, i) for e in range(owner * El, (owner + 1) * El) for s in range(R) for i in range(acc[s, e])]
+        place = {key: n for n, key in enumerate(order)}
+        for s in range(R):
+            base = ep.dest_base(acc, s, R)
+            for e in range(owner * El, (owner + 1) * El):
+                for i in range(acc[s, e]):
+                    assert base[e] + i == place[(s, e, i)]
+        # the owner's expert offsets are the starts of its experts in that order
+        _, offsets = ep.regroup(acc, owner, R)
+        for j in range(El):
+            e = owner * El + j
+            first = [n for n, key in enumerate(order) if key[1] == e]
+            assert offsets[j] == (first[0] if first else offsets[j + 1] if j + 1 <= El else offsets[j])

@@ -20,6 +20,7 @@ if not torch.cuda.is_available():  # pragma: no cover - GPU tests need a device
 import sparse_mixture_experts_25_b200 as moe  # noqa: E402
 from sparse_mixture_experts_25_b200 import expert_parallel as ep  # noqa: E402
 from sparse_mixture_experts_25_b200 import sharded  # noqa: E402
+from tests import ep_host_plan  # noqa: E402
 
 W = si.WORKLOADS
 CASES = {
@@ -46,25 +47,44 @@ def _ranks(w, R, dev):
     return layers, xs
 
 
+@pytest.mark.parametrize("path", ["collectives", "fused"])
 @pytest.mark.parametrize("name,R", [("qwen3_skewed_capped", 2), ("qwen3_skewed_capped", 4),
                                     ("deepseek_shared", 4), ("mixtral_pairs", 2), ("switch_f32_capped", 4)])
-def test_expert_parallel_emulated(name, R):
+def test_expert_parallel_emulated(name, R, path):
+    """R ranks in one process: with the rows moved by (emulated) all-to-all
+    collectives, or written straight into the owners' expert-major buffers and
+    read back from them (the fused exchange, the owners' buffers local here)."""
     w = CASES[name]
     inp = si.inputs(w)
     full = parity.gpu_forward(w, inp)
     dev = full["dev"]
     layers, xs = _ranks(w, R, dev)
     Ys = [torch.full((x.shape[0], w.d), float("nan"), device="cuda") for x in xs]
-    ep.emulate(layers, xs, Ys)
+    (ep.emulate if path == "collectives" else ep.emulate_peer)(layers, xs, Ys)
     torch.cuda.synchronize()
+    # the device plan against the host restatement
+    counts_all = np.stack([L.counts.cpu().numpy() for L in layers])
+    acc = ep_host_plan.accepted_counts(counts_all, layers[0].C)
+    rows = ep_host_plan.send_rows(acc, R)
+    for r, L in enumerate(layers):
+        send, recv = L.split_sizes()
+        assert send == [int(v) for v in rows[r]] and recv == [int(v) for v in rows[:, r]]
+        index, offsets = ep_host_plan.regroup(acc, r, R)
+        np.testing.assert_array_equal(L.local_offsets.cpu().numpy(), offsets)
+        if path == "collectives":
+            np.testing.assert_array_equal(L.regroup[:index.size].cpu().numpy(), index)
+        views = moe.workspace_views(L.p, L.ws)
+        np.testing.assert_array_equal(views["acc"].cpu().numpy(), acc[r])
     ids = np.concatenate([moe.workspace_views(L.p, L.ws)["ids"].cpu().numpy() for L in layers])
     np.testing.assert_array_equal(ids, full["rec"]["ids"])
     slot = np.concatenate([moe.workspace_views(L.p, L.ws)["slot"].cpu().numpy() for L in layers])
     np.testing.assert_array_equal(slot, full["rec"]["slot"])
     if full["stats"]["rejected"]:
         assert (slot < 0).any()
+    # the owners run the unfused expert kernels: outputs against the oracle on
+    # the (identical) routing records, at the layer's tolerance
     Y = np.concatenate([y.cpu().numpy() for y in Ys]).astype(np.float64)
-    assert parity.rel_err(Y, full["Y"]) <= 1e-5
+    parity.check_rows(w, inp, full["rec"], Y)
 
 
 def test_expert_parallel_forward_one_rank_nccl():
@@ -86,6 +106,6 @@ def test_expert_parallel_forward_one_rank_nccl():
         Y = torch.full((w.N, w.d), float("nan"), device="cuda")
         layer.forward(x, Y)
         torch.cuda.synchronize()
-        assert parity.rel_err(Y.cpu().numpy().astype(np.float64), full["Y"]) <= 1e-5
+        parity.check_rows(w, inp, full["rec"], Y.cpu().numpy().astype(np.float64))
     finally:
         dist.destroy_process_group()
