@@ -162,10 +162,8 @@ typedef struct moe_stats {
                                 rerouted expert (included in accepted; rejected and
                                 tokens_affected / tokens_skipped then count the
                                 paths left without any expert); 0 otherwise       */
-    int64_t padded_rows;     /* rows the forward's routed expert GEMMs compute: fp32
-                                layers round each expert's accepted rows up to 64;
-                                bf16 layers run tiles of 256 tokens and round an
-                                expert's last tile up to 32 tokens               */
+    int64_t padded_rows;     /* rows the routed expert GEMMs compute: each expert's
+                                accepted rows rounded up to the GEMM's row tile    */
     double padding_ratio;    /* padded_rows / accepted (0 when nothing accepted)  */
     double aux_balance;      /* E_r sum_e f_e pbar_e ("LLM from scratch" ch. 36.4
                                 balance objective, value only): f_e = L_e / sum L,

@@ -830,363 +830,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Weight-stationary grouped GEMM on CTA pairs ("swapped" operands)
-// ---------------------------------------------------------------------------
-// The routed contractions put an expert's WEIGHT rows on the MMA's M side
-// (256 rows across a CTA pair, 128 in each CTA) and its TOKEN rows on the N
-// side (tiles of up to 256 tokens, the last tile of an expert rounded up to
-// 32): per expert the padding is at most 31 rows instead of up to 127 or 255,
-// and each SM reads 32 KB (16 KB of weights + 16 KB of tokens) per 512 tensor
-// cycles with 6 stages in flight.
-//   gate/up: CTA c of the pair holds the 64 gate rows and the 64 up rows of
-//            output columns j0 + 64 c .. j0 + 64 c + 63 (j0 = 128 m), so a
-//            TMEM lane holds gate (lanes 0-63) or up (lanes 64-127) of one
-//            column for every token of the tile; the epilogue warps of lane
-//            quarters 0/2 and 1/3 swap half a chunk through shared memory
-//            and each writes h for 16 tokens.
-//   down:    CTA c holds output features n0 + 128 c .. + 127 (n0 = 256 m);
-//            a TMEM lane holds one feature for every token, and the epilogue
-//            adds a_t * value into Y[token] (32 x 32 chunks transposed
-//            through shared memory: 16-byte red.add, 4 tokens x 128 bytes
-//            per warp instruction).
-// Tiles are ordered expert by expert, weight tile by weight tile, token
-// tiles fastest, so the pairs working on one weight tile run together and
-// share it through L2, and an expert's tokens stay in L2 across its weight
-// tiles.  Loads, MMAs, barriers and bounded waits follow tc_grouped_kernel's
-// CTA-pair mode.
-constexpr int SW_STAGES = 6;
-constexpr int SW_A_BYTES = 128 * BK * 2;
-constexpr int SW_B_MAX_BYTES = 128 * BK * 2;
-constexpr int SW_STAGE_BYTES = SW_A_BYTES + SW_B_MAX_BYTES;
-constexpr int SW_TOK = 256;   // tokens per tile
-constexpr int SW_GRAN = 32;   // MMA N of a tile: its tokens rounded up to a multiple of this
-constexpr int kXchLd = 17;    // floats per row of the gate/up exchange buffers
-constexpr size_t kXchBytes = 2 * 2 * 32 * kXchLd * sizeof(float);
-// kind::f16, D fp32, A and B bf16 K-major, M = 256 across the pair; N per tile
-constexpr uint32_t kIdescSwapBase = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 4) << 24);
-
-// Exchange handshake of the two epilogue warps of a gate/up column group: all
-// 64 threads arrive on the group's mbarrier, then wait (bounded) for the
-// phase; k counts the group's handshakes.  A wait that gives up leaves the
-// kernel through the abort path like every other wait.
-__device__ __forceinline__ bool xch_sync(uint64_t* bar, uint32_t& k, volatile int* abort_flag,
-                                         unsigned long long* counters) {
-    __syncwarp();
-    mbar_arrive(bar);
-    const bool ok = warp_wait_bounded(bar, k & 1u, abort_flag, counters);
-    ++k;
-    return ok;
-}
-
-__device__ __forceinline__ int swap_tile_n(int rows) {
-    const int n = (rows + SW_GRAN - 1) / SW_GRAN * SW_GRAN;
-    return n < SW_GRAN ? SW_GRAN : (n > SW_TOK ? SW_TOK : n);
-}
-
-// TMEM lane = weight row, column = token.  Gate/up: gate in lane quarters 0-1,
-// up in 2-3 (the same 64 output columns); the two warps of a column group
-// trade half of each 32-token chunk.  Returns false if a handshake gave up.
-__device__ __forceinline__ bool swap_epilogue_swiglu(const TcArgs& a, const Tile& ti, uint32_t t_row, int quarter,
-                                                     int lane, int nt, uint32_t crank, float* xch, uint64_t* xbar,
-                                                     uint32_t& xk, volatile int* abort_flag) {
-    const bool gate = quarter < 2;
-    const int grp = quarter & 1;
-    const int j = ti.n_tile * 128 + (int)crank * 64 + grp * 32 + lane;  // output column of this lane
-    const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
-    const int ld = ti.shared ? a.ld_out_sh : a.ld_out;
-    __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(ti.shared ? a.out_sh : a.out);
-    float* xg = xch + grp * (2 * 32 * kXchLd);  // gate values of tokens 16-31 (written by the gate warp)
-    float* xu = xg + 32 * kXchLd;               // up values of tokens 0-15 (written by the up warp)
-    const bool col_ok = j < n_valid;
-#pragma unroll 1
-    for (int c0 = 0; c0 < nt; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(t_row + (uint32_t)c0, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (gate) xg[lane * kXchLd + i] = __uint_as_float(v[16 + i]);
-            else xu[lane * kXchLd + i] = __uint_as_float(v[i]);
-        }
-        if (!xch_sync(&xbar[grp], xk, abort_flag, a.counters)) return false;
-        const int tb = c0 + (gate ? 0 : 16);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float g = gate ? __uint_as_float(v[i]) : xg[lane * kXchLd + i];
-            const float u = gate ? xu[lane * kXchLd + i] : __uint_as_float(v[16 + i]);
-            const int tok = tb + i;
-            if (col_ok && tok < ti.rows)
-                outp[(int64_t)(ti.a_row + tok) * ld + j] = __float2bfloat16_rn(silu_f(g) * u);
-        }
-        // the exchange rows are free for the next chunk
-        if (!xch_sync(&xbar[grp], xk, abort_flag, a.counters)) return false;
-    }
-    return true;
-}
-
-// Down projection + weighted combine: TMEM lane = output feature, column = token.
-__device__ __forceinline__ void swap_epilogue_combine(const TcArgs& a, const Tile& ti, uint32_t t_row, int quarter,
-                                                      int lane, int nt, uint32_t crank, float* stg) {
-    const int nf = ti.n_tile * 256 + (int)crank * 128 + quarter * 32;  // first feature of this warp
-    const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
-    const int fc = (lane & 7) * 4;
-#pragma unroll 1
-    for (int c0 = 0; c0 < nt; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(t_row + (uint32_t)c0, v);
-        tmem_ld_wait();
-        // token and combine weight of column c0 + lane
-        int tok = -1;
-        float wt = 0.f;
-        const int tt = c0 + lane;
-        if (tt < ti.rows) {
-            const int row = ti.a_row + tt;
-            if (ti.shared) {
-                tok = row;
-                wt = 1.f;
-            } else if (row < a.max_rows) {
-                tok = a.slot_token[row];
-                wt = a.slot_w[row];
-            }
-            if (tok < 0 || tok >= a.n_tokens) tok = -1;
-        }
-#pragma unroll
-        for (int t = 0; t < 32; ++t) stg[t * kStgLd + lane] = __uint_as_float(v[t]) * __shfl_sync(0xffffffffu, wt, t);
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int rr = i * 4 + (lane >> 3);
-            const int tk = __shfl_sync(0xffffffffu, tok, rr);
-            if (tk >= 0 && nf + fc < n_valid) {
-                const float4 val = *reinterpret_cast<const float4*>(stg + rr * kStgLd + fc);
-                red_add_v4(a.Y + (int64_t)tk * a.ldY + nf + fc, val.x, val.y, val.z, val.w);
-            }
-        }
-        __syncwarp();
-    }
-}
-
-// mW0 / mW1: routed weights (gate/up: W_g and W_u in 64-row boxes; down: W_d
-// in 128-row boxes, mW1 unused); mX / mX16: routed token rows (x_perm or h)
-// in 128- and 16-row boxes; the _sh maps the same for the shared expert.
-template <int EPI>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    tc_swap_kernel(const __grid_constant__ CUtensorMap mW0, const __grid_constant__ CUtensorMap mW1,
-                   const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mX16,
-                   const __grid_constant__ CUtensorMap mW0_sh, const __grid_constant__ CUtensorMap mW1_sh,
-                   const __grid_constant__ CUtensorMap mX_sh, const __grid_constant__ CUtensorMap mX16_sh,
-                   const TcArgs a) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~uintptr_t(1023));
-    uint8_t* stage_base = smem;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + SW_STAGES * SW_STAGE_BYTES);
-    uint64_t* empty = full + SW_STAGES;
-    uint64_t* tfull = empty + SW_STAGES;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* done = tempty + 2;
-    uint64_t* xbar = done + 1;  // [2] gate/up exchange handshakes
-    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(xbar + 2);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
-    SchedSmem* sched = reinterpret_cast<SchedSmem*>(smem + SW_STAGES * SW_STAGE_BYTES + 256);
-    float* epi_smem = reinterpret_cast<float*>(
-        (reinterpret_cast<uintptr_t>(sched) + sizeof(SchedSmem) + 127) & ~static_cast<uintptr_t>(127));
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t crank = cluster_ctarank();
-    const bool leader = crank == 0;
-    const int unit = (int)(blockIdx.x >> 1);
-    const int n_units = (int)(gridDim.x >> 1);
-
-    if (a.has_routed) {
-        for (int i = threadIdx.x; i <= a.E; i += NUM_THREADS) {
-            sched->mt[i] = a.mt_start[i];
-            sched->off[i] = a.offsets[i];
-        }
-    }
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < SW_STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 8);  // one arrival per epilogue warp of both CTAs
-        }
-        mbar_init(done, 1);
-        mbar_init(&xbar[0], 64);
-        mbar_init(&xbar[1], 64);
-        *abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    if (warp == 1) tmem_alloc_pair(tmem_base_s, TMEM_COLS);
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&mW0);
-        if (EPI == EPI_SWIGLU) tma_prefetch_desc(&mW1);
-        tma_prefetch_desc(&mX);
-        tma_prefetch_desc(&mX16);
-        if (a.M_sh > 0) {
-            tma_prefetch_desc(&mW0_sh);
-            if (EPI == EPI_SWIGLU) tma_prefetch_desc(&mW1_sh);
-            tma_prefetch_desc(&mX_sh);
-            tma_prefetch_desc(&mX16_sh);
-        }
-    }
-    tc_fence_before();
-    cluster_sync_all();  // the peer's barriers exist before any remote arrival
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_base_s;
-
-    const int routed_tiles = a.has_routed ? sched->mt[a.E] * a.nt_r : 0;
-    const int total_tiles =
-        (routed_tiles + (a.M_sh > 0 ? ((a.M_sh + SW_TOK - 1) / SW_TOK) * a.nt_sh : 0)) * a.ks;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int issued_parity[SW_STAGES];
-            for (int s = 0; s < SW_STAGES; ++s) issued_parity[s] = -1;
-            bool ok = true;
-            for (int t = unit; t < total_tiles && ok; t += n_units) {
-                Tile ti;
-                decode_tile<SW_TOK>(t, *sched, a, routed_tiles, ti);
-                const int half = swap_tile_n(ti.rows) / 2;  // token rows this CTA loads
-                const CUtensorMap* pw0 = ti.shared ? &mW0_sh : &mW0;
-                const CUtensorMap* pw1 = ti.shared ? &mW1_sh : &mW1;
-                const CUtensorMap* px = ti.shared ? &mX_sh : &mX;
-                const CUtensorMap* px16 = ti.shared ? &mX16_sh : &mX16;
-                const int wbase = ti.shared ? 0 : ti.g * a.b_rows_r;
-                const int w_row = EPI == EPI_SWIGLU ? wbase + ti.n_tile * 128 + (int)crank * 64
-                                                    : wbase + ti.n_tile * 256 + (int)crank * 128;
-                const int x_row = ti.a_row + (int)crank * half;
-                const uint32_t bytes = 2u * (uint32_t)(SW_A_BYTES + half * BK * 2);
-                for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, a.counters)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* sa = stage_base + stage * SW_STAGE_BYTES;
-                    uint8_t* sb = sa + SW_A_BYTES;
-                    const uint32_t fb = map_shared_rank(smem_u32(&full[stage]), 0);
-                    if (leader) mbar_expect_tx(&full[stage], bytes);
-                    if (EPI == EPI_SWIGLU) {
-                        tma_load_2d_pair(sa, pw0, fb, kb * BK, w_row);
-                        tma_load_2d_pair(sa + SW_A_BYTES / 2, pw1, fb, kb * BK, w_row);
-                    } else {
-                        tma_load_2d_pair(sa, pw0, fb, kb * BK, w_row);
-                    }
-                    if (half == 128) {
-                        tma_load_2d_pair(sb, px, fb, kb * BK, x_row);
-                    } else {
-                        for (int r = 0; r < half; r += 16)
-                            tma_load_2d_pair(sb + r * BK * 2, px16, fb, kb * BK, x_row + r);
-                    }
-                    issued_parity[stage] = (int)phase;
-                    if (++stage == SW_STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-            }
-            if (*abort_flag && leader) {
-                for (int s = 0; s < SW_STAGES; ++s)
-                    if (issued_parity[s] >= 0)
-                        wait_bounded(&full[s], (uint32_t)issued_parity[s], abort_flag, a.counters, kTimeoutNs / 4);
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0 && leader) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
-            bool ok = true;
-            for (int t = unit; t < total_tiles && ok; t += n_units) {
-                Tile ti;
-                decode_tile<SW_TOK>(t, *sched, a, routed_tiles, ti);
-                const uint32_t idesc = kIdescSwapBase | ((uint32_t)(swap_tile_n(ti.rows) >> 3) << 17);
-                if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, a.counters)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-                    if (!wait_bounded(&full[stage], phase, abort_flag, a.counters)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sa = smem_u32(stage_base + stage * SW_STAGE_BYTES);
-                    const uint64_t ad = smem_desc_sw128(sa);
-                    const uint64_t bd = smem_desc_sw128(sa + SW_A_BYTES);
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_bf16_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc,
-                                       (kb > ti.kb0 || kk > 0) ? 1u : 0u);
-                    umma_commit_pair_both(&empty[stage]);
-                    if (++stage == SW_STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-                if (!ok) break;
-                umma_commit_pair_both(&tfull[acc]);
-                if (++acc == 2) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
-            }
-            umma_commit_pair_local(done);
-            wait_bounded(done, 0, abort_flag, a.counters, kTimeoutNs / 4);
-        }
-    } else {
-        // epilogue warps 2..5: TMEM lane quarter = warp % 4
-        if (a.zero_ptr) {
-            const int64_t per = (a.zero_n4 + gridDim.x - 1) / gridDim.x;
-            const int64_t lo = per * blockIdx.x;
-            const int64_t hi = min64(a.zero_n4, lo + per);
-            float4* z = reinterpret_cast<float4*>(a.zero_ptr);
-            for (int64_t i = lo + (threadIdx.x - 64); i < hi; i += 128) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        const int quarter = warp & 3;
-        int acc = 0;
-        uint32_t acc_phase = 0;
-        uint32_t xk = 0;  // handshakes of this warp's gate/up column group
-        for (int t = unit; t < total_tiles; t += n_units) {
-            Tile ti;
-            decode_tile<SW_TOK>(t, *sched, a, routed_tiles, ti);
-            const int nt = swap_tile_n(ti.rows);
-            if (!warp_wait_bounded(&tfull[acc], acc_phase, abort_flag, a.counters)) break;
-            tc_fence_after();
-            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-            if (EPI == EPI_SWIGLU) {
-                if (!swap_epilogue_swiglu(a, ti, t_row, quarter, lane, nt, crank, epi_smem, xbar, xk, abort_flag))
-                    break;
-            } else {
-                swap_epilogue_combine(a, ti, t_row, quarter, lane, nt, crank, epi_smem + (warp - 2) * 32 * kStgLd);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(map_shared_rank(smem_u32(&tempty[acc]), 0));
-            if (++acc == 2) {
-                acc = 0;
-                acc_phase ^= 1u;
-            }
-        }
-    }
-
-    __syncwarp();
-    if (*abort_flag) {
-        const unsigned long long t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 2000000ull) {
-        }
-    }
-    tc_fence_before();
-    cluster_sync_all();
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
-}
-
-// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -1440,41 +1083,6 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
     return launch_tc<EPI_STORE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles, st);
 }
 
-// the swapped-operand kernel: stages, barriers, schedule, epilogue buffers
-constexpr size_t swap_smem_bytes(int epi) {
-    return 1024 + (size_t)SW_STAGES * SW_STAGE_BYTES + 256 + sizeof(SchedSmem) + 128 +
-           (epi == EPI_SWIGLU ? kXchBytes : (size_t)4 * 32 * kStgLd * sizeof(float));
-}
-static_assert(swap_smem_bytes(EPI_SWIGLU) <= 232448 && swap_smem_bytes(EPI_COMBINE) <= 232448,
-              "shared memory per CTA");
-
-template <int EPI>
-cudaError_t launch_swap(const CUtensorMap& mW0, const CUtensorMap& mW1, const CUtensorMap& mX, const CUtensorMap& mX16,
-                        const CUtensorMap& mW0_sh, const CUtensorMap& mW1_sh, const CUtensorMap& mX_sh,
-                        const CUtensorMap& mX16_sh, const TcArgs& a, int64_t max_tiles, cudaStream_t st) {
-    auto kern = tc_swap_kernel<EPI>;
-    const size_t smem = swap_smem_bytes(EPI);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int pairs = (int)min64(max_tiles, num_sms() / 2);
-    if (pairs <= 0) return cudaSuccess;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mW0, mW1, mX, mX16, mW0_sh, mW1_sh, mX_sh, mX16_sh, a);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
-}
-
 cudaError_t launch_tc_dense(int64_t M, int64_t Nc, int64_t K, const void* A, const void* B, float* out,
                             unsigned long long* counters, cudaStream_t st, int* status) {
     *status = MOE_OK;
@@ -1503,112 +1111,6 @@ cudaError_t launch_tc_dense(int64_t M, int64_t Nc, int64_t K, const void* A, con
         if (e != cudaSuccess) return e;
     }
     return launch_tc<EPI_STORE, false>(mA, mB, mB, mA, mB, mB, mA, mA, a, tiles * a.ks, st);
-}
-
-cudaError_t launch_swap_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
-                                const int32_t* offsets, const int32_t* mt_start, const ExpertWeights& W, void* h,
-                                void* h_shared, float* Y_zero, unsigned long long* counters, cudaStream_t st,
-                                int* status) {
-    *status = MOE_OK;
-    CUtensorMap mW0, mW1, mX, mX16, mW0_sh, mW1_sh, mX_sh, mX16_sh;
-    const uint64_t rows = (uint64_t)(p.N * p.k);
-    bool ok = make_map(&mW0, W.W_g, (uint64_t)p.E_r * p.d_f, p.d, 64) &&
-              make_map(&mW1, W.W_u, (uint64_t)p.E_r * p.d_f, p.d, 64) && make_map(&mX, x_perm, rows, p.d, 128) &&
-              make_map(&mX16, x_perm, rows, p.d, 16);
-    const bool sh = p.d_f_shared > 0;
-    if (ok && sh) {
-        ok = make_map(&mW0_sh, W.Ws_g, (uint64_t)p.d_f_shared, p.d, 64) &&
-             make_map(&mW1_sh, W.Ws_u, (uint64_t)p.d_f_shared, p.d, 64) &&
-             make_map(&mX_sh, x_shared, (uint64_t)p.N, p.d, 128) && make_map(&mX16_sh, x_shared, (uint64_t)p.N, p.d, 16);
-    } else {
-        mW0_sh = mW0;
-        mW1_sh = mW1;
-        mX_sh = mX;
-        mX16_sh = mX16;
-    }
-    if (!ok) {
-        *status = MOE_ERR_CUDA;
-        return cudaErrorInvalidValue;
-    }
-    TcArgs a{};
-    a.mt_start = mt_start;
-    a.offsets = offsets;
-    a.E = p.E_r;
-    a.nt_r = (p.d_f + 127) / 128;
-    a.nkb_r = (p.d + BK - 1) / BK;
-    a.b_rows_r = p.d_f;
-    a.M_sh = sh ? (int)p.N : 0;
-    a.nt_sh = sh ? (p.d_f_shared + 127) / 128 : 0;
-    a.nkb_sh = a.nkb_r;
-    a.n_valid_r = p.d_f;
-    a.n_valid_sh = p.d_f_shared;
-    a.out = h;
-    a.out_sh = h_shared;
-    a.ld_out = p.d_f;
-    a.ld_out_sh = p.d_f_shared;
-    a.max_rows = (int)(p.N * p.k);
-    a.n_tokens = (int)p.N;
-    a.has_routed = 1;
-    a.ks = 1;
-    a.zero_ptr = Y_zero;
-    a.zero_n4 = Y_zero ? p.N * (int64_t)p.d / 4 : 0;
-    a.counters = counters;
-    int64_t max_tiles = routed_mtile_bound(p, SW_TOK) * a.nt_r + (sh ? ((p.N + SW_TOK - 1) / SW_TOK) * a.nt_sh : 0);
-    if (Y_zero && max_tiles < num_sms() / 2) max_tiles = num_sms() / 2;  // every CTA zeroes a share
-    return launch_swap<EPI_SWIGLU>(mW0, mW1, mX, mX16, mW0_sh, mW1_sh, mX_sh, mX16_sh, a, max_tiles, st);
-}
-
-cudaError_t launch_swap_down(const moe_params& p, int64_t C, const void* h, const void* h_shared,
-                             const int32_t* offsets, const int32_t* mt_start, const ExpertWeights& W,
-                             const int32_t* slot_token, const float* slot_w, float* Y, unsigned long long* counters,
-                             cudaStream_t st, int* status) {
-    *status = MOE_OK;
-    CUtensorMap mW0, mX, mX16, mW0_sh, mX_sh, mX16_sh;
-    const uint64_t rows = (uint64_t)(p.N * p.k);
-    bool ok = make_map(&mW0, W.W_d, (uint64_t)p.E_r * p.d, p.d_f, 128) && make_map(&mX, h, rows, p.d_f, 128) &&
-              make_map(&mX16, h, rows, p.d_f, 16);
-    const bool sh = p.d_f_shared > 0;
-    if (ok && sh) {
-        ok = make_map(&mW0_sh, W.Ws_d, (uint64_t)p.d, p.d_f_shared, 128) &&
-             make_map(&mX_sh, h_shared, (uint64_t)p.N, p.d_f_shared, 128) &&
-             make_map(&mX16_sh, h_shared, (uint64_t)p.N, p.d_f_shared, 16);
-    } else {
-        mW0_sh = mW0;
-        mX_sh = mX;
-        mX16_sh = mX16;
-    }
-    if (!ok) {
-        *status = MOE_ERR_CUDA;
-        return cudaErrorInvalidValue;
-    }
-    TcArgs a{};
-    a.mt_start = mt_start;
-    a.offsets = offsets;
-    a.E = p.E_r;
-    a.nt_r = (p.d + 255) / 256;
-    a.nkb_r = (p.d_f + BK - 1) / BK;
-    a.b_rows_r = p.d;
-    a.M_sh = sh ? (int)p.N : 0;
-    a.nt_sh = sh ? a.nt_r : 0;
-    a.nkb_sh = sh ? (p.d_f_shared + BK - 1) / BK : 0;
-    a.n_valid_r = p.d;
-    a.n_valid_sh = p.d;
-    a.slot_token = slot_token;
-    a.slot_w = slot_w;
-    a.Y = Y;
-    a.ldY = p.d;
-    a.max_rows = (int)(p.N * p.k);
-    a.n_tokens = (int)p.N;
-    a.has_routed = 1;
-    a.counters = counters;
-    // the combine reduces with red.add into a zeroed Y: split K across pairs
-    // when the output tiles fill less than one wave of pairs
-    const double tiles = routed_mtile_estimate(p, C, SW_TOK) * a.nt_r +
-                         (sh ? (double)((p.N + SW_TOK - 1) / SW_TOK) * a.nt_sh : 0.0);
-    a.ks = choose_ksplit(2.0 * tiles, sh ? std::min(a.nkb_r, a.nkb_sh) : a.nkb_r);
-    const int64_t max_tiles =
-        (routed_mtile_bound(p, SW_TOK) * a.nt_r + (sh ? ((p.N + SW_TOK - 1) / SW_TOK) * a.nt_sh : 0)) * a.ks;
-    return launch_swap<EPI_COMBINE>(mW0, mW0, mX, mX16, mW0_sh, mW0_sh, mX_sh, mX16_sh, a, max_tiles, st);
 }
 
 cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,

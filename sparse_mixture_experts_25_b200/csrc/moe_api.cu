@@ -437,7 +437,7 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
                                   v.scratch.psum, st, v.cand, v.cand_w);
     if (e != cudaSuccess) return fail(e, "moe_forward router");
     if ((e0 = stage_mark(1, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
-    const int bm = p->dtype == MOE_BF16 ? kSwapTok : kSimtBM;
+    const int bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
     const char* where = "";
     e = launch_dispatch(*p, C, bm, v.ids, v.w, v.slot, v.offsets, v.L, v.acc, v.slot_token, v.slot_w,
                         x, v.x_perm, v.counters, v.scratch, st, &where);
@@ -449,12 +449,12 @@ moe_status moe_forward(const moe_params* p, const void* x, const void* W_r, cons
     if ((e0 = stage_mark(2, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
     int status = MOE_OK;
     if (p->dtype == MOE_BF16) {
-        e = launch_swap_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, Y, v.counters,
-                                st, &status);
+        e = launch_tc_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared,
+                              Y, v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_forward gate/up: tensor map encode" : "moe_forward gate/up (tcgen05)");
         if ((e0 = stage_mark(3, st)) != cudaSuccess) return fail(e0, "moe_forward stage event");
-        e = launch_swap_down(*p, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W, v.slot_token, v.slot_w, Y,
-                             v.counters, st, &status);
+        e = launch_tc_down(*p, DOWN_COMBINE, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
+                           v.slot_token, v.slot_w, Y, nullptr, v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, status != MOE_OK ? "moe_forward down: tensor map encode" : "moe_forward down+combine (tcgen05)");
     } else {
         e = launch_simt_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, st);
@@ -572,7 +572,7 @@ moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32
     if (e == cudaSuccess) e = cudaMemsetAsync(v.counters + CNT_L_MAX, 0, 2 * 8, st);
     if (e != cudaSuccess) return fail(e, "moe_forward_end memset");
     const bool bf16 = p->dtype == MOE_BF16;
-    const int bm = bf16 ? kSwapTok : kSimtBM;
+    const int bm = bf16 ? tc_tile_rows(*p) : kSimtBM;
     const char* where = "";
     e = launch_dispatch_ranked(*p, C, bm, counts_all, rank, n_ranks, N_group, v.ids, v.w, v.slot,
                                v.offsets, v.L, v.acc, v.slot_token, v.slot_w, x, v.x_perm,
@@ -586,12 +586,12 @@ moe_status moe_forward_end(const moe_params* p, const int32_t* counts_all, int32
     if ((e = stage_mark(2, st)) != cudaSuccess) return fail(e, "moe_forward_end stage event");
     int status = MOE_OK;
     if (bf16) {
-        e = launch_swap_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, Y, v.counters,
-                                st, &status);
+        e = launch_tc_gate_up(*p, v.x_perm, x, v.offsets, v.scratch.mt_start, W, v.h, v.h_shared, Y,
+                              v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, "moe_forward_end gate/up (tcgen05)");
         if ((e = stage_mark(3, st)) != cudaSuccess) return fail(e, "moe_forward_end stage event");
-        e = launch_swap_down(*p, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W, v.slot_token, v.slot_w, Y,
-                             v.counters, st, &status);
+        e = launch_tc_down(*p, DOWN_COMBINE, C, v.h, v.h_shared, v.offsets, v.scratch.mt_start, W,
+                           v.slot_token, v.slot_w, Y, nullptr, v.counters, st, &status);
         if (e != cudaSuccess) return fail(e, "moe_forward_end down+combine (tcgen05)");
     } else {
         e = launch_zero_f32(Y, p->N * (int64_t)p->d, st);
@@ -668,17 +668,12 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
         const double n_group = cnt[CNT_N_GROUP] ? (double)cnt[CNT_N_GROUP] : (double)p->N;
         out->rho_max = (double)out->L_max * (double)p->E_r / (n_group * (double)p->k);
         out->reject_rate = out->requested ? (double)out->rejected / (double)out->requested : 0.0;
-        // rows the forward's routed GEMMs compute: fp32 layers round each
-        // expert's accepted rows up to the 64-row tile; bf16 layers run full
-        // token tiles of kSwapTok plus a last tile rounded up to kSwapGran
+        // rows the routed GEMMs compute: accepted rows per expert rounded up
+        // to the row tile of the kernels that run them
+        const int64_t bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
         int64_t padded = 0, accepted = 0;
         for (int32_t a : acc) {
-            if (p->dtype == MOE_BF16) {
-                const int64_t full = a / kSwapTok * kSwapTok, tail = a - full;
-                padded += full + (tail + kSwapGran - 1) / kSwapGran * kSwapGran;
-            } else {
-                padded += (a + kSimtBM - 1) / kSimtBM * kSimtBM;
-            }
+            padded += (a + bm - 1) / bm * bm;
             accepted += a;
         }
         out->padded_rows = padded;

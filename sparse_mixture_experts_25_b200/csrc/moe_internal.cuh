@@ -159,19 +159,6 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
 // rows of one output tile of the tcgen05 grouped GEMMs for these params
 // (256 when CTA pairs are used, else 128): the dispatch's M-tile prefix unit
 int tc_tile_rows(const moe_params& p);
-// The forward's routed GEMMs of bf16 layers: weight-stationary tiles on CTA
-// pairs (expert weight rows on the MMA's M side, up to kSwapTok tokens on its
-// N side); mt_start is the prefix of ceil(rows / kSwapTok) per expert.
-constexpr int kSwapTok = 256;
-constexpr int kSwapGran = 32;   // a tile's tokens are rounded up to a multiple of this
-cudaError_t launch_swap_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
-                                const int32_t* offsets, const int32_t* mt_start, const ExpertWeights& W, void* h,
-                                void* h_shared, float* Y_zero, unsigned long long* counters, cudaStream_t st,
-                                int* status);
-cudaError_t launch_swap_down(const moe_params& p, int64_t C, const void* h, const void* h_shared,
-                             const int32_t* offsets, const int32_t* mt_start, const ExpertWeights& W,
-                             const int32_t* slot_token, const float* slot_w, float* Y, unsigned long long* counters,
-                             cudaStream_t st, int* status);
 // out[M, Nc] (fp32, row-major) = A[M, K] B[Nc, K]^T, bf16 operands with rows
 // of K elements (K % 8 == 0, 16-byte aligned bases), tcgen05 tiles of 128 x 256
 cudaError_t launch_tc_dense(int64_t M, int64_t Nc, int64_t K, const void* A, const void* B, float* out,

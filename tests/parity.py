@@ -161,13 +161,11 @@ def check_dispatch(w: si.Workload, rec: dict, stats: dict):
     for key in ("requested", "accepted", "rejected", "O", "tokens_affected", "tokens_skipped", "L_max"):
         assert stats[key] == s[key], (key, stats[key], s[key])
     assert stats["C"] == C
-    # tile padding of the forward's routed GEMMs: fp32 layers round each
-    # expert's accepted rows up to 64; bf16 layers run 256-token tiles and a
-    # last tile rounded up to 32 tokens
-    if w.dtype == si.DT_F32:
-        padded = int(sum(-(-int(a) // 64) * 64 for a in d["acc"]))
-    else:
-        padded = int(sum(int(a) // 256 * 256 + -(-(int(a) % 256) // 32) * 32 for a in d["acc"]))
+    # tile padding of the routed GEMMs: each expert's accepted rows rounded up
+    # to the row tile (64 rows for fp32 layers; 128, or 256 on CTA pairs when
+    # experts average >= 768 rows, for bf16 layers)
+    bm = 64 if w.dtype == si.DT_F32 else (256 if w.N * w.k >= 768 * w.E else 128)
+    padded = int(sum(-(-int(a) // bm) * bm for a in d["acc"]))
     assert stats["padded_rows"] == padded
     assert stats["padding_ratio"] == pytest.approx(padded / s["accepted"] if s["accepted"] else 0.0)
     if w.N:
