@@ -461,11 +461,15 @@ __global__ void prio_token_kernel(const int32_t* __restrict__ ids, const float* 
 // Then the final offsets (prefix of acc), and the rows of every served path
 // (first choices at offsets[e] + slot, rerouted ones at offsets[e] + rr_slot)
 // with the per-token statistics.
+// rr_stop: set by the scan of a round that had no offers; every later round
+// returns at once (a round without offers leaves nothing for the next).
 __global__ void reroute_offer_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ slot,
                                      const int32_t* __restrict__ cand, int X, const int32_t* __restrict__ acc,
                                      int64_t C, int64_t N, int k, int E, int tile_tokens, int n_tiles,
                                      const int32_t* __restrict__ rr_e, int32_t* __restrict__ rr_next,
-                                     int32_t* __restrict__ rr_offer, int32_t* __restrict__ hist) {
+                                     int32_t* __restrict__ rr_offer, int32_t* __restrict__ hist,
+                                     const int32_t* __restrict__ rr_stop) {
+    if (*rr_stop) return;
     extern __shared__ int h[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
     __syncthreads();
@@ -502,22 +506,30 @@ __global__ void reroute_offer_kernel(const int32_t* __restrict__ ids, const int3
 }
 
 __global__ void reroute_scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int64_t C,
-                                    int32_t* __restrict__ acc, int32_t* __restrict__ base) {
+                                    int32_t* __restrict__ acc, int32_t* __restrict__ base,
+                                    int32_t* __restrict__ rr_stop) {
     __shared__ int sL[kMaxExperts];
+    __shared__ int any;
+    if (*rr_stop) return;  // uniform: every thread reads the same flag
+    if (threadIdx.x == 0) any = 0;
     tile_scan(hist, n_tiles, E, sL);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         const int a = acc[e];
         base[e] = a;
         acc[e] = (int)min64((int64_t)a + sL[e], C);
+        if (sL[e]) any = 1;
     }
+    __syncthreads();
+    if (threadIdx.x == 0 && !any) *rr_stop = 1;
 }
 
 __global__ void reroute_assign_kernel(const int32_t* __restrict__ rr_offer, const int32_t* __restrict__ cand,
                                       int X, int64_t N, int k, int E, int64_t C, int tile_tokens, int n_tiles,
                                       const int32_t* __restrict__ hist, const int32_t* __restrict__ base,
                                       int32_t* __restrict__ rr_e, int32_t* __restrict__ rr_slot,
-                                      int32_t* __restrict__ rr_q) {
+                                      int32_t* __restrict__ rr_q, const int32_t* __restrict__ rr_stop) {
+    if (*rr_stop) return;
     extern __shared__ int run[];
     const int lane = threadIdx.x;
     const int tile = blockIdx.x;
@@ -734,19 +746,20 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
         if ((e = cudaMemsetAsync(sc.rr_slot, 0xff, nk * 4, st)) != cudaSuccess) return e;
         if ((e = cudaMemsetAsync(sc.rr_q, 0xff, nk * 4, st)) != cudaSuccess) return e;
         if ((e = cudaMemsetAsync(sc.rr_next, 0, (size_t)p.N * 4, st)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(sc.rr_stop, 0, 4, st)) != cudaSuccess) return e;
         for (int r = 0; r < X; ++r) {
             *where = "reroute offer";
             reroute_offer_kernel<<<n_tiles, 256, sizeof(int) * E, st>>>(ids, slot, sc.cand, X, acc, C, p.N, k, E,
                                                                          sc.tile_tokens, n_tiles, sc.rr_e,
-                                                                         sc.rr_next, sc.rr_offer, sc.hist);
+                                                                         sc.rr_next, sc.rr_offer, sc.hist, sc.rr_stop);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             *where = "reroute scan";
-            reroute_scan_kernel<<<1, 1024, 0, st>>>(sc.hist, n_tiles, E, C, acc, sc.base);
+            reroute_scan_kernel<<<1, 1024, 0, st>>>(sc.hist, n_tiles, E, C, acc, sc.base, sc.rr_stop);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             *where = "reroute assign";
             reroute_assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(sc.rr_offer, sc.cand, X, p.N, k, E, C,
                                                                          sc.tile_tokens, n_tiles, sc.hist, sc.base,
-                                                                         sc.rr_e, sc.rr_slot, sc.rr_q);
+                                                                         sc.rr_e, sc.rr_slot, sc.rr_q, sc.rr_stop);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
         *where = "reroute offsets";

@@ -72,7 +72,7 @@ static bool layout(const moe_params& p, moe_ws_layout& L, int& n_tiles, int& til
     // the per-expert probability sums and (rerouting) the rounds' state
     L.scratch = take(align_up(E * (size_t)std::max(n_tiles, 1) * 4 + (E + 1) * 4 + E * 4, 256) +
                      align_up((size_t)p.N * E * 4, 256) + align_up((3 * E + 1) * 4, 256) + align_up(2 * Nk * 4, 256) +
-                     align_up(E * 4, 256) + (rr ? align_up(2 * Nk * 4 + (size_t)p.N * 4, 256) : 0) +
+                     align_up(E * 4, 256) + (rr ? align_up(2 * Nk * 4 + (size_t)p.N * 4 + 16, 256) : 0) +
                      align_up(2 * E * 4, 256));
     L.total = off;
     return true;
@@ -117,8 +117,9 @@ bool make_view(const moe_params& p, void* ws, WsView& v) {
         v.scratch.rr_q = reinterpret_cast<int32_t*>(rq);
         v.scratch.rr_offer = v.scratch.rr_q + Nk;
         v.scratch.rr_next = v.scratch.rr_offer + Nk;
+        v.scratch.rr_stop = v.scratch.rr_next + p.N;
         const bool rr = p.reject_policy == MOE_REJECT_REROUTE;
-        char* ep = rq + (rr ? align_up(2 * Nk * 4 + (size_t)p.N * 4, 256) : 0);
+        char* ep = rq + (rr ? align_up(2 * Nk * 4 + (size_t)p.N * 4 + 16, 256) : 0);
         v.scratch.ep_dest = reinterpret_cast<int32_t*>(ep);
         v.scratch.ep_recv_base = v.scratch.ep_dest + p.E_r;
     }

@@ -62,6 +62,7 @@ struct Scratch {
     int32_t* rr_q;        // [N k] candidate index used
     int32_t* rr_offer;    // [N k] candidate index offered in the current round, -1
     int32_t* rr_next;     // [N] next unused candidate of each token
+    int32_t* rr_stop;     // [1] set once a round made no offer
     // expert parallelism: position of this rank's first row of each expert in
     // its owner's buffer, and (receiving side) source-major row starts [R][El]
     int32_t* ep_dest;     // [E]
