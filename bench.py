@@ -660,11 +660,11 @@ def run_gpu(args):
 
 
 def backward_kernels(w: si.Workload) -> int:
-    """Kernels one moe_backward launches: tables (4), scores (1), weight
-    transposes (3), dY gather (1), z / u / W_d^T dY / dx-row GEMMs (4),
-    SwiGLU backward (1), router (1), router contractions (2, plus the slice
-    sum when dW_r = dG^T X is split over the tokens), db (2), dx (1), row
-    transposes (5), weight-gradient prefixes (2) and GEMMs (3); the shared
+    """Kernels one moe_backward launches: offsets check (1), tables (5), scores
+    (1), dY gather (1), z / u / W_d^T dY / dx-row GEMMs (4; W_d, W_g, W_u read
+    as stored), SwiGLU backward (1), router (1), router contractions (2, plus
+    the slice sum when dW_r = dG^T X is split over the tokens), db (2), dx (1),
+    row transposes (5), weight-gradient prefixes (2) and GEMMs (3); the shared
     expert adds 19."""
     tiles = ((w.E + 63) // 64) * ((w.d + 63) // 64)
     sms = 148
@@ -672,8 +672,8 @@ def backward_kernels(w: si.Workload) -> int:
     if w.dtype != si.DT_BF16:
         # fp32: scores, two gathers, SwiGLU, router chain, dx; per touched expert
         # z, u, W_d^T dY, two dx-row and three weight-gradient contractions
-        return 1 + 2 + 1 + (3 + 2 + (1 if slices > 1 else 0)) + 1 + 8 * w.E + (8 if w.d_f_shared else 0)
-    return 30 + (1 if slices > 1 else 0) + (19 if w.d_f_shared else 0)
+        return 1 + 1 + 2 + 1 + (3 + 2 + (1 if slices > 1 else 0)) + 1 + 8 * w.E + (8 if w.d_f_shared else 0)
+    return 29 + (1 if slices > 1 else 0) + (19 if w.d_f_shared else 0)
 
 
 def run_gpu_backward(args):

@@ -19,11 +19,13 @@
 // dW_r = dG^T X, db = column sums of dG (fp32 CUDA-core kernels: E_r is
 // small).  dx gathers the expert rows' dx_perm in token order.
 //
-// Layout choices for the tcgen05 GEMM (out = A B^T, both operands K-major):
-// the row-grouped contractions run on the grouped kernel in store mode with
-// the dimensions relabelled (its "d_f" is K, its "d" the output width), which
-// needs W_d^T [E, d_f, d] and [W_g^T | W_u^T] [E, d, 2 d_f]: both are written
-// once per call by a batched transpose.  The weight gradients contract over an
+// Layout choices for the tcgen05 GEMM (out = A B^T, A K-major): z and u run
+// on the grouped kernel in store mode with the dimensions relabelled (its
+// "d_f" is K, its "d" the output width; W_g, W_u are K-major as stored); W_d^T
+// dY and [dz | du] [W_g ; W_u] read W_d, W_g and W_u as stored, as MN-major B
+// operands (launch_tc_store_bmn), so no weight is transposed.  The shared
+// expert's dense contractions still read transposed copies of its three
+// matrices (one expert: small).  The weight gradients contract over an
 // expert's rows, so their operands are transposed into blocks [E][C][Kmax]
 // (expert e's C rows hold its R_e row values as columns, zero-padded to whole
 // 64-wide K blocks; Kmax = the largest padded R_e, from the host offsets).
@@ -611,7 +613,7 @@ cudaError_t simt_gemm_sliced(int64_t M, int64_t N, int64_t K, const TA* A, int64
 // ---------------------------------------------------------------------------
 struct BwdLayout {
     size_t tstart, nkb, mt_start, offs_d, offs_f, mt_d, mt_f, sh_off, sh_tstart, sh_nkb, counters;
-    size_t logits, dG, part, part_db, dwc, doP, Wt_d, Wt_gu, dYp, Z, U, Gd, dzu, dxp, doT, xT, hT, dzT, duT;
+    size_t logits, dG, part, part_db, dwc, doP, mt128, dYp, Z, U, Gd, dzu, dxp, doT, xT, hT, dzT, duT;
     size_t dYs, Zs, Us, Gs, dzus, dxs, WsT_d, WsT_gu, dYsT, xsT, hsT, dzsT, dusT;
     int64_t Kmax, Kmax_sh;
     size_t total;
@@ -672,8 +674,7 @@ BwdLayout bwd_layout(const moe_params& p, int64_t Kmax) {
     L.part_db = take((size_t)kMaxSlices * E * 4);
     L.dwc = take(rows * 4);
     L.doP = take((1 - tb) * rows * d * 4);
-    L.Wt_d = take(tb * E * df * d * 2);
-    L.Wt_gu = take(tb * E * d * 2 * df * 2);
+    L.mt128 = take((E + 1) * 4);  // 128-row tile prefix for the MN-major weight contractions
     L.dYp = take(rows * d * es);
     L.Z = take(rows * df * 4);
     L.U = take(rows * df * 4);
@@ -962,7 +963,8 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     float* logits = F32(L.logits);
     float* dG = F32(L.dG);
     float* dwc = F32(L.dwc);
-    bf16 *Wt_d = B16(L.Wt_d), *Wt_gu = B16(L.Wt_gu), *dYp = B16(L.dYp), *dzu = B16(L.dzu);
+    bf16 *dYp = B16(L.dYp), *dzu = B16(L.dzu);
+    int32_t* mt128 = I32(L.mt128);
     float *Z = F32(L.Z), *U = F32(L.U), *Gd = F32(L.Gd), *dxp = F32(L.dxp);
     bf16 *doT = B16(L.doT), *xT = B16(L.xT), *hT = B16(L.hT), *dzT = B16(L.dzT), *duT = B16(L.duT);
     const bf16* xp = static_cast<const bf16*>(v.x_perm);
@@ -982,6 +984,7 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     bwd_strided_offsets_kernel<<<1, 256, 0, st>>>((int)E, (int32_t)df, offs_f);
     if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "tables");
     e = launch_mtile_prefix((int)E, tc_tile_rows(*p), v.offsets, mt_start, st);
+    if (e == cudaSuccess) e = launch_mtile_prefix((int)E, 128, v.offsets, mt128, st);
     if (e != cudaSuccess) return bwd_fail(e, "tables");
     // router scores (bias added in the router kernel): tensor cores when the
     // fp32 epilogue's 4-column groups tile E_r, else the CUDA-core GEMM
@@ -991,17 +994,10 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
         e = simt_gemm<bf16, bf16>(N, E, d, static_cast<const bf16*>(x), d, 1, static_cast<const bf16*>(W_r), d, 1,
                                   logits, E, st);
     if (e != cudaSuccess) return bwd_fail(e, "scores");
-    // W_d^T [E, d_f, d] and [W_g^T | W_u^T] [E, d, 2 d_f]
-    bwd_batched_transpose_kernel<<<dim3((unsigned)((d + kTT - 1) / kTT), (unsigned)((df + kTT - 1) / kTT), (unsigned)E),
-                                   256, 0, st>>>(static_cast<const bf16*>(W_d), d, df, Wt_d, d, df * d);
-    bwd_batched_transpose_kernel<<<dim3((unsigned)((df + kTT - 1) / kTT), (unsigned)((d + kTT - 1) / kTT), (unsigned)E),
-                                   256, 0, st>>>(static_cast<const bf16*>(W_g), df, d, Wt_gu, 2 * df, d * 2 * df);
-    bwd_batched_transpose_kernel<<<dim3((unsigned)((df + kTT - 1) / kTT), (unsigned)((d + kTT - 1) / kTT), (unsigned)E),
-                                   256, 0, st>>>(static_cast<const bf16*>(W_u), df, d, Wt_gu + df, 2 * df, d * 2 * df);
     // dY rows of the accepted paths, bf16
     bwd_gather_dy_kernel<bf16><<<grid_for(8, rows), 256, 0, st>>>(dY, d, v.slot_token, n_rows, 0, rows, N, nullptr,
                                                                   dYp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "transposes");
+    if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "dY rows");
 
     // row-grouped contractions on the grouped tcgen05 kernel (store mode):
     // its output width is q.d and its K is q.d_f
@@ -1018,20 +1014,17 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     e = launch_tc_down(q, DOWN_STORE, N, xp, nullptr, v.offsets, mt_start, W0, nullptr, nullptr, nullptr, U, counters,
                        st, &status);
     if (e != cudaSuccess) return bwd_fail(e, "u (tcgen05)");
-    W0.W_d = Wt_d;
-    e = launch_tc_down(q, DOWN_STORE, N, dYp, nullptr, v.offsets, mt_start, W0, nullptr, nullptr, nullptr, Gd,
-                       counters, st, &status);
+    // W_d^T dY: W_d [E, d, d_f] read as stored (MN-major B operand)
+    e = launch_tc_store_bmn(*p, df, d, dYp, d, W_d, nullptr, 0, nullptr, v.offsets, mt128, Gd, counters, st,
+                            &status);
     if (e != cudaSuccess) return bwd_fail(e, "W_d^T dY (tcgen05)");
     bwd_swiglu_kernel<bf16, bf16><<<grid_for(8, rows), 256, 0, st>>>(Z, U, Gd, hp, df, v.slot_w, n_rows, 0, rows, dzu,
                                                                      dwc);
     if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "SwiGLU backward");
-    moe_params q2 = *p;
-    q2.d_f_shared = 0;
-    q2.d = (int32_t)d;
-    q2.d_f = (int32_t)(2 * df);
-    W0.W_d = Wt_gu;
-    e = launch_tc_down(q2, DOWN_STORE, N, dzu, nullptr, v.offsets, mt_start, W0, nullptr, nullptr, nullptr, dxp,
-                       counters, st, &status);
+    // dx rows = dz W_g + du W_u: W_g, W_u [E, d_f, d] read as stored (MN-major
+    // B operands), dz and du the two halves of each [dz | du] row
+    e = launch_tc_store_bmn(*p, d, df, dzu, 2 * df, W_g, dzu + df, 2 * df, W_u, v.offsets, mt128, dxp, counters,
+                            st, &status);
     if (e != cudaSuccess) return bwd_fail(e, "dx rows (tcgen05)");
 
     const bf16* xb = static_cast<const bf16*>(x);

@@ -10,15 +10,16 @@
 // waiting:
 //   hist   one CTA per tile of tokens counts its requests per expert
 //          (shared-memory atomics; order does not matter for counts);
-//   scan   one CTA turns the [E][tiles] counts into exclusive per-tile bases
-//          (a warp per expert, each lane a contiguous run of tiles), then scans the accepted
-//          counts min(L_e, C) over experts into row offsets and the M-tile
-//          prefix used by the grouped GEMMs, and writes the statistics;
+//   scan   a warp per expert turns its row of the [E][tiles] counts into
+//          exclusive per-tile bases (each lane a contiguous run of tiles);
+//          the block that finishes last (a ticket, no waiting) scans the
+//          accepted counts min(L_e, C) over experts into row offsets and the
+//          M-tile prefix used by the grouped GEMMs, and writes the statistics;
 //   assign one warp per tile walks its requests in token order, 32 at a
 //          time; __match_any_sync groups equal experts so a lane's slot is
 //          base + running count + its rank among earlier equal lanes.
-// gather then copies x rows into the per-expert row buffer with 16-byte
-// vector loads (HBM-bound, coalesced along each row).
+// gather then copies x rows into the per-expert row buffer, a warp per row
+// with 16-byte vector loads (HBM-bound, coalesced along each row).
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -58,6 +59,10 @@ __global__ void hist_kernel(const int32_t* __restrict__ ids, int64_t N, int k, i
                             unsigned long long* counters) {
     extern __shared__ int h[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {  // the scans that follow count finished blocks from 0
+        counters[CNT_SCAN_TICKET] = 0;
+        counters[CNT_SCAN_ANY] = 0;
+    }
     __syncthreads();
     const int64_t t0 = (int64_t)blockIdx.x * tile_tokens;
     const int64_t t1 = min64(N, t0 + tile_tokens);
@@ -113,40 +118,96 @@ __device__ void tile_scan(int32_t* __restrict__ hist, int n_tiles, int E, int* s
     }
 }
 
+// Expert e's per-tile request counts (one row of hist) become exclusive bases
+// in place, by one warp: each lane sums a contiguous run of tiles (independent
+// loads), one warp scan turns the sums into run bases, and each lane rewrites
+// its run.  Returns the expert's total in every lane.
+__device__ int warp_tile_scan(int32_t* __restrict__ row, int n_tiles, int lane) {
+    const int seg = (n_tiles + 31) / 32;
+    const int i0 = min(n_tiles, lane * seg), i1 = min(n_tiles, i0 + seg);
+    int sum = 0;
+#pragma unroll 8
+    for (int i = i0; i < i1; ++i) sum += row[i];
+    const int inc = warp_incl_scan(sum, lane);
+    int run = inc - sum;
+#pragma unroll 8
+    for (int i = i0; i < i1; ++i) {
+        const int v = row[i];
+        row[i] = run;
+        run += v;
+    }
+    return __shfl_sync(0xffffffffu, inc, 31);
+}
+
+// True in the block that finishes last (each block fences its global writes
+// before taking a ticket, so the last one sees them all).  No block waits for
+// another.  The last block puts the ticket back to 0 for the next launch.
+__device__ bool last_block_done(unsigned long long* ticket) {
+    __shared__ int last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        last = atomicAdd(ticket, 1ull) == (unsigned long long)gridDim.x - 1;
+        if (last) *ticket = 0;
+    }
+    __syncthreads();
+    if (last) __threadfence();
+    return last;
+}
+
+constexpr int kScanWarps = 8;  // experts per scan block (one warp each)
+
+// Per-tile bases (one warp per expert, kScanWarps experts per block), then,
+// in the block that finishes last, the scans over experts: accepted counts
+// min(L_e, C) into row offsets, M-tiles into the prefix used by the grouped
+// GEMMs, requests into all_offsets (acceptance by weight), and the
+// statistics.
 __global__ void scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int64_t C, int bm,
                             int32_t* __restrict__ L, int32_t* __restrict__ acc,
                             int32_t* __restrict__ offsets, int32_t* __restrict__ mt_start,
                             int32_t* __restrict__ all_offsets, unsigned long long* counters) {
-    __shared__ int sL[kMaxExperts];
     __shared__ int warp_tot[33];
-    tile_scan(hist, n_tiles, E, sL);
-    __syncthreads();
-    // one thread per expert (blockDim.x >= E)
-    const int e = threadIdx.x;
-    const int Le = e < E ? sL[e] : 0;
-    const int a = e < E ? (int)min64(Le, C) : 0;
-    const int mt = (a + bm - 1) / bm;
-    int tot_a, tot_mt, tot_L, tot_O;
-    const int ex_a = block_excl_scan(a, warp_tot, &tot_a);
-    const int ex_mt = block_excl_scan(mt, warp_tot, &tot_mt);
-    const int ex_L = block_excl_scan(Le, warp_tot, &tot_L);
-    block_excl_scan(Le > C ? (int)(Le - C) : 0, warp_tot, &tot_O);
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * kScanWarps + (threadIdx.x >> 5);
     if (e < E) {
-        L[e] = Le;
-        acc[e] = a;
-        offsets[e] = ex_a;
-        mt_start[e] = ex_mt;
-        if (all_offsets) all_offsets[e] = ex_L;
-        atomicMax(counters + CNT_L_MAX, (unsigned long long)Le);
+        const int tot = warp_tile_scan(hist + (int64_t)e * n_tiles, n_tiles, lane);
+        if (lane == 0) L[e] = tot;
     }
+    if (!last_block_done(counters + CNT_SCAN_TICKET)) return;
+    int car_a = 0, car_mt = 0, car_L = 0, car_O = 0, lmax = 0;
+    for (int e0 = 0; e0 < E; e0 += blockDim.x) {  // uniform over the block
+        const int ex = e0 + (int)threadIdx.x;
+        const int Le = ex < E ? __ldcg(L + ex) : 0;
+        const int a = (int)min64(Le, C);
+        const int mt = (a + bm - 1) / bm;
+        int t_a, t_mt, t_L, t_O;
+        const int ex_a = block_excl_scan(a, warp_tot, &t_a);
+        const int ex_mt = block_excl_scan(mt, warp_tot, &t_mt);
+        const int ex_L = block_excl_scan(Le, warp_tot, &t_L);
+        block_excl_scan(Le > C ? (int)(Le - C) : 0, warp_tot, &t_O);
+        if (ex < E) {
+            acc[ex] = a;
+            offsets[ex] = car_a + ex_a;
+            mt_start[ex] = car_mt + ex_mt;
+            if (all_offsets) all_offsets[ex] = car_L + ex_L;
+        }
+        lmax = max(lmax, Le);
+        car_a += t_a;
+        car_mt += t_mt;
+        car_L += t_L;
+        car_O += t_O;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    if (lane == 0 && lmax > 0) atomicMax(counters + CNT_L_MAX, (unsigned long long)lmax);
     if (threadIdx.x == 0) {
-        if (all_offsets) all_offsets[E] = tot_L;
-        offsets[E] = tot_a;
-        mt_start[E] = tot_mt;
-        counters[CNT_REQUESTED] = (unsigned long long)tot_L;
-        counters[CNT_ACCEPTED] = (unsigned long long)tot_a;
-        counters[CNT_REJECTED] = (unsigned long long)(tot_L - tot_a);
-        counters[CNT_O] = (unsigned long long)tot_O;
+        if (all_offsets) all_offsets[E] = car_L;
+        offsets[E] = car_a;
+        mt_start[E] = car_mt;
+        counters[CNT_REQUESTED] = (unsigned long long)car_L;
+        counters[CNT_ACCEPTED] = (unsigned long long)car_a;
+        counters[CNT_REJECTED] = (unsigned long long)(car_L - car_a);
+        counters[CNT_O] = (unsigned long long)car_O;
         counters[CNT_C] = (unsigned long long)C;
     }
 }
@@ -505,23 +566,29 @@ __global__ void reroute_offer_kernel(const int32_t* __restrict__ ids, const int3
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)e * n_tiles + blockIdx.x] = h[e];
 }
 
+// One rerouting round's offers per expert (one warp each): per-tile bases of
+// the offers, base[e] = slots taken before the round, acc[e] grows by the
+// offers it accepts.  The block that finishes last sets rr_stop when no
+// expert received an offer (the later rounds then return at once).
 __global__ void reroute_scan_kernel(int32_t* __restrict__ hist, int n_tiles, int E, int64_t C,
                                     int32_t* __restrict__ acc, int32_t* __restrict__ base,
-                                    int32_t* __restrict__ rr_stop) {
-    __shared__ int sL[kMaxExperts];
-    __shared__ int any;
+                                    int32_t* __restrict__ rr_stop, unsigned long long* counters) {
     if (*rr_stop) return;  // uniform: every thread reads the same flag
-    if (threadIdx.x == 0) any = 0;
-    tile_scan(hist, n_tiles, E, sL);
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        const int a = acc[e];
-        base[e] = a;
-        acc[e] = (int)min64((int64_t)a + sL[e], C);
-        if (sL[e]) any = 1;
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * kScanWarps + (threadIdx.x >> 5);
+    if (e < E) {
+        const int offers = warp_tile_scan(hist + (int64_t)e * n_tiles, n_tiles, lane);
+        if (lane == 0) {
+            const int a = acc[e];
+            base[e] = a;
+            acc[e] = (int)min64((int64_t)a + offers, C);
+            if (offers) atomicAdd(counters + CNT_SCAN_ANY, 1ull);
+        }
     }
-    __syncthreads();
-    if (threadIdx.x == 0 && !any) *rr_stop = 1;
+    if (!last_block_done(counters + CNT_SCAN_TICKET)) return;
+    if (threadIdx.x == 0) {
+        if (atomicExch(counters + CNT_SCAN_ANY, 0ull) == 0ull) *rr_stop = 1;
+    }
 }
 
 __global__ void reroute_assign_kernel(const int32_t* __restrict__ rr_offer, const int32_t* __restrict__ cand,
@@ -646,15 +713,33 @@ __global__ void reroute_rows_kernel(const int32_t* __restrict__ ids, const float
     }
 }
 
+// One warp copies a row of row_vec 16-byte words; four loads per lane are in
+// flight before their stores, so that each SM keeps enough bytes outstanding
+// to draw the HBM rate.
+__device__ __forceinline__ void copy_row_warp(const uint4* __restrict__ src, uint4* __restrict__ dst, int row_vec,
+                                              int lane) {
+    int i = lane;
+    for (; i + 96 < row_vec; i += 128) {
+        const uint4 v0 = src[i], v1 = src[i + 32], v2 = src[i + 64], v3 = src[i + 96];
+        dst[i] = v0;
+        dst[i + 32] = v1;
+        dst[i + 64] = v2;
+        dst[i + 96] = v3;
+    }
+    for (; i < row_vec; i += 32) dst[i] = src[i];
+}
+
+constexpr int kGatherThreads = 256;
+
 __global__ void gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ x_perm,
                               const int32_t* __restrict__ slot_token,
                               const int32_t* __restrict__ offsets, int E, int row_vec) {
     const int total = offsets[E];
-    for (int r = blockIdx.x; r < total; r += gridDim.x) {
+    const int lane = threadIdx.x & 31;
+    const int wpb = blockDim.x >> 5;
+    for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < total; r += gridDim.x * wpb) {
         const int64_t t = slot_token[r];
-        const uint4* src = x + t * row_vec;
-        uint4* dst = x_perm + (int64_t)r * row_vec;
-        for (int i = threadIdx.x; i < row_vec; i += blockDim.x) dst[i] = src[i];
+        copy_row_warp(x + t * row_vec, x_perm + (int64_t)r * row_vec, row_vec, lane);
     }
 }
 
@@ -662,11 +747,10 @@ __global__ void gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ x
 // regrouping of exchanged rows)
 __global__ void gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ index, int64_t n,
                                    int row_vec, uint4* __restrict__ dst) {
-    for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
-        const uint4* a = src + (int64_t)index[r] * row_vec;
-        uint4* b = dst + r * row_vec;
-        for (int i = threadIdx.x; i < row_vec; i += blockDim.x) b[i] = a[i];
-    }
+    const int lane = threadIdx.x & 31;
+    const int wpb = blockDim.x >> 5;
+    for (int64_t r = (int64_t)blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += (int64_t)gridDim.x * wpb)
+        copy_row_warp(src + (int64_t)index[r] * row_vec, dst + r * row_vec, row_vec, lane);
 }
 
 __global__ void combine_kernel(const float* __restrict__ H, const int32_t* __restrict__ offsets,
@@ -726,8 +810,9 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
     // one thread per expert (E <= kMaxExperts = 1024)
     *where = "scan";
     const bool by_weight = p.accept_order == MOE_ACCEPT_WEIGHT;
-    scan_kernel<<<1, 1024, 0, st>>>(sc.hist, n_tiles, E, C, bm, L, acc, offsets, sc.mt_start,
-                                    by_weight ? sc.all_offsets : nullptr, counters);
+    const int scan_blocks = (E + kScanWarps - 1) / kScanWarps;
+    scan_kernel<<<scan_blocks, 32 * kScanWarps, 0, st>>>(sc.hist, n_tiles, E, C, bm, L, acc, offsets, sc.mt_start,
+                                                         by_weight ? sc.all_offsets : nullptr, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int renorm = p.reject_policy == MOE_REJECT_RENORM;
     const bool reroute = p.reject_policy == MOE_REJECT_REROUTE;
@@ -754,7 +839,8 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
                                                                          sc.rr_next, sc.rr_offer, sc.hist, sc.rr_stop);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             *where = "reroute scan";
-            reroute_scan_kernel<<<1, 1024, 0, st>>>(sc.hist, n_tiles, E, C, acc, sc.base, sc.rr_stop);
+            reroute_scan_kernel<<<scan_blocks, 32 * kScanWarps, 0, st>>>(sc.hist, n_tiles, E, C, acc, sc.base,
+                                                                          sc.rr_stop, counters);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             *where = "reroute assign";
             reroute_assign_kernel<<<n_tiles, 32, sizeof(int) * E, st>>>(sc.rr_offer, sc.cand, X, p.N, k, E, C,
@@ -800,8 +886,8 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
         *where = "gather";
         const int row_vec = (int)(p.d * esize(p.dtype) / 16);
         const int64_t rows = p.N * p.k;
-        const int blocks = (int)min64(rows, (int64_t)num_sms() * 8);
-        gather_kernel<<<blocks, 128, 0, st>>>(static_cast<const uint4*>(x),
+        const int blocks = (int)min64((rows + kGatherThreads / 32 - 1) / (kGatherThreads / 32), (int64_t)num_sms() * 8);
+        gather_kernel<<<blocks, kGatherThreads, 0, st>>>(static_cast<const uint4*>(x),
                                               static_cast<uint4*>(x_perm), slot_token, offsets, E,
                                               row_vec);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -843,8 +929,8 @@ cudaError_t launch_dispatch_ranked(const moe_params& p, int64_t C, int bm, const
         *where = "gather";
         const int row_vec = (int)(p.d * esize(p.dtype) / 16);
         const int64_t rows = p.N * p.k;
-        const int blocks = (int)min64(rows, (int64_t)num_sms() * 8);
-        gather_kernel<<<blocks, 128, 0, st>>>(static_cast<const uint4*>(x),
+        const int blocks = (int)min64((rows + kGatherThreads / 32 - 1) / (kGatherThreads / 32), (int64_t)num_sms() * 8);
+        gather_kernel<<<blocks, kGatherThreads, 0, st>>>(static_cast<const uint4*>(x),
                                               static_cast<uint4*>(x_perm), slot_token, offsets, E,
                                               row_vec);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -854,8 +940,10 @@ cudaError_t launch_dispatch_ranked(const moe_params& p, int64_t C, int bm, const
 
 cudaError_t launch_gather_rows(const void* src, const int32_t* index, int64_t n_rows, int64_t row_bytes, void* dst,
                                cudaStream_t st) {
-    const int blocks = (int)min64(n_rows, (int64_t)num_sms() * 8);
-    gather_rows_kernel<<<blocks, 128, 0, st>>>(static_cast<const uint4*>(src), index, n_rows, (int)(row_bytes / 16),
+    if (n_rows <= 0) return cudaSuccess;
+    const int blocks =
+        (int)min64((n_rows + kGatherThreads / 32 - 1) / (kGatherThreads / 32), (int64_t)num_sms() * 8);
+    gather_rows_kernel<<<blocks, kGatherThreads, 0, st>>>(static_cast<const uint4*>(src), index, n_rows, (int)(row_bytes / 16),
                                                static_cast<uint4*>(dst));
     return cudaGetLastError();
 }

@@ -93,6 +93,10 @@ struct TcArgs {
     int64_t zero_n4;          // its size in float4
     int ks;                   // K splits per output tile (partial sums reduced with red.add)
     const int32_t* grp_nkb;   // [E] K blocks of each routed group (null: nkb_r for all; ks must be 1)
+    int b_mn;                 // 1: B is read MN-major (single-CTA store mode): per K block,
+                              //    four 64 x 64 boxes of a [K rows, N cols] matrix
+    int nkb_split;            // b_mn: K blocks >= nkb_split take A from mA_h and B from mB1
+                              //    (a second K segment); 0: one segment
     unsigned long long* counters;
 };
 
@@ -224,6 +228,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
     return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major operand, 128-byte swizzle:
+// each 128-byte row holds 64 consecutive N (or M) elements of one K index,
+// 8-row atoms of 1024 bytes follow each other along K (SBO = 1024 bytes), and
+// the next 64 N elements start 8 KB further (LBO = 8 KB: one 64 x 64 box).
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(8192 >> 4) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
 // N = 256, M = 128.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -236,6 +254,19 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint6
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+// the same MMA with B MN-major (instruction descriptor bit 16)
+constexpr uint32_t kIdescBmn = kIdesc | (1u << 16);
+
+__device__ __forceinline__ void umma_bf16_bmn(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(kIdescBmn), "r"(accumulate)
         : "memory");
 }
 
@@ -670,6 +701,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         } else {
                             tma_load_2d_pair(sb, pb1, fb, kb * BK, b_row1);
                         }
+                    } else if (a.b_mn) {
+                        // B MN-major: rows of the group's [K, N] matrix; a second
+                        // K segment (nkb_split) takes A from mA_h and B from mB1
+                        const bool seg1 = a.nkb_split > 0 && kb >= a.nkb_split;
+                        const int kbs = seg1 ? kb - a.nkb_split : kb;
+                        const CUtensorMap* pbm = seg1 ? &mB1 : &mB0;
+                        const int brow = ti.g * a.b_rows_r + kbs * BK;
+                        mbar_expect_tx(&full[stage], SBYTES);
+                        tma_load_2d(sa, seg1 ? &mA_h : pa, &full[stage], kbs * BK, a_row);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            tma_load_2d(sb + c * (B_HALF_BYTES / 2), pbm, &full[stage], ti.n_tile * 256 + c * BK,
+                                        brow);
                     } else {
                         mbar_expect_tx(&full[stage], SBYTES);
                         tma_load_2d(sa, pa, &full[stage], kb * BK, a_row);
@@ -714,15 +758,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t sa = smem_u32(stage_base + stage * SBYTES);
                     const uint32_t sb = sa + A_BYTES;
                     const uint64_t ad = smem_desc_sw128(sa);
-                    const uint64_t bd = smem_desc_sw128(sb);
+                    if (!PAIR && a.b_mn) {
+                        // B MN-major: 16 K indices are 16 rows of 128 bytes (2 KB)
+                        const uint64_t bd = smem_desc_mn_sw128(sb);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        // advance 16 elements (32 bytes) along K inside the swizzled row
-                        const uint32_t accum = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
-                        if (PAIR)
-                            umma_bf16_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc_pair,
-                                           accum);
-                        else umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), accum);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            umma_bf16_bmn(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 128),
+                                          (kb > ti.kb0 || kk > 0) ? 1u : 0u);
+                    } else {
+                        const uint64_t bd = smem_desc_sw128(sb);
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            // advance 16 elements (32 bytes) along K inside the swizzled row
+                            const uint32_t accum = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
+                            if (PAIR)
+                                umma_bf16_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc_pair,
+                                               accum);
+                            else umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), accum);
+                        }
                     }
                     if (PAIR) umma_commit_pair_both(&empty[stage]);
                     else umma_commit(&empty[stage]);
@@ -844,12 +897,14 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// 2-D bf16 row-major matrix [rows, cols] read in boxes of box_rows rows x 64 columns
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows = 128) {
+// 2-D bf16 row-major matrix [rows, cols] (row stride ld elements, default
+// cols) read in boxes of box_rows rows x 64 columns
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows = 128,
+              uint64_t ld = 0) {
     auto enc = get_encode();
     if (!enc || rows == 0 || cols == 0) return false;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
+    cuuint64_t strides[1] = {(ld ? ld : cols) * 2};
     cuuint32_t box[2] = {BK, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
@@ -1081,6 +1136,49 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
     if (pair)
         return launch_tc<EPI_STORE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles, st);
     return launch_tc<EPI_STORE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles, st);
+}
+
+cudaError_t launch_tc_store_bmn(const moe_params& p, int64_t n_out, int64_t K, const void* A0, int64_t ldA0,
+                                const void* B0, const void* A1, int64_t ldA1, const void* B1,
+                                const int32_t* offsets, const int32_t* mt_start128, float* out,
+                                unsigned long long* counters, cudaStream_t st, int* status) {
+    *status = MOE_OK;
+    CUtensorMap mA, mA2, mB0, mB1;
+    const uint64_t rows = (uint64_t)(p.N * p.k);
+    const bool two = A1 && B1;
+    bool ok = make_map(&mA, A0, rows, (uint64_t)K, 128, (uint64_t)ldA0) &&
+              make_map(&mB0, B0, (uint64_t)p.E_r * K, (uint64_t)n_out, 64);
+    if (ok && two)
+        ok = make_map(&mA2, A1, rows, (uint64_t)K, 128, (uint64_t)ldA1) &&
+             make_map(&mB1, B1, (uint64_t)p.E_r * K, (uint64_t)n_out, 64);
+    if (!two) {
+        mA2 = mA;
+        mB1 = mB0;
+    }
+    if (!ok) {
+        *status = MOE_ERR_CUDA;
+        return cudaErrorInvalidValue;
+    }
+    const int nkb = (int)((K + BK - 1) / BK);
+    TcArgs a{};
+    a.mt_start = mt_start128;
+    a.offsets = offsets;
+    a.E = p.E_r;
+    a.nt_r = (int)((n_out + BN - 1) / BN);
+    a.nkb_r = two ? 2 * nkb : nkb;
+    a.b_rows_r = (int)K;
+    a.b_mn = 1;
+    a.nkb_split = two ? nkb : 0;
+    a.n_valid_r = (int)n_out;
+    a.out = out;
+    a.ld_out = (int)n_out;
+    a.max_rows = (int)(p.N * p.k);
+    a.n_tokens = (int)p.N;
+    a.has_routed = 1;
+    a.ks = 1;
+    a.counters = counters;
+    const int64_t max_tiles = routed_mtile_bound(p, 128) * a.nt_r;
+    return launch_tc<EPI_STORE, false>(mA, mB0, mB1, mA, mB0, mB1, mA2, mA, a, max_tiles, st);
 }
 
 cudaError_t launch_tc_dense(int64_t M, int64_t Nc, int64_t K, const void* A, const void* B, float* out,

@@ -34,6 +34,8 @@ enum Counter {
     CNT_DEVICE_ERROR = 10,  // bit flags, see DevErr
     CNT_N_GROUP = 11,       // tokens of the whole routing group (sharded runs; 0 = N)
     CNT_REROUTED = 12,      // rejected paths served by a rerouted expert
+    CNT_SCAN_TICKET = 13,   // dispatch scans: blocks finished (reset by hist_kernel and the last block)
+    CNT_SCAN_ANY = 14,      // rerouting scan: experts that received offers this round
     CNT_COUNT = 16
 };
 
@@ -157,6 +159,15 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
                            const float* slot_w, float* Y, float* H_out,
                            unsigned long long* counters, cudaStream_t st, int* status,
                            const int32_t* grp_nkb = nullptr);
+// out[r, :] = A0[r, :K] B0[e] (+ A1[r, :K] B1[e]) for the rows r of each group e
+// (offsets), with B0, B1 [E_r][K][n_out] read as stored (MN-major operands:
+// no transposed copies); A rows K-major with leading dimensions ldA0 / ldA1;
+// fp32 out [N k, n_out].  Single-CTA 128-row tiles: mt_start128 is the
+// 128-row tile prefix of offsets.
+cudaError_t launch_tc_store_bmn(const moe_params& p, int64_t n_out, int64_t K, const void* A0, int64_t ldA0,
+                                const void* B0, const void* A1, int64_t ldA1, const void* B1,
+                                const int32_t* offsets, const int32_t* mt_start128, float* out,
+                                unsigned long long* counters, cudaStream_t st, int* status);
 // rows of one output tile of the tcgen05 grouped GEMMs for these params
 // (256 when CTA pairs are used, else 128): the dispatch's M-tile prefix unit
 int tc_tile_rows(const moe_params& p);
