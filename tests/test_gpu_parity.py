@@ -51,6 +51,9 @@ SMALL = {
     "wide_router_f32": W["switch_top1_f32"].scaled("wide_router_f32", N=200, d=64, d_f=64, E=48, k=3,
                                                    norm=si.NORM_RENORM, c=0.0),
     "odd_experts_bf16": W["mixtral_bf16"].scaled("odd_experts_bf16", N=200, d=64, d_f=64, E=34, k=3),
+    # d not a multiple of the 64-wide K block: the gate/up kernel's own row
+    # gather zero-fills the last block's columns past d (single-CTA tiles)
+    "ragged_k_bf16": W["qwen3_skew_bf16"].scaled("ragged_k_bf16", N=300, d=200, d_f=136, E=16, k=4),
     # >= 768 rows per expert: 256-row tiles on CTA pairs (ragged last pair tile)
     "pair_bf16": W["mixtral_bf16"].scaled("pair_bf16", N=1600, d=320, d_f=384, E=2, k=1),
     "pair_shared_bf16": W["mixtral_bf16"].scaled("pair_shared_bf16", N=1700, d=256, d_f=256, E=2, k=1,
