@@ -20,8 +20,11 @@
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator rows (one TMEM lane
 //              per row), then SwiGLU -> bf16 h (gate/up) or the weighted
 //              scatter-combine with 16-byte fp32 red.global.add (down), each
-//              32-column chunk transposed through a per-warp shared-memory
-//              tile so one warp instruction adds 4 rows x 128 contiguous bytes.
+//              32-column chunk transposed through a per-warp 128-byte-swizzled
+//              shared-memory tile so one warp instruction adds 4 rows x 128
+//              contiguous bytes.  Plain fp32 outputs (the store epilogue)
+//              leave that tile by TMA store, 32 rows x 32 columns at a time,
+//              when all 32 rows of the warp's slab are valid.
 // For gate/up the two B tiles are the gate and up rows of the same 128
 // output columns, so one N=256 MMA yields both and the SwiGLU is local to a
 // thread.  For the down projection they are two consecutive 128-row halves
@@ -64,8 +67,12 @@ constexpr int STAGE_BYTES = A_BYTES + 2 * B_HALF_BYTES;
 constexpr int STAGES_PAIR = 6;                            // CTA pair: A + one B half per CTA
 constexpr int STAGE_BYTES_PAIR = A_BYTES + B_HALF_BYTES;
 constexpr int NUM_THREADS = 192;
-constexpr int kStgLd = 36;  // floats per staging row (32 + 4: conflict-free 16-byte access)
-constexpr size_t kStgBytes = 4 * 32 * kStgLd * sizeof(float) + 128;  // + alignment slack
+// Per epilogue warp, a 32 x 32 fp32 staging tile (4 KB, 1024-byte aligned) in
+// the 128-byte-swizzle layout: row r at byte r * 128, its 16-byte chunk j at
+// chunk j ^ (r & 7).  Row-wise writes and 4-rows-at-a-time reads are both
+// conflict-free, and it is the layout a TMA store of a 32 x 32 fp32 box reads.
+constexpr int kStgTile = 32 * 32 * 4;
+constexpr size_t kStgBytes = 4 * kStgTile + 1024;  // + alignment slack
 constexpr int TMEM_COLS = 512;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
@@ -97,6 +104,8 @@ struct TcArgs {
                               //    four 64 x 64 boxes of a [K rows, N cols] matrix
     int nkb_split;            // b_mn: K blocks >= nkb_split take A from mA_h and B from mB1
                               //    (a second K segment); 0: one segment
+    int tma_out;              // store epilogue without K split: warp slabs whose 32 rows
+                              //    are all valid leave by TMA store (tensor map mOut)
     unsigned long long* counters;
 };
 
@@ -189,6 +198,30 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
+}
+
+// TMA store of one box from shared memory (bulk async-group completion)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// this thread's bulk stores have read their shared-memory source
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// this thread's bulk stores are complete
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// orders this thread's shared-memory writes before reads by the async proxy (TMA)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
@@ -479,7 +512,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 template <int EPI>
 __device__ __forceinline__ void epilogue_segment(const TcArgs& a, const Tile& ti, uint32_t t_row,
                                                  int lane, bool row_ok, int grow, int cb, int ob,
-                                                 int width, int up_off, float* stg) {
+                                                 int width, int up_off, float* stg, const CUtensorMap* mOut) {
     const int n_valid = ti.shared ? a.n_valid_sh : a.n_valid_r;
     if (EPI == EPI_SWIGLU) {
         const int ld = ti.shared ? a.ld_out_sh : a.ld_out;
@@ -511,10 +544,11 @@ __device__ __forceinline__ void epilogue_segment(const TcArgs& a, const Tile& ti
             }
         }
     } else {
-        // fp32 rows (combine into Y, or plain stores): each 32-column chunk is
-        // transposed through this warp's staging tile so that one warp
-        // instruction covers 4 rows x 128 contiguous bytes (8 lanes per row)
-        // instead of 32 rows x 16 bytes
+        // fp32 rows (combine into Y, or plain stores), 32 columns at a time
+        // through this warp's swizzled staging tile: each lane writes its row;
+        // then one TMA store takes the 32 x 32 box (store epilogue, every row
+        // of the warp's slab valid), or each warp instruction covers 4 rows x
+        // 128 contiguous bytes (8 lanes per row) instead of 32 rows x 16 bytes
         float wgt = 1.f;
         long long dst_off = -1;  // element offset of this row in the destination, -1: none
         float* dst_base = EPI == EPI_COMBINE ? a.Y : static_cast<float*>(a.out);
@@ -533,25 +567,43 @@ __device__ __forceinline__ void epilogue_segment(const TcArgs& a, const Tile& ti
             }
         }
         const bool reduce = EPI == EPI_COMBINE || a.ks > 1;
+        const bool tma_path = EPI == EPI_STORE && !reduce && a.tma_out;
+        const bool use_tma = tma_path && __all_sync(0xffffffffu, dst_off >= 0);
+        const int row0 = __shfl_sync(0xffffffffu, grow, 0);
+        uint8_t* sbuf = reinterpret_cast<uint8_t*>(stg);
+        const uint32_t sbuf_u = smem_u32(sbuf);
+        const int jj = lane & 7;
 #pragma unroll 1
         for (int c = 0; c < width; c += 32) {
             uint32_t v[32];
             tmem_ld32(t_row + (uint32_t)(cb + c), v);
             tmem_ld_wait();
-            float4* my = reinterpret_cast<float4*>(stg + lane * kStgLd);
+            if (tma_path) {  // the last TMA store from the tile has read it
+                if (lane == 0) bulk_wait_read();
+                __syncwarp();
+            }
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-                my[q] = make_float4(__uint_as_float(v[4 * q]) * wgt, __uint_as_float(v[4 * q + 1]) * wgt,
-                                    __uint_as_float(v[4 * q + 2]) * wgt, __uint_as_float(v[4 * q + 3]) * wgt);
-            __syncwarp();
+                *reinterpret_cast<float4*>(sbuf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                    make_float4(__uint_as_float(v[4 * q]) * wgt, __uint_as_float(v[4 * q + 1]) * wgt,
+                                __uint_as_float(v[4 * q + 2]) * wgt, __uint_as_float(v[4 * q + 3]) * wgt);
             const int col0 = ob + c;
-            const int cg = (lane & 7) * 4;
+            if (use_tma) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                // columns past n_valid are outside the tensor map and not written
+                if (lane == 0 && col0 < n_valid) tma_store_2d(mOut, sbuf_u, col0, row0);
+                continue;
+            }
+            __syncwarp();
+            const int cg = jj * 4;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int rr = i * 4 + (lane >> 3);
                 const long long off = __shfl_sync(0xffffffffu, dst_off, rr);
                 if (off >= 0 && col0 + cg < n_valid) {
-                    const float4 val = *reinterpret_cast<const float4*>(stg + rr * kStgLd + cg);
+                    const float4 val =
+                        *reinterpret_cast<const float4*>(sbuf + rr * 128 + ((jj ^ (rr & 7)) << 4));
                     float* p = dst_base + off + col0 + cg;
                     if (reduce) red_add_v4(p, val.x, val.y, val.z, val.w);
                     else *reinterpret_cast<float4*>(p) = val;
@@ -579,7 +631,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       const __grid_constant__ CUtensorMap mB0_sh,
                       const __grid_constant__ CUtensorMap mB1_sh,
                       const __grid_constant__ CUtensorMap mA_h,
-                      const __grid_constant__ CUtensorMap mA_sh_h, const TcArgs a) {
+                      const __grid_constant__ CUtensorMap mA_sh_h,
+                      const __grid_constant__ CUtensorMap mOut, const TcArgs a) {
     constexpr int NST = PAIR ? STAGES_PAIR : STAGES;
     constexpr int SBYTES = PAIR ? STAGE_BYTES_PAIR : STAGE_BYTES;
     constexpr int TM = PAIR ? 256 : 128;
@@ -596,9 +649,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
     SchedSmem* sched = reinterpret_cast<SchedSmem*>(smem + NST * SBYTES + 256);
-    // per-epilogue-warp staging tiles [32 rows][kStgLd floats]
+    // per-epilogue-warp staging tiles (kStgTile bytes each, 1024-byte aligned)
     float* stg_all = reinterpret_cast<float*>(
-        (reinterpret_cast<uintptr_t>(sched) + sizeof(SchedSmem) + 127) & ~static_cast<uintptr_t>(127));
+        (reinterpret_cast<uintptr_t>(sched) + sizeof(SchedSmem) + 1023) & ~static_cast<uintptr_t>(1023));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
@@ -810,7 +863,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
-        float* stg = stg_all + (warp - 2) * 32 * kStgLd;
+        float* stg = stg_all + (warp - 2) * (kStgTile / 4);
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = unit; t < total_tiles; t += n_units) {
@@ -823,20 +876,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // lane r = row r; gate/up: gate columns 0-127, up 128-255
                 const bool ok = r < ti.rows;
                 if (EPI == EPI_SWIGLU)
-                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + r, 0, ti.n_tile * 128, 128, 128, stg);
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + r, 0, ti.n_tile * 128, 128, 128, stg, &mOut);
                 else
-                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + r, 0, ti.n_tile * BN, BN, 0, stg);
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + r, 0, ti.n_tile * BN, BN, 0, stg, &mOut);
             } else if (ti.rows > 128) {
                 // 256-row tile: lane r = row crank * 128 + r, all 256 columns
                 const int lr = (int)crank * 128 + r;
                 const bool ok = lr < ti.rows;
                 if (EPI == EPI_SWIGLU) {
                     // each CTA's B half is 64 gate rows then 64 up rows
-                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 0, ti.n_tile * 128, 64, 64, stg);
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 0, ti.n_tile * 128, 64, 64, stg, &mOut);
                     epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 128, ti.n_tile * 128 + 64, 64,
-                                          64, stg);
+                                          64, stg, &mOut);
                 } else {
-                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 0, ti.n_tile * BN, BN, 0, stg);
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 0, ti.n_tile * BN, BN, 0, stg, &mOut);
                 }
             } else {
                 // 128-row tile (64 rows per CTA): lanes 0-63 hold the first
@@ -846,10 +899,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const bool ok = lr < ti.rows;
                 if (EPI == EPI_SWIGLU)
                     epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 0, ti.n_tile * 128 + hf * 64, 64,
-                                          64, stg);
+                                          64, stg, &mOut);
                 else
                     epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + lr, 0, ti.n_tile * BN + hf * 128, 128,
-                                          0, stg);
+                                          0, stg, &mOut);
             }
             tc_fence_before();
             __syncwarp();
@@ -862,6 +915,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 acc_phase ^= 1u;
             }
         }
+        // this warp's TMA stores are complete before its shared memory goes away
+        if (EPI == EPI_STORE && a.tma_out && lane == 0) bulk_wait_all();
     }
 
     __syncwarp();
@@ -913,12 +968,30 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
     return r == CUDA_SUCCESS;
 }
 
+// fp32 output [rows, cols] (row stride ld elements) written by TMA stores of
+// 32 x 32 boxes from the epilogue's swizzled staging tiles; false (plain
+// stores) when the address or the stride is not 16-byte aligned
+bool make_map_out(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t ld) {
+    auto enc = get_encode();
+    if (!enc || !ptr || rows == 0 || cols == 0 || (reinterpret_cast<uintptr_t>(ptr) & 15) || (ld * 4) % 16)
+        return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 4};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // the fp32 epilogues stage through shared memory; the SwiGLU epilogue does not
 constexpr size_t smem_bytes(int epi, bool pair) {
     return 1024 + (pair ? (size_t)STAGES_PAIR * STAGE_BYTES_PAIR : (size_t)STAGES * STAGE_BYTES) + 256 +
            sizeof(SchedSmem) + (epi == EPI_SWIGLU ? 0 : kStgBytes);
 }
-static_assert(smem_bytes(EPI_COMBINE, false) <= 232448 && smem_bytes(EPI_COMBINE, true) <= 232448,
+static_assert(smem_bytes(EPI_COMBINE, false) <= 232448 && smem_bytes(EPI_COMBINE, true) <= 232448 &&
+                  smem_bytes(EPI_STORE, false) <= 232448 && smem_bytes(EPI_STORE, true) <= 232448,
               "shared memory per CTA");
 
 // mA_h / mA_sh_h: the A matrices again in 64-row boxes (CTA-pair tiles of at
@@ -926,8 +999,8 @@ static_assert(smem_bytes(EPI_COMBINE, false) <= 232448 && smem_bytes(EPI_COMBINE
 template <int EPI, bool PAIR>
 cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mB0, const CUtensorMap& mB1,
                       const CUtensorMap& mA_sh, const CUtensorMap& mB0_sh, const CUtensorMap& mB1_sh,
-                      const CUtensorMap& mA_h, const CUtensorMap& mA_sh_h, const TcArgs& a,
-                      int64_t max_tiles, cudaStream_t st) {
+                      const CUtensorMap& mA_h, const CUtensorMap& mA_sh_h, const CUtensorMap& mOut,
+                      const TcArgs& a, int64_t max_tiles, cudaStream_t st) {
     auto kern = tc_grouped_kernel<EPI, PAIR>;
     const size_t smem = smem_bytes(EPI, PAIR);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -935,7 +1008,7 @@ cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mB0, const CUten
     if (!PAIR) {
         const int grid = (int)min64(max_tiles, num_sms());
         if (grid <= 0) return cudaSuccess;
-        kern<<<grid, NUM_THREADS, smem, st>>>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, a);
+        kern<<<grid, NUM_THREADS, smem, st>>>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, mOut, a);
         return cudaGetLastError();
     }
     // clusters of two CTAs, one tile per cluster at a time
@@ -953,7 +1026,7 @@ cudaError_t launch_tc(const CUtensorMap& mA, const CUtensorMap& mB0, const CUten
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, a);
+    e = cudaLaunchKernelEx(&cfg, kern, mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, mOut, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1060,9 +1133,10 @@ cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const voi
     const int units = pair ? num_sms() / 2 : num_sms();
     if (Y_zero && max_tiles < units) max_tiles = units;  // every CTA zeroes a share
     if (pair)
-        return launch_tc<EPI_SWIGLU, true>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, a, max_tiles,
+        return launch_tc<EPI_SWIGLU, true>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, mA, a, max_tiles,
                                            st);
-    return launch_tc<EPI_SWIGLU, false>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, a, max_tiles, st);
+    return launch_tc<EPI_SWIGLU, false>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, mA, a, max_tiles,
+                                        st);
 }
 
 cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void* h,
@@ -1128,14 +1202,21 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
         (routed_mtile_bound(p, tm) * a.nt_r + (sh ? ((p.N + tm - 1) / tm) * a.nt_sh : 0)) * a.ks;
     if (mode == DOWN_COMBINE) {
         if (pair)
-            return launch_tc<EPI_COMBINE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles,
+            return launch_tc<EPI_COMBINE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, mA, a, max_tiles,
                                                 st);
-        return launch_tc<EPI_COMBINE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles,
+        return launch_tc<EPI_COMBINE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, mA, a, max_tiles,
                                              st);
     }
+    // plain stores: whole 32-row slabs of the output leave by TMA store
+    CUtensorMap mOut = mA;
+    a.tma_out = (a.ks == 1 && make_map_out(&mOut, H_out, (uint64_t)a.max_rows, (uint64_t)a.n_valid_r,
+                                           (uint64_t)a.ld_out))
+                    ? 1
+                    : 0;
     if (pair)
-        return launch_tc<EPI_STORE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles, st);
-    return launch_tc<EPI_STORE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, a, max_tiles, st);
+        return launch_tc<EPI_STORE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, mOut, a, max_tiles,
+                                          st);
+    return launch_tc<EPI_STORE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, mOut, a, max_tiles, st);
 }
 
 cudaError_t launch_tc_store_bmn(const moe_params& p, int64_t n_out, int64_t K, const void* A0, int64_t ldA0,
@@ -1178,7 +1259,9 @@ cudaError_t launch_tc_store_bmn(const moe_params& p, int64_t n_out, int64_t K, c
     a.ks = 1;
     a.counters = counters;
     const int64_t max_tiles = routed_mtile_bound(p, 128) * a.nt_r;
-    return launch_tc<EPI_STORE, false>(mA, mB0, mB1, mA, mB0, mB1, mA2, mA, a, max_tiles, st);
+    CUtensorMap mOut = mA;
+    a.tma_out = make_map_out(&mOut, out, (uint64_t)a.max_rows, (uint64_t)n_out, (uint64_t)n_out) ? 1 : 0;
+    return launch_tc<EPI_STORE, false>(mA, mB0, mB1, mA, mB0, mB1, mA2, mA, mOut, a, max_tiles, st);
 }
 
 cudaError_t launch_tc_dense(int64_t M, int64_t Nc, int64_t K, const void* A, const void* B, float* out,
@@ -1208,7 +1291,9 @@ cudaError_t launch_tc_dense(int64_t M, int64_t Nc, int64_t K, const void* A, con
         cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)M * (size_t)Nc, st);
         if (e != cudaSuccess) return e;
     }
-    return launch_tc<EPI_STORE, false>(mA, mB, mB, mA, mB, mB, mA, mA, a, tiles * a.ks, st);
+    CUtensorMap mOut = mA;
+    a.tma_out = (a.ks == 1 && make_map_out(&mOut, out, (uint64_t)M, (uint64_t)Nc, (uint64_t)Nc)) ? 1 : 0;
+    return launch_tc<EPI_STORE, false>(mA, mB, mB, mA, mB, mB, mA, mA, mOut, a, tiles * a.ks, st);
 }
 
 cudaError_t launch_tc_logits(const moe_params& p, const void* x, const void* W_r, float* logits,
