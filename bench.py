@@ -663,7 +663,8 @@ def backward_kernels(w: si.Workload) -> int:
     """Kernels one moe_backward launches: offsets check (1), tables (5), scores
     (1), dY gather (1), z / u / W_d^T dY / dx-row GEMMs (4; W_d, W_g, W_u read
     as stored), SwiGLU backward (1), router (1), router contractions (2, plus
-    the slice sum when dW_r = dG^T X is split over the tokens), db (2), dx (1),
+    the slice sum when dW_r = dG^T X is split over the tokens on the CUDA
+    cores, or the score split and its tables on the tensor cores), db (2), dx (1),
     row transposes (5), weight-gradient prefixes (2) and GEMMs (3); the shared
     expert adds 19."""
     tiles = ((w.E + 63) // 64) * ((w.d + 63) // 64)
@@ -673,7 +674,10 @@ def backward_kernels(w: si.Workload) -> int:
         # fp32: scores, two gathers, SwiGLU, router chain, dx; per touched expert
         # z, u, W_d^T dY, two dx-row and three weight-gradient contractions
         return 1 + 1 + 2 + 1 + (3 + 2 + (1 if slices > 1 else 0)) + 1 + 8 * w.E + (8 if w.d_f_shared else 0)
-    return 29 + (1 if slices > 1 else 0) + (19 if w.d_f_shared else 0)
+    # E_r % 64 == 0: the router contractions run on the tensor cores, after a
+    # score split and a table kernel (no slice sum)
+    router_tc = w.E % 64 == 0 and w.N % 8 == 0
+    return 29 + (2 if router_tc else (1 if slices > 1 else 0)) + (19 if w.d_f_shared else 0)
 
 
 def run_gpu_backward(args):

@@ -16,8 +16,10 @@
 // Router (one warp per token): dwc -> routing-weight gradient (overflow
 // policy, renormalisation) -> probability gradient -> score gradient dG
 // (softmax Jacobian) + the balance objective's term; dx += dG W_r,
-// dW_r = dG^T X, db = column sums of dG (fp32 CUDA-core kernels: E_r is
-// small).  dx gathers the expert rows' dx_perm in token order.
+// dW_r = dG^T X, db = column sums of dG.  With E_r a multiple of 64 (bf16)
+// the two contractions run on the tensor cores, dG split into bf16 hi + lo
+// parts (two K segments of one launch, W_r and X read as stored); otherwise
+// fp32 CUDA-core kernels.  dx gathers the expert rows' dx_perm in token order.
 //
 // Layout choices for the tcgen05 GEMM (out = A B^T, A K-major): z and u run
 // on the grouped kernel in store mode with the dimensions relabelled (its
@@ -611,9 +613,11 @@ cudaError_t simt_gemm_sliced(int64_t M, int64_t N, int64_t K, const TA* A, int64
 // ---------------------------------------------------------------------------
 // Workspace
 // ---------------------------------------------------------------------------
+bool router_on_tensor_cores(const moe_params& p);
+
 struct BwdLayout {
     size_t tstart, nkb, mt_start, offs_d, offs_f, mt_d, mt_f, sh_off, sh_tstart, sh_nkb, counters;
-    size_t logits, dG, part, part_db, dwc, doP, mt128, dYp, Z, U, Gd, dzu, dxp, doT, xT, hT, dzT, duT;
+    size_t logits, dG, part, part_db, dwc, doP, mt128, rsplit, rtab, dYp, Z, U, Gd, dzu, dxp, doT, xT, hT, dzT, duT;
     size_t dYs, Zs, Us, Gs, dzus, dxs, WsT_d, WsT_gu, dYsT, xsT, hsT, dzsT, dusT;
     int64_t Kmax, Kmax_sh;
     size_t total;
@@ -675,6 +679,9 @@ BwdLayout bwd_layout(const moe_params& p, int64_t Kmax) {
     L.dwc = take(rows * 4);
     L.doP = take((1 - tb) * rows * d * 4);
     L.mt128 = take((E + 1) * 4);  // 128-row tile prefix for the MN-major weight contractions
+    // the score gradient's bf16 parts for the tensor-core router contractions
+    L.rsplit = take(router_on_tensor_cores(p) ? 4 * N * E * 2 : 0);
+    L.rtab = take(8 * 4);
     L.dYp = take(rows * d * es);
     L.Z = take(rows * df * 4);
     L.U = take(rows * df * 4);
@@ -738,10 +745,72 @@ unsigned grid_for(int64_t items_per_block_units, int64_t n) {
 
 // Router chain of the backward: score gradient dG (bwd_router_kernel), then
 // dx = dG W_r (written), dW_r = dG^T X (sliced over the tokens) and db_r.
+// The score gradient dG [N, E] (fp32) as two bf16 parts, hi = bf16(dG) and
+// lo = bf16(dG - hi), each also transposed to [E, N]: the tensor-core router
+// contractions multiply both parts by the exact bf16 W_r or x and add them, so
+// dG enters with about 16 mantissa bits instead of 8.  32 x 32 tiles through
+// shared memory, so both layouts are written row-contiguously.
+__global__ void __launch_bounds__(256)
+    bwd_split_scores_kernel(const float* __restrict__ dG, int64_t N, int E, bf16* __restrict__ hi,
+                            bf16* __restrict__ lo, bf16* __restrict__ hiT, bf16* __restrict__ loT) {
+    __shared__ float tile[32][33];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
+    const int64_t t0 = (int64_t)blockIdx.y * 32;
+    const int e0 = blockIdx.x * 32;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t t = t0 + ty + 8 * i;
+        const int e = e0 + tx;
+        float v = 0.f;
+        if (t < N && e < E) {
+            v = dG[t * E + e];
+            const bf16 h = __float2bfloat16_rn(v);
+            hi[t * E + e] = h;
+            lo[t * E + e] = __float2bfloat16_rn(v - __bfloat162float(h));
+        }
+        tile[ty + 8 * i][tx] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int e = e0 + ty + 8 * i;
+        const int64_t t = t0 + tx;
+        if (t < N && e < E) {
+            const float v = tile[tx][ty + 8 * i];
+            const bf16 h = __float2bfloat16_rn(v);
+            hiT[(int64_t)e * N + t] = h;
+            loT[(int64_t)e * N + t] = __float2bfloat16_rn(v - __bfloat162float(h));
+        }
+    }
+}
+
+// One-group row offsets and 128-row tile prefixes for the two router
+// contractions: t[0..1] = {0, N}, t[2..3] = {0, tiles(N)}, t[4..5] = {0, E},
+// t[6..7] = {0, tiles(E)}.
+__global__ void bwd_router_tables_kernel(int32_t* t, int32_t N, int32_t E) {
+    if (threadIdx.x == 0) {
+        t[0] = 0;
+        t[1] = N;
+        t[2] = 0;
+        t[3] = (N + 127) / 128;
+        t[4] = 0;
+        t[5] = E;
+        t[6] = 0;
+        t[7] = (E + 127) / 128;
+    }
+}
+
+// Whether the bf16 router contractions run on the tensor cores: E_r a
+// multiple of the 64-wide K block and 16-byte rows of the transposed scores.
+bool router_on_tensor_cores(const moe_params& p) {
+    return p.dtype == MOE_BF16 && p.E_r % 64 == 0 && p.N % 8 == 0 && p.N > 0 && p.d % 8 == 0;
+}
+
 template <typename T>
 moe_status router_backward(const moe_params& p, float aux_coef, const T* x, const T* W_r, const float* b_r,
                            const WsView& v, const float* logits, const float* dwc, float* dG, float* part,
-                           float* part_db, const moe_grads* gr, cudaStream_t st) {
+                           float* part_db, const moe_grads* gr, cudaStream_t st, bf16* split = nullptr,
+                           int32_t* tables = nullptr, unsigned long long* counters = nullptr) {
     const int64_t N = p.N, d = p.d, E = p.E_r;
     RouterBwd ra{};
     ra.logits = logits;
@@ -764,10 +833,34 @@ moe_status router_backward(const moe_params& p, float aux_coef, const T* x, cons
     bwd_router_kernel<<<grid_for(8, N), 256, 0, st>>>(ra);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return bwd_fail(e, "router");
-    e = simt_gemm<float, T>(N, d, E, dG, E, 1, W_r, 1, d, gr->dx, d, st);
-    if (e == cudaSuccess)  // K = N tokens, few output tiles: sliced over the tokens
-        e = simt_gemm_sliced<float, T>(E, d, N, dG, 1, E, x, 1, d, gr->dW_r, part, st);
-    if (e != cudaSuccess) return bwd_fail(e, "router contractions");
+    if (split && tables) {
+        // tensor cores: dx = dG W_r and dW_r = dG^T x, each as hi + lo parts of
+        // dG in two K segments of one launch, W_r and x read as stored (MN-major)
+        bf16 *hi = split, *lo = split + N * E, *hiT = split + 2 * N * E, *loT = split + 3 * N * E;
+        bwd_split_scores_kernel<<<dim3((unsigned)((E + 31) / 32), (unsigned)((N + 31) / 32)), 256, 0, st>>>(
+            dG, N, (int)E, hi, lo, hiT, loT);
+        bwd_router_tables_kernel<<<1, 32, 0, st>>>(tables, (int32_t)N, (int32_t)E);
+        if ((e = cudaGetLastError()) != cudaSuccess) return bwd_fail(e, "score split");
+        int status = MOE_OK;
+        moe_params q = p;  // one group of N rows, K = E_r
+        q.E_r = 1;
+        q.k = 1;
+        q.d_f_shared = 0;
+        e = launch_tc_store_bmn(q, d, E, hi, E, W_r, lo, E, W_r, tables, tables + 2, gr->dx, counters, st, &status);
+        if (e != cudaSuccess) return bwd_fail(e, "router dx (tcgen05)");
+        q.N = E;  // one group of E_r rows, K = N tokens, split over the tokens
+        const bool split_k = tc_store_bmn_split(q, d, N, true) > 1;
+        if (split_k && (e = cudaMemsetAsync(gr->dW_r, 0, sizeof(float) * E * d, st)) != cudaSuccess)
+            return bwd_fail(e, "memset");
+        e = launch_tc_store_bmn(q, d, N, hiT, N, x, loT, N, x, tables + 4, tables + 6, gr->dW_r, counters, st,
+                                &status, split_k);
+        if (e != cudaSuccess) return bwd_fail(e, "router dW_r (tcgen05)");
+    } else {
+        e = simt_gemm<float, T>(N, d, E, dG, E, 1, W_r, 1, d, gr->dx, d, st);
+        if (e == cudaSuccess)  // K = N tokens, few output tiles: sliced over the tokens
+            e = simt_gemm_sliced<float, T>(E, d, N, dG, 1, E, x, 1, d, gr->dW_r, part, st);
+        if (e != cudaSuccess) return bwd_fail(e, "router contractions");
+    }
     if (gr->db_r) {
         const int64_t chunk = (N + kMaxSlices - 1) / kMaxSlices;
         bwd_colsum_kernel<<<dim3((unsigned)((E + 31) / 32), (unsigned)kMaxSlices), 256, 0, st>>>(dG, N, (int)E, chunk,
@@ -1028,8 +1121,10 @@ moe_status moe_backward(const moe_params* p, float aux_coef, const int32_t* offs
     if (e != cudaSuccess) return bwd_fail(e, "dx rows (tcgen05)");
 
     const bf16* xb = static_cast<const bf16*>(x);
+    const bool rtc = router_on_tensor_cores(*p);
     if ((s = router_backward<bf16>(*p, aux_coef, xb, static_cast<const bf16*>(W_r), b_r, v, logits, dwc, dG,
-                                   F32(L.part), F32(L.part_db), gr, st)) != MOE_OK)
+                                   F32(L.part), F32(L.part_db), gr, st, rtc ? B16(L.rsplit) : nullptr,
+                                   rtc ? I32(L.rtab) : nullptr, counters)) != MOE_OK)
         return s;
 
     // shared expert: weight 1 on every token

@@ -1219,10 +1219,17 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
     return launch_tc<EPI_STORE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, mOut, a, max_tiles, st);
 }
 
+int tc_store_bmn_split(const moe_params& p, int64_t n_out, int64_t K, bool two_segments) {
+    const int nkb = (int)((K + BK - 1) / BK) * (two_segments ? 2 : 1);
+    const double tiles = (double)((p.N * p.k + 127) / 128 + p.E_r - 1) * (double)((n_out + BN - 1) / BN);
+    return choose_ksplit(tiles, nkb);
+}
+
 cudaError_t launch_tc_store_bmn(const moe_params& p, int64_t n_out, int64_t K, const void* A0, int64_t ldA0,
                                 const void* B0, const void* A1, int64_t ldA1, const void* B1,
                                 const int32_t* offsets, const int32_t* mt_start128, float* out,
-                                unsigned long long* counters, cudaStream_t st, int* status) {
+                                unsigned long long* counters, cudaStream_t st, int* status, bool split_k,
+                                int* ks_out) {
     *status = MOE_OK;
     CUtensorMap mA, mA2, mB0, mB1;
     const uint64_t rows = (uint64_t)(p.N * p.k);
@@ -1256,11 +1263,14 @@ cudaError_t launch_tc_store_bmn(const moe_params& p, int64_t n_out, int64_t K, c
     a.max_rows = (int)(p.N * p.k);
     a.n_tokens = (int)p.N;
     a.has_routed = 1;
-    a.ks = 1;
+    a.ks = split_k ? tc_store_bmn_split(p, n_out, K, two) : 1;
+    if (ks_out) *ks_out = a.ks;
     a.counters = counters;
-    const int64_t max_tiles = routed_mtile_bound(p, 128) * a.nt_r;
+    const int64_t max_tiles = routed_mtile_bound(p, 128) * a.nt_r * a.ks;
     CUtensorMap mOut = mA;
-    a.tma_out = make_map_out(&mOut, out, (uint64_t)a.max_rows, (uint64_t)n_out, (uint64_t)n_out) ? 1 : 0;
+    a.tma_out = (a.ks == 1 && make_map_out(&mOut, out, (uint64_t)a.max_rows, (uint64_t)n_out, (uint64_t)n_out))
+                    ? 1
+                    : 0;
     return launch_tc<EPI_STORE, false>(mA, mB0, mB1, mA, mB0, mB1, mA2, mA, mOut, a, max_tiles, st);
 }
 

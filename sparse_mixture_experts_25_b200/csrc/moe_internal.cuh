@@ -163,11 +163,18 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
 // (offsets), with B0, B1 [E_r][K][n_out] read as stored (MN-major operands:
 // no transposed copies); A rows K-major with leading dimensions ldA0 / ldA1;
 // fp32 out [N k, n_out].  Single-CTA 128-row tiles: mt_start128 is the
-// 128-row tile prefix of offsets.
+// 128-row tile prefix of offsets.  split_k: when the output tiles fill less
+// than one wave, the K blocks are split across CTAs and added into `out`
+// with red.add, so the caller zeroes it first (the function returns the
+// split it chose in *ks_out when that is not null; pass split_k = false to
+// keep one CTA per tile).
 cudaError_t launch_tc_store_bmn(const moe_params& p, int64_t n_out, int64_t K, const void* A0, int64_t ldA0,
                                 const void* B0, const void* A1, int64_t ldA1, const void* B1,
                                 const int32_t* offsets, const int32_t* mt_start128, float* out,
-                                unsigned long long* counters, cudaStream_t st, int* status);
+                                unsigned long long* counters, cudaStream_t st, int* status,
+                                bool split_k = false, int* ks_out = nullptr);
+// K blocks split that launch_tc_store_bmn uses for these sizes with split_k
+int tc_store_bmn_split(const moe_params& p, int64_t n_out, int64_t K, bool two_segments);
 // rows of one output tile of the tcgen05 grouped GEMMs for these params
 // (256 when CTA pairs are used, else 128): the dispatch's M-tile prefix unit
 int tc_tile_rows(const moe_params& p);

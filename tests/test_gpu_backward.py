@@ -52,6 +52,9 @@ CASES = {
     "weight_order": W["qwen3_skew_bf16"].scaled("bwd_weight_order", N=700, d=128, d_f=192, E=16, k=2, c=0.8,
                                                 accept_order=1, reject_policy=1),
     "odd_experts": W["mixtral_bf16"].scaled("bwd_odd_experts", N=200, d=64, d_f=64, E=34, k=3, c=1.0),
+    # 128 experts: router contractions on the tensor cores (bf16 hi + lo parts of
+    # the score gradient), N not a multiple of 32, K split over the tokens for dW_r
+    "wide_router_aux": W["qwen3_skew_bf16"].scaled("bwd_wide_router", N=520, d=192, d_f=128, E=128, k=8),
     "one_expert_ragged": W["mixtral_bf16"].scaled("bwd_one_expert", N=200, d=64, d_f=136, E=1, k=1),
     # fp32 layers (every contraction on the CUDA cores, nothing rounded)
     "switch_f32_capped": W["switch_top1_f32"].scaled("bwd_switch_f32", N=1000, d=72, d_f=96, c=0.9),
@@ -59,7 +62,8 @@ CASES = {
                                                             norm=si.NORM_RENORM, c=0.8, d_f_shared=40,
                                                             reject_policy=1),
 }
-AUX = {"qwen3_capped_aux": 0.5, "weight_order": 0.3, "odd_experts": 1.0, "switch_f32_capped": 0.5}
+AUX = {"qwen3_capped_aux": 0.5, "weight_order": 0.3, "odd_experts": 1.0, "switch_f32_capped": 0.5,
+       "wide_router_aux": 0.5}
 
 
 def _grads(w, device="cuda"):
