@@ -259,6 +259,7 @@ __global__ void __launch_bounds__(256)
         const bool ok = tok >= 0 && tok < n_tokens;
         const float s = scale ? scale[r] : 1.f;
         const float* src = dY + (ok ? tok : 0) * d;
+#pragma unroll 4
         for (int64_t c = lane; c < d / 4; c += 32) {
             float4 v = ok ? ld4(src + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
             v.x *= s; v.y *= s; v.z *= s; v.w *= s;
@@ -486,22 +487,38 @@ __global__ void __launch_bounds__(256)
     const int64_t wpb = blockDim.x >> 5;
     for (int64_t t = blockIdx.x * wpb + (threadIdx.x >> 5); t < N; t += (int64_t)gridDim.x * wpb) {
         float4* o = reinterpret_cast<float4*>(dx + t * d);
-        for (int64_t c = lane; c < d / 4; c += 32) {
-            float4 v = o[c];
-            if (dxs) {
-                const float4 s = reinterpret_cast<const float4*>(dxs + t * d)[c];
-                v.x += s.x; v.y += s.y; v.z += s.z; v.w += s.w;
+        // the token's accepted rows, resolved once: lane j holds path j's row
+        // (-1: rejected), for paths j0 .. j0 + 31
+        for (int j0 = 0; j0 < k; j0 += 32) {
+            int64_t my_row = -1;
+            if (j0 + lane < k) {
+                const int e = ids[t * k + j0 + lane];
+                const int s = slot[t * k + j0 + lane];
+                if (e >= 0 && e < E && s >= 0) {
+                    const int64_t row = (int64_t)offsets[e] + s;
+                    if (row < max_rows) my_row = row;
+                }
             }
-            for (int j = 0; j < k; ++j) {
-                const int e = ids[t * k + j];
-                const int s = slot[t * k + j];
-                if (e < 0 || e >= E || s < 0) continue;
-                const int64_t row = (int64_t)offsets[e] + s;
-                if (row >= max_rows) continue;
-                const float4 q = reinterpret_cast<const float4*>(dxp + row * d)[c];
-                v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
+            const int nj = min(32, k - j0);
+            // every lane runs the same trip count (the shuffles need the whole warp)
+            for (int64_t c0 = 0; c0 < d / 4; c0 += 32) {
+                const int64_t c = c0 + lane;
+                const bool in = c < d / 4;
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (in) v = o[c];
+                if (in && dxs && j0 == 0) {
+                    const float4 q = reinterpret_cast<const float4*>(dxs + t * d)[c];
+                    v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
+                }
+#pragma unroll 4
+                for (int j = 0; j < nj; ++j) {
+                    const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
+                    if (row < 0 || !in) continue;
+                    const float4 q = reinterpret_cast<const float4*>(dxp + row * d)[c];
+                    v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
+                }
+                if (in) o[c] = v;
             }
-            o[c] = v;
         }
     }
 }
