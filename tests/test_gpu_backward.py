@@ -43,6 +43,9 @@ W = si.WORKLOADS
 CASES = {
     "mixtral_small": W["mixtral_bf16"].scaled("bwd_mixtral_small", N=512, d=320, d_f=384),
     "pair_tiles": W["mixtral_bf16"].scaled("bwd_pair", N=1600, d=320, d_f=384, E=2, k=1),
+    # d_f = 800 >= 768: dW_g and dW_u run on CTA pairs (and d = 192: dW_d on
+    # single CTAs), both with the weight-gradient epilogue and ragged tiles
+    "pair_weight_grads": W["mixtral_bf16"].scaled("bwd_pair_dw", N=300, d=192, d_f=800, E=4, k=2),
     "qwen3_capped_aux": W["qwen3_skew_bf16"].scaled("bwd_qwen3", N=1024, d=256, d_f=192, E=32, k=4),
     "deepseek_shared": W["deepseek_shared_bf16"].scaled("bwd_deepseek", N=384, d=448, d_f=128, E=64, k=6,
                                                         d_f_shared=192),
