@@ -530,4 +530,5 @@ def round_bf16(v: float) -> float:
 
 
 # gradients of the layer (numpy, float64): oracle/backward.py
-from oracle.backward import backward, bf16_round, score_gradient  # noqa: E402,F401
+from oracle.backward import (backward, bf16_round, combine_weights, expert_backward_columns,  # noqa: E402,F401
+                             score_gradient, token_dx)

@@ -242,3 +242,96 @@ def backward(x, W_r, Wg, Wu, Wd, dY, ids, w, slot, *, norm: int, reject_policy: 
     out.update({"dx": dx, "dW_r": dG.T @ X, "db_r": dG.sum(axis=0), "dW_g": dWg, "dW_u": dWu, "dW_d": dWd,
                 "dG": dG, "dwc": dwc})
     return out
+
+
+# ---------------------------------------------------------------------------
+# Samples of the same gradients, for layers too large to run whole: each is the
+# definition above restricted to some hidden units or some tokens (the hidden
+# units of an expert are independent of each other, and with aux_coef = 0 a
+# token's dx depends on that token's rows only).  Pinned against backward()
+# in the CPU tests.
+# ---------------------------------------------------------------------------
+def expert_backward_columns(X, Wg, Wu, Wd, dY, wc, cols, *, bf16: bool):
+    """One expert's weight gradients restricted to hidden units `cols`: rows
+    `cols` of dW_g and dW_u and columns `cols` of dW_d, for the expert's
+    accepted rows X [R, d] (any order), their upstream rows dY [R, d] (fp32)
+    and combine weights wc [R].  Weights as stored (bf16 bit patterns or
+    fp32): Wg, Wu [d_f, d], Wd [d, d_f].  Returns float64 (dWg [c, d],
+    dWu [c, d], dWd [d, c])."""
+    rnd = bf16_round if bf16 else (lambda v: v)
+    cols = np.asarray(cols, np.int64)
+    X = _f64(X)
+    Wg_c, Wu_c = _f64(np.asarray(Wg)[cols]), _f64(np.asarray(Wu)[cols])
+    Wd_c = _f64(np.asarray(Wd)[:, cols])
+    wc = np.asarray(wc, np.float64)
+    dYb = rnd(np.asarray(dY, np.float64))
+    Z = X @ Wg_c.T
+    U = X @ Wu_c.T
+    S, dS = _silu_parts(Z)
+    H = S * U
+    if bf16:
+        H = bf16_round(H)
+    dH = wc[:, None] * (dYb @ Wd_c)
+    dZ = rnd(dH * U * dS)
+    dU = rnd(dH * S)
+    dO = rnd(wc[:, None] * dYb)
+    return dZ.T @ X, dU.T @ X, dO.T @ H
+
+
+def token_dx(x, W_r, expert_weights, dY, ids, w, slot, *, norm: int, reject_policy: int = 0, b_r=None,
+             bf16: bool):
+    """dx of some tokens with aux_coef = 0: x [n, d] their rows, dY [n, d],
+    ids / w / slot [n, k] their routing records; expert_weights(e) returns
+    (W_g[e], W_u[e], W_d[e]) as stored.  The same chain as backward(): each
+    accepted path's expert backward on the token's row, the score gradient
+    from its dwc, and dx = sum of the paths' W_g^T dz + W_u^T du + dG W_r.
+    Returns float64 [n, d]."""
+    rnd = bf16_round if bf16 else (lambda v: v)
+    X, Wr = _f64(x), _f64(W_r)
+    ids = np.asarray(ids, np.int64)
+    slot = np.asarray(slot, np.int64)
+    w = np.asarray(w, np.float64)
+    n, d = X.shape
+    k = ids.shape[1]
+    dYb = rnd(np.asarray(dY, np.float64))
+    G = X @ Wr.T
+    if b_r is not None:
+        G = G + np.asarray(b_r, np.float64)[None, :]
+    valid = np.isfinite(G).all(axis=1)
+    P = np.zeros_like(G)
+    if valid.any():
+        Gv = G[valid]
+        Pv = np.exp(Gv - Gv.max(axis=1, keepdims=True))
+        P[valid] = Pv / Pv.sum(axis=1, keepdims=True)
+    _, wc, q = _weights(P, valid, ids, w, slot, norm, reject_policy)
+    acc = q["acc"]
+    dx = np.zeros((n, d))
+    dwc = np.zeros((n, k))
+    for e in np.unique(ids[acc]):  # each expert's weights converted once, its paths together
+        tt, jj = np.nonzero(acc & (ids == e))
+        Wg, Wu, Wd = (_f64(a_) for a_ in expert_weights(int(e)))
+        dXe, _, _, _, dwe = _expert_backward(X[tt], Wg, Wu, Wd, dYb[tt], wc[tt, jj], rnd, bf16)
+        np.add.at(dx, tt, dXe)
+        dwc[tt, jj] = dwe
+    dG = score_gradient(P, valid, ids, w, slot, dwc, norm=norm, reject_policy=reject_policy, aux_coef=0.0)
+    return dx + dG @ Wr
+
+
+def combine_weights(x, W_r, ids, w, slot, *, norm: int, reject_policy: int = 0, b_r=None):
+    """The combine weight wc [n, k] of each accepted path of some tokens (0
+    elsewhere), from their rows x [n, d] and routing records: the router's
+    probabilities, the routing-weight rule of the layer's normalisation, and
+    the overflow policy's rescaling (w is read only for its zero pattern)."""
+    X, Wr = _f64(x), _f64(W_r)
+    G = X @ Wr.T
+    if b_r is not None:
+        G = G + np.asarray(b_r, np.float64)[None, :]
+    valid = np.isfinite(G).all(axis=1)
+    P = np.zeros_like(G)
+    if valid.any():
+        Gv = G[valid]
+        Pv = np.exp(Gv - Gv.max(axis=1, keepdims=True))
+        P[valid] = Pv / Pv.sum(axis=1, keepdims=True)
+    _, wc, _ = _weights(P, valid, np.asarray(ids, np.int64), np.asarray(w, np.float64), np.asarray(slot, np.int64),
+                        norm, reject_policy)
+    return wc

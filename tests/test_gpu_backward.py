@@ -178,3 +178,62 @@ def test_backward_check_reports_stale_host_offsets():
         moe.moe_backward(p, offs, dev["x"], dev["W_r"], None, dev["W_g"], dev["W_u"], dev["W_d"], None, None, None,
                          dY, full["ws"], g, bws)
         assert moe.moe_backward_check(p, bws) == want
+
+
+@pytest.mark.parametrize("name", ["mixtral_bf16", "qwen3_skew_bf16"])
+def test_full_size_backward_sampled(name):
+    """The backward of the page-shaped layers at full size, in the benchmark's
+    launch configuration (CTA-pair weight gradients on the Mixtral shape, the
+    tensor-core router contractions on the Qwen3 shape), checked on samples the
+    oracle computes one by one: rows of dW_g and dW_u and columns of dW_d for
+    six hidden units of three experts (the most loaded, a middle one and the
+    least loaded), and dx of 16 tokens (every path, including rejected ones).
+    Each sampled row within the bf16 bound on its own; aux_coef = 0, so a
+    token's dx depends on its own rows only."""
+    w = si.WORKLOADS[name]
+    inp = si.inputs(w)
+    full = parity.gpu_forward(w, inp)
+    assert full["status"] == moe.MOE_OK
+    rec = full["rec"]
+    p, dev, ws = full["p"], full["dev"], full["ws"]
+    dY = si.upstream_gradient(w)
+    g = _grads(w)
+    bws = torch.empty(moe.moe_backward_workspace_size(p, rec["offsets"]), dtype=torch.uint8, device="cuda")
+    moe.moe_backward(p, rec["offsets"], dev["x"], dev["W_r"], dev.get("b_r"), dev["W_g"], dev["W_u"], dev["W_d"],
+                     None, None, None, torch.from_numpy(dY).cuda(), ws, g, bws, aux_coef=0.0)
+    assert moe.moe_backward_check(p, bws) == moe.MOE_OK
+    ids, wts, slot = rec["ids"], rec["w"], rec["slot"]
+    acc_rows = np.array([int(((ids == e) & (slot >= 0)).sum()) for e in range(w.E)])
+    live = np.nonzero(acc_rows > 0)[0]
+    order = live[np.argsort(acc_rows[live], kind="stable")]
+    experts = [int(order[-1]), int(order[len(order) // 2]), int(order[0])]
+    rng = np.random.default_rng(17)
+    cols = np.unique(np.concatenate([[0, w.d_f // 3, 2 * w.d_f // 3, w.d_f - 1], rng.integers(0, w.d_f, 2)]))
+    wc = oracle.combine_weights(inp["x"], inp["W_r"], ids, wts, slot, norm=w.norm, reject_policy=w.reject_policy,
+                                b_r=inp.get("b_r"))
+    cols_t = torch.from_numpy(cols).cuda()
+    worst = {}
+    for e in experts:
+        tt, jj = np.nonzero((ids == e) & (slot >= 0))
+        ref = oracle.expert_backward_columns(inp["x"][tt], inp["W_g"][e], inp["W_u"][e], inp["W_d"][e], dY[tt],
+                                             wc[tt, jj], cols, bf16=True)
+        got = (g["dW_g"][e].index_select(0, cols_t), g["dW_u"][e].index_select(0, cols_t),
+               g["dW_d"][e].index_select(1, cols_t).T)
+        for n, r_, g_ in zip(("dW_g", "dW_u", "dW_d"), (ref[0], ref[1], ref[2].T), got):
+            g_ = g_.cpu().numpy().astype(np.float64)
+            assert np.isfinite(g_).all()
+            err, row = parity.rel_err(g_, r_), parity.row_rel_err(g_, r_)
+            worst[n] = max(worst.get(n, 0.0), row)
+            assert err <= 5e-3 and row <= 1e-2, (name, n, e, err, row)
+    # tokens: seeded, plus (when the capacity binds) tokens that lost a path
+    lost = np.nonzero(((ids >= 0) & (slot < 0)).any(axis=1))[0]
+    toks = np.union1d(rng.choice(w.N, size=12, replace=False), lost[:4])
+    ref = oracle.token_dx(inp["x"][toks], inp["W_r"], lambda e: (inp["W_g"][e], inp["W_u"][e], inp["W_d"][e]),
+                          dY[toks], ids[toks], wts[toks], slot[toks], norm=w.norm, reject_policy=w.reject_policy,
+                          b_r=inp.get("b_r"), bf16=True)
+    got = g["dx"].index_select(0, torch.from_numpy(toks).cuda()).cpu().numpy().astype(np.float64)
+    err, row = parity.rel_err(got, ref), parity.row_rel_err(got, ref)
+    worst["dx"] = row
+    assert err <= 5e-3 and row <= 1e-2, (name, "dx", err, row)
+    print(f"{name}: largest per-row error {worst}, experts {experts} with {acc_rows[experts].tolist()} rows, "
+          f"{toks.size} tokens ({min(lost.size, 4)} with a rejected path)")
