@@ -275,8 +275,8 @@ MOE_API moe_status moe_dispatch(const moe_params* p, const int32_t* ids, const f
  * counters) lives in a 1 MiB array inside the library, which every GPU that
  * loads the library holds until the process exits.  Limit:
  * E_r * n_tiles + 3 E_r + 33 four-byte words must fit in 1 MiB, with
- * n_tiles = ceil(N / max(8, floor(256 / k))) (for example N = 8192, k = 8,
- * E_r = 128 needs 132 KB); larger sizes return MOE_ERR_UNSUPPORTED with the
+ * n_tiles = ceil(N / max(8, floor(128 / k))) (for example N = 8192, k = 8,
+ * E_r = 128 needs 258 KB); larger sizes return MOE_ERR_UNSUPPORTED with the
  * required size in moe_last_error.  The routing statistics of this call
  * stay inside the array and are not readable through moe_get_stats.
  *

@@ -715,18 +715,47 @@ __global__ void reroute_rows_kernel(const int32_t* __restrict__ ids, const float
 
 // One warp copies a row of row_vec 16-byte words; four loads per lane are in
 // flight before their stores, so that each SM keeps enough bytes outstanding
-// to draw the HBM rate.
+// to draw the HBM rate.  The source rows are read with an evict-last L2
+// policy and the destination written evict-first: a token's row is read once
+// per path (k times), and the copies streaming out must not push the source
+// rows out of L2 between those reads.
+__device__ __forceinline__ uint4 ld_keep(const uint4* p, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+__device__ __forceinline__ void st_stream(uint4* p, uint4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w), "l"(pol)
+                 : "memory");
+}
+
 __device__ __forceinline__ void copy_row_warp(const uint4* __restrict__ src, uint4* __restrict__ dst, int row_vec,
                                               int lane) {
+    uint64_t keep, stream;
+#ifndef MOE_GATHER_HINTS
+#define MOE_GATHER_HINTS 1
+#endif
+    if (MOE_GATHER_HINTS) {
+        asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
+        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(stream));
+    } else {  // both normal priority
+        asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(keep));
+        stream = keep;
+    }
     int i = lane;
     for (; i + 96 < row_vec; i += 128) {
-        const uint4 v0 = src[i], v1 = src[i + 32], v2 = src[i + 64], v3 = src[i + 96];
-        dst[i] = v0;
-        dst[i + 32] = v1;
-        dst[i + 64] = v2;
-        dst[i + 96] = v3;
+        const uint4 v0 = ld_keep(src + i, keep), v1 = ld_keep(src + i + 32, keep);
+        const uint4 v2 = ld_keep(src + i + 64, keep), v3 = ld_keep(src + i + 96, keep);
+        st_stream(dst + i, v0, stream);
+        st_stream(dst + i + 32, v1, stream);
+        st_stream(dst + i + 64, v2, stream);
+        st_stream(dst + i + 96, v3, stream);
     }
-    for (; i < row_vec; i += 32) dst[i] = src[i];
+    for (; i < row_vec; i += 32) st_stream(dst + i, ld_keep(src + i, keep), stream);
 }
 
 constexpr int kGatherThreads = 256;

@@ -124,7 +124,7 @@ moe_status moe_dispatch_noalloc(const moe_params* p, const int32_t* ids, const f
         char msg[256];
         snprintf(msg, sizeof(msg),
                  "moe_dispatch_noalloc: these sizes need %zu bytes of scratch, the static buffer "
-                 "holds %zu (E_r per-tile counts for each tile of max(8, 256/k) tokens); use moe_dispatch",
+                 "holds %zu (E_r per-tile counts for each tile of max(8, 128/k) tokens); use moe_dispatch",
                  need, kScratchBytes);
         record_error(msg);
         return MOE_ERR_UNSUPPORTED;

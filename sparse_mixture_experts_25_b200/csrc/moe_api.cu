@@ -17,8 +17,11 @@ namespace moe {
 size_t esize(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
 
 int dispatch_tile_tokens(int k) {
-    // about 256 requests per dispatch tile (one warp walks a tile)
-    int t = 256 / (k > 0 ? k : 1);
+    // about 128 requests per dispatch tile (one warp walks a tile)
+#ifndef MOE_DISPATCH_TILE_REQUESTS
+#define MOE_DISPATCH_TILE_REQUESTS 128
+#endif
+    int t = MOE_DISPATCH_TILE_REQUESTS / (k > 0 ? k : 1);
     return t < 8 ? 8 : t;
 }
 
