@@ -55,7 +55,7 @@ def kernels_per_step(w: si.Workload, sharded: bool) -> int:
         router = 1                      # fused FFMA router
     dispatch = 5 if sharded else 4      # hist, scan(s), assign, gather
     if w.accept_order == 1:
-        dispatch += 3                   # placement, rank, numbering, per-token pass replace assign
+        dispatch += 2                   # placement, select + numbering, per-token pass replace assign
     if w.reject_policy == 2:
         dispatch += 3 * w.reroute_depth + 2   # offer, scan, assign per round; final offsets; rows
     experts = 2 if w.dtype == si.DT_BF16 else 3   # fp32 layers zero Y in the router or a kernel

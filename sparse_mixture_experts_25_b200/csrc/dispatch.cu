@@ -386,12 +386,13 @@ __device__ void token_pass(const int32_t* __restrict__ ids, const float* __restr
 // indices), expert e's requests sit in token order at seg_req / seg_w
 // [all_offsets[e], all_offsets[e+1]).  An expert with more than C requests
 // accepts the C with the largest weight, equal weights to the earlier
-// request.  prio_select_kernel finds, per such expert, the C-th largest
+// request.  prio_accept_kernel (one block per expert) finds the C-th largest
 // weight W* by a radix select over the order-preserving bit pattern of the
-// fp32 weights (four passes of 8-bit digits, 256-bin shared-memory
-// histograms) and how many of the requests equal to W* are taken; requests
+// fp32 weights (four passes of 8-bit digits into a 256-bin shared-memory
+// histogram) and how many of the requests equal to W* are taken; requests
 // above W* are all accepted, and those equal to W* in token order up to that
-// count.
+// count.  It then numbers the accepted requests in token order and writes the
+// routing records.
 
 // fp32 bits -> unsigned integer with the same order as the floats
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -399,95 +400,123 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__global__ void prio_select_kernel(int64_t C, const int32_t* __restrict__ all_offsets,
-                                   const float* __restrict__ seg_w, uint32_t* __restrict__ sel_key,
-                                   int32_t* __restrict__ sel_take) {
+// One block of 1024 threads per expert.
+//   select  per pass, lanes of a warp with the same digit add to the
+//           histogram once (match_any), and warp 0 finds the digit that holds
+//           the rem-th largest candidate with a scan over 8 bins per lane;
+//   number  each thread takes a contiguous run of the expert's requests, so
+//           the whole numbering costs two block scans (equal keys before the
+//           run, accepted requests before the run) whatever the request count.
+// An expert with at most C requests accepts them all: slot = position.
+__global__ void __launch_bounds__(1024)
+    prio_accept_kernel(int k, int64_t C, const int32_t* __restrict__ all_offsets,
+                       const int32_t* __restrict__ offsets, const int32_t* __restrict__ seg_req,
+                       const float* __restrict__ seg_w, const float* __restrict__ w,
+                       uint32_t* __restrict__ sel_key, int32_t* __restrict__ sel_take,
+                       int32_t* __restrict__ slot, int32_t* __restrict__ slot_token,
+                       float* __restrict__ slot_w) {
     __shared__ int hist[256];
-    __shared__ uint32_t s_prefix, s_mask;
+    __shared__ int warp_tot[33];
+    __shared__ uint32_t s_prefix;
     __shared__ int s_rem;
     const int e = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int s0 = all_offsets[e], Le = all_offsets[e + 1] - s0;
-    if (Le <= C) return;  // every request accepted; nothing to select
-    if (threadIdx.x == 0) {
-        s_prefix = 0;
-        s_mask = 0;
-        s_rem = (int)C;  // rank (1-based, from the top) of the wanted key among the candidates
+    const int64_t o = offsets[e];
+    if (Le <= C) {
+        for (int i = threadIdx.x; i < Le; i += blockDim.x) {
+            const int req = seg_req[s0 + i];
+            slot[req] = i;
+            slot_token[o + i] = req / k;
+            slot_w[o + i] = w[req];
+        }
+        return;
     }
+    uint32_t prefix = 0, mask = 0;
+    int rem = (int)C;  // rank (1-based, from the top) of the wanted key among the candidates
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0;
         __syncthreads();
-        const uint32_t prefix = s_prefix, mask = s_mask;
-        for (int i = threadIdx.x; i < Le; i += blockDim.x) {
-            const uint32_t key = order_key(seg_w[s0 + i]);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            // the digit holding the s_rem-th largest candidate, counting from digit 255 down
-            int cum = 0, rem = s_rem, d = 255;
-            for (; d > 0; --d) {
-                if (cum + hist[d] >= rem) break;
-                cum += hist[d];
+        for (int i0 = 0; i0 < Le; i0 += blockDim.x) {  // warp-uniform trip count
+            const int i = i0 + threadIdx.x;
+            bool cand = false;
+            uint32_t dg = 0;
+            if (i < Le) {
+                const uint32_t key = order_key(seg_w[s0 + i]);
+                cand = (key & mask) == prefix;
+                dg = (key >> shift) & 255u;
             }
-            s_rem = rem - cum;
-            s_prefix = prefix | ((uint32_t)d << shift);
-            s_mask = mask | (255u << shift);
+            const unsigned act = __ballot_sync(0xffffffffu, cand);
+            if (cand) {
+                const unsigned peers = __match_any_sync(act, dg);
+                if (__ffs(peers) - 1 == lane) atomicAdd(&hist[dg], __popc(peers));
+            }
         }
         __syncthreads();
+        if (warp == 0) {
+            // lane l holds digits 255 - 8l down to 248 - 8l (largest first)
+            int c[8], sum = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                c[j] = hist[255 - 8 * lane - j];
+                sum += c[j];
+            }
+            const int incl = warp_incl_scan(sum, lane);
+            const unsigned hit = __ballot_sync(0xffffffffu, incl >= rem);
+            // the candidates always number at least rem; lane 31 if not
+            const int l0 = hit ? __ffs(hit) - 1 : 31;
+            if (lane == l0) {
+                int cum = incl - sum, d = 248 - 8 * lane;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (cum + c[j] >= rem) {
+                        d = 255 - 8 * lane - j;
+                        break;
+                    }
+                    cum += c[j];
+                }
+                s_rem = rem - cum;
+                s_prefix = prefix | ((uint32_t)d << shift);
+            }
+        }
+        __syncthreads();
+        prefix = s_prefix;
+        rem = s_rem;
+        mask |= 255u << shift;
     }
+    const uint32_t T = prefix;  // key of the C-th largest weight
+    const int take = rem;       // requests with exactly that key to accept, earliest first
     if (threadIdx.x == 0) {
-        sel_key[e] = s_prefix;  // key of the C-th largest weight
-        sel_take[e] = s_rem;    // requests with exactly that key to accept, earliest first
+        sel_key[e] = T;
+        sel_take[e] = take;
     }
-}
-
-// One block per expert: walks its requests in token order, decides which are
-// accepted (all of them for an expert with at most C requests), numbers the
-// accepted ones (block-wide scans) and writes the routing records: slot of
-// each request (-1 if rejected) and the token / weight of each accepted row.
-__global__ void prio_scatter_kernel(int k, int64_t C, const int32_t* __restrict__ all_offsets,
-                                    const int32_t* __restrict__ offsets,
-                                    const int32_t* __restrict__ seg_req, const float* __restrict__ seg_w,
-                                    const uint32_t* __restrict__ sel_key,
-                                    const int32_t* __restrict__ sel_take, const float* __restrict__ w,
-                                    int32_t* __restrict__ slot, int32_t* __restrict__ slot_token,
-                                    float* __restrict__ slot_w) {
-    __shared__ int warp_tot[33];
-    const int e = blockIdx.x;
-    const int s0 = all_offsets[e], Le = all_offsets[e + 1] - s0;
-    const bool all_in = Le <= C;
-    // accepted rows of e: Le or C (the cap also keeps a caller's NaN weight,
-    // whose key is arbitrary, from numbering a row past the expert's block)
-    const int cap = all_in ? Le : (int)C;
-    const uint32_t T = all_in ? 0u : sel_key[e];
-    const int take = all_in ? 0 : sel_take[e];
-    int run = 0, run_eq = 0;
-    for (int b = 0; b < Le; b += blockDim.x) {
-        const int i = b + threadIdx.x;
-        const bool in = i < Le;
-        int f = in ? 1 : 0;
-        if (!all_in) {
-            const uint32_t key = in ? order_key(seg_w[s0 + i]) : 0u;
-            const int eq = (in && key == T) ? 1 : 0;
-            int tot_eq;
-            const int ex_eq = block_excl_scan(eq, warp_tot, &tot_eq);
-            f = in && (key > T || (eq && run_eq + ex_eq < take)) ? 1 : 0;
-            run_eq += tot_eq;
+    const int per = (Le + blockDim.x - 1) / blockDim.x;
+    const int b0 = min(Le, (int)threadIdx.x * per), b1 = min(Le, b0 + per);
+    int n_eq = 0;
+    for (int i = b0; i < b1; ++i) n_eq += order_key(seg_w[s0 + i]) == T ? 1 : 0;
+    int tot;
+    const int eq0 = block_excl_scan(n_eq, warp_tot, &tot);
+    int n_f = 0;
+    for (int i = b0, eq = eq0; i < b1; ++i) {
+        const uint32_t key = order_key(seg_w[s0 + i]);
+        if (key > T) ++n_f;
+        else if (key == T && eq++ < take) ++n_f;
+    }
+    int sl = block_excl_scan(n_f, warp_tot, &tot);
+    // accepted rows of e: C (the cap also keeps a caller's NaN weight, whose
+    // key is arbitrary, from numbering a row past the expert's block)
+    for (int i = b0, eq = eq0; i < b1; ++i) {
+        const uint32_t key = order_key(seg_w[s0 + i]);
+        const bool f = key > T || (key == T && eq++ < take);
+        const int req = seg_req[s0 + i];
+        if (f && sl < C) {
+            slot[req] = sl;
+            slot_token[o + sl] = req / k;
+            slot_w[o + sl] = w[req];
+        } else {
+            slot[req] = -1;
         }
-        int tot;
-        const int ex = block_excl_scan(f, warp_tot, &tot);
-        if (in) {
-            const int req = seg_req[s0 + i];
-            if (f && run + ex < cap) {
-                const int sl = run + ex;
-                slot[req] = sl;
-                slot_token[(int64_t)offsets[e] + sl] = req / k;
-                slot_w[(int64_t)offsets[e] + sl] = w[req];
-            } else {
-                slot[req] = -1;
-            }
-        }
-        run += tot;
+        if (f) ++sl;
     }
 }
 
@@ -900,11 +929,8 @@ cudaError_t launch_dispatch(const moe_params& p, int64_t C, int bm, const int32_
                                                              slot, sc.seg_req, sc.seg_w, counters);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         *where = "select";
-        prio_select_kernel<<<E, 1024, 0, st>>>(C, sc.all_offsets, sc.seg_w, sc.sel_key, sc.sel_take);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        *where = "number";
-        prio_scatter_kernel<<<E, 1024, 0, st>>>(k, C, sc.all_offsets, offsets, sc.seg_req, sc.seg_w, sc.sel_key,
-                                              sc.sel_take, w, slot, slot_token, slot_w);
+        prio_accept_kernel<<<E, 1024, 0, st>>>(k, C, sc.all_offsets, offsets, sc.seg_req, sc.seg_w, w,
+                                               sc.sel_key, sc.sel_take, slot, slot_token, slot_w);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         *where = "tokens";
         prio_token_kernel<<<n_tiles, 32, 0, st>>>(ids, w, p.N, k, E, sc.tile_tokens, offsets, renorm, slot,
