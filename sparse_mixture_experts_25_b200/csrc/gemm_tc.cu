@@ -106,6 +106,11 @@ struct TcArgs {
                               //    (a second K segment); 0: one segment
     int tma_out;              // store epilogue without K split: warp slabs whose 32 rows
                               //    are all valid leave by TMA store (tensor map mOut)
+    int swap_tails;           // CTA pairs: the rows of each group past its last 256-row
+                              //    boundary, when at most 128, run as one weight-stationary
+                              //    tile (see group_tail_rows); the M-tile prefix is then
+                              //    built from offsets inside the kernel, and mOut holds the
+                              //    A rows in 16-row boxes
     unsigned long long* counters;
 };
 
@@ -433,12 +438,41 @@ struct Tile {
     int rows;       // valid rows of the tile (<= TM)
     int n_tile;     // output-column tile
     int kb0, kb1;   // K blocks [kb0, kb1) of this tile
+    int swap;       // 1: weight-stationary tail tile (CTA pairs with swap_tails)
 };
 
 struct SchedSmem {
     int32_t mt[kMaxExperts + 1];
     int32_t off[kMaxExperts + 1];
 };
+
+// Weight-stationary tail tiles (CTA pairs, swap_tails).  A pair tile of at
+// most 128 rows costs as long as a full one: an M=128 pair MMA uses half of
+// each SM's tensor datapath.  So the rows of a group of L rows past its last
+// 256-row boundary, when there are at most 128 of them, run as one tile with
+// the operands swapped: the 256 weight rows of the output-column tile on the
+// MMA's M side (128 per CTA, the same boxes a row tile loads as B) and the
+// tail's tokens on its N side, rounded up to 32, so the tile costs in
+// proportion to its rows.  The group's other rows run in 256-row tiles (the
+// last of 129..255 rows).
+__device__ __forceinline__ int group_tail_rows(int L) {
+    const int rem = L > 0 ? (L & 255) : 0;
+    return rem <= 128 ? rem : 0;
+}
+
+__device__ __forceinline__ int group_swap_tiles(int L) {
+    const int tail = group_tail_rows(L);
+    return ((max(L, 0) - tail + 255) >> 8) + (tail > 0 ? 1 : 0);
+}
+
+// MMA N of a tail tile: its rows rounded up to 32 (each CTA loads half)
+__device__ __forceinline__ int swap_tile_n(int rows) {
+    const int n = (rows + 31) / 32 * 32;
+    return n < 32 ? 32 : (n > 128 ? 128 : n);
+}
+
+// kind::f16, D fp32, A and B bf16 K-major, M = 256 across the pair; N per tile
+constexpr uint32_t kIdescSwapBase = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 4) << 24);
 
 // TM: rows of one output tile (128 for one CTA, 256 for a CTA pair); the
 // M-tile prefix in `s.mt` counts tiles of TM rows.
@@ -471,14 +505,26 @@ __device__ __forceinline__ bool decode_tile(int t_in, const SchedSmem& s, const 
             ti.n_tile = 0;
             ti.a_row = 0;
             ti.rows = 0;
+            ti.swap = 0;
             return true;
         }
         const int local = t - s.mt[g] * a.nt_r;
         const int m_tile = local % mtiles;
         ti.n_tile = local / mtiles;
         ti.a_row = s.off[g] + m_tile * TM;
+        int r_end = s.off[g + 1];
+        ti.swap = 0;
+        if (a.swap_tails) {
+            const int tail = group_tail_rows(r_end - s.off[g]);
+            if (tail > 0 && ti.a_row >= r_end - tail) {  // the group's last tile
+                ti.swap = 1;
+                ti.a_row = r_end - tail;
+            } else {
+                r_end -= tail;
+            }
+        }
         // rows of this tile inside the group and inside the row buffer
-        ti.rows = max(0, min(min(TM, s.off[g + 1] - ti.a_row), a.max_rows - ti.a_row));
+        ti.rows = max(0, min(min(TM, r_end - ti.a_row), a.max_rows - ti.a_row));
         if (ti.a_row < 0) ti.rows = 0;
         return true;
     }
@@ -486,6 +532,7 @@ __device__ __forceinline__ bool decode_tile(int t_in, const SchedSmem& s, const 
     const int local = t - routed_tiles;
     if (a.M_sh <= 0 || local >= mt_sh * a.nt_sh) return false;
     ti.shared = 1;
+    ti.swap = 0;
     ti.g = 0;
     ti.n_tile = local / mt_sh;
     ti.a_row = (local % mt_sh) * TM;
@@ -493,6 +540,15 @@ __device__ __forceinline__ bool decode_tile(int t_in, const SchedSmem& s, const 
     ti.kb0 = (int)((int64_t)kq * a.nkb_sh / a.ks);
     ti.kb1 = (int)((int64_t)(kq + 1) * a.nkb_sh / a.ks);
     return true;
+}
+
+__device__ __forceinline__ int warp_incl_sum(int v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    return v;
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
@@ -614,6 +670,112 @@ __device__ __forceinline__ void epilogue_segment(const TcArgs& a, const Tile& ti
     }
 }
 
+// --- tail tiles (CTA pairs): TMEM lane = weight row, column = token --------
+// Exchange handshake of the two epilogue warps of a gate/up column group: all
+// 64 threads arrive on the group's mbarrier, then wait (bounded) for its
+// phase; xk counts this warp's handshakes (both warps of a group make the same
+// number).  A wait that gives up leaves through the abort path.
+__device__ __forceinline__ bool xch_sync(uint64_t* bar, uint32_t& xk, volatile int* abort_flag,
+                                         unsigned long long* counters) {
+    __syncwarp();
+    mbar_arrive(bar);
+    const bool ok = warp_wait_bounded(bar, xk & 1u, abort_flag, counters);
+    ++xk;
+    return ok;
+}
+
+constexpr int kXchLd = 17;  // floats per lane row of the exchange buffers (conflict-free)
+
+// Gate/up tail tile: CTA c holds gate rows of output columns
+// j0 + 64 c .. + 63 in TMEM lanes 0-63 and the up rows of the same columns in
+// lanes 64-127.  The gate and up warps of a column group (lane quarters 0/2
+// and 1/3) trade half of each 32-token chunk through shared memory, and each
+// writes h for 16 tokens: 32 lanes store 32 consecutive columns of a token.
+__device__ __forceinline__ bool tail_epilogue_swiglu(const TcArgs& a, const Tile& ti, uint32_t t_row, int quarter,
+                                                     int lane, uint32_t crank, float* xch, uint64_t* xbar,
+                                                     uint32_t& xk, volatile int* abort_flag) {
+    const int nt = swap_tile_n(ti.rows);
+    const bool gate = quarter < 2;
+    const int grp = quarter & 1;
+    const int j = ti.n_tile * 128 + (int)crank * 64 + grp * 32 + lane;  // output column of this lane
+    const bool col_ok = j < a.n_valid_r;
+    __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(a.out);
+    float* xg = xch + grp * (2 * 32 * kXchLd);  // gate of tokens 16-31 (from the gate warp)
+    float* xu = xg + 32 * kXchLd;               // up of tokens 0-15 (from the up warp)
+#pragma unroll 1
+    for (int c0 = 0; c0 < nt; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(t_row + (uint32_t)c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (gate) xg[lane * kXchLd + i] = __uint_as_float(v[16 + i]);
+            else xu[lane * kXchLd + i] = __uint_as_float(v[i]);
+        }
+        if (!xch_sync(&xbar[grp], xk, abort_flag, a.counters)) return false;
+        const int tb = c0 + (gate ? 0 : 16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float g = gate ? __uint_as_float(v[i]) : xg[lane * kXchLd + i];
+            const float u = gate ? xu[lane * kXchLd + i] : __uint_as_float(v[16 + i]);
+            const int tok = tb + i;
+            if (col_ok && tok < ti.rows)
+                outp[(int64_t)(ti.a_row + tok) * a.ld_out + j] = __float2bfloat16_rn(silu_f(g) * u);
+        }
+        // the exchange rows are free for the next chunk
+        if (!xch_sync(&xbar[grp], xk, abort_flag, a.counters)) return false;
+    }
+    return true;
+}
+
+// Down + combine tail tile: CTA c holds output features n0 + 128 c .. + 127
+// (lane quarter q: 32 of them), a column per token.  Each 32-token chunk is
+// transposed through the warp's swizzled staging tile (row = token) and added
+// into Y[token] with 16-byte red.add, 4 tokens x 128 bytes per instruction.
+__device__ __forceinline__ void tail_epilogue_combine(const TcArgs& a, const Tile& ti, uint32_t t_row, int quarter,
+                                                      int lane, uint32_t crank, float* stg) {
+    const int nt = swap_tile_n(ti.rows);
+    const int nf = ti.n_tile * BN + (int)crank * 128 + quarter * 32;  // first feature of this warp
+    uint8_t* sbuf = reinterpret_cast<uint8_t*>(stg);
+    const int jj = lane & 7;
+#pragma unroll 1
+    for (int c0 = 0; c0 < nt; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(t_row + (uint32_t)c0, v);
+        tmem_ld_wait();
+        // token and combine weight of column c0 + lane
+        long long dst_off = -1;
+        float wt = 0.f;
+        const int tt = c0 + lane;
+        if (tt < ti.rows) {
+            const int row = ti.a_row + tt;
+            if (row < a.max_rows) {
+                const int tok = a.slot_token[row];
+                wt = a.slot_w[row];
+                if (tok >= 0 && tok < a.n_tokens) dst_off = (long long)tok * a.ldY;
+            }
+        }
+        // staging row = token t, column = this lane's feature
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const float val = __uint_as_float(v[t]) * __shfl_sync(0xffffffffu, wt, t);
+            *reinterpret_cast<float*>(sbuf + t * 128 + (((lane >> 2) ^ (t & 7)) << 4) + ((lane & 3) << 2)) = val;
+        }
+        __syncwarp();
+        const int cg = jj * 4;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int rr = i * 4 + (lane >> 3);
+            const long long off = __shfl_sync(0xffffffffu, dst_off, rr);
+            if (off >= 0 && nf + cg < a.n_valid_r) {
+                const float4 val = *reinterpret_cast<const float4*>(sbuf + rr * 128 + ((jj ^ (rr & 7)) << 4));
+                red_add_v4(a.Y + off + nf + cg, val.x, val.y, val.z, val.w);
+            }
+        }
+        __syncwarp();
+    }
+}
+
 // PAIR = false: one CTA computes a 128 x 256 tile (A 128 rows, B 256 rows:
 //   4 stages of 48 KB).
 // PAIR = true: a cluster of two CTAs computes a 256 x 256 tile with
@@ -646,7 +808,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t* tfull = empty + NST;
     uint64_t* tempty = tfull + 2;
     uint64_t* done = tempty + 2;
-    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* xbar = done + 1;  // [2] tail-tile gate/up exchange handshakes (CTA pairs)
+    uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(xbar + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
     SchedSmem* sched = reinterpret_cast<SchedSmem*>(smem + NST * SBYTES + 256);
     // per-epilogue-warp staging tiles (kStgTile bytes each, 1024-byte aligned)
@@ -659,9 +822,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;   // tile-processing unit
     const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
+    const bool swap_tails = PAIR && a.swap_tails;
     if (a.has_routed) {
         for (int i = threadIdx.x; i <= a.E; i += NUM_THREADS) {
-            sched->mt[i] = a.mt_start[i];
+            if (!swap_tails) sched->mt[i] = a.mt_start[i];
             sched->off[i] = a.offsets[i];
         }
     }
@@ -675,6 +839,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&tempty[b], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
         }
         mbar_init(done, 1);
+        mbar_init(&xbar[0], 64);  // the two epilogue warps of a column group
+        mbar_init(&xbar[1], 64);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -701,6 +867,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_s;
+    if (a.has_routed && swap_tails) {
+        // M-tile prefix with tail tiles, from the row offsets (both CTAs of a
+        // pair compute the same one)
+        if (warp == 2) {
+            int carry = 0;
+            for (int base = 0; base < a.E; base += 32) {
+                const int g = base + lane;
+                const int c = g < a.E ? group_swap_tiles(sched->off[g + 1] - sched->off[g]) : 0;
+                const int v = warp_incl_sum(c, lane);
+                if (g < a.E) sched->mt[g] = carry + v - c;
+                carry += __shfl_sync(0xffffffffu, v, 31);
+            }
+            if (lane == 0) sched->mt[a.E] = carry;
+        }
+        __syncthreads();
+    }
 
     const int routed_tiles = a.has_routed ? sched->mt[a.E] * a.nt_r : 0;
     const int total_tiles =
@@ -738,7 +920,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     uint8_t* sa = stage_base + stage * SBYTES;
                     uint8_t* sb = sa + A_BYTES;
-                    if (PAIR) {
+                    if (PAIR && ti.swap) {
+                        // tail tile: this CTA's 128 weight rows (the row tile's B
+                        // boxes) as A, half of the tail's token rows (16-row
+                        // boxes; rows past the tail only feed unused columns) as B
+                        const uint32_t fb = map_shared_rank(smem_u32(&full[stage]), 0);
+                        const int hrows = swap_tile_n(ti.rows) / 2;
+                        if (leader) mbar_expect_tx(&full[stage], 2u * (uint32_t)(A_BYTES + hrows * BK * 2));
+                        if (EPI == EPI_SWIGLU) {
+                            tma_load_2d_pair(sa, pb0, fb, kb * BK, b_row0 + (int)crank * 64);
+                            tma_load_2d_pair(sa + A_BYTES / 2, pb1, fb, kb * BK, b_row0 + (int)crank * 64);
+                        } else {
+                            tma_load_2d_pair(sa, crank == 0 ? pb0 : pb1, fb, kb * BK, crank == 0 ? b_row0 : b_row1);
+                        }
+                        const int x_row = ti.a_row + (int)crank * hrows;
+                        for (int r16 = 0; r16 < hrows; r16 += 16)
+                            tma_load_2d_pair(sb + r16 * BK * 2, &mOut, fb, kb * BK, x_row + r16);
+                    } else if (PAIR) {
                         // both CTAs' bytes complete on the leader's full barrier
                         const uint32_t fb = map_shared_rank(smem_u32(&full[stage]), 0);
                         if (leader) mbar_expect_tx(&full[stage], 2 * (a_bytes + B_HALF_BYTES));
@@ -798,7 +996,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int t = unit; t < total_tiles && ok; t += n_units) {
                 Tile ti;
                 decode_tile<TM>(t, *sched, a, routed_tiles, ti);
-                const uint32_t idesc_pair = ti.rows <= 128 ? kIdescPairHalf : kIdescPair;
+                const uint32_t idesc_pair =
+                    ti.swap ? (kIdescSwapBase | ((uint32_t)(swap_tile_n(ti.rows) >> 3) << 17))
+                            : (ti.rows <= 128 ? kIdescPairHalf : kIdescPair);
                 if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, a.counters)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -866,13 +1066,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float* stg = stg_all + (warp - 2) * (kStgTile / 4);
         int acc = 0;
         uint32_t acc_phase = 0;
+        uint32_t xk = 0;  // tail-tile exchange handshakes of this warp
         for (int t = unit; t < total_tiles; t += n_units) {
             Tile ti;
             decode_tile<TM>(t, *sched, a, routed_tiles, ti);
             if (!warp_wait_bounded(&tfull[acc], acc_phase, abort_flag, a.counters)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-            if (!PAIR) {
+            if (PAIR && ti.swap) {
+                if (EPI == EPI_SWIGLU) {
+                    if (!tail_epilogue_swiglu(a, ti, t_row, quarter, lane, crank, stg_all, xbar, xk, abort_flag))
+                        break;
+                } else if (EPI == EPI_COMBINE) {
+                    tail_epilogue_combine(a, ti, t_row, quarter, lane, crank, stg);
+                }
+            } else if (!PAIR) {
                 // lane r = row r; gate/up: gate columns 0-127, up 128-255
                 const bool ok = r < ti.rows;
                 if (EPI == EPI_SWIGLU)
@@ -985,12 +1193,15 @@ bool make_map_out(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
     return r == CUDA_SUCCESS;
 }
 
-// the fp32 epilogues stage through shared memory; the SwiGLU epilogue does not
+// the fp32 epilogues stage through shared memory, and on CTA pairs the tail
+// tiles' SwiGLU epilogue trades values through the same area; the single-CTA
+// SwiGLU epilogue needs none
 constexpr size_t smem_bytes(int epi, bool pair) {
     return 1024 + (pair ? (size_t)STAGES_PAIR * STAGE_BYTES_PAIR : (size_t)STAGES * STAGE_BYTES) + 256 +
-           sizeof(SchedSmem) + (epi == EPI_SWIGLU ? 0 : kStgBytes);
+           sizeof(SchedSmem) + (epi == EPI_SWIGLU && !pair ? 0 : kStgBytes);
 }
-static_assert(smem_bytes(EPI_COMBINE, false) <= 232448 && smem_bytes(EPI_COMBINE, true) <= 232448 &&
+static_assert(smem_bytes(EPI_SWIGLU, true) <= 232448 &&
+                  smem_bytes(EPI_COMBINE, false) <= 232448 && smem_bytes(EPI_COMBINE, true) <= 232448 &&
                   smem_bytes(EPI_STORE, false) <= 232448 && smem_bytes(EPI_STORE, true) <= 232448,
               "shared memory per CTA");
 
@@ -1069,11 +1280,23 @@ int choose_ksplit(double tiles, int nkb_min) {
 
 }  // namespace
 
+#ifndef MOE_TC_PAIR_MIN_ROWS
+#define MOE_TC_PAIR_MIN_ROWS 768
+#endif
+#ifndef MOE_TC_SWAP_TAILS
+#define MOE_TC_SWAP_TAILS 1
+#endif
+#ifndef MOE_TC_COMBINE_PAIR_MIN_ROWS
+#define MOE_TC_COMBINE_PAIR_MIN_ROWS 384
+#endif
+
 int tc_tile_rows(const moe_params& p) {
     // CTA pairs (256-row tiles) when experts average enough rows to fill them
     const double mu = (double)p.N * p.k / p.E_r;
-    return (p.dtype == MOE_BF16 && mu >= 768.0) ? 256 : 128;
+    return (p.dtype == MOE_BF16 && mu >= (double)MOE_TC_PAIR_MIN_ROWS) ? 256 : 128;
 }
+
+bool tc_swap_tails(const moe_params& p) { return MOE_TC_SWAP_TAILS && tc_tile_rows(p) == 256; }
 
 cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const void* x_shared,
                               const int32_t* offsets, const int32_t* mt_start,
@@ -1132,9 +1355,19 @@ cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const voi
         routed_mtile_bound(p, tm) * a.nt_r + (sh ? ((p.N + tm - 1) / tm) * a.nt_sh : 0);
     const int units = pair ? num_sms() / 2 : num_sms();
     if (Y_zero && max_tiles < units) max_tiles = units;  // every CTA zeroes a share
-    if (pair)
-        return launch_tc<EPI_SWIGLU, true>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, mA, a, max_tiles,
+    if (pair) {
+        // tail tiles read the gathered rows in 16-row boxes (the mOut slot)
+        CUtensorMap mX16 = mA;
+        if (tc_swap_tails(p)) {
+            if (!make_map(&mX16, x_perm, rows, p.d, 16)) {
+                *status = MOE_ERR_CUDA;
+                return cudaErrorInvalidValue;
+            }
+            a.swap_tails = 1;
+        }
+        return launch_tc<EPI_SWIGLU, true>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, mX16, a, max_tiles,
                                            st);
+    }
     return launch_tc<EPI_SWIGLU, false>(mA, mB0, mB1, mA_sh, mB0_sh, mB1_sh, mA_h, mA_sh_h, mA, a, max_tiles,
                                         st);
 }
@@ -1188,7 +1421,13 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
     a.has_routed = 1;
     a.ks = 1;
     a.grp_nkb = grp_nkb;
-    const bool pair = tc_tile_rows(p) == 256;
+    // the combine runs on CTA pairs with tail tiles also where the layer's row
+    // tiles are 128 rows (its tile list comes from the offsets, not from the
+    // dispatch's M-tile prefix): measured faster than single CTAs on layers of
+    // 384..767 requests per expert, whose gate/up stays on single CTAs
+    const bool combine_swap = mode == DOWN_COMBINE && MOE_TC_SWAP_TAILS && p.dtype == MOE_BF16 &&
+                              (double)p.N * p.k >= (double)MOE_TC_COMBINE_PAIR_MIN_ROWS * p.E_r;
+    const bool pair = tc_tile_rows(p) == 256 || combine_swap;
     const int tm = pair ? 256 : 128;
     if (mode == DOWN_COMBINE) {
         // the combine reduces with red.add into a zeroed Y, so K slices of one
@@ -1201,9 +1440,19 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
     int64_t max_tiles =
         (routed_mtile_bound(p, tm) * a.nt_r + (sh ? ((p.N + tm - 1) / tm) * a.nt_sh : 0)) * a.ks;
     if (mode == DOWN_COMBINE) {
-        if (pair)
-            return launch_tc<EPI_COMBINE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, mA, a, max_tiles,
-                                                st);
+        if (pair) {
+            // tail tiles read the h rows in 16-row boxes (the mOut slot)
+            CUtensorMap mX16 = mA;
+            if (tc_swap_tails(p) || combine_swap) {
+                if (!make_map(&mX16, h, rows, p.d_f, 16)) {
+                    *status = MOE_ERR_CUDA;
+                    return cudaErrorInvalidValue;
+                }
+                a.swap_tails = 1;
+            }
+            return launch_tc<EPI_COMBINE, true>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, mX16, a,
+                                                max_tiles, st);
+        }
         return launch_tc<EPI_COMBINE, false>(mA, mB0, mB0, mA_sh, mB0_sh, mB0_sh, mA_h, mA_sh_h, mA, a, max_tiles,
                                              st);
     }

@@ -675,9 +675,12 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
         // rows the routed GEMMs compute: accepted rows per expert rounded up
         // to the row tile of the kernels that run them
         const int64_t bm = p->dtype == MOE_BF16 ? tc_tile_rows(*p) : kSimtBM;
+        const bool swap = p->dtype == MOE_BF16 && tc_swap_tails(*p);
         int64_t padded = 0, accepted = 0;
         for (int32_t a : acc) {
-            padded += (a + bm - 1) / bm * bm;
+            const int64_t rem = a % 256, tail = swap && rem <= 128 ? rem : 0;
+            // a tail of at most 128 rows runs as one tile of its tokens rounded up to 32
+            padded += (a - tail + bm - 1) / bm * bm + (tail + 31) / 32 * 32;
             accepted += a;
         }
         out->padded_rows = padded;

@@ -178,6 +178,9 @@ int tc_store_bmn_split(const moe_params& p, int64_t n_out, int64_t K, bool two_s
 // rows of one output tile of the tcgen05 grouped GEMMs for these params
 // (256 when CTA pairs are used, else 128): the dispatch's M-tile prefix unit
 int tc_tile_rows(const moe_params& p);
+// CTA-pair layers run each expert's tail of at most 128 rows past its last
+// 256-row boundary as one weight-stationary tile (tokens rounded up to 32)
+bool tc_swap_tails(const moe_params& p);
 // out[M, Nc] (fp32, row-major) = A[M, K] B[Nc, K]^T, bf16 operands with rows
 // of K elements (K % 8 == 0, 16-byte aligned bases), tcgen05 tiles of 128 x 256
 cudaError_t launch_tc_dense(int64_t M, int64_t Nc, int64_t K, const void* A, const void* B, float* out,

@@ -163,9 +163,17 @@ def check_dispatch(w: si.Workload, rec: dict, stats: dict):
     assert stats["C"] == C
     # tile padding of the routed GEMMs: each expert's accepted rows rounded up
     # to the row tile (64 rows for fp32 layers; 128, or 256 on CTA pairs when
-    # experts average >= 768 rows, for bf16 layers)
-    bm = 64 if w.dtype == si.DT_F32 else (256 if w.N * w.k >= 768 * w.E else 128)
-    padded = int(sum(-(-int(a) // bm) * bm for a in d["acc"]))
+    # experts average >= 768 rows, for bf16 layers).  On CTA pairs a tail of
+    # at most 128 rows past the last 256-row boundary runs as one tile of its
+    # rows rounded up to 32.
+    pair = w.dtype != si.DT_F32 and w.N * w.k >= 768 * w.E
+    bm = 64 if w.dtype == si.DT_F32 else (256 if pair else 128)
+
+    def padded_rows(a):
+        tail = a % 256 if pair and a % 256 <= 128 else 0
+        return -(-(a - tail) // bm) * bm + -(-tail // 32) * 32
+
+    padded = int(sum(padded_rows(int(a)) for a in d["acc"]))
     assert stats["padded_rows"] == padded
     assert stats["padding_ratio"] == pytest.approx(padded / s["accepted"] if s["accepted"] else 0.0)
     if w.N:

@@ -60,6 +60,13 @@ SMALL = {
                                                  d_f_shared=128),
     "pair_capped_bf16": W["mixtral_bf16"].scaled("pair_capped_bf16", N=2000, d=128, d_f=256, E=2, k=1,
                                                  c=0.9),
+    # CTA pairs with skewed experts: tails of at most 128 rows past the last
+    # 256-row boundary run as weight-stationary tiles (16, 28, 108 rows here;
+    # the others end in ragged 256-row tiles), and with C = 117 every expert
+    # is a single tail tile
+    "pair_tails_bf16": W["qwen3_skew_bf16"].scaled("pair_tails_bf16", N=2080, d=256, d_f=192, E=8, k=3),
+    "pair_all_tails_bf16": W["qwen3_skew_bf16"].scaled("pair_all_tails_bf16", N=6200, d=192, d_f=128, E=8, k=1,
+                                                       c=0.15),
     # overflow policy: a token that loses a path renormalises its accepted ones
     "renorm_reject_bf16": W["qwen3_skew_bf16"].scaled("renorm_reject_bf16", N=1024, d=256, d_f=192,
                                                      E=32, k=4, reject_policy=1),
