@@ -162,8 +162,10 @@ typedef struct moe_stats {
                                 rerouted expert (included in accepted; rejected and
                                 tokens_affected / tokens_skipped then count the
                                 paths left without any expert); 0 otherwise       */
-    int64_t padded_rows;     /* rows the routed expert GEMMs compute: each expert's
-                                accepted rows rounded up to the GEMM's row tile    */
+    int64_t padded_rows;     /* rows the routed gate/up GEMM computes: each expert's
+                                accepted rows rounded up to the GEMM's row tile (on
+                                CTA pairs a tail of at most 128 rows past the last
+                                256-row boundary rounded up to 32 instead)         */
     double padding_ratio;    /* padded_rows / accepted (0 when nothing accepted)  */
     double aux_balance;      /* E_r sum_e f_e pbar_e ("LLM from scratch" ch. 36.4
                                 balance objective, value only): f_e = L_e / sum L,
