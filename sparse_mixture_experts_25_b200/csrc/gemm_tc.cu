@@ -455,14 +455,9 @@ struct SchedSmem {
 // tail's tokens on its N side, rounded up to 32, so the tile costs in
 // proportion to its rows.  The group's other rows run in 256-row tiles (the
 // last of 129..255 rows).
-#ifndef MOE_TC_SWAP_MAX_TAIL
-#define MOE_TC_SWAP_MAX_TAIL 128
-#endif
-constexpr int kSwapMaxTail = MOE_TC_SWAP_MAX_TAIL;
-
 __device__ __forceinline__ int group_tail_rows(int L) {
     const int rem = L > 0 ? (L & 255) : 0;
-    return rem <= kSwapMaxTail ? rem : 0;
+    return rem <= 128 ? rem : 0;
 }
 
 __device__ __forceinline__ int group_swap_tiles(int L) {
@@ -473,7 +468,7 @@ __device__ __forceinline__ int group_swap_tiles(int L) {
 // MMA N of a tail tile: its rows rounded up to 32 (each CTA loads half)
 __device__ __forceinline__ int swap_tile_n(int rows) {
     const int n = (rows + 31) / 32 * 32;
-    return n < 32 ? 32 : (n > 256 ? 256 : n);
+    return n < 32 ? 32 : (n > 128 ? 128 : n);
 }
 
 // kind::f16, D fp32, A and B bf16 K-major, M = 256 across the pair; N per tile
