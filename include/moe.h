@@ -165,7 +165,8 @@ typedef struct moe_stats {
     int64_t padded_rows;     /* rows the routed gate/up GEMM computes: each expert's
                                 accepted rows rounded up to the GEMM's row tile (on
                                 CTA pairs a tail of at most 128 rows past the last
-                                256-row boundary rounded up to 32 instead)         */
+                                256-row boundary rounded up to 32 instead; on single
+                                CTAs a last tile of at most 64 rows to 64)         */
     double padding_ratio;    /* padded_rows / accepted (0 when nothing accepted)  */
     double aux_balance;      /* E_r sum_e f_e pbar_e ("LLM from scratch" ch. 36.4
                                 balance objective, value only): f_e = L_e / sum L,

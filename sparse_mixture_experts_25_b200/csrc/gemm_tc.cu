@@ -106,6 +106,8 @@ struct TcArgs {
                               //    (a second K segment); 0: one segment
     int tma_out;              // store epilogue without K split: warp slabs whose 32 rows
                               //    are all valid leave by TMA store (tensor map mOut)
+    int a_h64;                // single CTA: mA_h / mA_sh_h hold the A rows in 64-row boxes,
+                              //    so tiles of at most 64 rows run as M=64 MMAs
     int swap_tails;           // CTA pairs: the rows of each group past its last 256-row
                               //    boundary, when at most 128, run as one weight-stationary
                               //    tile (see group_tail_rows); the M-tile prefix is then
@@ -285,13 +287,18 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t addr) {
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
 
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t accumulate) {
+// M = 64 (one CTA): accumulator row i in TMEM lane (i mod 16) + 32 (i / 16),
+// lanes 0-15 of each 32-lane quarter; the other lanes are not written
+constexpr uint32_t kIdescM64 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                               ((uint32_t)(64 >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16_id(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -439,6 +446,7 @@ struct Tile {
     int n_tile;     // output-column tile
     int kb0, kb1;   // K blocks [kb0, kb1) of this tile
     int swap;       // 1: weight-stationary tail tile (CTA pairs with swap_tails)
+    int m64;        // 1: single-CTA tile of at most 64 rows, run as an M=64 MMA
 };
 
 struct SchedSmem {
@@ -506,6 +514,7 @@ __device__ __forceinline__ bool decode_tile(int t_in, const SchedSmem& s, const 
             ti.a_row = 0;
             ti.rows = 0;
             ti.swap = 0;
+            ti.m64 = 0;
             return true;
         }
         const int local = t - s.mt[g] * a.nt_r;
@@ -526,6 +535,7 @@ __device__ __forceinline__ bool decode_tile(int t_in, const SchedSmem& s, const 
         // rows of this tile inside the group and inside the row buffer
         ti.rows = max(0, min(min(TM, r_end - ti.a_row), a.max_rows - ti.a_row));
         if (ti.a_row < 0) ti.rows = 0;
+        ti.m64 = (TM == 128 && a.a_h64 && !a.b_mn && ti.rows > 0 && ti.rows <= 64) ? 1 : 0;
         return true;
     }
     const int mt_sh = (a.M_sh + TM - 1) / TM;
@@ -537,6 +547,7 @@ __device__ __forceinline__ bool decode_tile(int t_in, const SchedSmem& s, const 
     ti.n_tile = local / mt_sh;
     ti.a_row = (local % mt_sh) * TM;
     ti.rows = min(TM, a.M_sh - ti.a_row);
+    ti.m64 = (TM == 128 && a.a_h64 && !a.b_mn && ti.rows > 0 && ti.rows <= 64) ? 1 : 0;
     ti.kb0 = (int)((int64_t)kq * a.nkb_sh / a.ks);
     ti.kb1 = (int)((int64_t)(kq + 1) * a.nkb_sh / a.ks);
     return true;
@@ -965,6 +976,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         for (int c = 0; c < 4; ++c)
                             tma_load_2d(sb + c * (B_HALF_BYTES / 2), pbm, &full[stage], ti.n_tile * 256 + c * BK,
                                         brow);
+                    } else if (ti.m64) {
+                        // at most 64 rows: the first 64 A rows of the stage (an M=64 MMA)
+                        mbar_expect_tx(&full[stage], SBYTES - A_BYTES / 2);
+                        tma_load_2d(sa, ti.shared ? &mA_sh_h : &mA_h, &full[stage], kb * BK, a_row);
+                        tma_load_2d(sb, pb0, &full[stage], kb * BK, b_row0);
+                        tma_load_2d(sb + B_HALF_BYTES, pb1, &full[stage], kb * BK, b_row1);
                     } else {
                         mbar_expect_tx(&full[stage], SBYTES);
                         tma_load_2d(sa, pa, &full[stage], kb * BK, a_row);
@@ -1027,7 +1044,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             if (PAIR)
                                 umma_bf16_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc_pair,
                                                accum);
-                            else umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), accum);
+                            else
+                                umma_bf16_id(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2),
+                                             ti.m64 ? kIdescM64 : kIdesc, accum);
                         }
                     }
                     if (PAIR) umma_commit_pair_both(&empty[stage]);
@@ -1081,12 +1100,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     tail_epilogue_combine(a, ti, t_row, quarter, lane, crank, stg);
                 }
             } else if (!PAIR) {
-                // lane r = row r; gate/up: gate columns 0-127, up 128-255
-                const bool ok = r < ti.rows;
+                // lane r = row r (M=64 tiles: lanes 0-15 of quarter q hold rows
+                // 16 q .. 16 q + 15); gate/up: gate columns 0-127, up 128-255
+                const int rr = ti.m64 ? (lane < 16 ? quarter * 16 + lane : TM) : r;
+                const bool ok = rr < ti.rows;
                 if (EPI == EPI_SWIGLU)
-                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + r, 0, ti.n_tile * 128, 128, 128, stg, &mOut);
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + rr, 0, ti.n_tile * 128, 128, 128, stg, &mOut);
                 else
-                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + r, 0, ti.n_tile * BN, BN, 0, stg, &mOut);
+                    epilogue_segment<EPI>(a, ti, t_row, lane, ok, ti.a_row + rr, 0, ti.n_tile * BN, BN, 0, stg, &mOut);
             } else if (ti.rows > 128) {
                 // 256-row tile: lane r = row crank * 128 + r, all 256 columns
                 const int lr = (int)crank * 128 + r;
@@ -1346,6 +1367,7 @@ cudaError_t launch_tc_gate_up(const moe_params& p, const void* x_perm, const voi
     a.max_rows = (int)(p.N * p.k);
     a.n_tokens = (int)p.N;
     a.has_routed = 1;
+    a.a_h64 = 1;
     a.ks = 1;  // the SwiGLU epilogue needs the whole K sum
     a.zero_ptr = Y_zero;
     a.zero_n4 = Y_zero ? p.N * (int64_t)p.d / 4 : 0;
@@ -1419,6 +1441,7 @@ cudaError_t launch_tc_down(const moe_params& p, int mode, int64_t C, const void*
     a.max_rows = (int)(p.N * p.k);
     a.n_tokens = (int)p.N;
     a.has_routed = 1;
+    a.a_h64 = 1;
     a.ks = 1;
     a.grp_nkb = grp_nkb;
     // the combine runs on CTA pairs with tail tiles also where the layer's row

@@ -681,6 +681,8 @@ moe_status moe_get_stats(const moe_params* p, const void* ws, moe_stats* out, mo
             const int64_t rem = a % 256, tail = swap && rem <= 128 ? rem : 0;
             // a tail of at most 128 rows runs as one tile of its tokens rounded up to 32
             padded += (a - tail + bm - 1) / bm * bm + (tail + 31) / 32 * 32;
+            // single-CTA tcgen05 tiles: a last tile of at most 64 rows is an M=64 MMA
+            if (p->dtype == MOE_BF16 && bm == 128 && a % 128 > 0 && a % 128 <= 64) padded -= 64;
             accepted += a;
         }
         out->padded_rows = padded;

@@ -171,7 +171,11 @@ def check_dispatch(w: si.Workload, rec: dict, stats: dict):
 
     def padded_rows(a):
         tail = a % 256 if pair and a % 256 <= 128 else 0
-        return -(-(a - tail) // bm) * bm + -(-tail // 32) * 32
+        rows = -(-(a - tail) // bm) * bm + -(-tail // 32) * 32
+        # single-CTA tensor-core tiles: a last tile of at most 64 rows is an M=64 MMA
+        if bm == 128 and 0 < a % 128 <= 64:
+            rows -= 64
+        return rows
 
     padded = int(sum(padded_rows(int(a)) for a in d["acc"]))
     assert stats["padded_rows"] == padded
