@@ -525,6 +525,73 @@ def test_wlr_disconnected_expert_and_tie():
     assert list(r["ids"][0]) == [0, -1]
 
 
+def _wlr_random(seed, theta, scale=None):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((64, 8)).astype(np.float32)
+    W_r = rng.standard_normal((7, 8)).astype(np.float32)
+    lat = np.exp(rng.standard_normal((64, 7))).astype(np.float32)
+    if scale is not None:
+        lat = (lat * scale[:, None]).astype(np.float32)
+    return x, W_r, lat, oracle.route(x, W_r, k=4, norm=oracle.NORM_WLR, theta=theta, lat=lat)
+
+
+@pytest.mark.parametrize("theta", [0.1, 0.25, 0.4])
+def test_wlr_kept_set_is_the_rules_fixpoint(theta):
+    """On random tokens, by brute force from the rule's statement: the kept
+    experts are the top-k experts of largest WLR = p / t (ties: the higher
+    index goes first), the kept set passes the test (one expert, or min WLR /
+    (min + max) > theta), and putting back the last expert dropped fails it;
+    weights are the kept probabilities renormalised."""
+    x, W_r, lat, r = _wlr_random(7, theta)
+    topk = oracle.route(x, W_r, k=4, norm=oracle.NORM_RENORM)["ids"]
+    logits = x.astype(np.float64) @ W_r.astype(np.float64).T
+    prob = np.exp(logits - logits.max(axis=1, keepdims=True))
+    prob /= prob.sum(axis=1, keepdims=True)
+    pruned_any = False
+    for t in range(x.shape[0]):
+        S = [int(e) for e in topk[t]]
+        wlr = {e: prob[t, e] / float(lat[t, e]) for e in S}
+        # drop order: smallest WLR first, on equal WLR the higher index first
+        order = sorted(S, key=lambda e: (wlr[e], -e))
+        kept = {int(e) for e in r["ids"][t] if e >= 0}
+        m = len(kept)
+        assert m >= 1 and kept == set(order[len(S) - m:])
+
+        def passes(group):
+            if len(group) < 2:
+                return True
+            lo, hi = min(wlr[e] for e in group), max(wlr[e] for e in group)
+            return lo / (lo + hi) > theta
+
+        assert passes(kept)
+        if m < len(S):
+            pruned_any = True
+            assert not passes(kept | {order[len(S) - m - 1]})
+        want = np.array([prob[t, e] if e in kept else 0.0 for e in S])
+        want /= want.sum()
+        got = np.array([r["w"][t][list(r["ids"][t]).index(e)] if e in kept else 0.0 for e in S])
+        np.testing.assert_allclose(got, want, rtol=1e-6, atol=1e-7)
+    assert pruned_any
+
+
+def test_wlr_latency_scale_and_theta_monotone():
+    """Scaling a token's latencies by one factor changes no WLR ratio, so
+    neither the kept set nor the weights; a larger theta keeps a subset."""
+    rng = np.random.default_rng(8)
+    scale = np.exp(rng.standard_normal(64)).astype(np.float32)
+    _, _, _, a = _wlr_random(9, 0.25)
+    _, _, _, b = _wlr_random(9, 0.25, scale=scale)
+    assert (a["ids"] == b["ids"]).all()
+    np.testing.assert_allclose(a["w"], b["w"], rtol=1e-5, atol=1e-7)
+    prev = None
+    for theta in (0.0, 0.1, 0.2, 0.3, 0.45):
+        _, _, _, r = _wlr_random(9, theta)
+        kept = [set(int(e) for e in row if e >= 0) for row in r["ids"]]
+        if prev is not None:
+            assert all(k <= p for k, p in zip(kept, prev))
+        prev = kept
+
+
 # ---------------------------------------------------------------------------
 # dispatch invariants (Algorithm 36.1) on random requests, checked by brute force
 # ---------------------------------------------------------------------------
